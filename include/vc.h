@@ -1,0 +1,224 @@
+/*
+ * vc.h -- C ABI of the VeriCache hot-path library (libvc_b200.so, sm_100a).
+ *
+ * VeriCache drafts tokens from a compressed KV cache and verifies them against
+ * the full KV cache, keeping exactly the tokens full-cache greedy decoding
+ * would produce ("VeriCache: making lossy KV compression exact", devshah.ca,
+ * section "The Core Idea"; "VeriCache: Turning Lossy KV Cache into Lossless
+ * LLM Inference", menfem.com, section "Key Contributions").  This library is
+ * the data-parallel hot path of one round:
+ *
+ *   draft attention   one query token per request over the compressed cache,
+ *                     either quantised (vc_draft_attn_quant) or token-dropped
+ *                     (vc_draft_attn_sparse);
+ *   verify attention  nq = K + 1 causal query rows per request over the full
+ *                     bf16 cache (vc_verify_attn);
+ *   acceptance        argmax of the K + 1 verifier logit rows, first mismatch,
+ *                     accepted length and correction token (vc_accept).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers are DEVICE pointers unless a parameter says "host".  The caller
+ *   owns all memory; the library never allocates device memory in these
+ *   calls.  Element types are given per argument: bf16 and fp16 arrays are
+ *   passed as `const void*` holding IEEE binary16 / bfloat16 bit patterns.
+ * - Layouts are dense, row-major, with the shapes written in brackets
+ *   (last index fastest).  Every device pointer must be 16-byte aligned.
+ * - `stream` is a cudaStream_t passed as `void*` (NULL = legacy default
+ *   stream).  Calls only enqueue work on that stream and return; nothing
+ *   blocks the host.
+ * - Workspace: each kernel that splits the context across thread blocks
+ *   needs a caller-owned workspace of at least the size its
+ *   *_workspace_size() function returns.  The workspace must be zero-filled
+ *   once before its first use (e.g. cudaMemsetAsync); every call leaves it
+ *   ready for the next call.  Calls that share one workspace must not
+ *   overlap on the GPU (use one workspace per stream in flight).
+ * - Errors: invalid shapes, sizes, alignments or null pointers are detected
+ *   on the host before any launch and return VC_ERR_INVALID_ARG (nothing is
+ *   enqueued); unsupported but well-formed configurations return
+ *   VC_ERR_UNSUPPORTED; a failed launch returns VC_ERR_CUDA.  A thread-local
+ *   message for the last error is available from vc_last_error().  Data
+ *   errors that only the device can see (an out-of-range kept position, a
+ *   bounded wait that timed out) skip the offending access and set a flag
+ *   in the workspace, readable with vc_workspace_flags().
+ */
+#ifndef VC_H_
+#define VC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VC_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define VC_API __attribute__((visibility("default")))
+#else
+#define VC_API
+#endif
+
+typedef enum vc_status {
+  VC_OK = 0,
+  VC_ERR_INVALID_ARG = -1,
+  VC_ERR_UNSUPPORTED = -2,
+  VC_ERR_CUDA = -3,
+  VC_ERR_TIMEOUT = -4,
+  VC_ERR_WORKSPACE = -5
+} vc_status;
+
+typedef enum vc_dtype { VC_F32 = 0, VC_BF16 = 1, VC_F16 = 2 } vc_dtype;
+
+/* Device-side flags reported through the workspace (bit mask). */
+#define VC_FLAG_BAD_INDEX 1u   /* a kept position was outside [0, T_store) */
+#define VC_FLAG_WAIT_TIMEOUT 2u /* a bounded on-chip wait gave up */
+
+/* Message for the last error returned on the calling thread ("" if none). */
+VC_API const char* vc_last_error(void);
+/* ABI version of the loaded library (VC_ABI_VERSION at build time). */
+VC_API int vc_abi_version(void);
+
+/* Attention geometry of one call (one layer).
+ *   B    requests in the batch, >= 1
+ *   Hq   query heads, Hkv KV heads; Hq % Hkv == 0 and g = Hq / Hkv <= 8.
+ *        Query head hq reads KV head hq / g (grouped-query attention).
+ *   D    head dimension, 64 or 128
+ *   sm_scale  softmax scale; a value <= 0 selects 1 / sqrt(D). */
+typedef struct vc_attn_shape {
+  int B;
+  int Hq;
+  int Hkv;
+  int D;
+  float sm_scale;
+} vc_attn_shape;
+
+/* One layer of a quantised draft cache.  Quantisation keeps every position
+ * and lowers the precision of each stored number (devshah.ca page, section
+ * "The Tradeoff VeriCache Is Trying to Escape"); the system sees a compressor
+ * only through its bit width and its dropped positions (menfem.com source
+ * page, section "Key Contributions").  The pages fix no format; this one is
+ * KIVI-style asymmetric uniform quantisation:
+ *
+ *   keys:   per channel over groups of `group` consecutive tokens,
+ *           k_hat[t][c] = code * k_scale[t / group][c] + k_zero[t / group][c]
+ *   values: per token over groups of `group` consecutive channels,
+ *           v_hat[t][c] = code * v_scale[t][c / group] + v_zero[t][c / group]
+ *
+ * evaluated as one fp32 fused multiply-add.  Codes of a token row are packed
+ * little-endian: channel c sits in bits [(c % (8/bits)) * bits, +bits) of byte
+ * c * bits / 8.  The oldest L_q tokens are quantised; the newest R tokens are
+ * kept in bf16 (the residual window, rows 0..R-1 of a buffer of R_cap rows).
+ *
+ *   k_codes, v_codes  uint8 [B][Hkv][L_q][D * bits / 8]
+ *   k_scale, k_zero   fp16  [B][Hkv][L_q / group][D]
+ *   v_scale, v_zero   fp16  [B][Hkv][L_q][D / group]
+ *   k_res, v_res      bf16  [B][Hkv][R_cap][D]
+ *   bits in {2, 4}; group in {32, 64}; L_q >= 0 and a multiple of group;
+ *   0 <= R <= R_cap; L_q + R >= 1.  Scales, zeros and codes must be finite
+ *   and q * scale must stay inside the fp16 range (|q * scale| < 65504). */
+typedef struct vc_quant_cache {
+  const void* k_codes;
+  const void* v_codes;
+  const void* k_scale;
+  const void* k_zero;
+  const void* v_scale;
+  const void* v_zero;
+  const void* k_res;
+  const void* v_res;
+  int bits;
+  int group;
+  int64_t L_q;
+  int R;
+  int R_cap;
+} vc_quant_cache;
+
+/* One layer of a token-dropped draft cache: every (request, KV head) keeps
+ * the same number n_keep of positions (the pages restrict the method to equal
+ * drop counts per layer and head, menfem.com source page, section
+ * "Limitations"; a dropping compressor is described by its positions,
+ * section "Key Contributions").
+ *   k, v   bf16  [B][Hkv][T_store][D]   rows addressed by idx
+ *   idx    int32 [B][Hkv][n_keep]       each in [0, T_store); order free
+ *   n_keep >= 1. */
+typedef struct vc_sparse_cache {
+  const void* k;
+  const void* v;
+  int64_t T_store;
+  const int32_t* idx;
+  int n_keep;
+} vc_sparse_cache;
+
+/* ---- draft attention over a quantised cache --------------------------------
+ * out[b][hq][:] = softmax(q[b][hq] . K_hat^T * sm_scale) . V_hat over the
+ * L_q dequantised tokens followed by the R residual tokens of KV head hq / g.
+ * Drafting decodes one token per step against the compressed cache held in
+ * HBM (menfem.com source page, "Key Contributions").
+ *   q    bf16 [B][Hq][D]        (|q| < 65504)
+ *   out  fp32 [B][Hq][D]
+ *   ws   workspace of vc_draft_attn_quant_workspace_size() bytes. */
+VC_API size_t vc_draft_attn_quant_workspace_size(const vc_attn_shape* shape, const vc_quant_cache* cache);
+VC_API vc_status vc_draft_attn_quant(const vc_attn_shape* shape, const vc_quant_cache* cache, const void* q,
+                              float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- draft attention over a token-dropped cache ----------------------------
+ * out[b][hq][:] = softmax(q . K[idx]^T * sm_scale) . V[idx] over the n_keep
+ * kept rows of KV head hq / g.
+ *   q    bf16 [B][Hq][D];  out fp32 [B][Hq][D]. */
+VC_API size_t vc_draft_attn_sparse_workspace_size(const vc_attn_shape* shape, const vc_sparse_cache* cache);
+VC_API vc_status vc_draft_attn_sparse(const vc_attn_shape* shape, const vc_sparse_cache* cache, const void* q,
+                               float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- block verification attention -----------------------------------------
+ * One pass over the full cache scores every drafted position at once and
+ * yields one extra prediction past the last drafted token (devshah.ca page,
+ * "The Core Idea").  Row i (0 <= i < nq) of
+ * query head hq attends causally to keys 0 .. T - nq + i of KV head hq / g;
+ * the block's own keys are the last nq rows of the cache.
+ *   q    bf16 [B][nq][Hq][D]
+ *   k, v bf16 [B][Hkv][T][D]   (HBM-resident or a staging buffer)
+ *   out  fp32 [B][nq][Hq][D]
+ *   lse  fp32 [B][nq][Hq] natural-log softmax denominators, or NULL
+ *   1 <= nq <= 32, T >= nq. */
+VC_API size_t vc_verify_attn_workspace_size(const vc_attn_shape* shape, int64_t T, int nq);
+VC_API vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* k, const void* v, int64_t T,
+                         int nq, float* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- greedy acceptance -----------------------------------------------------
+ * target[b][i] = argmax_v logits[b][i][v] for i = 0..K (lowest index wins a
+ * tie, +0 and -0 tie, the first NaN counts as the maximum).  accept_len[b] =
+ * the first i < K with draft[b][i] != target[b][i], or K when all match;
+ * correction[b] = target[b][accept_len[b]] (the bonus token when all match).
+ * The emitted run is draft[b][0 .. a-1] followed by correction[b]
+ * (devshah.ca page, "The Core Idea": accept until the first mismatch, insert
+ * the full-cache correction, keep the bonus token when everything matches).
+ *   logits  fp32 or bf16 [B][K+1][V] (dtype VC_F32 or VC_BF16)
+ *   draft   int32 [B][K]; target int32 [B][K+1];
+ *   accept_len, correction int32 [B].   B >= 1, 0 <= K <= 64, V >= 1. */
+VC_API size_t vc_accept_workspace_size(int B, int K, int V);
+VC_API vc_status vc_accept(const void* logits, int dtype, int B, int K, int V, const int32_t* draft, int32_t* target,
+                    int32_t* accept_len, int32_t* correction, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- workspace flags -------------------------------------------------------
+ * Copies the device-side flag word of a workspace to *host_flags and clears
+ * it (a synchronous read on `stream`).  Returns VC_OK or VC_ERR_CUDA. */
+VC_API vc_status vc_workspace_flags(void* ws, size_t ws_bytes, uint32_t* host_flags, void* stream);
+
+/* ---- test exports ------------------------------------------------------------
+ * vc_debug_dequant writes the dequantised L_q rows of every (request, head)
+ * with the same code unpacking the draft kernel uses:
+ *   k_out, v_out fp32 [B][Hkv][L_q][D]   (R residual rows are not included)
+ * vc_debug_gather writes the kept rows the sparse draft kernel reads:
+ *   k_out, v_out bf16 [B][Hkv][n_keep][D]; out-of-range positions write
+ *   zeros and raise VC_FLAG_BAD_INDEX in `ws` (which may be NULL). */
+VC_API vc_status vc_debug_dequant(const vc_attn_shape* shape, const vc_quant_cache* cache, float* k_out, float* v_out,
+                           void* stream);
+VC_API vc_status vc_debug_gather(const vc_attn_shape* shape, const vc_sparse_cache* cache, void* k_out, void* v_out,
+                          void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VC_H_ */

@@ -1,0 +1,194 @@
+"""Python binding of the C ABI in include/vc.h (ctypes; argument marshalling
+only -- every step of the hot path runs in the CUDA library).
+
+Function names match the C entry points.  Tensor arguments are torch CUDA
+tensors (or raw integer device pointers); their data pointers and the current
+CUDA stream are passed through unchanged.  A non-VC_OK status raises VcError
+with the library's message.  If ``libvc_b200.so`` is missing this module
+raises on import of any entry point: there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, Structure, c_char_p, c_float, c_int, c_int32, c_int64, c_size_t, c_uint32, c_void_p
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvc_b200.so")
+
+VC_OK = 0
+VC_ERR_INVALID_ARG = -1
+VC_ERR_UNSUPPORTED = -2
+VC_ERR_CUDA = -3
+VC_ERR_TIMEOUT = -4
+VC_ERR_WORKSPACE = -5
+VC_F32, VC_BF16, VC_F16 = 0, 1, 2
+VC_FLAG_BAD_INDEX = 1
+VC_FLAG_WAIT_TIMEOUT = 2
+
+
+class VcError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"vc status {status}: {msg}")
+        self.status = status
+
+
+class vc_attn_shape(Structure):
+    _fields_ = [("B", c_int), ("Hq", c_int), ("Hkv", c_int), ("D", c_int), ("sm_scale", c_float)]
+
+
+class vc_quant_cache(Structure):
+    _fields_ = [("k_codes", c_void_p), ("v_codes", c_void_p), ("k_scale", c_void_p), ("k_zero", c_void_p),
+                ("v_scale", c_void_p), ("v_zero", c_void_p), ("k_res", c_void_p), ("v_res", c_void_p),
+                ("bits", c_int), ("group", c_int), ("L_q", c_int64), ("R", c_int), ("R_cap", c_int)]
+
+
+class vc_sparse_cache(Structure):
+    _fields_ = [("k", c_void_p), ("v", c_void_p), ("T_store", c_int64), ("idx", c_void_p), ("n_keep", c_int)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvc_b200.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with lossless_draft_verify_vc_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P = POINTER
+        sigs = {
+            "vc_last_error": (c_char_p, []),
+            "vc_abi_version": (c_int, []),
+            "vc_draft_attn_quant_workspace_size": (c_size_t, [P(vc_attn_shape), P(vc_quant_cache)]),
+            "vc_draft_attn_quant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p,
+                                            c_size_t, c_void_p]),
+            "vc_draft_attn_sparse_workspace_size": (c_size_t, [P(vc_attn_shape), P(vc_sparse_cache)]),
+            "vc_draft_attn_sparse": (c_int, [P(vc_attn_shape), P(vc_sparse_cache), c_void_p, c_void_p, c_void_p,
+                                             c_size_t, c_void_p]),
+            "vc_verify_attn_workspace_size": (c_size_t, [P(vc_attn_shape), c_int64, c_int]),
+            "vc_verify_attn": (c_int, [P(vc_attn_shape), c_void_p, c_void_p, c_void_p, c_int64, c_int, c_void_p,
+                                       c_void_p, c_void_p, c_size_t, c_void_p]),
+            "vc_accept_workspace_size": (c_size_t, [c_int, c_int, c_int]),
+            "vc_accept": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, c_size_t, c_void_p]),
+            "vc_workspace_flags": (c_int, [c_void_p, c_size_t, P(c_uint32), c_void_p]),
+            "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
+            "vc_debug_gather": (c_int, [P(vc_attn_shape), P(vc_sparse_cache), c_void_p, c_void_p, c_void_p,
+                                        c_size_t, c_void_p]),
+        }
+        for name, (res, args) in sigs.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(st: int):
+    if st != VC_OK:
+        raise VcError(st, lib().vc_last_error().decode())
+
+
+def _p(x) -> int:
+    """Device pointer of a tensor (or pass an int / None through)."""
+    if x is None:
+        return 0
+    if isinstance(x, int):
+        return x
+    if not x.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def shape(B: int, Hq: int, Hkv: int, D: int, sm_scale: float = 0.0) -> vc_attn_shape:
+    return vc_attn_shape(B, Hq, Hkv, D, sm_scale)
+
+
+def quant_cache(t: dict) -> vc_quant_cache:
+    """Descriptor of a quantised cache given as a dict of CUDA tensors with the
+    keys k_codes, v_codes, k_scale, k_zero, v_scale, v_zero, k_res, v_res and
+    ints bits, group, L_q, R, R_cap (the layout documented in vc.h)."""
+    return vc_quant_cache(_p(t["k_codes"]), _p(t["v_codes"]), _p(t["k_scale"]), _p(t["k_zero"]),
+                          _p(t["v_scale"]), _p(t["v_zero"]), _p(t.get("k_res")), _p(t.get("v_res")),
+                          int(t["bits"]), int(t["group"]), int(t["L_q"]), int(t["R"]), int(t["R_cap"]))
+
+
+def sparse_cache(k, v, idx) -> vc_sparse_cache:
+    return vc_sparse_cache(_p(k), _p(v), int(k.shape[2]), _p(idx), int(idx.shape[-1]))
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace of at least nbytes (16-byte aligned)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+# ---- entry points (same names as the C ABI) ---------------------------------
+
+def vc_abi_version() -> int:
+    return lib().vc_abi_version()
+
+
+def vc_draft_attn_quant_workspace_size(sh: vc_attn_shape, qc: vc_quant_cache) -> int:
+    return lib().vc_draft_attn_quant_workspace_size(ctypes.byref(sh), ctypes.byref(qc))
+
+
+def vc_draft_attn_quant(sh, qc, q, out, ws, stream=None):
+    _check(lib().vc_draft_attn_quant(ctypes.byref(sh), ctypes.byref(qc), _p(q), _p(out), _p(ws),
+                                     ws.numel() if hasattr(ws, "numel") else 1 << 62, _stream(stream)))
+
+
+def vc_draft_attn_sparse_workspace_size(sh, sc) -> int:
+    return lib().vc_draft_attn_sparse_workspace_size(ctypes.byref(sh), ctypes.byref(sc))
+
+
+def vc_draft_attn_sparse(sh, sc, q, out, ws, stream=None):
+    _check(lib().vc_draft_attn_sparse(ctypes.byref(sh), ctypes.byref(sc), _p(q), _p(out), _p(ws),
+                                      ws.numel() if hasattr(ws, "numel") else 1 << 62, _stream(stream)))
+
+
+def vc_verify_attn_workspace_size(sh, T: int, nq: int) -> int:
+    return lib().vc_verify_attn_workspace_size(ctypes.byref(sh), int(T), int(nq))
+
+
+def vc_verify_attn(sh, q, k, v, T: int, nq: int, out, lse, ws, stream=None):
+    _check(lib().vc_verify_attn(ctypes.byref(sh), _p(q), _p(k), _p(v), int(T), int(nq), _p(out), _p(lse), _p(ws),
+                                ws.numel() if hasattr(ws, "numel") else 1 << 62, _stream(stream)))
+
+
+def vc_accept_workspace_size(B: int, K: int, V: int) -> int:
+    return lib().vc_accept_workspace_size(int(B), int(K), int(V))
+
+
+def vc_accept(logits, B: int, K: int, V: int, draft, target, accept_len, correction, ws, stream=None):
+    dtype = VC_BF16 if logits.dtype == torch.bfloat16 else VC_F32
+    if logits.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("logits must be fp32 or bf16")
+    _check(lib().vc_accept(_p(logits), dtype, int(B), int(K), int(V), _p(draft), _p(target), _p(accept_len),
+                           _p(correction), _p(ws), ws.numel(), _stream(stream)))
+
+
+def vc_workspace_flags(ws, stream=None) -> int:
+    v = c_uint32(0)
+    _check(lib().vc_workspace_flags(_p(ws), ws.numel(), ctypes.byref(v), _stream(stream)))
+    return int(v.value)
+
+
+def vc_debug_dequant(sh, qc, k_out, v_out, stream=None):
+    _check(lib().vc_debug_dequant(ctypes.byref(sh), ctypes.byref(qc), _p(k_out), _p(v_out), _stream(stream)))
+
+
+def vc_debug_gather(sh, sc, k_out, v_out, ws=None, stream=None):
+    _check(lib().vc_debug_gather(ctypes.byref(sh), ctypes.byref(sc), _p(k_out), _p(v_out), _p(ws),
+                                 0 if ws is None else ws.numel(), _stream(stream)))
