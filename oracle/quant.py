@@ -2,11 +2,12 @@
 
 What the pages fix
 ------------------
-[P2] "Key Contributions": the compressor interface exposes only dropped-token
-positions and *bits per element*; KIVI and KVQuant are named as quantising
-drafters.  [P2] "Limitations": one bit precision for all layers and tokens.
-[P1] "The Tradeoff VeriCache Is Trying to Escape": quantisation keeps every
-position and stores each entry with fewer bits.
+[P2] "Key Contributions": a compressor is known to the system only through
+the positions it drops and the bit width it stores; KIVI and KVQuant are
+among the quantising drafters it wraps.  [P2] "Limitations": a single bit
+width is shared by every layer and token.  [P1] "The Tradeoff VeriCache Is
+Trying to Escape": quantisation keeps all positions and lowers the precision
+of each stored number.
 
 Readings taken where the pages are silent (all listed in the design doc)
 ------------------------------------------------------------------
