@@ -259,7 +259,7 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
       issue(i + C::NST - 1);
     }
     const int s = i % C::NST;
-    if (!mbar_wait_bounded(&bars[s], (i / C::NST) & 1, a.flags)) {
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (i / C::NST) & 1, a.flags))) {  // warp-uniform
       ok = false;
       for (int k = i; k < my_n && k < i + C::NST; ++k)
         mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
@@ -488,7 +488,7 @@ __device__ void residual_role(const QArgs& a, unsigned char* smem, int unit, int
     __syncwarp();
     const __nv_bfloat16* src = (lane < 16 ? kr : vr) + static_cast<size_t>(valid ? t0 + r : 0) * D;
     bulk_g2s(ring + lane * RSTRIDE, src, ROW_B, bar);
-    if (!mbar_wait_bounded(bar, i & 1, a.flags)) {
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar, i & 1, a.flags))) {  // warp-uniform
       ok = false;
       break;
     }
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(kQNW * 32) draft_quant_kernel(QArgs a) {
   __syncthreads();
   const int hq0 = b * a.Hq + h * a.g;
   splitk_finish<D>(
-      reinterpret_cast<const float*>(smem), C::WARP_B / 4, wst_ml, kQNW, a.g, a.S, chunk, unit, a.o,
+      reinterpret_cast<const float*>(smem), C::WARP_B / 4, wst_ml, kQNW, a.g, a.g, a.S, chunk, unit, a.o,
       [&](int r) { return static_cast<size_t>(hq0 + r) * D; }, [&](int r) { return static_cast<size_t>(hq0 + r); },
       smem_w);
 }

@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kSpNW * 32) draft_sparse_kernel(SpArgs a) {
       issue(i + kSpNST - 1);
     }
     const int s = i % kSpNST;
-    ok = mbar_wait_bounded(&bars[s], (i / kSpNST) & 1, a.flags);
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (i / kSpNST) & 1, a.flags));  // warp-uniform
     if (!ok) break;
     const unsigned char* Ks = ring + s * C::STAGE_B;
     const unsigned char* Vs = Ks + 16 * C::RS;
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kSpNW * 32) draft_sparse_kernel(SpArgs a) {
   __syncthreads();
   const int hq0 = b * a.Hq + h * a.g;
   splitk_finish<D>(
-      reinterpret_cast<const float*>(smem), C::WARP_B / 4, wst_ml, kSpNW, a.g, a.S, chunk, unit, a.o,
+      reinterpret_cast<const float*>(smem), C::WARP_B / 4, wst_ml, kSpNW, a.g, a.g, a.S, chunk, unit, a.o,
       [&](int r) { return static_cast<size_t>(hq0 + r) * D; }, [&](int r) { return static_cast<size_t>(hq0 + r); },
       smem_w);
 }

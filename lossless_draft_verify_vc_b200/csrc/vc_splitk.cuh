@@ -33,10 +33,11 @@ __device__ __forceinline__ float lse_from(float m, float l) {
 // Block-wide: every thread of the block must call it.  `row_out(r)` gives the
 // element offset of row r in `out` (and `row_lse(r)` in lse).
 // wst_o: warp w's rows start at wst_o + w * o_wstride (floats), row r at +r*D.
+// rows_cap: rows reserved per (unit, chunk) in the partial arrays (>= rows).
 template <int D, typename RowOff, typename RowLse>
-__device__ void splitk_finish(const float* wst_o, int o_wstride, const float* wst_ml, int nw, int rows, int S,
-                              int chunk, int unit, const SplitKOut& o, RowOff row_out, RowLse row_lse,
-                              float* smem_w) {
+__device__ void splitk_finish(const float* wst_o, int o_wstride, const float* wst_ml, int nw, int rows,
+                              int rows_cap, int S, int chunk, int unit, const SplitKOut& o, RowOff row_out,
+                              RowLse row_lse, float* smem_w) {
   const int tid = threadIdx.x;
   const int nthr = blockDim.x;
   // per-row block max and weights of each warp
@@ -68,8 +69,8 @@ __device__ void splitk_finish(const float* wst_o, int o_wstride, const float* ws
         o.lse[row_lse(r)] = lse_from(smem_w[nw * rows + 2 * r], smem_w[nw * rows + 2 * r + 1]);
     return;
   }
-  float* po = o.part_o + (static_cast<size_t>(unit) * S + chunk) * rows * D;
-  float* pml = o.part_ml + (static_cast<size_t>(unit) * S + chunk) * rows * 2;
+  float* po = o.part_o + (static_cast<size_t>(unit) * S + chunk) * rows_cap * D;
+  float* pml = o.part_ml + (static_cast<size_t>(unit) * S + chunk) * rows_cap * 2;
   for (int e = tid; e < total; e += nthr) {
     const int r = e / D, d = e - r * D;
     float acc = 0.f;
@@ -88,15 +89,15 @@ __device__ void splitk_finish(const float* wst_o, int o_wstride, const float* ws
   if (ticket != static_cast<uint32_t>(S - 1)) return;
   __threadfence();
   // last block of this unit: merge the S partials
-  const float* uo = o.part_o + static_cast<size_t>(unit) * S * rows * D;
-  const float* uml = o.part_ml + static_cast<size_t>(unit) * S * rows * 2;
+  const float* uo = o.part_o + static_cast<size_t>(unit) * S * rows_cap * D;
+  const float* uml = o.part_ml + static_cast<size_t>(unit) * S * rows_cap * 2;
   for (int r = tid; r < rows; r += nthr) {
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(uml + (s * rows + r) * 2));
+    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(uml + (s * rows_cap + r) * 2));
     float L = 0.f;
     for (int s = 0; s < S; ++s) {
-      const float ms = __ldcg(uml + (s * rows + r) * 2);
-      if (ms != -INFINITY) L += ex2(ms - M) * __ldcg(uml + (s * rows + r) * 2 + 1);
+      const float ms = __ldcg(uml + (s * rows_cap + r) * 2);
+      if (ms != -INFINITY) L += ex2(ms - M) * __ldcg(uml + (s * rows_cap + r) * 2 + 1);
     }
     smem_w[2 * r] = M;
     smem_w[2 * r + 1] = L;
@@ -107,8 +108,8 @@ __device__ void splitk_finish(const float* wst_o, int o_wstride, const float* ws
     const float M = smem_w[2 * r];
     float acc = 0.f;
     for (int s = 0; s < S; ++s) {
-      const float ms = __ldcg(uml + (s * rows + r) * 2);
-      if (ms != -INFINITY) acc += ex2(ms - M) * __ldcg(uo + (static_cast<size_t>(s) * rows + r) * D + d);
+      const float ms = __ldcg(uml + (s * rows_cap + r) * 2);
+      if (ms != -INFINITY) acc += ex2(ms - M) * __ldcg(uo + (static_cast<size_t>(s) * rows_cap + r) * D + d);
     }
     const float L = smem_w[2 * r + 1];
     o.out[row_out(r) + d] = L > 0.f ? acc / L : 0.f;

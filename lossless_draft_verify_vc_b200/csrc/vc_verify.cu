@@ -1,19 +1,444 @@
-// vc_verify.cu -- block verification attention (placeholder until the
-// tcgen05 kernel lands in this file).
-#include "vc_common.cuh"
+// vc_verify.cu -- block verification attention on the sm_100a tensor cores.
+//
+// The verifier checks every drafted position in one pass over the full KV
+// cache and yields one prediction more than there are drafted tokens
+// (devshah.ca page "VeriCache: making lossy KV compression exact", section
+// "The Core Idea"); verification is bound by the interconnect and by FLOPs
+// ("VeriCache: Turning Lossy KV Cache into Lossless LLM Inference",
+// menfem.com, "Key Contributions").  The pages give no kernel.
+//
+// Design.  For one (request, KV head) the nq query rows of all g heads of the
+// GQA group form the MMA's M dimension (row r = position i * g + head), so each
+// K/V tile is read from HBM once for the whole group.  Blocks split the
+// context (split-K) and merge through the workspace.  Per block:
+//   * Q (<= 128 rows) is written once into shared memory in the 128-byte
+//     swizzled K-major layout;
+//   * K and V tiles of BN = 64 keys stream in through a 2-stage ring of tiled
+//     TMA loads (3-D tensor maps, rows past T read as zeros, no multicast);
+//   * one thread issues tcgen05.mma: S = Q K^T into tensor memory (TMEM);
+//   * each of the 128 threads owns one row: it reads its scores from TMEM,
+//     applies the causal mask (row i sees keys 0 .. T - nq + i), updates an
+//     online softmax with lazy rescaling (O is rescaled only when the running
+//     maximum grows by more than 8 in log2 units), and writes P back to TMEM
+//     as a bf16 high part and a bf16 low part (P keeps ~16 bits);
+//   * O += P_hi V + P_lo V as tcgen05.mma with A read from TMEM and V from
+//     shared memory (MN-major), accumulating in TMEM.
+// All waits are bounded; TMEM is always released.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "vc_splitk.cuh"
+#include "vc_tc.cuh"
+
+namespace vc {
+namespace {
+
+constexpr int kVBN = 64;        // keys per tile
+constexpr int kVThreads = 128;  // one warpgroup; thread r owns row r
+constexpr int kVTmemCols = 256;
+// TMEM column map
+constexpr uint32_t kColS = 0;     // S: kVBN fp32 columns
+constexpr uint32_t kColPhi = 64;  // P high part: kVBN / 2 columns (bf16 pairs)
+constexpr uint32_t kColPlo = 96;  // P low part
+constexpr uint32_t kColO = 128;   // O: D fp32 columns
+
+template <int D>
+struct VCfg {
+  static constexpr int HALVES = D / 64;              // 128-byte swizzle atoms across D
+  static constexpr int Q_B = 128 * D * 2;            // 128 rows
+  static constexpr int KV_B = kVBN * D * 2;          // one of K or V per stage
+  static constexpr int STAGE_B = 2 * KV_B;
+  static constexpr int Q_OFF = 0;
+  static constexpr int ST_OFF = Q_B;                 // 2 stages
+  static constexpr int BAR_OFF = ST_OFF + 2 * STAGE_B;
+  static constexpr int SMEM_B = BAR_OFF + 64 + 1024;  // + alignment slack
+  static_assert(2 * STAGE_B >= 128 * D * 4, "stages must hold the fp32 output tile");
+};
+
+struct VArgs {
+  const __nv_bfloat16* q;
+  int64_t T;
+  int nq, Hq, Hkv, g, nqt, RT, C, tiles_per_chunk;
+  float scale_log2;
+  uint32_t* flags;
+  SplitKOut o;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                           const __grid_constant__ CUtensorMap tm_v, VArgs a) {
+  using C = VCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* q_s = smem + C::Q_OFF;
+  unsigned char* st_s = smem + C::ST_OFF;
+  uint64_t* bar_kv = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);  // [2]
+  uint64_t* bar_s = bar_kv + 2;
+  uint64_t* bar_pv = bar_kv + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_kv + 4);
+  __shared__ float wst_ml[128 * 2];
+  __shared__ float smem_w[3 * 128];
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int chunk = blockIdx.x;
+  const int unit = blockIdx.y;  // b * Hkv + h
+  const int rt = blockIdx.z;    // row tile
+  const int b = unit / a.Hkv, h = unit - b * a.Hkv;
+  const int i0 = rt * a.nqt;
+  const int nq_t = min(a.nqt, a.nq - i0);
+  const int M = nq_t * a.g;  // valid rows
+  const int64_t k_begin = static_cast<int64_t>(chunk) * a.tiles_per_chunk * kVBN;
+  const int64_t k_end = min(a.T, k_begin + static_cast<int64_t>(a.tiles_per_chunk) * kVBN);
+  const int ntiles = static_cast<int>((k_end - k_begin + kVBN - 1) / kVBN);
+
+  if (tid == 0) {
+    mbar_init(&bar_kv[0], 1);
+    mbar_init(&bar_kv[1], 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_pv, 1);
+  }
+  fence_mbar_init();
+  if (warp == 0) tc::alloc(tmem_slot, kVTmemCols);
+
+  // ---- Q rows -> shared memory, 128-byte swizzled K-major (zeros past M)
+  {
+    const int r = tid;
+    const bool valid = r < M;
+    const int i = i0 + (valid ? r / a.g : 0);
+    const int hq = h * a.g + (valid ? r % a.g : 0);
+    const uint4* src = reinterpret_cast<const uint4*>(a.q + ((static_cast<size_t>(b) * a.nq + i) * a.Hq + hq) * D);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
+      const int half = c >> 3, k = c & 7;
+      *reinterpret_cast<uint4*>(q_s + half * (128 * 128) + r * 128 + ((k ^ (r & 7)) << 4)) = v;
+    }
+  }
+  fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  auto issue_tile = [&](int i) {  // thread 0 only
+    const int s = i & 1;
+    unsigned char* ks = st_s + s * C::STAGE_B;
+    unsigned char* vs = ks + C::KV_B;
+    const int y = static_cast<int>(k_begin + static_cast<int64_t>(i) * kVBN);
+    mbar_arrive_expect_tx(&bar_kv[s], C::STAGE_B);
+#pragma unroll
+    for (int hf = 0; hf < C::HALVES; ++hf) {
+      tc::tma_load_3d(ks + hf * kVBN * 128, &tm_k, hf * 64, y, unit, &bar_kv[s]);
+      tc::tma_load_3d(vs + hf * kVBN * 128, &tm_v, hf * 64, y, unit, &bar_kv[s]);
+    }
+  };
+
+  constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, kVBN, false);
+  constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(128, D, true);
+  const uint32_t q_base = smem_addr(q_s);
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;  // this warp's TMEM lanes
+
+  // row state
+  const int r = tid;
+  const int i_row = i0 + (r < M ? r / a.g : 0);
+  const int64_t vis_end = a.T - a.nq + i_row + 1;  // keys [0, vis_end) visible to this row
+  float m_run = -INFINITY, l_run = 0.f;
+
+  if (tid == 0) {
+    if (ntiles > 0) issue_tile(0);
+    if (ntiles > 1) issue_tile(1);
+  }
+
+  // Failure handling: every wait is bounded; a thread that sees a timeout sets
+  // its sticky `fail`.  tcgen05.ld / st are warp-collective, so each warp
+  // decides them with __any_sync; the loop exits on a block-wide
+  // __syncthreads_or, so all threads leave together.
+  bool fail = false;
+  constexpr unsigned FULL = 0xffffffffu;
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i & 1;
+    const uint32_t ks_addr = smem_addr(st_s + s * C::STAGE_B);
+    const uint32_t vs_addr = ks_addr + C::KV_B;
+    if (tid == 0 && !fail) {
+      if (!mbar_wait_bounded(&bar_kv[s], (i >> 1) & 1, a.flags)) {
+        fail = true;
+      } else {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int hf = kk >> 2, ko = (kk & 3) * 32;
+          const uint64_t ad = tc::smem_desc_sw128(q_base + hf * (128 * 128) + ko, 16, 1024);
+          const uint64_t bd = tc::smem_desc_sw128(ks_addr + hf * (kVBN * 128) + ko, 16, 1024);
+          tc::mma_ss(tmem + kColS, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        tc::commit(bar_s);
+      }
+    }
+    if (!fail && !mbar_wait_bounded(bar_s, i & 1, a.flags)) fail = true;
+    tc::fence_after_sync();
+    bool wfail = __any_sync(FULL, fail);
+    uint32_t sr[2][32];
+    if (!wfail) {
+      tc::ld32(tmem + lane_off + kColS, sr[0]);
+      tc::ld32(tmem + lane_off + kColS + 32, sr[1]);
+      tc::wait_ld();
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) sr[0][j] = sr[1][j] = 0u;
+    }
+    const int64_t t0 = k_begin + static_cast<int64_t>(i) * kVBN;
+    const int64_t lim = min(vis_end, k_end) - t0;  // keys [t0, t0 + lim) are live
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) * a.scale_log2 : -INFINITY;
+        sr[c][j] = __float_as_uint(x);
+        tmax = fmaxf(tmax, x);
+      }
+    // lazy rescale: keep the stale maximum unless the new one exceeds it by > 8
+    float m_use = m_run;
+    float alpha = 1.f;
+    if (tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY)) {
+      m_use = tmax;
+      if (m_run != -INFINITY) alpha = ex2(m_run - m_use);
+      m_run = m_use;
+    }
+    const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+    uint32_t phi[32], plo[32];
+    float psum = 0.f;
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float p0 = ex2(__uint_as_float(sr[c][j]) - m_sub);
+        const float p1 = ex2(__uint_as_float(sr[c][j + 1]) - m_sub);
+        psum += p0 + p1;
+        const uint32_t hw = pack_bf2(p0, p1);
+        const float2 hf = unpack_bf2(hw);
+        phi[c * 16 + j / 2] = hw;
+        plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
+      }
+    l_run = l_run * alpha + psum;
+    // the previous P.V must be done before P is overwritten / O is touched
+    if (i > 0 && !fail && !mbar_wait_bounded(bar_pv, (i - 1) & 1, a.flags)) fail = true;
+    tc::fence_after_sync();
+    wfail = __any_sync(FULL, fail);
+    if (!wfail && __any_sync(FULL, alpha != 1.f)) {  // warp-uniform: lanes without a new max scale by 1
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tc::ld32(tmem + lane_off + kColO + c0, o);
+        tc::wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+        tc::st32(tmem + lane_off + kColO + c0, o);
+      }
+    }
+    if (!wfail) {
+      tc::st32(tmem + lane_off + kColPhi, phi);
+      tc::st32(tmem + lane_off + kColPlo, plo);
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    if (__syncthreads_or(fail)) break;
+    if (tid == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int j = 0; j < kVBN / 16; ++j) {
+        const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
+        tc::mma_ts(tmem + kColO, tmem + kColPhi + 8 * j, vd, IDESC_PV, (i > 0 || j > 0) ? 1u : 0u);
+      }
+#pragma unroll
+      for (int j = 0; j < kVBN / 16; ++j) {
+        const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
+        tc::mma_ts(tmem + kColO, tmem + kColPlo + 8 * j, vd, IDESC_PV, 1u);
+      }
+      tc::commit(bar_pv);
+      if (i + 2 < ntiles) {
+        // the stage is free once this tile's MMAs are done
+        if (!mbar_wait_bounded(bar_pv, i & 1, a.flags)) {
+          fail = true;
+        } else {
+          fence_proxy_async_smem();
+          issue_tile(i + 2);
+        }
+      }
+    }
+  }
+
+  // ---- drain, read O, release TMEM
+  if (!fail && ntiles > 0 && !mbar_wait_bounded(bar_pv, (ntiles - 1) & 1, a.flags)) fail = true;
+  tc::fence_after_sync();
+  const bool aborted = __syncthreads_or(fail) != 0;
+  if (aborted && tid == 0) {
+    // let MMAs already issued finish before TMEM is released (bounded)
+    mbar_wait_bounded(bar_pv, 0, nullptr, 100000000ull);
+    mbar_wait_bounded(bar_pv, 1, nullptr, 100000000ull);
+    mbar_wait_bounded(bar_s, 0, nullptr, 100000000ull);
+    mbar_wait_bounded(bar_s, 1, nullptr, 100000000ull);
+  }
+  __syncthreads();
+  float* wst_o = reinterpret_cast<float*>(st_s);  // [128][D] fp32 (stages are idle now)
+  const bool ok = !aborted;
+  if (ok && ntiles > 0) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t o[32];
+      tc::ld32(tmem + lane_off + kColO + c0, o);
+      tc::wait_ld();
+      float4* dst = reinterpret_cast<float4*>(wst_o + r * D + c0);
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        dst[j / 4] = make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]), __uint_as_float(o[j + 2]),
+                                 __uint_as_float(o[j + 3]));
+    }
+  } else {
+    for (int c0 = 0; c0 < D; ++c0) wst_o[r * D + c0] = 0.f;
+  }
+  wst_ml[2 * r] = (ok && ntiles > 0) ? m_run : -INFINITY;
+  wst_ml[2 * r + 1] = (ok && ntiles > 0) ? l_run : 0.f;
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::dealloc(tmem, kVTmemCols);
+  }
+  if (!ok) return;  // the flag tells the caller; partials of this unit are left unmerged
+  const int hq0 = h * a.g;
+  const int g = a.g;
+  const int nq = a.nq;
+  const int Hq = a.Hq;
+  splitk_finish<D>(
+      wst_o, 0, wst_ml, 1, M, a.nqt * a.g, a.C, chunk, unit * a.RT + rt, a.o,
+      [&](int rr) {
+        return ((static_cast<size_t>(b) * nq + i0 + rr / g) * Hq + hq0 + rr % g) * D;
+      },
+      [&](int rr) { return (static_cast<size_t>(b) * nq + i0 + rr / g) * Hq + hq0 + rr % g; }, smem_w);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D map over [units][T][D] bf16 with a box of 64 channels x kVBN keys x 1.
+bool make_kv_map(CUtensorMap* m, const void* base, int64_t T, int D, int units) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(units)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(T) * D * 2};
+  cuuint32_t box[3] = {64, kVBN, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct VPlan {
+  int nqt, RT, C, tiles_per_chunk;
+  size_t off_tick, off_ml, off_o, total;
+};
+
+VPlan plan_verify(const vc_attn_shape& sh, int64_t T, int nq) {
+  VPlan p{};
+  const int g = sh.Hq / sh.Hkv;
+  p.nqt = 128 / g;
+  if (p.nqt > nq) p.nqt = nq;
+  p.RT = (nq + p.nqt - 1) / p.nqt;
+  const int units = sh.B * sh.Hkv;
+  const int64_t tiles = (T + kVBN - 1) / kVBN;
+  const int64_t slots = 2LL * sm_count();
+  int64_t c = slots / (static_cast<int64_t>(units) * p.RT);
+  if (c < 1) c = 1;
+  if (c > tiles) c = tiles;
+  int64_t tpc = (tiles + c - 1) / c;
+  p.tiles_per_chunk = static_cast<int>(tpc);
+  p.C = static_cast<int>((tiles + tpc - 1) / tpc);
+  const int rows = p.nqt * g;
+  const size_t nunit = static_cast<size_t>(units) * p.RT;
+  p.off_tick = sizeof(WsHeader);
+  p.off_ml = align_up(p.off_tick + nunit * 4, 256);
+  p.off_o = align_up(p.off_ml + nunit * p.C * rows * 2 * 4, 256);
+  p.total = align_up(p.off_o + nunit * p.C * rows * sh.D * 4, 256);
+  return p;
+}
+
+vc_status check_verify(const vc_attn_shape* sh, int64_t T, int nq, const char* who) {
+  VC_REQUIRE(sh, "%s: null shape", who);
+  VC_REQUIRE(sh->B >= 1 && sh->Hkv >= 1 && sh->Hq >= 1 && sh->Hq % sh->Hkv == 0 && sh->Hq / sh->Hkv <= 8,
+             "%s: need B >= 1, Hq a multiple of Hkv, Hq/Hkv <= 8", who);
+  VC_REQUIRE(sh->D == 64 || sh->D == 128, "%s: head dim must be 64 or 128 (got %d)", who, sh->D);
+  VC_REQUIRE(nq >= 1 && nq <= 32, "%s: need 1 <= nq <= 32 (got %d)", who, nq);
+  VC_REQUIRE(T >= nq && T < (int64_t(1) << 31), "%s: need nq <= T < 2^31", who);
+  VC_REQUIRE(static_cast<int64_t>(sh->B) * sh->Hkv <= 65535, "%s: too many (request, head) pairs", who);
+  return VC_OK;
+}
+
+}  // namespace
+}  // namespace vc
 
 extern "C" {
 
 size_t vc_verify_attn_workspace_size(const vc_attn_shape* shape, int64_t T, int nq) {
-  (void)shape;
-  (void)T;
-  (void)nq;
-  return 0;
+  if (vc::check_verify(shape, T, nq, "vc_verify_attn_workspace_size") != VC_OK) return 0;
+  return vc::plan_verify(*shape, T, nq).total;
 }
 
-vc_status vc_verify_attn(const vc_attn_shape*, const void*, const void*, const void*, int64_t, int, float*, float*,
-                         void*, size_t, void*) {
-  return vc::set_error(VC_ERR_UNSUPPORTED, "vc_verify_attn: not built yet");
+vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* k, const void* v, int64_t T, int nq,
+                         float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  vc_status st = vc::check_verify(shape, T, nq, "vc_verify_attn");
+  if (st != VC_OK) return st;
+  VC_REQUIRE(q && k && v && out && ws, "vc_verify_attn: null pointer argument");
+  VC_REQUIRE(vc::aligned16(q) && vc::aligned16(k) && vc::aligned16(v) && vc::aligned16(out) && vc::aligned16(ws),
+             "vc_verify_attn: q, k, v, out and workspace must be 16-byte aligned");
+  const vc::VPlan p = vc::plan_verify(*shape, T, nq);
+  VC_REQUIRE(ws_bytes >= p.total, "vc_verify_attn: workspace too small (%zu < %zu)", ws_bytes, p.total);
+  const int units = shape->B * shape->Hkv;
+  CUtensorMap tk, tv;
+  if (!vc::make_kv_map(&tk, k, T, shape->D, units) || !vc::make_kv_map(&tv, v, T, shape->D, units))
+    return vc::set_error(VC_ERR_CUDA, "vc_verify_attn: could not encode the K/V tensor maps");
+  char* w = static_cast<char*>(ws);
+  vc::VArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.T = T;
+  a.nq = nq;
+  a.Hq = shape->Hq;
+  a.Hkv = shape->Hkv;
+  a.g = shape->Hq / shape->Hkv;
+  a.nqt = p.nqt;
+  a.RT = p.RT;
+  a.C = p.C;
+  a.tiles_per_chunk = p.tiles_per_chunk;
+  const float sm = shape->sm_scale > 0.f ? shape->sm_scale : 1.0f / sqrtf(static_cast<float>(shape->D));
+  a.scale_log2 = sm * 1.4426950408889634f;
+  a.flags = reinterpret_cast<uint32_t*>(w);
+  a.o.out = out;
+  a.o.lse = lse;
+  a.o.tickets = reinterpret_cast<uint32_t*>(w + p.off_tick);
+  a.o.part_ml = reinterpret_cast<float*>(w + p.off_ml);
+  a.o.part_o = reinterpret_cast<float*>(w + p.off_o);
+  dim3 grid(p.C, units, p.RT);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (shape->D == 128) {
+    using C = vc::VCfg<128>;
+    cudaFuncSetAttribute(vc::verify_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
+    vc::verify_kernel<128><<<grid, vc::kVThreads, C::SMEM_B, s>>>(tk, tv, a);
+  } else {
+    using C = vc::VCfg<64>;
+    cudaFuncSetAttribute(vc::verify_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
+    vc::verify_kernel<64><<<grid, vc::kVThreads, C::SMEM_B, s>>>(tk, tv, a);
+  }
+  return vc::launch_status("vc_verify_attn");
 }
 
 }  // extern "C"
