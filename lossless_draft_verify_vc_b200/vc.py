@@ -119,14 +119,21 @@ def shape(B: int, Hq: int, Hkv: int, D: int, sm_scale: float = 0.0) -> vc_attn_s
 def quant_cache(t: dict) -> vc_quant_cache:
     """Descriptor of a quantised cache given as a dict of CUDA tensors with the
     keys k_codes, v_codes, k_scale, k_zero, v_scale, v_zero, k_res, v_res and
-    ints bits, group, L_q, R, R_cap (the layout documented in vc.h)."""
-    return vc_quant_cache(_p(t["k_codes"]), _p(t["v_codes"]), _p(t["k_scale"]), _p(t["k_zero"]),
-                          _p(t["v_scale"]), _p(t["v_zero"]), _p(t.get("k_res")), _p(t.get("v_res")),
-                          int(t["bits"]), int(t["group"]), int(t["L_q"]), int(t["R"]), int(t["R_cap"]))
+    ints bits, group, L_q, R, R_cap (the layout documented in vc.h).  The
+    descriptor holds raw device pointers; it keeps references to the tensors so
+    they stay allocated while it lives."""
+    d = vc_quant_cache(_p(t["k_codes"]), _p(t["v_codes"]), _p(t["k_scale"]), _p(t["k_zero"]),
+                       _p(t["v_scale"]), _p(t["v_zero"]), _p(t.get("k_res")), _p(t.get("v_res")),
+                       int(t["bits"]), int(t["group"]), int(t["L_q"]), int(t["R"]), int(t["R_cap"]))
+    d._keep = dict(t)
+    return d
 
 
 def sparse_cache(k, v, idx) -> vc_sparse_cache:
-    return vc_sparse_cache(_p(k), _p(v), int(k.shape[2]), _p(idx), int(idx.shape[-1]))
+    """Descriptor of a token-dropped cache (keeps references to its tensors)."""
+    d = vc_sparse_cache(_p(k), _p(v), int(k.shape[2]), _p(idx), int(idx.shape[-1]))
+    d._keep = (k, v, idx)
+    return d
 
 
 def workspace(nbytes: int, device=None) -> torch.Tensor:
