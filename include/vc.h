@@ -162,6 +162,26 @@ VC_API size_t vc_draft_attn_quant_workspace_size(const vc_attn_shape* shape, con
 VC_API vc_status vc_draft_attn_quant(const vc_attn_shape* shape, const vc_quant_cache* cache, const void* q,
                               float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- allocation-free quantised draft attention -----------------------------
+ * The pages have no counterpart to this entry point; it serves callers that
+ * cannot allocate device memory or pass a workspace -- code running inside a
+ * host framework whose memory pool owns all device memory, or latency-
+ * critical paths that must never reach an allocator.  It computes exactly
+ * what vc_draft_attn_quant computes, with the same arguments minus the
+ * workspace: the split-K scratch lives in a fixed device array of
+ * VC_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.  Nothing is allocated.
+ *   - The first call on a device looks up that array's address (with the
+ *     device current); make that first call before any stream capture.
+ *   - All calls share the one array; each call clears the counters it needs
+ *     at zero.  Calls that overlap on the GPU (different streams or host
+ *     threads) race on it and must be serialised by the caller.
+ *   - A call whose scratch would exceed VC_NOALLOC_SCRATCH_BYTES returns
+ *     VC_ERR_WORKSPACE with a message and enqueues nothing. */
+#define VC_NOALLOC_SCRATCH_BYTES (4u << 20)
+VC_API vc_status vc_draft_attn_quant_noalloc(const vc_attn_shape* shape, const vc_quant_cache* cache,
+                                             const void* q, float* out, void* stream);
+
 /* ---- draft attention over a token-dropped cache ----------------------------
  * out[b][hq][:] = softmax(q . K[idx]^T * sm_scale) . V[idx] over the n_keep
  * kept rows of KV head hq / g.

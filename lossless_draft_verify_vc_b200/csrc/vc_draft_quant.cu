@@ -36,6 +36,8 @@
 // Code bits are moved into fp16 mantissas with one LOP3 (magic 0x6400 = 1024)
 // and rescaled with one HFMA2; the assignment of MMA k-slots / rows to
 // channels is chosen so that each lane's codes sit at fixed bit positions.
+#include <mutex>
+
 #include "vc_splitk.cuh"
 
 namespace vc {
@@ -852,6 +854,99 @@ vc_status vc_debug_dequant(const vc_attn_shape* shape, const vc_quant_cache* cac
     vc::debug_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value>(a, *shape, k_out, v_out, s);
   });
   return vc::launch_status("vc_debug_dequant");
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of vc_draft_attn_quant.
+//
+// Some callers cannot call cudaMalloc or hand the library a workspace: code
+// that runs inside a host framework whose memory pool owns every byte of
+// device memory, or latency-critical paths that must never reach an
+// allocator (cudaMalloc may implicitly synchronise the device).  For them
+// this entry point keeps the split-K scratch (flag word, tickets, partials)
+// in a file-scope device array of fixed size, VC_NOALLOC_SCRATCH_BYTES, that
+// every GPU which loads the library holds until the process exits.
+//
+// The array's address is looked up once per device, with that device
+// current, on the first call made on it (cudaGetSymbolAddress); make that
+// first call before any stream capture.  Every call shares the one array:
+// each call clears the words that must start at zero, and calls that
+// overlap on the GPU (other streams, other host threads) race on it.
+namespace vc {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = VC_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device (nullptr + error
+// status on failure).  Host code must not use the symbol's name as an
+// address: it is a host-side stand-in.
+vc_status noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(VC_ERR_CUDA, "vc_draft_attn_quant_noalloc: no usable current device");
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return set_error(VC_ERR_CUDA, "vc_draft_attn_quant_noalloc: cudaGetSymbolAddress failed: %s",
+                       cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return VC_OK;
+}
+
+}  // namespace
+}  // namespace vc
+
+extern "C" {
+
+vc_status vc_draft_attn_quant_noalloc(const vc_attn_shape* shape, const vc_quant_cache* cache, const void* q,
+                                      float* out, void* stream) {
+  vc_status st = vc::check_quant(shape, cache, "vc_draft_attn_quant_noalloc");
+  if (st != VC_OK) return st;
+  VC_REQUIRE(q && out, "vc_draft_attn_quant_noalloc: null q or out");
+  VC_REQUIRE(vc::aligned16(q) && vc::aligned16(out), "vc_draft_attn_quant_noalloc: q and out must be 16-byte aligned");
+  vc::QPlan p{};
+  if (!vc::quant_plan(*shape, *cache, &p))
+    return vc::set_error(VC_ERR_UNSUPPORTED, "vc_draft_attn_quant_noalloc: no kernel for this configuration");
+  if (p.total > vc::kNoAllocScratchBytes)
+    return vc::set_error(VC_ERR_WORKSPACE,
+                         "vc_draft_attn_quant_noalloc: this call needs %zu bytes of scratch, more than the fixed "
+                         "%zu-byte device array; use vc_draft_attn_quant with a caller workspace",
+                         p.total, vc::kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  st = vc::noalloc_scratch(&scratch);
+  if (st != VC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // flag word and tickets must start at zero; partials need no clearing
+  if (cudaMemsetAsync(scratch, 0, p.off_ml, s) != cudaSuccess)
+    return vc::set_error(VC_ERR_CUDA, "vc_draft_attn_quant_noalloc: clearing the scratch failed: %s",
+                         cudaGetErrorString(cudaGetLastError()));
+  vc::QArgs a = vc::make_args(*shape, *cache, q);
+  char* w = static_cast<char*>(scratch);
+  a.S = p.S;
+  a.Sq = p.Sq;
+  a.GPC = p.GPC;
+  a.res_first = p.res;
+  a.flags = reinterpret_cast<uint32_t*>(w);
+  a.o.out = out;
+  a.o.lse = nullptr;
+  a.o.tickets = reinterpret_cast<uint32_t*>(w + p.off_tick);
+  a.o.part_ml = reinterpret_cast<float*>(w + p.off_ml);
+  a.o.part_o = reinterpret_cast<float*>(w + p.off_o);
+  const int nt = a.g <= 4 ? 1 : 2;
+  vc::dispatch(cache->bits, cache->group, shape->D, nt, [&](auto BI, auto GR, auto DD, auto NN) {
+    vc::launch_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value, decltype(NN)::value>(a, p, *shape,
+                                                                                                     s);
+  });
+  return vc::launch_status("vc_draft_attn_quant_noalloc");
 }
 
 }  // extern "C"

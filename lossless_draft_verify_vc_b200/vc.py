@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
             "vc_draft_attn_quant_workspace_size": (c_size_t, [P(vc_attn_shape), P(vc_quant_cache)]),
             "vc_draft_attn_quant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p,
                                             c_size_t, c_void_p]),
+            "vc_draft_attn_quant_noalloc": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p,
+                                                    c_void_p]),
             "vc_draft_attn_sparse_workspace_size": (c_size_t, [P(vc_attn_shape), P(vc_sparse_cache)]),
             "vc_draft_attn_sparse": (c_int, [P(vc_attn_shape), P(vc_sparse_cache), c_void_p, c_void_p, c_void_p,
                                              c_size_t, c_void_p]),
@@ -154,6 +156,13 @@ def vc_draft_attn_quant_workspace_size(sh: vc_attn_shape, qc: vc_quant_cache) ->
 def vc_draft_attn_quant(sh, qc, q, out, ws, stream=None):
     _check(lib().vc_draft_attn_quant(ctypes.byref(sh), ctypes.byref(qc), _p(q), _p(out), _p(ws),
                                      ws.numel() if hasattr(ws, "numel") else 1 << 62, _stream(stream)))
+
+
+def vc_draft_attn_quant_noalloc(sh, qc, q, out, stream=None):
+    """vc_draft_attn_quant without a workspace: the scratch is a fixed device
+    array inside the library (for callers that cannot allocate device memory);
+    calls sharing it must not overlap on the GPU."""
+    _check(lib().vc_draft_attn_quant_noalloc(ctypes.byref(sh), ctypes.byref(qc), _p(q), _p(out), _stream(stream)))
 
 
 def vc_draft_attn_sparse_workspace_size(sh, sc) -> int:
