@@ -33,9 +33,9 @@
 //   scores:  D[token][col] = codes[token][chan] x qfold[chan][col]
 //            col = 2 * head + part (part 0 = high, 1 = low), 4 heads per n-tile
 //   values:  D[chan][col]  = codes^T[chan][token] x pfold[token][col]
-// Code bits are moved into fp16 mantissas with one LOP3 (magic 0x6400 = 1024)
-// and rescaled with one HFMA2; the assignment of MMA k-slots / rows to
-// channels is chosen so that each lane's codes sit at fixed bit positions.
+// Code bits reach the tensor cores as fp16 subnormals (one AND per two codes,
+// see KLane / VLane); the assignment of MMA k-slots / rows to channels is
+// chosen so that each lane's codes sit at fixed bit positions.
 #include <mutex>
 
 #include "vc_splitk.cuh"
@@ -44,7 +44,6 @@ namespace vc {
 namespace {
 
 constexpr int kQNW = 4;  // warps per block
-constexpr uint32_t kMagic = 0x64006400u;
 
 template <int BITS, int G, int D, int NT>
 struct QCfg {
@@ -57,8 +56,8 @@ struct QCfg {
   static constexpr int RS = D * 2 + 16;             // residual smem row stride
   static constexpr int RSTAGE = 32 * RS;            // 16 K + 16 V residual rows
   static constexpr int RING = (NST * QSTAGE > RSTAGE) ? NST * QSTAGE : RSTAGE;
-  static constexpr int PS_FLOATS = 4 * NT * G;      // probabilities [heads][G]
-  static constexpr int WARP_B = RING + PS_FLOATS * 4;
+  static constexpr int PS_B = 2 * (4 * NT * G) * 2;  // p high/low parts, fp16 [heads][G] each
+  static constexpr int WARP_B = RING + PS_B;
   static constexpr int BAR_OFF = kQNW * WARP_B;
   static constexpr int SMEM_B = BAR_OFF + kQNW * NST * 8 + 16;
   static constexpr int KT = D / 16;                 // channel tiles
@@ -85,8 +84,6 @@ struct QArgs {
   SplitKOut o;
 };
 
-__device__ __forceinline__ uint32_t h2_const(float lo, float hi) { return pack_h2(lo, hi); }
-
 // Online-softmax update of one head state with 4 new (already scaled) scores.
 __device__ __forceinline__ float softmax_step(float (&x)[4], float& m_run, float& l_run, int xor0) {
   float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
@@ -108,57 +105,56 @@ __device__ __forceinline__ float softmax_step(float (&x)[4], float& m_run, float
 }
 
 // ---- code extraction shared by the attention kernel and vc_debug_dequant
+//
+// A code is handed to the tensor core as an fp16 SUBNORMAL: AND-ing the packed
+// word with a mask that keeps one code per 16-bit half at bit position pos
+// (0 <= pos <= 9) yields the fp16 value code * 2^(pos - 24) exactly, and the
+// tensor cores multiply subnormal inputs exactly.  One LOP3 per two codes; the
+// power-of-two factors 2^(pos - 24) are folded into the other operand (key
+// side) or undone per output row (value side).
+//
 // Key side (MMA rows = tokens, k = channels): inside a 16-channel tile, k-slots
-// (2t, 2t+1) of lane t hold channels (cA, cB), slots (2t+8, 2t+9) hold
-// (cA+1, cB+1).
+// (2t, 2t+1) of lane t hold channels (cA, cB) at bit position posA, slots
+// (2t+8, 2t+9) hold (cA+1, cB+1) at position posC.
 template <int BITS>
 struct KLane {
-  int cA, cB, shK;
-  uint32_t m1, m2, d1s, d1b, d2s, d2b;
+  int cA, cB, shK, posA, posC;
+  uint32_t m1, m2;
   __device__ __forceinline__ explicit KLane(int tig) {
     cA = BITS == 2 ? 2 * tig : 8 * (tig >> 1) + 2 * (tig & 1);
     cB = cA + (BITS == 2 ? 8 : 4);
     shK = BITS == 2 ? 8 * (tig >> 1) : 8 * (tig & 1);
-    const int p = BITS == 2 ? 4 * (tig & 1) : 0;
-    m1 = BITS == 2 ? (0x00030003u << p) : 0x000F000Fu;
-    m2 = BITS == 2 ? (0x000C000Cu << p) : 0x00F000F0u;
-    const float f1 = BITS == 2 ? (p ? 1.f / 16.f : 1.f) : 1.f;
-    const float f2 = BITS == 2 ? (p ? 1.f / 64.f : 1.f / 4.f) : 1.f / 16.f;
-    d1s = pack_h2(f1, f1);
-    d1b = pack_h2(-1024.f * f1, -1024.f * f1);
-    d2s = pack_h2(f2, f2);
-    d2b = pack_h2(-1024.f * f2, -1024.f * f2);
+    posA = BITS == 2 ? 4 * (tig & 1) : 0;
+    posC = posA + (BITS == 2 ? 2 : 4);
+    m1 = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << posA;
+    m2 = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << posC;
   }
   // word of a token row holding this lane's codes of channel tile kt
   __device__ __forceinline__ int word(int kt, int tig) const { return BITS == 2 ? kt : 2 * kt + (tig >> 1); }
   // A fragment of one 16x16 tile from the words of rows gid and gid + 8
   __device__ __forceinline__ void frag(uint32_t w0, uint32_t w1, uint32_t (&af)[4]) const {
     const uint32_t x0 = w0 >> shK, x1 = w1 >> shK;
-    af[0] = hfma2(and_or(x0, m1, kMagic), d1s, d1b);
-    af[1] = hfma2(and_or(x1, m1, kMagic), d1s, d1b);
-    af[2] = hfma2(and_or(x0, m2, kMagic), d2s, d2b);
-    af[3] = hfma2(and_or(x1, m2, kMagic), d2s, d2b);
+    af[0] = x0 & m1;
+    af[1] = x1 & m1;
+    af[2] = x0 & m2;
+    af[3] = x1 & m2;
   }
 };
 
 // Value side (MMA rows = channels, k = tokens): row gid of a 16-channel tile
-// is channel `row`, row gid + 8 is channel row + 1; k-slots are tokens.
+// is channel `row` (bit position posR0), row gid + 8 is channel row + 1
+// (position posR1); k-slots are tokens.
 template <int BITS>
 struct VLane {
-  int row;
-  uint32_t sel, m1, m2, d1s, d1b, d2s, d2b;
+  int row, posR0, posR1;
+  uint32_t sel, m1, m2;
   __device__ __forceinline__ explicit VLane(int gid) {
     const int k = BITS == 2 ? (gid >> 1) : (gid & 3);
     sel = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
-    const int p = BITS == 2 ? 4 * (gid & 1) : 0;
-    m1 = BITS == 2 ? (0x00030003u << p) : 0x000F000Fu;
-    m2 = BITS == 2 ? (0x000C000Cu << p) : 0x00F000F0u;
-    const float f1 = BITS == 2 ? (p ? 1.f / 16.f : 1.f) : 1.f;
-    const float f2 = BITS == 2 ? (p ? 1.f / 64.f : 1.f / 4.f) : 1.f / 16.f;
-    d1s = pack_h2(f1, f1);
-    d1b = pack_h2(-1024.f * f1, -1024.f * f1);
-    d2s = pack_h2(f2, f2);
-    d2b = pack_h2(-1024.f * f2, -1024.f * f2);
+    posR0 = BITS == 2 ? 4 * (gid & 1) : 0;
+    posR1 = posR0 + (BITS == 2 ? 2 : 4);
+    m1 = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << posR0;
+    m2 = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << posR1;
     row = BITS == 2 ? 4 * (gid >> 1) + 2 * (gid & 1) : 2 * gid;
   }
   __device__ __forceinline__ int word(int mc, int gid) const { return BITS == 2 ? mc : 2 * mc + (gid >> 2); }
@@ -166,23 +162,40 @@ struct VLane {
   __device__ __forceinline__ void frag(uint32_t w0, uint32_t w1, uint32_t w8, uint32_t w9,
                                        uint32_t (&af)[4]) const {
     const uint32_t y01 = prmt(w0, w1, sel), y89 = prmt(w8, w9, sel);
-    af[0] = hfma2(and_or(y01, m1, kMagic), d1s, d1b);
-    af[1] = hfma2(and_or(y01, m2, kMagic), d2s, d2b);
-    af[2] = hfma2(and_or(y89, m1, kMagic), d1s, d1b);
-    af[3] = hfma2(and_or(y89, m2, kMagic), d2s, d2b);
+    af[0] = y01 & m1;
+    af[1] = y01 & m2;
+    af[2] = y89 & m1;
+    af[3] = y89 & m2;
   }
 };
+
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// value scales of tokens (t, t+1) for value group cg as one f16x2 word
+template <int CPG>
+__device__ __forceinline__ uint32_t pair_of(const __half* base, int t, int cg) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(base + t * CPG);
+  if constexpr (CPG == 1) {
+    return w[0];
+  } else if constexpr (CPG == 2) {
+    return prmt(w[0], w[1], cg ? 0x7632 : 0x5410);
+  } else {
+    return prmt(w[cg >> 1], w[2 + (cg >> 1)], (cg & 1) ? 0x7632 : 0x5410);
+  }
+}
 
 // ----------------------------------------------------------- quantised part
 template <int BITS, int G, int D, int NT>
 __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b, int h, int qchunk,
                            float* wst_ml, bool& ok) {
   using C = QCfg<BITS, G, D, NT>;
+  constexpr unsigned FULL = 0xffffffffu;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int part = gid & 1;
   unsigned char* ring = smem + warp * C::WARP_B;
-  float* P_s = reinterpret_cast<float*>(ring + C::RING);
+  __half* Ph = reinterpret_cast<__half*>(ring + C::RING);  // [4 * NT][G] fp16 high parts of p
+  __half* Pl = Ph + 4 * NT * G;                            // low parts
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + warp * C::NST;
 
   const int64_t n_groups = a.L_q / G;
@@ -215,12 +228,14 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
   const KLane<BITS> kl(tig);
   const VLane<BITS> vl(gid);
   const int cA = kl.cA, cB = kl.cB;
-  const uint32_t keep = part ? 0u : 0xffffffffu;  // high columns keep, low columns zero
-  const uint32_t lomask = part ? 0xffffffffu : 0u;
+  const uint32_t lomask = part ? 0xffffffffu : 0u;  // low-part columns
 
-  // ---- query fragments (fp16, exact from bf16), column head = nt*4 + gid/2
-  uint32_t q2[C::KT][NT][2];
+  // ---- query registers (fp16, exact from bf16), column head = nt*4 + gid/2
+  //   q2s: q at the k-slot channels, scaled by 2^-pos of the code encoding
+  //   qb : q at natural channel pairs for the zero-point MMA (high columns only)
+  uint32_t q2s[C::KT][NT][2], qb[C::KT][NT][2];
   {
+    const float fA = pow2i(-kl.posA), fC = pow2i(-kl.posC);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int hh = nt * 4 + (gid >> 1);
@@ -228,13 +243,19 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
       const __nv_bfloat16* qp = a.q + (static_cast<size_t>(b) * a.Hq + h * a.g + (hv ? hh : 0)) * D;
 #pragma unroll
       for (int kt = 0; kt < C::KT; ++kt) {
-        const float qa = __bfloat162float(qp[kt * 16 + cA]), qb = __bfloat162float(qp[kt * 16 + cB]);
+        const float qa = __bfloat162float(qp[kt * 16 + cA]), qbb = __bfloat162float(qp[kt * 16 + cB]);
         const float qc = __bfloat162float(qp[kt * 16 + cA + 1]), qd = __bfloat162float(qp[kt * 16 + cB + 1]);
-        q2[kt][nt][0] = hv ? pack_h2(qa, qb) : 0u;
-        q2[kt][nt][1] = hv ? pack_h2(qc, qd) : 0u;
+        q2s[kt][nt][0] = hv ? pack_h2(qa * fA, qbb * fA) : 0u;
+        q2s[kt][nt][1] = hv ? pack_h2(qc * fC, qd * fC) : 0u;
+        const uint32_t n0 = *reinterpret_cast<const uint32_t*>(qp + kt * 16 + 2 * tig);
+        const uint32_t n8 = *reinterpret_cast<const uint32_t*>(qp + kt * 16 + 8 + 2 * tig);
+        qb[kt][nt][0] = (hv && !part) ? bf2_to_h2(n0) : 0u;
+        qb[kt][nt][1] = (hv && !part) ? bf2_to_h2(n8) : 0u;
       }
     }
   }
+  // the score MMAs accumulate (scores) * 2^-24; undo it together with the softmax scale
+  const float scl = a.scale_log2 * 16777216.0f;
 
   float acc[C::KT][NT][4];
   float vb[NT][4];
@@ -261,7 +282,7 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
       issue(i + C::NST - 1);
     }
     const int s = i % C::NST;
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (i / C::NST) & 1, a.flags))) {  // warp-uniform
+    if (!__all_sync(FULL, mbar_wait_bounded(&bars[s], (i / C::NST) & 1, a.flags))) {  // warp-uniform
       ok = false;
       for (int k = i; k < my_n && k < i + C::NST; ++k)
         mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
@@ -275,30 +296,32 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
     const __half* sv = zk + D;
     const __half* zv = sv + D;
 
-    // (1) fold the key scales into q (high/low fp16 parts) and form the
-    //     zero-point term sum_c q_c z_c as an MMA with z broadcast on rows
+    // (1) fold the key scales into q (fp16 high part in part-0 columns, low
+    //     part in part-1 columns) and the zero-point term sum_c q_c z_c
     uint32_t qf[C::KT][NT][2];
-    float kbias[NT][4];
+    float kb[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) kbias[nt][0] = kbias[nt][1] = kbias[nt][2] = kbias[nt][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt) kb[nt][0] = kb[nt][1] = kb[nt][2] = kb[nt][3] = 0.f;
 #pragma unroll
     for (int kt = 0; kt < C::KT; ++kt) {
       const uint32_t sw1 = *reinterpret_cast<const uint32_t*>(sk + kt * 16 + cA);
       const uint32_t sw2 = *reinterpret_cast<const uint32_t*>(sk + kt * 16 + cB);
-      const uint32_t zw1 = *reinterpret_cast<const uint32_t*>(zk + kt * 16 + cA);
-      const uint32_t zw2 = *reinterpret_cast<const uint32_t*>(zk + kt * 16 + cB);
       const uint32_t sA = prmt(sw1, sw2, 0x5410), sC = prmt(sw1, sw2, 0x7632);
-      const uint32_t zA = prmt(zw1, zw2, 0x5410), zC = prmt(zw1, zw2, 0x7632);
-      const uint32_t za[4] = {zA, zA, zC, zC};
+      const uint32_t z0 = *reinterpret_cast<const uint32_t*>(zk + kt * 16 + 2 * tig);
+      const uint32_t z8 = *reinterpret_cast<const uint32_t*>(zk + kt * 16 + 8 + 2 * tig);
+      const uint32_t za[4] = {z0, z0, z8, z8};
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t qa = q2[kt][nt][0], qc = q2[kt][nt][1];
-        const uint32_t qan = (qa ^ 0x80008000u) & lomask, qcn = (qc ^ 0x80008000u) & lomask;
-        qf[kt][nt][0] = hfma2(qa, sA, hmul2(qan, sA));
-        qf[kt][nt][1] = hfma2(qc, sC, hmul2(qcn, sC));
-        mma_f16(kbias[nt], za, qa & keep, qc & keep);
+        const uint32_t qa = q2s[kt][nt][0], qc = q2s[kt][nt][1];
+        qf[kt][nt][0] = hfma2(qa, sA, hmul2((qa ^ 0x80008000u) & lomask, sA));
+        qf[kt][nt][1] = hfma2(qc, sC, hmul2((qc ^ 0x80008000u) & lomask, sC));
+        mma_f16(kb[nt], za, qb[kt][nt][0], qb[kt][nt][1]);
       }
     }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kb[nt][e] *= 5.9604644775390625e-8f;  // 2^-24
 
     // (2) 32-token sub-blocks: scores, softmax, P . V
 #pragma unroll 1
@@ -307,60 +330,84 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         const int r0 = sb * 32 + mt * 16 + gid;
-        const uint32_t* row0 = kcw + r0 * C::WPR;
-        const uint32_t* row1 = row0 + 8 * C::WPR;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sc[mt][nt][e] = kbias[nt][e];
+          for (int e = 0; e < 4; ++e) sc[mt][nt][e] = kb[nt][e];
+        if constexpr (BITS == 2) {
+          uint32_t w0[C::WPR], w1[C::WPR];
 #pragma unroll
-        for (int kt = 0; kt < C::KT; ++kt) {
-          const int wi = kl.word(kt, tig);
-          uint32_t af[4];
-          kl.frag(row0[wi], row1[wi], af);
+          for (int v = 0; v < C::WPR / 4; ++v) {
+            const uint4 x = reinterpret_cast<const uint4*>(kcw + r0 * C::WPR)[v];
+            const uint4 y = reinterpret_cast<const uint4*>(kcw + (r0 + 8) * C::WPR)[v];
+            w0[4 * v] = x.x, w0[4 * v + 1] = x.y, w0[4 * v + 2] = x.z, w0[4 * v + 3] = x.w;
+            w1[4 * v] = y.x, w1[4 * v + 1] = y.y, w1[4 * v + 2] = y.z, w1[4 * v + 3] = y.w;
+          }
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_f16(sc[mt][nt], af, qf[kt][nt][0], qf[kt][nt][1]);
+          for (int kt = 0; kt < C::KT; ++kt) {
+            uint32_t af[4];
+            kl.frag(w0[kt], w1[kt], af);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_f16(sc[mt][nt], af, qf[kt][nt][0], qf[kt][nt][1]);
+          }
+        } else {
+          const uint32_t* row0 = kcw + r0 * C::WPR + (tig >> 1);
+          const uint32_t* row1 = row0 + 8 * C::WPR;
+#pragma unroll
+          for (int kt = 0; kt < C::KT; ++kt) {
+            uint32_t af[4];
+            kl.frag(row0[2 * kt], row1[2 * kt], af);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_f16(sc[mt][nt], af, qf[kt][nt][0], qf[kt][nt][1]);
+          }
         }
       }
       // softmax per head nt*4 + tig over tokens sb*32 + {gid, gid+8, gid+16, gid+24}
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float x[4] = {(sc[0][nt][0] + sc[0][nt][1]) * a.scale_log2, (sc[0][nt][2] + sc[0][nt][3]) * a.scale_log2,
-                      (sc[1][nt][0] + sc[1][nt][1]) * a.scale_log2, (sc[1][nt][2] + sc[1][nt][3]) * a.scale_log2};
+        float x[4] = {(sc[0][nt][0] + sc[0][nt][1]) * scl, (sc[0][nt][2] + sc[0][nt][3]) * scl,
+                      (sc[1][nt][0] + sc[1][nt][1]) * scl, (sc[1][nt][2] + sc[1][nt][3]) * scl};
         const float alpha = softmax_step(x, m_run[nt], l_run[nt], 4);
+        if (__any_sync(FULL, alpha != 1.f)) {
 #pragma unroll
-        for (int mc = 0; mc < C::KT; ++mc) {
-          acc[mc][nt][0] *= alpha;
-          acc[mc][nt][1] *= alpha;
-          acc[mc][nt][2] *= alpha;
-          acc[mc][nt][3] *= alpha;
+          for (int mc = 0; mc < C::KT; ++mc) {
+            acc[mc][nt][0] *= alpha;
+            acc[mc][nt][1] *= alpha;
+            acc[mc][nt][2] *= alpha;
+            acc[mc][nt][3] *= alpha;
+          }
+          vb[nt][0] *= alpha;
+          vb[nt][1] *= alpha;
+          vb[nt][2] *= alpha;
+          vb[nt][3] *= alpha;
         }
-        vb[nt][0] *= alpha;
-        vb[nt][1] *= alpha;
-        vb[nt][2] *= alpha;
-        vb[nt][3] *= alpha;
-        float* ps = P_s + (nt * 4 + tig) * G + sb * 32 + gid;
-        ps[0] = x[0];
-        ps[8] = x[1];
-        ps[16] = x[2];
-        ps[24] = x[3];
+        // p as fp16 high + low parts, split once here for the value side
+        const uint32_t h01 = pack_h2(x[0], x[1]), h23 = pack_h2(x[2], x[3]);
+        const float2 f01 = unpack_h2(h01), f23 = unpack_h2(h23);
+        const uint32_t l01 = pack_h2(x[0] - f01.x, x[1] - f01.y), l23 = pack_h2(x[2] - f23.x, x[3] - f23.y);
+        unsigned short* ph = reinterpret_cast<unsigned short*>(Ph + (nt * 4 + tig) * G + sb * 32 + gid);
+        unsigned short* pl = reinterpret_cast<unsigned short*>(Pl + (nt * 4 + tig) * G + sb * 32 + gid);
+        ph[0] = static_cast<unsigned short>(h01);
+        ph[8] = static_cast<unsigned short>(h01 >> 16);
+        ph[16] = static_cast<unsigned short>(h23);
+        ph[24] = static_cast<unsigned short>(h23 >> 16);
+        pl[0] = static_cast<unsigned short>(l01);
+        pl[8] = static_cast<unsigned short>(l01 >> 16);
+        pl[16] = static_cast<unsigned short>(l23);
+        pl[24] = static_cast<unsigned short>(l23 >> 16);
       }
       __syncwarp();
 #pragma unroll
       for (int ktt = 0; ktt < 2; ++ktt) {
         const int t0 = sb * 32 + ktt * 16 + 2 * tig;  // tokens t0, t0+1, t0+8, t0+9
-        // probabilities as fp16 high/low parts for column head nt*4 + gid/2
-        uint32_t ph[NT][2], pl[NT][2];
+        uint32_t ph01[NT], ph89[NT], pl01[NT], pl89[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const float* pp = P_s + (nt * 4 + (gid >> 1)) * G + t0;
-          const float2 p01 = *reinterpret_cast<const float2*>(pp);
-          const float2 p89 = *reinterpret_cast<const float2*>(pp + 8);
-          ph[nt][0] = pack_h2(p01.x, p01.y);
-          ph[nt][1] = pack_h2(p89.x, p89.y);
-          const float2 f01 = unpack_h2(ph[nt][0]), f89 = unpack_h2(ph[nt][1]);
-          pl[nt][0] = pack_h2(p01.x - f01.x, p01.y - f01.y);
-          pl[nt][1] = pack_h2(p89.x - f89.x, p89.y - f89.y);
+          const int hh = nt * 4 + (gid >> 1);
+          ph01[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0);
+          ph89[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0 + 8);
+          pl01[nt] = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0);
+          pl89[nt] = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0 + 8);
         }
         // value zero-point term: A = z_v^T (row = value group gid), B = p
         {
@@ -375,34 +422,31 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
           }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
-            mma_f16(vb[nt], za, part ? pl[nt][0] : ph[nt][0], part ? pl[nt][1] : ph[nt][1]);
+            mma_f16(vb[nt], za, part ? pl01[nt] : ph01[nt], part ? pl89[nt] : ph89[nt]);
         }
-        // code words of the four tokens
-        const uint32_t* w0 = vcw + t0 * C::WPR;
-        const uint32_t* w1 = w0 + C::WPR;
-        const uint32_t* w8 = w0 + 8 * C::WPR;
-        const uint32_t* w9 = w0 + 9 * C::WPR;
+        const uint32_t* T0 = vcw + t0 * C::WPR;
+        const uint32_t* T1 = T0 + C::WPR;
+        const uint32_t* T8 = T0 + 8 * C::WPR;
+        const uint32_t* T9 = T0 + 9 * C::WPR;
 #pragma unroll
         for (int cg = 0; cg < C::CPG; ++cg) {
           // folded p*s for this value group: high part (part 0) or low part (part 1)
-          const uint32_t s01 = __half_as_ushort(sv[t0 * C::CPG + cg]) |
-                               (static_cast<uint32_t>(__half_as_ushort(sv[(t0 + 1) * C::CPG + cg])) << 16);
-          const uint32_t s89 = __half_as_ushort(sv[(t0 + 8) * C::CPG + cg]) |
-                               (static_cast<uint32_t>(__half_as_ushort(sv[(t0 + 9) * C::CPG + cg])) << 16);
+          const uint32_t s01 = pair_of<C::CPG>(sv, t0, cg);
+          const uint32_t s89 = pair_of<C::CPG>(sv, t0 + 8, cg);
           uint32_t pf[NT][2];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const uint32_t phn0 = (ph[nt][0] ^ 0x80008000u) & lomask, phn1 = (ph[nt][1] ^ 0x80008000u) & lomask;
-            const uint32_t plm0 = pl[nt][0] & lomask, plm1 = pl[nt][1] & lomask;
-            pf[nt][0] = hfma2(plm0, s01, hfma2(ph[nt][0], s01, hmul2(phn0, s01)));
-            pf[nt][1] = hfma2(plm1, s89, hfma2(ph[nt][1], s89, hmul2(phn1, s89)));
+            pf[nt][0] = hfma2(pl01[nt] & lomask, s01,
+                              hfma2(ph01[nt], s01, hmul2((ph01[nt] ^ 0x80008000u) & lomask, s01)));
+            pf[nt][1] = hfma2(pl89[nt] & lomask, s89,
+                              hfma2(ph89[nt], s89, hmul2((ph89[nt] ^ 0x80008000u) & lomask, s89)));
           }
 #pragma unroll
           for (int mq = 0; mq < G / 16; ++mq) {
             const int mc = cg * (G / 16) + mq;  // 16-channel tile
             const int wi = vl.word(mc, gid);
             uint32_t af[4];
-            vl.frag(w0[wi], w1[wi], w8[wi], w9[wi], af);
+            vl.frag(T0[wi], T1[wi], T8[wi], T9[wi], af);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) mma_f16(acc[mc][nt], af, pf[nt][0], pf[nt][1]);
           }
@@ -415,22 +459,23 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
   // ---- this warp's state -> its own (finished) ring, natural channel order
   __syncwarp();
   float* my_o = reinterpret_cast<float*>(ring);  // [g][D]
+  const float u0 = pow2i(24 - vl.posR0), u1 = pow2i(24 - vl.posR1);  // undo the code encoding
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int hh = nt * 4 + tig;
     float l = l_run[nt];
-    l += __shfl_xor_sync(0xffffffffu, l, 4);
-    l += __shfl_xor_sync(0xffffffffu, l, 8);
-    l += __shfl_xor_sync(0xffffffffu, l, 16);
+    l += __shfl_xor_sync(FULL, l, 4);
+    l += __shfl_xor_sync(FULL, l, 8);
+    l += __shfl_xor_sync(FULL, l, 16);
     const float vbs = vb[nt][0] + vb[nt][1];  // value-zero term of group gid, head hh
 #pragma unroll
     for (int mc = 0; mc < C::KT; ++mc) {
       const int cg = mc * 16 / G;
-      const float zb = __shfl_sync(0xffffffffu, vbs, cg * 4 + tig);
+      const float zb = __shfl_sync(FULL, vbs, cg * 4 + tig);
       if (hh < a.g) {
         float* wo = my_o + hh * D + mc * 16 + vl.row;
-        wo[0] = acc[mc][nt][0] + acc[mc][nt][1] + zb;
-        wo[1] = acc[mc][nt][2] + acc[mc][nt][3] + zb;
+        wo[0] = (acc[mc][nt][0] + acc[mc][nt][1]) * u0 + zb;
+        wo[1] = (acc[mc][nt][2] + acc[mc][nt][3]) * u1 + zb;
       }
     }
     if (hh < a.g && gid == 0) {
@@ -574,7 +619,7 @@ __device__ void residual_role(const QArgs& a, unsigned char* smem, int unit, int
 
 
 template <int BITS, int G, int D, int NT>
-__global__ void __launch_bounds__(kQNW * 32) draft_quant_kernel(QArgs a) {
+__global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kernel(QArgs a) {
   using C = QCfg<BITS, G, D, NT>;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ float wst_ml[kQNW * 8 * 2];
@@ -623,9 +668,10 @@ __global__ void __launch_bounds__(32) debug_dequant_kernel(QArgs a, float* ko, f
       kl.frag(kc[t * WPR + wi], kc[(t + 8) * WPR + wi], af);
       const int ch[4][2] = {{kl.cA, kl.cB}, {kl.cA, kl.cB}, {kl.cA + 1, kl.cB + 1}, {kl.cA + 1, kl.cB + 1}};
       const int64_t tok[4] = {t, t + 8, t, t + 8};
+      const float undo[4] = {pow2i(24 - kl.posA), pow2i(24 - kl.posA), pow2i(24 - kl.posC), pow2i(24 - kl.posC)};
       for (int e = 0; e < 4; ++e) {
         const float2 code = unpack_h2(af[e]);
-        const float cc[2] = {code.x, code.y};
+        const float cc[2] = {code.x * undo[e], code.y * undo[e]};
         for (int u = 0; u < 2; ++u) {
           const int c = kt * 16 + ch[e][u];
           kou[tok[e] * D + c] = __fmaf_rn(cc[u], __half2float(sk[c]), __half2float(zk[c]));
@@ -642,9 +688,10 @@ __global__ void __launch_bounds__(32) debug_dequant_kernel(QArgs a, float* ko, f
       vl.frag(vc[t0 * WPR + wi], vc[(t0 + 1) * WPR + wi], vc[(t0 + 8) * WPR + wi], vc[(t0 + 9) * WPR + wi], af);
       const int chs[4] = {vl.row, vl.row + 1, vl.row, vl.row + 1};
       const int64_t tk[4][2] = {{t0, t0 + 1}, {t0, t0 + 1}, {t0 + 8, t0 + 9}, {t0 + 8, t0 + 9}};
+      const float undo[4] = {pow2i(24 - vl.posR0), pow2i(24 - vl.posR1), pow2i(24 - vl.posR0), pow2i(24 - vl.posR1)};
       for (int e = 0; e < 4; ++e) {
         const float2 code = unpack_h2(af[e]);
-        const float cc[2] = {code.x, code.y};
+        const float cc[2] = {code.x * undo[e], code.y * undo[e]};
         const int c = mc * 16 + chs[e];
         for (int u = 0; u < 2; ++u) {
           const int64_t tt = tk[e][u];
