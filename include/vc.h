@@ -220,6 +220,114 @@ VC_API size_t vc_accept_workspace_size(int B, int K, int V);
 VC_API vc_status vc_accept(const void* logits, int dtype, int B, int K, int V, const int32_t* draft, int32_t* target,
                     int32_t* accept_len, int32_t* correction, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- host -> HBM streaming of the full KV for verification ----------------
+ * The full cache may live in host memory and be brought to the GPU only for
+ * verification (devshah.ca page, "Verifying Without Giving Back the
+ * Speedup"; menfem.com source page, "Key Contributions": the verifier reads
+ * the full KV from CPU memory over the interconnect).  A vc_kvstream moves one
+ * layer at a time into one of two caller-owned device staging slots with
+ * cudaMemcpyAsync on a copy stream, so the copy of layer l + 1 overlaps the
+ * verification of layer l.  Layer l always uses slot l % 2.  Everything is
+ * stream-ordered with events; no call blocks the host except destroy.
+ *   host_k[l], host_v[l]  pinned host memory, bytes_per_layer each (caller-owned)
+ *   dev_k[0..1], dev_v[0..1]  device staging slots, bytes_per_layer each
+ *   copy_stream  the stream that carries the copies (caller-owned)
+ * Protocol per layer l: prefetch(l) (enqueues the copies once the slot's
+ * previous layer was released), acquire(l, compute) (the compute stream
+ * waits for the copies; returns the slot's pointers), launch the work,
+ * release(l, compute) (the slot may be overwritten after the work).  Calling
+ * acquire on a layer that was not prefetched, or prefetch on a slot whose
+ * previous layer was not yet released, returns VC_ERR_INVALID_ARG. */
+typedef struct vc_kvstream vc_kvstream;
+VC_API vc_status vc_kvstream_create(vc_kvstream** out, int n_layers, const void* const* host_k,
+                                    const void* const* host_v, size_t bytes_per_layer, void* const* dev_k,
+                                    void* const* dev_v, void* copy_stream);
+VC_API vc_status vc_kvstream_prefetch(vc_kvstream* s, int layer);
+VC_API vc_status vc_kvstream_acquire(vc_kvstream* s, int layer, void* compute_stream, const void** k,
+                                     const void** v);
+VC_API vc_status vc_kvstream_release(vc_kvstream* s, int layer, void* compute_stream);
+VC_API vc_status vc_kvstream_destroy(vc_kvstream* s);
+
+/* ---- cross-request staggering scheduler -------------------------------------
+ * Drafting is bound by HBM bandwidth and verification by the host link, so
+ * the pages interleave different requests' draft and verify phases instead
+ * of running all drafts and then all verifications (devshah.ca page,
+ * "Verifying Without Giving Back the Speedup", Figure 2; menfem.com source
+ * page, "Key Contributions").  vc_sched runs rounds for n requests:
+ *   draft   draft_len x n_layers calls of the request's draft attention on the
+ *           request's stream;
+ *   verify  n_layers of host-streamed verification (vc_kvstream over the
+ *           shared copy stream, kernels on the request's stream);
+ *   accept  one vc_accept call.
+ * VC_SCHED_LOCKSTEP: every request drafts, then (after all drafts) the
+ * verifications run one after another; the next round starts when all are
+ * done.  VC_SCHED_STAGGER: a request starts verifying as soon as its own
+ * draft is done and the link is free, and starts its next round's draft as
+ * soon as its own round is done, so one request's verification overlaps
+ * other requests' drafting.  The host polls events (never blocks a device)
+ * and gives up with VC_ERR_TIMEOUT after timeout_ms.  Inputs and outputs
+ * of every call are the caller's (device pointers, as in the calls above);
+ * the round's synthetic inputs do not change between rounds. */
+#define VC_DRAFT_QUANT 0
+#define VC_DRAFT_SPARSE 1
+#define VC_SCHED_LOCKSTEP 0
+#define VC_SCHED_STAGGER 1
+typedef struct vc_sched_request {
+  vc_attn_shape shape;               /* B, Hq, Hkv, D, sm_scale of the request */
+  int draft_kind;                    /* VC_DRAFT_QUANT or VC_DRAFT_SPARSE */
+  const vc_quant_cache* qcaches;     /* host array [n_layers] (quant) */
+  const vc_sparse_cache* scaches;    /* host array [n_layers] (sparse) */
+  const void* draft_q;               /* bf16 [draft_len][n_layers][B][Hq][D] */
+  float* draft_out;                  /* fp32 [B][Hq][D] */
+  void* draft_ws;
+  size_t draft_ws_bytes;
+  const void* const* host_k;         /* host array [n_layers] of pinned host pointers */
+  const void* const* host_v;
+  size_t kv_bytes_per_layer;         /* B * Hkv * T * D * 2 */
+  void* stage_k[2];                  /* device staging slots, kv_bytes_per_layer each */
+  void* stage_v[2];
+  const void* verify_q;              /* bf16 [n_layers][B][nq][Hq][D] */
+  float* verify_out;                 /* fp32 [B][nq][Hq][D] (last layer's result remains) */
+  void* verify_ws;
+  size_t verify_ws_bytes;
+  int64_t T;
+  int nq;
+  const void* logits;                /* [B][draft_len + 1][V], dtype logits_dtype */
+  int logits_dtype;
+  int V;
+  const int32_t* draft_tokens;       /* [B][draft_len] */
+  int32_t* target;                   /* [B][draft_len + 1] */
+  int32_t* accept_len;               /* [B] */
+  int32_t* correction;               /* [B] */
+  void* accept_ws;
+  size_t accept_ws_bytes;
+  void* stream;                      /* the request's compute stream */
+} vc_sched_request;
+typedef struct vc_sched_stats {
+  double elapsed_ms;      /* device time from the first enqueued work to the last completion */
+  double link_busy_ms;    /* device time the copy stream spent copying */
+  double draft_ms;        /* summed device time of the draft phases */
+  double verify_ms;       /* summed device time of the verify + accept phases */
+  int rounds;
+  int requests;
+} vc_sched_stats;
+typedef struct vc_sched vc_sched;
+VC_API vc_status vc_sched_create(vc_sched** out, int n_requests, const vc_sched_request* reqs, int n_layers,
+                                 int draft_len, int policy, void* copy_stream, int timeout_ms);
+VC_API vc_status vc_sched_run_rounds(vc_sched* s, int n_rounds, vc_sched_stats* stats);
+VC_API vc_status vc_sched_destroy(vc_sched* s);
+
+/* Host-only model of the same policy on a simulated timeline (no GPU): each
+ * request's draft takes draft_ms of the GPU (drafts share the GPU one at a
+ * time) and its verification verify_ms of the link (one at a time).  Writes
+ * the finishing time of the last round to *makespan_ms.  A request index
+ * `never_done` >= 0 makes that request's first verification never complete,
+ * which exercises the timeout path (VC_ERR_TIMEOUT after timeout_ms of
+ * simulated time).  Used by the CPU tests of the policy. */
+VC_API vc_status vc_sched_simulate(int n_requests, int n_rounds, int policy, const double* draft_ms,
+                                   const double* verify_ms, int never_done, double timeout_ms,
+                                   double* makespan_ms);
+
 /* ---- workspace flags -------------------------------------------------------
  * Copies the device-side flag word of a workspace to *host_flags and clears
  * it (a synchronous read on `stream`).  Returns VC_OK or VC_ERR_CUDA. */

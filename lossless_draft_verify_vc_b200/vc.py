@@ -49,6 +49,26 @@ class vc_sparse_cache(Structure):
     _fields_ = [("k", c_void_p), ("v", c_void_p), ("T_store", c_int64), ("idx", c_void_p), ("n_keep", c_int)]
 
 
+class vc_sched_request(Structure):
+    _fields_ = [("shape", vc_attn_shape), ("draft_kind", c_int), ("qcaches", c_void_p), ("scaches", c_void_p),
+                ("draft_q", c_void_p), ("draft_out", c_void_p), ("draft_ws", c_void_p), ("draft_ws_bytes", c_size_t),
+                ("host_k", c_void_p), ("host_v", c_void_p), ("kv_bytes_per_layer", c_size_t),
+                ("stage_k", c_void_p * 2), ("stage_v", c_void_p * 2), ("verify_q", c_void_p),
+                ("verify_out", c_void_p), ("verify_ws", c_void_p), ("verify_ws_bytes", c_size_t), ("T", c_int64),
+                ("nq", c_int), ("logits", c_void_p), ("logits_dtype", c_int), ("V", c_int),
+                ("draft_tokens", c_void_p), ("target", c_void_p), ("accept_len", c_void_p),
+                ("correction", c_void_p), ("accept_ws", c_void_p), ("accept_ws_bytes", c_size_t),
+                ("stream", c_void_p)]
+
+
+class vc_sched_stats(Structure):
+    _fields_ = [("elapsed_ms", ctypes.c_double), ("link_busy_ms", ctypes.c_double), ("draft_ms", ctypes.c_double),
+                ("verify_ms", ctypes.c_double), ("rounds", c_int), ("requests", c_int)]
+
+
+VC_DRAFT_QUANT, VC_DRAFT_SPARSE = 0, 1
+VC_SCHED_LOCKSTEP, VC_SCHED_STAGGER = 0, 1
+
 _lib = None
 
 
@@ -79,6 +99,18 @@ def lib() -> ctypes.CDLL:
                                   c_void_p, c_size_t, c_void_p]),
             "vc_workspace_flags": (c_int, [c_void_p, c_size_t, P(c_uint32), c_void_p]),
             "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
+            "vc_kvstream_create": (c_int, [P(c_void_p), c_int, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p,
+                                           c_void_p]),
+            "vc_kvstream_prefetch": (c_int, [c_void_p, c_int]),
+            "vc_kvstream_acquire": (c_int, [c_void_p, c_int, c_void_p, P(c_void_p), P(c_void_p)]),
+            "vc_kvstream_release": (c_int, [c_void_p, c_int, c_void_p]),
+            "vc_kvstream_destroy": (c_int, [c_void_p]),
+            "vc_sched_create": (c_int, [P(c_void_p), c_int, P(vc_sched_request), c_int, c_int, c_int, c_void_p,
+                                        c_int]),
+            "vc_sched_run_rounds": (c_int, [c_void_p, c_int, P(vc_sched_stats)]),
+            "vc_sched_destroy": (c_int, [c_void_p]),
+            "vc_sched_simulate": (c_int, [c_int, c_int, c_int, P(ctypes.c_double), P(ctypes.c_double), c_int,
+                                          ctypes.c_double, P(ctypes.c_double)]),
             "vc_debug_gather": (c_int, [P(vc_attn_shape), P(vc_sparse_cache), c_void_p, c_void_p, c_void_p,
                                         c_size_t, c_void_p]),
         }
@@ -208,3 +240,125 @@ def vc_debug_dequant(sh, qc, k_out, v_out, stream=None):
 def vc_debug_gather(sh, sc, k_out, v_out, ws=None, stream=None):
     _check(lib().vc_debug_gather(ctypes.byref(sh), ctypes.byref(sc), _p(k_out), _p(v_out), _p(ws),
                                  0 if ws is None else ws.numel(), _stream(stream)))
+
+
+# ---- host -> HBM layer streaming ------------------------------------------------
+
+class KvStream:
+    """Handle of a vc_kvstream (double-buffered per-layer host -> device copies).
+
+    host_k / host_v: lists of pinned host tensors, one per layer; dev_k / dev_v:
+    two device staging tensors each; copy_stream: a torch.cuda.Stream."""
+
+    def __init__(self, host_k, host_v, dev_k, dev_v, copy_stream):
+        n = len(host_k)
+        self._keep = (host_k, host_v, dev_k, dev_v, copy_stream)
+        self._hk = (c_void_p * n)(*[_p(t) for t in host_k])
+        self._hv = (c_void_p * n)(*[_p(t) for t in host_v])
+        self._dk = (c_void_p * 2)(*[_p(t) for t in dev_k])
+        self._dv = (c_void_p * 2)(*[_p(t) for t in dev_v])
+        nbytes = host_k[0].numel() * host_k[0].element_size()
+        h = c_void_p()
+        _check(lib().vc_kvstream_create(ctypes.byref(h), n, self._hk, self._hv, nbytes, self._dk, self._dv,
+                                        _stream(copy_stream)))
+        self.h = h
+
+    def prefetch(self, layer: int):
+        _check(lib().vc_kvstream_prefetch(self.h, int(layer)))
+
+    def acquire(self, layer: int, stream=None):
+        k, v = c_void_p(), c_void_p()
+        _check(lib().vc_kvstream_acquire(self.h, int(layer), _stream(stream), ctypes.byref(k), ctypes.byref(v)))
+        return k.value, v.value
+
+    def release(self, layer: int, stream=None):
+        _check(lib().vc_kvstream_release(self.h, int(layer), _stream(stream)))
+
+    def close(self):
+        if self.h:
+            _check(lib().vc_kvstream_destroy(self.h))
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ---- stagger scheduler ----------------------------------------------------------
+
+class Sched:
+    """Handle of a vc_sched.  `requests` is a list of vc_sched_request structs
+    (see make_sched_request); keep-alive references travel with them."""
+
+    def __init__(self, requests, n_layers: int, draft_len: int, policy: int, copy_stream, timeout_ms: int = 60000):
+        n = len(requests)
+        self._arr = (vc_sched_request * n)(*requests)
+        self._keep = [getattr(r, "_keep", None) for r in requests] + [copy_stream]
+        h = c_void_p()
+        _check(lib().vc_sched_create(ctypes.byref(h), n, self._arr, int(n_layers), int(draft_len), int(policy),
+                                     _stream(copy_stream), int(timeout_ms)))
+        self.h = h
+
+    def run_rounds(self, n_rounds: int) -> dict:
+        st = vc_sched_stats()
+        _check(lib().vc_sched_run_rounds(self.h, int(n_rounds), ctypes.byref(st)))
+        return dict(elapsed_ms=st.elapsed_ms, link_busy_ms=st.link_busy_ms, draft_ms=st.draft_ms,
+                    verify_ms=st.verify_ms, rounds=st.rounds, requests=st.requests)
+
+    def close(self):
+        if self.h:
+            _check(lib().vc_sched_destroy(self.h))
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def make_sched_request(sh, kind, caches, draft_q, draft_out, draft_ws, host_k, host_v, stage_k, stage_v, verify_q,
+                       verify_out, verify_ws, T, nq, logits, V, draft_tokens, target, accept_len, correction,
+                       accept_ws, stream):
+    """Marshal one request of the scheduler; `caches` are per-layer
+    vc_quant_cache (kind VC_DRAFT_QUANT) or vc_sparse_cache descriptors."""
+    n = len(caches)
+    carr = ((vc_quant_cache if kind == VC_DRAFT_QUANT else vc_sparse_cache) * n)(*caches)
+    hk = (c_void_p * n)(*[_p(t) for t in host_k])
+    hv = (c_void_p * n)(*[_p(t) for t in host_v])
+    r = vc_sched_request()
+    r.shape = sh
+    r.draft_kind = kind
+    r.qcaches = ctypes.cast(carr, c_void_p) if kind == VC_DRAFT_QUANT else None
+    r.scaches = ctypes.cast(carr, c_void_p) if kind != VC_DRAFT_QUANT else None
+    r.draft_q, r.draft_out, r.draft_ws, r.draft_ws_bytes = _p(draft_q), _p(draft_out), _p(draft_ws), draft_ws.numel()
+    r.host_k = ctypes.cast(hk, c_void_p)
+    r.host_v = ctypes.cast(hv, c_void_p)
+    r.kv_bytes_per_layer = host_k[0].numel() * host_k[0].element_size()
+    r.stage_k[0], r.stage_k[1] = _p(stage_k[0]), _p(stage_k[1])
+    r.stage_v[0], r.stage_v[1] = _p(stage_v[0]), _p(stage_v[1])
+    r.verify_q, r.verify_out, r.verify_ws, r.verify_ws_bytes = _p(verify_q), _p(verify_out), _p(verify_ws), verify_ws.numel()
+    r.T, r.nq = int(T), int(nq)
+    r.logits = _p(logits)
+    r.logits_dtype = VC_BF16 if logits.dtype == torch.bfloat16 else VC_F32
+    r.V = int(V)
+    r.draft_tokens, r.target, r.accept_len, r.correction = _p(draft_tokens), _p(target), _p(accept_len), _p(correction)
+    r.accept_ws, r.accept_ws_bytes = _p(accept_ws), accept_ws.numel()
+    r.stream = _stream(stream)
+    r._keep = (caches, carr, hk, hv, host_k, host_v, stage_k, stage_v, draft_q, draft_out, draft_ws, verify_q,
+               verify_out, verify_ws, logits, draft_tokens, target, accept_len, correction, accept_ws, stream)
+    return r
+
+
+def vc_sched_simulate(draft_ms, verify_ms, n_rounds: int, policy: int, never_done: int = -1,
+                      timeout_ms: float = 1e9) -> float:
+    """Makespan of the scheduling policy on a simulated timeline (host only)."""
+    n = len(draft_ms)
+    d = (ctypes.c_double * n)(*draft_ms)
+    v = (ctypes.c_double * n)(*verify_ms)
+    out = ctypes.c_double()
+    _check(lib().vc_sched_simulate(n, int(n_rounds), int(policy), d, v, int(never_done), float(timeout_ms),
+                                   ctypes.byref(out)))
+    return out.value
