@@ -106,15 +106,34 @@ typedef struct vc_attn_shape {
  *   values: per token over groups of `group` consecutive channels,
  *           v_hat[t][c] = code * v_scale[t][c / group] + v_zero[t][c / group]
  *
- * evaluated as one fp32 fused multiply-add.  Codes of a token row are packed
- * little-endian: channel c sits in bits [(c % (8/bits)) * bits, +bits) of byte
- * c * bits / 8.  The oldest L_q tokens are quantised; the newest R tokens are
- * kept in bf16 (the residual window, rows 0..R-1 of a buffer of R_cap rows).
+ * evaluated as one fp32 fused multiply-add.  The oldest L_q tokens are
+ * quantised; the newest R tokens are kept in bf16 (the residual window, rows
+ * 0..R-1 of a buffer of R_cap rows).
  *
- *   k_codes, v_codes  uint8 [B][Hkv][L_q][D * bits / 8]
+ *   k_codes, v_codes  uint8 [B][Hkv][L_q / group][group * D * bits / 8]
  *   k_scale, k_zero   fp16  [B][Hkv][L_q / group][D]
- *   v_scale, v_zero   fp16  [B][Hkv][L_q][D / group]
+ *   v_scale, v_zero   fp16  [B][Hkv][L_q / 2][D / group][2]
  *   k_res, v_res      bf16  [B][Hkv][R_cap][D]
+ *
+ * Code blocks are stored in fragment-native order, the order in which the
+ * tensor-core tiles of the draft kernel consume them.  For one group (a
+ * group x D code matrix C[t][c]) split tokens and channels into tiles of 16;
+ * lane L = 4 gid + tig (gid 0..7, tig 0..3) owns, per (token tile, channel
+ * tile), four registers of two codes:
+ *   keys:   reg0 = C[16tt+gid][16ct+2tig+{0,1}],  reg1 = same with token +8,
+ *           reg2 = C[16tt+gid][16ct+2tig+8+{0,1}], reg3 = reg2 with token +8
+ *   values: reg0 = C[16tt+2tig+{0,1}][16ct+gid],  reg1 = same with channel +8,
+ *           reg2 = C[16tt+2tig+8+{0,1}][16ct+gid], reg3 = reg2 with channel +8
+ * Words X_j / Y_j (j = 0 .. NW/2 - 1, NW = 2 (D/16) / TPW, TPW = 8 / bits)
+ * cover the channel tiles ct = TPW j + i; keys: X_j = (reg0, reg1), Y_j =
+ * (reg2, reg3); values: X_j = (reg0, reg2), Y_j = (reg1, reg3).  In a word,
+ * local tile i puts the first register's two codes at bits [bits*i, +bits)
+ * and [16 + bits*i, +bits), the second register's at [8 + bits*i, +bits) and
+ * [24 + bits*i, +bits).  Lane L's word w of token tile tt is 32-bit word
+ * (tt * 32 + L) * NW + w of the group's block.  Value scales and zeros hold,
+ * for each token pair (2p, 2p+1) and value group g, the two tokens' entries
+ * side by side.
+ *
  *   bits in {2, 4}; group in {32, 64}; L_q >= 0 and a multiple of group;
  *   0 <= R <= R_cap; L_q + R >= 1.  Scales, zeros and codes must be finite
  *   and q * scale must stay inside the fp16 range (|q * scale| < 65504). */
@@ -335,7 +354,8 @@ VC_API vc_status vc_workspace_flags(void* ws, size_t ws_bytes, uint32_t* host_fl
 
 /* ---- test exports ------------------------------------------------------------
  * vc_debug_dequant writes the dequantised L_q rows of every (request, head)
- * with the same code unpacking the draft kernel uses:
+ * in natural [token][channel] order, extracting the codes with the same
+ * word layout and masks the draft kernel uses:
  *   k_out, v_out fp32 [B][Hkv][L_q][D]   (R residual rows are not included)
  * vc_debug_gather writes the kept rows the sparse draft kernel reads:
  *   k_out, v_out bf16 [B][Hkv][n_keep][D]; out-of-range positions write

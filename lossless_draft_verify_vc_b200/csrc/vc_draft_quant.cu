@@ -106,81 +106,55 @@ __device__ __forceinline__ float softmax_step(float (&x)[4], float& m_run, float
 
 // ---- code extraction shared by the attention kernel and vc_debug_dequant
 //
-// A code is handed to the tensor core as an fp16 SUBNORMAL: AND-ing the packed
-// word with a mask that keeps one code per 16-bit half at bit position pos
-// (0 <= pos <= 9) yields the fp16 value code * 2^(pos - 24) exactly, and the
-// tensor cores multiply subnormal inputs exactly.  One LOP3 per two codes; the
-// power-of-two factors 2^(pos - 24) are folded into the other operand (key
-// side) or undone per output row (value side).
+// Storage: the codes of a group of G tokens form one block in fragment-native
+// order (include/vc.h): for each 16-token tile, lane L of the warp finds its
+// NW 32-bit words at word (tile * 32 + L) * NW.  Words come in pairs (X_j,
+// Y_j) covering TPW = 8 / bits channel tiles; a word holds two MMA registers
+// ("first" in the low byte of each 16-bit half, "second" in the high byte),
+// each register two codes (one per half), local tile i at bit position
+// bits * i.
 //
-// Key side (MMA rows = tokens, k = channels): inside a 16-channel tile, k-slots
-// (2t, 2t+1) of lane t hold channels (cA, cB) at bit position posA, slots
-// (2t+8, 2t+9) hold (cA+1, cB+1) at position posC.
+// A code reaches the tensor core as an fp16 SUBNORMAL: AND-ing a word with a
+// mask that keeps one code per half at bit position pos (< 10) yields the
+// fp16 value code * 2^(pos - 24) exactly, and the tensor cores multiply
+// subnormal inputs exactly.  So a register costs one AND (the second
+// register of a word also shares one shift).  The factors 2^(pos - 24) are
+// folded into the query operand (keys) or undone per output row (values).
 template <int BITS>
-struct KLane {
-  int cA, cB, shK, posA, posC;
-  uint32_t m1, m2;
-  __device__ __forceinline__ explicit KLane(int tig) {
-    cA = BITS == 2 ? 2 * tig : 8 * (tig >> 1) + 2 * (tig & 1);
-    cB = cA + (BITS == 2 ? 8 : 4);
-    shK = BITS == 2 ? 8 * (tig >> 1) : 8 * (tig & 1);
-    posA = BITS == 2 ? 4 * (tig & 1) : 0;
-    posC = posA + (BITS == 2 ? 2 : 4);
-    m1 = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << posA;
-    m2 = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << posC;
-  }
-  // word of a token row holding this lane's codes of channel tile kt
-  __device__ __forceinline__ int word(int kt, int tig) const { return BITS == 2 ? kt : 2 * kt + (tig >> 1); }
-  // A fragment of one 16x16 tile from the words of rows gid and gid + 8
-  __device__ __forceinline__ void frag(uint32_t w0, uint32_t w1, uint32_t (&af)[4]) const {
-    const uint32_t x0 = w0 >> shK, x1 = w1 >> shK;
-    af[0] = x0 & m1;
-    af[1] = x1 & m1;
-    af[2] = x0 & m2;
-    af[3] = x1 & m2;
-  }
-};
-
-// Value side (MMA rows = channels, k = tokens): row gid of a 16-channel tile
-// is channel `row` (bit position posR0), row gid + 8 is channel row + 1
-// (position posR1); k-slots are tokens.
-template <int BITS>
-struct VLane {
-  int row, posR0, posR1;
-  uint32_t sel, m1, m2;
-  __device__ __forceinline__ explicit VLane(int gid) {
-    const int k = BITS == 2 ? (gid >> 1) : (gid & 3);
-    sel = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
-    posR0 = BITS == 2 ? 4 * (gid & 1) : 0;
-    posR1 = posR0 + (BITS == 2 ? 2 : 4);
-    m1 = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << posR0;
-    m2 = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << posR1;
-    row = BITS == 2 ? 4 * (gid >> 1) + 2 * (gid & 1) : 2 * gid;
-  }
-  __device__ __forceinline__ int word(int mc, int gid) const { return BITS == 2 ? mc : 2 * mc + (gid >> 2); }
-  // A fragment from the words of tokens (t0, t0+1) and (t0+8, t0+9)
-  __device__ __forceinline__ void frag(uint32_t w0, uint32_t w1, uint32_t w8, uint32_t w9,
-                                       uint32_t (&af)[4]) const {
-    const uint32_t y01 = prmt(w0, w1, sel), y89 = prmt(w8, w9, sel);
-    af[0] = y01 & m1;
-    af[1] = y01 & m2;
-    af[2] = y89 & m1;
-    af[3] = y89 & m2;
-  }
+struct Frag {
+  static constexpr int TPW = 8 / BITS;  // channel (key) or row (value) tiles per word
+  static constexpr uint32_t BASE = BITS == 2 ? 0x00030003u : 0x000F000Fu;
+  __device__ __forceinline__ static uint32_t mask(int i) { return BASE << (BITS * i); }
 };
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
-// value scales of tokens (t, t+1) for value group cg as one f16x2 word
-template <int CPG>
-__device__ __forceinline__ uint32_t pair_of(const __half* base, int t, int cg) {
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(base + t * CPG);
-  if constexpr (CPG == 1) {
-    return w[0];
-  } else if constexpr (CPG == 2) {
-    return prmt(w[0], w[1], cg ? 0x7632 : 0x5410);
+template <int N>
+__device__ __forceinline__ void load_words(const uint32_t* p, uint32_t (&w)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int v = 0; v < N / 4; ++v) {
+      const uint4 x = reinterpret_cast<const uint4*>(p)[v];
+      w[4 * v] = x.x, w[4 * v + 1] = x.y, w[4 * v + 2] = x.z, w[4 * v + 3] = x.w;
+    }
   } else {
-    return prmt(w[cg >> 1], w[2 + (cg >> 1)], (cg & 1) ? 0x7632 : 0x5410);
+    static_assert(N == 2, "two or a multiple of four words");
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    w[0] = x.x, w[1] = x.y;
+  }
+}
+
+// the CPG words (one per value group) of a token pair
+template <int CPG>
+__device__ __forceinline__ void load_cpg(const uint32_t* p, uint32_t (&w)[CPG]) {
+  if constexpr (CPG == 4) {
+    const uint4 x = *reinterpret_cast<const uint4*>(p);
+    w[0] = x.x, w[1] = x.y, w[2] = x.z, w[3] = x.w;
+  } else if constexpr (CPG == 2) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    w[0] = x.x, w[1] = x.y;
+  } else {
+    w[0] = p[0];
   }
 }
 
@@ -189,7 +163,9 @@ template <int BITS, int G, int D, int NT>
 __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b, int h, int qchunk,
                            float* wst_ml, bool& ok) {
   using C = QCfg<BITS, G, D, NT>;
+  using F = Frag<BITS>;
   constexpr unsigned FULL = 0xffffffffu;
+  constexpr int NW = 2 * C::KT / F::TPW;  // words per lane per 16-token tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int part = gid & 1;
@@ -215,46 +191,41 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
     const int s = i % C::NST;
     const int64_t j = g_begin + warp + static_cast<int64_t>(i) * kQNW;
     unsigned char* st = ring + s * C::QSTAGE;
-    if (lane == 0) mbar_arrive_expect_tx(&bars[s], C::QSTAGE);
-    __syncwarp();
-    if (lane == 0) bulk_g2s(st, kc_u + j * C::KC_B, C::KC_B, &bars[s]);
-    if (lane == 1) bulk_g2s(st + C::KC_B, vc_u + j * C::KC_B, C::KC_B, &bars[s]);
-    if (lane == 2) bulk_g2s(st + 2 * C::KC_B, sk_u + j * D, C::SC_B, &bars[s]);
-    if (lane == 3) bulk_g2s(st + 2 * C::KC_B + C::SC_B, zk_u + j * D, C::SC_B, &bars[s]);
-    if (lane == 4) bulk_g2s(st + 2 * C::KC_B + 2 * C::SC_B, sv_u + j * G * C::CPG, C::SC_B, &bars[s]);
-    if (lane == 5) bulk_g2s(st + 2 * C::KC_B + 3 * C::SC_B, zv_u + j * G * C::CPG, C::SC_B, &bars[s]);
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[s], C::QSTAGE);
+      bulk_g2s(st, kc_u + j * C::KC_B, C::KC_B, &bars[s]);
+      bulk_g2s(st + C::KC_B, vc_u + j * C::KC_B, C::KC_B, &bars[s]);
+      bulk_g2s(st + 2 * C::KC_B, sk_u + j * D, C::SC_B, &bars[s]);
+      bulk_g2s(st + 2 * C::KC_B + C::SC_B, zk_u + j * D, C::SC_B, &bars[s]);
+      bulk_g2s(st + 2 * C::KC_B + 2 * C::SC_B, sv_u + j * G * C::CPG, C::SC_B, &bars[s]);
+      bulk_g2s(st + 2 * C::KC_B + 3 * C::SC_B, zv_u + j * G * C::CPG, C::SC_B, &bars[s]);
+    }
   };
 
-  const KLane<BITS> kl(tig);
-  const VLane<BITS> vl(gid);
-  const int cA = kl.cA, cB = kl.cB;
   const uint32_t lomask = part ? 0xffffffffu : 0u;  // low-part columns
 
-  // ---- query registers (fp16, exact from bf16), column head = nt*4 + gid/2
-  //   q2s: q at the k-slot channels, scaled by 2^-pos of the code encoding
-  //   qb : q at natural channel pairs for the zero-point MMA (high columns only)
+  // ---- query registers (fp16, exact from bf16), column head = nt*4 + gid/2,
+  //      natural channel pairs (16kt + 2tig, +1) and (16kt + 2tig + 8, +9)
+  //   q2s: scaled by 2^-(bits * (kt % TPW)) of the code encoding
+  //   qb : unscaled, high columns only (zero-point MMA)
   uint32_t q2s[C::KT][NT][2], qb[C::KT][NT][2];
-  {
-    const float fA = pow2i(-kl.posA), fC = pow2i(-kl.posC);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int hh = nt * 4 + (gid >> 1);
-      const bool hv = hh < a.g;
-      const __nv_bfloat16* qp = a.q + (static_cast<size_t>(b) * a.Hq + h * a.g + (hv ? hh : 0)) * D;
+  for (int nt = 0; nt < NT; ++nt) {
+    const int hh = nt * 4 + (gid >> 1);
+    const bool hv = hh < a.g;
+    const __nv_bfloat16* qp = a.q + (static_cast<size_t>(b) * a.Hq + h * a.g + (hv ? hh : 0)) * D;
 #pragma unroll
-      for (int kt = 0; kt < C::KT; ++kt) {
-        const float qa = __bfloat162float(qp[kt * 16 + cA]), qbb = __bfloat162float(qp[kt * 16 + cB]);
-        const float qc = __bfloat162float(qp[kt * 16 + cA + 1]), qd = __bfloat162float(qp[kt * 16 + cB + 1]);
-        q2s[kt][nt][0] = hv ? pack_h2(qa * fA, qbb * fA) : 0u;
-        q2s[kt][nt][1] = hv ? pack_h2(qc * fC, qd * fC) : 0u;
-        const uint32_t n0 = *reinterpret_cast<const uint32_t*>(qp + kt * 16 + 2 * tig);
-        const uint32_t n8 = *reinterpret_cast<const uint32_t*>(qp + kt * 16 + 8 + 2 * tig);
-        qb[kt][nt][0] = (hv && !part) ? bf2_to_h2(n0) : 0u;
-        qb[kt][nt][1] = (hv && !part) ? bf2_to_h2(n8) : 0u;
-      }
+    for (int kt = 0; kt < C::KT; ++kt) {
+      const float f = pow2i(-BITS * (kt % F::TPW));
+      const float2 lo = unpack_bf2(*reinterpret_cast<const uint32_t*>(qp + kt * 16 + 2 * tig));
+      const float2 hi = unpack_bf2(*reinterpret_cast<const uint32_t*>(qp + kt * 16 + 8 + 2 * tig));
+      q2s[kt][nt][0] = hv ? pack_h2(lo.x * f, lo.y * f) : 0u;
+      q2s[kt][nt][1] = hv ? pack_h2(hi.x * f, hi.y * f) : 0u;
+      qb[kt][nt][0] = (hv && !part) ? pack_h2(lo.x, lo.y) : 0u;
+      qb[kt][nt][1] = (hv && !part) ? pack_h2(hi.x, hi.y) : 0u;
     }
   }
-  // the score MMAs accumulate (scores) * 2^-24; undo it together with the softmax scale
+  // the score MMAs accumulate scores * 2^-24; undo it together with the softmax scale
   const float scl = a.scale_log2 * 16777216.0f;
 
   float acc[C::KT][NT][4];
@@ -279,6 +250,7 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
   for (int i = 0; i < my_n; ++i) {
     if (i + C::NST - 1 < my_n) {
       fence_proxy_async_smem();
+      __syncwarp();
       issue(i + C::NST - 1);
     }
     const int s = i % C::NST;
@@ -293,8 +265,8 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
     const uint32_t* vcw = reinterpret_cast<const uint32_t*>(st + C::KC_B);
     const __half* sk = reinterpret_cast<const __half*>(st + 2 * C::KC_B);
     const __half* zk = sk + D;
-    const __half* sv = zk + D;
-    const __half* zv = sv + D;
+    const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(zk + D);      // [G/2][CPG] token pairs
+    const uint32_t* zv32 = sv32 + G / 2 * C::CPG;
 
     // (1) fold the key scales into q (fp16 high part in part-0 columns, low
     //     part in part-1 columns) and the zero-point term sum_c q_c z_c
@@ -304,9 +276,8 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
     for (int nt = 0; nt < NT; ++nt) kb[nt][0] = kb[nt][1] = kb[nt][2] = kb[nt][3] = 0.f;
 #pragma unroll
     for (int kt = 0; kt < C::KT; ++kt) {
-      const uint32_t sw1 = *reinterpret_cast<const uint32_t*>(sk + kt * 16 + cA);
-      const uint32_t sw2 = *reinterpret_cast<const uint32_t*>(sk + kt * 16 + cB);
-      const uint32_t sA = prmt(sw1, sw2, 0x5410), sC = prmt(sw1, sw2, 0x7632);
+      const uint32_t sA = *reinterpret_cast<const uint32_t*>(sk + kt * 16 + 2 * tig);
+      const uint32_t sC = *reinterpret_cast<const uint32_t*>(sk + kt * 16 + 8 + 2 * tig);
       const uint32_t z0 = *reinterpret_cast<const uint32_t*>(zk + kt * 16 + 2 * tig);
       const uint32_t z8 = *reinterpret_cast<const uint32_t*>(zk + kt * 16 + 8 + 2 * tig);
       const uint32_t za[4] = {z0, z0, z8, z8};
@@ -329,34 +300,20 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
       float sc[2][NT][4];
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
-        const int r0 = sb * 32 + mt * 16 + gid;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) sc[mt][nt][e] = kb[nt][e];
-        if constexpr (BITS == 2) {
-          uint32_t w0[C::WPR], w1[C::WPR];
+        uint32_t w[NW];
+        load_words(kcw + ((sb * 2 + mt) * 32 + lane) * NW, w);
 #pragma unroll
-          for (int v = 0; v < C::WPR / 4; ++v) {
-            const uint4 x = reinterpret_cast<const uint4*>(kcw + r0 * C::WPR)[v];
-            const uint4 y = reinterpret_cast<const uint4*>(kcw + (r0 + 8) * C::WPR)[v];
-            w0[4 * v] = x.x, w0[4 * v + 1] = x.y, w0[4 * v + 2] = x.z, w0[4 * v + 3] = x.w;
-            w1[4 * v] = y.x, w1[4 * v + 1] = y.y, w1[4 * v + 2] = y.z, w1[4 * v + 3] = y.w;
-          }
+        for (int j = 0; j < NW / 2; ++j) {
+          const uint32_t X = w[2 * j], Y = w[2 * j + 1], xs = X >> 8, ys = Y >> 8;
 #pragma unroll
-          for (int kt = 0; kt < C::KT; ++kt) {
-            uint32_t af[4];
-            kl.frag(w0[kt], w1[kt], af);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_f16(sc[mt][nt], af, qf[kt][nt][0], qf[kt][nt][1]);
-          }
-        } else {
-          const uint32_t* row0 = kcw + r0 * C::WPR + (tig >> 1);
-          const uint32_t* row1 = row0 + 8 * C::WPR;
-#pragma unroll
-          for (int kt = 0; kt < C::KT; ++kt) {
-            uint32_t af[4];
-            kl.frag(row0[2 * kt], row1[2 * kt], af);
+          for (int i = 0; i < F::TPW; ++i) {
+            const int kt = F::TPW * j + i;
+            const uint32_t m = F::mask(i);
+            const uint32_t af[4] = {X & m, xs & m, Y & m, ys & m};
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) mma_f16(sc[mt][nt], af, qf[kt][nt][0], qf[kt][nt][1]);
           }
@@ -368,19 +325,17 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
         float x[4] = {(sc[0][nt][0] + sc[0][nt][1]) * scl, (sc[0][nt][2] + sc[0][nt][3]) * scl,
                       (sc[1][nt][0] + sc[1][nt][1]) * scl, (sc[1][nt][2] + sc[1][nt][3]) * scl};
         const float alpha = softmax_step(x, m_run[nt], l_run[nt], 4);
-        if (__any_sync(FULL, alpha != 1.f)) {
 #pragma unroll
-          for (int mc = 0; mc < C::KT; ++mc) {
-            acc[mc][nt][0] *= alpha;
-            acc[mc][nt][1] *= alpha;
-            acc[mc][nt][2] *= alpha;
-            acc[mc][nt][3] *= alpha;
-          }
-          vb[nt][0] *= alpha;
-          vb[nt][1] *= alpha;
-          vb[nt][2] *= alpha;
-          vb[nt][3] *= alpha;
+        for (int mc = 0; mc < C::KT; ++mc) {
+          acc[mc][nt][0] *= alpha;
+          acc[mc][nt][1] *= alpha;
+          acc[mc][nt][2] *= alpha;
+          acc[mc][nt][3] *= alpha;
         }
+        vb[nt][0] *= alpha;
+        vb[nt][1] *= alpha;
+        vb[nt][2] *= alpha;
+        vb[nt][3] *= alpha;
         // p as fp16 high + low parts, split once here for the value side
         const uint32_t h01 = pack_h2(x[0], x[1]), h23 = pack_h2(x[2], x[3]);
         const float2 f01 = unpack_h2(h01), f23 = unpack_h2(h23);
@@ -400,55 +355,53 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
 #pragma unroll
       for (int ktt = 0; ktt < 2; ++ktt) {
         const int t0 = sb * 32 + ktt * 16 + 2 * tig;  // tokens t0, t0+1, t0+8, t0+9
-        uint32_t ph01[NT], ph89[NT], pl01[NT], pl89[NT];
+        uint32_t ph01[NT], ph89[NT], plm01[NT], plm89[NT], phn01[NT], phn89[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int hh = nt * 4 + (gid >> 1);
           ph01[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0);
           ph89[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0 + 8);
-          pl01[nt] = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0);
-          pl89[nt] = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0 + 8);
-        }
-        // value zero-point term: A = z_v^T (row = value group gid), B = p
-        {
+          const uint32_t pl01 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0);
+          const uint32_t pl89 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0 + 8);
+          plm01[nt] = pl01 & lomask;
+          plm89[nt] = pl89 & lomask;
+          phn01[nt] = (ph01[nt] ^ 0x80008000u) & lomask;
+          phn89[nt] = (ph89[nt] ^ 0x80008000u) & lomask;
+          // value zero-point term: A = z_v^T (row = value group gid), B = p (high or low column)
           uint32_t za[4] = {0u, 0u, 0u, 0u};
           if (gid < C::CPG) {
-            const uint32_t z0 = __half_as_ushort(zv[t0 * C::CPG + gid]);
-            const uint32_t z1 = __half_as_ushort(zv[(t0 + 1) * C::CPG + gid]);
-            const uint32_t z8 = __half_as_ushort(zv[(t0 + 8) * C::CPG + gid]);
-            const uint32_t z9 = __half_as_ushort(zv[(t0 + 9) * C::CPG + gid]);
-            za[0] = z0 | (z1 << 16);
-            za[2] = z8 | (z9 << 16);
+            za[0] = zv32[(t0 >> 1) * C::CPG + gid];
+            za[2] = zv32[((t0 + 8) >> 1) * C::CPG + gid];
           }
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_f16(vb[nt], za, part ? pl01[nt] : ph01[nt], part ? pl89[nt] : ph89[nt]);
+          mma_f16(vb[nt], za, part ? pl01 : ph01[nt], part ? pl89 : ph89[nt]);
         }
-        const uint32_t* T0 = vcw + t0 * C::WPR;
-        const uint32_t* T1 = T0 + C::WPR;
-        const uint32_t* T8 = T0 + 8 * C::WPR;
-        const uint32_t* T9 = T0 + 9 * C::WPR;
+        // folded p*s for every value group: high part (part 0) or low part (part 1)
+        uint32_t pf[C::CPG][NT][2];
+        {
+          uint32_t s01[C::CPG], s89[C::CPG];
+          load_cpg<C::CPG>(sv32 + (t0 >> 1) * C::CPG, s01);
+          load_cpg<C::CPG>(sv32 + ((t0 + 8) >> 1) * C::CPG, s89);
 #pragma unroll
-        for (int cg = 0; cg < C::CPG; ++cg) {
-          // folded p*s for this value group: high part (part 0) or low part (part 1)
-          const uint32_t s01 = pair_of<C::CPG>(sv, t0, cg);
-          const uint32_t s89 = pair_of<C::CPG>(sv, t0 + 8, cg);
-          uint32_t pf[NT][2];
+          for (int cg = 0; cg < C::CPG; ++cg)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            pf[nt][0] = hfma2(pl01[nt] & lomask, s01,
-                              hfma2(ph01[nt], s01, hmul2((ph01[nt] ^ 0x80008000u) & lomask, s01)));
-            pf[nt][1] = hfma2(pl89[nt] & lomask, s89,
-                              hfma2(ph89[nt], s89, hmul2((ph89[nt] ^ 0x80008000u) & lomask, s89)));
-          }
+            for (int nt = 0; nt < NT; ++nt) {
+              pf[cg][nt][0] = hfma2(plm01[nt], s01[cg], hfma2(ph01[nt], s01[cg], hmul2(phn01[nt], s01[cg])));
+              pf[cg][nt][1] = hfma2(plm89[nt], s89[cg], hfma2(ph89[nt], s89[cg], hmul2(phn89[nt], s89[cg])));
+            }
+        }
+        uint32_t w[NW];
+        load_words(vcw + ((sb * 2 + ktt) * 32 + lane) * NW, w);
 #pragma unroll
-          for (int mq = 0; mq < G / 16; ++mq) {
-            const int mc = cg * (G / 16) + mq;  // 16-channel tile
-            const int wi = vl.word(mc, gid);
-            uint32_t af[4];
-            vl.frag(T0[wi], T1[wi], T8[wi], T9[wi], af);
+        for (int j = 0; j < NW / 2; ++j) {
+          const uint32_t X = w[2 * j], Y = w[2 * j + 1], xs = X >> 8, ys = Y >> 8;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_f16(acc[mc][nt], af, pf[nt][0], pf[nt][1]);
+          for (int i = 0; i < F::TPW; ++i) {
+            const int mc = F::TPW * j + i;  // 16-channel tile
+            const int cg = mc * 16 / G;
+            const uint32_t m = F::mask(i);
+            const uint32_t af[4] = {X & m, Y & m, xs & m, ys & m};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_f16(acc[mc][nt], af, pf[cg][nt][0], pf[cg][nt][1]);
           }
         }
       }
@@ -459,7 +412,6 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
   // ---- this warp's state -> its own (finished) ring, natural channel order
   __syncwarp();
   float* my_o = reinterpret_cast<float*>(ring);  // [g][D]
-  const float u0 = pow2i(24 - vl.posR0), u1 = pow2i(24 - vl.posR1);  // undo the code encoding
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int hh = nt * 4 + tig;
@@ -472,10 +424,11 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
     for (int mc = 0; mc < C::KT; ++mc) {
       const int cg = mc * 16 / G;
       const float zb = __shfl_sync(FULL, vbs, cg * 4 + tig);
+      const float u = pow2i(24 - BITS * (mc % F::TPW));  // undo the code encoding of this tile
       if (hh < a.g) {
-        float* wo = my_o + hh * D + mc * 16 + vl.row;
-        wo[0] = (acc[mc][nt][0] + acc[mc][nt][1]) * u0 + zb;
-        wo[1] = (acc[mc][nt][2] + acc[mc][nt][3]) * u1 + zb;
+        float* wo = my_o + hh * D + mc * 16 + gid;
+        wo[0] = (acc[mc][nt][0] + acc[mc][nt][1]) * u + zb;
+        wo[8] = (acc[mc][nt][2] + acc[mc][nt][3]) * u + zb;
       }
     }
     if (hh < a.g && gid == 0) {
@@ -641,63 +594,63 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
       smem_w);
 }
 
-// vc_debug_dequant: one warp per (group, unit); the codes are extracted with
-// the same KLane / VLane fragment code the attention kernel uses, then
-// dequantised with one fp32 FMA each and stored at their natural positions.
+// vc_debug_dequant: one warp per (group, unit).  The codes are extracted with
+// the same word layout, masks and subnormal encoding the attention kernel
+// uses (Frag), then dequantised with one fp32 FMA each and stored at their
+// natural positions.
 template <int BITS, int G, int D>
 __global__ void __launch_bounds__(32) debug_dequant_kernel(QArgs a, float* ko, float* vo) {
-  constexpr int RB = D * BITS / 8, WPR = RB / 4, CPG = D / G;
+  using F = Frag<BITS>;
+  constexpr int RB = D * BITS / 8, CPG = D / G, KT = D / 16, NW = 2 * KT / F::TPW;
   const int lane = threadIdx.x, gid = lane >> 2, tig = lane & 3;
   const int unit = blockIdx.y;
   const int64_t j = blockIdx.x;
   const int64_t n_groups = a.L_q / G;
-  const uint32_t* kc = reinterpret_cast<const uint32_t*>(a.kc + static_cast<size_t>(unit) * a.L_q * RB);
-  const uint32_t* vc = reinterpret_cast<const uint32_t*>(a.vc + static_cast<size_t>(unit) * a.L_q * RB);
+  const uint32_t* kc = reinterpret_cast<const uint32_t*>(a.kc + (static_cast<size_t>(unit) * a.L_q + j * G) * RB);
+  const uint32_t* vcw = reinterpret_cast<const uint32_t*>(a.vc + (static_cast<size_t>(unit) * a.L_q + j * G) * RB);
   const __half* sk = a.sk + (static_cast<size_t>(unit) * n_groups + j) * D;
   const __half* zk = a.zk + (static_cast<size_t>(unit) * n_groups + j) * D;
-  const __half* sv = a.sv + static_cast<size_t>(unit) * a.L_q * CPG;
-  const __half* zv = a.zv + static_cast<size_t>(unit) * a.L_q * CPG;
-  float* kou = ko + static_cast<size_t>(unit) * a.L_q * D;
-  float* vou = vo + static_cast<size_t>(unit) * a.L_q * D;
-  const KLane<BITS> kl(tig);
-  for (int mt = 0; mt < G / 16; ++mt) {
-    const int64_t t = j * G + mt * 16 + gid;
-    for (int kt = 0; kt < D / 16; ++kt) {
-      uint32_t af[4];
-      const int wi = kl.word(kt, tig);
-      kl.frag(kc[t * WPR + wi], kc[(t + 8) * WPR + wi], af);
-      const int ch[4][2] = {{kl.cA, kl.cB}, {kl.cA, kl.cB}, {kl.cA + 1, kl.cB + 1}, {kl.cA + 1, kl.cB + 1}};
-      const int64_t tok[4] = {t, t + 8, t, t + 8};
-      const float undo[4] = {pow2i(24 - kl.posA), pow2i(24 - kl.posA), pow2i(24 - kl.posC), pow2i(24 - kl.posC)};
-      for (int e = 0; e < 4; ++e) {
-        const float2 code = unpack_h2(af[e]);
-        const float cc[2] = {code.x * undo[e], code.y * undo[e]};
-        for (int u = 0; u < 2; ++u) {
-          const int c = kt * 16 + ch[e][u];
-          kou[tok[e] * D + c] = __fmaf_rn(cc[u], __half2float(sk[c]), __half2float(zk[c]));
-        }
+  const __half* sv = a.sv + (static_cast<size_t>(unit) * a.L_q + j * G) * CPG;  // pair-interleaved
+  const __half* zv = a.zv + (static_cast<size_t>(unit) * a.L_q + j * G) * CPG;
+  float* kou = ko + (static_cast<size_t>(unit) * a.L_q + j * G) * D;
+  float* vou = vo + (static_cast<size_t>(unit) * a.L_q + j * G) * D;
+  auto code = [](uint32_t reg, int half, float undo) {
+    const float2 f = unpack_h2(reg);
+    return (half ? f.y : f.x) * undo;
+  };
+  for (int tt = 0; tt < G / 16; ++tt) {
+    for (int jw = 0; jw < NW / 2; ++jw) {
+      const uint32_t X = kc[(tt * 32 + lane) * NW + 2 * jw], Y = kc[(tt * 32 + lane) * NW + 2 * jw + 1];
+      for (int i = 0; i < F::TPW; ++i) {
+        const int kt = F::TPW * jw + i;
+        const uint32_t m = F::mask(i);
+        const float undo = pow2i(24 - BITS * i);
+        // reg0: token gid, channels 2tig+{0,1}; reg1: token gid+8; reg2/3: channels +8
+        const uint32_t regs[4] = {X & m, (X >> 8) & m, Y & m, (Y >> 8) & m};
+        for (int r = 0; r < 4; ++r)
+          for (int e = 0; e < 2; ++e) {
+            const int t = tt * 16 + gid + ((r & 1) ? 8 : 0);
+            const int c = kt * 16 + 2 * tig + ((r & 2) ? 8 : 0) + e;
+            kou[t * D + c] = __fmaf_rn(code(regs[r], e, undo), __half2float(sk[c]), __half2float(zk[c]));
+          }
       }
     }
-  }
-  const VLane<BITS> vl(gid);
-  for (int ktt = 0; ktt < G / 16; ++ktt) {
-    const int64_t t0 = j * G + ktt * 16 + 2 * tig;
-    for (int mc = 0; mc < D / 16; ++mc) {
-      uint32_t af[4];
-      const int wi = vl.word(mc, gid);
-      vl.frag(vc[t0 * WPR + wi], vc[(t0 + 1) * WPR + wi], vc[(t0 + 8) * WPR + wi], vc[(t0 + 9) * WPR + wi], af);
-      const int chs[4] = {vl.row, vl.row + 1, vl.row, vl.row + 1};
-      const int64_t tk[4][2] = {{t0, t0 + 1}, {t0, t0 + 1}, {t0 + 8, t0 + 9}, {t0 + 8, t0 + 9}};
-      const float undo[4] = {pow2i(24 - vl.posR0), pow2i(24 - vl.posR1), pow2i(24 - vl.posR0), pow2i(24 - vl.posR1)};
-      for (int e = 0; e < 4; ++e) {
-        const float2 code = unpack_h2(af[e]);
-        const float cc[2] = {code.x * undo[e], code.y * undo[e]};
-        const int c = mc * 16 + chs[e];
-        for (int u = 0; u < 2; ++u) {
-          const int64_t tt = tk[e][u];
-          vou[tt * D + c] =
-              __fmaf_rn(cc[u], __half2float(sv[tt * CPG + c / G]), __half2float(zv[tt * CPG + c / G]));
-        }
+    for (int jw = 0; jw < NW / 2; ++jw) {
+      const uint32_t X = vcw[(tt * 32 + lane) * NW + 2 * jw], Y = vcw[(tt * 32 + lane) * NW + 2 * jw + 1];
+      for (int i = 0; i < F::TPW; ++i) {
+        const int mc = F::TPW * jw + i;
+        const uint32_t m = F::mask(i);
+        const float undo = pow2i(24 - BITS * i);
+        // reg0: channel gid, tokens 2tig+{0,1}; reg1: channel gid+8; reg2/3: tokens +8
+        const uint32_t regs[4] = {X & m, Y & m, (X >> 8) & m, (Y >> 8) & m};
+        for (int r = 0; r < 4; ++r)
+          for (int e = 0; e < 2; ++e) {
+            const int t = tt * 16 + 2 * tig + ((r & 2) ? 8 : 0) + e;
+            const int c = mc * 16 + gid + ((r & 1) ? 8 : 0);
+            const int cg = c / G;
+            const int pi = ((t >> 1) * CPG + cg) * 2 + (t & 1);
+            vou[t * D + c] = __fmaf_rn(code(regs[r], e, undo), __half2float(sv[pi]), __half2float(zv[pi]));
+          }
       }
     }
   }

@@ -105,9 +105,10 @@ def random_quant_cache(B: int, Hkv: int, L_q: int, R_cap: int, D: int, bits: int
     """A quantised cache drawn directly in compressed form for throughput runs:
     uniform random packed codes, scales ~U(0.05, 1.5), zeros ~U(-3, -0.5)
     (magnitudes of 2/4-bit groups of N(0, 1) data), bf16 residual ~N(0, 1).
-    Layouts match the library's quantised-cache descriptor."""
+    Shapes match the library's quantised-cache descriptor (codes per group
+    block, value scales/zeros per token pair)."""
     g = _gen(seed, device)
-    row = D * bits // 8
+    blk = group * D * bits // 8
     f16 = torch.float16
 
     def u(shape, lo, hi):
@@ -115,12 +116,14 @@ def random_quant_cache(B: int, Hkv: int, L_q: int, R_cap: int, D: int, bits: int
 
     return dict(
         bits=bits, group=group, L_q=L_q, R=R_cap, R_cap=R_cap,
-        k_codes=torch.randint(0, 256, (B, Hkv, L_q, row), generator=g, device=device, dtype=torch.int32).to(torch.uint8),
-        v_codes=torch.randint(0, 256, (B, Hkv, L_q, row), generator=g, device=device, dtype=torch.int32).to(torch.uint8),
+        k_codes=torch.randint(0, 256, (B, Hkv, L_q // group, blk), generator=g, device=device,
+                              dtype=torch.int32).to(torch.uint8),
+        v_codes=torch.randint(0, 256, (B, Hkv, L_q // group, blk), generator=g, device=device,
+                              dtype=torch.int32).to(torch.uint8),
         k_scale=u((B, Hkv, L_q // group, D), 0.05, 1.5),
         k_zero=u((B, Hkv, L_q // group, D), -3.0, -0.5),
-        v_scale=u((B, Hkv, L_q, D // group), 0.05, 1.5),
-        v_zero=u((B, Hkv, L_q, D // group), -3.0, -0.5),
+        v_scale=u((B, Hkv, L_q // 2, D // group, 2), 0.05, 1.5),
+        v_zero=u((B, Hkv, L_q // 2, D // group, 2), -3.0, -0.5),
         k_res=normal((B, Hkv, R_cap, D), seed + 11, device),
         v_res=normal((B, Hkv, R_cap, D), seed + 12, device),
     )

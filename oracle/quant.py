@@ -22,9 +22,17 @@ Readings taken where the pages are silent (all listed in the design doc)
   multiply-add).  In float64 the product and sum below are exact (code < 2**4,
   s and z are fp16), so rounding the float64 result to float32 once is exactly
   that single rounding.
-* Packing: code of channel c of a token occupies bits
-  [(c mod (8/b)) * b, +b) of byte floor(c * b / 8) of that token's row
-  (little-endian within the byte, channels contiguous along the row).
+* Storage order of the codes (a choice of this library, the pages fix
+  none): the codes of each group of G tokens form one block in the
+  "fragment-native" order defined in key_code_positions /
+  value_code_positions below -- the order in which a warp of the draft
+  kernel feeds them to its tensor-core tiles.  Value scales and zeros are
+  stored pair-interleaved: for tokens (2p, 2p+1) the CPG = D / G groups
+  hold (s[2p][cg], s[2p+1][cg]) next to each other.  Key scales and zeros
+  keep the natural [group][channel] order.  pack_codes / unpack_codes
+  (the plain row order: channel c of a token at bits [(c mod (8/b)) * b,
+  +b) of byte c * b / 8) remain as the reference from which the block order
+  is a fixed permutation.
 * The oldest L_q = T - R tokens are quantised; the newest R stay bf16
   (the "recent-token residual window").
 """
@@ -123,6 +131,113 @@ def unpack_codes(packed: np.ndarray, bits: int) -> np.ndarray:
     return np.stack(parts, axis=-1).reshape(*packed.shape[:-1], packed.shape[-1] * per)
 
 
+# ---------------------------------------------------------------------------
+# Fragment-native block order of the codes of one group.
+#
+# Keys (a G x D block C[t][c], t token in the group, c channel): tokens in
+# tiles of 16 (t = 16 mt + r), channels in tiles of 16 (c = 16 kt + j).
+# Lane L = 4 gid + tig (gid 0..7, tig 0..3) of a 32-lane warp owns, per
+# (mt, kt), four registers of two codes each (first code = even slot):
+#   reg0 = C[16mt+gid  ][16kt+2tig+{0,1}]    reg1 = C[16mt+gid+8][16kt+2tig+{0,1}]
+#   reg2 = C[16mt+gid  ][16kt+2tig+8+{0,1}]  reg3 = C[16mt+gid+8][16kt+2tig+8+{0,1}]
+# The lane's 32-bit words, per mt, are X_0, Y_0, X_1, Y_1, ... where X_j holds
+# (reg0, reg1) and Y_j holds (reg2, reg3) of the TPW = 8 / b tiles
+# kt = TPW j + i.  Inside a word, for local tile i and the pair
+# (first register F, second register S):
+#   F.code0 at bits [b i, +b)        F.code1 at bits [16 + b i, +b)
+#   S.code0 at bits [8 + b i, +b)    S.code1 at bits [24 + b i, +b)
+# Word w of lane L in token tile mt is the 32-bit word number
+# (mt * 32 + L) * NW + w of the block (little-endian), NW = 2 (D/16) / TPW.
+#
+# Values (a G x D block C[t][c]): tokens in tiles of 16 (t = 16 kk + k),
+# channels in tiles of 16 (c = 16 mc + r); per (kk, mc) lane L owns
+#   reg0 = C[16kk+2tig+{0,1}][16mc+gid]      reg1 = C[16kk+2tig+{0,1}][16mc+gid+8]
+#   reg2 = C[16kk+2tig+8+{0,1}][16mc+gid]    reg3 = C[16kk+2tig+8+{0,1}][16mc+gid+8]
+# X_j holds (reg0, reg2), Y_j holds (reg1, reg3) of tiles mc = TPW j + i, with
+# the same bit rule and word numbering (token tile kk in place of mt).
+# ---------------------------------------------------------------------------
+
+def _block_positions(bits: int, G: int, D: int, values: bool):
+    """(byte index, bit shift) of every code of a G x D group block."""
+    tpw = 8 // bits
+    ntile_c = D // 16
+    nw = 2 * ntile_c // tpw
+    byte = np.full((G, D), -1, np.int64)
+    shift = np.zeros((G, D), np.int64)
+    for tt in range(G // 16):
+        for L in range(32):
+            gid, tig = L // 4, L % 4
+            for ct in range(ntile_c):
+                j, i = divmod(ct, tpw)
+                if not values:
+                    # (token, channel) of reg0..reg3, code0/code1
+                    regs = [[(16 * tt + gid, 16 * ct + 2 * tig + e) for e in (0, 1)],
+                            [(16 * tt + gid + 8, 16 * ct + 2 * tig + e) for e in (0, 1)],
+                            [(16 * tt + gid, 16 * ct + 2 * tig + 8 + e) for e in (0, 1)],
+                            [(16 * tt + gid + 8, 16 * ct + 2 * tig + 8 + e) for e in (0, 1)]]
+                    words = [(2 * j, regs[0], regs[1]), (2 * j + 1, regs[2], regs[3])]
+                else:
+                    regs = [[(16 * tt + 2 * tig + e, 16 * ct + gid) for e in (0, 1)],
+                            [(16 * tt + 2 * tig + e, 16 * ct + gid + 8) for e in (0, 1)],
+                            [(16 * tt + 2 * tig + 8 + e, 16 * ct + gid) for e in (0, 1)],
+                            [(16 * tt + 2 * tig + 8 + e, 16 * ct + gid + 8) for e in (0, 1)]]
+                    words = [(2 * j, regs[0], regs[2]), (2 * j + 1, regs[1], regs[3])]
+                for w, F, S in words:
+                    word_index = (tt * 32 + L) * nw + w
+                    for (t, c), bit in ((F[0], bits * i), (F[1], 16 + bits * i),
+                                        (S[0], 8 + bits * i), (S[1], 24 + bits * i)):
+                        byte[t, c] = word_index * 4 + bit // 8
+                        shift[t, c] = bit % 8
+    assert (byte >= 0).all(), "every code must have a place"
+    return byte, shift
+
+
+def key_code_positions(bits: int, G: int, D: int):
+    return _block_positions(bits, G, D, values=False)
+
+
+def value_code_positions(bits: int, G: int, D: int):
+    return _block_positions(bits, G, D, values=True)
+
+
+def pack_group_blocks(codes: np.ndarray, bits: int, G: int, values: bool) -> np.ndarray:
+    """[..., L, D] codes -> [..., L/G, G*D*bits/8] bytes in block order."""
+    codes = np.asarray(codes, np.uint8)
+    *lead, L, D = codes.shape
+    byte, shift = _block_positions(bits, G, D, values)
+    c = codes.reshape(*lead, L // G, G, D).astype(np.uint32)
+    out = np.zeros((*lead, L // G, G * D * bits // 8), np.uint32)
+    flat_out = out.reshape(-1, out.shape[-1])
+    flat_c = c.reshape(-1, G, D)
+    for n in range(flat_c.shape[0]):
+        np.bitwise_or.at(flat_out[n], byte.ravel(), (flat_c[n] << shift).ravel())
+    return out.astype(np.uint8)
+
+
+def unpack_group_blocks(blocks: np.ndarray, bits: int, G: int, D: int, values: bool) -> np.ndarray:
+    """Inverse of pack_group_blocks: [..., L/G, G*D*bits/8] -> [..., L, D]."""
+    blocks = np.asarray(blocks, np.uint8)
+    byte, shift = _block_positions(bits, G, D, values)
+    mask = (1 << bits) - 1
+    out = (blocks[..., byte] >> shift) & mask
+    *lead, ng, _, _ = out.shape
+    return out.reshape(*lead, ng * G, D).astype(np.uint8)
+
+
+def pair_interleave(params: np.ndarray) -> np.ndarray:
+    """Value scales or zeros [..., L, CPG] -> [..., L/2, CPG, 2]: the two tokens
+    of a pair sit next to each other for every value group."""
+    p = np.asarray(params)
+    *lead, L, cpg = p.shape
+    return np.ascontiguousarray(p.reshape(*lead, L // 2, 2, cpg).swapaxes(-1, -2))
+
+
+def pair_deinterleave(params: np.ndarray) -> np.ndarray:
+    p = np.asarray(params)
+    *lead, P, cpg, two = p.shape
+    return np.ascontiguousarray(p.swapaxes(-1, -2)).reshape(*lead, 2 * P, cpg)
+
+
 def dequantize_keys(codes: np.ndarray, s: np.ndarray, z: np.ndarray, group: int) -> np.ndarray:
     """k_hat[t, c] = fp32(code[t, c] * s[t // G, c] + z[t // G, c]) (single rounding)."""
     codes = np.asarray(codes, np.float64)
@@ -144,11 +259,14 @@ def build_quant_cache(k: np.ndarray, v: np.ndarray, bits: int, group: int, resid
 
     k, v: [B, Hkv, T, D] bf16 values (as float32).  The oldest
     L_q = T - residual tokens are quantised, the newest ``residual`` stay bf16.
-    Returns a dict with the packed codes, fp16 scales/zeros and the residual
-    rows, in the layouts the library's quantised-cache descriptor names."""
+    Returns a dict in the library's storage layout:
+      k_codes, v_codes  uint8 [B, Hkv, L_q/G, G*D*bits/8]  (block order)
+      k_scale, k_zero   fp16  [B, Hkv, L_q/G, D]
+      v_scale, v_zero   fp16  [B, Hkv, L_q/2, D/G, 2]      (pair-interleaved)
+      k_res, v_res      bf16 values [B, Hkv, residual, D]"""
     k = np.asarray(k, np.float32)
     v = np.asarray(v, np.float32)
-    T = k.shape[-2]
+    T, D = k.shape[-2], k.shape[-1]
     L_q = T - residual
     if L_q < 0 or L_q % group:
         raise ValueError("T - residual must be a non-negative multiple of the group size")
@@ -156,8 +274,9 @@ def build_quant_cache(k: np.ndarray, v: np.ndarray, bits: int, group: int, resid
     vc, sv, zv = quantize_values(v[..., :L_q, :], bits, group)
     return dict(
         bits=bits, group=group, L_q=L_q, R=residual,
-        k_codes=pack_codes(kc, bits), v_codes=pack_codes(vc, bits),
-        k_scale=sk, k_zero=zk, v_scale=sv, v_zero=zv,
+        k_codes=pack_group_blocks(kc, bits, group, values=False),
+        v_codes=pack_group_blocks(vc, bits, group, values=True),
+        k_scale=sk, k_zero=zk, v_scale=pair_interleave(sv), v_zero=pair_interleave(zv),
         k_res=k[..., L_q:, :].copy(), v_res=v[..., L_q:, :].copy(),
     )
 
@@ -166,10 +285,11 @@ def dequantize_cache(cache: dict):
     """Full-length (K_hat, V_hat) of a quantised cache: dequantised rows
     followed by the bf16 residual rows.  Float32 arrays [B, Hkv, L_q + R, D]."""
     bits, G = cache["bits"], cache["group"]
-    kc = unpack_codes(cache["k_codes"], bits)
-    vc = unpack_codes(cache["v_codes"], bits)
+    D = cache["k_scale"].shape[-1]
+    kc = unpack_group_blocks(cache["k_codes"], bits, G, D, values=False)
+    vc = unpack_group_blocks(cache["v_codes"], bits, G, D, values=True)
     kh = dequantize_keys(kc, cache["k_scale"], cache["k_zero"], G)
-    vh = dequantize_values(vc, cache["v_scale"], cache["v_zero"], G)
+    vh = dequantize_values(vc, pair_deinterleave(cache["v_scale"]), pair_deinterleave(cache["v_zero"]), G)
     R = cache["R"]
     kr = np.asarray(cache["k_res"], np.float32)[..., :R, :]
     vr = np.asarray(cache["v_res"], np.float32)[..., :R, :]

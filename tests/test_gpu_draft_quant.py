@@ -42,10 +42,10 @@ def test_dequant_bit_exact(bits, G, D):
     vo = torch.empty_like(ko)
     vc.vc_debug_dequant(vc.shape(B, 2 * Hkv, Hkv, D), vc.quant_cache(tc), ko, vo)
     torch.cuda.synchronize()
-    kc = Q.unpack_codes(cache["k_codes"], bits)
-    vcd = Q.unpack_codes(cache["v_codes"], bits)
+    kc = Q.unpack_group_blocks(cache["k_codes"], bits, G, D, values=False)
+    vcd = Q.unpack_group_blocks(cache["v_codes"], bits, G, D, values=True)
     kw = Q.dequantize_keys(kc, cache["k_scale"], cache["k_zero"], G)
-    vw = Q.dequantize_values(vcd, cache["v_scale"], cache["v_zero"], G)
+    vw = Q.dequantize_values(vcd, Q.pair_deinterleave(cache["v_scale"]), Q.pair_deinterleave(cache["v_zero"]), G)
     assert np.array_equal(ko.cpu().numpy().view(np.uint32), kw.view(np.uint32))
     assert np.array_equal(vo.cpu().numpy().view(np.uint32), vw.view(np.uint32))
 

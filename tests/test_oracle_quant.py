@@ -105,15 +105,47 @@ def test_round_to_nearest_error_bound(bits, G):
     assert np.all(np.abs(xh - x) <= bound)
 
 
+def test_block_positions_worked_by_hand(golden_dir):
+    with open(os.path.join(golden_dir, "code_block_positions.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        fn = quant.key_code_positions if c["kind"] == "key" else quant.value_code_positions
+        byte, shift = fn(c["bits"], c["group"], c["D"])
+        assert (int(byte[c["token"], c["channel"]]), int(shift[c["token"], c["channel"]])) == (c["byte"], c["shift"]), c["why"]
+
+
+@pytest.mark.parametrize("bits,G,D", [(2, 32, 128), (2, 64, 128), (4, 64, 128), (4, 32, 128), (2, 32, 64), (4, 64, 64)])
+@pytest.mark.parametrize("values", [False, True])
+def test_block_order_is_a_permutation(bits, G, D, values):
+    """Every code of a group gets its own bits, the block is exactly G*D*b/8
+    bytes, and pack/unpack round-trip."""
+    byte, shift = quant._block_positions(bits, G, D, values)
+    slots = byte * 8 + shift
+    assert len(np.unique(slots)) == G * D
+    assert np.all(shift % bits == 0) and byte.max() == G * D * bits // 8 - 1
+    rng = np.random.default_rng(bits + G + D)
+    c = rng.integers(0, 1 << bits, size=(2, 3 * G, D)).astype(np.uint8)
+    blk = quant.pack_group_blocks(c, bits, G, values)
+    assert np.array_equal(quant.unpack_group_blocks(blk, bits, G, D, values), c)
+
+
+def test_pair_interleave():
+    p = np.arange(2 * 6 * 4).reshape(2, 6, 4)
+    q = quant.pair_interleave(p)
+    assert q.shape == (2, 3, 4, 2)
+    assert q[1, 2, 3].tolist() == [p[1, 4, 3], p[1, 5, 3]]
+    assert np.array_equal(quant.pair_deinterleave(q), p)
+
+
 def test_build_cache_layout():
     rng = np.random.default_rng(0)
     B, H, T, D, R, G = 2, 3, 96, 64, 32, 32
     k = rng.standard_normal((B, H, T, D)).astype(np.float32)
     v = rng.standard_normal((B, H, T, D)).astype(np.float32)
     c = quant.build_quant_cache(k, v, 2, G, R)
-    assert c["k_codes"].shape == (B, H, T - R, D // 4)
+    assert c["k_codes"].shape == (B, H, (T - R) // G, G * D // 4)
     assert c["k_scale"].shape == (B, H, (T - R) // G, D)
-    assert c["v_scale"].shape == (B, H, T - R, D // G)
+    assert c["v_scale"].shape == (B, H, (T - R) // 2, D // G, 2)
     kh, vh = quant.dequantize_cache(c)
     assert kh.shape == (B, H, T, D)
     assert np.array_equal(kh[:, :, T - R:], k[:, :, T - R:])
