@@ -314,11 +314,8 @@ def oracle_sample(w, budget_s: float):
         threads = os.cpu_count() or 1
     g = w["Hq"] // w["Hkv"]
     c = synth.random_quant_cache(1, 1, w["T"] - w["R"], w["R"], w["D"], w["bits"], w["G"], seed=7, device="cpu")
-    cache = dict(bits=c["bits"], group=c["group"], L_q=c["L_q"], R=c["R"],
-                 k_codes=c["k_codes"].numpy(), v_codes=c["v_codes"].numpy(),
-                 k_scale=c["k_scale"].numpy(), k_zero=c["k_zero"].numpy(),
-                 v_scale=c["v_scale"].numpy(), v_zero=c["v_zero"].numpy(),
-                 k_res=c["k_res"].float().numpy(), v_res=c["v_res"].float().numpy())
+    cache = dict(bits=c["bits"], group=c["group"], L_q=c["L_q"], R=c["R"], D=c["D"],
+                 records=c["records"].numpy(), k_res=c["k_res"].float().numpy(), v_res=c["v_res"].float().numpy())
     q = synth.normal((1, g, w["D"]), 8).float().numpy()
     per_slice = draft_bytes_per_layer(dict(w, B=1, Hkv=1))
     n = 0
@@ -340,10 +337,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama-3.1-8b-32k-kivi2", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the layer count (small cases for profiler captures; 0 = the workload's)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    w = WORKLOADS[args.workload]
+    w = dict(WORKLOADS[args.workload])
+    if args.layers > 0:
+        w["NL"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     peak, peak_kind = read_peaks()

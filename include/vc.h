@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define VC_ABI_VERSION 1
+#define VC_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define VC_API __attribute__((visibility("default")))
@@ -110,10 +110,26 @@ typedef struct vc_attn_shape {
  * quantised; the newest R tokens are kept in bf16 (the residual window, rows
  * 0..R-1 of a buffer of R_cap rows).
  *
- *   k_codes, v_codes  uint8 [B][Hkv][L_q / group][group * D * bits / 8]
- *   k_scale, k_zero   fp16  [B][Hkv][L_q / group][D]
- *   v_scale, v_zero   fp16  [B][Hkv][L_q / 2][D / group][2]
+ * Storage (this library's choice; the pages fix none).  Everything one group
+ * of `group` quantised tokens needs is one contiguous RECORD, so a stage of
+ * the draft kernel is a single bulk copy:
+ *
+ *   records   uint8 [B][Hkv][L_q / group][REC],  REC = 2 * CB + 8 * D,
+ *             CB = group * D * bits / 8
+ *   record:   [0, CB)            key codes of the group (block order below)
+ *             [CB, 2CB)          value codes of the group (block order below)
+ *             [2CB, +2D)         key scales, D fp16 in key-parameter order
+ *             [2CB + 2D, +2D)    key zeros, same order
+ *             [2CB + 4D, +2D)    value scales of the group's tokens, fp16
+ *                                [group/2][D/group][2]: for token pair
+ *                                (2p, 2p+1) and value group v, the two
+ *                                tokens' entries side by side
+ *             [2CB + 6D, +2D)    value zeros, same shape
  *   k_res, v_res      bf16  [B][Hkv][R_cap][D]
+ *
+ * Key-parameter order: channel c = 16 kt + 8 h + 2 t + e (h, e in {0,1},
+ * t in 0..3) sits at fp16 slot 2 (t * 2 (D/16) + 2 kt + h) + e, so the
+ * channel pairs one MMA lane multiplies form one contiguous run.
  *
  * Code blocks are stored in fragment-native order, the order in which the
  * tensor-core tiles of the draft kernel consume them.  For one group (a
@@ -130,20 +146,14 @@ typedef struct vc_attn_shape {
  * local tile i puts the first register's two codes at bits [bits*i, +bits)
  * and [16 + bits*i, +bits), the second register's at [8 + bits*i, +bits) and
  * [24 + bits*i, +bits).  Lane L's word w of token tile tt is 32-bit word
- * (tt * 32 + L) * NW + w of the group's block.  Value scales and zeros hold,
- * for each token pair (2p, 2p+1) and value group g, the two tokens' entries
- * side by side.
+ * (tt * 32 + L) * NW + w of the group's block.
  *
  *   bits in {2, 4}; group in {32, 64}; L_q >= 0 and a multiple of group;
- *   0 <= R <= R_cap; L_q + R >= 1.  Scales, zeros and codes must be finite
- *   and q * scale must stay inside the fp16 range (|q * scale| < 65504). */
+ *   0 <= R <= R_cap; L_q + R >= 1; records, k_res and v_res 16-byte
+ *   aligned.  Scales, zeros and codes must be finite and q * scale must stay
+ *   inside the fp16 range (|q * scale| < 65504). */
 typedef struct vc_quant_cache {
-  const void* k_codes;
-  const void* v_codes;
-  const void* k_scale;
-  const void* k_zero;
-  const void* v_scale;
-  const void* v_zero;
+  const void* records;
   const void* k_res;
   const void* v_res;
   int bits;
@@ -364,6 +374,19 @@ VC_API vc_status vc_debug_dequant(const vc_attn_shape* shape, const vc_quant_cac
                            void* stream);
 VC_API vc_status vc_debug_gather(const vc_attn_shape* shape, const vc_sparse_cache* cache, void* k_out, void* v_out,
                           void* ws, size_t ws_bytes, void* stream);
+
+/* vc_debug_quant_partition reports, without touching a GPU, how
+ * vc_draft_attn_quant cuts one call into blocks when at most target_blocks
+ * blocks are allowed (the real call uses SMs x resident blocks).  The call is
+ * one axis of stages: every (request, head) unit's quantised groups
+ * (n_quant_stages in all), then every unit's residual rows, 16 per stage
+ * (n_stages in all).  Block k owns stages [first_stage[k], first_stage[k+1]);
+ * *max_segments is the most unit parts (quantised or residual part of one
+ * unit) one block touches.  first_stage may be NULL; else it needs
+ * max_blocks >= *n_blocks + 1 entries. */
+VC_API vc_status vc_debug_quant_partition(const vc_attn_shape* shape, const vc_quant_cache* cache,
+                                          int target_blocks, int64_t* first_stage, int max_blocks, int* n_blocks,
+                                          int* max_segments, int64_t* n_stages, int64_t* n_quant_stages);
 
 #ifdef __cplusplus
 }

@@ -20,89 +20,131 @@
 // fp32.  The result equals attention over fp32-dequantised values up to fp32
 // rounding (the oracle dequantises with one fp32 FMA per element).
 //
-// Work layout.  grid (S, B * Hkv): block x < units-with-residual ... see
-// plan_quant(); a block owns a contiguous run of groups (G tokens each) of one
-// (request, KV head), or that head's bf16 residual rows.  Each of its 4 warps
-// takes groups round-robin and streams them through a private ring of
-// shared-memory stages filled by 1-D bulk copies (codes, scales, zeros of a
-// group are contiguous in HBM, so one group = 6 bulk copies) completed on
-// mbarriers; waits are bounded.  All g query heads of the GQA group share each
-// group read (they are the MMA's N columns).
+// Work layout.  The job is one axis of STAGES: first every (request, KV
+// head) unit's quantised groups, NG consecutive group records per stage,
+// then every unit's bf16 residual, 16 rows per stage.  A persistent grid of
+// (SMs x resident blocks) blocks cuts that axis into equal-cost contiguous
+// ranges (Partition); inside a block the 4 warps take the range's stages
+// round-robin.  A quantised stage is ONE bulk copy of contiguous records into
+// the warp's private ring (NST stages deep, completed on mbarriers, waits
+// bounded).  Wherever the range crosses from one unit's segment to the next,
+// the block merges its warps' online-softmax states into one partial of that
+// segment; the last block to finish a unit (atomic ticket) merges the unit's
+// partials into the output.  All g query heads of a GQA group share each
+// record (they are the MMA's N columns).
 //
 // MMA arrangement (mma.sync m16n8k16, fp16 x fp16 -> fp32):
 //   scores:  D[token][col] = codes[token][chan] x qfold[chan][col]
 //            col = 2 * head + part (part 0 = high, 1 = low), 4 heads per n-tile
 //   values:  D[chan][col]  = codes^T[chan][token] x pfold[token][col]
 // Code bits reach the tensor cores as fp16 subnormals (one AND per two codes,
-// see KLane / VLane); the assignment of MMA k-slots / rows to channels is
-// chosen so that each lane's codes sit at fixed bit positions.
+// see Frag); the record layout puts each lane's codes at fixed bit positions
+// and each lane's key scales in one contiguous run.
 #include <mutex>
 
-#include "vc_splitk.cuh"
+#include "vc_common.cuh"
 
 namespace vc {
 namespace {
 
-constexpr int kQNW = 4;  // warps per block
+constexpr int kQNW = 4;          // warps per block
+constexpr int kResRows = 16;     // residual rows per stage
+constexpr int kMergeChunk = 64;  // partials weighed per pass when a unit is finished
+constexpr int kResCostWeight = 2;  // residual stages are not pipelined: count their bytes twice
 
 template <int BITS, int G, int D, int NT>
 struct QCfg {
-  static constexpr int RB = D * BITS / 8;           // bytes per packed token row
-  static constexpr int WPR = RB / 4;                // 32-bit words per row
-  static constexpr int KC_B = G * RB;               // key (or value) codes per group
-  static constexpr int SC_B = 2 * D;                // each of sk, zk, sv, zv per group
-  static constexpr int QSTAGE = 2 * KC_B + 4 * SC_B;
-  static constexpr int NST = QSTAGE <= 4096 ? 4 : 2;
-  static constexpr int RS = D * 2 + 16;             // residual smem row stride
-  static constexpr int RSTAGE = 32 * RS;            // 16 K + 16 V residual rows
-  static constexpr int RING = (NST * QSTAGE > RSTAGE) ? NST * QSTAGE : RSTAGE;
-  static constexpr int PS_B = 2 * (4 * NT * G) * 2;  // p high/low parts, fp16 [heads][G] each
+  static constexpr int CB = G * D * BITS / 8;  // one code block (keys or values) of a group
+  static constexpr int REC = 2 * CB + 8 * D;   // group record: kc | vc | sk | zk | sv | zv
+  static constexpr int OFF_VC = CB;
+  static constexpr int OFF_SK = 2 * CB;
+  static constexpr int OFF_ZK = 2 * CB + 2 * D;
+  static constexpr int OFF_SV = 2 * CB + 4 * D;
+  static constexpr int OFF_ZV = 2 * CB + 6 * D;
+  static constexpr int NG = REC >= 3072 ? 1 : 3072 / REC;  // records per stage
+  static constexpr int STAGE = NG * REC;
+  static constexpr int NST0 = (NT == 1 ? 9216 : 18432) / STAGE;
+  static constexpr int NST = NST0 < 2 ? 2 : (NST0 > 4 ? 4 : NST0);  // ring depth
+  static constexpr int RS = D * 2 + 16;                              // residual smem row stride
+  static constexpr int RSTAGE = 2 * kResRows * RS;                   // 16 K + 16 V rows
+  static constexpr int RING0 = NST * STAGE > RSTAGE ? NST * STAGE : RSTAGE;
+  static constexpr int RING = (RING0 + 127) / 128 * 128;
+  static constexpr int HEADS = 4 * NT;
+  static constexpr int PS_B = 2 * HEADS * G * 2;  // p high / low parts, fp16 [HEADS][G] each
   static constexpr int WARP_B = RING + PS_B;
-  static constexpr int BAR_OFF = kQNW * WARP_B;
-  static constexpr int SMEM_B = BAR_OFF + kQNW * NST * 8 + 16;
-  static constexpr int KT = D / 16;                 // channel tiles
-  static constexpr int CPG = D / G;                 // value groups per token
+  static constexpr int STATE_OFF = kQNW * WARP_B;                       // fp32 [kQNW][HEADS][D]
+  static constexpr int ML_OFF = STATE_OFF + kQNW * HEADS * D * 4;       // fp32 [kQNW][HEADS][2]
+  static constexpr int MW_OFF = ML_OFF + kQNW * HEADS * 2 * 4;          // merge weights + (M, L)
+  static constexpr int MW_FLOATS = kMergeChunk * HEADS + 2 * HEADS;
+  static constexpr int SLOT_OFF = (MW_OFF + MW_FLOATS * 4 + 15) / 16 * 16;  // int64 [kMergeChunk]
+  static constexpr int BAR_OFF = SLOT_OFF + kMergeChunk * 8;
+  static constexpr int TICK_OFF = BAR_OFF + kQNW * (NST + 1) * 8;
+  static constexpr int SMEM_B = TICK_OFF + 16;
+  static constexpr int KT = D / 16;   // channel tiles
+  static constexpr int CPG = D / G;   // value groups per token
   static_assert(G % 32 == 0, "group must be a multiple of 32");
+  static_assert(REC % 16 == 0 && STAGE % 16 == 0, "bulk copies need 16-byte multiples");
+  static_assert(PS_B >= HEADS * kResRows * 4, "residual scores share the p buffer");
+  static_assert(WARP_B % 128 == 0, "warp areas stay 128-byte aligned");
+};
+
+// The stage axis and its cut into blocks; the same arithmetic runs on the
+// host (planning, workspace size) and on the device.
+//   stage s <  QZ : quantised stage s % sq of unit s / sq   (cost cq)
+//   stage s >= QZ : residual stage (s - QZ) % sr of unit (s - QZ) / sr (cost cr)
+// Block k owns the stages whose start cost c_s satisfies
+// ceil(k C / n) <= c_s < ceil((k + 1) C / n); equivalently the block of stage
+// s is floor(c_s n / C).  The host keeps n <= C / max(cq, cr), so every block
+// owns at least one stage.  Segment of a stage: its unit's quantised part
+// (id u) or residual part (id U + u).
+struct Partition {
+  int64_t ng;      // groups per unit
+  int64_t QZ;      // stages in the quantised zone = U * sq
+  int64_t S_tot;   // all stages
+  int64_t cq, cr;  // cost of one quantised / residual stage
+  int64_t C;       // total cost
+  int U, sq, sr, nblk;
+
+  __host__ __device__ int64_t cost(int64_t s) const { return s < QZ ? s * cq : QZ * cq + (s - QZ) * cr; }
+  __host__ __device__ int64_t first(int k) const {
+    if (k <= 0) return 0;
+    if (k >= nblk) return S_tot;
+    const int64_t T = (static_cast<int64_t>(k) * C + nblk - 1) / nblk;
+    if (QZ > 0 && T <= (QZ - 1) * cq) return (T + cq - 1) / cq;
+    const int64_t base = QZ * cq;
+    if (T <= base) return QZ;
+    const int64_t s = QZ + (T - base + cr - 1) / cr;
+    return s < S_tot ? s : S_tot;
+  }
+  __host__ __device__ int block_of(int64_t s) const {
+    const int64_t k = cost(s) * nblk / C;
+    return k < nblk ? static_cast<int>(k) : nblk - 1;
+  }
+  __host__ __device__ int seg_of(int64_t s) const {
+    return s < QZ ? static_cast<int>(s / sq) : U + static_cast<int>((s - QZ) / sr);
+  }
+  __host__ __device__ int64_t seg_begin(int seg) const {
+    return seg < U ? static_cast<int64_t>(seg) * sq : QZ + static_cast<int64_t>(seg - U) * sr;
+  }
+  __host__ __device__ int64_t seg_end(int seg) const { return seg_begin(seg) + (seg < U ? sq : sr); }
 };
 
 struct QArgs {
-  const uint8_t* kc;
-  const uint8_t* vc;
-  const __half* sk;
-  const __half* zk;
-  const __half* sv;
-  const __half* zv;
+  const uint8_t* rec;  // [U][ng][REC] group records
   const __nv_bfloat16* kr;
   const __nv_bfloat16* vr;
   const __nv_bfloat16* q;
-  int64_t L_q;
+  Partition P;
   int R, R_cap;
   int Hq, Hkv, g;
-  int S, Sq, GPC, res_first;  // chunks; quant chunks; groups per chunk; residual blocks lead
+  int MAXS;  // partial slots per block
   float scale_log2;
   uint32_t* flags;
-  SplitKOut o;
+  uint32_t* tickets;  // [U], zero between calls
+  float* part_o;      // [nblk * MAXS][g][D]
+  float* part_ml;     // [nblk * MAXS][g][2]
+  float* out;         // [B][Hq][D]
 };
-
-// Online-softmax update of one head state with 4 new (already scaled) scores.
-__device__ __forceinline__ float softmax_step(float (&x)[4], float& m_run, float& l_run, int xor0) {
-  float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-  tmax = warp_max_xor(tmax, xor0);
-  tmax = warp_max_xor(tmax, xor0 * 2);
-  tmax = warp_max_xor(tmax, xor0 * 4);
-  const float m_new = fmaxf(m_run, tmax);
-  const float m_use = m_new == -INFINITY ? 0.f : m_new;
-  const float alpha = ex2(m_run - m_use);
-  float ps = 0.f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    x[j] = ex2(x[j] - m_use);
-    ps += x[j];
-  }
-  l_run = l_run * alpha + ps;
-  m_run = m_new;
-  return alpha;
-}
 
 // ---- code extraction shared by the attention kernel and vc_debug_dequant
 //
@@ -158,10 +200,43 @@ __device__ __forceinline__ void load_cpg(const uint32_t* p, uint32_t (&w)[CPG]) 
   }
 }
 
+// Where this warp's next quantised stage to fetch lives: unit u, stage ls of
+// that unit.  Advancing by kQNW stages needs no division.
+struct IssuePtr {
+  int64_t u, ls;
+  __device__ void start(const Partition& P, int64_t s) {
+    u = s / P.sq;
+    ls = s - u * P.sq;
+  }
+  __device__ void advance(const Partition& P) {
+    ls += kQNW;
+    while (ls >= P.sq) {
+      ls -= P.sq;
+      ++u;
+    }
+  }
+};
+
+// One bulk copy of this warp's quantised stage number i (at ip) into its ring slot.
+template <typename C>
+__device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring, uint64_t* bars, int lane, int i,
+                                            const IssuePtr& ip) {
+  const int64_t g0 = ip.ls * C::NG;
+  const int64_t left = a.P.ng - g0;
+  const uint32_t bytes = static_cast<uint32_t>((left < C::NG ? left : C::NG) * C::REC);
+  const int slot = i % C::NST;
+  if (lane == 0) {
+    mbar_arrive_expect_tx(&bars[slot], bytes);
+    bulk_g2s(ring + slot * C::STAGE, a.rec + (ip.u * a.P.ng + g0) * C::REC, bytes, &bars[slot]);
+  }
+}
+
 // ----------------------------------------------------------- quantised part
+// Processes this warp's stages of unit u's quantised segment (the prefetch
+// pipeline runs on across segments) and leaves the warp's state in its slot.
 template <int BITS, int G, int D, int NT>
-__device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b, int h, int qchunk,
-                           float* wst_ml, bool& ok) {
+__device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, int u, int64_t B0, int my_nq,
+                          int& iq, int& issued, IssuePtr& ip, bool& ok, float* st_o, float* st_ml) {
   using C = QCfg<BITS, G, D, NT>;
   using F = Frag<BITS>;
   constexpr unsigned FULL = 0xffffffffu;
@@ -169,46 +244,20 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int part = gid & 1;
-  unsigned char* ring = smem + warp * C::WARP_B;
-  __half* Ph = reinterpret_cast<__half*>(ring + C::RING);  // [4 * NT][G] fp16 high parts of p
-  __half* Pl = Ph + 4 * NT * G;                            // low parts
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + warp * C::NST;
+  __half* Ph = reinterpret_cast<__half*>(ring + C::RING);  // [HEADS][G] fp16 high parts of p
+  __half* Pl = Ph + C::HEADS * G;                          // low parts
+  const int b = u / a.Hkv, h = u - b * a.Hkv;
 
-  const int64_t n_groups = a.L_q / G;
-  const int64_t g_begin = static_cast<int64_t>(qchunk) * a.GPC;
-  const int64_t g_end = min(n_groups, g_begin + a.GPC);
-  const int ngr = static_cast<int>(g_end - g_begin);
-  const int my_n = ngr > warp ? (ngr - warp + kQNW - 1) / kQNW : 0;
-
-  const uint8_t* kc_u = a.kc + static_cast<size_t>(unit) * a.L_q * C::RB;
-  const uint8_t* vc_u = a.vc + static_cast<size_t>(unit) * a.L_q * C::RB;
-  const __half* sk_u = a.sk + static_cast<size_t>(unit) * n_groups * D;
-  const __half* zk_u = a.zk + static_cast<size_t>(unit) * n_groups * D;
-  const __half* sv_u = a.sv + static_cast<size_t>(unit) * a.L_q * C::CPG;
-  const __half* zv_u = a.zv + static_cast<size_t>(unit) * a.L_q * C::CPG;
-
-  auto issue = [&](int i) {
-    const int s = i % C::NST;
-    const int64_t j = g_begin + warp + static_cast<int64_t>(i) * kQNW;
-    unsigned char* st = ring + s * C::QSTAGE;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bars[s], C::QSTAGE);
-      bulk_g2s(st, kc_u + j * C::KC_B, C::KC_B, &bars[s]);
-      bulk_g2s(st + C::KC_B, vc_u + j * C::KC_B, C::KC_B, &bars[s]);
-      bulk_g2s(st + 2 * C::KC_B, sk_u + j * D, C::SC_B, &bars[s]);
-      bulk_g2s(st + 2 * C::KC_B + C::SC_B, zk_u + j * D, C::SC_B, &bars[s]);
-      bulk_g2s(st + 2 * C::KC_B + 2 * C::SC_B, sv_u + j * G * C::CPG, C::SC_B, &bars[s]);
-      bulk_g2s(st + 2 * C::KC_B + 3 * C::SC_B, zv_u + j * G * C::CPG, C::SC_B, &bars[s]);
-    }
-  };
-
-  const uint32_t lomask = part ? 0xffffffffu : 0u;  // low-part columns
+  // per-lane constants of the high/low split: part 0 lanes keep the rounded
+  // product, part 1 lanes its rounding error
+  const uint32_t kap = part ? 0xBC00BC00u : 0u;  // (-1, -1) or (0, 0) in fp16
+  const uint32_t mu = part ? 0x3C003C00u : 0u;   // (1, 1) or (0, 0)
 
   // ---- query registers (fp16, exact from bf16), column head = nt*4 + gid/2,
   //      natural channel pairs (16kt + 2tig, +1) and (16kt + 2tig + 8, +9)
-  //   q2s: scaled by 2^-(bits * (kt % TPW)) of the code encoding
-  //   qb : unscaled, high columns only (zero-point MMA)
-  uint32_t q2s[C::KT][NT][2], qb[C::KT][NT][2];
+  //   q2s: scaled by 2^-(bits * (kt % TPW)) of the code encoding (the
+  //        zero-point MMA uses it too, with the zeros scaled up to match)
+  uint32_t q2s[C::KT][NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int hh = nt * 4 + (gid >> 1);
@@ -221,8 +270,6 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
       const float2 hi = unpack_bf2(*reinterpret_cast<const uint32_t*>(qp + kt * 16 + 8 + 2 * tig));
       q2s[kt][nt][0] = hv ? pack_h2(lo.x * f, lo.y * f) : 0u;
       q2s[kt][nt][1] = hv ? pack_h2(hi.x * f, hi.y * f) : 0u;
-      qb[kt][nt][0] = (hv && !part) ? pack_h2(lo.x, lo.y) : 0u;
-      qb[kt][nt][1] = (hv && !part) ? pack_h2(hi.x, hi.y) : 0u;
     }
   }
   // the score MMAs accumulate scores * 2^-24; undo it together with the softmax scale
@@ -240,178 +287,209 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
     for (int mc = 0; mc < C::KT; ++mc) acc[mc][nt][0] = acc[mc][nt][1] = acc[mc][nt][2] = acc[mc][nt][3] = 0.f;
   }
 
-  if (lane == 0)
-    for (int s = 0; s < C::NST; ++s) mbar_init(&bars[s], 1);
-  fence_mbar_init();
-  __syncwarp();
-  const int pre = my_n < C::NST - 1 ? my_n : C::NST - 1;
-  for (int i = 0; i < pre; ++i) issue(i);
-
-  for (int i = 0; i < my_n; ++i) {
-    if (i + C::NST - 1 < my_n) {
+  const int64_t seg_lo = static_cast<int64_t>(u) * a.P.sq, seg_hi = seg_lo + a.P.sq;
+  for (; iq < my_nq; ++iq) {
+    const int64_t s = B0 + warp + static_cast<int64_t>(iq) * kQNW;
+    if (s >= seg_hi) break;
+    if (!ok) continue;
+    if (issued < my_nq && issued <= iq + C::NST - 1) {
       fence_proxy_async_smem();
       __syncwarp();
-      issue(i + C::NST - 1);
+      issue_stage<C>(a, ring, bars, lane, issued, ip);
+      ip.advance(a.P);
+      ++issued;
     }
-    const int s = i % C::NST;
-    if (!__all_sync(FULL, mbar_wait_bounded(&bars[s], (i / C::NST) & 1, a.flags))) {  // warp-uniform
+    const int slot = iq % C::NST;
+    if (!__all_sync(FULL, mbar_wait_bounded(&bars[slot], (iq / C::NST) & 1, a.flags))) {  // warp-uniform
       ok = false;
-      for (int k = i; k < my_n && k < i + C::NST; ++k)
-        mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
-      break;
+      for (int k = iq; k < issued; ++k) mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
+      continue;
     }
-    const unsigned char* st = ring + s * C::QSTAGE;
-    const uint32_t* kcw = reinterpret_cast<const uint32_t*>(st);
-    const uint32_t* vcw = reinterpret_cast<const uint32_t*>(st + C::KC_B);
-    const __half* sk = reinterpret_cast<const __half*>(st + 2 * C::KC_B);
-    const __half* zk = sk + D;
-    const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(zk + D);      // [G/2][CPG] token pairs
-    const uint32_t* zv32 = sv32 + G / 2 * C::CPG;
-
-    // (1) fold the key scales into q (fp16 high part in part-0 columns, low
-    //     part in part-1 columns) and the zero-point term sum_c q_c z_c
-    uint32_t qf[C::KT][NT][2];
-    float kb[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) kb[nt][0] = kb[nt][1] = kb[nt][2] = kb[nt][3] = 0.f;
-#pragma unroll
-    for (int kt = 0; kt < C::KT; ++kt) {
-      const uint32_t sA = *reinterpret_cast<const uint32_t*>(sk + kt * 16 + 2 * tig);
-      const uint32_t sC = *reinterpret_cast<const uint32_t*>(sk + kt * 16 + 8 + 2 * tig);
-      const uint32_t z0 = *reinterpret_cast<const uint32_t*>(zk + kt * 16 + 2 * tig);
-      const uint32_t z8 = *reinterpret_cast<const uint32_t*>(zk + kt * 16 + 8 + 2 * tig);
-      const uint32_t za[4] = {z0, z0, z8, z8};
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t qa = q2s[kt][nt][0], qc = q2s[kt][nt][1];
-        qf[kt][nt][0] = hfma2(qa, sA, hmul2((qa ^ 0x80008000u) & lomask, sA));
-        qf[kt][nt][1] = hfma2(qc, sC, hmul2((qc ^ 0x80008000u) & lomask, sC));
-        mma_f16(kb[nt], za, qb[kt][nt][0], qb[kt][nt][1]);
-      }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) kb[nt][e] *= 5.9604644775390625e-8f;  // 2^-24
-
-    // (2) 32-token sub-blocks: scores, softmax, P . V
+    const int64_t g0 = (s - seg_lo) * C::NG;
+    const int n_here = a.P.ng - g0 < C::NG ? static_cast<int>(a.P.ng - g0) : C::NG;
 #pragma unroll 1
-    for (int sb = 0; sb < G / 32; ++sb) {
-      float sc[2][NT][4];
+    for (int gi = 0; gi < n_here; ++gi) {
+      const unsigned char* rs = ring + slot * C::STAGE + gi * C::REC;
+      const uint32_t* kcw = reinterpret_cast<const uint32_t*>(rs);
+      const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
+      const uint4* skw = reinterpret_cast<const uint4*>(rs + C::OFF_SK) + tig * (C::KT / 2);
+      const uint4* zkw = reinterpret_cast<const uint4*>(rs + C::OFF_ZK) + tig * (C::KT / 2);
+      const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);  // [G/2][CPG] token pairs
+      const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
+
+      // (2) 32-token sub-blocks: scores, softmax, P . V
+      float kb[NT][4];  // zero-point term sum_c q_c z_c (high columns), from sub-block 0
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
+      for (int nt = 0; nt < NT; ++nt) kb[nt][0] = kb[nt][1] = kb[nt][2] = kb[nt][3] = 0.f;
+#pragma unroll 1
+      for (int sb = 0; sb < G / 32; ++sb) {
+        // scores of token tiles mt = 0, 1.  Per channel tile kt the key scales
+        // are folded into q right before use (fp16 high part in part-0
+        // columns, low part in part-1 columns); lane tig's scale words for
+        // (kt, h) are word 2kt + h of its run.
+        float sc[2][NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sc[mt][nt][e] = kb[nt][e];
-        uint32_t w[NW];
-        load_words(kcw + ((sb * 2 + mt) * 32 + lane) * NW, w);
+          for (int nt = 0; nt < NT; ++nt) sc[mt][nt][0] = sc[mt][nt][1] = sc[mt][nt][2] = sc[mt][nt][3] = 0.f;
 #pragma unroll
         for (int j = 0; j < NW / 2; ++j) {
-          const uint32_t X = w[2 * j], Y = w[2 * j + 1], xs = X >> 8, ys = Y >> 8;
+          const uint2 w0 = *reinterpret_cast<const uint2*>(kcw + ((sb * 2 + 0) * 32 + lane) * NW + 2 * j);
+          const uint2 w1 = *reinterpret_cast<const uint2*>(kcw + ((sb * 2 + 1) * 32 + lane) * NW + 2 * j);
+          const uint32_t xs0 = w0.x >> 8, ys0 = w0.y >> 8, xs1 = w1.x >> 8, ys1 = w1.y >> 8;
 #pragma unroll
           for (int i = 0; i < F::TPW; ++i) {
             const int kt = F::TPW * j + i;
+            const uint4 s4 = skw[kt >> 1];
+            const uint32_t sA = (kt & 1) ? s4.z : s4.x, sC = (kt & 1) ? s4.w : s4.y;
             const uint32_t m = F::mask(i);
-            const uint32_t af[4] = {X & m, xs & m, Y & m, ys & m};
+            const uint32_t a0[4] = {w0.x & m, xs0 & m, w0.y & m, ys0 & m};
+            const uint32_t a1[4] = {w1.x & m, xs1 & m, w1.y & m, ys1 & m};
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_f16(sc[mt][nt], af, qf[kt][nt][0], qf[kt][nt][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+              const uint32_t qa = q2s[kt][nt][0], qc = q2s[kt][nt][1];
+              const uint32_t fa = hfma2(qa, sA, hmul2(hmul2(qa, sA), kap));
+              const uint32_t fc = hfma2(qc, sC, hmul2(hmul2(qc, sC), kap));
+              mma_f16(sc[0][nt], a0, fa, fc);
+              mma_f16(sc[1][nt], a1, fa, fc);
+            }
+            if (sb == 0) {
+              // zeros times 2^(bits i) (exact) against q2s: sum_c z_c q_c, in
+              // both columns of a head (only the high one is used)
+              const uint4 z4 = zkw[kt >> 1];
+              uint32_t z0 = (kt & 1) ? z4.z : z4.x, z8 = (kt & 1) ? z4.w : z4.y;
+              if (i > 0) {
+                const uint32_t f2 = static_cast<uint32_t>(15 + BITS * i) << 10;  // fp16 2^(bits i)
+                z0 = hmul2(z0, f2 | (f2 << 16));
+                z8 = hmul2(z8, f2 | (f2 << 16));
+              }
+              const uint32_t za[4] = {z0, z0, z8, z8};
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma_f16(kb[nt], za, q2s[kt][nt][0], q2s[kt][nt][1]);
+            }
           }
         }
-      }
-      // softmax per head nt*4 + tig over tokens sb*32 + {gid, gid+8, gid+16, gid+24}
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float x[4] = {(sc[0][nt][0] + sc[0][nt][1]) * scl, (sc[0][nt][2] + sc[0][nt][3]) * scl,
-                      (sc[1][nt][0] + sc[1][nt][1]) * scl, (sc[1][nt][2] + sc[1][nt][3]) * scl};
-        const float alpha = softmax_step(x, m_run[nt], l_run[nt], 4);
-#pragma unroll
-        for (int mc = 0; mc < C::KT; ++mc) {
-          acc[mc][nt][0] *= alpha;
-          acc[mc][nt][1] *= alpha;
-          acc[mc][nt][2] *= alpha;
-          acc[mc][nt][3] *= alpha;
-        }
-        vb[nt][0] *= alpha;
-        vb[nt][1] *= alpha;
-        vb[nt][2] *= alpha;
-        vb[nt][3] *= alpha;
-        // p as fp16 high + low parts, split once here for the value side
-        const uint32_t h01 = pack_h2(x[0], x[1]), h23 = pack_h2(x[2], x[3]);
-        const float2 f01 = unpack_h2(h01), f23 = unpack_h2(h23);
-        const uint32_t l01 = pack_h2(x[0] - f01.x, x[1] - f01.y), l23 = pack_h2(x[2] - f23.x, x[3] - f23.y);
-        unsigned short* ph = reinterpret_cast<unsigned short*>(Ph + (nt * 4 + tig) * G + sb * 32 + gid);
-        unsigned short* pl = reinterpret_cast<unsigned short*>(Pl + (nt * 4 + tig) * G + sb * 32 + gid);
-        ph[0] = static_cast<unsigned short>(h01);
-        ph[8] = static_cast<unsigned short>(h01 >> 16);
-        ph[16] = static_cast<unsigned short>(h23);
-        ph[24] = static_cast<unsigned short>(h23 >> 16);
-        pl[0] = static_cast<unsigned short>(l01);
-        pl[8] = static_cast<unsigned short>(l01 >> 16);
-        pl[16] = static_cast<unsigned short>(l23);
-        pl[24] = static_cast<unsigned short>(l23 >> 16);
-      }
-      __syncwarp();
-#pragma unroll
-      for (int ktt = 0; ktt < 2; ++ktt) {
-        const int t0 = sb * 32 + ktt * 16 + 2 * tig;  // tokens t0, t0+1, t0+8, t0+9
-        uint32_t ph01[NT], ph89[NT], plm01[NT], plm89[NT], phn01[NT], phn89[NT];
+        // softmax per head nt*4 + tig over tokens sb*32 + {gid, gid+8, gid+16, gid+24};
+        // the running max is raised only when a score exceeds it by more
+        // than 2^8 (lazy rescale; p <= 256 keeps every fp16/fp32 value in range)
+        float x[NT][4], tmax[NT];
+        bool need = false;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const int hh = nt * 4 + (gid >> 1);
-          ph01[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0);
-          ph89[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0 + 8);
-          const uint32_t pl01 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0);
-          const uint32_t pl89 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0 + 8);
-          plm01[nt] = pl01 & lomask;
-          plm89[nt] = pl89 & lomask;
-          phn01[nt] = (ph01[nt] ^ 0x80008000u) & lomask;
-          phn89[nt] = (ph89[nt] ^ 0x80008000u) & lomask;
-          // value zero-point term: A = z_v^T (row = value group gid), B = p (high or low column)
-          uint32_t za[4] = {0u, 0u, 0u, 0u};
-          if (gid < C::CPG) {
-            za[0] = zv32[(t0 >> 1) * C::CPG + gid];
-            za[2] = zv32[((t0 + 8) >> 1) * C::CPG + gid];
-          }
-          mma_f16(vb[nt], za, part ? pl01 : ph01[nt], part ? pl89 : ph89[nt]);
+          // zero-point term (exact fp32, rows gid and gid+8 alike) into the 2^-24 domain
+          const float k0 = kb[nt][0] * 5.9604644775390625e-8f;
+          const float k8 = kb[nt][2] * 5.9604644775390625e-8f;
+          x[nt][0] = (sc[0][nt][0] + sc[0][nt][1] + k0) * scl;
+          x[nt][1] = (sc[0][nt][2] + sc[0][nt][3] + k8) * scl;
+          x[nt][2] = (sc[1][nt][0] + sc[1][nt][1] + k0) * scl;
+          x[nt][3] = (sc[1][nt][2] + sc[1][nt][3] + k8) * scl;
+          float t = fmaxf(fmaxf(x[nt][0], x[nt][1]), fmaxf(x[nt][2], x[nt][3]));
+          t = warp_max_xor(t, 4);
+          t = warp_max_xor(t, 8);
+          t = warp_max_xor(t, 16);
+          tmax[nt] = t;
+          need |= t > m_run[nt] + 8.f;
         }
-        // folded p*s for every value group: high part (part 0) or low part (part 1)
-        uint32_t pf[C::CPG][NT][2];
-        {
+        if (__any_sync(FULL, need)) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const float m_new = fmaxf(m_run[nt], tmax[nt]);
+            const float alpha = ex2(m_run[nt] - m_new);
+            m_run[nt] = m_new;
+            l_run[nt] *= alpha;
+#pragma unroll
+            for (int mc = 0; mc < C::KT; ++mc) {
+              acc[mc][nt][0] *= alpha;
+              acc[mc][nt][1] *= alpha;
+              acc[mc][nt][2] *= alpha;
+              acc[mc][nt][3] *= alpha;
+            }
+            vb[nt][0] *= alpha;
+            vb[nt][1] *= alpha;
+            vb[nt][2] *= alpha;
+            vb[nt][3] *= alpha;
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float p[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) p[j] = ex2(x[nt][j] - m_run[nt]);
+          l_run[nt] += (p[0] + p[1]) + (p[2] + p[3]);
+          // p as fp16 high + low parts, split once here for the value side
+          const uint32_t h01 = pack_h2(p[0], p[1]), h23 = pack_h2(p[2], p[3]);
+          const float2 f01 = unpack_h2(h01), f23 = unpack_h2(h23);
+          const uint32_t l01 = pack_h2(p[0] - f01.x, p[1] - f01.y), l23 = pack_h2(p[2] - f23.x, p[3] - f23.y);
+          unsigned short* ph = reinterpret_cast<unsigned short*>(Ph + (nt * 4 + tig) * G + sb * 32 + gid);
+          unsigned short* pl = reinterpret_cast<unsigned short*>(Pl + (nt * 4 + tig) * G + sb * 32 + gid);
+          ph[0] = static_cast<unsigned short>(h01);
+          ph[8] = static_cast<unsigned short>(h01 >> 16);
+          ph[16] = static_cast<unsigned short>(h23);
+          ph[24] = static_cast<unsigned short>(h23 >> 16);
+          pl[0] = static_cast<unsigned short>(l01);
+          pl[8] = static_cast<unsigned short>(l01 >> 16);
+          pl[16] = static_cast<unsigned short>(l23);
+          pl[24] = static_cast<unsigned short>(l23 >> 16);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int ktt = 0; ktt < 2; ++ktt) {
+          const int t0 = sb * 32 + ktt * 16 + 2 * tig;  // tokens t0, t0+1, t0+8, t0+9
+          uint32_t ph01[NT], ph89[NT], plm01[NT], plm89[NT], phn01[NT], phn89[NT];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const int hh = nt * 4 + (gid >> 1);
+            ph01[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0);
+            ph89[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0 + 8);
+            const uint32_t pl01 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0);
+            const uint32_t pl89 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0 + 8);
+            plm01[nt] = hmul2(pl01, mu);
+            plm89[nt] = hmul2(pl89, mu);
+            phn01[nt] = hmul2(ph01[nt], kap);
+            phn89[nt] = hmul2(ph89[nt], kap);
+            // value zero-point term: A = z_v^T (row = value group gid), B = p (high or low column)
+            uint32_t za[4] = {0u, 0u, 0u, 0u};
+            if (gid < C::CPG) {
+              za[0] = zv32[(t0 >> 1) * C::CPG + gid];
+              za[2] = zv32[((t0 + 8) >> 1) * C::CPG + gid];
+            }
+            mma_f16(vb[nt], za, part ? pl01 : ph01[nt], part ? pl89 : ph89[nt]);
+          }
+          // folded p*s per value group, made right before the channel tiles
+          // that use it: high part (part 0) or low part (part 1)
           uint32_t s01[C::CPG], s89[C::CPG];
           load_cpg<C::CPG>(sv32 + (t0 >> 1) * C::CPG, s01);
           load_cpg<C::CPG>(sv32 + ((t0 + 8) >> 1) * C::CPG, s89);
+          uint32_t w[NW];
+          load_words(vcw + ((sb * 2 + ktt) * 32 + lane) * NW, w);
+          uint32_t pf[NT][2];
 #pragma unroll
-          for (int cg = 0; cg < C::CPG; ++cg)
+          for (int j = 0; j < NW / 2; ++j) {
+            const uint32_t X = w[2 * j], Y = w[2 * j + 1], xs = X >> 8, ys = Y >> 8;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              pf[cg][nt][0] = hfma2(plm01[nt], s01[cg], hfma2(ph01[nt], s01[cg], hmul2(phn01[nt], s01[cg])));
-              pf[cg][nt][1] = hfma2(plm89[nt], s89[cg], hfma2(ph89[nt], s89[cg], hmul2(phn89[nt], s89[cg])));
+            for (int i = 0; i < F::TPW; ++i) {
+              const int mc = F::TPW * j + i;  // 16-channel tile
+              const int cg = mc * 16 / G;
+              if (mc == 0 || (mc - 1) * 16 / G != cg) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                  pf[nt][0] = hfma2(plm01[nt], s01[cg], hfma2(ph01[nt], s01[cg], hmul2(phn01[nt], s01[cg])));
+                  pf[nt][1] = hfma2(plm89[nt], s89[cg], hfma2(ph89[nt], s89[cg], hmul2(phn89[nt], s89[cg])));
+                }
+              }
+              const uint32_t m = F::mask(i);
+              const uint32_t af[4] = {X & m, Y & m, xs & m, ys & m};
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma_f16(acc[mc][nt], af, pf[nt][0], pf[nt][1]);
             }
-        }
-        uint32_t w[NW];
-        load_words(vcw + ((sb * 2 + ktt) * 32 + lane) * NW, w);
-#pragma unroll
-        for (int j = 0; j < NW / 2; ++j) {
-          const uint32_t X = w[2 * j], Y = w[2 * j + 1], xs = X >> 8, ys = Y >> 8;
-#pragma unroll
-          for (int i = 0; i < F::TPW; ++i) {
-            const int mc = F::TPW * j + i;  // 16-channel tile
-            const int cg = mc * 16 / G;
-            const uint32_t m = F::mask(i);
-            const uint32_t af[4] = {X & m, Y & m, xs & m, ys & m};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_f16(acc[mc][nt], af, pf[cg][nt][0], pf[cg][nt][1]);
           }
         }
+        __syncwarp();
       }
-      __syncwarp();
     }
   }
 
-  // ---- this warp's state -> its own (finished) ring, natural channel order
-  __syncwarp();
-  float* my_o = reinterpret_cast<float*>(ring);  // [g][D]
+  // ---- this warp's state -> its slot, natural channel order
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int hh = nt * 4 + tig;
@@ -424,36 +502,36 @@ __device__ void quant_role(const QArgs& a, unsigned char* smem, int unit, int b,
     for (int mc = 0; mc < C::KT; ++mc) {
       const int cg = mc * 16 / G;
       const float zb = __shfl_sync(FULL, vbs, cg * 4 + tig);
-      const float u = pow2i(24 - BITS * (mc % F::TPW));  // undo the code encoding of this tile
+      const float uf = pow2i(24 - BITS * (mc % F::TPW));  // undo the code encoding of this tile
       if (hh < a.g) {
-        float* wo = my_o + hh * D + mc * 16 + gid;
-        wo[0] = (acc[mc][nt][0] + acc[mc][nt][1]) * u + zb;
-        wo[8] = (acc[mc][nt][2] + acc[mc][nt][3]) * u + zb;
+        float* wo = st_o + (warp * C::HEADS + hh) * D + mc * 16 + gid;
+        wo[0] = (acc[mc][nt][0] + acc[mc][nt][1]) * uf + zb;
+        wo[8] = (acc[mc][nt][2] + acc[mc][nt][3]) * uf + zb;
       }
     }
     if (hh < a.g && gid == 0) {
-      wst_ml[(warp * a.g + hh) * 2] = ok ? m_run[nt] : -INFINITY;
-      wst_ml[(warp * a.g + hh) * 2 + 1] = ok ? l : 0.f;
+      st_ml[(warp * C::HEADS + hh) * 2] = ok ? m_run[nt] : -INFINITY;
+      st_ml[(warp * C::HEADS + hh) * 2 + 1] = ok ? l : 0.f;
     }
   }
 }
 
 // -------------------------------------------------------- bf16 residual part
-template <int D, int NT, int RSTRIDE, int WARPB>
-__device__ void residual_role(const QArgs& a, unsigned char* smem, int unit, int b, int h, float* wst_ml,
-                              bool& ok, int bar_off) {
+// This warp's residual stages of unit u (16 rows each, one bulk copy per row,
+// not pipelined; the residual is a few percent of the bytes).  Leaves the
+// warp's state in its slot.
+template <int D, int NT, int RSTRIDE, int HEADS>
+__device__ __noinline__ void residual_seg(const QArgs& a, unsigned char* ring, float* P_s, uint64_t* bar, int& rph, int u,
+                             int64_t first_s, int64_t end_s, int64_t seg_b, bool& ok, float* st_o, float* st_ml) {
   constexpr int KT = D / 16;
   constexpr int ROW_B = D * 2;
+  constexpr unsigned FULL = 0xffffffffu;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int part = gid & 1;
-  unsigned char* ring = smem + warp * WARPB;  // one stage: 16 K rows + 16 V rows
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + bar_off) + warp;
-  float* P_s = reinterpret_cast<float*>(ring + 32 * RSTRIDE);  // [4*NT][16]
-  const int ntiles = (a.R + 15) / 16;
-  const int my_n = ntiles > warp ? (ntiles - warp + kQNW - 1) / kQNW : 0;
-  const __nv_bfloat16* kr = a.kr + static_cast<size_t>(unit) * a.R_cap * D;
-  const __nv_bfloat16* vr = a.vr + static_cast<size_t>(unit) * a.R_cap * D;
+  const int b = u / a.Hkv, h = u - b * a.Hkv;
+  const __nv_bfloat16* kr = a.kr + static_cast<size_t>(u) * a.R_cap * D;
+  const __nv_bfloat16* vr = a.vr + static_cast<size_t>(u) * a.R_cap * D;
 
   // query B fragments (bf16, natural channels): high columns = q, low = 0
   uint32_t qb[KT][NT][2];
@@ -477,21 +555,23 @@ __device__ void residual_role(const QArgs& a, unsigned char* smem, int unit, int
 #pragma unroll
     for (int mc = 0; mc < KT; ++mc) acc[mc][nt][0] = acc[mc][nt][1] = acc[mc][nt][2] = acc[mc][nt][3] = 0.f;
   }
-  if (lane == 0) mbar_init(bar, 1);
-  fence_mbar_init();
-  __syncwarp();
-  for (int i = 0; i < my_n; ++i) {
-    const int t0 = (warp + i * kQNW) * 16;
+  for (int64_t s = first_s; s < end_s && ok; s += kQNW) {
+    const int t0 = static_cast<int>(s - seg_b) * kResRows;
     const int r = lane & 15;
     const bool valid = t0 + r < a.R;
+    fence_proxy_async_smem();
+    __syncwarp();
     if (lane == 0) mbar_arrive_expect_tx(bar, 32u * ROW_B);
     __syncwarp();
     const __nv_bfloat16* src = (lane < 16 ? kr : vr) + static_cast<size_t>(valid ? t0 + r : 0) * D;
     bulk_g2s(ring + lane * RSTRIDE, src, ROW_B, bar);
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar, i & 1, a.flags))) {  // warp-uniform
+    if (!__all_sync(FULL, mbar_wait_bounded(bar, rph & 1, a.flags))) {  // warp-uniform
       ok = false;
+      mbar_wait_bounded(bar, rph & 1, nullptr, 100000000ull);
+      ++rph;
       break;
     }
+    ++rph;
     const unsigned char* Ks = ring;
     const unsigned char* Vs = ring + 16 * RSTRIDE;
     const int mi = lane >> 3, ri = lane & 7;
@@ -509,9 +589,19 @@ __device__ void residual_role(const QArgs& a, unsigned char* smem, int unit, int
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const bool v0 = t0 + gid < a.R, v1 = t0 + gid + 8 < a.R;
-      float x[4] = {v0 ? (sc[nt][0] + sc[nt][1]) * a.scale_log2 : -INFINITY,
-                    v1 ? (sc[nt][2] + sc[nt][3]) * a.scale_log2 : -INFINITY, -INFINITY, -INFINITY};
-      const float alpha = softmax_step(x, m_run[nt], l_run[nt], 4);
+      float x[2] = {v0 ? (sc[nt][0] + sc[nt][1]) * a.scale_log2 : -INFINITY,
+                    v1 ? (sc[nt][2] + sc[nt][3]) * a.scale_log2 : -INFINITY};
+      float t = fmaxf(x[0], x[1]);
+      t = warp_max_xor(t, 4);
+      t = warp_max_xor(t, 8);
+      t = warp_max_xor(t, 16);
+      const float m_new = fmaxf(m_run[nt], t);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = ex2(m_run[nt] - m_use);
+      x[0] = ex2(x[0] - m_use);
+      x[1] = ex2(x[1] - m_use);
+      l_run[nt] = l_run[nt] * alpha + x[0] + x[1];
+      m_run[nt] = m_new;
 #pragma unroll
       for (int mc = 0; mc < KT; ++mc) {
         acc[mc][nt][0] *= alpha;
@@ -546,52 +636,237 @@ __device__ void residual_role(const QArgs& a, unsigned char* smem, int unit, int
     }
     __syncwarp();
   }
-  __syncwarp();
-  float* my_o = reinterpret_cast<float*>(ring);  // [g][D]
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int hh = nt * 4 + tig;
     float l = l_run[nt];
-    l += __shfl_xor_sync(0xffffffffu, l, 4);
-    l += __shfl_xor_sync(0xffffffffu, l, 8);
-    l += __shfl_xor_sync(0xffffffffu, l, 16);
+    l += __shfl_xor_sync(FULL, l, 4);
+    l += __shfl_xor_sync(FULL, l, 8);
+    l += __shfl_xor_sync(FULL, l, 16);
     if (hh < a.g) {
 #pragma unroll
       for (int mc = 0; mc < KT; ++mc) {
-        float* wo = my_o + hh * D + mc * 16 + gid;
+        float* wo = st_o + (warp * HEADS + hh) * D + mc * 16 + gid;
         wo[0] = acc[mc][nt][0] + acc[mc][nt][1];
         wo[8] = acc[mc][nt][2] + acc[mc][nt][3];
       }
       if (gid == 0) {
-        wst_ml[(warp * a.g + hh) * 2] = ok ? m_run[nt] : -INFINITY;
-        wst_ml[(warp * a.g + hh) * 2 + 1] = ok ? l : 0.f;
+        st_ml[(warp * HEADS + hh) * 2] = ok ? m_run[nt] : -INFINITY;
+        st_ml[(warp * HEADS + hh) * 2 + 1] = ok ? l : 0.f;
       }
     }
   }
 }
 
+// Number of block partials of unit u and the slot of partial p of it.  A
+// unit's partials are those of its quantised segment (blocks block_of(begin)
+// .. block_of(end - 1)) followed by those of its residual segment.  Every
+// block after the first one of a segment starts inside it, so its local
+// segment index is 0; only the first block's index needs computing.
+struct UnitPartials {
+  int seg[2];
+  int kb[2];
+  int cnt[2];
+  int loc0[2];
+  __device__ void init(const Partition& P, int u) {
+    int n = 0;
+    if (P.sq > 0) seg[n++] = u;
+    if (P.sr > 0) seg[n++] = P.U + u;
+    for (int i = 0; i < 2; ++i) {
+      if (i < n) {
+        kb[i] = P.block_of(P.seg_begin(seg[i]));
+        cnt[i] = P.block_of(P.seg_end(seg[i]) - 1) - kb[i] + 1;
+        loc0[i] = seg[i] - P.seg_of(P.first(kb[i]));
+      } else {
+        seg[i] = 0, kb[i] = 0, cnt[i] = 0, loc0[i] = 0;
+      }
+    }
+  }
+  __device__ int total() const { return cnt[0] + cnt[1]; }
+  __device__ int64_t slot(int maxs, int p) const {
+    const int i = p < cnt[0] ? 0 : 1;
+    const int pl = i ? p - cnt[0] : p;
+    return static_cast<int64_t>(kb[i] + pl) * maxs + (pl == 0 ? loc0[i] : 0);
+  }
+};
+
+// Block-wide: merges the kQNW warp states of segment `seg` (local index j of
+// block k) into the block's partial; the block that completes unit u's last
+// partial merges all of them into out (one online pass over chunks of
+// kMergeChunk partials: their (m, l) pairs are staged in shared memory, the
+// running maximum rescales the running sums).
+template <int D, int HEADS>
+__device__ __noinline__ void merge_segment(const QArgs& a, int k, int j, int seg, const float* st_o,
+                                           const float* st_ml, float* mw, int64_t* slots_s, uint32_t* tick_s) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int g = a.g;
+  const Partition& P = a.P;
+  float* wts = mw;                       // [kQNW][HEADS]  (block merge)  /  [kMergeChunk][HEADS]
+  float* ML = mw + kMergeChunk * HEADS;  // [HEADS][2]
+  for (int r = tid; r < g; r += nthr) {
+    float M = -INFINITY;
+    for (int w = 0; w < kQNW; ++w) M = fmaxf(M, st_ml[(w * HEADS + r) * 2]);
+    float L = 0.f;
+    for (int w = 0; w < kQNW; ++w) {
+      const float mw_ = st_ml[(w * HEADS + r) * 2];
+      const float sc = (mw_ == -INFINITY) ? 0.f : ex2(mw_ - M);
+      wts[w * HEADS + r] = sc;
+      L += sc * st_ml[(w * HEADS + r) * 2 + 1];
+    }
+    ML[2 * r] = M;
+    ML[2 * r + 1] = L;
+  }
+  __syncthreads();
+  const int64_t slot = static_cast<int64_t>(k) * a.MAXS + j;
+  float* po = a.part_o + slot * g * D;
+  float* pml = a.part_ml + slot * g * 2;
+  for (int e = tid; e < g * D; e += nthr) {
+    const int r = e / D, d = e - r * D;
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kQNW; ++w) acc += wts[w * HEADS + r] * st_o[(w * HEADS + r) * D + d];
+    po[e] = acc;
+  }
+  for (int r = tid; r < g; r += nthr) {
+    pml[2 * r] = ML[2 * r];
+    pml[2 * r + 1] = ML[2 * r + 1];
+  }
+  __threadfence();
+  __syncthreads();
+  const int u = seg < P.U ? seg : seg - P.U;
+  UnitPartials up;
+  up.init(P, u);
+  if (tid == 0) *tick_s = atomicAdd(&a.tickets[u], 1u);
+  __syncthreads();
+  const int np = up.total();
+  if (*tick_s == static_cast<uint32_t>(np - 1)) {
+    __threadfence();
+    constexpr int EPT = (8 * D + 127) / 128;  // elements per thread for g <= 8, 128 threads
+    float acc[EPT];
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) acc[i] = 0.f;
+    float* Mrun = ML;  // [HEADS][2]: running max, running denominator
+    for (int r = tid; r < g; r += nthr) {
+      Mrun[2 * r] = -INFINITY;
+      Mrun[2 * r + 1] = 0.f;
+    }
+    for (int p0 = 0; p0 < np; p0 += kMergeChunk) {
+      const int nc = np - p0 < kMergeChunk ? np - p0 : kMergeChunk;
+      __syncthreads();
+      for (int p = tid; p < nc; p += nthr) slots_s[p] = up.slot(a.MAXS, p0 + p);
+      __syncthreads();
+      // partial maxima of the chunk into wts (as m), then the new running max per row
+      for (int idx = tid; idx < nc * g; idx += nthr) {
+        const int p = idx / g, r = idx - p * g;
+        wts[p * HEADS + r] = __ldcg(a.part_ml + slots_s[p] * g * 2 + 2 * r);
+      }
+      __syncthreads();
+      __shared__ float resc[8];  // factor applied to the running sums of each row
+      for (int r = tid; r < g; r += nthr) {
+        float M = Mrun[2 * r];
+        for (int p = 0; p < nc; ++p) M = fmaxf(M, wts[p * HEADS + r]);
+        resc[r] = Mrun[2 * r] == -INFINITY ? 0.f : ex2(Mrun[2 * r] - M);
+        Mrun[2 * r] = M;
+      }
+      __syncthreads();
+      // weights of the chunk's partials against the new running max; denominators
+      for (int idx = tid; idx < nc * g; idx += nthr) {
+        const int p = idx / g, r = idx - p * g;
+        const float mp = wts[p * HEADS + r];
+        wts[p * HEADS + r] = mp == -INFINITY ? 0.f : ex2(mp - Mrun[2 * r]);
+      }
+      __syncthreads();
+      for (int r = tid; r < g; r += nthr) {
+        float L = Mrun[2 * r + 1] * resc[r];
+        for (int p = 0; p < nc; ++p) L += wts[p * HEADS + r] * __ldcg(a.part_ml + slots_s[p] * g * 2 + 2 * r + 1);
+        Mrun[2 * r + 1] = L;
+      }
+#pragma unroll
+      for (int i = 0; i < EPT; ++i) {
+        const int e = tid + i * nthr;
+        if (e < g * D) {
+          const int r = e / D;
+          float s0 = acc[i] * resc[r], s1 = 0.f, s2 = 0.f, s3 = 0.f;
+          int p = 0;
+          for (; p + 4 <= nc; p += 4) {
+            const float v0 = __ldcg(a.part_o + slots_s[p] * g * D + e);
+            const float v1 = __ldcg(a.part_o + slots_s[p + 1] * g * D + e);
+            const float v2 = __ldcg(a.part_o + slots_s[p + 2] * g * D + e);
+            const float v3 = __ldcg(a.part_o + slots_s[p + 3] * g * D + e);
+            s0 += wts[p * HEADS + r] * v0;
+            s1 += wts[(p + 1) * HEADS + r] * v1;
+            s2 += wts[(p + 2) * HEADS + r] * v2;
+            s3 += wts[(p + 3) * HEADS + r] * v3;
+          }
+          for (; p < nc; ++p) s0 += wts[p * HEADS + r] * __ldcg(a.part_o + slots_s[p] * g * D + e);
+          acc[i] = (s0 + s1) + (s2 + s3);
+        }
+      }
+    }
+    __syncthreads();
+    const int b = u / a.Hkv, h = u - b * a.Hkv;
+    float* o = a.out + (static_cast<size_t>(b) * a.Hq + h * g) * D;
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+      const int e = tid + i * nthr;
+      if (e < g * D) {
+        const float L = Mrun[2 * (e / D) + 1];
+        o[e] = L > 0.f ? acc[i] / L : 0.f;
+      }
+    }
+    if (tid == 0) a.tickets[u] = 0;
+  }
+  __syncthreads();
+}
 
 template <int BITS, int G, int D, int NT>
 __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kernel(QArgs a) {
   using C = QCfg<BITS, G, D, NT>;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ float wst_ml[kQNW * 8 * 2];
-  __shared__ float smem_w[kQNW * 8 + 2 * 8];
-  const int unit = blockIdx.y;
-  const int b = unit / a.Hkv, h = unit - b * a.Hkv;
-  const int chunk = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.x;
+  const Partition& P = a.P;
+  const int64_t B0 = P.first(k), B1 = P.first(k + 1);
+  if (B0 >= B1) return;  // the host sizes the grid so that this never happens
+  const int seg0 = P.seg_of(B0), seg1 = P.seg_of(B1 - 1);
+  unsigned char* ring = smem + warp * C::WARP_B;
+  float* P_res = reinterpret_cast<float*>(ring + C::RING);  // residual scores share the p buffer
+  float* st_o = reinterpret_cast<float*>(smem + C::STATE_OFF);
+  float* st_ml = reinterpret_cast<float*>(smem + C::ML_OFF);
+  float* mw = reinterpret_cast<float*>(smem + C::MW_OFF);
+  int64_t* slots_s = reinterpret_cast<int64_t*>(smem + C::SLOT_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + warp * (C::NST + 1);
+  uint32_t* tick_s = reinterpret_cast<uint32_t*>(smem + C::TICK_OFF);
+
+  const int64_t B1q = B1 < P.QZ ? B1 : P.QZ;
+  const int my_nq = B1q > B0 + warp ? static_cast<int>((B1q - B0 - warp + kQNW - 1) / kQNW) : 0;
+  if (lane == 0)
+    for (int s = 0; s <= C::NST; ++s) mbar_init(&bars[s], 1);
+  fence_mbar_init();
+  __syncwarp();
   bool ok = true;
-  // chunk numbering: the residual block (if any) first, then quantised chunks
-  if (a.res_first && chunk == 0)
-    residual_role<D, NT, C::RS, C::WARP_B>(a, smem, unit, b, h, wst_ml, ok, C::BAR_OFF);
-  else
-    quant_role<BITS, G, D, NT>(a, smem, unit, b, h, chunk - a.res_first, wst_ml, ok);
-  __syncthreads();
-  const int hq0 = b * a.Hq + h * a.g;
-  splitk_finish<D>(
-      reinterpret_cast<const float*>(smem), C::WARP_B / 4, wst_ml, kQNW, a.g, a.g, a.S, chunk, unit, a.o,
-      [&](int r) { return static_cast<size_t>(hq0 + r) * D; }, [&](int r) { return static_cast<size_t>(hq0 + r); },
-      smem_w);
+  int iq = 0, issued = 0, rph = 0;
+  IssuePtr ip;
+  if (my_nq > 0) ip.start(P, B0 + warp);
+  while (issued < my_nq && issued < C::NST - 1) {
+    issue_stage<C>(a, ring, bars, lane, issued, ip);
+    ip.advance(P);
+    ++issued;
+  }
+  for (int seg = seg0; seg <= seg1; ++seg) {
+    if (seg < P.U) {
+      quant_seg<BITS, G, D, NT>(a, ring, bars, seg, B0, my_nq, iq, issued, ip, ok, st_o, st_ml);
+    } else {
+      const int64_t sb = P.seg_begin(seg), se = P.seg_end(seg);
+      const int64_t lo = sb > B0 ? sb : B0;
+      const int64_t off = lo - B0;
+      const int64_t i0 = off <= warp ? 0 : (off - warp + kQNW - 1) / kQNW;
+      residual_seg<D, NT, C::RS, C::HEADS>(a, ring, P_res, &bars[C::NST], rph, seg - P.U,
+                                           B0 + warp + i0 * kQNW, se < B1 ? se : B1, sb, ok, st_o, st_ml);
+    }
+    __syncthreads();
+    merge_segment<D, C::HEADS>(a, k, seg - seg0, seg, st_o, st_ml, mw, slots_s, tick_s);
+  }
 }
 
 // vc_debug_dequant: one warp per (group, unit).  The codes are extracted with
@@ -599,24 +874,30 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
 // uses (Frag), then dequantised with one fp32 FMA each and stored at their
 // natural positions.
 template <int BITS, int G, int D>
-__global__ void __launch_bounds__(32) debug_dequant_kernel(QArgs a, float* ko, float* vo) {
+__global__ void __launch_bounds__(32) debug_dequant_kernel(const uint8_t* recs, int64_t ng, float* ko, float* vo) {
   using F = Frag<BITS>;
-  constexpr int RB = D * BITS / 8, CPG = D / G, KT = D / 16, NW = 2 * KT / F::TPW;
+  using C = QCfg<BITS, G, D, 1>;
+  constexpr int CPG = D / G, KT = D / 16, NW = 2 * KT / F::TPW;
   const int lane = threadIdx.x, gid = lane >> 2, tig = lane & 3;
   const int unit = blockIdx.y;
   const int64_t j = blockIdx.x;
-  const int64_t n_groups = a.L_q / G;
-  const uint32_t* kc = reinterpret_cast<const uint32_t*>(a.kc + (static_cast<size_t>(unit) * a.L_q + j * G) * RB);
-  const uint32_t* vcw = reinterpret_cast<const uint32_t*>(a.vc + (static_cast<size_t>(unit) * a.L_q + j * G) * RB);
-  const __half* sk = a.sk + (static_cast<size_t>(unit) * n_groups + j) * D;
-  const __half* zk = a.zk + (static_cast<size_t>(unit) * n_groups + j) * D;
-  const __half* sv = a.sv + (static_cast<size_t>(unit) * a.L_q + j * G) * CPG;  // pair-interleaved
-  const __half* zv = a.zv + (static_cast<size_t>(unit) * a.L_q + j * G) * CPG;
-  float* kou = ko + (static_cast<size_t>(unit) * a.L_q + j * G) * D;
-  float* vou = vo + (static_cast<size_t>(unit) * a.L_q + j * G) * D;
+  const uint8_t* rs = recs + (static_cast<size_t>(unit) * ng + j) * C::REC;
+  const uint32_t* kc = reinterpret_cast<const uint32_t*>(rs);
+  const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
+  const __half* sk = reinterpret_cast<const __half*>(rs + C::OFF_SK);
+  const __half* zk = reinterpret_cast<const __half*>(rs + C::OFF_ZK);
+  const __half* sv = reinterpret_cast<const __half*>(rs + C::OFF_SV);  // pair-interleaved
+  const __half* zv = reinterpret_cast<const __half*>(rs + C::OFF_ZV);
+  float* kou = ko + (static_cast<size_t>(unit) * ng + j) * G * D;
+  float* vou = vo + (static_cast<size_t>(unit) * ng + j) * G * D;
   auto code = [](uint32_t reg, int half, float undo) {
     const float2 f = unpack_h2(reg);
     return (half ? f.y : f.x) * undo;
+  };
+  // fp16 slot of channel c in the key-parameter row: word tig*2KT + 2kt + h
+  auto kslot = [](int c) {
+    const int kt = c >> 4, h = (c >> 3) & 1, t = (c >> 1) & 3, e = c & 1;
+    return 2 * (t * 2 * KT + 2 * kt + h) + e;
   };
   for (int tt = 0; tt < G / 16; ++tt) {
     for (int jw = 0; jw < NW / 2; ++jw) {
@@ -631,7 +912,8 @@ __global__ void __launch_bounds__(32) debug_dequant_kernel(QArgs a, float* ko, f
           for (int e = 0; e < 2; ++e) {
             const int t = tt * 16 + gid + ((r & 1) ? 8 : 0);
             const int c = kt * 16 + 2 * tig + ((r & 2) ? 8 : 0) + e;
-            kou[t * D + c] = __fmaf_rn(code(regs[r], e, undo), __half2float(sk[c]), __half2float(zk[c]));
+            kou[t * D + c] =
+                __fmaf_rn(code(regs[r], e, undo), __half2float(sk[kslot(c)]), __half2float(zk[kslot(c)]));
           }
       }
     }
@@ -657,7 +939,8 @@ __global__ void __launch_bounds__(32) debug_dequant_kernel(QArgs a, float* ko, f
 }
 
 struct QPlan {
-  int S, Sq, GPC, res;
+  Partition P;
+  int MAXS;
   size_t off_tick, off_ml, off_o, total;
 };
 
@@ -681,48 +964,62 @@ int quant_occupancy() {
   return cache[dev];
 }
 
-QPlan make_plan(const vc_attn_shape& sh, const vc_quant_cache& c, int occ) {
+// The stage axis of one call and its cut into at most `target_blocks` blocks.
+QPlan make_plan(const vc_attn_shape& sh, const vc_quant_cache& c, int ng_per_stage, int rec_bytes,
+                int64_t target_blocks) {
   QPlan p{};
-  const int units = sh.B * sh.Hkv;
-  const int64_t n_groups = c.L_q / c.group;
-  p.res = c.R > 0 ? 1 : 0;
-  if (n_groups > 0) {
-    const int64_t slots = static_cast<int64_t>(occ) * sm_count();
-    int64_t sq = (slots - static_cast<int64_t>(units) * p.res) / units;
-    if (sq < 1) sq = 1;
-    int64_t gpc = (n_groups + sq - 1) / sq;
-    if (gpc < 4) gpc = 4;
-    p.GPC = static_cast<int>(gpc);
-    p.Sq = static_cast<int>((n_groups + gpc - 1) / gpc);
+  Partition& P = p.P;
+  P.U = sh.B * sh.Hkv;
+  P.ng = c.L_q / c.group;
+  P.sq = static_cast<int>((P.ng + ng_per_stage - 1) / ng_per_stage);
+  P.sr = (c.R + kResRows - 1) / kResRows;
+  P.QZ = static_cast<int64_t>(P.U) * P.sq;
+  P.S_tot = P.QZ + static_cast<int64_t>(P.U) * P.sr;
+  P.cq = static_cast<int64_t>(ng_per_stage) * rec_bytes;
+  P.cr = P.sr > 0 ? static_cast<int64_t>(kResRows) * 4 * sh.D * kResCostWeight : 1;
+  P.C = P.QZ * P.cq + (P.S_tot - P.QZ) * P.cr;
+  const int64_t mx = P.sq > 0 && P.sr > 0 ? (P.cq > P.cr ? P.cq : P.cr) : (P.sq > 0 ? P.cq : P.cr);
+  int64_t n = target_blocks;
+  if (n > P.S_tot) n = P.S_tot;
+  if (n > P.C / mx) n = P.C / mx;
+  if (n < 1) n = 1;
+  P.nblk = static_cast<int>(n);
+  int maxs = 1;
+  for (int k = 0; k < P.nblk; ++k) {
+    const int64_t b0 = P.first(k), b1 = P.first(k + 1);
+    const int segs = P.seg_of(b1 - 1) - P.seg_of(b0) + 1;
+    if (segs > maxs) maxs = segs;
   }
-  p.S = p.Sq + p.res;
+  p.MAXS = maxs;
   const int g = sh.Hq / sh.Hkv;
+  const size_t slots = static_cast<size_t>(P.nblk) * maxs;
   p.off_tick = sizeof(WsHeader);
-  p.off_ml = align_up(p.off_tick + static_cast<size_t>(units) * 4, 256);
-  p.off_o = align_up(p.off_ml + static_cast<size_t>(units) * p.S * g * 2 * 4, 256);
-  p.total = align_up(p.off_o + static_cast<size_t>(units) * p.S * g * sh.D * 4, 256);
+  p.off_ml = align_up(p.off_tick + static_cast<size_t>(P.U) * 4, 256);
+  p.off_o = align_up(p.off_ml + slots * g * 2 * 4, 256);
+  p.total = align_up(p.off_o + slots * g * sh.D * 4, 256);
   return p;
 }
 
 template <int BITS, int G, int D, int NT>
-QPlan plan_t(const vc_attn_shape& sh, const vc_quant_cache& c) {
-  return make_plan(sh, c, quant_occupancy<BITS, G, D, NT>());
+QPlan plan_t(const vc_attn_shape& sh, const vc_quant_cache& c, int64_t target_blocks) {
+  using C = QCfg<BITS, G, D, NT>;
+  if (target_blocks <= 0) target_blocks = static_cast<int64_t>(quant_occupancy<BITS, G, D, NT>()) * sm_count();
+  return make_plan(sh, c, C::NG, C::REC, target_blocks);
 }
 
 template <int BITS, int G, int D, int NT>
-void launch_t(const QArgs& a, const QPlan& p, const vc_attn_shape& sh, cudaStream_t s) {
+void launch_t(const QArgs& a, const QPlan& p, cudaStream_t s) {
   using C = QCfg<BITS, G, D, NT>;
   quant_occupancy<BITS, G, D, NT>();  // sets the shared-memory attribute once per device
-  dim3 grid(p.S, sh.B * sh.Hkv);
-  draft_quant_kernel<BITS, G, D, NT><<<grid, kQNW * 32, C::SMEM_B, s>>>(a);
+  draft_quant_kernel<BITS, G, D, NT><<<p.P.nblk, kQNW * 32, C::SMEM_B, s>>>(a);
 }
 
 template <int BITS, int G, int D>
-void debug_t(const QArgs& a, const vc_attn_shape& sh, float* ko, float* vo, cudaStream_t s) {
-  const int64_t n_groups = a.L_q / G;
+void debug_t(const vc_quant_cache& c, const vc_attn_shape& sh, float* ko, float* vo, cudaStream_t s) {
+  const int64_t n_groups = c.L_q / G;
   if (n_groups == 0) return;
   dim3 grid(static_cast<unsigned>(n_groups), sh.B * sh.Hkv);
-  debug_dequant_kernel<BITS, G, D><<<grid, 32, 0, s>>>(a, ko, vo);
+  debug_dequant_kernel<BITS, G, D><<<grid, 32, 0, s>>>(static_cast<const uint8_t*>(c.records), n_groups, ko, vo);
 }
 
 // Dispatch over the compiled instances: bits {2,4} x group {32,64} x D
@@ -754,13 +1051,11 @@ vc_status check_quant(const vc_attn_shape* sh, const vc_quant_cache* c, const ch
   VC_REQUIRE(c->L_q / c->group < (int64_t(1) << 30), "%s: L_q too large", who);
   VC_REQUIRE(c->R >= 0 && c->R <= c->R_cap, "%s: need 0 <= R <= R_cap", who);
   VC_REQUIRE(c->L_q + c->R >= 1, "%s: the cache holds no token", who);
-  VC_REQUIRE(static_cast<int64_t>(sh->B) * sh->Hkv <= 65535, "%s: too many (request, head) pairs", who);
+  VC_REQUIRE(static_cast<int64_t>(sh->B) * sh->Hkv <= (int64_t(1) << 24), "%s: too many (request, head) pairs",
+             who);
   if (c->L_q > 0) {
-    VC_REQUIRE(c->k_codes && c->v_codes && c->k_scale && c->k_zero && c->v_scale && c->v_zero,
-               "%s: null quantised-cache pointer", who);
-    VC_REQUIRE(aligned16(c->k_codes) && aligned16(c->v_codes) && aligned16(c->k_scale) && aligned16(c->k_zero) &&
-                   aligned16(c->v_scale) && aligned16(c->v_zero),
-               "%s: quantised-cache arrays must be 16-byte aligned", who);
+    VC_REQUIRE(c->records, "%s: null group-record pointer", who);
+    VC_REQUIRE(aligned16(c->records), "%s: group records must be 16-byte aligned", who);
   }
   if (c->R > 0) {
     VC_REQUIRE(c->k_res && c->v_res, "%s: null residual pointer", who);
@@ -771,16 +1066,10 @@ vc_status check_quant(const vc_attn_shape* sh, const vc_quant_cache* c, const ch
 
 QArgs make_args(const vc_attn_shape& sh, const vc_quant_cache& c, const void* q) {
   QArgs a{};
-  a.kc = static_cast<const uint8_t*>(c.k_codes);
-  a.vc = static_cast<const uint8_t*>(c.v_codes);
-  a.sk = static_cast<const __half*>(c.k_scale);
-  a.zk = static_cast<const __half*>(c.k_zero);
-  a.sv = static_cast<const __half*>(c.v_scale);
-  a.zv = static_cast<const __half*>(c.v_zero);
+  a.rec = static_cast<const uint8_t*>(c.records);
   a.kr = static_cast<const __nv_bfloat16*>(c.k_res);
   a.vr = static_cast<const __nv_bfloat16*>(c.v_res);
   a.q = static_cast<const __nv_bfloat16*>(q);
-  a.L_q = c.L_q;
   a.R = c.R;
   a.R_cap = c.R_cap;
   a.Hq = sh.Hq;
@@ -791,10 +1080,29 @@ QArgs make_args(const vc_attn_shape& sh, const vc_quant_cache& c, const void* q)
   return a;
 }
 
-bool quant_plan(const vc_attn_shape& sh, const vc_quant_cache& c, QPlan* out) {
+bool quant_plan(const vc_attn_shape& sh, const vc_quant_cache& c, QPlan* out, int64_t target_blocks = 0) {
   const int nt = (sh.Hq / sh.Hkv) <= 4 ? 1 : 2;
   return dispatch(c.bits, c.group, sh.D, nt, [&](auto BI, auto GR, auto DD, auto NN) {
-    *out = plan_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value, decltype(NN)::value>(sh, c);
+    *out = plan_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value, decltype(NN)::value>(
+        sh, c, target_blocks);
+  });
+}
+
+void bind_scratch(QArgs& a, const QPlan& p, void* scratch, float* out) {
+  char* w = static_cast<char*>(scratch);
+  a.P = p.P;
+  a.MAXS = p.MAXS;
+  a.flags = reinterpret_cast<uint32_t*>(w);
+  a.tickets = reinterpret_cast<uint32_t*>(w + p.off_tick);
+  a.part_ml = reinterpret_cast<float*>(w + p.off_ml);
+  a.part_o = reinterpret_cast<float*>(w + p.off_o);
+  a.out = out;
+}
+
+void launch_quant(const vc_attn_shape& sh, const vc_quant_cache& c, const QArgs& a, const QPlan& p, cudaStream_t s) {
+  const int nt = a.g <= 4 ? 1 : 2;
+  dispatch(c.bits, c.group, sh.D, nt, [&](auto BI, auto GR, auto DD, auto NN) {
+    launch_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value, decltype(NN)::value>(a, p, s);
   });
 }
 
@@ -822,23 +1130,8 @@ vc_status vc_draft_attn_quant(const vc_attn_shape* shape, const vc_quant_cache* 
     return vc::set_error(VC_ERR_UNSUPPORTED, "vc_draft_attn_quant: no kernel for this configuration");
   VC_REQUIRE(ws_bytes >= p.total, "vc_draft_attn_quant: workspace too small (%zu < %zu)", ws_bytes, p.total);
   vc::QArgs a = vc::make_args(*shape, *cache, q);
-  char* w = static_cast<char*>(ws);
-  a.S = p.S;
-  a.Sq = p.Sq;
-  a.GPC = p.GPC;
-  a.res_first = p.res;
-  a.flags = reinterpret_cast<uint32_t*>(w);
-  a.o.out = out;
-  a.o.lse = nullptr;
-  a.o.tickets = reinterpret_cast<uint32_t*>(w + p.off_tick);
-  a.o.part_ml = reinterpret_cast<float*>(w + p.off_ml);
-  a.o.part_o = reinterpret_cast<float*>(w + p.off_o);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int nt = a.g <= 4 ? 1 : 2;
-  vc::dispatch(cache->bits, cache->group, shape->D, nt, [&](auto BI, auto GR, auto DD, auto NN) {
-    vc::launch_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value, decltype(NN)::value>(a, p, *shape,
-                                                                                                     s);
-  });
+  vc::bind_scratch(a, p, ws, out);
+  vc::launch_quant(*shape, *cache, a, p, static_cast<cudaStream_t>(stream));
   return vc::launch_status("vc_draft_attn_quant");
 }
 
@@ -848,12 +1141,34 @@ vc_status vc_debug_dequant(const vc_attn_shape* shape, const vc_quant_cache* cac
   if (st != VC_OK) return st;
   VC_REQUIRE(k_out && v_out, "vc_debug_dequant: null output");
   VC_REQUIRE(cache->L_q / cache->group <= 2147483647, "vc_debug_dequant: too many groups");
-  vc::QArgs a = vc::make_args(*shape, *cache, nullptr);
+  VC_REQUIRE(static_cast<int64_t>(shape->B) * shape->Hkv <= 65535, "vc_debug_dequant: too many units");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   vc::dispatch(cache->bits, cache->group, shape->D, 1, [&](auto BI, auto GR, auto DD, auto) {
-    vc::debug_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value>(a, *shape, k_out, v_out, s);
+    vc::debug_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value>(*cache, *shape, k_out, v_out, s);
   });
   return vc::launch_status("vc_debug_dequant");
+}
+
+vc_status vc_debug_quant_partition(const vc_attn_shape* shape, const vc_quant_cache* cache, int target_blocks,
+                                   int64_t* first_stage, int max_blocks, int* n_blocks, int* max_segments,
+                                   int64_t* n_stages, int64_t* n_quant_stages) {
+  vc_status st = vc::check_quant(shape, cache, "vc_debug_quant_partition");
+  if (st != VC_OK) return st;
+  VC_REQUIRE(target_blocks >= 1, "vc_debug_quant_partition: target_blocks must be >= 1");
+  VC_REQUIRE(n_blocks && max_segments && n_stages && n_quant_stages, "vc_debug_quant_partition: null output");
+  vc::QPlan p{};
+  if (!vc::quant_plan(*shape, *cache, &p, target_blocks))
+    return vc::set_error(VC_ERR_UNSUPPORTED, "vc_debug_quant_partition: no kernel for this configuration");
+  *n_blocks = p.P.nblk;
+  *max_segments = p.MAXS;
+  *n_stages = p.P.S_tot;
+  *n_quant_stages = p.P.QZ;
+  if (first_stage) {
+    VC_REQUIRE(max_blocks >= p.P.nblk + 1, "vc_debug_quant_partition: first_stage needs %d entries",
+               p.P.nblk + 1);
+    for (int k = 0; k <= p.P.nblk; ++k) first_stage[k] = p.P.first(k);
+  }
+  return VC_OK;
 }
 
 }  // extern "C"
@@ -930,22 +1245,8 @@ vc_status vc_draft_attn_quant_noalloc(const vc_attn_shape* shape, const vc_quant
     return vc::set_error(VC_ERR_CUDA, "vc_draft_attn_quant_noalloc: clearing the scratch failed: %s",
                          cudaGetErrorString(cudaGetLastError()));
   vc::QArgs a = vc::make_args(*shape, *cache, q);
-  char* w = static_cast<char*>(scratch);
-  a.S = p.S;
-  a.Sq = p.Sq;
-  a.GPC = p.GPC;
-  a.res_first = p.res;
-  a.flags = reinterpret_cast<uint32_t*>(w);
-  a.o.out = out;
-  a.o.lse = nullptr;
-  a.o.tickets = reinterpret_cast<uint32_t*>(w + p.off_tick);
-  a.o.part_ml = reinterpret_cast<float*>(w + p.off_ml);
-  a.o.part_o = reinterpret_cast<float*>(w + p.off_o);
-  const int nt = a.g <= 4 ? 1 : 2;
-  vc::dispatch(cache->bits, cache->group, shape->D, nt, [&](auto BI, auto GR, auto DD, auto NN) {
-    vc::launch_t<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value, decltype(NN)::value>(a, p, *shape,
-                                                                                                     s);
-  });
+  vc::bind_scratch(a, p, scratch, out);
+  vc::launch_quant(*shape, *cache, a, p, s);
   return vc::launch_status("vc_draft_attn_quant_noalloc");
 }
 

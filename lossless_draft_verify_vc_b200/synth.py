@@ -103,27 +103,24 @@ def planted_logits(B: int, K: int, V: int, draft: torch.Tensor, accept_lens, see
 def random_quant_cache(B: int, Hkv: int, L_q: int, R_cap: int, D: int, bits: int, group: int,
                        seed: int, device="cpu") -> dict:
     """A quantised cache drawn directly in compressed form for throughput runs:
-    uniform random packed codes, scales ~U(0.05, 1.5), zeros ~U(-3, -0.5)
-    (magnitudes of 2/4-bit groups of N(0, 1) data), bf16 residual ~N(0, 1).
-    Shapes match the library's quantised-cache descriptor (codes per group
-    block, value scales/zeros per token pair)."""
+    group records (the library's descriptor layout: two code blocks of
+    group * D * bits / 8 uniform random bytes, then four parameter rows of D
+    fp16 each -- key scales, key zeros, value scales, value zeros), scales
+    ~U(0.05, 1.5), zeros ~U(-3, -0.5) (magnitudes of 2/4-bit groups of N(0, 1)
+    data), bf16 residual ~N(0, 1)."""
     g = _gen(seed, device)
-    blk = group * D * bits // 8
-    f16 = torch.float16
+    ng = L_q // group
+    cb = group * D * bits // 8
 
     def u(shape, lo, hi):
-        return (torch.rand(shape, generator=g, device=device) * (hi - lo) + lo).to(f16)
+        return (torch.rand(shape, generator=g, device=device) * (hi - lo) + lo).to(torch.float16)
 
+    codes = torch.randint(0, 256, (B, Hkv, ng, 2 * cb), generator=g, device=device, dtype=torch.int32)
+    params = torch.cat([u((B, Hkv, ng, D), 0.05, 1.5), u((B, Hkv, ng, D), -3.0, -0.5),
+                        u((B, Hkv, ng, D), 0.05, 1.5), u((B, Hkv, ng, D), -3.0, -0.5)], dim=-1)
+    records = torch.cat([codes.to(torch.uint8), params.view(torch.uint8)], dim=-1).contiguous()
     return dict(
-        bits=bits, group=group, L_q=L_q, R=R_cap, R_cap=R_cap,
-        k_codes=torch.randint(0, 256, (B, Hkv, L_q // group, blk), generator=g, device=device,
-                              dtype=torch.int32).to(torch.uint8),
-        v_codes=torch.randint(0, 256, (B, Hkv, L_q // group, blk), generator=g, device=device,
-                              dtype=torch.int32).to(torch.uint8),
-        k_scale=u((B, Hkv, L_q // group, D), 0.05, 1.5),
-        k_zero=u((B, Hkv, L_q // group, D), -3.0, -0.5),
-        v_scale=u((B, Hkv, L_q // 2, D // group, 2), 0.05, 1.5),
-        v_zero=u((B, Hkv, L_q // 2, D // group, 2), -3.0, -0.5),
+        bits=bits, group=group, L_q=L_q, R=R_cap, R_cap=R_cap, D=D, records=records,
         k_res=normal((B, Hkv, R_cap, D), seed + 11, device),
         v_res=normal((B, Hkv, R_cap, D), seed + 12, device),
     )

@@ -40,8 +40,7 @@ class vc_attn_shape(Structure):
 
 
 class vc_quant_cache(Structure):
-    _fields_ = [("k_codes", c_void_p), ("v_codes", c_void_p), ("k_scale", c_void_p), ("k_zero", c_void_p),
-                ("v_scale", c_void_p), ("v_zero", c_void_p), ("k_res", c_void_p), ("v_res", c_void_p),
+    _fields_ = [("records", c_void_p), ("k_res", c_void_p), ("v_res", c_void_p),
                 ("bits", c_int), ("group", c_int), ("L_q", c_int64), ("R", c_int), ("R_cap", c_int)]
 
 
@@ -99,6 +98,8 @@ def lib() -> ctypes.CDLL:
                                   c_void_p, c_size_t, c_void_p]),
             "vc_workspace_flags": (c_int, [c_void_p, c_size_t, P(c_uint32), c_void_p]),
             "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
+            "vc_debug_quant_partition": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_int, c_void_p, c_int,
+                                                 P(c_int), P(c_int), P(c_int64), P(c_int64)]),
             "vc_kvstream_create": (c_int, [P(c_void_p), c_int, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p,
                                            c_void_p]),
             "vc_kvstream_prefetch": (c_int, [c_void_p, c_int]),
@@ -152,12 +153,10 @@ def shape(B: int, Hq: int, Hkv: int, D: int, sm_scale: float = 0.0) -> vc_attn_s
 
 def quant_cache(t: dict) -> vc_quant_cache:
     """Descriptor of a quantised cache given as a dict of CUDA tensors with the
-    keys k_codes, v_codes, k_scale, k_zero, v_scale, v_zero, k_res, v_res and
-    ints bits, group, L_q, R, R_cap (the layout documented in vc.h).  The
-    descriptor holds raw device pointers; it keeps references to the tensors so
-    they stay allocated while it lives."""
-    d = vc_quant_cache(_p(t["k_codes"]), _p(t["v_codes"]), _p(t["k_scale"]), _p(t["k_zero"]),
-                       _p(t["v_scale"]), _p(t["v_zero"]), _p(t.get("k_res")), _p(t.get("v_res")),
+    keys records, k_res, v_res and ints bits, group, L_q, R, R_cap (the layout
+    documented in vc.h).  The descriptor holds raw device pointers; it keeps
+    references to the tensors so they stay allocated while it lives."""
+    d = vc_quant_cache(_p(t["records"]), _p(t.get("k_res")), _p(t.get("v_res")),
                        int(t["bits"]), int(t["group"]), int(t["L_q"]), int(t["R"]), int(t["R_cap"]))
     d._keep = dict(t)
     return d
@@ -235,6 +234,22 @@ def vc_workspace_flags(ws, stream=None) -> int:
 
 def vc_debug_dequant(sh, qc, k_out, v_out, stream=None):
     _check(lib().vc_debug_dequant(ctypes.byref(sh), ctypes.byref(qc), _p(k_out), _p(v_out), _stream(stream)))
+
+
+def vc_debug_quant_partition(sh, qc, target_blocks: int) -> dict:
+    """How vc_draft_attn_quant cuts a call into at most target_blocks blocks
+    (no GPU needed): first stage of every block plus the stage counts."""
+    L = lib()
+    nb, ms = ctypes.c_int(), ctypes.c_int()
+    ns, nqs = ctypes.c_int64(), ctypes.c_int64()
+    _check(L.vc_debug_quant_partition(ctypes.byref(sh), ctypes.byref(qc), int(target_blocks), None, 0,
+                                      ctypes.byref(nb), ctypes.byref(ms), ctypes.byref(ns), ctypes.byref(nqs)))
+    first = (ctypes.c_int64 * (nb.value + 1))()
+    _check(L.vc_debug_quant_partition(ctypes.byref(sh), ctypes.byref(qc), int(target_blocks), first,
+                                      nb.value + 1, ctypes.byref(nb), ctypes.byref(ms), ctypes.byref(ns),
+                                      ctypes.byref(nqs)))
+    return dict(first=list(first), n_blocks=nb.value, max_segments=ms.value, n_stages=ns.value,
+                n_quant_stages=nqs.value)
 
 
 def vc_debug_gather(sh, sc, k_out, v_out, ws=None, stream=None):

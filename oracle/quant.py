@@ -22,17 +22,19 @@ Readings taken where the pages are silent (all listed in the design doc)
   multiply-add).  In float64 the product and sum below are exact (code < 2**4,
   s and z are fp16), so rounding the float64 result to float32 once is exactly
   that single rounding.
-* Storage order of the codes (a choice of this library, the pages fix
-  none): the codes of each group of G tokens form one block in the
-  "fragment-native" order defined in key_code_positions /
-  value_code_positions below -- the order in which a warp of the draft
-  kernel feeds them to its tensor-core tiles.  Value scales and zeros are
-  stored pair-interleaved: for tokens (2p, 2p+1) the CPG = D / G groups
-  hold (s[2p][cg], s[2p+1][cg]) next to each other.  Key scales and zeros
-  keep the natural [group][channel] order.  pack_codes / unpack_codes
-  (the plain row order: channel c of a token at bits [(c mod (8/b)) * b,
-  +b) of byte c * b / 8) remain as the reference from which the block order
-  is a fixed permutation.
+* Storage (a choice of this library, the pages fix none): everything one
+  group of G quantised tokens needs is one contiguous RECORD (record_layout
+  below): the key-code block, the value-code block, the key scales and
+  zeros of the group's D channels, and the value scales and zeros of its G
+  tokens.  Code blocks are in the "fragment-native" order defined in
+  key_code_positions / value_code_positions -- the order in which a warp of
+  the draft kernel feeds them to its tensor-core tiles.  Key scales and
+  zeros are in the fragment order of key_param_positions.  Value scales and
+  zeros are pair-interleaved: for tokens (2p, 2p+1) the CPG = D / G groups
+  hold (s[2p][cg], s[2p+1][cg]) next to each other.  pack_codes /
+  unpack_codes (the plain row order: channel c of a token at bits
+  [(c mod (8/b)) * b, +b) of byte c * b / 8) remain as the reference from
+  which the block order is a fixed permutation.
 * The oldest L_q = T - R tokens are quantised; the newest R stay bf16
   (the "recent-token residual window").
 """
@@ -254,16 +256,98 @@ def dequantize_values(codes: np.ndarray, s: np.ndarray, z: np.ndarray, group: in
     return (codes * s_c + z_c).astype(np.float32)
 
 
+# ---------------------------------------------------------------------------
+# Key scales / zeros of a group in fragment order.  A lane with tig (0..3)
+# multiplies, for every 16-channel tile kt, the channel pairs
+# (16kt + 2tig, +1) and (16kt + 8 + 2tig, +1); the row of D fp16 entries is
+# stored so that those pairs are one run of 2 * (D/16) 32-bit words per tig:
+#   channel c = 16 kt + 8 h + 2 tig + e   (h, e in {0, 1})
+#   -> 32-bit word tig * 2 (D/16) + 2 kt + h, fp16 slot e of that word.
+# ---------------------------------------------------------------------------
+
+def key_param_positions(D: int) -> np.ndarray:
+    """fp16 index, inside a group's key-scale (or key-zero) row, of channel c."""
+    KT = D // 16
+    pos = np.empty(D, np.int64)
+    for c in range(D):
+        kt, r = divmod(c, 16)
+        h, r2 = divmod(r, 8)
+        tig, e = divmod(r2, 2)
+        pos[c] = 2 * (tig * 2 * KT + 2 * kt + h) + e
+    return pos
+
+
+def record_layout(bits: int, G: int, D: int) -> dict:
+    """Byte offsets of the parts of one group record and its size.
+      kc  key codes,   G*D*bits/8 bytes (fragment-native block)
+      vc  value codes, G*D*bits/8 bytes (fragment-native block)
+      sk  key scales,  D fp16 (key_param_positions order)
+      zk  key zeros,   D fp16 (same order)
+      sv  value scales of the G tokens, [G/2][D/G][2] fp16 (pair-interleaved)
+      zv  value zeros, same shape"""
+    cb = G * D * bits // 8
+    off = dict(kc=0, vc=cb, sk=2 * cb, zk=2 * cb + 2 * D, sv=2 * cb + 4 * D, zv=2 * cb + 6 * D)
+    off["size"] = 2 * cb + 8 * D
+    return off
+
+
+def pack_group_records(kc_blocks, vc_blocks, sk, zk, sv_pairs, zv_pairs, bits: int, G: int) -> np.ndarray:
+    """Assemble records [..., L/G, size] from code blocks [..., L/G, CB], key
+    scales/zeros [..., L/G, D] (natural channel order) and pair-interleaved
+    value scales/zeros [..., L/2, D/G, 2]."""
+    kc_blocks = np.asarray(kc_blocks, np.uint8)
+    *lead, ng, _ = kc_blocks.shape
+    D = np.asarray(sk).shape[-1]
+    lay = record_layout(bits, G, D)
+    out = np.zeros((*lead, ng, lay["size"]), np.uint8)
+    pos = key_param_positions(D)
+
+    def put(name, arr16):
+        b = np.ascontiguousarray(arr16.astype(np.float16)).view(np.uint8)
+        out[..., lay[name]:lay[name] + b.shape[-1]] = b
+
+    out[..., lay["kc"]:lay["vc"]] = kc_blocks
+    out[..., lay["vc"]:lay["sk"]] = np.asarray(vc_blocks, np.uint8)
+    for name, row in (("sk", sk), ("zk", zk)):
+        perm = np.empty_like(np.asarray(row, np.float16))
+        perm[..., pos] = np.asarray(row, np.float16)
+        put(name, perm)
+    for name, pr in (("sv", sv_pairs), ("zv", zv_pairs)):
+        pr = np.asarray(pr, np.float16)
+        put(name, pr.reshape(*lead, ng, (G // 2) * pr.shape[-2] * 2))
+    return out
+
+
+def unpack_group_records(records, bits: int, G: int, D: int):
+    """Inverse of pack_group_records: (kc_blocks, vc_blocks, sk, zk, sv_pairs,
+    zv_pairs) with key parameters back in natural channel order."""
+    rec = np.asarray(records, np.uint8)
+    *lead, ng, size = rec.shape
+    lay = record_layout(bits, G, D)
+    if size != lay["size"]:
+        raise ValueError("record size does not match bits, group and head dim")
+    pos = key_param_positions(D)
+
+    def get16(name, n):
+        return np.ascontiguousarray(rec[..., lay[name]:lay[name] + 2 * n]).view(np.float16)
+
+    sk = get16("sk", D)[..., pos]
+    zk = get16("zk", D)[..., pos]
+    cpg = D // G
+    sv = get16("sv", D).reshape(*lead, ng * G // 2, cpg, 2)
+    zv = get16("zv", D).reshape(*lead, ng * G // 2, cpg, 2)
+    return (rec[..., lay["kc"]:lay["vc"]].copy(), rec[..., lay["vc"]:lay["sk"]].copy(), sk, zk, sv, zv)
+
+
 def build_quant_cache(k: np.ndarray, v: np.ndarray, bits: int, group: int, residual: int) -> dict:
     """Compress one layer's full cache into the quantised draft cache.
 
     k, v: [B, Hkv, T, D] bf16 values (as float32).  The oldest
     L_q = T - residual tokens are quantised, the newest ``residual`` stay bf16.
     Returns a dict in the library's storage layout:
-      k_codes, v_codes  uint8 [B, Hkv, L_q/G, G*D*bits/8]  (block order)
-      k_scale, k_zero   fp16  [B, Hkv, L_q/G, D]
-      v_scale, v_zero   fp16  [B, Hkv, L_q/2, D/G, 2]      (pair-interleaved)
-      k_res, v_res      bf16 values [B, Hkv, residual, D]"""
+      records     uint8 [B, Hkv, L_q/G, size]  (record_layout)
+      k_res, v_res bf16 values [B, Hkv, residual, D]
+    plus bits, group, L_q, R, D."""
     k = np.asarray(k, np.float32)
     v = np.asarray(v, np.float32)
     T, D = k.shape[-2], k.shape[-1]
@@ -272,24 +356,30 @@ def build_quant_cache(k: np.ndarray, v: np.ndarray, bits: int, group: int, resid
         raise ValueError("T - residual must be a non-negative multiple of the group size")
     kc, sk, zk = quantize_keys(k[..., :L_q, :], bits, group)
     vc, sv, zv = quantize_values(v[..., :L_q, :], bits, group)
-    return dict(
-        bits=bits, group=group, L_q=L_q, R=residual,
-        k_codes=pack_group_blocks(kc, bits, group, values=False),
-        v_codes=pack_group_blocks(vc, bits, group, values=True),
-        k_scale=sk, k_zero=zk, v_scale=pair_interleave(sv), v_zero=pair_interleave(zv),
-        k_res=k[..., L_q:, :].copy(), v_res=v[..., L_q:, :].copy(),
-    )
+    records = pack_group_records(pack_group_blocks(kc, bits, group, values=False),
+                                 pack_group_blocks(vc, bits, group, values=True),
+                                 sk, zk, pair_interleave(sv), pair_interleave(zv), bits, group)
+    return dict(bits=bits, group=group, L_q=L_q, R=residual, D=D, records=records,
+                k_res=k[..., L_q:, :].copy(), v_res=v[..., L_q:, :].copy())
+
+
+def cache_parts(cache: dict):
+    """Codes and parameters of a quantised cache in natural order:
+    (k_codes [.., L_q, D], k_scale, k_zero [.., L_q/G, D],
+     v_codes [.., L_q, D], v_scale, v_zero [.., L_q, D/G])."""
+    bits, G, D = cache["bits"], cache["group"], cache["D"]
+    kb, vb, sk, zk, sv, zv = unpack_group_records(cache["records"], bits, G, D)
+    return (unpack_group_blocks(kb, bits, G, D, values=False), sk, zk,
+            unpack_group_blocks(vb, bits, G, D, values=True), pair_deinterleave(sv), pair_deinterleave(zv))
 
 
 def dequantize_cache(cache: dict):
     """Full-length (K_hat, V_hat) of a quantised cache: dequantised rows
     followed by the bf16 residual rows.  Float32 arrays [B, Hkv, L_q + R, D]."""
-    bits, G = cache["bits"], cache["group"]
-    D = cache["k_scale"].shape[-1]
-    kc = unpack_group_blocks(cache["k_codes"], bits, G, D, values=False)
-    vc = unpack_group_blocks(cache["v_codes"], bits, G, D, values=True)
-    kh = dequantize_keys(kc, cache["k_scale"], cache["k_zero"], G)
-    vh = dequantize_values(vc, pair_deinterleave(cache["v_scale"]), pair_deinterleave(cache["v_zero"]), G)
+    G = cache["group"]
+    kc, sk, zk, vc, sv, zv = cache_parts(cache)
+    kh = dequantize_keys(kc, sk, zk, G)
+    vh = dequantize_values(vc, sv, zv, G)
     R = cache["R"]
     kr = np.asarray(cache["k_res"], np.float32)[..., :R, :]
     vr = np.asarray(cache["v_res"], np.float32)[..., :R, :]

@@ -42,10 +42,9 @@ def test_dequant_bit_exact(bits, G, D):
     vo = torch.empty_like(ko)
     vc.vc_debug_dequant(vc.shape(B, 2 * Hkv, Hkv, D), vc.quant_cache(tc), ko, vo)
     torch.cuda.synchronize()
-    kc = Q.unpack_group_blocks(cache["k_codes"], bits, G, D, values=False)
-    vcd = Q.unpack_group_blocks(cache["v_codes"], bits, G, D, values=True)
-    kw = Q.dequantize_keys(kc, cache["k_scale"], cache["k_zero"], G)
-    vw = Q.dequantize_values(vcd, Q.pair_deinterleave(cache["v_scale"]), Q.pair_deinterleave(cache["v_zero"]), G)
+    kc, sk, zk, vcd, sv, zv = Q.cache_parts(cache)
+    kw = Q.dequantize_keys(kc, sk, zk, G)
+    vw = Q.dequantize_values(vcd, sv, zv, G)
     assert np.array_equal(ko.cpu().numpy().view(np.uint32), kw.view(np.uint32))
     assert np.array_equal(vo.cpu().numpy().view(np.uint32), vw.view(np.uint32))
 

@@ -137,15 +137,84 @@ def test_pair_interleave():
     assert np.array_equal(quant.pair_deinterleave(q), p)
 
 
+def _records(golden_dir):
+    with open(os.path.join(golden_dir, "record_positions.json")) as f:
+        return json.load(f)
+
+
+def test_key_param_slots_worked_by_hand(golden_dir):
+    for c in _records(golden_dir)["key_param_slots"]:
+        assert int(quant.key_param_positions(c["D"])[c["channel"]]) == c["slot"], c["why"]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_key_param_order_gives_each_tig_one_run(D):
+    """Permutation of the D slots; lane tig's channel pairs are the words
+    [tig*2KT, (tig+1)*2KT) in the order (kt, h) -- one contiguous run."""
+    pos = quant.key_param_positions(D)
+    assert sorted(pos.tolist()) == list(range(D))
+    KT = D // 16
+    for tig in range(4):
+        chans = [16 * kt + 8 * h + 2 * tig + e for kt in range(KT) for h in (0, 1) for e in (0, 1)]
+        assert pos[chans].tolist() == list(range(tig * 4 * KT, (tig + 1) * 4 * KT))
+
+
+def test_record_sizes_worked_by_hand(golden_dir):
+    for c in _records(golden_dir)["record_size"]:
+        assert quant.record_layout(c["bits"], c["group"], c["D"])["size"] == c["size"]
+
+
+def test_planted_parameters_land_on_hand_worked_bytes(golden_dir):
+    """Quantise data whose scales / zeros are known, then read the fp16 at the
+    byte offset worked by hand."""
+    for c in _records(golden_dir)["record_bytes"]:
+        bits, G, D = c["bits"], c["group"], c["D"]
+        levels = (1 << bits) - 1
+        rng = np.random.default_rng(1)
+        x = rng.integers(0, levels + 1, size=(1, 1, G, D)).astype(np.float64)
+        if c["part"] in ("key_scale", "key_zero"):
+            ch = c["channel"]
+            x[..., ch] = 0.25
+            x[..., 1, ch] = 0.25 + 0.5 * levels                         # zero 0.25, scale 0.5
+            want = 0.5 if c["part"] == "key_scale" else 0.25
+            cache = quant.build_quant_cache(x, np.zeros_like(x), bits, G, 0)
+        else:
+            t, vg = c["token"], c["vgroup"]
+            v = np.zeros_like(x)
+            v[..., t, vg * G:(vg + 1) * G] = -0.75
+            v[..., t, vg * G + 1] = -0.75 + 0.125 * levels                  # zero -0.75, scale 0.125
+            want = 0.125 if c["part"] == "value_scale" else -0.75
+            cache = quant.build_quant_cache(x, v, bits, G, 0)
+        rec = cache["records"][0, 0, 0]
+        got = float(rec[c["byte"]:c["byte"] + 2].view(np.float16)[0])
+        assert got == want, c["why"]
+
+
+@pytest.mark.parametrize("bits,G,D", [(2, 32, 128), (4, 64, 128), (2, 64, 64), (4, 32, 64)])
+def test_records_round_trip_and_match_direct_quantisation(bits, G, D):
+    rng = np.random.default_rng(bits * G + D)
+    B, H, T, R = 2, 3, 3 * G + 5, 5
+    k = (rng.standard_normal((B, H, T, D)) * np.exp(rng.standard_normal((B, H, 1, D)))).astype(np.float32)
+    v = rng.standard_normal((B, H, T, D)).astype(np.float32)
+    c = quant.build_quant_cache(k, v, bits, G, R)
+    assert c["records"].shape == (B, H, (T - R) // G, quant.record_layout(bits, G, D)["size"])
+    kc, sk, zk, vc, sv, zv = quant.cache_parts(c)
+    kc0, sk0, zk0 = quant.quantize_keys(k[..., :T - R, :], bits, G)
+    vc0, sv0, zv0 = quant.quantize_values(v[..., :T - R, :], bits, G)
+    for a, b in ((kc, kc0), (sk, sk0), (zk, zk0), (vc, vc0), (sv, sv0), (zv, zv0)):
+        assert np.array_equal(a, b)
+    parts = quant.unpack_group_records(c["records"], bits, G, D)
+    again = quant.pack_group_records(*parts, bits, G)
+    assert np.array_equal(again, c["records"])
+
+
 def test_build_cache_layout():
     rng = np.random.default_rng(0)
     B, H, T, D, R, G = 2, 3, 96, 64, 32, 32
     k = rng.standard_normal((B, H, T, D)).astype(np.float32)
     v = rng.standard_normal((B, H, T, D)).astype(np.float32)
     c = quant.build_quant_cache(k, v, 2, G, R)
-    assert c["k_codes"].shape == (B, H, (T - R) // G, G * D // 4)
-    assert c["k_scale"].shape == (B, H, (T - R) // G, D)
-    assert c["v_scale"].shape == (B, H, (T - R) // 2, D // G, 2)
+    assert c["records"].shape == (B, H, (T - R) // G, 2 * G * D // 4 + 8 * D)
     kh, vh = quant.dequantize_cache(c)
     assert kh.shape == (B, H, T, D)
     assert np.array_equal(kh[:, :, T - R:], k[:, :, T - R:])

@@ -45,13 +45,9 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
 def test_noalloc_refuses_a_call_larger_than_its_scratch():
     # 1600 (request, head) pairs need more split-K scratch than the fixed array
     B, Hq, Hkv, D, Lq = 200, 64, 8, 128, 64
+    rec = 2 * 32 * D * 2 // 8 + 8 * D
     tc = dict(bits=2, group=32, L_q=Lq, R=0, R_cap=1,
-              k_codes=torch.zeros(B, Hkv, Lq, D // 4, dtype=torch.uint8, device=dev),
-              v_codes=torch.zeros(B, Hkv, Lq, D // 4, dtype=torch.uint8, device=dev),
-              k_scale=torch.ones(B, Hkv, Lq // 32, D, dtype=torch.float16, device=dev),
-              k_zero=torch.zeros(B, Hkv, Lq // 32, D, dtype=torch.float16, device=dev),
-              v_scale=torch.ones(B, Hkv, Lq, D // 32, dtype=torch.float16, device=dev),
-              v_zero=torch.zeros(B, Hkv, Lq, D // 32, dtype=torch.float16, device=dev),
+              records=torch.zeros(B, Hkv, Lq // 32, rec, dtype=torch.uint8, device=dev),
               k_res=torch.zeros(B, Hkv, 1, D, dtype=torch.bfloat16, device=dev),
               v_res=torch.zeros(B, Hkv, 1, D, dtype=torch.bfloat16, device=dev))
     sh = vc.shape(B, Hq, Hkv, D)

@@ -34,8 +34,8 @@ def quant_cache_to_torch(cache: dict, device, R_cap: int | None = None, pad_valu
     a kernel that reads them produces NaN."""
     R = cache["R"]
     R_cap = R if R_cap is None else R_cap
-    B, H = cache["k_codes"].shape[:2]
-    D = cache["k_scale"].shape[-1]
+    B, H = cache["records"].shape[:2]
+    D = cache["D"]
 
     def res(x):
         out = torch.full((B, H, max(R_cap, 1), D), pad_value, dtype=torch.float32)
@@ -43,21 +43,16 @@ def quant_cache_to_torch(cache: dict, device, R_cap: int | None = None, pad_valu
             out[:, :, :R] = torch.from_numpy(np.ascontiguousarray(x[:, :, :R]))
         return out.to(torch.bfloat16).to(device)
 
-    f16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).astype(np.float16)).to(device)
-    u8 = lambda a: torch.from_numpy(np.ascontiguousarray(a).astype(np.uint8)).to(device)
+    rec = torch.from_numpy(np.ascontiguousarray(cache["records"]).astype(np.uint8)).to(device)
     return dict(bits=cache["bits"], group=cache["group"], L_q=cache["L_q"], R=R, R_cap=max(R_cap, 1),
-                k_codes=u8(cache["k_codes"]), v_codes=u8(cache["v_codes"]),
-                k_scale=f16(cache["k_scale"]), k_zero=f16(cache["k_zero"]),
-                v_scale=f16(cache["v_scale"]), v_zero=f16(cache["v_zero"]),
-                k_res=res(cache["k_res"]), v_res=res(cache["v_res"]))
+                records=rec, k_res=res(cache["k_res"]), v_res=res(cache["v_res"]))
 
 
 def quant_cache_from_torch(t: dict) -> dict:
     """Device quantised cache (e.g. drawn on the GPU for a full-size run) as the
     oracle's numpy dict; only rows 0..R-1 of the residual are kept."""
     R = int(t["R"])
-    c = lambda x: x.detach().cpu().numpy()
-    return dict(bits=int(t["bits"]), group=int(t["group"]), L_q=int(t["L_q"]), R=R,
-                k_codes=c(t["k_codes"]), v_codes=c(t["v_codes"]),
-                k_scale=c(t["k_scale"]), k_zero=c(t["k_zero"]), v_scale=c(t["v_scale"]), v_zero=c(t["v_zero"]),
+    D = int(t["k_res"].shape[-1])
+    return dict(bits=int(t["bits"]), group=int(t["group"]), L_q=int(t["L_q"]), R=R, D=D,
+                records=t["records"].detach().cpu().numpy(),
                 k_res=np32(t["k_res"][:, :, :R]), v_res=np32(t["v_res"][:, :, :R]))
