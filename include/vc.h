@@ -378,9 +378,9 @@ VC_API vc_status vc_debug_gather(const vc_attn_shape* shape, const vc_sparse_cac
 /* vc_debug_quant_partition reports, without touching a GPU, how
  * vc_draft_attn_quant cuts one call into blocks when at most target_blocks
  * blocks are allowed (the real call uses SMs x resident blocks).  The call is
- * one axis of stages: every (request, head) unit's quantised groups
- * (n_quant_stages in all), then every unit's residual rows, 16 per stage
- * (n_stages in all).  Block k owns stages [first_stage[k], first_stage[k+1]);
+ * one axis of stages: every (request, head) unit's residual rows, 16 per
+ * stage, then every unit's quantised groups (n_quant_stages of the n_stages
+ * stages).  Block k owns stages [first_stage[k], first_stage[k+1]);
  * *max_segments is the most unit parts (quantised or residual part of one
  * unit) one block touches.  first_stage may be NULL; else it needs
  * max_blocks >= *n_blocks + 1 entries. */

@@ -80,6 +80,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test, but a thread whose phase is not complete is suspended until it
+// completes or about hint_ns nanoseconds pass (so waiting warps do not take
+// issue slots from the warps that compute).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -88,14 +103,15 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 // Waits for phase `parity` of an mbarrier, giving up after ~limit_ns.  On
 // give-up it ORs VC_FLAG_WAIT_TIMEOUT into *flags (if non-null) and returns
-// false.  No unbounded spin exists anywhere in this library.
+// false.  No unbounded spin exists anywhere in this library.  Each test
+// suspends the thread for up to 20 us while the phase is incomplete.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* flags,
                                                   uint64_t limit_ns = 2000000000ull) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 255u && global_timer_ns() - t0 > limit_ns) {
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if (global_timer_ns() - t0 > limit_ns) {
       if (flags) atomicOr(flags, VC_FLAG_WAIT_TIMEOUT);
       return false;
     }

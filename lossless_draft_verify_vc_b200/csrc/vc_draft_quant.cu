@@ -49,7 +49,6 @@ namespace {
 
 constexpr int kQNW = 4;          // warps per block
 constexpr int kResRows = 16;     // residual rows per stage
-constexpr int kMergeChunk = 64;  // partials weighed per pass when a unit is finished
 constexpr int kResCostWeight = 2;  // residual stages are not pipelined: count their bytes twice
 
 template <int BITS, int G, int D, int NT>
@@ -65,8 +64,7 @@ struct QCfg {
   static constexpr int STAGE = NG * REC;
   static constexpr int NST0 = (NT == 1 ? 9216 : 18432) / STAGE;
   static constexpr int NST = NST0 < 2 ? 2 : (NST0 > 4 ? 4 : NST0);  // ring depth
-  static constexpr int RS = D * 2 + 16;                              // residual smem row stride
-  static constexpr int RSTAGE = 2 * kResRows * RS;                   // 16 K + 16 V rows
+  static constexpr int RSTAGE = 2 * kResRows * D * 2;                // 16 K + 16 V bf16 rows
   static constexpr int RING0 = NST * STAGE > RSTAGE ? NST * STAGE : RSTAGE;
   static constexpr int RING = (RING0 + 127) / 128 * 128;
   static constexpr int HEADS = 4 * NT;
@@ -75,11 +73,9 @@ struct QCfg {
   static constexpr int STATE_OFF = kQNW * WARP_B;                       // fp32 [kQNW][HEADS][D]
   static constexpr int ML_OFF = STATE_OFF + kQNW * HEADS * D * 4;       // fp32 [kQNW][HEADS][2]
   static constexpr int MW_OFF = ML_OFF + kQNW * HEADS * 2 * 4;          // merge weights + (M, L)
-  static constexpr int MW_FLOATS = kMergeChunk * HEADS + 2 * HEADS;
-  static constexpr int SLOT_OFF = (MW_OFF + MW_FLOATS * 4 + 15) / 16 * 16;  // int64 [kMergeChunk]
-  static constexpr int BAR_OFF = SLOT_OFF + kMergeChunk * 8;
-  static constexpr int TICK_OFF = BAR_OFF + kQNW * (NST + 1) * 8;
-  static constexpr int SMEM_B = TICK_OFF + 16;
+  static constexpr int MW_FLOATS = kQNW * HEADS + 2 * HEADS;
+  static constexpr int BAR_OFF = (MW_OFF + MW_FLOATS * 4 + 15) / 16 * 16;
+  static constexpr int SMEM_B = BAR_OFF + kQNW * (NST + 1) * 8;
   static constexpr int KT = D / 16;   // channel tiles
   static constexpr int CPG = D / G;   // value groups per token
   static_assert(G % 32 == 0, "group must be a multiple of 32");
@@ -90,30 +86,32 @@ struct QCfg {
 
 // The stage axis and its cut into blocks; the same arithmetic runs on the
 // host (planning, workspace size) and on the device.
-//   stage s <  QZ : quantised stage s % sq of unit s / sq   (cost cq)
-//   stage s >= QZ : residual stage (s - QZ) % sr of unit (s - QZ) / sr (cost cr)
+//   stage s <  RZ : residual stage s % sr of unit s / sr            (cost cr)
+//   stage s >= RZ : quantised stage (s - RZ) % sq of unit (s - RZ) / sq (cost cq)
+// The residual zone comes first so that a unit's last partial (whose block
+// finishes the unit) comes from the quantised zone, spread over many blocks.
 // Block k owns the stages whose start cost c_s satisfies
 // ceil(k C / n) <= c_s < ceil((k + 1) C / n); equivalently the block of stage
 // s is floor(c_s n / C).  The host keeps n <= C / max(cq, cr), so every block
-// owns at least one stage.  Segment of a stage: its unit's quantised part
-// (id u) or residual part (id U + u).
+// owns at least one stage.  Segments along the axis: the residual part of
+// unit u (id u), then the quantised part of unit u (id U + u).
 struct Partition {
   int64_t ng;      // groups per unit
-  int64_t QZ;      // stages in the quantised zone = U * sq
-  int64_t S_tot;   // all stages
+  int64_t RZ;      // stages in the residual zone = U * sr
+  int64_t S_tot;   // all stages = RZ + U * sq
   int64_t cq, cr;  // cost of one quantised / residual stage
   int64_t C;       // total cost
   int U, sq, sr, nblk;
 
-  __host__ __device__ int64_t cost(int64_t s) const { return s < QZ ? s * cq : QZ * cq + (s - QZ) * cr; }
+  __host__ __device__ int64_t cost(int64_t s) const { return s < RZ ? s * cr : RZ * cr + (s - RZ) * cq; }
   __host__ __device__ int64_t first(int k) const {
     if (k <= 0) return 0;
     if (k >= nblk) return S_tot;
     const int64_t T = (static_cast<int64_t>(k) * C + nblk - 1) / nblk;
-    if (QZ > 0 && T <= (QZ - 1) * cq) return (T + cq - 1) / cq;
-    const int64_t base = QZ * cq;
-    if (T <= base) return QZ;
-    const int64_t s = QZ + (T - base + cr - 1) / cr;
+    if (RZ > 0 && T <= (RZ - 1) * cr) return (T + cr - 1) / cr;
+    const int64_t base = RZ * cr;
+    if (T <= base) return RZ;
+    const int64_t s = RZ + (T - base + cq - 1) / cq;
     return s < S_tot ? s : S_tot;
   }
   __host__ __device__ int block_of(int64_t s) const {
@@ -121,12 +119,12 @@ struct Partition {
     return k < nblk ? static_cast<int>(k) : nblk - 1;
   }
   __host__ __device__ int seg_of(int64_t s) const {
-    return s < QZ ? static_cast<int>(s / sq) : U + static_cast<int>((s - QZ) / sr);
+    return s < RZ ? static_cast<int>(s / sr) : U + static_cast<int>((s - RZ) / sq);
   }
   __host__ __device__ int64_t seg_begin(int seg) const {
-    return seg < U ? static_cast<int64_t>(seg) * sq : QZ + static_cast<int64_t>(seg - U) * sr;
+    return seg < U ? static_cast<int64_t>(seg) * sr : RZ + static_cast<int64_t>(seg - U) * sq;
   }
-  __host__ __device__ int64_t seg_end(int seg) const { return seg_begin(seg) + (seg < U ? sq : sr); }
+  __host__ __device__ int64_t seg_end(int seg) const { return seg_begin(seg) + (seg < U ? sr : sq); }
 };
 
 struct QArgs {
@@ -140,7 +138,6 @@ struct QArgs {
   int MAXS;  // partial slots per block
   float scale_log2;
   uint32_t* flags;
-  uint32_t* tickets;  // [U], zero between calls
   float* part_o;      // [nblk * MAXS][g][D]
   float* part_ml;     // [nblk * MAXS][g][2]
   float* out;         // [B][Hq][D]
@@ -201,12 +198,13 @@ __device__ __forceinline__ void load_cpg(const uint32_t* p, uint32_t (&w)[CPG]) 
 }
 
 // Where this warp's next quantised stage to fetch lives: unit u, stage ls of
-// that unit.  Advancing by kQNW stages needs no division.
+// that unit (both < 2^31: units are capped at 2^24, groups per unit at 2^30).
+// Advancing by kQNW stages needs no division.
 struct IssuePtr {
-  int64_t u, ls;
+  int u, ls;
   __device__ void start(const Partition& P, int64_t s) {
-    u = s / P.sq;
-    ls = s - u * P.sq;
+    u = static_cast<int>(s / P.sq);
+    ls = static_cast<int>(s - static_cast<int64_t>(u) * P.sq);
   }
   __device__ void advance(const Partition& P) {
     ls += kQNW;
@@ -221,13 +219,14 @@ struct IssuePtr {
 template <typename C>
 __device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring, uint64_t* bars, int lane, int i,
                                             const IssuePtr& ip) {
-  const int64_t g0 = ip.ls * C::NG;
+  const int64_t g0 = static_cast<int64_t>(ip.ls) * C::NG;
   const int64_t left = a.P.ng - g0;
   const uint32_t bytes = static_cast<uint32_t>((left < C::NG ? left : C::NG) * C::REC);
   const int slot = i % C::NST;
   if (lane == 0) {
     mbar_arrive_expect_tx(&bars[slot], bytes);
-    bulk_g2s(ring + slot * C::STAGE, a.rec + (ip.u * a.P.ng + g0) * C::REC, bytes, &bars[slot]);
+    bulk_g2s(ring + slot * C::STAGE, a.rec + (static_cast<int64_t>(ip.u) * a.P.ng + g0) * C::REC, bytes,
+             &bars[slot]);
   }
 }
 
@@ -235,12 +234,13 @@ __device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring,
 // Processes this warp's stages of unit u's quantised segment (the prefetch
 // pipeline runs on across segments) and leaves the warp's state in its slot.
 template <int BITS, int G, int D, int NT>
-__device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, int u, int64_t B0, int my_nq,
+__device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, int u, int64_t qs0, int my_nq,
                           int& iq, int& issued, IssuePtr& ip, bool& ok, float* st_o, float* st_ml) {
   using C = QCfg<BITS, G, D, NT>;
   using F = Frag<BITS>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int NW = 2 * C::KT / F::TPW;  // words per lane per 16-token tile
+  constexpr int MT = G / 16;              // token tiles per group
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int part = gid & 1;
@@ -287,10 +287,19 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
     for (int mc = 0; mc < C::KT; ++mc) acc[mc][nt][0] = acc[mc][nt][1] = acc[mc][nt][2] = acc[mc][nt][3] = 0.f;
   }
 
-  const int64_t seg_lo = static_cast<int64_t>(u) * a.P.sq, seg_hi = seg_lo + a.P.sq;
-  for (; iq < my_nq; ++iq) {
-    const int64_t s = B0 + warp + static_cast<int64_t>(iq) * kQNW;
-    if (s >= seg_hi) break;
+  // this warp's stages of the segment: local stages ls0, ls0 + kQNW, ...
+  // (qs: index inside the quantised zone; this warp's i-th one is qs0 + kQNW i)
+  int n_seg = 0, ls0 = 0;
+  {
+    const int64_t seg_lo = static_cast<int64_t>(u) * a.P.sq, seg_hi = seg_lo + a.P.sq;
+    const int64_t s_first = qs0 + static_cast<int64_t>(iq) * kQNW;
+    if (iq < my_nq && s_first < seg_hi) {
+      const int64_t n = (seg_hi - s_first + kQNW - 1) / kQNW;
+      n_seg = n < my_nq - iq ? static_cast<int>(n) : my_nq - iq;
+      ls0 = static_cast<int>(s_first - seg_lo);
+    }
+  }
+  for (int kk = 0; kk < n_seg; ++kk, ++iq) {
     if (!ok) continue;
     if (issued < my_nq && issued <= iq + C::NST - 1) {
       fence_proxy_async_smem();
@@ -305,7 +314,7 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
       for (int k = iq; k < issued; ++k) mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
       continue;
     }
-    const int64_t g0 = (s - seg_lo) * C::NG;
+    const int64_t g0 = static_cast<int64_t>(ls0 + kk * kQNW) * C::NG;
     const int n_here = a.P.ng - g0 < C::NG ? static_cast<int>(a.P.ng - g0) : C::NG;
 #pragma unroll 1
     for (int gi = 0; gi < n_here; ++gi) {
@@ -317,175 +326,179 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
       const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);  // [G/2][CPG] token pairs
       const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
 
-      // (2) 32-token sub-blocks: scores, softmax, P . V
-      float kb[NT][4];  // zero-point term sum_c q_c z_c (high columns), from sub-block 0
+      // (1) scores of the group's MT token tiles in one pass over the channel
+      //     tiles kt.  Per kt the key scales are folded into q right before
+      //     use (fp16 high part in part-0 columns, low part in part-1
+      //     columns); lane tig's scale words for (kt, h) are word 2kt + h of
+      //     its run.  The zero-point term sum_c q_c z_c comes from the zeros
+      //     times 2^(bits i) (exact) against q2s, in both columns of a head
+      //     (only the high one is used).
+      float sc[MT][NT][4];
+      float kb[NT][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) kb[nt][0] = kb[nt][1] = kb[nt][2] = kb[nt][3] = 0.f;
-#pragma unroll 1
-      for (int sb = 0; sb < G / 32; ++sb) {
-        // scores of token tiles mt = 0, 1.  Per channel tile kt the key scales
-        // are folded into q right before use (fp16 high part in part-0
-        // columns, low part in part-1 columns); lane tig's scale words for
-        // (kt, h) are word 2kt + h of its run.
-        float sc[2][NT][4];
+      for (int nt = 0; nt < NT; ++nt) {
+        kb[nt][0] = kb[nt][1] = kb[nt][2] = kb[nt][3] = 0.f;
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int mt = 0; mt < MT; ++mt) sc[mt][nt][0] = sc[mt][nt][1] = sc[mt][nt][2] = sc[mt][nt][3] = 0.f;
+      }
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) sc[mt][nt][0] = sc[mt][nt][1] = sc[mt][nt][2] = sc[mt][nt][3] = 0.f;
+      for (int j = 0; j < NW / 2; ++j) {
+        uint2 w[MT];
+        uint32_t xs[MT], ys[MT];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          w[mt] = *reinterpret_cast<const uint2*>(kcw + (mt * 32 + lane) * NW + 2 * j);
+          xs[mt] = w[mt].x >> 8;
+          ys[mt] = w[mt].y >> 8;
+        }
+#pragma unroll
+        for (int i = 0; i < F::TPW; ++i) {
+          const int kt = F::TPW * j + i;
+          const uint4 s4 = skw[kt >> 1];
+          const uint32_t sA = (kt & 1) ? s4.z : s4.x, sC = (kt & 1) ? s4.w : s4.y;
+          const uint32_t m = F::mask(i);
+          uint32_t fa[NT], fc[NT];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint32_t qa = q2s[kt][nt][0], qc = q2s[kt][nt][1];
+            fa[nt] = hfma2(qa, sA, hmul2(hmul2(qa, sA), kap));
+            fc[nt] = hfma2(qc, sC, hmul2(hmul2(qc, sC), kap));
+          }
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const uint32_t af[4] = {w[mt].x & m, xs[mt] & m, w[mt].y & m, ys[mt] & m};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_f16(sc[mt][nt], af, fa[nt], fc[nt]);
+          }
+          const uint4 z4 = zkw[kt >> 1];
+          uint32_t z0 = (kt & 1) ? z4.z : z4.x, z8 = (kt & 1) ? z4.w : z4.y;
+          if (i > 0) {
+            const uint32_t f2 = static_cast<uint32_t>(15 + BITS * i) << 10;  // fp16 2^(bits i)
+            z0 = hmul2(z0, f2 | (f2 << 16));
+            z8 = hmul2(z8, f2 | (f2 << 16));
+          }
+          const uint32_t za[4] = {z0, z0, z8, z8};
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_f16(kb[nt], za, q2s[kt][nt][0], q2s[kt][nt][1]);
+        }
+      }
+
+      // (2) softmax per head nt*4 + tig over the lane's tokens 16 mt + gid (+8);
+      //     the running max is raised only when a score exceeds it by more
+      //     than 2^8 (lazy rescale; p <= 256 keeps every fp16/fp32 value in range)
+      float x[NT][2 * MT], tmax[NT];
+      bool need = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float kz = kb[nt][0] * 5.9604644775390625e-8f;  // zero-point term in the 2^-24 domain
+        float t = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          x[nt][2 * mt] = (sc[mt][nt][0] + sc[mt][nt][1] + kz) * scl;
+          x[nt][2 * mt + 1] = (sc[mt][nt][2] + sc[mt][nt][3] + kz) * scl;
+          t = fmaxf(t, fmaxf(x[nt][2 * mt], x[nt][2 * mt + 1]));
+        }
+        t = warp_max_xor(t, 4);
+        t = warp_max_xor(t, 8);
+        t = warp_max_xor(t, 16);
+        tmax[nt] = t;
+        need |= t > m_run[nt] + 8.f;
+      }
+      if (__any_sync(FULL, need)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const float m_new = fmaxf(m_run[nt], tmax[nt]);
+          const float alpha = ex2(m_run[nt] - m_new);
+          m_run[nt] = m_new;
+          l_run[nt] *= alpha;
+#pragma unroll
+          for (int mc = 0; mc < C::KT; ++mc) {
+            acc[mc][nt][0] *= alpha;
+            acc[mc][nt][1] *= alpha;
+            acc[mc][nt][2] *= alpha;
+            acc[mc][nt][3] *= alpha;
+          }
+          vb[nt][0] *= alpha;
+          vb[nt][1] *= alpha;
+          vb[nt][2] *= alpha;
+          vb[nt][3] *= alpha;
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        unsigned short* ph = reinterpret_cast<unsigned short*>(Ph + (nt * 4 + tig) * G + gid);
+        unsigned short* pl = reinterpret_cast<unsigned short*>(Pl + (nt * 4 + tig) * G + gid);
+        float ls = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const float p0 = ex2(x[nt][2 * mt] - m_run[nt]), p1 = ex2(x[nt][2 * mt + 1] - m_run[nt]);
+          ls += p0 + p1;
+          // p as fp16 high + low parts (tokens 16mt + gid and +8), split once for the value side
+          const uint32_t hh = pack_h2(p0, p1);
+          const float2 f = unpack_h2(hh);
+          const uint32_t ll = pack_h2(p0 - f.x, p1 - f.y);
+          ph[16 * mt] = static_cast<unsigned short>(hh);
+          ph[16 * mt + 8] = static_cast<unsigned short>(hh >> 16);
+          pl[16 * mt] = static_cast<unsigned short>(ll);
+          pl[16 * mt + 8] = static_cast<unsigned short>(ll >> 16);
+        }
+        l_run[nt] += ls;
+      }
+      __syncwarp();
+
+      // (3) P . V over the group's MT token tiles
+#pragma unroll
+      for (int ktt = 0; ktt < MT; ++ktt) {
+        const int t0 = ktt * 16 + 2 * tig;  // tokens t0, t0+1, t0+8, t0+9
+        uint32_t ph01[NT], ph89[NT], plm01[NT], plm89[NT], phn01[NT], phn89[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hh = nt * 4 + (gid >> 1);
+          ph01[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0);
+          ph89[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0 + 8);
+          const uint32_t pl01 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0);
+          const uint32_t pl89 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0 + 8);
+          plm01[nt] = hmul2(pl01, mu);
+          plm89[nt] = hmul2(pl89, mu);
+          phn01[nt] = hmul2(ph01[nt], kap);
+          phn89[nt] = hmul2(ph89[nt], kap);
+          // value zero-point term: A = z_v^T (row = value group gid), B = p (high or low column)
+          uint32_t za[4] = {0u, 0u, 0u, 0u};
+          if (gid < C::CPG) {
+            za[0] = zv32[(t0 >> 1) * C::CPG + gid];
+            za[2] = zv32[((t0 + 8) >> 1) * C::CPG + gid];
+          }
+          mma_f16(vb[nt], za, part ? pl01 : ph01[nt], part ? pl89 : ph89[nt]);
+        }
+        // folded p*s per value group, made right before the channel tiles
+        // that use it: high part (part 0) or low part (part 1)
+        uint32_t s01[C::CPG], s89[C::CPG];
+        load_cpg<C::CPG>(sv32 + (t0 >> 1) * C::CPG, s01);
+        load_cpg<C::CPG>(sv32 + ((t0 + 8) >> 1) * C::CPG, s89);
+        uint32_t wv[NW];
+        load_words(vcw + (ktt * 32 + lane) * NW, wv);
+        uint32_t pf[NT][2];
 #pragma unroll
         for (int j = 0; j < NW / 2; ++j) {
-          const uint2 w0 = *reinterpret_cast<const uint2*>(kcw + ((sb * 2 + 0) * 32 + lane) * NW + 2 * j);
-          const uint2 w1 = *reinterpret_cast<const uint2*>(kcw + ((sb * 2 + 1) * 32 + lane) * NW + 2 * j);
-          const uint32_t xs0 = w0.x >> 8, ys0 = w0.y >> 8, xs1 = w1.x >> 8, ys1 = w1.y >> 8;
+          const uint32_t X = wv[2 * j], Y = wv[2 * j + 1], xsv = X >> 8, ysv = Y >> 8;
 #pragma unroll
           for (int i = 0; i < F::TPW; ++i) {
-            const int kt = F::TPW * j + i;
-            const uint4 s4 = skw[kt >> 1];
-            const uint32_t sA = (kt & 1) ? s4.z : s4.x, sC = (kt & 1) ? s4.w : s4.y;
-            const uint32_t m = F::mask(i);
-            const uint32_t a0[4] = {w0.x & m, xs0 & m, w0.y & m, ys0 & m};
-            const uint32_t a1[4] = {w1.x & m, xs1 & m, w1.y & m, ys1 & m};
+            const int mc = F::TPW * j + i;  // 16-channel tile
+            const int cg = mc * 16 / G;
+            if (mc == 0 || (mc - 1) * 16 / G != cg) {
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              const uint32_t qa = q2s[kt][nt][0], qc = q2s[kt][nt][1];
-              const uint32_t fa = hfma2(qa, sA, hmul2(hmul2(qa, sA), kap));
-              const uint32_t fc = hfma2(qc, sC, hmul2(hmul2(qc, sC), kap));
-              mma_f16(sc[0][nt], a0, fa, fc);
-              mma_f16(sc[1][nt], a1, fa, fc);
-            }
-            if (sb == 0) {
-              // zeros times 2^(bits i) (exact) against q2s: sum_c z_c q_c, in
-              // both columns of a head (only the high one is used)
-              const uint4 z4 = zkw[kt >> 1];
-              uint32_t z0 = (kt & 1) ? z4.z : z4.x, z8 = (kt & 1) ? z4.w : z4.y;
-              if (i > 0) {
-                const uint32_t f2 = static_cast<uint32_t>(15 + BITS * i) << 10;  // fp16 2^(bits i)
-                z0 = hmul2(z0, f2 | (f2 << 16));
-                z8 = hmul2(z8, f2 | (f2 << 16));
+              for (int nt = 0; nt < NT; ++nt) {
+                pf[nt][0] = hfma2(plm01[nt], s01[cg], hfma2(ph01[nt], s01[cg], hmul2(phn01[nt], s01[cg])));
+                pf[nt][1] = hfma2(plm89[nt], s89[cg], hfma2(ph89[nt], s89[cg], hmul2(phn89[nt], s89[cg])));
               }
-              const uint32_t za[4] = {z0, z0, z8, z8};
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) mma_f16(kb[nt], za, q2s[kt][nt][0], q2s[kt][nt][1]);
             }
+            const uint32_t af[4] = {X & F::mask(i), Y & F::mask(i), xsv & F::mask(i), ysv & F::mask(i)};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_f16(acc[mc][nt], af, pf[nt][0], pf[nt][1]);
           }
         }
-        // softmax per head nt*4 + tig over tokens sb*32 + {gid, gid+8, gid+16, gid+24};
-        // the running max is raised only when a score exceeds it by more
-        // than 2^8 (lazy rescale; p <= 256 keeps every fp16/fp32 value in range)
-        float x[NT][4], tmax[NT];
-        bool need = false;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          // zero-point term (exact fp32, rows gid and gid+8 alike) into the 2^-24 domain
-          const float k0 = kb[nt][0] * 5.9604644775390625e-8f;
-          const float k8 = kb[nt][2] * 5.9604644775390625e-8f;
-          x[nt][0] = (sc[0][nt][0] + sc[0][nt][1] + k0) * scl;
-          x[nt][1] = (sc[0][nt][2] + sc[0][nt][3] + k8) * scl;
-          x[nt][2] = (sc[1][nt][0] + sc[1][nt][1] + k0) * scl;
-          x[nt][3] = (sc[1][nt][2] + sc[1][nt][3] + k8) * scl;
-          float t = fmaxf(fmaxf(x[nt][0], x[nt][1]), fmaxf(x[nt][2], x[nt][3]));
-          t = warp_max_xor(t, 4);
-          t = warp_max_xor(t, 8);
-          t = warp_max_xor(t, 16);
-          tmax[nt] = t;
-          need |= t > m_run[nt] + 8.f;
-        }
-        if (__any_sync(FULL, need)) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const float m_new = fmaxf(m_run[nt], tmax[nt]);
-            const float alpha = ex2(m_run[nt] - m_new);
-            m_run[nt] = m_new;
-            l_run[nt] *= alpha;
-#pragma unroll
-            for (int mc = 0; mc < C::KT; ++mc) {
-              acc[mc][nt][0] *= alpha;
-              acc[mc][nt][1] *= alpha;
-              acc[mc][nt][2] *= alpha;
-              acc[mc][nt][3] *= alpha;
-            }
-            vb[nt][0] *= alpha;
-            vb[nt][1] *= alpha;
-            vb[nt][2] *= alpha;
-            vb[nt][3] *= alpha;
-          }
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          float p[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) p[j] = ex2(x[nt][j] - m_run[nt]);
-          l_run[nt] += (p[0] + p[1]) + (p[2] + p[3]);
-          // p as fp16 high + low parts, split once here for the value side
-          const uint32_t h01 = pack_h2(p[0], p[1]), h23 = pack_h2(p[2], p[3]);
-          const float2 f01 = unpack_h2(h01), f23 = unpack_h2(h23);
-          const uint32_t l01 = pack_h2(p[0] - f01.x, p[1] - f01.y), l23 = pack_h2(p[2] - f23.x, p[3] - f23.y);
-          unsigned short* ph = reinterpret_cast<unsigned short*>(Ph + (nt * 4 + tig) * G + sb * 32 + gid);
-          unsigned short* pl = reinterpret_cast<unsigned short*>(Pl + (nt * 4 + tig) * G + sb * 32 + gid);
-          ph[0] = static_cast<unsigned short>(h01);
-          ph[8] = static_cast<unsigned short>(h01 >> 16);
-          ph[16] = static_cast<unsigned short>(h23);
-          ph[24] = static_cast<unsigned short>(h23 >> 16);
-          pl[0] = static_cast<unsigned short>(l01);
-          pl[8] = static_cast<unsigned short>(l01 >> 16);
-          pl[16] = static_cast<unsigned short>(l23);
-          pl[24] = static_cast<unsigned short>(l23 >> 16);
-        }
-        __syncwarp();
-#pragma unroll
-        for (int ktt = 0; ktt < 2; ++ktt) {
-          const int t0 = sb * 32 + ktt * 16 + 2 * tig;  // tokens t0, t0+1, t0+8, t0+9
-          uint32_t ph01[NT], ph89[NT], plm01[NT], plm89[NT], phn01[NT], phn89[NT];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int hh = nt * 4 + (gid >> 1);
-            ph01[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0);
-            ph89[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0 + 8);
-            const uint32_t pl01 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0);
-            const uint32_t pl89 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0 + 8);
-            plm01[nt] = hmul2(pl01, mu);
-            plm89[nt] = hmul2(pl89, mu);
-            phn01[nt] = hmul2(ph01[nt], kap);
-            phn89[nt] = hmul2(ph89[nt], kap);
-            // value zero-point term: A = z_v^T (row = value group gid), B = p (high or low column)
-            uint32_t za[4] = {0u, 0u, 0u, 0u};
-            if (gid < C::CPG) {
-              za[0] = zv32[(t0 >> 1) * C::CPG + gid];
-              za[2] = zv32[((t0 + 8) >> 1) * C::CPG + gid];
-            }
-            mma_f16(vb[nt], za, part ? pl01 : ph01[nt], part ? pl89 : ph89[nt]);
-          }
-          // folded p*s per value group, made right before the channel tiles
-          // that use it: high part (part 0) or low part (part 1)
-          uint32_t s01[C::CPG], s89[C::CPG];
-          load_cpg<C::CPG>(sv32 + (t0 >> 1) * C::CPG, s01);
-          load_cpg<C::CPG>(sv32 + ((t0 + 8) >> 1) * C::CPG, s89);
-          uint32_t w[NW];
-          load_words(vcw + ((sb * 2 + ktt) * 32 + lane) * NW, w);
-          uint32_t pf[NT][2];
-#pragma unroll
-          for (int j = 0; j < NW / 2; ++j) {
-            const uint32_t X = w[2 * j], Y = w[2 * j + 1], xs = X >> 8, ys = Y >> 8;
-#pragma unroll
-            for (int i = 0; i < F::TPW; ++i) {
-              const int mc = F::TPW * j + i;  // 16-channel tile
-              const int cg = mc * 16 / G;
-              if (mc == 0 || (mc - 1) * 16 / G != cg) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                  pf[nt][0] = hfma2(plm01[nt], s01[cg], hfma2(ph01[nt], s01[cg], hmul2(phn01[nt], s01[cg])));
-                  pf[nt][1] = hfma2(plm89[nt], s89[cg], hfma2(ph89[nt], s89[cg], hmul2(phn89[nt], s89[cg])));
-                }
-              }
-              const uint32_t m = F::mask(i);
-              const uint32_t af[4] = {X & m, Y & m, xs & m, ys & m};
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) mma_f16(acc[mc][nt], af, pf[nt][0], pf[nt][1]);
-            }
-          }
-        }
-        __syncwarp();
       }
+      __syncwarp();
     }
   }
 
@@ -520,7 +533,7 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
 // This warp's residual stages of unit u (16 rows each, one bulk copy per row,
 // not pipelined; the residual is a few percent of the bytes).  Leaves the
 // warp's state in its slot.
-template <int D, int NT, int RSTRIDE, int HEADS>
+template <int D, int NT, int HEADS>
 __device__ __noinline__ void residual_seg(const QArgs& a, unsigned char* ring, float* P_s, uint64_t* bar, int& rph, int u,
                              int64_t first_s, int64_t end_s, int64_t seg_b, bool& ok, float* st_o, float* st_ml) {
   constexpr int KT = D / 16;
@@ -557,14 +570,22 @@ __device__ __noinline__ void residual_seg(const QArgs& a, unsigned char* ring, f
   }
   for (int64_t s = first_s; s < end_s && ok; s += kQNW) {
     const int t0 = static_cast<int>(s - seg_b) * kResRows;
-    const int r = lane & 15;
-    const bool valid = t0 + r < a.R;
+    const int nv = a.R - t0 < kResRows ? a.R - t0 : kResRows;  // rows of this tile inside the window
     fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) mbar_arrive_expect_tx(bar, 32u * ROW_B);
+    if (nv < kResRows) {
+      // V rows the copy does not fill must read as zeros (their p is 0, but
+      // whatever a buffer holds past the window must not reach the MMA)
+      uint4* vz = reinterpret_cast<uint4*>(ring + (kResRows + nv) * ROW_B);
+      for (int e = lane; e < (kResRows - nv) * ROW_B / 16; e += 32) vz[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // the tile's K rows and V rows are contiguous: two bulk copies
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, 2u * nv * ROW_B);
+      bulk_g2s(ring, kr + static_cast<size_t>(t0) * D, nv * ROW_B, bar);
+      bulk_g2s(ring + kResRows * ROW_B, vr + static_cast<size_t>(t0) * D, nv * ROW_B, bar);
+    }
     __syncwarp();
-    const __nv_bfloat16* src = (lane < 16 ? kr : vr) + static_cast<size_t>(valid ? t0 + r : 0) * D;
-    bulk_g2s(ring + lane * RSTRIDE, src, ROW_B, bar);
     if (!__all_sync(FULL, mbar_wait_bounded(bar, rph & 1, a.flags))) {  // warp-uniform
       ok = false;
       mbar_wait_bounded(bar, rph & 1, nullptr, 100000000ull);
@@ -573,7 +594,7 @@ __device__ __noinline__ void residual_seg(const QArgs& a, unsigned char* ring, f
     }
     ++rph;
     const unsigned char* Ks = ring;
-    const unsigned char* Vs = ring + 16 * RSTRIDE;
+    const unsigned char* Vs = ring + kResRows * ROW_B;
     const int mi = lane >> 3, ri = lane & 7;
     float sc[NT][4];
 #pragma unroll
@@ -582,7 +603,7 @@ __device__ __noinline__ void residual_seg(const QArgs& a, unsigned char* ring, f
     for (int kt = 0; kt < KT; ++kt) {
       // A = K rows (tokens x channels): matrices (rows 0-7,k 0-7) (8-15,0-7) (0-7,8-15) (8-15,8-15)
       uint32_t af[4];
-      ldsm_x4(af, Ks + (ri + (mi & 1) * 8) * RSTRIDE + (kt * 16 + (mi >> 1) * 8) * 2);
+      ldsm_x4(af, Ks + (ri + (mi & 1) * 8) * ROW_B + (kt * 16 + (mi >> 1) * 8) * 2);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], af, qb[kt][nt][0], qb[kt][nt][1]);
     }
@@ -630,7 +651,7 @@ __device__ __noinline__ void residual_seg(const QArgs& a, unsigned char* ring, f
     for (int mc = 0; mc < KT; ++mc) {
       // A[chan][token]: matrices (ch 0-7, tok 0-7) (ch 8-15, tok 0-7) (ch 0-7, tok 8-15) (ch 8-15, tok 8-15)
       uint32_t af[4];
-      ldsm_x4_t(af, Vs + (ri + (mi >> 1) * 8) * RSTRIDE + (mc * 16 + (mi & 1) * 8) * 2);
+      ldsm_x4_t(af, Vs + (ri + (mi >> 1) * 8) * ROW_B + (mc * 16 + (mi & 1) * 8) * 2);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[mc][nt], af, pb[nt][0], pb[nt][1]);
     }
@@ -659,8 +680,8 @@ __device__ __noinline__ void residual_seg(const QArgs& a, unsigned char* ring, f
 }
 
 // Number of block partials of unit u and the slot of partial p of it.  A
-// unit's partials are those of its quantised segment (blocks block_of(begin)
-// .. block_of(end - 1)) followed by those of its residual segment.  Every
+// unit's partials are those of its residual segment (blocks block_of(begin)
+// .. block_of(end - 1)) followed by those of its quantised segment.  Every
 // block after the first one of a segment starts inside it, so its local
 // segment index is 0; only the first block's index needs computing.
 struct UnitPartials {
@@ -670,8 +691,8 @@ struct UnitPartials {
   int loc0[2];
   __device__ void init(const Partition& P, int u) {
     int n = 0;
-    if (P.sq > 0) seg[n++] = u;
-    if (P.sr > 0) seg[n++] = P.U + u;
+    if (P.sr > 0) seg[n++] = u;
+    if (P.sq > 0) seg[n++] = P.U + u;
     for (int i = 0; i < 2; ++i) {
       if (i < n) {
         kb[i] = P.block_of(P.seg_begin(seg[i]));
@@ -691,18 +712,14 @@ struct UnitPartials {
 };
 
 // Block-wide: merges the kQNW warp states of segment `seg` (local index j of
-// block k) into the block's partial; the block that completes unit u's last
-// partial merges all of them into out (one online pass over chunks of
-// kMergeChunk partials: their (m, l) pairs are staged in shared memory, the
-// running maximum rescales the running sums).
+// block k) into the block's partial of that segment.
 template <int D, int HEADS>
-__device__ __noinline__ void merge_segment(const QArgs& a, int k, int j, int seg, const float* st_o,
-                                           const float* st_ml, float* mw, int64_t* slots_s, uint32_t* tick_s) {
+__device__ __noinline__ void merge_segment(const QArgs& a, int k, int j, const float* st_o, const float* st_ml,
+                                           float* mw) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int g = a.g;
-  const Partition& P = a.P;
-  float* wts = mw;                       // [kQNW][HEADS]  (block merge)  /  [kMergeChunk][HEADS]
-  float* ML = mw + kMergeChunk * HEADS;  // [HEADS][2]
+  float* wts = mw;               // [kQNW][HEADS]
+  float* ML = mw + kQNW * HEADS;  // [HEADS][2]
   for (int r = tid; r < g; r += nthr) {
     float M = -INFINITY;
     for (int w = 0; w < kQNW; ++w) M = fmaxf(M, st_ml[(w * HEADS + r) * 2]);
@@ -731,92 +748,100 @@ __device__ __noinline__ void merge_segment(const QArgs& a, int k, int j, int seg
     pml[2 * r] = ML[2 * r];
     pml[2 * r + 1] = ML[2 * r + 1];
   }
-  __threadfence();
-  __syncthreads();
-  const int u = seg < P.U ? seg : seg - P.U;
+  __syncthreads();  // the warp slots are reused by the next segment
+}
+
+// Merges every unit's block partials into out.  One block of 128 threads per
+// (unit, head r): the (m, l) pairs of the unit's partials are staged in
+// shared memory, a block max / denominator is formed, then each warp sums a
+// quarter of the partials over all D channels (D/32 consecutive channels per
+// lane) and the four sums are added through shared memory.
+struct CArgs {
+  Partition P;
+  int MAXS, g, Hq, Hkv;
+  const float* part_o;
+  const float* part_ml;
+  float* out;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) combine_kernel(CArgs a) {
+  extern __shared__ __align__(16) float csm[];  // [np][2] (m, l), then [4][D] warp sums, then [2] (M, L)
+  const int u = blockIdx.x, r = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = a.g;
   UnitPartials up;
-  up.init(P, u);
-  if (tid == 0) *tick_s = atomicAdd(&a.tickets[u], 1u);
-  __syncthreads();
+  up.init(a.P, u);
   const int np = up.total();
-  if (*tick_s == static_cast<uint32_t>(np - 1)) {
-    __threadfence();
-    constexpr int EPT = (8 * D + 127) / 128;  // elements per thread for g <= 8, 128 threads
-    float acc[EPT];
-#pragma unroll
-    for (int i = 0; i < EPT; ++i) acc[i] = 0.f;
-    float* Mrun = ML;  // [HEADS][2]: running max, running denominator
-    for (int r = tid; r < g; r += nthr) {
-      Mrun[2 * r] = -INFINITY;
-      Mrun[2 * r + 1] = 0.f;
-    }
-    for (int p0 = 0; p0 < np; p0 += kMergeChunk) {
-      const int nc = np - p0 < kMergeChunk ? np - p0 : kMergeChunk;
-      __syncthreads();
-      for (int p = tid; p < nc; p += nthr) slots_s[p] = up.slot(a.MAXS, p0 + p);
-      __syncthreads();
-      // partial maxima of the chunk into wts (as m), then the new running max per row
-      for (int idx = tid; idx < nc * g; idx += nthr) {
-        const int p = idx / g, r = idx - p * g;
-        wts[p * HEADS + r] = __ldcg(a.part_ml + slots_s[p] * g * 2 + 2 * r);
-      }
-      __syncthreads();
-      __shared__ float resc[8];  // factor applied to the running sums of each row
-      for (int r = tid; r < g; r += nthr) {
-        float M = Mrun[2 * r];
-        for (int p = 0; p < nc; ++p) M = fmaxf(M, wts[p * HEADS + r]);
-        resc[r] = Mrun[2 * r] == -INFINITY ? 0.f : ex2(Mrun[2 * r] - M);
-        Mrun[2 * r] = M;
-      }
-      __syncthreads();
-      // weights of the chunk's partials against the new running max; denominators
-      for (int idx = tid; idx < nc * g; idx += nthr) {
-        const int p = idx / g, r = idx - p * g;
-        const float mp = wts[p * HEADS + r];
-        wts[p * HEADS + r] = mp == -INFINITY ? 0.f : ex2(mp - Mrun[2 * r]);
-      }
-      __syncthreads();
-      for (int r = tid; r < g; r += nthr) {
-        float L = Mrun[2 * r + 1] * resc[r];
-        for (int p = 0; p < nc; ++p) L += wts[p * HEADS + r] * __ldcg(a.part_ml + slots_s[p] * g * 2 + 2 * r + 1);
-        Mrun[2 * r + 1] = L;
-      }
-#pragma unroll
-      for (int i = 0; i < EPT; ++i) {
-        const int e = tid + i * nthr;
-        if (e < g * D) {
-          const int r = e / D;
-          float s0 = acc[i] * resc[r], s1 = 0.f, s2 = 0.f, s3 = 0.f;
-          int p = 0;
-          for (; p + 4 <= nc; p += 4) {
-            const float v0 = __ldcg(a.part_o + slots_s[p] * g * D + e);
-            const float v1 = __ldcg(a.part_o + slots_s[p + 1] * g * D + e);
-            const float v2 = __ldcg(a.part_o + slots_s[p + 2] * g * D + e);
-            const float v3 = __ldcg(a.part_o + slots_s[p + 3] * g * D + e);
-            s0 += wts[p * HEADS + r] * v0;
-            s1 += wts[(p + 1) * HEADS + r] * v1;
-            s2 += wts[(p + 2) * HEADS + r] * v2;
-            s3 += wts[(p + 3) * HEADS + r] * v3;
-          }
-          for (; p < nc; ++p) s0 += wts[p * HEADS + r] * __ldcg(a.part_o + slots_s[p] * g * D + e);
-          acc[i] = (s0 + s1) + (s2 + s3);
-        }
-      }
-    }
-    __syncthreads();
-    const int b = u / a.Hkv, h = u - b * a.Hkv;
-    float* o = a.out + (static_cast<size_t>(b) * a.Hq + h * g) * D;
-#pragma unroll
-    for (int i = 0; i < EPT; ++i) {
-      const int e = tid + i * nthr;
-      if (e < g * D) {
-        const float L = Mrun[2 * (e / D) + 1];
-        o[e] = L > 0.f ? acc[i] / L : 0.f;
-      }
-    }
-    if (tid == 0) a.tickets[u] = 0;
+  float* mls = csm;
+  float* wsum = csm + 2 * np;
+  float* ML = wsum + 4 * D;
+  for (int p = tid; p < np; p += 128) {
+    const float2 ml = *reinterpret_cast<const float2*>(a.part_ml + up.slot(a.MAXS, p) * g * 2 + 2 * r);
+    mls[2 * p] = ml.x;
+    mls[2 * p + 1] = ml.y;
   }
   __syncthreads();
+  if (warp == 0) {
+    float M = -INFINITY;
+    for (int p = lane; p < np; p += 32) M = fmaxf(M, mls[2 * p]);
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int p = lane; p < np; p += 32) {
+      const float mp = mls[2 * p];
+      L += mp == -INFINITY ? 0.f : ex2(mp - M) * mls[2 * p + 1];
+    }
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) {
+      ML[0] = M;
+      ML[1] = L;
+    }
+  }
+  __syncthreads();
+  const float M = ML[0];
+  constexpr int PER = D / 32;  // channels per lane
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  int p = warp;
+  for (; p + 12 < np; p += 16) {  // four partials of this warp in flight
+    float v[4][PER];
+    float w[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const float* src = a.part_o + (up.slot(a.MAXS, p + 4 * q4) * g + r) * D + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(src);
+        v[q4][0] = t.x, v[q4][1] = t.y, v[q4][2] = t.z, v[q4][3] = t.w;
+      } else {
+        const float2 t = *reinterpret_cast<const float2*>(src);
+        v[q4][0] = t.x, v[q4][1] = t.y;
+      }
+      const float mp = mls[2 * (p + 4 * q4)];
+      w[q4] = mp == -INFINITY ? 0.f : ex2(mp - M);
+    }
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] += w[q4] * v[q4][i];
+  }
+  for (; p < np; p += 4) {
+    const float* src = a.part_o + (up.slot(a.MAXS, p) * g + r) * D + lane * PER;
+    const float mp = mls[2 * p];
+    const float w = mp == -INFINITY ? 0.f : ex2(mp - M);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] += w * src[i];
+  }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) wsum[warp * D + lane * PER + i] = acc[i];
+  __syncthreads();
+  const int b = u / a.Hkv, h = u - b * a.Hkv;
+  float* o = a.out + (static_cast<size_t>(b) * a.Hq + h * g + r) * D;
+  const float L = ML[1];
+  for (int d = tid; d < D; d += 128) {
+    const float t = (wsum[d] + wsum[D + d]) + (wsum[2 * D + d] + wsum[3 * D + d]);
+    o[d] = L > 0.f ? t / L : 0.f;
+  }
 }
 
 template <int BITS, int G, int D, int NT>
@@ -834,38 +859,44 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
   float* st_o = reinterpret_cast<float*>(smem + C::STATE_OFF);
   float* st_ml = reinterpret_cast<float*>(smem + C::ML_OFF);
   float* mw = reinterpret_cast<float*>(smem + C::MW_OFF);
-  int64_t* slots_s = reinterpret_cast<int64_t*>(smem + C::SLOT_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + warp * (C::NST + 1);
-  uint32_t* tick_s = reinterpret_cast<uint32_t*>(smem + C::TICK_OFF);
 
-  const int64_t B1q = B1 < P.QZ ? B1 : P.QZ;
-  const int my_nq = B1q > B0 + warp ? static_cast<int>((B1q - B0 - warp + kQNW - 1) / kQNW) : 0;
+  // this warp's quantised stages: s = sQ0 + kQNW i (s >= RZ), i < my_nq
+  const int64_t lo_q = B0 > P.RZ ? B0 : P.RZ;
+  const int64_t off_q = lo_q - B0;
+  const int64_t sQ0 = B0 + warp + (off_q <= warp ? 0 : (off_q - warp + kQNW - 1) / kQNW) * kQNW;
+  const int my_nq = sQ0 < B1 ? static_cast<int>((B1 - sQ0 + kQNW - 1) / kQNW) : 0;
   if (lane == 0)
     for (int s = 0; s <= C::NST; ++s) mbar_init(&bars[s], 1);
   fence_mbar_init();
   __syncwarp();
-  bool ok = true;
+  bool ok = true, primed = false;
   int iq = 0, issued = 0, rph = 0;
   IssuePtr ip;
-  if (my_nq > 0) ip.start(P, B0 + warp);
-  while (issued < my_nq && issued < C::NST - 1) {
-    issue_stage<C>(a, ring, bars, lane, issued, ip);
-    ip.advance(P);
-    ++issued;
-  }
   for (int seg = seg0; seg <= seg1; ++seg) {
-    if (seg < P.U) {
-      quant_seg<BITS, G, D, NT>(a, ring, bars, seg, B0, my_nq, iq, issued, ip, ok, st_o, st_ml);
+    if (seg >= P.U) {
+      if (!primed) {  // the ring is free of residual tiles from here on
+        primed = true;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (my_nq > 0) ip.start(P, sQ0 - P.RZ);
+        while (issued < my_nq && issued < C::NST - 1) {
+          issue_stage<C>(a, ring, bars, lane, issued, ip);
+          ip.advance(P);
+          ++issued;
+        }
+      }
+      quant_seg<BITS, G, D, NT>(a, ring, bars, seg - P.U, sQ0 - P.RZ, my_nq, iq, issued, ip, ok, st_o, st_ml);
     } else {
       const int64_t sb = P.seg_begin(seg), se = P.seg_end(seg);
       const int64_t lo = sb > B0 ? sb : B0;
       const int64_t off = lo - B0;
       const int64_t i0 = off <= warp ? 0 : (off - warp + kQNW - 1) / kQNW;
-      residual_seg<D, NT, C::RS, C::HEADS>(a, ring, P_res, &bars[C::NST], rph, seg - P.U,
-                                           B0 + warp + i0 * kQNW, se < B1 ? se : B1, sb, ok, st_o, st_ml);
+      residual_seg<D, NT, C::HEADS>(a, ring, P_res, &bars[C::NST], rph, seg,
+                                    B0 + warp + i0 * kQNW, se < B1 ? se : B1, sb, ok, st_o, st_ml);
     }
     __syncthreads();
-    merge_segment<D, C::HEADS>(a, k, seg - seg0, seg, st_o, st_ml, mw, slots_s, tick_s);
+    merge_segment<D, C::HEADS>(a, k, seg - seg0, st_o, st_ml, mw);
   }
 }
 
@@ -941,7 +972,7 @@ __global__ void __launch_bounds__(32) debug_dequant_kernel(const uint8_t* recs, 
 struct QPlan {
   Partition P;
   int MAXS;
-  size_t off_tick, off_ml, off_o, total;
+  size_t off_ml, off_o, total;
 };
 
 // Blocks per SM for one kernel instance (cached per device).
@@ -973,11 +1004,11 @@ QPlan make_plan(const vc_attn_shape& sh, const vc_quant_cache& c, int ng_per_sta
   P.ng = c.L_q / c.group;
   P.sq = static_cast<int>((P.ng + ng_per_stage - 1) / ng_per_stage);
   P.sr = (c.R + kResRows - 1) / kResRows;
-  P.QZ = static_cast<int64_t>(P.U) * P.sq;
-  P.S_tot = P.QZ + static_cast<int64_t>(P.U) * P.sr;
-  P.cq = static_cast<int64_t>(ng_per_stage) * rec_bytes;
+  P.RZ = static_cast<int64_t>(P.U) * P.sr;
+  P.S_tot = P.RZ + static_cast<int64_t>(P.U) * P.sq;
+  P.cq = P.sq > 0 ? static_cast<int64_t>(ng_per_stage) * rec_bytes : 1;
   P.cr = P.sr > 0 ? static_cast<int64_t>(kResRows) * 4 * sh.D * kResCostWeight : 1;
-  P.C = P.QZ * P.cq + (P.S_tot - P.QZ) * P.cr;
+  P.C = P.RZ * P.cr + (P.S_tot - P.RZ) * P.cq;
   const int64_t mx = P.sq > 0 && P.sr > 0 ? (P.cq > P.cr ? P.cq : P.cr) : (P.sq > 0 ? P.cq : P.cr);
   int64_t n = target_blocks;
   if (n > P.S_tot) n = P.S_tot;
@@ -993,8 +1024,7 @@ QPlan make_plan(const vc_attn_shape& sh, const vc_quant_cache& c, int ng_per_sta
   p.MAXS = maxs;
   const int g = sh.Hq / sh.Hkv;
   const size_t slots = static_cast<size_t>(P.nblk) * maxs;
-  p.off_tick = sizeof(WsHeader);
-  p.off_ml = align_up(p.off_tick + static_cast<size_t>(P.U) * 4, 256);
+  p.off_ml = align_up(sizeof(WsHeader), 256);
   p.off_o = align_up(p.off_ml + slots * g * 2 * 4, 256);
   p.total = align_up(p.off_o + slots * g * sh.D * 4, 256);
   return p;
@@ -1012,6 +1042,18 @@ void launch_t(const QArgs& a, const QPlan& p, cudaStream_t s) {
   using C = QCfg<BITS, G, D, NT>;
   quant_occupancy<BITS, G, D, NT>();  // sets the shared-memory attribute once per device
   draft_quant_kernel<BITS, G, D, NT><<<p.P.nblk, kQNW * 32, C::SMEM_B, s>>>(a);
+  CArgs c{};
+  c.P = p.P;
+  c.MAXS = p.MAXS;
+  c.g = a.g;
+  c.Hq = a.Hq;
+  c.Hkv = a.Hkv;
+  c.part_o = a.part_o;
+  c.part_ml = a.part_ml;
+  c.out = a.out;
+  // a unit has at most one partial per block plus one (its residual and quantised parts may share a block)
+  const size_t smem = (2 * static_cast<size_t>(p.P.nblk + 1) + 4 * D + 2) * sizeof(float);
+  combine_kernel<D><<<dim3(static_cast<unsigned>(p.P.U), static_cast<unsigned>(a.g)), 128, smem, s>>>(c);
 }
 
 template <int BITS, int G, int D>
@@ -1093,7 +1135,6 @@ void bind_scratch(QArgs& a, const QPlan& p, void* scratch, float* out) {
   a.P = p.P;
   a.MAXS = p.MAXS;
   a.flags = reinterpret_cast<uint32_t*>(w);
-  a.tickets = reinterpret_cast<uint32_t*>(w + p.off_tick);
   a.part_ml = reinterpret_cast<float*>(w + p.off_ml);
   a.part_o = reinterpret_cast<float*>(w + p.off_o);
   a.out = out;
@@ -1162,7 +1203,7 @@ vc_status vc_debug_quant_partition(const vc_attn_shape* shape, const vc_quant_ca
   *n_blocks = p.P.nblk;
   *max_segments = p.MAXS;
   *n_stages = p.P.S_tot;
-  *n_quant_stages = p.P.QZ;
+  *n_quant_stages = p.P.S_tot - p.P.RZ;
   if (first_stage) {
     VC_REQUIRE(max_blocks >= p.P.nblk + 1, "vc_debug_quant_partition: first_stage needs %d entries",
                p.P.nblk + 1);
@@ -1180,7 +1221,7 @@ vc_status vc_debug_quant_partition(const vc_attn_shape* shape, const vc_quant_ca
 // that runs inside a host framework whose memory pool owns every byte of
 // device memory, or latency-critical paths that must never reach an
 // allocator (cudaMalloc may implicitly synchronise the device).  For them
-// this entry point keeps the split-K scratch (flag word, tickets, partials)
+// this entry point keeps the split-K scratch (flag word, partials)
 // in a file-scope device array of fixed size, VC_NOALLOC_SCRATCH_BYTES, that
 // every GPU which loads the library holds until the process exits.
 //
@@ -1240,7 +1281,7 @@ vc_status vc_draft_attn_quant_noalloc(const vc_attn_shape* shape, const vc_quant
   st = vc::noalloc_scratch(&scratch);
   if (st != VC_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // flag word and tickets must start at zero; partials need no clearing
+  // the flag word must start at zero; partials need no clearing
   if (cudaMemsetAsync(scratch, 0, p.off_ml, s) != cudaSuccess)
     return vc::set_error(VC_ERR_CUDA, "vc_draft_attn_quant_noalloc: clearing the scratch failed: %s",
                          cudaGetErrorString(cudaGetLastError()));

@@ -1,7 +1,7 @@
 """The work partition of vc_draft_attn_quant, checked on the CPU through
 vc_debug_quant_partition (no GPU call): the stages of one call -- every
-(request, head) unit's quantised groups, then every unit's residual rows,
-16 per stage -- are cut into contiguous, non-empty, cost-balanced block
+(request, head) unit's residual rows, 16 per stage, then every unit's
+quantised groups -- are cut into contiguous, non-empty, cost-balanced block
 ranges, and the segment bound the workspace is sized with holds."""
 
 import pytest
@@ -58,11 +58,13 @@ def test_partition_covers_every_stage_once_in_balanced_ranges(Bq, Hq, Hkv, D, L_
     assert 1 <= n <= target
     assert first[0] == 0 and first[n] == p["n_stages"]
     assert all(first[k] < first[k + 1] for k in range(n)), "a block without a stage"
-    # cost of a stage: its bytes (residual stages count double: they are not pipelined)
+    # cost of a stage: its bytes (records), or twice its bytes (16 bf16 K and V
+    # rows, fetched without a pipeline)
     cq, cr = ng_stage * rec, 16 * 4 * D * 2
+    RZ = U * sr
 
     def cost(s):
-        return s * cq if s < U * sq else U * sq * cq + (s - U * sq) * cr
+        return s * cr if s < RZ else RZ * cr + (s - RZ) * cq
 
     total = cost(p["n_stages"])
     for k in range(n):
@@ -70,7 +72,7 @@ def test_partition_covers_every_stage_once_in_balanced_ranges(Bq, Hq, Hkv, D, L_
         assert abs(c - total / n) <= max(cq, cr) + 1, (k, c, total / n)
 
     def seg(s):
-        return s // sq if s < U * sq else U + (s - U * sq) // sr
+        return s // sr if s < RZ else U + (s - RZ) // sq
 
     segs = max(seg(first[k + 1] - 1) - seg(first[k]) + 1 for k in range(n))
     assert p["max_segments"] == segs
