@@ -42,10 +42,21 @@ sys.path.insert(0, ROOT)
 METRIC = "draft-attn HBM GB/s (% of peak); K=30 verify-round µs vs PCIe/HBM roofline"
 
 WORKLOADS = {
-    "llama-3.1-8b-32k-kivi2": dict(NL=32, B=8, Hq=32, Hkv=8, D=128, T=32768, bits=2, G=32, R=128, K=30,
-                                   V=128256, logits="bf16", p_mismatch=0.2),
-    "llama-3.1-8b-1m-500k-kivi2": dict(NL=32, B=1, Hq=32, Hkv=8, D=128, T=500000, bits=2, G=32, R=128, K=30,
-                                       V=128256, logits="bf16", p_mismatch=0.2),
+    # quantised draft cache in HBM, full KV resident in HBM
+    "llama-3.1-8b-32k-kivi2": dict(kind="resident", NL=32, B=8, Hq=32, Hkv=8, D=128, T=32768, bits=2, G=32,
+                                   R=128, K=30, V=128256, logits="bf16", p_mismatch=0.2),
+    # the same shapes at 500K context; verification runs resident and host-streamed
+    "llama-3.1-8b-1m-500k-kivi2": dict(kind="resident", streamed_too=True, NL=32, B=1, Hq=32, Hkv=8, D=128,
+                                       T=500000, bits=2, G=32, R=128, K=30, V=128256, logits="bf16",
+                                       p_mismatch=0.2, host_pool=2),
+    # token-dropped draft cache (25% kept per layer-head) in HBM, full KV in pinned host memory
+    "qwen-32b-100k-tokdrop4-streamed": dict(kind="streamed", NL=64, B=1, Hq=40, Hkv=8, D=128, T=100000,
+                                            n_keep=25000, K=30, V=152064, logits="bf16", p_mismatch=0.2,
+                                            host_pool=4),
+    # four requests, 4-bit group-64 draft caches, full KV in pinned host memory, staggered by the scheduler
+    "llama-70b-4x131k-4bit-stagger": dict(kind="stagger", NL=80, B=1, n_req=4, Hq=64, Hkv=8, D=128, T=131072,
+                                          bits=4, G=64, R=128, K=30, V=128256, logits="bf16", p_mismatch=0.2,
+                                          host_pool=2),
 }
 
 
@@ -61,6 +72,63 @@ def draft_bytes_per_layer(w) -> int:
 
 def verify_bytes_per_layer(w) -> int:
     return 4 * w["T"] * w["Hkv"] * w["D"] * w["B"]
+
+
+def sparse_bytes_per_layer(w) -> int:
+    """Algorithmic HBM bytes of one token-dropped draft layer call: the kept
+    bf16 K and V rows plus their int32 indices."""
+    return w["n_keep"] * w["Hkv"] * (4 * w["D"] + 4) * w["B"]
+
+
+def measure_pcie_h2d(dev, nbytes: int = 1 << 30, reps: int = 5) -> float:
+    """Pinned host -> device copy bandwidth (GB/s, best of reps) of one
+    cudaMemcpyAsync of nbytes: the host-link peak the streamed verification
+    is measured against."""
+    import torch
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    st = torch.cuda.Stream(dev)
+    best = 0.0
+    with torch.cuda.stream(st):
+        d.copy_(h, non_blocking=True)
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            d.copy_(h, non_blocking=True)
+            e1.record(st)
+            e1.synchronize()
+            best = max(best, nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del h, d
+    return best
+
+
+def host_pool(w, dev_dtype, n: int):
+    """n distinct pinned host layers of full bf16 K and V [B, Hkv, T, D]; the
+    streamed layers cycle through them (the host link moves every layer's
+    bytes; only the host RAM they come from is shared)."""
+    import torch
+    from lossless_draft_verify_vc_b200 import synth
+    hk, hv = [], []
+    for i in range(n):
+        k, v = synth.kv_full(w["B"], w["Hkv"], w["T"], w["D"], seed=900 + i, device="cuda")
+        hk.append(k.cpu().pin_memory())
+        hv.append(v.cpu().pin_memory())
+        del k, v
+    return hk, hv
+
+
+def streamed_verify_pass(vc, ks, sh, q_ver, T, nq, NL, out_v, ws_v, comp):
+    """One verification pass over NL layers streamed from host memory: the copy
+    of layer l + 2 overlaps the verification of layer l (two staging slots)."""
+    ks.prefetch(0)
+    if NL > 1:
+        ks.prefetch(1)
+    for l in range(NL):
+        kp, vp = ks.acquire(l, comp)
+        vc.vc_verify_attn(sh, q_ver[l], kp, vp, T, nq, out_v, None, ws_v, comp)
+        ks.release(l, comp)
+        if l + 2 < NL:
+            ks.prefetch(l + 2)
 
 
 def read_peaks():
@@ -287,6 +355,10 @@ def run_gpu(args, w, rank, world):
            + h_lg.numel() * h_lg.element_size() + h_dt.numel() * h_dt.element_size())
     d2h = h_res.numel() * h_res.element_size()
 
+    streamed = None
+    if w.get("streamed_too"):
+        streamed = time_streamed_verify(args, w, dev, inp, sh, ws_v, out_v, stream)
+
     times = torch.tensor([total_ms, draft_ms, verify_ms, accept_ms, e2e_total_ms, e2e_draft_ms], dtype=torch.float64)
     if world > 1:
         tt = times.to(dev)
@@ -294,7 +366,196 @@ def run_gpu(args, w, rank, world):
         times = tt.cpu()
     total_ms, draft_ms, verify_ms, accept_ms, e2e_total_ms, e2e_draft_ms = times.tolist()
     return dict(total_ms=total_ms, draft_ms=draft_ms, verify_ms=verify_ms, accept_ms=accept_ms,
-                e2e_total_ms=e2e_total_ms, e2e_draft_ms=e2e_draft_ms, h2d=h2d, d2h=d2h, clocks=clk)
+                e2e_total_ms=e2e_total_ms, e2e_draft_ms=e2e_draft_ms, h2d=h2d, d2h=d2h, clocks=clk,
+                streamed=streamed)
+
+
+def time_streamed_verify(args, w, dev, inp, sh, ws_v, out_v, comp):
+    """Verification rounds with every layer's full K and V streamed from
+    pinned host memory (double-buffered staging); returns the round time,
+    the link bytes per second and the measured link peak."""
+    import torch
+    from lossless_draft_verify_vc_b200 import vc
+    NL, T, nq = w["NL"], w["T"], w["K"] + 1
+    pcie = measure_pcie_h2d(dev)
+    hk, hv = host_pool(w, torch.bfloat16, w.get("host_pool", 2))
+    host_k = [hk[l % len(hk)] for l in range(NL)]
+    host_v = [hv[l % len(hv)] for l in range(NL)]
+    stage_k = [torch.empty_like(hk[0], device=dev) for _ in range(2)]
+    stage_v = [torch.empty_like(hv[0], device=dev) for _ in range(2)]
+    copy = torch.cuda.Stream(dev)
+    ks = vc.KvStream(host_k, host_v, stage_k, stage_v, copy)
+    steps = max(1, min(args.steps, 3))
+    for _ in range(1):
+        streamed_verify_pass(vc, ks, sh, inp["q_ver"], T, nq, NL, out_v, ws_v, comp)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    copy.wait_event(e0)
+    for _ in range(steps):
+        streamed_verify_pass(vc, ks, sh, inp["q_ver"], T, nq, NL, out_v, ws_v, comp)
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    ks.close()
+    ms = e0.elapsed_time(e1) / steps
+    link_bytes = 2 * hk[0].numel() * hk[0].element_size() * NL
+    return dict(round_us=ms * 1e3, link_gbps=link_bytes / (ms * 1e-3) / 1e9, pcie_peak_gbps=pcie,
+                rounds=steps, host_pool_layers=len(hk))
+
+
+def run_streamed(args, w, rank, world):
+    """Token-dropped draft over a kept-row pool in HBM, verification streamed
+    per layer from pinned host memory, greedy acceptance."""
+    import torch
+    from lossless_draft_verify_vc_b200 import synth, vc
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    vc.lib()
+    NL, B, Hq, Hkv, D, T, K, V, nk = w["NL"], w["B"], w["Hq"], w["Hkv"], w["D"], w["T"], w["K"], w["V"], w["n_keep"]
+    nq = K + 1
+    seed0 = 1000 * rank
+    sh = vc.shape(B, Hq, Hkv, D)
+    # kept-row pools: the n_keep kept K and V rows of every layer-head, addressed
+    # through index lists (here the pool slots 0..n_keep-1)
+    idx = torch.arange(nk, dtype=torch.int32, device=dev).expand(B, Hkv, nk).contiguous()
+    pools = [synth.kv_full(B, Hkv, nk, D, seed=seed0 + l, device=dev) for l in range(NL)]
+    scs = [vc.sparse_cache(k, v, idx) for k, v in pools]
+    q_draft = synth.normal((K, NL, B, Hq, D), seed0 + 1, dev)
+    q_ver = synth.normal((NL, B, nq, Hq, D), seed0 + 2, dev)
+    draft_tok = synth.tokens((B, K), V, seed0 + 3, dev)
+    lens = synth.geometric_accept_lengths(B, K, w["p_mismatch"], seed0 + 3)
+    logits = synth.planted_logits(B, K, V, draft_tok.cpu(), lens, seed0 + 4, device="cpu",
+                                  dtype=torch.bfloat16).to(dev)
+    ws_d = vc.workspace(vc.vc_draft_attn_sparse_workspace_size(sh, scs[0]), dev)
+    ws_v = vc.workspace(vc.vc_verify_attn_workspace_size(sh, T, nq), dev)
+    ws_a = vc.workspace(vc.vc_accept_workspace_size(B, K, V), dev)
+    out_d = torch.empty(B, Hq, D, device=dev)
+    out_v = torch.empty(B, nq, Hq, D, device=dev)
+    tgt = torch.empty(B, K + 1, dtype=torch.int32, device=dev)
+    acc = torch.empty(B, dtype=torch.int32, device=dev)
+    cor = torch.empty(B, dtype=torch.int32, device=dev)
+    pcie = measure_pcie_h2d(dev)
+    hk, hv = host_pool(w, torch.bfloat16, w["host_pool"])
+    host_k = [hk[l % len(hk)] for l in range(NL)]
+    host_v = [hv[l % len(hv)] for l in range(NL)]
+    stage_k = [torch.empty_like(hk[0], device=dev) for _ in range(2)]
+    stage_v = [torch.empty_like(hv[0], device=dev) for _ in range(2)]
+    comp = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+    ks = vc.KvStream(host_k, host_v, stage_k, stage_v, copy)
+
+    def step(ev=None):
+        if ev: ev[0].record(comp)
+        for t in range(K):
+            for l in range(NL):
+                vc.vc_draft_attn_sparse(sh, scs[l], q_draft[t, l], out_d, ws_d, comp)
+        if ev:
+            ev[1].record(comp)
+            copy.wait_event(ev[1])  # the timed verification starts its copies here
+        streamed_verify_pass(vc, ks, sh, q_ver, T, nq, NL, out_v, ws_v, comp)
+        if ev: ev[2].record(comp)
+        vc.vc_accept(logits, B, K, V, draft_tok, tgt, acc, cor, ws_a, comp)
+        if ev: ev[3].record(comp)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert acc.cpu().tolist() == lens, "acceptance mismatch on the planted logits"
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(comp)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(comp)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ks.close()
+    draft_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    verify_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    accept_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    return dict(total_ms=t0.elapsed_time(t1), draft_ms=draft_ms, verify_ms=verify_ms, accept_ms=accept_ms,
+                clocks=clk, pcie=pcie, link_bytes=2 * hk[0].numel() * hk[0].element_size() * NL,
+                host_pool_layers=len(hk))
+
+
+def run_stagger(args, w, rank, world):
+    """Several requests, each a 4-bit draft over its quantised cache and a
+    host-streamed verification, run by the scheduler in lock-step and in the
+    staggered order; both policies' round times are reported."""
+    import torch
+    from lossless_draft_verify_vc_b200 import synth, vc
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    vc.lib()
+    NL, B, Hq, Hkv, D, T, K, V, n = (w["NL"], w["B"], w["Hq"], w["Hkv"], w["D"], w["T"], w["K"], w["V"],
+                                     w["n_req"])
+    nq = K + 1
+    sh = vc.shape(B, Hq, Hkv, D)
+    pcie = measure_pcie_h2d(dev)
+    hk, hv = host_pool(w, torch.bfloat16, w["host_pool"])
+    copy = torch.cuda.Stream(dev)
+    reqs, keep = [], []
+    for i in range(n):
+        seed0 = 1000 * rank + 100 * i
+        caches = [synth.random_quant_cache(B, Hkv, T - w["R"], w["R"], D, w["bits"], w["G"], seed=seed0 + l,
+                                           device=dev) for l in range(NL)]
+        qcs = [vc.quant_cache(c) for c in caches]
+        q_draft = synth.normal((K, NL, B, Hq, D), seed0 + 1, dev)
+        q_ver = synth.normal((NL, B, nq, Hq, D), seed0 + 2, dev)
+        toks = synth.tokens((B, K), V, seed0 + 3, dev)
+        lens = synth.geometric_accept_lengths(B, K, w["p_mismatch"], seed0 + 3)
+        logits = synth.planted_logits(B, K, V, toks.cpu(), lens, seed0 + 4, device="cpu",
+                                      dtype=torch.bfloat16).to(dev)
+        st_k = [torch.empty_like(hk[0], device=dev) for _ in range(2)]
+        st_v = [torch.empty_like(hv[0], device=dev) for _ in range(2)]
+        out = dict(d=torch.empty(B, Hq, D, device=dev), v=torch.empty(B, nq, Hq, D, device=dev),
+                   t=torch.empty(B, K + 1, dtype=torch.int32, device=dev),
+                   a=torch.empty(B, dtype=torch.int32, device=dev), c=torch.empty(B, dtype=torch.int32, device=dev))
+        dws = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, qcs[0]), dev)
+        vws = vc.workspace(vc.vc_verify_attn_workspace_size(sh, T, nq), dev)
+        aws = vc.workspace(vc.vc_accept_workspace_size(B, K, V), dev)
+        stream = torch.cuda.Stream(dev)
+        reqs.append(vc.make_sched_request(sh, vc.VC_DRAFT_QUANT, qcs, q_draft, out["d"], dws,
+                                          [hk[l % len(hk)] for l in range(NL)], [hv[l % len(hv)] for l in range(NL)],
+                                          st_k, st_v, q_ver, out["v"], vws, T, nq, logits, V, toks, out["t"],
+                                          out["a"], out["c"], aws, stream))
+        keep.append((caches, qcs, out, lens, q_draft))
+    # draft kernel alone (request 0), as in the resident workload
+    qcs0, q_draft0, out0 = keep[0][1], keep[0][4], keep[0][2]["d"]
+    dws0 = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, qcs0[0]), dev)
+    comp = torch.cuda.current_stream(dev)
+    for l in range(NL):
+        vc.vc_draft_attn_quant(sh, qcs0[l], q_draft0[0, l], out0, dws0, comp)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for t in range(K):
+        for l in range(NL):
+            vc.vc_draft_attn_quant(sh, qcs0[l], q_draft0[t, l], out0, dws0, comp)
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    draft_ms = e0.elapsed_time(e1)
+    res = {}
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    for name, pol in (("lockstep", vc.VC_SCHED_LOCKSTEP), ("stagger", vc.VC_SCHED_STAGGER)):
+        sch = vc.Sched(reqs, NL, K, pol, copy, timeout_ms=600000)
+        sch.run_rounds(1)  # warm-up round
+        torch.cuda.synchronize(dev)
+        st = sch.run_rounds(max(1, min(args.steps, 2)))
+        torch.cuda.synchronize(dev)
+        sch.close()
+        for r, (_, _, out, lens, _) in zip(reqs, keep):
+            assert out["a"].cpu().tolist() == lens, "acceptance mismatch under the scheduler"
+        res[name] = st
+    clk = clocks.stop()
+    return dict(draft_ms=draft_ms, sched=res, pcie=pcie, clocks=clk,
+                link_bytes_per_request=2 * hk[0].numel() * hk[0].element_size() * NL, host_pool_layers=len(hk))
 
 
 # ----------------------------------------------------------------------------- oracle leg
@@ -349,11 +610,20 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     peak, peak_kind = read_peaks()
     nq = w["K"] + 1
-    config = {"workload": args.workload, "layers": w["NL"], "requests_per_gpu": w["B"], "context": w["T"],
-              "heads": [w["Hq"], w["Hkv"]], "head_dim": w["D"], "bits": w["bits"], "group": w["G"],
-              "residual": w["R"], "draft_len": w["K"], "verify_rows": nq, "vocab": w["V"],
-              "l2": "inputs larger than L2 (draft cache and full KV are tens of GB; no flush needed)",
+    config = {"workload": args.workload, "layers": w["NL"], "requests_per_gpu": w["B"] * w.get("n_req", 1),
+              "context": w["T"], "heads": [w["Hq"], w["Hkv"]], "head_dim": w["D"], "draft_len": w["K"],
+              "verify_rows": nq, "vocab": w["V"],
+              "l2": "inputs larger than L2 (draft caches and KV are GBs; no flush needed)",
               "parallelism": f"replicas x{args.gpus}"}
+    if "bits" in w:
+        config.update(bits=w["bits"], group=w["G"], residual=w["R"])
+    if "n_keep" in w:
+        config.update(kept_per_head=w["n_keep"], kept_row_pool="idx = pool slots 0..n_keep-1")
+    if w["kind"] != "resident" or w.get("streamed_too"):
+        config.update(full_kv="pinned host memory, streamed per layer",
+                      host_pool_layers=w.get("host_pool", 2))
+    if w["kind"] == "stagger":
+        config.update(requests=w["n_req"])
 
     if args.impl == "reference":
         if rank != 0:
@@ -380,6 +650,85 @@ def main():
         import torch
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if w["kind"] == "streamed":
+        line = streamed_line(args, w, rank, world, config, peak, peak_kind)
+    elif w["kind"] == "stagger":
+        line = stagger_line(args, w, rank, world, config, peak, peak_kind)
+    else:
+        line = resident_line(args, w, rank, world, config, peak, peak_kind)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch
+        torch.distributed.destroy_process_group()
+
+
+def _common(args, config, value, peak, peak_kind, r, dtype):
+    return {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": dtype, "data": "synthetic (seeded random KV, queries and logits; no model weights)",
+            "config": config, "clocks": r["clocks"]}
+
+
+def streamed_line(args, w, rank, world, config, peak, peak_kind):
+    r = run_streamed(args, w, rank, world)
+    K, NL = w["K"], w["NL"]
+    db = sparse_bytes_per_layer(w)
+    value = db * K * NL * args.steps * world / (r["draft_ms"] * 1e-3) / 1e9
+    achieved = db / (r["draft_ms"] * 1e3 / (K * NL * args.steps) * 1e-6) / 1e9
+    vr_us = r["verify_ms"] * 1e3 / args.steps
+    link = r["link_bytes"] / (vr_us * 1e-6) / 1e9
+    line = _common(args, config, value, peak, peak_kind, r, "bf16 rows -> bf16 MMA, fp32 accumulate")
+    line.update({
+        "ms_per_step": r["total_ms"] / args.steps,
+        "draft_frac_of_hbm_peak": value / world / peak,
+        "verify_round_us": vr_us, "verify_link_gbps": link, "pcie_peak_gbps": r["pcie"],
+        "verify_frac_of_pcie_peak": link / r["pcie"], "accept_us": r["accept_ms"] * 1e3 / args.steps,
+        "phases_ms_per_step": {"draft": r["draft_ms"] / args.steps, "verify_streamed": vr_us / 1e3,
+                               "accept": r["accept_ms"] / args.steps},
+        "roofline": {"kernel": "vc_draft_attn_sparse (draft_sparse_kernel)", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)", "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "algorithmic_bytes_per_launch": db},
+        "link_roofline": {"phase": "host-streamed verification", "bound": "pcie", "achieved": link,
+                          "peak": r["pcie"], "peak_kind": "pinned host->device cudaMemcpyAsync of 1 GiB, measured "
+                                                          "in this run", "unit": "GB/s",
+                          "frac": link / r["pcie"], "bytes_per_round": r["link_bytes"]},
+        "gpu_launches": (K * NL + NL + 1) * args.steps,
+    })
+    return line
+
+
+def stagger_line(args, w, rank, world, config, peak, peak_kind):
+    r = run_stagger(args, w, rank, world)
+    K, NL, n = w["K"], w["NL"], w["n_req"]
+    db = draft_bytes_per_layer(w)
+    value = db * K * NL * world / (r["draft_ms"] * 1e-3) / 1e9
+    lk, sg = r["sched"]["lockstep"], r["sched"]["stagger"]
+    per = lambda st: st["elapsed_ms"] / st["rounds"]
+    link_bytes_round = r["link_bytes_per_request"] * n
+    line = _common(args, config, value, peak, peak_kind, r, "int4 codes + bf16 -> fp16/bf16 MMA, fp32 accumulate")
+    line.update({
+        "ms_per_step": per(sg),
+        "draft_frac_of_hbm_peak": value / world / peak,
+        "stagger": {"lockstep_ms_per_round": per(lk), "stagger_ms_per_round": per(sg),
+                    "speedup": per(lk) / per(sg),
+                    "link_busy_frac_stagger": sg["link_busy_ms"] / sg["elapsed_ms"],
+                    "link_busy_frac_lockstep": lk["link_busy_ms"] / lk["elapsed_ms"],
+                    "link_gbps_stagger": link_bytes_round / (per(sg) * 1e-3) / 1e9,
+                    "pcie_peak_gbps": r["pcie"],
+                    "verify_frac_of_pcie_peak_stagger": link_bytes_round / (per(sg) * 1e-3) / 1e9 / r["pcie"],
+                    "rounds": sg["rounds"]},
+        "roofline": {"kernel": "vc_draft_attn_quant (draft_quant_kernel)", "bound": "hbm",
+                     "achieved": db / (r["draft_ms"] * 1e3 / (K * NL) * 1e-6) / 1e9, "peak": peak,
+                     "peak_kind": f"{peak_kind} hbm_gbs (burst copy)", "unit": "GB/s",
+                     "frac": db / (r["draft_ms"] * 1e3 / (K * NL) * 1e-6) / 1e9 / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": db},
+        "gpu_launches": 2 * K * NL,
+    })
+    return line
+
+
+def resident_line(args, w, rank, world, config, peak, peak_kind):
     r = run_gpu(args, w, rank, world)
     K, NL = w["K"], w["NL"]
     db = draft_bytes_per_layer(w)
@@ -410,19 +759,21 @@ def main():
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "note": "draft phase timed with its queries copied from pinned host memory; every step also "
                         "copies verify queries, logits and draft tokens in and reads target/accept/correction out"},
-        "gpu_launches": (K * NL + NL + 1) * args.steps,
+        "gpu_launches": (2 * K * NL + NL + 1) * args.steps,
         "clocks": r["clocks"],
     }
+    if r.get("streamed"):
+        sv = r["streamed"]
+        line["verify_streamed"] = {"round_us": sv["round_us"], "link_gbps": sv["link_gbps"],
+                                   "pcie_peak_gbps": sv["pcie_peak_gbps"],
+                                   "frac_of_pcie_peak": sv["link_gbps"] / sv["pcie_peak_gbps"],
+                                   "rounds": sv["rounds"], "host_pool_layers": sv["host_pool_layers"]}
     if rank == 0 and world == 1:
         gbs, n, el, threads, per_slice = oracle_sample(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                                 "sample": f"{n} x (request 0, KV head 0) of one layer ({per_slice} bytes each) "
                                           f"in {el:.1f} s"}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch
-        torch.distributed.destroy_process_group()
+    return line
 
 
 if __name__ == "__main__":
