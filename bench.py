@@ -150,7 +150,6 @@ def kernel_source_hash(files) -> str:
 
 
 DRAFT_SOURCES = ["lossless_draft_verify_vc_b200/csrc/vc_draft_quant.cu",
-                 "lossless_draft_verify_vc_b200/csrc/vc_splitk.cuh",
                  "lossless_draft_verify_vc_b200/csrc/vc_common.cuh"]
 
 
