@@ -215,14 +215,13 @@ struct IssuePtr {
   }
 };
 
-// One bulk copy of this warp's quantised stage number i (at ip) into its ring slot.
+// One bulk copy of this warp's next quantised stage (at ip) into ring slot `slot`.
 template <typename C>
-__device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring, uint64_t* bars, int lane, int i,
+__device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring, uint64_t* bars, int lane, int slot,
                                             const IssuePtr& ip) {
   const int64_t g0 = static_cast<int64_t>(ip.ls) * C::NG;
   const int64_t left = a.P.ng - g0;
   const uint32_t bytes = static_cast<uint32_t>((left < C::NG ? left : C::NG) * C::REC);
-  const int slot = i % C::NST;
   if (lane == 0) {
     mbar_arrive_expect_tx(&bars[slot], bytes);
     bulk_g2s(ring + slot * C::STAGE, a.rec + (static_cast<int64_t>(ip.u) * a.P.ng + g0) * C::REC, bytes,
@@ -235,7 +234,8 @@ __device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring,
 // pipeline runs on across segments) and leaves the warp's state in its slot.
 template <int BITS, int G, int D, int NT>
 __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, int u, int64_t qs0, int my_nq,
-                          int& iq, int& issued, IssuePtr& ip, bool& ok, float* st_o, float* st_ml) {
+                          int& iq, int& issued, IssuePtr& ip, int& islot, int& cslot, uint32_t& cphase, bool& ok,
+                          float* st_o, float* st_ml) {
   using C = QCfg<BITS, G, D, NT>;
   using F = Frag<BITS>;
   constexpr unsigned FULL = 0xffffffffu;
@@ -304,12 +304,16 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
     if (issued < my_nq && issued <= iq + C::NST - 1) {
       fence_proxy_async_smem();
       __syncwarp();
-      issue_stage<C>(a, ring, bars, lane, issued, ip);
+      issue_stage<C>(a, ring, bars, lane, islot, ip);
       ip.advance(a.P);
       ++issued;
+      islot = islot + 1 == C::NST ? 0 : islot + 1;
     }
-    const int slot = iq % C::NST;
-    if (!__all_sync(FULL, mbar_wait_bounded(&bars[slot], (iq / C::NST) & 1, a.flags))) {  // warp-uniform
+    const int slot = cslot;  // = iq mod NST, with phase cphase = (iq / NST) mod 2
+    cslot = cslot + 1 == C::NST ? 0 : cslot + 1;
+    const uint32_t phase = cphase;
+    cphase ^= cslot == 0 ? 1u : 0u;
+    if (!__all_sync(FULL, mbar_wait_bounded(&bars[slot], phase, a.flags))) {  // warp-uniform
       ok = false;
       for (int k = iq; k < issued; ++k) mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
       continue;
@@ -317,7 +321,7 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
     const int64_t g0 = static_cast<int64_t>(ls0 + kk * kQNW) * C::NG;
     const int n_here = a.P.ng - g0 < C::NG ? static_cast<int>(a.P.ng - g0) : C::NG;
 #pragma unroll 1
-    for (int gi = 0; gi < n_here; ++gi) {
+    for (int gi = 0; gi < (C::NG == 1 ? 1 : n_here); ++gi) {
       const unsigned char* rs = ring + slot * C::STAGE + gi * C::REC;
       const uint32_t* kcw = reinterpret_cast<const uint32_t*>(rs);
       const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
@@ -714,7 +718,7 @@ struct UnitPartials {
 // Block-wide: merges the kQNW warp states of segment `seg` (local index j of
 // block k) into the block's partial of that segment.
 template <int D, int HEADS>
-__device__ __noinline__ void merge_segment(const QArgs& a, int k, int j, const float* st_o, const float* st_ml,
+__device__ __forceinline__ void merge_segment(const QArgs& a, int k, int j, const float* st_o, const float* st_ml,
                                            float* mw) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int g = a.g;
@@ -767,6 +771,9 @@ struct CArgs {
 template <int D>
 __global__ void __launch_bounds__(128) combine_kernel(CArgs a) {
   extern __shared__ __align__(16) float csm[];  // [np][2] (m, l), then [4][D] warp sums, then [2] (M, L)
+  // launched as a programmatic dependent of draft_quant_kernel: wait until that
+  // grid has completed and its partials are visible
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int u = blockIdx.x, r = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = a.g;
@@ -851,6 +858,9 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x;
   const Partition& P = a.P;
+  // let the combine grid be scheduled as this grid's blocks retire (it waits
+  // for this grid's completion before reading anything)
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int64_t B0 = P.first(k), B1 = P.first(k + 1);
   if (B0 >= B1) return;  // the host sizes the grid so that this never happens
   const int seg0 = P.seg_of(B0), seg1 = P.seg_of(B1 - 1);
@@ -871,7 +881,8 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
   fence_mbar_init();
   __syncwarp();
   bool ok = true, primed = false;
-  int iq = 0, issued = 0, rph = 0;
+  int iq = 0, issued = 0, rph = 0, islot = 0, cslot = 0;
+  uint32_t cphase = 0;
   IssuePtr ip;
   for (int seg = seg0; seg <= seg1; ++seg) {
     if (seg >= P.U) {
@@ -881,12 +892,14 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
         __syncwarp();
         if (my_nq > 0) ip.start(P, sQ0 - P.RZ);
         while (issued < my_nq && issued < C::NST - 1) {
-          issue_stage<C>(a, ring, bars, lane, issued, ip);
+          issue_stage<C>(a, ring, bars, lane, islot, ip);
           ip.advance(P);
           ++issued;
+          islot = islot + 1 == C::NST ? 0 : islot + 1;
         }
       }
-      quant_seg<BITS, G, D, NT>(a, ring, bars, seg - P.U, sQ0 - P.RZ, my_nq, iq, issued, ip, ok, st_o, st_ml);
+      quant_seg<BITS, G, D, NT>(a, ring, bars, seg - P.U, sQ0 - P.RZ, my_nq, iq, issued, ip, islot, cslot, cphase,
+                                ok, st_o, st_ml);
     } else {
       const int64_t sb = P.seg_begin(seg), se = P.seg_end(seg);
       const int64_t lo = sb > B0 ? sb : B0;
@@ -1053,7 +1066,17 @@ void launch_t(const QArgs& a, const QPlan& p, cudaStream_t s) {
   c.out = a.out;
   // a unit has at most one partial per block plus one (its residual and quantised parts may share a block)
   const size_t smem = (2 * static_cast<size_t>(p.P.nblk + 1) + 4 * D + 2) * sizeof(float);
-  combine_kernel<D><<<dim3(static_cast<unsigned>(p.P.U), static_cast<unsigned>(a.g)), 128, smem, s>>>(c);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.P.U), static_cast<unsigned>(a.g));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, combine_kernel<D>, c);
 }
 
 template <int BITS, int G, int D>

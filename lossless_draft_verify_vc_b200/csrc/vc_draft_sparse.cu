@@ -6,7 +6,8 @@
 // menfem.com, "Key Contributions"); a dropping compressor is described by its
 // kept positions, with equal counts per layer and head ("Limitations").
 //
-// Design (sm_100a, HBM-bound): grid (S chunks, B * Hkv).  A block owns CH
+// Design (sm_100a, HBM-bound): grid (S chunks, B * Hkv), one wave of the
+// resident blocks (plan_sparse).  A block owns CH
 // consecutive kept positions of one (request, KV head); its warps take
 // 16-row tiles round-robin.  Each warp gathers its tile's K and V rows with
 // one 1-D bulk copy per row (lane l copies K row l, lane 16 + l V row l) into
@@ -55,6 +56,9 @@ struct SpArgs {
 template <int D>
 __global__ void __launch_bounds__(kSpNW * 32) draft_sparse_kernel(SpArgs a) {
   using C = SpCfg<D>;
+  // the chunk-merge launch that follows may be scheduled as this grid's blocks
+  // retire; it waits for this grid's completion before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   extern __shared__ __align__(128) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -239,26 +243,64 @@ __global__ void __launch_bounds__(kSpNW * 32) draft_sparse_kernel(SpArgs a) {
   }
   __syncthreads();
   const int hq0 = b * a.Hq + h * a.g;
-  splitk_finish<D>(
+  splitk_store<D>(
       reinterpret_cast<const float*>(smem), C::WARP_B / 4, wst_ml, kSpNW, a.g, a.g, a.S, chunk, unit, a.o,
       [&](int r) { return static_cast<size_t>(hq0 + r) * D; }, [&](int r) { return static_cast<size_t>(hq0 + r); },
       smem_w);
 }
+
+// Output row of flattened partial row fr = unit * g + r (query head h * g + r).
+struct SparseRowMap {
+  int g, Hq, Hkv, D;
+  __device__ bool locate(int64_t fr, int& unit, int& r, size_t& out_off, size_t& lse_off) const {
+    unit = static_cast<int>(fr / g);
+    r = static_cast<int>(fr - static_cast<int64_t>(unit) * g);
+    const int b = unit / Hkv, h = unit - b * Hkv;
+    out_off = (static_cast<size_t>(b) * Hq + h * g + r) * D;
+    lse_off = 0;
+    return true;
+  }
+};
 
 struct SpPlan {
   int S, CH;
   size_t off_tick, off_ml, off_o, total;
 };
 
+// Resident blocks per SM of one instance (cached per device; also sets the
+// kernel's shared-memory attribute on that device).
+template <int D>
+int sparse_occupancy() {
+  using C = SpCfg<D>;
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    cudaFuncSetAttribute(draft_sparse_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, draft_sparse_kernel<D>, kSpNW * 32, C::SMEM_B) !=
+            cudaSuccess ||
+        n < 1)
+      n = 1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Chunks of CH kept rows per block, sized so that the grid is one wave of
+// the resident blocks (SMs x occupancy).
 SpPlan plan_sparse(const vc_attn_shape& sh, int n_keep) {
   SpPlan p{};
   const int units = sh.B * sh.Hkv;
   const int64_t rows = static_cast<int64_t>(units) * n_keep;
-  const int64_t target_blocks = static_cast<int64_t>(sm_count()) * 4;
+  const int occ = sh.D == 128 ? sparse_occupancy<128>() : sparse_occupancy<64>();
+  const int64_t target_blocks = static_cast<int64_t>(sm_count()) * occ;
+  // smallest multiple of 16 rows that keeps units * ceil(n_keep / ch) <= target_blocks
   int64_t ch = (rows + target_blocks - 1) / target_blocks;
-  ch = (ch + 63) / 64 * 64;
+  ch = (ch + 15) / 16 * 16;
   if (ch < 64) ch = 64;
-  if (ch > 2048) ch = 2048;
+  while (units * ((n_keep + ch - 1) / ch) > target_blocks && ch < n_keep) ch += 16;
   p.CH = static_cast<int>(ch);
   p.S = static_cast<int>((n_keep + p.CH - 1) / p.CH);
   const int g = sh.Hq / sh.Hkv;
@@ -340,21 +382,19 @@ vc_status vc_draft_attn_sparse(const vc_attn_shape* shape, const vc_sparse_cache
   dim3 grid(pl.S, shape->B * shape->Hkv);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (shape->D == 128) {
-    using C = vc::SpCfg<128>;
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(vc::draft_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
-      attr = true;
-    }
-    vc::draft_sparse_kernel<128><<<grid, vc::kSpNW * 32, C::SMEM_B, s>>>(a);
+    vc::sparse_occupancy<128>();  // sets the shared-memory attribute once per device
+    vc::draft_sparse_kernel<128><<<grid, vc::kSpNW * 32, vc::SpCfg<128>::SMEM_B, s>>>(a);
   } else {
-    using C = vc::SpCfg<64>;
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(vc::draft_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
-      attr = true;
-    }
-    vc::draft_sparse_kernel<64><<<grid, vc::kSpNW * 32, C::SMEM_B, s>>>(a);
+    vc::sparse_occupancy<64>();
+    vc::draft_sparse_kernel<64><<<grid, vc::kSpNW * 32, vc::SpCfg<64>::SMEM_B, s>>>(a);
+  }
+  if (pl.S > 1) {  // chunk partials -> output rows
+    const vc::SparseRowMap map{a.g, shape->Hq, shape->Hkv, shape->D};
+    const int64_t n_rows = static_cast<int64_t>(shape->B) * shape->Hkv * a.g;
+    if (shape->D == 128)
+      vc::launch_splitk_combine<128>(a.o, pl.S, a.g, n_rows, map, s);
+    else
+      vc::launch_splitk_combine<64>(a.o, pl.S, a.g, n_rows, map, s);
   }
   return vc::launch_status("vc_draft_attn_sparse");
 }

@@ -1,7 +1,8 @@
 // vc_splitk.cuh -- split-K bookkeeping shared by the attention kernels: the
-// in-block merge of per-warp online-softmax states and the cross-block merge
-// of per-chunk partials (the last block of a unit, found with an atomic
-// ticket, merges; nobody waits).
+// in-block merge of per-warp online-softmax states into a per-chunk partial
+// (splitk_store), and the cross-chunk merge, either by the last block of a
+// unit found with an atomic ticket (splitk_finish) or by a separate launch
+// with one warp per output row (splitk_combine_kernel).
 //
 // A partial of one (unit, chunk) holds, per query row r < rows:
 //   o[r][0..D)  unnormalised sum_j 2^(s_j - m) v_j
@@ -117,6 +118,132 @@ __device__ void splitk_finish(const float* wst_o, int o_wstride, const float* ws
   if (o.lse)
     for (int r = tid; r < rows; r += nthr) o.lse[row_lse(r)] = lse_from(smem_w[2 * r], smem_w[2 * r + 1]);
   if (tid == 0) o.tickets[unit] = 0;
+}
+
+// Block-wide: merges the per-warp states of one (unit, chunk) like
+// splitk_finish, but only stores: with S == 1 the normalised output rows,
+// otherwise the chunk's partial, which splitk_combine_kernel merges later.
+template <int D, typename RowOff, typename RowLse>
+__device__ void splitk_store(const float* wst_o, int o_wstride, const float* wst_ml, int nw, int rows, int rows_cap,
+                             int S, int chunk, int unit, const SplitKOut& o, RowOff row_out, RowLse row_lse,
+                             float* smem_w) {
+  const int tid = threadIdx.x;
+  const int nthr = blockDim.x;
+  for (int r = tid; r < rows; r += nthr) {
+    float M = -INFINITY;
+    for (int w = 0; w < nw; ++w) M = fmaxf(M, wst_ml[(w * rows + r) * 2]);
+    float L = 0.f;
+    for (int w = 0; w < nw; ++w) {
+      const float mw = wst_ml[(w * rows + r) * 2];
+      const float sc = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+      smem_w[w * rows + r] = sc;
+      L += sc * wst_ml[(w * rows + r) * 2 + 1];
+    }
+    smem_w[nw * rows + 2 * r] = M;
+    smem_w[nw * rows + 2 * r + 1] = L;
+  }
+  __syncthreads();
+  const int total = rows * D;
+  if (S == 1) {
+    for (int e = tid; e < total; e += nthr) {
+      const int r = e / D, d = e - r * D;
+      float acc = 0.f;
+      for (int w = 0; w < nw; ++w) acc += smem_w[w * rows + r] * wst_o[w * o_wstride + r * D + d];
+      const float L = smem_w[nw * rows + 2 * r + 1];
+      o.out[row_out(r) + d] = L > 0.f ? acc / L : 0.f;
+    }
+    if (o.lse)
+      for (int r = tid; r < rows; r += nthr)
+        o.lse[row_lse(r)] = lse_from(smem_w[nw * rows + 2 * r], smem_w[nw * rows + 2 * r + 1]);
+    return;
+  }
+  float* po = o.part_o + (static_cast<size_t>(unit) * S + chunk) * rows_cap * D;
+  float* pml = o.part_ml + (static_cast<size_t>(unit) * S + chunk) * rows_cap * 2;
+  for (int e = tid; e < total; e += nthr) {
+    const int r = e / D, d = e - r * D;
+    float acc = 0.f;
+    for (int w = 0; w < nw; ++w) acc += smem_w[w * rows + r] * wst_o[w * o_wstride + r * D + d];
+    po[e] = acc;
+  }
+  for (int r = tid; r < rows; r += nthr) {
+    pml[2 * r] = smem_w[nw * rows + 2 * r];
+    pml[2 * r + 1] = smem_w[nw * rows + 2 * r + 1];
+  }
+}
+
+// Cross-chunk merge as its own launch: warp w of block b merges row
+// (b * 4 + w) of the flattened (unit, row) list over the S chunk partials.
+// Each lane owns D/32 consecutive channels; the S (m, l) pairs are reduced by
+// warp shuffles; the S partial loads of a lane are independent.  Map gives,
+// for a flattened row, its unit, its row inside the unit's partials, whether
+// it exists, and its output / lse element offsets.  Launched as a
+// programmatic dependent of the attention kernel: it waits for that grid.
+template <int D, typename Map>
+__global__ void __launch_bounds__(128) splitk_combine_kernel(SplitKOut o, int S, int rows_cap, int64_t n_rows,
+                                                             Map map) {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t fr = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  if (fr >= n_rows) return;
+  int unit, r;
+  size_t out_off, lse_off;
+  if (!map.locate(fr, unit, r, out_off, lse_off)) return;
+  const float* pml = o.part_ml + static_cast<size_t>(unit) * S * rows_cap * 2 + 2 * r;
+  float M = -INFINITY;
+  for (int s = lane; s < S; s += 32) M = fmaxf(M, pml[static_cast<size_t>(s) * rows_cap * 2]);
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
+  float L = 0.f;
+  for (int s = lane; s < S; s += 32) {
+    const float ms = pml[static_cast<size_t>(s) * rows_cap * 2];
+    if (ms != -INFINITY) L += ex2(ms - M) * pml[static_cast<size_t>(s) * rows_cap * 2 + 1];
+  }
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
+  constexpr int PER = D / 32;
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  const float* po = o.part_o + (static_cast<size_t>(unit) * S * rows_cap + r) * D + lane * PER;
+#pragma unroll 4
+  for (int s = 0; s < S; ++s) {
+    const float ms = pml[static_cast<size_t>(s) * rows_cap * 2];
+    const float w = ms == -INFINITY ? 0.f : ex2(ms - M);
+    const float* src = po + static_cast<size_t>(s) * rows_cap * D;
+    if constexpr (PER == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      acc[0] += w * v.x, acc[1] += w * v.y, acc[2] += w * v.z, acc[3] += w * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      acc[0] += w * v.x, acc[1] += w * v.y;
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  float* dst = o.out + out_off + lane * PER;
+  if constexpr (PER == 4) {
+    *reinterpret_cast<float4*>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  } else {
+    *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+  }
+  if (o.lse && lane == 0) o.lse[lse_off] = lse_from(M, L);
+}
+
+// Host: launches splitk_combine_kernel<D> as a programmatic dependent of the
+// kernel just enqueued on s.
+template <int D, typename Map>
+inline void launch_splitk_combine(const SplitKOut& o, int S, int rows_cap, int64_t n_rows, const Map& map,
+                                  cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((n_rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, splitk_combine_kernel<D, Map>, o, S, rows_cap, n_rows, map);
 }
 
 }  // namespace vc

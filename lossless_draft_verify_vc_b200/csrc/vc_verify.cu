@@ -68,6 +68,9 @@ template <int D>
 __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                            const __grid_constant__ CUtensorMap tm_v, VArgs a) {
   using C = VCfg<D>;
+  // the chunk-merge launch that follows may be scheduled as this grid's blocks
+  // retire; it waits for this grid's completion before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_s = smem + C::Q_OFF;
@@ -310,13 +313,34 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
   const int g = a.g;
   const int nq = a.nq;
   const int Hq = a.Hq;
-  splitk_finish<D>(
+  splitk_store<D>(
       wst_o, 0, wst_ml, 1, M, a.nqt * a.g, a.C, chunk, unit * a.RT + rt, a.o,
       [&](int rr) {
         return ((static_cast<size_t>(b) * nq + i0 + rr / g) * Hq + hq0 + rr % g) * D;
       },
       [&](int rr) { return (static_cast<size_t>(b) * nq + i0 + rr / g) * Hq + hq0 + rr % g; }, smem_w);
 }
+
+// Output row of flattened partial row fr = ((unit * RT + rt) * rows_cap + r),
+// for splitk_combine_kernel: row r of row tile rt is query i = rt * nqt + r / g
+// of head h * g + r % g.
+struct VerifyRowMap {
+  int rows_cap, RT, Hkv, nq, nqt, g, Hq, D;
+  __device__ bool locate(int64_t fr, int& unit_rt, int& r, size_t& out_off, size_t& lse_off) const {
+    const int64_t uu = fr / rows_cap;
+    r = static_cast<int>(fr - uu * rows_cap);
+    const int rt = static_cast<int>(uu % RT);
+    const int64_t unit = uu / RT;
+    const int i = rt * nqt + r / g;
+    if (r / g >= nqt || i >= nq) return false;
+    const int b = static_cast<int>(unit / Hkv), h = static_cast<int>(unit % Hkv);
+    const size_t row = (static_cast<size_t>(b) * nq + i) * Hq + h * g + r % g;
+    out_off = row * D;
+    lse_off = row;
+    unit_rt = static_cast<int>(uu);
+    return true;
+  }
+};
 
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -349,6 +373,30 @@ struct VPlan {
   size_t off_tick, off_ml, off_o, total;
 };
 
+// Resident blocks per SM of one instance (cached per device; also sets the
+// kernel's shared-memory attribute on that device).
+template <int D>
+int verify_occupancy() {
+  using C = VCfg<D>;
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    cudaFuncSetAttribute(verify_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, verify_kernel<D>, kVThreads, C::SMEM_B) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Split of the context into C chunks per (unit, row tile): the C that
+// minimises waves x (tiles per chunk + 2), where a wave is SMs x resident
+// blocks and the 2 stands for a block's fixed cost (its query load, pipeline
+// fill and partial write).
 VPlan plan_verify(const vc_attn_shape& sh, int64_t T, int nq) {
   VPlan p{};
   const int g = sh.Hq / sh.Hkv;
@@ -357,10 +405,18 @@ VPlan plan_verify(const vc_attn_shape& sh, int64_t T, int nq) {
   p.RT = (nq + p.nqt - 1) / p.nqt;
   const int units = sh.B * sh.Hkv;
   const int64_t tiles = (T + kVBN - 1) / kVBN;
-  const int64_t slots = 2LL * sm_count();
-  int64_t c = slots / (static_cast<int64_t>(units) * p.RT);
-  if (c < 1) c = 1;
-  if (c > tiles) c = tiles;
+  const int occ = sh.D == 128 ? verify_occupancy<128>() : verify_occupancy<64>();
+  const int64_t slots = static_cast<int64_t>(occ) * sm_count();
+  const int64_t n = static_cast<int64_t>(units) * p.RT;
+  int64_t c = 1, best = -1;
+  for (int64_t cc = 1; cc <= tiles && cc <= 256; ++cc) {
+    const int64_t waves = (n * cc + slots - 1) / slots;
+    const int64_t cost = waves * ((tiles + cc - 1) / cc + 2);
+    if (best < 0 || cost < best) {
+      best = cost;
+      c = cc;
+    }
+  }
   int64_t tpc = (tiles + c - 1) / c;
   p.tiles_per_chunk = static_cast<int>(tpc);
   p.C = static_cast<int>((tiles + tpc - 1) / tpc);
@@ -430,13 +486,20 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
   dim3 grid(p.C, units, p.RT);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (shape->D == 128) {
-    using C = vc::VCfg<128>;
-    cudaFuncSetAttribute(vc::verify_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
-    vc::verify_kernel<128><<<grid, vc::kVThreads, C::SMEM_B, s>>>(tk, tv, a);
+    vc::verify_occupancy<128>();  // sets the shared-memory attribute once per device
+    vc::verify_kernel<128><<<grid, vc::kVThreads, vc::VCfg<128>::SMEM_B, s>>>(tk, tv, a);
   } else {
-    using C = vc::VCfg<64>;
-    cudaFuncSetAttribute(vc::verify_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
-    vc::verify_kernel<64><<<grid, vc::kVThreads, C::SMEM_B, s>>>(tk, tv, a);
+    vc::verify_occupancy<64>();
+    vc::verify_kernel<64><<<grid, vc::kVThreads, vc::VCfg<64>::SMEM_B, s>>>(tk, tv, a);
+  }
+  if (p.C > 1) {  // chunk partials -> output rows (and lse)
+    const int rows_cap = p.nqt * a.g;
+    const vc::VerifyRowMap map{rows_cap, p.RT, shape->Hkv, nq, p.nqt, a.g, shape->Hq, shape->D};
+    const int64_t n_rows = static_cast<int64_t>(units) * p.RT * rows_cap;
+    if (shape->D == 128)
+      vc::launch_splitk_combine<128>(a.o, p.C, rows_cap, n_rows, map, s);
+    else
+      vc::launch_splitk_combine<64>(a.o, p.C, rows_cap, n_rows, map, s);
   }
   return vc::launch_status("vc_verify_attn");
 }
