@@ -25,7 +25,7 @@ namespace vc {
 namespace {
 
 constexpr int kSpNW = 4;   // warps per block
-constexpr int kSpNST = 3;  // ring stages per warp
+constexpr int kSpNST = 2;  // ring stages per warp (3 blocks per SM)
 
 template <int D>
 struct SpCfg {
