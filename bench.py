@@ -692,7 +692,9 @@ def streamed_line(args, w, rank, world, config, peak, peak_kind):
                           "peak": r["pcie"], "peak_kind": "pinned host->device cudaMemcpyAsync of 1 GiB, measured "
                                                           "in this run", "unit": "GB/s",
                           "frac": link / r["pcie"], "bytes_per_round": r["link_bytes"]},
-        "gpu_launches": (K * NL + NL + 1) * args.steps,
+        # per step: K*NL token-drop draft calls and NL verify calls (each an
+        # attention kernel + its chunk-merge kernel), one accept kernel
+        "gpu_launches": (2 * K * NL + 2 * NL + 1) * args.steps,
     })
     return line
 
@@ -758,7 +760,9 @@ def resident_line(args, w, rank, world, config, peak, peak_kind):
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "note": "draft phase timed with its queries copied from pinned host memory; every step also "
                         "copies verify queries, logits and draft tokens in and reads target/accept/correction out"},
-        "gpu_launches": (2 * K * NL + NL + 1) * args.steps,
+        # per step: K*NL quantised draft calls and NL verify calls (each an
+        # attention kernel + its merge kernel), one accept kernel
+        "gpu_launches": (2 * K * NL + 2 * NL + 1) * args.steps,
         "clocks": r["clocks"],
     }
     if r.get("streamed"):

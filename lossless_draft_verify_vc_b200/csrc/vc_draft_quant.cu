@@ -756,10 +756,10 @@ __device__ __forceinline__ void merge_segment(const QArgs& a, int k, int j, cons
 }
 
 // Merges every unit's block partials into out.  One block of 128 threads per
-// (unit, head r): the (m, l) pairs of the unit's partials are staged in
-// shared memory, a block max / denominator is formed, then each warp sums a
-// quarter of the partials over all D channels (D/32 consecutive channels per
-// lane) and the four sums are added through shared memory.
+// (unit, head r): warp w takes partials w, w + 4, ...; each lane keeps a
+// running online-softmax merge (M, L, D/32 channels) of them, loading a
+// partial's (m, l) and its channel slice together (independent loads, one
+// round trip); the four warp states are then merged through shared memory.
 struct CArgs {
   Partition P;
   int MAXS, g, Hq, Hkv;
@@ -770,7 +770,8 @@ struct CArgs {
 
 template <int D>
 __global__ void __launch_bounds__(128) combine_kernel(CArgs a) {
-  extern __shared__ __align__(16) float csm[];  // [np][2] (m, l), then [4][D] warp sums, then [2] (M, L)
+  __shared__ float wsum[4][D];
+  __shared__ float wml[4][2];
   // launched as a programmatic dependent of draft_quant_kernel: wait until that
   // grid has completed and its partials are visible
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
@@ -780,74 +781,67 @@ __global__ void __launch_bounds__(128) combine_kernel(CArgs a) {
   UnitPartials up;
   up.init(a.P, u);
   const int np = up.total();
-  float* mls = csm;
-  float* wsum = csm + 2 * np;
-  float* ML = wsum + 4 * D;
-  for (int p = tid; p < np; p += 128) {
-    const float2 ml = *reinterpret_cast<const float2*>(a.part_ml + up.slot(a.MAXS, p) * g * 2 + 2 * r);
-    mls[2 * p] = ml.x;
-    mls[2 * p + 1] = ml.y;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    float M = -INFINITY;
-    for (int p = lane; p < np; p += 32) M = fmaxf(M, mls[2 * p]);
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    for (int p = lane; p < np; p += 32) {
-      const float mp = mls[2 * p];
-      L += mp == -INFINITY ? 0.f : ex2(mp - M) * mls[2 * p + 1];
-    }
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) {
-      ML[0] = M;
-      ML[1] = L;
-    }
-  }
-  __syncthreads();
-  const float M = ML[0];
   constexpr int PER = D / 32;  // channels per lane
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  int p = warp;
-  for (; p + 12 < np; p += 16) {  // four partials of this warp in flight
-    float v[4][PER];
-    float w[4];
+  float M = -INFINITY, L = 0.f;
+  for (int p0 = warp; p0 < np; p0 += 8) {  // two partials of this warp per trip
+    float v[2][PER];
+    float2 ml[2];
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const float* src = a.part_o + (up.slot(a.MAXS, p + 4 * q4) * g + r) * D + lane * PER;
-      if constexpr (PER == 4) {
-        const float4 t = *reinterpret_cast<const float4*>(src);
-        v[q4][0] = t.x, v[q4][1] = t.y, v[q4][2] = t.z, v[q4][3] = t.w;
+    for (int t = 0; t < 2; ++t) {
+      const int p = p0 + 4 * t;
+      if (p < np) {
+        const int64_t slot = up.slot(a.MAXS, p);
+        ml[t] = *reinterpret_cast<const float2*>(a.part_ml + slot * g * 2 + 2 * r);
+        const float* src = a.part_o + (slot * g + r) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(src);
+          v[t][0] = x.x, v[t][1] = x.y, v[t][2] = x.z, v[t][3] = x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(src);
+          v[t][0] = x.x, v[t][1] = x.y;
+        }
       } else {
-        const float2 t = *reinterpret_cast<const float2*>(src);
-        v[q4][0] = t.x, v[q4][1] = t.y;
+        ml[t] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) v[t][i] = 0.f;
       }
-      const float mp = mls[2 * (p + 4 * q4)];
-      w[q4] = mp == -INFINITY ? 0.f : ex2(mp - M);
     }
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4)
+    for (int t = 0; t < 2; ++t) {
+      if (ml[t].x == -INFINITY) continue;
+      const float Mn = fmaxf(M, ml[t].x);
+      const float ro = M == -INFINITY ? 0.f : ex2(M - Mn);
+      const float rn = ex2(ml[t].x - Mn);
+      L = L * ro + ml[t].y * rn;
 #pragma unroll
-      for (int i = 0; i < PER; ++i) acc[i] += w[q4] * v[q4][i];
+      for (int i = 0; i < PER; ++i) acc[i] = acc[i] * ro + v[t][i] * rn;
+      M = Mn;
+    }
   }
-  for (; p < np; p += 4) {
-    const float* src = a.part_o + (up.slot(a.MAXS, p) * g + r) * D + lane * PER;
-    const float mp = mls[2 * p];
-    const float w = mp == -INFINITY ? 0.f : ex2(mp - M);
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] += w * src[i];
+  if (lane == 0) {
+    wml[warp][0] = M;
+    wml[warp][1] = L;
   }
 #pragma unroll
-  for (int i = 0; i < PER; ++i) wsum[warp * D + lane * PER + i] = acc[i];
+  for (int i = 0; i < PER; ++i) wsum[warp][lane * PER + i] = acc[i];
   __syncthreads();
+  float Mb = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) Mb = fmaxf(Mb, wml[w][0]);
+  float f[4], Lb = 0.f;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    f[w] = wml[w][0] == -INFINITY ? 0.f : ex2(wml[w][0] - Mb);
+    Lb += f[w] * wml[w][1];
+  }
   const int b = u / a.Hkv, h = u - b * a.Hkv;
   float* o = a.out + (static_cast<size_t>(b) * a.Hq + h * g + r) * D;
-  const float L = ML[1];
   for (int d = tid; d < D; d += 128) {
-    const float t = (wsum[d] + wsum[D + d]) + (wsum[2 * D + d] + wsum[3 * D + d]);
-    o[d] = L > 0.f ? t / L : 0.f;
+    const float t = (f[0] * wsum[0][d] + f[1] * wsum[1][d]) + (f[2] * wsum[2][d] + f[3] * wsum[3][d]);
+    o[d] = Lb > 0.f ? t / Lb : 0.f;
   }
 }
 
@@ -1064,12 +1058,10 @@ void launch_t(const QArgs& a, const QPlan& p, cudaStream_t s) {
   c.part_o = a.part_o;
   c.part_ml = a.part_ml;
   c.out = a.out;
-  // a unit has at most one partial per block plus one (its residual and quantised parts may share a block)
-  const size_t smem = (2 * static_cast<size_t>(p.P.nblk + 1) + 4 * D + 2) * sizeof(float);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.P.U), static_cast<unsigned>(a.g));
   cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
