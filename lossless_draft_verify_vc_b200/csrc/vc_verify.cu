@@ -147,36 +147,38 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
   const int64_t vis_end = a.T - a.nq + i_row + 1;  // keys [0, vis_end) visible to this row
   float m_run = -INFINITY, l_run = 0.f;
 
+  // S = Q K^T of tile i: thread 0, once tile i's K and V have landed
+  auto issue_s = [&](int i) -> bool {
+    const uint32_t ks_addr = smem_addr(st_s + (i & 1) * C::STAGE_B);
+    if (!mbar_wait_bounded(&bar_kv[i & 1], (i >> 1) & 1, a.flags)) return false;
+    tc::fence_after_sync();
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int hf = kk >> 2, ko = (kk & 3) * 32;
+      const uint64_t ad = tc::smem_desc_sw128(q_base + hf * (128 * 128) + ko, 16, 1024);
+      const uint64_t bd = tc::smem_desc_sw128(ks_addr + hf * (kVBN * 128) + ko, 16, 1024);
+      tc::mma_ss(tmem + kColS, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+    }
+    tc::commit(bar_s);
+    return true;
+  };
+
+  bool fail = false;
   if (tid == 0) {
     if (ntiles > 0) issue_tile(0);
     if (ntiles > 1) issue_tile(1);
+    if (ntiles > 0 && !issue_s(0)) fail = true;
   }
 
   // Failure handling: every wait is bounded; a thread that sees a timeout sets
   // its sticky `fail`.  tcgen05.ld / st are warp-collective, so each warp
   // decides them with __any_sync; the loop exits on a block-wide
   // __syncthreads_or, so all threads leave together.
-  bool fail = false;
   constexpr unsigned FULL = 0xffffffffu;
   for (int i = 0; i < ntiles; ++i) {
     const int s = i & 1;
     const uint32_t ks_addr = smem_addr(st_s + s * C::STAGE_B);
     const uint32_t vs_addr = ks_addr + C::KV_B;
-    if (tid == 0 && !fail) {
-      if (!mbar_wait_bounded(&bar_kv[s], (i >> 1) & 1, a.flags)) {
-        fail = true;
-      } else {
-        tc::fence_after_sync();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int hf = kk >> 2, ko = (kk & 3) * 32;
-          const uint64_t ad = tc::smem_desc_sw128(q_base + hf * (128 * 128) + ko, 16, 1024);
-          const uint64_t bd = tc::smem_desc_sw128(ks_addr + hf * (kVBN * 128) + ko, 16, 1024);
-          tc::mma_ss(tmem + kColS, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-        tc::commit(bar_s);
-      }
-    }
     if (!fail && !mbar_wait_bounded(bar_s, i & 1, a.flags)) fail = true;
     tc::fence_after_sync();
     bool wfail = __any_sync(FULL, fail);
@@ -259,7 +261,10 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
         tc::mma_ts(tmem + kColO, tmem + kColPlo + 8 * j, vd, IDESC_PV, 1u);
       }
       tc::commit(bar_pv);
-      if (i + 2 < ntiles) {
+      // feed the tensor pipe the next S right behind this P.V (other TMEM
+      // columns, a stage already loaded); its commit also covers this P.V
+      if (i + 1 < ntiles && !issue_s(i + 1)) fail = true;
+      if (!fail && i + 2 < ntiles) {
         // the stage is free once this tile's MMAs are done
         if (!mbar_wait_bounded(bar_pv, i & 1, a.flags)) {
           fail = true;
