@@ -193,15 +193,24 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
     }
     const int64_t t0 = k_begin + static_cast<int64_t>(i) * kVBN;
     const int64_t lim = min(vis_end, k_end) - t0;  // keys [t0, t0 + lim) are live
+    // raw scores; the scale (> 0) is applied in the exponent's FMA below
     float tmax = -INFINITY;
+    if (__all_sync(FULL, lim >= kVBN)) {  // whole tile visible to the warp's rows: no mask
 #pragma unroll
-    for (int c = 0; c < 2; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) * a.scale_log2 : -INFINITY;
-        sr[c][j] = __float_as_uint(x);
-        tmax = fmaxf(tmax, x);
-      }
+        for (int j = 0; j < 32; ++j) tmax = fmaxf(tmax, __uint_as_float(sr[c][j]));
+    } else {
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
+          sr[c][j] = __float_as_uint(x);
+          tmax = fmaxf(tmax, x);
+        }
+    }
+    tmax *= a.scale_log2;
     // lazy rescale: keep the stale maximum unless the new one exceeds it by > 8
     float m_use = m_run;
     float alpha = 1.f;
@@ -217,8 +226,8 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
     for (int c = 0; c < 2; ++c)
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
-        const float p0 = ex2(__uint_as_float(sr[c][j]) - m_sub);
-        const float p1 = ex2(__uint_as_float(sr[c][j + 1]) - m_sub);
+        const float p0 = ex2(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, -m_sub));
+        const float p1 = ex2(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, -m_sub));
         psum += p0 + p1;
         const uint32_t hw = pack_bf2(p0, p1);
         const float2 hf = unpack_bf2(hw);
