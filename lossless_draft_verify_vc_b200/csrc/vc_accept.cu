@@ -112,7 +112,21 @@ __global__ void __launch_bounds__(kAcceptThreads) accept_kernel(const T* __restr
   const int a = v0 + head;
   const int nvec = (v1 - a) / VEC;
   if (threadIdx.x < head) take(b, to_f32(p[v0 + threadIdx.x]), v0 + threadIdx.x);
-  for (int j = threadIdx.x; j < nvec; j += kAcceptThreads) {
+  // four independent 16-byte loads in flight per thread before they are used
+  // (the comparison rule does not depend on the order values are taken in)
+  int j = threadIdx.x;
+  for (; j + 3 * kAcceptThreads < nvec; j += 4 * kAcceptThreads) {
+    const int b0 = a + j * VEC;
+    const auto x0 = ld_stream(p + b0);
+    const auto x1 = ld_stream(p + b0 + kAcceptThreads * VEC);
+    const auto x2 = ld_stream(p + b0 + 2 * kAcceptThreads * VEC);
+    const auto x3 = ld_stream(p + b0 + 3 * kAcceptThreads * VEC);
+    take_vec<T>(b, x0, b0);
+    take_vec<T>(b, x1, b0 + kAcceptThreads * VEC);
+    take_vec<T>(b, x2, b0 + 2 * kAcceptThreads * VEC);
+    take_vec<T>(b, x3, b0 + 3 * kAcceptThreads * VEC);
+  }
+  for (; j < nvec; j += kAcceptThreads) {
     const int base = a + j * VEC;
     take_vec<T>(b, ld_stream(p + base), base);
   }

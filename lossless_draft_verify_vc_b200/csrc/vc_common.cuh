@@ -36,8 +36,9 @@ inline vc_status launch_status(const char* what) {
   return VC_OK;
 }
 
-// Workspace header: a flag word, then per-unit ticket counters, then
-// kernel-specific partials at WS_PARTIAL_OFFSET-aligned offsets.
+// Workspace header: a flag word (device-side errors, read and cleared by
+// vc_workspace_flags); kernel-specific counters and partials follow at
+// 256-byte-aligned offsets.
 struct WsHeader {
   uint32_t flags;
   uint32_t pad[3];

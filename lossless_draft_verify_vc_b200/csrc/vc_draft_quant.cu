@@ -21,17 +21,17 @@
 // rounding (the oracle dequantises with one fp32 FMA per element).
 //
 // Work layout.  The job is one axis of STAGES: first every (request, KV
-// head) unit's quantised groups, NG consecutive group records per stage,
-// then every unit's bf16 residual, 16 rows per stage.  A persistent grid of
+// head) unit's bf16 residual, 16 rows per stage, then every unit's quantised
+// groups, NG consecutive group records per stage.  A persistent grid of
 // (SMs x resident blocks) blocks cuts that axis into equal-cost contiguous
 // ranges (Partition); inside a block the 4 warps take the range's stages
 // round-robin.  A quantised stage is ONE bulk copy of contiguous records into
 // the warp's private ring (NST stages deep, completed on mbarriers, waits
 // bounded).  Wherever the range crosses from one unit's segment to the next,
 // the block merges its warps' online-softmax states into one partial of that
-// segment; the last block to finish a unit (atomic ticket) merges the unit's
-// partials into the output.  All g query heads of a GQA group share each
-// record (they are the MMA's N columns).
+// segment; a second launch (combine_kernel, one block per (unit, head))
+// merges each unit's partials into the output.  All g query heads of a GQA
+// group share each record (they are the MMA's N columns).
 //
 // MMA arrangement (mma.sync m16n8k16, fp16 x fp16 -> fp32):
 //   scores:  D[token][col] = codes[token][chan] x qfold[chan][col]

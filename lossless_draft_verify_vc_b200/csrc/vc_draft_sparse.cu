@@ -264,7 +264,7 @@ struct SparseRowMap {
 
 struct SpPlan {
   int S, CH;
-  size_t off_tick, off_ml, off_o, total;
+  size_t off_ml, off_o, total;
 };
 
 // Resident blocks per SM of one instance (cached per device; also sets the
@@ -304,8 +304,7 @@ SpPlan plan_sparse(const vc_attn_shape& sh, int n_keep) {
   p.CH = static_cast<int>(ch);
   p.S = static_cast<int>((n_keep + p.CH - 1) / p.CH);
   const int g = sh.Hq / sh.Hkv;
-  p.off_tick = sizeof(WsHeader);
-  p.off_ml = align_up(p.off_tick + static_cast<size_t>(units) * 4, 256);
+  p.off_ml = align_up(sizeof(WsHeader), 256);
   p.off_o = align_up(p.off_ml + static_cast<size_t>(units) * p.S * g * 2 * 4, 256);
   p.total = align_up(p.off_o + static_cast<size_t>(units) * p.S * g * sh.D * 4, 256);
   return p;
@@ -376,7 +375,6 @@ vc_status vc_draft_attn_sparse(const vc_attn_shape* shape, const vc_sparse_cache
   a.flags = reinterpret_cast<uint32_t*>(w);
   a.o.out = out;
   a.o.lse = nullptr;
-  a.o.tickets = reinterpret_cast<uint32_t*>(w + pl.off_tick);
   a.o.part_ml = reinterpret_cast<float*>(w + pl.off_ml);
   a.o.part_o = reinterpret_cast<float*>(w + pl.off_o);
   dim3 grid(pl.S, shape->B * shape->Hkv);

@@ -384,7 +384,7 @@ bool make_kv_map(CUtensorMap* m, const void* base, int64_t T, int D, int units) 
 
 struct VPlan {
   int nqt, RT, C, tiles_per_chunk;
-  size_t off_tick, off_ml, off_o, total;
+  size_t off_ml, off_o, total;
 };
 
 // Resident blocks per SM of one instance (cached per device; also sets the
@@ -436,8 +436,7 @@ VPlan plan_verify(const vc_attn_shape& sh, int64_t T, int nq) {
   p.C = static_cast<int>((tiles + tpc - 1) / tpc);
   const int rows = p.nqt * g;
   const size_t nunit = static_cast<size_t>(units) * p.RT;
-  p.off_tick = sizeof(WsHeader);
-  p.off_ml = align_up(p.off_tick + nunit * 4, 256);
+  p.off_ml = align_up(sizeof(WsHeader), 256);
   p.off_o = align_up(p.off_ml + nunit * p.C * rows * 2 * 4, 256);
   p.total = align_up(p.off_o + nunit * p.C * rows * sh.D * 4, 256);
   return p;
@@ -494,7 +493,6 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
   a.flags = reinterpret_cast<uint32_t*>(w);
   a.o.out = out;
   a.o.lse = lse;
-  a.o.tickets = reinterpret_cast<uint32_t*>(w + p.off_tick);
   a.o.part_ml = reinterpret_cast<float*>(w + p.off_ml);
   a.o.part_o = reinterpret_cast<float*>(w + p.off_o);
   dim3 grid(p.C, units, p.RT);
