@@ -131,6 +131,24 @@ def streamed_verify_pass(vc, ks, sh, q_ver, T, nq, NL, out_v, ws_v, comp):
             ks.prefetch(l + 2)
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of a list of floats over all ranks of the default
+    process group (identity without one): multi-GPU times are the slowest
+    rank's."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist = torch.distributed
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def whole_job_rate(bytes_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput of independent replicas (GB/s): every rank
+    processes the same work per step; the job takes the slowest rank's time."""
+    return bytes_per_rank_step * steps * world / (max_ms * 1e-3) / 1e9
+
+
 def read_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -358,12 +376,8 @@ def run_gpu(args, w, rank, world):
     if w.get("streamed_too"):
         streamed = time_streamed_verify(args, w, dev, inp, sh, ws_v, out_v, stream)
 
-    times = torch.tensor([total_ms, draft_ms, verify_ms, accept_ms, e2e_total_ms, e2e_draft_ms], dtype=torch.float64)
-    if world > 1:
-        tt = times.to(dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        times = tt.cpu()
-    total_ms, draft_ms, verify_ms, accept_ms, e2e_total_ms, e2e_draft_ms = times.tolist()
+    total_ms, draft_ms, verify_ms, accept_ms, e2e_total_ms, e2e_draft_ms = max_over_ranks(
+        [total_ms, draft_ms, verify_ms, accept_ms, e2e_total_ms, e2e_draft_ms], dev)
     return dict(total_ms=total_ms, draft_ms=draft_ms, verify_ms=verify_ms, accept_ms=accept_ms,
                 e2e_total_ms=e2e_total_ms, e2e_draft_ms=e2e_draft_ms, h2d=h2d, d2h=d2h, clocks=clk,
                 streamed=streamed)
@@ -463,6 +477,8 @@ def run_streamed(args, w, rank, world):
     assert acc.cpu().tolist() == lens, "acceptance mismatch on the planted logits"
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     clocks = ClockSampler(dev.index)
+    if world > 1:
+        torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -473,10 +489,10 @@ def run_streamed(args, w, rank, world):
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     ks.close()
-    draft_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    verify_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    accept_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
-    return dict(total_ms=t0.elapsed_time(t1), draft_ms=draft_ms, verify_ms=verify_ms, accept_ms=accept_ms,
+    total_ms, draft_ms, verify_ms, accept_ms = max_over_ranks(
+        [t0.elapsed_time(t1), sum(e[0].elapsed_time(e[1]) for e in evs), sum(e[1].elapsed_time(e[2]) for e in evs),
+         sum(e[2].elapsed_time(e[3]) for e in evs)], dev)
+    return dict(total_ms=total_ms, draft_ms=draft_ms, verify_ms=verify_ms, accept_ms=accept_ms,
                 clocks=clk, pcie=pcie, link_bytes=2 * hk[0].numel() * hk[0].element_size() * NL,
                 host_pool_layers=len(hk))
 
@@ -531,6 +547,8 @@ def run_stagger(args, w, rank, world):
     for l in range(NL):
         vc.vc_draft_attn_quant(sh, qcs0[l], q_draft0[0, l], out0, dws0, comp)
     torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(comp)
     for t in range(K):
@@ -538,7 +556,7 @@ def run_stagger(args, w, rank, world):
             vc.vc_draft_attn_quant(sh, qcs0[l], q_draft0[t, l], out0, dws0, comp)
     e1.record(comp)
     torch.cuda.synchronize(dev)
-    draft_ms = e0.elapsed_time(e1)
+    draft_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
     res = {}
     clocks = ClockSampler(dev.index)
     clocks.start()
@@ -546,9 +564,12 @@ def run_stagger(args, w, rank, world):
         sch = vc.Sched(reqs, NL, K, pol, copy, timeout_ms=600000)
         sch.run_rounds(1)  # warm-up round
         torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
         st = sch.run_rounds(max(1, min(args.steps, 2)))
         torch.cuda.synchronize(dev)
         sch.close()
+        st["elapsed_ms"], st["link_busy_ms"] = max_over_ranks([st["elapsed_ms"], st["link_busy_ms"]], dev)
         for r, (_, _, out, lens, _) in zip(reqs, keep):
             assert out["a"].cpu().tolist() == lens, "acceptance mismatch under the scheduler"
         res[name] = st
@@ -673,7 +694,7 @@ def streamed_line(args, w, rank, world, config, peak, peak_kind):
     r = run_streamed(args, w, rank, world)
     K, NL = w["K"], w["NL"]
     db = sparse_bytes_per_layer(w)
-    value = db * K * NL * args.steps * world / (r["draft_ms"] * 1e-3) / 1e9
+    value = whole_job_rate(db * K * NL, args.steps, world, r["draft_ms"])
     achieved = db / (r["draft_ms"] * 1e3 / (K * NL * args.steps) * 1e-6) / 1e9
     vr_us = r["verify_ms"] * 1e3 / args.steps
     link = r["link_bytes"] / (vr_us * 1e-6) / 1e9
@@ -703,7 +724,7 @@ def stagger_line(args, w, rank, world, config, peak, peak_kind):
     r = run_stagger(args, w, rank, world)
     K, NL, n = w["K"], w["NL"], w["n_req"]
     db = draft_bytes_per_layer(w)
-    value = db * K * NL * world / (r["draft_ms"] * 1e-3) / 1e9
+    value = whole_job_rate(db * K * NL, 1, world, r["draft_ms"])
     lk, sg = r["sched"]["lockstep"], r["sched"]["stagger"]
     per = lambda st: st["elapsed_ms"] / st["rounds"]
     link_bytes_round = r["link_bytes_per_request"] * n
@@ -735,13 +756,13 @@ def resident_line(args, w, rank, world, config, peak, peak_kind):
     db = draft_bytes_per_layer(w)
     vb = verify_bytes_per_layer(w)
     draft_bytes_step = db * K * NL
-    value = draft_bytes_step * args.steps * world / (r["draft_ms"] * 1e-3) / 1e9
+    value = whole_job_rate(draft_bytes_step, args.steps, world, r["draft_ms"])
     launches_draft = K * NL * args.steps
     avg_launch_us = r["draft_ms"] * 1e3 / launches_draft
     achieved = db / (avg_launch_us * 1e-6) / 1e9
     verify_round_us = r["verify_ms"] * 1e3 / args.steps
     verify_gbs = vb * NL / (verify_round_us * 1e-6) / 1e9
-    e2e_value = draft_bytes_step * args.steps * world / (r["e2e_draft_ms"] * 1e-3) / 1e9
+    e2e_value = whole_job_rate(draft_bytes_step, args.steps, world, r["e2e_draft_ms"])
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True,
