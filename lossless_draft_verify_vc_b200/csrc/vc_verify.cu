@@ -15,8 +15,10 @@
 //     swizzled K-major layout;
 //   * K and V tiles of BN = 64 keys stream in through a 2-stage ring of tiled
 //     TMA loads (3-D tensor maps, rows past T read as zeros, no multicast);
-//   * one thread issues tcgen05.mma: S = Q K^T into tensor memory (TMEM);
-//   * each of the 128 threads owns one row: it reads its scores from TMEM,
+//   * a fifth warp issues the TMA loads and tcgen05.mma: S = Q K^T into
+//     tensor memory (TMEM), and P.V; it blocks on the tensor pipe's queue
+//     while the softmax warps work, so no row waits for it;
+//   * each of the 128 softmax threads owns one row: it reads its scores from TMEM,
 //     applies the causal mask (row i sees keys 0 .. T - nq + i), updates an
 //     online softmax with lazy rescaling (O is rescaled only when the running
 //     maximum grows by more than 8 in log2 units), and writes P back to TMEM
@@ -34,7 +36,9 @@ namespace vc {
 namespace {
 
 constexpr int kVBN = 64;        // keys per tile
-constexpr int kVThreads = 128;  // one warpgroup; thread r owns row r
+constexpr int kVThreads = 128;  // softmax warpgroup: thread r owns row r
+constexpr int kVBlock = kVThreads + 32;  // + the issuing warp
+constexpr int kVIssuer = kVThreads;      // its elected thread
 constexpr int kVTmemCols = 256;
 // TMEM column map
 constexpr uint32_t kColS = 0;     // S: kVBN fp32 columns
@@ -65,7 +69,7 @@ struct VArgs {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                            const __grid_constant__ CUtensorMap tm_v, VArgs a) {
   using C = VCfg<D>;
   // the chunk-merge launch that follows may be scheduled as this grid's blocks
@@ -104,7 +108,7 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
   if (warp == 0) tc::alloc(tmem_slot, kVTmemCols);
 
   // ---- Q rows -> shared memory, 128-byte swizzled K-major (zeros past M)
-  {
+  if (tid < kVThreads) {
     const int r = tid;
     const bool valid = r < M;
     const int i = i0 + (valid ? r / a.g : 0);
@@ -123,7 +127,9 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  auto issue_tile = [&](int i) {  // thread 0 only
+  int n_issued = 0, n_landed = 0;  // tiles whose loads were issued / waited (issuer)
+  auto issue_tile = [&](int i) {  // issuer only
+    n_issued = i + 1;
     const int s = i & 1;
     unsigned char* ks = st_s + s * C::STAGE_B;
     unsigned char* vs = ks + C::KV_B;
@@ -147,10 +153,11 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
   const int64_t vis_end = a.T - a.nq + i_row + 1;  // keys [0, vis_end) visible to this row
   float m_run = -INFINITY, l_run = 0.f;
 
-  // S = Q K^T of tile i: thread 0, once tile i's K and V have landed
+  // S = Q K^T of tile i: issuer, once tile i's K and V have landed
   auto issue_s = [&](int i) -> bool {
     const uint32_t ks_addr = smem_addr(st_s + (i & 1) * C::STAGE_B);
     if (!mbar_wait_bounded(&bar_kv[i & 1], (i >> 1) & 1, a.flags)) return false;
+    n_landed = i + 1;
     tc::fence_after_sync();
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
@@ -164,7 +171,8 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
   };
 
   bool fail = false;
-  if (tid == 0) {
+  const bool softmax_thread = tid < kVThreads;
+  if (tid == kVIssuer) {
     if (ntiles > 0) issue_tile(0);
     if (ntiles > 1) issue_tile(1);
     if (ntiles > 0 && !issue_s(0)) fail = true;
@@ -179,85 +187,87 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
     const int s = i & 1;
     const uint32_t ks_addr = smem_addr(st_s + s * C::STAGE_B);
     const uint32_t vs_addr = ks_addr + C::KV_B;
-    if (!fail && !mbar_wait_bounded(bar_s, i & 1, a.flags)) fail = true;
-    tc::fence_after_sync();
-    bool wfail = __any_sync(FULL, fail);
-    uint32_t sr[2][32];
-    if (!wfail) {
-      tc::ld32(tmem + lane_off + kColS, sr[0]);
-      tc::ld32(tmem + lane_off + kColS + 32, sr[1]);
-      tc::wait_ld();
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) sr[0][j] = sr[1][j] = 0u;
-    }
-    const int64_t t0 = k_begin + static_cast<int64_t>(i) * kVBN;
-    const int64_t lim = min(vis_end, k_end) - t0;  // keys [t0, t0 + lim) are live
-    // raw scores; the scale (> 0) is applied in the exponent's FMA below
-    float tmax = -INFINITY;
-    if (__all_sync(FULL, lim >= kVBN)) {  // whole tile visible to the warp's rows: no mask
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) tmax = fmaxf(tmax, __uint_as_float(sr[c][j]));
-    } else {
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
-          sr[c][j] = __float_as_uint(x);
-          tmax = fmaxf(tmax, x);
-        }
-    }
-    tmax *= a.scale_log2;
-    // lazy rescale: keep the stale maximum unless the new one exceeds it by > 8
-    float m_use = m_run;
-    float alpha = 1.f;
-    if (tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY)) {
-      m_use = tmax;
-      if (m_run != -INFINITY) alpha = ex2(m_run - m_use);
-      m_run = m_use;
-    }
-    const float m_sub = m_use == -INFINITY ? 0.f : m_use;
-    uint32_t phi[32], plo[32];
-    float psum = 0.f;
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float p0 = ex2(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, -m_sub));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, -m_sub));
-        psum += p0 + p1;
-        const uint32_t hw = pack_bf2(p0, p1);
-        const float2 hf = unpack_bf2(hw);
-        phi[c * 16 + j / 2] = hw;
-        plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
-      }
-    l_run = l_run * alpha + psum;
-    // the previous P.V must be done before P is overwritten / O is touched
-    if (i > 0 && !fail && !mbar_wait_bounded(bar_pv, (i - 1) & 1, a.flags)) fail = true;
-    tc::fence_after_sync();
-    wfail = __any_sync(FULL, fail);
-    if (!wfail && __any_sync(FULL, alpha != 1.f)) {  // warp-uniform: lanes without a new max scale by 1
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tc::ld32(tmem + lane_off + kColO + c0, o);
+    if (softmax_thread) {  // warp-uniform: warps 0-3
+      if (!fail && !mbar_wait_bounded(bar_s, i & 1, a.flags)) fail = true;
+      tc::fence_after_sync();
+      bool wfail = __any_sync(FULL, fail);
+      uint32_t sr[2][32];
+      if (!wfail) {
+        tc::ld32(tmem + lane_off + kColS, sr[0]);
+        tc::ld32(tmem + lane_off + kColS + 32, sr[1]);
         tc::wait_ld();
+      } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-        tc::st32(tmem + lane_off + kColO + c0, o);
+        for (int j = 0; j < 32; ++j) sr[0][j] = sr[1][j] = 0u;
       }
+      const int64_t t0 = k_begin + static_cast<int64_t>(i) * kVBN;
+      const int64_t lim = min(vis_end, k_end) - t0;  // keys [t0, t0 + lim) are live
+      // raw scores; the scale (> 0) is applied in the exponent's FMA below
+      float tmax = -INFINITY;
+      if (__all_sync(FULL, lim >= kVBN)) {  // whole tile visible to the warp's rows: no mask
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tmax = fmaxf(tmax, __uint_as_float(sr[c][j]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
+            sr[c][j] = __float_as_uint(x);
+            tmax = fmaxf(tmax, x);
+          }
+      }
+      tmax *= a.scale_log2;
+      // lazy rescale: keep the stale maximum unless the new one exceeds it by > 8
+      float m_use = m_run;
+      float alpha = 1.f;
+      if (tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY)) {
+        m_use = tmax;
+        if (m_run != -INFINITY) alpha = ex2(m_run - m_use);
+        m_run = m_use;
+      }
+      const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+      uint32_t phi[32], plo[32];
+      float psum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, -m_sub));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, -m_sub));
+          psum += p0 + p1;
+          const uint32_t hw = pack_bf2(p0, p1);
+          const float2 hf = unpack_bf2(hw);
+          phi[c * 16 + j / 2] = hw;
+          plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
+        }
+      l_run = l_run * alpha + psum;
+      // the previous P.V must be done before P is overwritten / O is touched
+      if (i > 0 && !fail && !mbar_wait_bounded(bar_pv, (i - 1) & 1, a.flags)) fail = true;
+      tc::fence_after_sync();
+      wfail = __any_sync(FULL, fail);
+      if (!wfail && __any_sync(FULL, alpha != 1.f)) {  // warp-uniform: lanes without a new max scale by 1
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tc::ld32(tmem + lane_off + kColO + c0, o);
+          tc::wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tc::st32(tmem + lane_off + kColO + c0, o);
+        }
+      }
+      if (!wfail) {
+        tc::st32(tmem + lane_off + kColPhi, phi);
+        tc::st32(tmem + lane_off + kColPlo, plo);
+        tc::wait_st();
+      }
+      tc::fence_before_sync();
     }
-    if (!wfail) {
-      tc::st32(tmem + lane_off + kColPhi, phi);
-      tc::st32(tmem + lane_off + kColPlo, plo);
-      tc::wait_st();
-    }
-    tc::fence_before_sync();
     if (__syncthreads_or(fail)) break;
-    if (tid == 0) {
+    if (tid == kVIssuer) {
       tc::fence_after_sync();
 #pragma unroll
       for (int j = 0; j < kVBN / 16; ++j) {
@@ -289,17 +299,21 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
   if (!fail && ntiles > 0 && !mbar_wait_bounded(bar_pv, (ntiles - 1) & 1, a.flags)) fail = true;
   tc::fence_after_sync();
   const bool aborted = __syncthreads_or(fail) != 0;
-  if (aborted && tid == 0) {
+  if (aborted && tid == kVIssuer) {
     // let MMAs already issued finish before TMEM is released (bounded)
     mbar_wait_bounded(bar_pv, 0, nullptr, 100000000ull);
     mbar_wait_bounded(bar_pv, 1, nullptr, 100000000ull);
     mbar_wait_bounded(bar_s, 0, nullptr, 100000000ull);
     mbar_wait_bounded(bar_s, 1, nullptr, 100000000ull);
+    // and the tile loads still in flight before the shared memory is reused
+    for (int j = n_landed; j < n_issued; ++j) mbar_wait_bounded(&bar_kv[j & 1], (j >> 1) & 1, nullptr, 100000000ull);
   }
   __syncthreads();
   float* wst_o = reinterpret_cast<float*>(st_s);  // [128][D] fp32 (stages are idle now)
   const bool ok = !aborted;
-  if (ok && ntiles > 0) {
+  if (!softmax_thread) {
+    // the issuing warp holds no rows
+  } else if (ok && ntiles > 0) {
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t o[32];
@@ -314,8 +328,10 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(const __grid_constant
   } else {
     for (int c0 = 0; c0 < D; ++c0) wst_o[r * D + c0] = 0.f;
   }
-  wst_ml[2 * r] = (ok && ntiles > 0) ? m_run : -INFINITY;
-  wst_ml[2 * r + 1] = (ok && ntiles > 0) ? l_run : 0.f;
+  if (softmax_thread) {
+    wst_ml[2 * r] = (ok && ntiles > 0) ? m_run : -INFINITY;
+    wst_ml[2 * r + 1] = (ok && ntiles > 0) ? l_run : 0.f;
+  }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -399,7 +415,7 @@ int verify_occupancy() {
   if (cache[dev] == 0) {
     cudaFuncSetAttribute(verify_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, verify_kernel<D>, kVThreads, C::SMEM_B) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, verify_kernel<D>, kVBlock, C::SMEM_B) != cudaSuccess ||
         n < 1)
       n = 1;
     cache[dev] = n;
@@ -499,10 +515,10 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (shape->D == 128) {
     vc::verify_occupancy<128>();  // sets the shared-memory attribute once per device
-    vc::verify_kernel<128><<<grid, vc::kVThreads, vc::VCfg<128>::SMEM_B, s>>>(tk, tv, a);
+    vc::verify_kernel<128><<<grid, vc::kVBlock, vc::VCfg<128>::SMEM_B, s>>>(tk, tv, a);
   } else {
     vc::verify_occupancy<64>();
-    vc::verify_kernel<64><<<grid, vc::kVThreads, vc::VCfg<64>::SMEM_B, s>>>(tk, tv, a);
+    vc::verify_kernel<64><<<grid, vc::kVBlock, vc::VCfg<64>::SMEM_B, s>>>(tk, tv, a);
   }
   if (p.C > 1) {  // chunk partials -> output rows (and lse)
     const int rows_cap = p.nqt * a.g;
