@@ -13,16 +13,20 @@
 // context (split-K) and merge through the workspace.  Per block:
 //   * Q (<= 128 rows) is written once into shared memory in the 128-byte
 //     swizzled K-major layout;
-//   * K and V tiles of BN = 64 keys stream in through a 2-stage ring of tiled
-//     TMA loads (3-D tensor maps, rows past T read as zeros, no multicast);
+//   * K and V tiles of BN = 64 keys stream in through 2-slot rings of tiled
+//     TMA loads (3-D tensor maps, rows past T read as zeros, no multicast),
+//     K and V on barriers of their own: a K slot is refilled as soon as the
+//     S that read it is done, a V slot once its P.V is done;
 //   * a fifth warp issues the TMA loads and tcgen05.mma: S = Q K^T into
 //     tensor memory (TMEM), and P.V; it blocks on the tensor pipe's queue
-//     while the softmax warps work, so no row waits for it;
+//     while the softmax warps work, so no row waits for it.  S is double
+//     buffered: S of tile i + 1 is computed while the softmax of tile i runs;
 //   * each of the 128 softmax threads owns one row: it reads its scores from TMEM,
 //     applies the causal mask (row i sees keys 0 .. T - nq + i), updates an
 //     online softmax with lazy rescaling (O is rescaled only when the running
 //     maximum grows by more than 8 in log2 units), and writes P back to TMEM
-//     as a bf16 high part and a bf16 low part (P keeps ~16 bits);
+//     over its own S as a bf16 high part and a bf16 low part (P keeps ~16
+//     bits);
 //   * O += P_hi V + P_lo V as tcgen05.mma with A read from TMEM and V from
 //     shared memory (MN-major), accumulating in TMEM.
 // All waits are bounded; TMEM is always released.
@@ -40,11 +44,12 @@ constexpr int kVThreads = 128;  // softmax warpgroup: thread r owns row r
 constexpr int kVBlock = kVThreads + 32;  // + the issuing warp
 constexpr int kVIssuer = kVThreads;      // its elected thread
 constexpr int kVTmemCols = 256;
-// TMEM column map
-constexpr uint32_t kColS = 0;     // S: kVBN fp32 columns
-constexpr uint32_t kColPhi = 64;  // P high part: kVBN / 2 columns (bf16 pairs)
-constexpr uint32_t kColPlo = 96;  // P low part
-constexpr uint32_t kColO = 128;   // O: D fp32 columns
+// TMEM column map: two S buffers of kVBN fp32 columns (tile i in buffer
+// i & 1), each overwritten by its P -- high part in the first kVBN / 2
+// columns, low part in the next (bf16 pairs) -- then O, D fp32 columns.
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColPlo = kVBN / 2;  // offset of P's low part inside a buffer
+constexpr uint32_t kColO = 2 * kVBN;
 
 template <int D>
 struct VCfg {
@@ -79,10 +84,11 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_s = smem + C::Q_OFF;
   unsigned char* st_s = smem + C::ST_OFF;
-  uint64_t* bar_kv = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);  // [2]
-  uint64_t* bar_s = bar_kv + 2;
-  uint64_t* bar_pv = bar_kv + 3;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_kv + 4);
+  uint64_t* bar_k = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);  // [2] K slot landed
+  uint64_t* bar_v = bar_k + 2;                                        // [2] V slot landed
+  uint64_t* bar_s = bar_k + 4;                                        // [2] S buffer computed
+  uint64_t* bar_pv = bar_k + 6;                                       // P.V done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_k + 7);
   __shared__ float wst_ml[128 * 2];
   __shared__ float smem_w[3 * 128];
 
@@ -99,10 +105,7 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   const int ntiles = static_cast<int>((k_end - k_begin + kVBN - 1) / kVBN);
 
   if (tid == 0) {
-    mbar_init(&bar_kv[0], 1);
-    mbar_init(&bar_kv[1], 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_pv, 1);
+    for (int j = 0; j < 7; ++j) mbar_init(&bar_k[j], 1);
   }
   fence_mbar_init();
   if (warp == 0) tc::alloc(tmem_slot, kVTmemCols);
@@ -127,19 +130,18 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  int n_issued = 0, n_landed = 0;  // tiles whose loads were issued / waited (issuer)
-  auto issue_tile = [&](int i) {  // issuer only
-    n_issued = i + 1;
-    const int s = i & 1;
-    unsigned char* ks = st_s + s * C::STAGE_B;
-    unsigned char* vs = ks + C::KV_B;
+  // K (v = 0) or V (v = 1) of tile i into slot i & 1; issuer only.  Loads of
+  // one kind land in order; [n_done[v], n_iss[v]) are still in flight.
+  int n_iss[2] = {0, 0}, n_done[2] = {0, 0};
+  auto issue_load = [&](int i, int v) {
+    n_iss[v] = i + 1;
+    unsigned char* dst = st_s + (i & 1) * C::STAGE_B + v * C::KV_B;
+    uint64_t* bar = v ? &bar_v[i & 1] : &bar_k[i & 1];
     const int y = static_cast<int>(k_begin + static_cast<int64_t>(i) * kVBN);
-    mbar_arrive_expect_tx(&bar_kv[s], C::STAGE_B);
+    mbar_arrive_expect_tx(bar, C::KV_B);
 #pragma unroll
-    for (int hf = 0; hf < C::HALVES; ++hf) {
-      tc::tma_load_3d(ks + hf * kVBN * 128, &tm_k, hf * 64, y, unit, &bar_kv[s]);
-      tc::tma_load_3d(vs + hf * kVBN * 128, &tm_v, hf * 64, y, unit, &bar_kv[s]);
-    }
+    for (int hf = 0; hf < C::HALVES; ++hf)
+      tc::tma_load_3d(dst + hf * kVBN * 128, v ? &tm_v : &tm_k, hf * 64, y, unit, bar);
   };
 
   constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, kVBN, false);
@@ -153,29 +155,39 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   const int64_t vis_end = a.T - a.nq + i_row + 1;  // keys [0, vis_end) visible to this row
   float m_run = -INFINITY, l_run = 0.f;
 
-  // S = Q K^T of tile i: issuer, once tile i's K and V have landed
+  // S = Q K^T of tile i into buffer i & 1: issuer, once tile i's K has landed
   auto issue_s = [&](int i) -> bool {
     const uint32_t ks_addr = smem_addr(st_s + (i & 1) * C::STAGE_B);
-    if (!mbar_wait_bounded(&bar_kv[i & 1], (i >> 1) & 1, a.flags)) return false;
-    n_landed = i + 1;
+    if (!mbar_wait_bounded(&bar_k[i & 1], (i >> 1) & 1, a.flags)) return false;
+    n_done[0] = i + 1;
     tc::fence_after_sync();
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const int hf = kk >> 2, ko = (kk & 3) * 32;
       const uint64_t ad = tc::smem_desc_sw128(q_base + hf * (128 * 128) + ko, 16, 1024);
       const uint64_t bd = tc::smem_desc_sw128(ks_addr + hf * (kVBN * 128) + ko, 16, 1024);
-      tc::mma_ss(tmem + kColS, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+      tc::mma_ss(tmem + kColS + (i & 1) * kVBN, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
     }
-    tc::commit(bar_s);
+    tc::commit(&bar_s[i & 1]);
     return true;
   };
 
   bool fail = false;
   const bool softmax_thread = tid < kVThreads;
   if (tid == kVIssuer) {
-    if (ntiles > 0) issue_tile(0);
-    if (ntiles > 1) issue_tile(1);
+    for (int j = 0; j < 2 && j < ntiles; ++j) {
+      issue_load(j, 0);
+      issue_load(j, 1);
+    }
     if (ntiles > 0 && !issue_s(0)) fail = true;
+    if (!fail && ntiles > 1 && !issue_s(1)) fail = true;
+    // S of tile 0 done: its K slot takes tile 2
+    if (!fail && ntiles > 2) {
+      if (!mbar_wait_bounded(&bar_s[0], 0, a.flags))
+        fail = true;
+      else
+        issue_load(2, 0);
+    }
   }
 
   // Failure handling: every wait is bounded; a thread that sees a timeout sets
@@ -188,13 +200,13 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
     const uint32_t ks_addr = smem_addr(st_s + s * C::STAGE_B);
     const uint32_t vs_addr = ks_addr + C::KV_B;
     if (softmax_thread) {  // warp-uniform: warps 0-3
-      if (!fail && !mbar_wait_bounded(bar_s, i & 1, a.flags)) fail = true;
+      if (!fail && !mbar_wait_bounded(&bar_s[s], (i >> 1) & 1, a.flags)) fail = true;
       tc::fence_after_sync();
       bool wfail = __any_sync(FULL, fail);
       uint32_t sr[2][32];
       if (!wfail) {
-        tc::ld32(tmem + lane_off + kColS, sr[0]);
-        tc::ld32(tmem + lane_off + kColS + 32, sr[1]);
+        tc::ld32(tmem + lane_off + kColS + s * kVBN, sr[0]);
+        tc::ld32(tmem + lane_off + kColS + s * kVBN + 32, sr[1]);
         tc::wait_ld();
       } else {
 #pragma unroll
@@ -260,8 +272,8 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
         }
       }
       if (!wfail) {
-        tc::st32(tmem + lane_off + kColPhi, phi);
-        tc::st32(tmem + lane_off + kColPlo, plo);
+        tc::st32(tmem + lane_off + kColS + s * kVBN, phi);
+        tc::st32(tmem + lane_off + kColS + s * kVBN + kColPlo, plo);
         tc::wait_st();
       }
       tc::fence_before_sync();
@@ -269,27 +281,38 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
     if (__syncthreads_or(fail)) break;
     if (tid == kVIssuer) {
       tc::fence_after_sync();
+      if (!mbar_wait_bounded(&bar_v[s], (i >> 1) & 1, a.flags))
+        fail = true;
+      else
+        n_done[1] = i + 1;
+      if (!fail) {
+        const uint32_t pcol = kColS + s * kVBN;
 #pragma unroll
-      for (int j = 0; j < kVBN / 16; ++j) {
-        const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
-        tc::mma_ts(tmem + kColO, tmem + kColPhi + 8 * j, vd, IDESC_PV, (i > 0 || j > 0) ? 1u : 0u);
-      }
+        for (int j = 0; j < kVBN / 16; ++j) {
+          const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
+          tc::mma_ts(tmem + kColO, tmem + pcol + 8 * j, vd, IDESC_PV, (i > 0 || j > 0) ? 1u : 0u);
+        }
 #pragma unroll
-      for (int j = 0; j < kVBN / 16; ++j) {
-        const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
-        tc::mma_ts(tmem + kColO, tmem + kColPlo + 8 * j, vd, IDESC_PV, 1u);
+        for (int j = 0; j < kVBN / 16; ++j) {
+          const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
+          tc::mma_ts(tmem + kColO, tmem + pcol + kColPlo + 8 * j, vd, IDESC_PV, 1u);
+        }
+        tc::commit(bar_pv);
+        // S of tile i + 1 (issued one tile ago) done: its K slot takes tile i + 3
+        if (i + 3 < ntiles) {
+          if (!mbar_wait_bounded(&bar_s[(i + 1) & 1], ((i + 1) >> 1) & 1, a.flags))
+            fail = true;
+          else
+            issue_load(i + 3, 0);
+        }
       }
-      tc::commit(bar_pv);
-      // feed the tensor pipe the next S right behind this P.V (other TMEM
-      // columns, a stage already loaded); its commit also covers this P.V
-      if (i + 1 < ntiles && !issue_s(i + 1)) fail = true;
       if (!fail && i + 2 < ntiles) {
-        // the stage is free once this tile's MMAs are done
+        // P.V of tile i done: its V slot and its S buffer take tile i + 2
         if (!mbar_wait_bounded(bar_pv, i & 1, a.flags)) {
           fail = true;
         } else {
-          fence_proxy_async_smem();
-          issue_tile(i + 2);
+          issue_load(i + 2, 1);
+          if (!issue_s(i + 2)) fail = true;
         }
       }
     }
@@ -303,10 +326,11 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
     // let MMAs already issued finish before TMEM is released (bounded)
     mbar_wait_bounded(bar_pv, 0, nullptr, 100000000ull);
     mbar_wait_bounded(bar_pv, 1, nullptr, 100000000ull);
-    mbar_wait_bounded(bar_s, 0, nullptr, 100000000ull);
-    mbar_wait_bounded(bar_s, 1, nullptr, 100000000ull);
+    for (int j = 0; j < 4; ++j) mbar_wait_bounded(&bar_s[j >> 1], j & 1, nullptr, 100000000ull);
     // and the tile loads still in flight before the shared memory is reused
-    for (int j = n_landed; j < n_issued; ++j) mbar_wait_bounded(&bar_kv[j & 1], (j >> 1) & 1, nullptr, 100000000ull);
+    for (int v = 0; v < 2; ++v)
+      for (int j = n_done[v]; j < n_iss[v]; ++j)
+        mbar_wait_bounded(v ? &bar_v[j & 1] : &bar_k[j & 1], (j >> 1) & 1, nullptr, 100000000ull);
   }
   __syncthreads();
   float* wst_o = reinterpret_cast<float*>(st_s);  // [128][D] fp32 (stages are idle now)
