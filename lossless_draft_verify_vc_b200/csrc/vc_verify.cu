@@ -17,10 +17,11 @@
 //     TMA loads (3-D tensor maps, rows past T read as zeros, no multicast),
 //     K and V on barriers of their own: a K slot is refilled as soon as the
 //     S that read it is done, a V slot once its P.V is done;
-//   * a fifth warp issues the TMA loads and tcgen05.mma: S = Q K^T into
-//     tensor memory (TMEM), and P.V; it blocks on the tensor pipe's queue
-//     while the softmax warps work, so no row waits for it.  S is double
-//     buffered: S of tile i + 1 is computed while the softmax of tile i runs;
+//   * a loader warp issues the TMA loads, an MMA warp issues tcgen05.mma:
+//     S = Q K^T into tensor memory (TMEM), and P.V; the MMA warp blocks on
+//     the tensor pipe's queue while the softmax warps work, so no row waits
+//     for it.  S is double buffered: S of tile i + 1 is computed while the
+//     softmax of tile i runs;
 //   * each of the 128 softmax threads owns one row: it reads its scores from TMEM,
 //     applies the causal mask (row i sees keys 0 .. T - nq + i), updates an
 //     online softmax with lazy rescaling (O is rescaled only when the running
@@ -41,8 +42,9 @@ namespace {
 
 constexpr int kVBN = 64;        // keys per tile
 constexpr int kVThreads = 128;  // softmax warpgroup: thread r owns row r
-constexpr int kVBlock = kVThreads + 32;  // + the issuing warp
-constexpr int kVIssuer = kVThreads;      // its elected thread
+constexpr int kVBlock = kVThreads + 64;  // + the MMA warp + the loader warp
+constexpr int kVIssuer = kVThreads;      // the MMA warp's elected thread
+constexpr int kVLoader = kVThreads + 32; // the loader warp's elected thread
 constexpr int kVTmemCols = 256;
 // TMEM column map: two S buffers of kVBN fp32 columns (tile i in buffer
 // i & 1), each overwritten by its P -- high part in the first kVBN / 2
@@ -60,7 +62,7 @@ struct VCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int ST_OFF = Q_B;                 // 2 stages
   static constexpr int BAR_OFF = ST_OFF + 2 * STAGE_B;
-  static constexpr int SMEM_B = BAR_OFF + 64 + 1024;  // + alignment slack
+  static constexpr int SMEM_B = BAR_OFF + 128 + 1024;  // 8 barriers + TMEM slot; + alignment slack
   static_assert(2 * STAGE_B >= 128 * D * 4, "stages must hold the fp32 output tile");
 };
 
@@ -72,6 +74,18 @@ struct VArgs {
   uint32_t* flags;
   SplitKOut o;
 };
+
+// Block-wide barrier of the softmax warps and the MMA warp only (the loader
+// warp runs its own loop); returns whether any participant passed true.
+__device__ __forceinline__ bool mma_group_sync_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "n"(kVThreads + 32)
+      : "memory");
+  return r != 0;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -87,8 +101,8 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   uint64_t* bar_k = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);  // [2] K slot landed
   uint64_t* bar_v = bar_k + 2;                                        // [2] V slot landed
   uint64_t* bar_s = bar_k + 4;                                        // [2] S buffer computed
-  uint64_t* bar_pv = bar_k + 6;                                       // P.V done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_k + 7);
+  uint64_t* bar_pv = bar_k + 6;                                       // [2] P.V of that buffer done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_k + 8);
   __shared__ float wst_ml[128 * 2];
   __shared__ float smem_w[3 * 128];
 
@@ -103,15 +117,36 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   const int64_t k_begin = static_cast<int64_t>(chunk) * a.tiles_per_chunk * kVBN;
   const int64_t k_end = min(a.T, k_begin + static_cast<int64_t>(a.tiles_per_chunk) * kVBN);
   const int ntiles = static_cast<int>((k_end - k_begin + kVBN - 1) / kVBN);
+  const bool softmax_thread = tid < kVThreads;
+  bool fail = false;
 
-  if (tid == 0) {
-    for (int j = 0; j < 7; ++j) mbar_init(&bar_k[j], 1);
+  // K (v = 0) or V (v = 1) of tile i into slot i & 1; loader only
+  auto issue_load = [&](int i, int v) {
+    unsigned char* dst = st_s + (i & 1) * C::STAGE_B + v * C::KV_B;
+    uint64_t* bar = v ? &bar_v[i & 1] : &bar_k[i & 1];
+    const int y = static_cast<int>(k_begin + static_cast<int64_t>(i) * kVBN);
+    mbar_arrive_expect_tx(bar, C::KV_B);
+#pragma unroll
+    for (int hf = 0; hf < C::HALVES; ++hf)
+      tc::tma_load_3d(dst + hf * kVBN * 128, v ? &tm_v : &tm_k, hf * 64, y, unit, bar);
+  };
+
+  // The loader owns the barriers' initialisation and starts the first two
+  // tiles' loads at once, while the softmax threads fetch Q; nobody else
+  // touches a barrier before the block-wide barrier below.
+  if (tid == kVLoader) {
+    for (int j = 0; j < 8; ++j) mbar_init(&bar_k[j], 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    for (int j = 0; j < 2 && j < ntiles; ++j) {
+      issue_load(j, 0);
+      issue_load(j, 1);
+    }
   }
-  fence_mbar_init();
   if (warp == 0) tc::alloc(tmem_slot, kVTmemCols);
 
   // ---- Q rows -> shared memory, 128-byte swizzled K-major (zeros past M)
-  if (tid < kVThreads) {
+  if (softmax_thread) {
     const int r = tid;
     const bool valid = r < M;
     const int i = i0 + (valid ? r / a.g : 0);
@@ -130,24 +165,10 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  // K (v = 0) or V (v = 1) of tile i into slot i & 1; issuer only.  Loads of
-  // one kind land in order; [n_done[v], n_iss[v]) are still in flight.
-  int n_iss[2] = {0, 0}, n_done[2] = {0, 0};
-  auto issue_load = [&](int i, int v) {
-    n_iss[v] = i + 1;
-    unsigned char* dst = st_s + (i & 1) * C::STAGE_B + v * C::KV_B;
-    uint64_t* bar = v ? &bar_v[i & 1] : &bar_k[i & 1];
-    const int y = static_cast<int>(k_begin + static_cast<int64_t>(i) * kVBN);
-    mbar_arrive_expect_tx(bar, C::KV_B);
-#pragma unroll
-    for (int hf = 0; hf < C::HALVES; ++hf)
-      tc::tma_load_3d(dst + hf * kVBN * 128, v ? &tm_v : &tm_k, hf * 64, y, unit, bar);
-  };
-
   constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, kVBN, false);
   constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(128, D, true);
   const uint32_t q_base = smem_addr(q_s);
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;  // this warp's TMEM lanes
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;  // this warp's TMEM lanes
 
   // row state
   const int r = tid;
@@ -155,11 +176,10 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   const int64_t vis_end = a.T - a.nq + i_row + 1;  // keys [0, vis_end) visible to this row
   float m_run = -INFINITY, l_run = 0.f;
 
-  // S = Q K^T of tile i into buffer i & 1: issuer, once tile i's K has landed
+  // S = Q K^T of tile i into buffer i & 1: MMA thread, once tile i's K has landed
   auto issue_s = [&](int i) -> bool {
     const uint32_t ks_addr = smem_addr(st_s + (i & 1) * C::STAGE_B);
     if (!mbar_wait_bounded(&bar_k[i & 1], (i >> 1) & 1, a.flags)) return false;
-    n_done[0] = i + 1;
     tc::fence_after_sync();
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
@@ -172,171 +192,174 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
     return true;
   };
 
-  bool fail = false;
-  const bool softmax_thread = tid < kVThreads;
   if (tid == kVIssuer) {
-    for (int j = 0; j < 2 && j < ntiles; ++j) {
-      issue_load(j, 0);
-      issue_load(j, 1);
-    }
     if (ntiles > 0 && !issue_s(0)) fail = true;
     if (!fail && ntiles > 1 && !issue_s(1)) fail = true;
-    // S of tile 0 done: its K slot takes tile 2
-    if (!fail && ntiles > 2) {
-      if (!mbar_wait_bounded(&bar_s[0], 0, a.flags))
-        fail = true;
-      else
-        issue_load(2, 0);
-    }
   }
 
   // Failure handling: every wait is bounded; a thread that sees a timeout sets
   // its sticky `fail`.  tcgen05.ld / st are warp-collective, so each warp
-  // decides them with __any_sync; the loop exits on a block-wide
-  // __syncthreads_or, so all threads leave together.
+  // decides them with __any_sync; the tile loop of the softmax and MMA warps
+  // exits on their common barrier's OR, so they leave together; the loader
+  // stops at its first failed wait.  All meet again after the loop.
   constexpr unsigned FULL = 0xffffffffu;
-  for (int i = 0; i < ntiles; ++i) {
-    const int s = i & 1;
-    const uint32_t ks_addr = smem_addr(st_s + s * C::STAGE_B);
-    const uint32_t vs_addr = ks_addr + C::KV_B;
-    if (softmax_thread) {  // warp-uniform: warps 0-3
-      if (!fail && !mbar_wait_bounded(&bar_s[s], (i >> 1) & 1, a.flags)) fail = true;
-      tc::fence_after_sync();
-      bool wfail = __any_sync(FULL, fail);
-      uint32_t sr[2][32];
-      if (!wfail) {
-        tc::ld32(tmem + lane_off + kColS + s * kVBN, sr[0]);
-        tc::ld32(tmem + lane_off + kColS + s * kVBN + 32, sr[1]);
-        tc::wait_ld();
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sr[0][j] = sr[1][j] = 0u;
-      }
-      const int64_t t0 = k_begin + static_cast<int64_t>(i) * kVBN;
-      const int64_t lim = min(vis_end, k_end) - t0;  // keys [t0, t0 + lim) are live
-      // raw scores; the scale (> 0) is applied in the exponent's FMA below
-      float tmax = -INFINITY;
-      if (__all_sync(FULL, lim >= kVBN)) {  // whole tile visible to the warp's rows: no mask
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) tmax = fmaxf(tmax, __uint_as_float(sr[c][j]));
-      } else {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
-            sr[c][j] = __float_as_uint(x);
-            tmax = fmaxf(tmax, x);
-          }
-      }
-      tmax *= a.scale_log2;
-      // lazy rescale: keep the stale maximum unless the new one exceeds it by > 8
-      float m_use = m_run;
-      float alpha = 1.f;
-      if (tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY)) {
-        m_use = tmax;
-        if (m_run != -INFINITY) alpha = ex2(m_run - m_use);
-        m_run = m_use;
-      }
-      const float m_sub = m_use == -INFINITY ? 0.f : m_use;
-      uint32_t phi[32], plo[32];
-      float psum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, -m_sub));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, -m_sub));
-          psum += p0 + p1;
-          const uint32_t hw = pack_bf2(p0, p1);
-          const float2 hf = unpack_bf2(hw);
-          phi[c * 16 + j / 2] = hw;
-          plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
-        }
-      l_run = l_run * alpha + psum;
-      // the previous P.V must be done before P is overwritten / O is touched
-      if (i > 0 && !fail && !mbar_wait_bounded(bar_pv, (i - 1) & 1, a.flags)) fail = true;
-      tc::fence_after_sync();
-      wfail = __any_sync(FULL, fail);
-      if (!wfail && __any_sync(FULL, alpha != 1.f)) {  // warp-uniform: lanes without a new max scale by 1
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tc::ld32(tmem + lane_off + kColO + c0, o);
-          tc::wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tc::st32(tmem + lane_off + kColO + c0, o);
-        }
-      }
-      if (!wfail) {
-        tc::st32(tmem + lane_off + kColS + s * kVBN, phi);
-        tc::st32(tmem + lane_off + kColS + s * kVBN + kColPlo, plo);
-        tc::wait_st();
-      }
-      tc::fence_before_sync();
-    }
-    if (__syncthreads_or(fail)) break;
-    if (tid == kVIssuer) {
-      tc::fence_after_sync();
-      if (!mbar_wait_bounded(&bar_v[s], (i >> 1) & 1, a.flags))
-        fail = true;
-      else
-        n_done[1] = i + 1;
-      if (!fail) {
-        const uint32_t pcol = kColS + s * kVBN;
-#pragma unroll
-        for (int j = 0; j < kVBN / 16; ++j) {
-          const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
-          tc::mma_ts(tmem + kColO, tmem + pcol + 8 * j, vd, IDESC_PV, (i > 0 || j > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int j = 0; j < kVBN / 16; ++j) {
-          const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
-          tc::mma_ts(tmem + kColO, tmem + pcol + kColPlo + 8 * j, vd, IDESC_PV, 1u);
-        }
-        tc::commit(bar_pv);
-        // S of tile i + 1 (issued one tile ago) done: its K slot takes tile i + 3
-        if (i + 3 < ntiles) {
-          if (!mbar_wait_bounded(&bar_s[(i + 1) & 1], ((i + 1) >> 1) & 1, a.flags))
-            fail = true;
-          else
-            issue_load(i + 3, 0);
-        }
-      }
-      if (!fail && i + 2 < ntiles) {
-        // P.V of tile i done: its V slot and its S buffer take tile i + 2
-        if (!mbar_wait_bounded(bar_pv, i & 1, a.flags)) {
+  int nk = ntiles < 2 ? ntiles : 2, nv = nk;  // K / V tiles issued so far (loader)
+  if (warp == kVLoader / 32) {
+    // ---- loader: K of tile j once S of tile j - 2 is done, V of tile j once
+    //      P.V of tile j - 2 is done, in the order those happen (S of tile
+    //      j - 1 finishes before P.V of tile j - 2, so K runs a tile ahead).
+    //      The next completion of the awaited barrier needs this very load,
+    //      so its phase cannot run ahead of the wait.
+    if (tid == kVLoader) {
+      while (nk < ntiles || nv < ntiles) {
+        const bool is_k = nk < ntiles && nk <= nv + 1;
+        const int j = is_k ? nk : nv;
+        if (!mbar_wait_bounded(is_k ? &bar_s[j & 1] : &bar_pv[j & 1], ((j - 2) >> 1) & 1, a.flags)) {
           fail = true;
+          break;
+        }
+        issue_load(j, is_k ? 0 : 1);
+        if (is_k)
+          nk = j + 1;
+        else
+          nv = j + 1;
+      }
+    }
+  } else {
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i & 1;
+      const uint32_t vs_addr = smem_addr(st_s + s * C::STAGE_B) + C::KV_B;
+      if (softmax_thread) {  // warp-uniform: warps 0-3
+        if (!fail && !mbar_wait_bounded(&bar_s[s], (i >> 1) & 1, a.flags)) fail = true;
+        tc::fence_after_sync();
+        bool wfail = __any_sync(FULL, fail);
+        uint32_t sr[2][32];
+        if (!wfail) {
+          tc::ld32(tmem + lane_off + kColS + s * kVBN, sr[0]);
+          tc::ld32(tmem + lane_off + kColS + s * kVBN + 32, sr[1]);
+          tc::wait_ld();
         } else {
-          issue_load(i + 2, 1);
-          if (!issue_s(i + 2)) fail = true;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sr[0][j] = sr[1][j] = 0u;
+        }
+        const int64_t t0 = k_begin + static_cast<int64_t>(i) * kVBN;
+        const int64_t lim = min(vis_end, k_end) - t0;  // keys [t0, t0 + lim) are live
+        // raw scores; the scale (> 0) is applied in the exponent's FMA below
+        float tmax = -INFINITY;
+        if (__all_sync(FULL, lim >= kVBN)) {  // whole tile visible to the warp's rows: no mask
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) tmax = fmaxf(tmax, __uint_as_float(sr[c][j]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
+              sr[c][j] = __float_as_uint(x);
+              tmax = fmaxf(tmax, x);
+            }
+        }
+        tmax *= a.scale_log2;
+        // lazy rescale: keep the stale maximum unless the new one exceeds it by > 8
+        float m_use = m_run;
+        float alpha = 1.f;
+        if (tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY)) {
+          m_use = tmax;
+          if (m_run != -INFINITY) alpha = ex2(m_run - m_use);
+          m_run = m_use;
+        }
+        const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+        uint32_t phi[32], plo[32];
+        float psum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, -m_sub));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, -m_sub));
+            psum += p0 + p1;
+            const uint32_t hw = pack_bf2(p0, p1);
+            const float2 hf = unpack_bf2(hw);
+            phi[c * 16 + j / 2] = hw;
+            plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
+          }
+        l_run = l_run * alpha + psum;
+        // the previous P.V must be done before O is touched
+        if (i > 0 && !fail && !mbar_wait_bounded(&bar_pv[(i - 1) & 1], ((i - 1) >> 1) & 1, a.flags)) fail = true;
+        tc::fence_after_sync();
+        wfail = __any_sync(FULL, fail);
+        if (!wfail && __any_sync(FULL, alpha != 1.f)) {  // warp-uniform: lanes without a new max scale by 1
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tc::ld32(tmem + lane_off + kColO + c0, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tc::st32(tmem + lane_off + kColO + c0, o);
+          }
+        }
+        if (!wfail) {  // P over this tile's S, read above
+          tc::st32(tmem + lane_off + kColS + s * kVBN, phi);
+          tc::st32(tmem + lane_off + kColS + s * kVBN + kColPlo, plo);
+          tc::wait_st();
+        }
+        tc::fence_before_sync();
+      }
+      if (mma_group_sync_or(fail)) break;
+      if (tid == kVIssuer) {
+        tc::fence_after_sync();
+        if (!mbar_wait_bounded(&bar_v[s], (i >> 1) & 1, a.flags)) fail = true;
+        if (!fail) {
+          const uint32_t pcol = kColS + s * kVBN;
+#pragma unroll
+          for (int j = 0; j < kVBN / 16; ++j) {
+            const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
+            tc::mma_ts(tmem + kColO, tmem + pcol + 8 * j, vd, IDESC_PV, (i > 0 || j > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int j = 0; j < kVBN / 16; ++j) {
+            const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
+            tc::mma_ts(tmem + kColO, tmem + pcol + kColPlo + 8 * j, vd, IDESC_PV, 1u);
+          }
+          tc::commit(&bar_pv[s]);
+        }
+        if (!fail && i + 2 < ntiles) {
+          // P.V of tile i done: its S buffer takes tile i + 2
+          if (!mbar_wait_bounded(&bar_pv[s], (i >> 1) & 1, a.flags) || !issue_s(i + 2)) fail = true;
         }
       }
     }
   }
 
   // ---- drain, read O, release TMEM
-  if (!fail && ntiles > 0 && !mbar_wait_bounded(bar_pv, (ntiles - 1) & 1, a.flags)) fail = true;
+  if (!fail && ntiles > 0 && !mbar_wait_bounded(&bar_pv[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, a.flags))
+    fail = true;
   tc::fence_after_sync();
   const bool aborted = __syncthreads_or(fail) != 0;
   if (aborted && tid == kVIssuer) {
     // let MMAs already issued finish before TMEM is released (bounded)
-    mbar_wait_bounded(bar_pv, 0, nullptr, 100000000ull);
-    mbar_wait_bounded(bar_pv, 1, nullptr, 100000000ull);
-    for (int j = 0; j < 4; ++j) mbar_wait_bounded(&bar_s[j >> 1], j & 1, nullptr, 100000000ull);
-    // and the tile loads still in flight before the shared memory is reused
-    for (int v = 0; v < 2; ++v)
-      for (int j = n_done[v]; j < n_iss[v]; ++j)
-        mbar_wait_bounded(v ? &bar_v[j & 1] : &bar_k[j & 1], (j >> 1) & 1, nullptr, 100000000ull);
+    for (int j = 0; j < 4; ++j) {
+      mbar_wait_bounded(&bar_s[j >> 1], j & 1, nullptr, 100000000ull);
+      mbar_wait_bounded(&bar_pv[j >> 1], j & 1, nullptr, 100000000ull);
+    }
+  }
+  if (aborted && tid == kVLoader) {
+    // and the tile loads still in flight: the last one issued into each slot
+    // (earlier ones into it were consumed, hence landed)
+    for (int v = 0; v < 2; ++v) {
+      const int n = v ? nv : nk;
+      for (int j = n - 2; j < n; ++j)
+        if (j >= 0) mbar_wait_bounded(v ? &bar_v[j & 1] : &bar_k[j & 1], (j >> 1) & 1, nullptr, 100000000ull);
+    }
   }
   __syncthreads();
   float* wst_o = reinterpret_cast<float*>(st_s);  // [128][D] fp32 (stages are idle now)
   const bool ok = !aborted;
   if (!softmax_thread) {
-    // the issuing warp holds no rows
+    // the issuing warps hold no rows
   } else if (ok && ntiles > 0) {
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
