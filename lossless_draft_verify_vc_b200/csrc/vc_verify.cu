@@ -11,8 +11,10 @@
 // GQA group form the MMA's M dimension (row r = position i * g + head), so each
 // K/V tile is read from HBM once for the whole group.  Blocks split the
 // context (split-K) and merge through the workspace.  Per block:
-//   * Q (<= 128 rows) is written once into shared memory in the 128-byte
-//     swizzled K-major layout;
+//   * Q (<= 128 rows) is staged once into shared memory in the 128-byte
+//     swizzled K-major layout by tiled TMA (a 3-D map over positions x heads
+//     x channels: the g heads of nqt positions are the tile's rows), the
+//     first request of the block so that it does not queue behind K and V;
 //   * K and V tiles of BN = 64 keys stream in through 2-slot rings of tiled
 //     TMA loads (3-D tensor maps, rows past T read as zeros, no multicast),
 //     K and V on barriers of their own: a K slot is refilled as soon as the
@@ -88,7 +90,8 @@ __device__ __forceinline__ bool mma_group_sync_or(bool v) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                           const __grid_constant__ CUtensorMap tm_k,
                                                            const __grid_constant__ CUtensorMap tm_v, VArgs a) {
   using C = VCfg<D>;
   // the chunk-merge launch that follows may be scheduled as this grid's blocks
@@ -102,9 +105,8 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   uint64_t* bar_v = bar_k + 2;                                        // [2] V slot landed
   uint64_t* bar_s = bar_k + 4;                                        // [2] S buffer computed
   uint64_t* bar_pv = bar_k + 6;                                       // [2] P.V of that buffer done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_k + 8);
-  __shared__ float wst_ml[128 * 2];
-  __shared__ float smem_w[3 * 128];
+  uint64_t* bar_q = bar_k + 8;                                        // Q staged
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_k + 9);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int chunk = blockIdx.x;
@@ -131,13 +133,17 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
       tc::tma_load_3d(dst + hf * kVBN * 128, v ? &tm_v : &tm_k, hf * 64, y, unit, bar);
   };
 
-  // The loader owns the barriers' initialisation and starts the first two
-  // tiles' loads at once, while the softmax threads fetch Q; nobody else
-  // touches a barrier before the block-wide barrier below.
+  // The loader owns the barriers' initialisation and requests Q, then the
+  // first two tiles; nobody else touches a barrier before the block-wide
+  // barrier below.
   if (tid == kVLoader) {
-    for (int j = 0; j < 8; ++j) mbar_init(&bar_k[j], 1);
+    for (int j = 0; j < 9; ++j) mbar_init(&bar_k[j], 1);
     fence_mbar_init();
     fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar_q, C::HALVES * 128 * a.g * a.nqt);
+#pragma unroll
+    for (int hf = 0; hf < C::HALVES; ++hf)
+      tc::tma_load_3d(q_s + hf * (128 * 128), &tm_q, hf * 64, h * a.g, b * a.nq + i0, bar_q);
     for (int j = 0; j < 2 && j < ntiles; ++j) {
       issue_load(j, 0);
       issue_load(j, 1);
@@ -145,19 +151,13 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   }
   if (warp == 0) tc::alloc(tmem_slot, kVTmemCols);
 
-  // ---- Q rows -> shared memory, 128-byte swizzled K-major (zeros past M)
-  if (softmax_thread) {
-    const int r = tid;
-    const bool valid = r < M;
-    const int i = i0 + (valid ? r / a.g : 0);
-    const int hq = h * a.g + (valid ? r % a.g : 0);
-    const uint4* src = reinterpret_cast<const uint4*>(a.q + ((static_cast<size_t>(b) * a.nq + i) * a.Hq + hq) * D);
+  // ---- Q rows past the TMA tile's g * nqt rows are zeros (rows of the tile
+  //      whose position is past nq hold finite data and are never stored)
+  if (softmax_thread && tid >= a.g * a.nqt) {
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
-      const int half = c >> 3, k = c & 7;
-      *reinterpret_cast<uint4*>(q_s + half * (128 * 128) + r * 128 + ((k ^ (r & 7)) << 4)) = v;
-    }
+    for (int c = 0; c < D / 8; ++c)
+      *reinterpret_cast<uint4*>(q_s + (c >> 3) * (128 * 128) + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) =
+          make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
   tc::fence_before_sync();
@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   };
 
   if (tid == kVIssuer) {
-    if (ntiles > 0 && !issue_s(0)) fail = true;
+    if (!mbar_wait_bounded(bar_q, 0, a.flags)) fail = true;
+    if (!fail && ntiles > 0 && !issue_s(0)) fail = true;
     if (!fail && ntiles > 1 && !issue_s(1)) fail = true;
   }
 
@@ -347,8 +348,9 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
     }
   }
   if (aborted && tid == kVLoader) {
-    // and the tile loads still in flight: the last one issued into each slot
-    // (earlier ones into it were consumed, hence landed)
+    // and the loads still in flight: Q, and the last tile issued into each
+    // slot (earlier ones into it were consumed, hence landed)
+    mbar_wait_bounded(bar_q, 0, nullptr, 100000000ull);
     for (int v = 0; v < 2; ++v) {
       const int n = v ? nv : nk;
       for (int j = n - 2; j < n; ++j)
@@ -356,28 +358,52 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
     }
   }
   __syncthreads();
-  float* wst_o = reinterpret_cast<float*>(st_s);  // [128][D] fp32 (stages are idle now)
   const bool ok = !aborted;
-  if (!softmax_thread) {
-    // the issuing warps hold no rows
-  } else if (ok && ntiles > 0) {
+  // ---- O rows straight from TMEM: with one chunk the normalised output rows
+  //      (and lse), otherwise this chunk's partial (unnormalised O, m, l) for
+  //      splitk_combine_kernel.  Rows past M are not stored.
+  if (softmax_thread && ok) {
+    const bool live = r < M;
+    const bool any = ntiles > 0;
+    float* dst = nullptr;
+    float sc = 1.f;
+    const size_t orow = (static_cast<size_t>(b) * a.nq + i0 + r / a.g) * a.Hq + h * a.g + r % a.g;
+    const int rows_cap = a.nqt * a.g;
+    const size_t slot = (static_cast<size_t>(unit) * a.RT + rt) * a.C + chunk;
+    if (a.C == 1) {
+      dst = a.o.out + orow * D;
+      sc = (any && l_run > 0.f) ? 1.f / l_run : 0.f;
+    } else {
+      dst = a.o.part_o + (slot * rows_cap + r) * D;
+    }
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t o[32];
-      tc::ld32(tmem + lane_off + kColO + c0, o);
-      tc::wait_ld();
-      float4* dst = reinterpret_cast<float4*>(wst_o + r * D + c0);
+      if (any) {
+        tc::ld32(tmem + lane_off + kColO + c0, o);  // warp-collective: every lane
+        tc::wait_ld();
+      } else {
 #pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        dst[j / 4] = make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]), __uint_as_float(o[j + 2]),
-                                 __uint_as_float(o[j + 3]));
+        for (int j = 0; j < 32; ++j) o[j] = 0u;
+      }
+      if (live) {
+        float4* d4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          d4[j / 4] = make_float4(__uint_as_float(o[j]) * sc, __uint_as_float(o[j + 1]) * sc,
+                                  __uint_as_float(o[j + 2]) * sc, __uint_as_float(o[j + 3]) * sc);
+      }
     }
-  } else {
-    for (int c0 = 0; c0 < D; ++c0) wst_o[r * D + c0] = 0.f;
-  }
-  if (softmax_thread) {
-    wst_ml[2 * r] = (ok && ntiles > 0) ? m_run : -INFINITY;
-    wst_ml[2 * r + 1] = (ok && ntiles > 0) ? l_run : 0.f;
+    const float m_out = any ? m_run : -INFINITY;
+    const float l_out = any ? l_run : 0.f;
+    if (live) {
+      if (a.C == 1) {
+        if (a.o.lse) a.o.lse[orow] = lse_from(m_out, l_out);
+      } else {
+        a.o.part_ml[(slot * rows_cap + r) * 2] = m_out;
+        a.o.part_ml[(slot * rows_cap + r) * 2 + 1] = l_out;
+      }
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -385,17 +411,6 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
     tc::fence_after_sync();
     tc::dealloc(tmem, kVTmemCols);
   }
-  if (!ok) return;  // the flag tells the caller; partials of this unit are left unmerged
-  const int hq0 = h * a.g;
-  const int g = a.g;
-  const int nq = a.nq;
-  const int Hq = a.Hq;
-  splitk_store<D>(
-      wst_o, 0, wst_ml, 1, M, a.nqt * a.g, a.C, chunk, unit * a.RT + rt, a.o,
-      [&](int rr) {
-        return ((static_cast<size_t>(b) * nq + i0 + rr / g) * Hq + hq0 + rr % g) * D;
-      },
-      [&](int rr) { return (static_cast<size_t>(b) * nq + i0 + rr / g) * Hq + hq0 + rr % g; }, smem_w);
 }
 
 // Output row of flattened partial row fr = ((unit * RT + rt) * rows_cap + r),
@@ -442,6 +457,21 @@ bool make_kv_map(CUtensorMap* m, const void* base, int64_t T, int D, int units) 
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over Q [B * nq][Hq][D] bf16 with a box of 64 channels x g heads x
+// nqt positions: one box is the 128-byte-swizzled rows (position, head) of a
+// row tile, for one half of the channels.
+bool make_q_map(CUtensorMap* m, const void* base, int64_t positions, int Hq, int D, int g, int nqt) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(positions)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hq) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(g), static_cast<cuuint32_t>(nqt)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -536,9 +566,10 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
   const vc::VPlan p = vc::plan_verify(*shape, T, nq);
   VC_REQUIRE(ws_bytes >= p.total, "vc_verify_attn: workspace too small (%zu < %zu)", ws_bytes, p.total);
   const int units = shape->B * shape->Hkv;
-  CUtensorMap tk, tv;
-  if (!vc::make_kv_map(&tk, k, T, shape->D, units) || !vc::make_kv_map(&tv, v, T, shape->D, units))
-    return vc::set_error(VC_ERR_CUDA, "vc_verify_attn: could not encode the K/V tensor maps");
+  CUtensorMap tq, tk, tv;
+  if (!vc::make_kv_map(&tk, k, T, shape->D, units) || !vc::make_kv_map(&tv, v, T, shape->D, units) ||
+      !vc::make_q_map(&tq, q, static_cast<int64_t>(shape->B) * nq, shape->Hq, shape->D, shape->Hq / shape->Hkv, p.nqt))
+    return vc::set_error(VC_ERR_CUDA, "vc_verify_attn: could not encode the Q/K/V tensor maps");
   char* w = static_cast<char*>(ws);
   vc::VArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -562,10 +593,10 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (shape->D == 128) {
     vc::verify_occupancy<128>();  // sets the shared-memory attribute once per device
-    vc::verify_kernel<128><<<grid, vc::kVBlock, vc::VCfg<128>::SMEM_B, s>>>(tk, tv, a);
+    vc::verify_kernel<128><<<grid, vc::kVBlock, vc::VCfg<128>::SMEM_B, s>>>(tq, tk, tv, a);
   } else {
     vc::verify_occupancy<64>();
-    vc::verify_kernel<64><<<grid, vc::kVBlock, vc::VCfg<64>::SMEM_B, s>>>(tk, tv, a);
+    vc::verify_kernel<64><<<grid, vc::kVBlock, vc::VCfg<64>::SMEM_B, s>>>(tq, tk, tv, a);
   }
   if (p.C > 1) {  // chunk partials -> output rows (and lse)
     const int rows_cap = p.nqt * a.g;
