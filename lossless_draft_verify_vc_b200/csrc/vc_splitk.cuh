@@ -1,7 +1,8 @@
-// vc_splitk.cuh -- split-K bookkeeping shared by the attention kernels: the
+// vc_splitk.cuh -- split-K bookkeeping of the attention kernels: the
 // in-block merge of per-warp online-softmax states into a per-chunk partial
-// (splitk_store), and the cross-chunk merge as a separate launch with one
-// warp per output row (splitk_combine_kernel).
+// (splitk_store; the token-dropped draft -- verification stores its one
+// state per row straight from tensor memory), and the cross-chunk merge as a
+// separate launch with one warp per output row (splitk_combine_kernel; both).
 //
 // A partial of one (unit, chunk) holds, per query row r < rows:
 //   o[r][0..D)  unnormalised sum_j 2^(s_j - m) v_j

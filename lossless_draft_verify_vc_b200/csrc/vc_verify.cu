@@ -31,7 +31,10 @@
 //     over its own S as a bf16 high part and a bf16 low part (P keeps ~16
 //     bits);
 //   * O += P_hi V + P_lo V as tcgen05.mma with A read from TMEM and V from
-//     shared memory (MN-major), accumulating in TMEM.
+//     shared memory (MN-major), accumulating in TMEM;
+//   * at the end each softmax thread moves its O row from TMEM to the output
+//     (one chunk) or to its chunk's partial, which splitk_combine_kernel
+//     merges in a programmatic-dependent launch.
 // All waits are bounded; TMEM is always released.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -64,8 +67,7 @@ struct VCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int ST_OFF = Q_B;                 // 2 stages
   static constexpr int BAR_OFF = ST_OFF + 2 * STAGE_B;
-  static constexpr int SMEM_B = BAR_OFF + 128 + 1024;  // 8 barriers + TMEM slot; + alignment slack
-  static_assert(2 * STAGE_B >= 128 * D * 4, "stages must hold the fp32 output tile");
+  static constexpr int SMEM_B = BAR_OFF + 128 + 1024;  // 9 barriers + TMEM slot (76 B); + alignment slack
 };
 
 struct VArgs {
