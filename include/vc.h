@@ -229,7 +229,10 @@ VC_API vc_status vc_draft_attn_sparse(const vc_attn_shape* shape, const vc_spars
  *   k, v bf16 [B][Hkv][T][D]   (HBM-resident or a staging buffer)
  *   out  fp32 [B][nq][Hq][D]
  *   lse  fp32 [B][nq][Hq] natural-log softmax denominators, or NULL
- *   1 <= nq <= 32, T >= nq. */
+ *   1 <= nq <= 32, nq <= T < 2^31, g = Hq / Hkv <= 8, D = 64 or 128,
+ *   B * Hkv <= 65535 (VC_ERR_INVALID_ARG otherwise).  q, k and v are read
+ *   through TMA tensor maps encoded per call; a map the driver refuses
+ *   returns VC_ERR_CUDA before any launch. */
 VC_API size_t vc_verify_attn_workspace_size(const vc_attn_shape* shape, int64_t T, int nq);
 VC_API vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* k, const void* v, int64_t T,
                          int nq, float* out, float* lse, void* ws, size_t ws_bytes, void* stream);
