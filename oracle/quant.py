@@ -9,8 +9,8 @@ width is shared by every layer and token.  [P1] "The Tradeoff VeriCache Is
 Trying to Escape": quantisation keeps all positions and lowers the precision
 of each stored number.
 
-Readings taken where the pages are silent (all listed in the design doc)
-------------------------------------------------------------------
+Readings taken where the pages are silent
+-----------------------------------------
 * Uniform asymmetric min/max quantisation, b in {2, 4} bits.
 * Keys are grouped per channel over G consecutive tokens; values are grouped
   per token over G consecutive channels (the KIVI split).
