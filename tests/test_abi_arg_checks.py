@@ -1,0 +1,118 @@
+"""The C boundary's documented error behaviour, on the CPU: invalid shapes,
+sizes, null or misaligned pointers return VC_ERR_INVALID_ARG with a message
+naming the entry point, from host-side checks that run before any CUDA call
+or launch (include/vc.h, "Conventions shared by every entry point").
+
+The pointers below are fake device addresses: the checks only look at their
+value (null, 16-byte alignment), and every case fails a check, so nothing is
+dereferenced and no CUDA call is reached."""
+
+import ctypes
+
+import pytest
+
+from lossless_draft_verify_vc_b200 import vc
+
+A = 0x100000  # aligned fake device address
+M = 0x100008  # 8 bytes off a 16-byte boundary
+INVALID = -1
+WS = 1 << 40
+
+
+@pytest.fixture(scope="module")
+def L():
+    return vc.lib()
+
+
+def _expect_invalid(L, status, who):
+    assert status == INVALID, status
+    msg = L.vc_last_error().decode()
+    assert who in msg, msg
+
+
+# ------------------------------------------------------------------ verify
+@pytest.mark.parametrize("B,Hq,Hkv,D,T,nq,q,k", [
+    (1, 4, 1, 128, 100, 0, A, A),        # nq < 1
+    (1, 4, 1, 128, 100, 33, A, A),       # nq > 32
+    (1, 4, 1, 128, 10, 31, A, A),        # T < nq
+    (1, 4, 1, 128, 1 << 31, 31, A, A),   # T >= 2^31
+    (1, 4, 1, 96, 100, 31, A, A),        # head dim
+    (1, 6, 4, 128, 100, 31, A, A),       # Hq not a multiple of Hkv
+    (1, 16, 1, 128, 100, 31, A, A),      # g > 8
+    (70000, 1, 1, 128, 100, 31, A, A),   # B * Hkv > 65535
+    (1, 4, 1, 128, 100, 31, 0, A),       # null q
+    (1, 4, 1, 128, 100, 31, A, M),       # misaligned k
+])
+def test_verify_rejects(L, B, Hq, Hkv, D, T, nq, q, k):
+    sh = vc.shape(B, Hq, Hkv, D)
+    st = L.vc_verify_attn(ctypes.byref(sh), q, k, A, T, nq, A, 0, A, WS, 0)
+    _expect_invalid(L, st, "vc_verify_attn")
+
+
+def test_verify_workspace_size_is_zero_for_invalid_shapes(L):
+    assert L.vc_verify_attn_workspace_size(ctypes.byref(vc.shape(1, 4, 1, 96)), 100, 31) == 0
+    assert L.vc_verify_attn_workspace_size(ctypes.byref(vc.shape(1, 4, 1, 128)), 100, 40) == 0
+
+
+# ------------------------------------------------------------ quantised draft
+def _qc(**kw):
+    f = dict(records=A, k_res=A, v_res=A, bits=2, group=32, L_q=1024, R=16, R_cap=32)
+    f.update(kw)
+    return vc.vc_quant_cache(f["records"], f["k_res"], f["v_res"], f["bits"], f["group"], f["L_q"], f["R"],
+                             f["R_cap"])
+
+
+@pytest.mark.parametrize("shape,cache,q,out", [
+    ((1, 4, 1, 128), dict(bits=3), A, A),
+    ((1, 4, 1, 128), dict(group=48), A, A),
+    ((1, 4, 1, 128), dict(L_q=1000), A, A),            # not whole groups
+    ((1, 4, 1, 128), dict(R=40), A, A),                # R > R_cap
+    ((1, 4, 1, 128), dict(L_q=0, R=0), A, A),          # no token at all
+    ((1, 4, 1, 128), dict(records=0), A, A),
+    ((1, 4, 1, 128), dict(records=M), A, A),
+    ((1, 4, 1, 128), dict(v_res=0), A, A),
+    ((1, 4, 1, 96), dict(), A, A),
+    ((1, 4, 1, 128), dict(), 0, A),                    # null q
+    ((1, 4, 1, 128), dict(), A, M),                    # misaligned out
+])
+def test_quant_draft_rejects(L, shape, cache, q, out):
+    sh = vc.shape(*shape)
+    qc = _qc(**cache)
+    st = L.vc_draft_attn_quant(ctypes.byref(sh), ctypes.byref(qc), q, out, A, WS, 0)
+    _expect_invalid(L, st, "vc_draft_attn_quant")
+
+
+def test_quant_noalloc_rejects_before_touching_its_scratch(L):
+    sh = vc.shape(1, 4, 1, 128)
+    st = L.vc_draft_attn_quant_noalloc(ctypes.byref(sh), ctypes.byref(_qc(bits=5)), A, A, 0)
+    _expect_invalid(L, st, "vc_draft_attn_quant_noalloc")
+
+
+# -------------------------------------------------------- token-dropped draft
+@pytest.mark.parametrize("k,T_store,idx,n_keep,q", [
+    (A, 100, A, 0, A),       # n_keep < 1
+    (A, 0, A, 10, A),        # empty store
+    (A, 100, 0, 10, A),      # null positions
+    (M, 100, A, 10, A),      # misaligned K store
+    (A, 100, A, 10, 0),      # null q
+])
+def test_sparse_draft_rejects(L, k, T_store, idx, n_keep, q):
+    sh = vc.shape(1, 4, 1, 128)
+    sc = vc.vc_sparse_cache(k, A, T_store, idx, n_keep)
+    st = L.vc_draft_attn_sparse(ctypes.byref(sh), ctypes.byref(sc), q, A, A, WS, 0)
+    _expect_invalid(L, st, "vc_draft_attn_sparse")
+
+
+# ----------------------------------------------------------------- acceptance
+@pytest.mark.parametrize("logits,dtype,B,K,V,target", [
+    (A, vc.VC_BF16, 0, 30, 1000, A),      # B < 1
+    (A, vc.VC_BF16, 1, 65, 1000, A),      # K > 64
+    (A, vc.VC_BF16, 1, 30, 0, A),         # V < 1
+    (A, 7, 1, 30, 1000, A),               # dtype
+    (A, vc.VC_BF16, 1, 30, 1000, 0),      # null target
+    (M, vc.VC_BF16, 1, 30, 1000, A),      # misaligned logits
+    (A, vc.VC_BF16, 3000, 30, 1000, A),   # more than 65535 logit rows
+])
+def test_accept_rejects(L, logits, dtype, B, K, V, target):
+    st = L.vc_accept(logits, dtype, B, K, V, A, target, A, A, A, WS, 0)
+    _expect_invalid(L, st, "vc_accept")
