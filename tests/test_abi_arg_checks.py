@@ -116,3 +116,69 @@ def test_sparse_draft_rejects(L, k, T_store, idx, n_keep, q):
 def test_accept_rejects(L, logits, dtype, B, K, V, target):
     st = L.vc_accept(logits, dtype, B, K, V, A, target, A, A, A, WS, 0)
     _expect_invalid(L, st, "vc_accept")
+
+
+# ------------------------------------------------------ host -> HBM streaming
+def _ptrs(*xs):
+    arr = (ctypes.c_void_p * len(xs))(*xs)
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+@pytest.mark.parametrize("n_layers,nbytes,host_k,dev_k0", [
+    (0, 4096, (A, A), A),      # no layer
+    (2, 0, (A, A), A),         # empty layer
+    (2, 4096, (A, 0), A),      # null host pointer of layer 1
+    (2, 4096, (A, A), M),      # misaligned staging slot
+    (2, 4096, (A, A), 0),      # null staging slot
+])
+def test_kvstream_create_rejects(L, n_layers, nbytes, host_k, dev_k0):
+    hk, _a = _ptrs(*host_k)
+    hv, _b = _ptrs(A, A)
+    dk, _c = _ptrs(dev_k0, A)
+    dv, _d = _ptrs(A, A)
+    handle = ctypes.c_void_p(0)
+    st = L.vc_kvstream_create(ctypes.byref(handle), n_layers, hk, hv, nbytes, dk, dv, 0)
+    _expect_invalid(L, st, "vc_kvstream_create")
+    assert not handle.value
+
+
+def test_kvstream_calls_reject_a_null_object(L):
+    k, v = ctypes.c_void_p(0), ctypes.c_void_p(0)
+    _expect_invalid(L, L.vc_kvstream_prefetch(None, 0), "vc_kvstream_prefetch")
+    _expect_invalid(L, L.vc_kvstream_acquire(None, 0, 0, ctypes.byref(k), ctypes.byref(v)), "vc_kvstream_acquire")
+    _expect_invalid(L, L.vc_kvstream_release(None, 0, 0), "vc_kvstream_release")
+    assert L.vc_kvstream_destroy(None) == 0  # destroying nothing is a no-op
+
+
+# ------------------------------------------------------------------ scheduler
+def _request(**kw):
+    r = vc.vc_sched_request()
+    r.shape = vc.shape(1, 4, 1, 128)
+    r.draft_kind = vc.VC_DRAFT_QUANT
+    r.T, r.nq, r.V = 256, 31, 1000
+    r.kv_bytes_per_layer = 1 * 1 * 256 * 128 * 2
+    for f in ("qcaches", "draft_q", "draft_out", "draft_ws", "host_k", "host_v", "verify_q", "verify_out",
+              "verify_ws", "logits", "draft_tokens", "target", "accept_len", "correction", "accept_ws"):
+        setattr(r, f, A)
+    r.stage_k[0] = r.stage_k[1] = r.stage_v[0] = r.stage_v[1] = A
+    r.draft_ws_bytes = r.verify_ws_bytes = r.accept_ws_bytes = WS
+    r.logits_dtype = vc.VC_BF16
+    for k, v in kw.items():
+        setattr(r, k, v)
+    return r
+
+
+@pytest.mark.parametrize("n_req,policy,timeout_ms,req", [
+    (0, vc.VC_SCHED_STAGGER, 1000, {}),                       # no request
+    (1, 9, 1000, {}),                                         # unknown policy
+    (1, vc.VC_SCHED_STAGGER, 0, {}),                          # no timeout
+    (1, vc.VC_SCHED_STAGGER, 1000, {"qcaches": 0}),           # quantised draft without caches
+    (1, vc.VC_SCHED_STAGGER, 1000, {"host_k": 0}),            # no host KV
+    (1, vc.VC_SCHED_STAGGER, 1000, {"kv_bytes_per_layer": 12345}),
+])
+def test_sched_create_rejects(L, n_req, policy, timeout_ms, req):
+    reqs = (vc.vc_sched_request * 1)(_request(**req))
+    handle = ctypes.c_void_p(0)
+    st = L.vc_sched_create(ctypes.byref(handle), n_req, reqs, 2, 30, policy, 0, timeout_ms)
+    _expect_invalid(L, st, "vc_sched_create")
+    assert not handle.value
