@@ -561,7 +561,7 @@ def run_stagger(args, w, rank, world):
     clocks = ClockSampler(dev.index)
     clocks.start()
     for name, pol in (("lockstep", vc.VC_SCHED_LOCKSTEP), ("stagger", vc.VC_SCHED_STAGGER)):
-        sch = vc.Sched(reqs, NL, K, pol, copy, timeout_ms=600000)
+        sch = vc.Sched(reqs, NL, K, pol, copy, timeout_ms=30000)
         sch.run_rounds(1)  # warm-up round
         torch.cuda.synchronize(dev)
         if world > 1:

@@ -297,7 +297,9 @@ VC_API vc_status vc_kvstream_destroy(vc_kvstream* s);
  * draft is done and the link is free, and starts its next round's draft as
  * soon as its own round is done, so one request's verification overlaps
  * other requests' drafting.  The host polls events (never blocks a device)
- * and gives up with VC_ERR_TIMEOUT after timeout_ms.  Inputs and outputs
+ * and gives up with VC_ERR_TIMEOUT once timeout_ms pass without progress
+ * (no draft, verification or round of any request completing or starting);
+ * a run that keeps progressing may last any time.  Inputs and outputs
  * of every call are the caller's (device pointers, as in the calls above);
  * the round's synthetic inputs do not change between rounds. */
 #define VC_DRAFT_QUANT 0
@@ -355,7 +357,7 @@ VC_API vc_status vc_sched_destroy(vc_sched* s);
  * the finishing time of the last round to *makespan_ms.  A request index
  * `never_done` >= 0 makes that request's first verification never complete,
  * which exercises the timeout path (VC_ERR_TIMEOUT after timeout_ms of
- * simulated time).  Used by the CPU tests of the policy. */
+ * simulated time without progress).  Used by the CPU tests of the policy. */
 VC_API vc_status vc_sched_simulate(int n_requests, int n_rounds, int policy, const double* draft_ms,
                                    const double* verify_ms, int never_done, double timeout_ms,
                                    double* makespan_ms);

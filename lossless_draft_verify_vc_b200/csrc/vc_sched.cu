@@ -46,14 +46,16 @@ enum Phase { kIdle, kDrafting, kReady, kVerifying, kFinished };
 //   STAGGER: a request drafts as soon as its previous round is done and
 //   verifies as soon as its draft is done and the link is free.
 // In both, one verification holds the link at a time (first ready, first
-// served).
+// served).  timeout_ms bounds the time WITHOUT progress (no phase of any
+// request changed): a long run that keeps completing phases never times out,
+// one whose outstanding work stops completing fails after timeout_ms.
 vc_status run_policy(Backend& be, int n, int n_rounds, int policy, double timeout_ms) {
   std::vector<Phase> ph(n, kIdle);
   std::vector<int> rnd(n, 0);
   std::deque<int> ready;
   int link_owner = -1;
   int finished = 0;
-  const double t0 = be.now_ms();
+  double t_progress = be.now_ms();
   if (n_rounds <= 0) return VC_OK;
   while (finished < n) {
     bool progressed = false;
@@ -110,8 +112,10 @@ vc_status run_policy(Backend& be, int n, int n_rounds, int policy, double timeou
         progressed = true;
       }
     }
-    if (!progressed) {
-      if (be.now_ms() - t0 > timeout_ms)
+    if (progressed) {
+      t_progress = be.now_ms();
+    } else {
+      if (be.now_ms() - t_progress > timeout_ms)
         return set_error(VC_ERR_TIMEOUT, "vc_sched: no progress within %.0f ms", timeout_ms);
       be.idle();
     }

@@ -68,6 +68,21 @@ def test_a_verification_that_never_completes_times_out():
     assert e.value.status == vc.VC_ERR_TIMEOUT
 
 
+def test_timeout_bounds_time_without_progress_not_the_whole_run():
+    # every phase completes within 30 ms of simulated time, the run lasts far
+    # longer than the 40 ms limit: it must finish
+    n, R, D, V = 3, 6, 10.0, 30.0
+    got = vc.vc_sched_simulate([D] * n, [V] * n, R, vc.VC_SCHED_STAGGER, timeout_ms=40.0)
+    assert got == pytest.approx(D + R * n * V)
+    assert got > 10 * 40.0
+    got = vc.vc_sched_simulate([D] * n, [V] * n, R, vc.VC_SCHED_LOCKSTEP, timeout_ms=40.0)
+    assert got == pytest.approx(R * n * (D + V))
+    # the same run with one verification that stops completing fails
+    with pytest.raises(vc.VcError) as e:
+        vc.vc_sched_simulate([D] * n, [V] * n, R, vc.VC_SCHED_STAGGER, never_done=2, timeout_ms=40.0)
+    assert e.value.status == vc.VC_ERR_TIMEOUT
+
+
 def test_invalid_arguments_are_refused_before_any_device_call():
     L = vc.lib()
     h = ctypes.c_void_p()
