@@ -202,14 +202,28 @@ VC_API vc_status vc_draft_attn_quant(const vc_attn_shape* shape, const vc_quant_
  * library holds until the process exits.  Nothing is allocated.
  *   - The first call on a device looks up that array's address (with the
  *     device current); make that first call before any stream capture.
- *   - All calls share the one array; each call clears the counters it needs
- *     at zero.  Calls that overlap on the GPU (different streams or host
- *     threads) race on it and must be serialised by the caller.
+ *   - All calls share the one array and leave in it whatever they wrote;
+ *     nothing in it has to start at zero except the flag word below, which
+ *     is zero when the library loads.  Calls that overlap on the GPU
+ *     (different streams or host threads) race on the array and must be
+ *     serialised by the caller.
+ *   - Device-side errors (a bounded on-chip wait that gave up: that call's
+ *     output is incomplete) are ORed into the array's flag word and stay
+ *     there across calls until vc_draft_attn_quant_noalloc_flags() reads
+ *     and clears them.
+ *   - The array's address is cached per device for the life of the process:
+ *     cudaDeviceReset() while the library is in use is not supported.
  *   - A call whose scratch would exceed VC_NOALLOC_SCRATCH_BYTES returns
  *     VC_ERR_WORKSPACE with a message and enqueues nothing. */
 #define VC_NOALLOC_SCRATCH_BYTES (4u << 20)
 VC_API vc_status vc_draft_attn_quant_noalloc(const vc_attn_shape* shape, const vc_quant_cache* cache,
                                              const void* q, float* out, void* stream);
+/* Reads the VC_FLAG_* bits that vc_draft_attn_quant_noalloc calls on the
+ * current device have set since the last read, writes them to *host_flags
+ * (host memory) and clears them.  Enqueues the read and the clear on
+ * `stream` and waits for that stream.  No counterpart in the pages; it is
+ * the allocation-free path's version of vc_workspace_flags(). */
+VC_API vc_status vc_draft_attn_quant_noalloc_flags(uint32_t* host_flags, void* stream);
 
 /* ---- draft attention over a token-dropped cache ----------------------------
  * out[b][hq][:] = softmax(q . K[idx]^T * sm_scale) . V[idx] over the n_keep

@@ -68,8 +68,8 @@ struct QCfg {
   static constexpr int RING0 = NST * STAGE > RSTAGE ? NST * STAGE : RSTAGE;
   static constexpr int RING = (RING0 + 127) / 128 * 128;
   static constexpr int HEADS = 4 * NT;
-  static constexpr int PS_B = 2 * HEADS * G * 2;  // p high / low parts, fp16 [HEADS][G] each
-  static constexpr int WARP_B = RING + PS_B;
+  static constexpr int RP_B = HEADS * kResRows * 4;  // residual tile scores, fp32 [HEADS][16]
+  static constexpr int WARP_B = RING + RP_B;
   static constexpr int STATE_OFF = kQNW * WARP_B;                       // fp32 [kQNW][HEADS][D]
   static constexpr int ML_OFF = STATE_OFF + kQNW * HEADS * D * 4;       // fp32 [kQNW][HEADS][2]
   static constexpr int MW_OFF = ML_OFF + kQNW * HEADS * 2 * 4;          // merge weights + (M, L)
@@ -80,7 +80,6 @@ struct QCfg {
   static constexpr int CPG = D / G;   // value groups per token
   static_assert(G % 32 == 0, "group must be a multiple of 32");
   static_assert(REC % 16 == 0 && STAGE % 16 == 0, "bulk copies need 16-byte multiples");
-  static_assert(PS_B >= HEADS * kResRows * 4, "residual scores share the p buffer");
   static_assert(WARP_B % 128 == 0, "warp areas stay 128-byte aligned");
 };
 
@@ -230,62 +229,457 @@ __device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring,
 }
 
 // ----------------------------------------------------------- quantised part
-// Processes this warp's stages of unit u's quantised segment (the prefetch
-// pipeline runs on across segments) and leaves the warp's state in its slot.
-template <int BITS, int G, int D, int NT>
-__device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, int u, int64_t qs0, int my_nq,
-                          int& iq, int& issued, IssuePtr& ip, int& islot, int& cslot, uint32_t& cphase, bool& ok,
-                          float* st_o, float* st_ml) {
-  using C = QCfg<BITS, G, D, NT>;
+//
+// Two arrangements of the same arithmetic, chosen by the GQA group size g:
+//
+//   TokM (g <= 4): scores D[token][col] = codes[token][chan] x qfold[chan][col]
+//     with col = 2 * head + part (part 0 = high, 1 = low fp16 part of q*s),
+//     so the 4 heads' two parts fill the MMA's N = 8.  The softmax weights
+//     of a lane (one head, four tokens) are moved into the value MMA's B
+//     layout with movmatrix (8x8 transposes in registers).
+//   HeadM (4 < g <= 8): scores D[row][token] = qfold[row][chan] x
+//     codes[chan][token] with row = head (high part) or 8 + head (low part),
+//     so the 8 heads' two parts fill M = 16; a lane ends up holding the
+//     weights of one head for the token pairs the value MMA's B operand
+//     needs, and no data moves between lanes.
+//
+// Both: values D[chan][col] = codes^T[chan][token] x pfold[token][col].
+// The softmax weights p (<= 2^kLazyLog2 by the lazy running maximum) are
+// rounded once to fp16 (p~) for the value side; the softmax denominator
+// sums the fp32 p.  p~ * s is split into an fp16 high part and the exact
+// fp16 remainder (one fma), so the value operand carries ~22 bits.
+
+constexpr float kLazy = 8.f;  // raise the running max only when a score exceeds it by > 2^8
+
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(x));
+  return d;
+}
+
+// a * b - c, f16x2
+__device__ __forceinline__ uint32_t hfms2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("{\n\t.reg .b32 t;\n\tneg.f16x2 t, %3;\n\tfma.rn.f16x2 %0, %1, %2, t;\n\t}\n"
+      : "=r"(d)
+      : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t zscale(uint32_t z, int i) {
+  // z * 2^(bits i) in fp16 (exact while |z| 2^(bits i) stays below 65504)
+  if (i == 0) return z;
+  const uint32_t f2 = static_cast<uint32_t>(15 + BITS * i) << 10;
+  return hmul2(z, f2 | (f2 << 16));
+}
+
+template <int BITS, int G, int D>
+struct TokM {
   using F = Frag<BITS>;
-  constexpr unsigned FULL = 0xffffffffu;
-  constexpr int NW = 2 * C::KT / F::TPW;  // words per lane per 16-token tile
-  constexpr int MT = G / 16;              // token tiles per group
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int part = gid & 1;
-  __half* Ph = reinterpret_cast<__half*>(ring + C::RING);  // [HEADS][G] fp16 high parts of p
-  __half* Pl = Ph + C::HEADS * G;                          // low parts
-  const int b = u / a.Hkv, h = u - b * a.Hkv;
+  static constexpr int KT = D / 16, TPW = F::TPW, NW = 2 * KT / TPW, MT = G / 16, CPG = D / G;
+  static constexpr int HEADS = 4;
+  uint32_t qs[KT][2];  // q * 2^-(bits i), negated in low-part lanes
+  uint32_t qm[KT][2];  // q * 2^-(bits i) in low-part lanes, 0 in high-part lanes
+  float acc[KT][4];    // D[channel][col]
+  float vb[4];         // value zero-point term: D[value group][col]
+  float m_run, m_lim, l_run;
 
-  // per-lane constants of the high/low split: part 0 lanes keep the rounded
-  // product, part 1 lanes its rounding error
-  const uint32_t kap = part ? 0xBC00BC00u : 0u;  // (-1, -1) or (0, 0) in fp16
-  const uint32_t mu = part ? 0x3C003C00u : 0u;   // (1, 1) or (0, 0)
-
-  // ---- query registers (fp16, exact from bf16), column head = nt*4 + gid/2,
-  //      natural channel pairs (16kt + 2tig, +1) and (16kt + 2tig + 8, +9)
-  //   q2s: scaled by 2^-(bits * (kt % TPW)) of the code encoding (the
-  //        zero-point MMA uses it too, with the zeros scaled up to match)
-  uint32_t q2s[C::KT][NT][2];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int hh = nt * 4 + (gid >> 1);
+  __device__ __forceinline__ void init(const QArgs& a, int b, int h, int lane) {
+    const int gid = lane >> 2, tig = lane & 3, part = gid & 1;
+    const int hh = gid >> 1;
     const bool hv = hh < a.g;
     const __nv_bfloat16* qp = a.q + (static_cast<size_t>(b) * a.Hq + h * a.g + (hv ? hh : 0)) * D;
 #pragma unroll
-    for (int kt = 0; kt < C::KT; ++kt) {
-      const float f = pow2i(-BITS * (kt % F::TPW));
+    for (int kt = 0; kt < KT; ++kt) {
+      const float f = pow2i(-BITS * (kt % TPW));
       const float2 lo = unpack_bf2(*reinterpret_cast<const uint32_t*>(qp + kt * 16 + 2 * tig));
       const float2 hi = unpack_bf2(*reinterpret_cast<const uint32_t*>(qp + kt * 16 + 8 + 2 * tig));
-      q2s[kt][nt][0] = hv ? pack_h2(lo.x * f, lo.y * f) : 0u;
-      q2s[kt][nt][1] = hv ? pack_h2(hi.x * f, hi.y * f) : 0u;
+      const uint32_t q0 = hv ? pack_h2(lo.x * f, lo.y * f) : 0u;
+      const uint32_t q1 = hv ? pack_h2(hi.x * f, hi.y * f) : 0u;
+      qs[kt][0] = part ? q0 ^ 0x80008000u : q0;
+      qs[kt][1] = part ? q1 ^ 0x80008000u : q1;
+      qm[kt][0] = part ? q0 : 0u;
+      qm[kt][1] = part ? q1 : 0u;
+    }
+#pragma unroll
+    for (int mc = 0; mc < KT; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
+    vb[0] = vb[1] = vb[2] = vb[3] = 0.f;
+    m_run = -INFINITY;
+    m_lim = -INFINITY;
+    l_run = 0.f;
+  }
+
+  // One group record at rs (shared memory).
+  __device__ __forceinline__ void group(const unsigned char* rs, int lane, float scl, float sl2) {
+    constexpr unsigned FULL = 0xffffffffu;
+    using C = QCfg<BITS, G, D, 1>;
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t* kcw = reinterpret_cast<const uint32_t*>(rs);
+    const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
+    const uint4* skw = reinterpret_cast<const uint4*>(rs + C::OFF_SK) + tig * (KT / 2);
+    const uint4* zkw = reinterpret_cast<const uint4*>(rs + C::OFF_ZK) + tig * (KT / 2);
+    const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);  // [G/2][CPG] token pairs
+    const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
+
+    // (1) scores: per channel tile kt the key scales are folded into q right
+    //     before use (high part in part-0 columns, low part in part-1
+    //     columns); the zero-point term sum_c q_c z_c is an MMA of the zeros
+    //     (times 2^(bits i), exact) against the signed q in the high columns.
+    float sc[MT][4], kb[4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
+    kb[0] = kb[1] = kb[2] = kb[3] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NW / 2; ++j) {
+      uint32_t X[MT], Y[MT], XS[MT], YS[MT];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const uint2 w = *reinterpret_cast<const uint2*>(kcw + (mt * 32 + lane) * NW + 2 * j);
+        X[mt] = w.x, Y[mt] = w.y, XS[mt] = w.x >> 8, YS[mt] = w.y >> 8;
+      }
+#pragma unroll
+      for (int i = 0; i < TPW; ++i) {
+        const int kt = TPW * j + i;
+        const uint4 s4 = skw[kt >> 1];
+        const uint32_t sA = (kt & 1) ? s4.z : s4.x, sC = (kt & 1) ? s4.w : s4.y;
+        const uint32_t fa = hfma2(qm[kt][0], sA, hmul2(qs[kt][0], sA));
+        const uint32_t fc = hfma2(qm[kt][1], sC, hmul2(qs[kt][1], sC));
+        const uint32_t m = F::mask(i);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const uint32_t af[4] = {X[mt] & m, XS[mt] & m, Y[mt] & m, YS[mt] & m};
+          mma_f16(sc[mt], af, fa, fc);
+        }
+        const uint4 z4 = zkw[kt >> 1];
+        const uint32_t z0 = zscale<BITS>((kt & 1) ? z4.z : z4.x, i);
+        const uint32_t z8 = zscale<BITS>((kt & 1) ? z4.w : z4.y, i);
+        const uint32_t za[4] = {z0, z0, z8, z8};
+        mma_f16(kb, za, qs[kt][0], qs[kt][1]);
+      }
+    }
+
+    // (2) softmax of head tig over the lane's tokens 16 mt + gid (+8); the
+    //     scores sit in the 2^-24 domain of the code encoding
+    const float kzs = kb[0] * sl2;
+    float x[MT][2];
+    float t = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      x[mt][0] = fmaf(sc[mt][0] + sc[mt][1], scl, kzs);
+      x[mt][1] = fmaf(sc[mt][2] + sc[mt][3], scl, kzs);
+      t = fmaxf(t, fmaxf(x[mt][0], x[mt][1]));
+    }
+    t = warp_max_xor(t, 4);
+    t = warp_max_xor(t, 8);
+    t = warp_max_xor(t, 16);
+    if (__any_sync(FULL, t > m_lim)) {
+      const float m_new = fmaxf(m_run, t);
+      const float alpha = ex2(m_run - m_new);
+      m_run = m_new;
+      m_lim = m_new + kLazy;
+      l_run *= alpha;
+#pragma unroll
+      for (int mc = 0; mc < KT; ++mc) {
+        acc[mc][0] *= alpha;
+        acc[mc][1] *= alpha;
+        acc[mc][2] *= alpha;
+        acc[mc][3] *= alpha;
+      }
+      vb[0] *= alpha;
+      vb[1] *= alpha;
+      vb[2] *= alpha;
+      vb[3] *= alpha;
+    }
+    // p~ into the value MMA's B layout: an 8x8 block [token][col] holds
+    // (p, -p) in a head's (high, low) columns for PA and (0, p) for PB;
+    // after the transpose lane (gid, tig) holds its column's entries for
+    // tokens 2 tig, 2 tig + 1 of the block.
+    uint32_t PA[MT][2], PB[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const float p = ex2(x[mt][hf] - m_run);
+        l_run += p;
+        PA[mt][hf] = movm_t(pack_h2(p, -p));
+        PB[mt][hf] = movm_t(pack_h2(0.f, p));
+      }
+    }
+
+    // (3) P . V: per 16-token tile, the folded operand of value group cg is
+    //     high (part 0 columns: 0 + fp16(p~ s)) or low (part 1 columns:
+    //     p~ s - fp16(p~ s), exact) -- the same two instructions in every lane
+#pragma unroll
+    for (int ktt = 0; ktt < MT; ++ktt) {
+      uint32_t s01[CPG], s89[CPG];
+      load_cpg<CPG>(sv32 + (ktt * 8 + tig) * CPG, s01);
+      load_cpg<CPG>(sv32 + (ktt * 8 + 4 + tig) * CPG, s89);
+      {
+        // value zero-point term: A = z_v^T (row = value group gid), B = p~ (low columns)
+        uint32_t za[4] = {0u, 0u, 0u, 0u};
+        if (gid < CPG) {
+          za[0] = zv32[(ktt * 8 + tig) * CPG + gid];
+          za[2] = zv32[(ktt * 8 + 4 + tig) * CPG + gid];
+        }
+        mma_f16(vb, za, PB[ktt][0], PB[ktt][1]);
+      }
+      uint32_t pf0 = 0u, pf1 = 0u;
+#pragma unroll
+      for (int j = 0; j < NW / 2; ++j) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vcw + (ktt * 32 + lane) * NW + 2 * j);
+        const uint32_t X = w.x, Y = w.y, XS = w.x >> 8, YS = w.y >> 8;
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+          const int mc = TPW * j + i;
+          const int cg = mc * 16 / G;
+          if (mc == 0 || (mc - 1) * 16 / G != cg) {
+            pf0 = hfma2(PB[ktt][0], s01[cg], hmul2(PA[ktt][0], s01[cg]));
+            pf1 = hfma2(PB[ktt][1], s89[cg], hmul2(PA[ktt][1], s89[cg]));
+          }
+          const uint32_t m = F::mask(i);
+          const uint32_t af[4] = {X & m, Y & m, XS & m, YS & m};
+          mma_f16(acc[mc], af, pf0, pf1);
+        }
+      }
     }
   }
+
+  // This warp's state -> its slot (natural channel order, unnormalised).
+  __device__ __forceinline__ void store(const QArgs& a, int warp, int lane, bool ok, float* st_o, float* st_ml) {
+    constexpr unsigned FULL = 0xffffffffu;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int hh = tig;
+    float l = l_run;
+    l += __shfl_xor_sync(FULL, l, 4);
+    l += __shfl_xor_sync(FULL, l, 8);
+    l += __shfl_xor_sync(FULL, l, 16);
+    const float vbs = vb[1];  // value-zero term of group gid, head tig (low column)
+#pragma unroll
+    for (int mc = 0; mc < KT; ++mc) {
+      const int cg = mc * 16 / G;
+      const float zb = __shfl_sync(FULL, vbs, cg * 4 + tig);
+      const float uf = pow2i(24 - BITS * (mc % TPW));  // undo the code encoding of this tile
+      if (hh < a.g) {
+        float* wo = st_o + (warp * HEADS + hh) * D + mc * 16 + gid;
+        wo[0] = (acc[mc][0] + acc[mc][1]) * uf + zb;
+        wo[8] = (acc[mc][2] + acc[mc][3]) * uf + zb;
+      }
+    }
+    if (hh < a.g && gid == 0) {
+      st_ml[(warp * HEADS + hh) * 2] = ok ? m_run : -INFINITY;
+      st_ml[(warp * HEADS + hh) * 2 + 1] = ok ? l : 0.f;
+    }
+  }
+};
+
+template <int BITS, int G, int D>
+struct HeadM {
+  using F = Frag<BITS>;
+  static constexpr int KT = D / 16, TPW = F::TPW, NW = 2 * KT / TPW, MT = G / 16, CPG = D / G;
+  static constexpr int HEADS = 8;
+  uint32_t q2[KT][2];  // head gid: q * 2^-(bits i), channel pairs (2 tig, +1), (2 tig + 8, +9)
+  float acc[KT][4];    // D[channel][head]: (channel gid, heads 2 tig, 2 tig + 1), channel + 8
+  float vb[4];         // D[value group][head]
+  float m_run, m_lim, l_run;  // head gid
+
+  __device__ __forceinline__ void init(const QArgs& a, int b, int h, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const bool hv = gid < a.g;
+    const __nv_bfloat16* qp = a.q + (static_cast<size_t>(b) * a.Hq + h * a.g + (hv ? gid : 0)) * D;
+#pragma unroll
+    for (int kt = 0; kt < KT; ++kt) {
+      const float f = pow2i(-BITS * (kt % TPW));
+      const float2 lo = unpack_bf2(*reinterpret_cast<const uint32_t*>(qp + kt * 16 + 2 * tig));
+      const float2 hi = unpack_bf2(*reinterpret_cast<const uint32_t*>(qp + kt * 16 + 8 + 2 * tig));
+      q2[kt][0] = hv ? pack_h2(lo.x * f, lo.y * f) : 0u;
+      q2[kt][1] = hv ? pack_h2(hi.x * f, hi.y * f) : 0u;
+    }
+#pragma unroll
+    for (int mc = 0; mc < KT; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
+    vb[0] = vb[1] = vb[2] = vb[3] = 0.f;
+    m_run = -INFINITY;
+    m_lim = -INFINITY;
+    l_run = 0.f;
+  }
+
+  __device__ __forceinline__ void group(const unsigned char* rs, int lane, float scl, float sl2) {
+    constexpr unsigned FULL = 0xffffffffu;
+    using C = QCfg<BITS, G, D, 2>;
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t* kcw = reinterpret_cast<const uint32_t*>(rs);
+    const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
+    const uint4* skw = reinterpret_cast<const uint4*>(rs + C::OFF_SK) + tig * (KT / 2);
+    const uint4* zkw = reinterpret_cast<const uint4*>(rs + C::OFF_ZK) + tig * (KT / 2);
+    const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);
+    const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
+
+    // (1) scores, n-tile nt = tokens 8 nt .. 8 nt + 7: rows gid (high part of
+    //     head gid's q*s) and gid + 8 (its low part); zero-point term from
+    //     rows = q (unfolded) against the zeros broadcast over the columns
+    float sc[2 * MT][4], kb[4];
+#pragma unroll
+    for (int n = 0; n < 2 * MT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+    kb[0] = kb[1] = kb[2] = kb[3] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NW / 2; ++j) {
+      uint32_t fa[TPW][4];
+#pragma unroll
+      for (int i = 0; i < TPW; ++i) {
+        const int kt = TPW * j + i;
+        const uint4 s4 = skw[kt >> 1];
+        const uint32_t sA = (kt & 1) ? s4.z : s4.x, sC = (kt & 1) ? s4.w : s4.y;
+        fa[i][0] = hmul2(q2[kt][0], sA);
+        fa[i][1] = hfms2(q2[kt][0], sA, fa[i][0]);
+        fa[i][2] = hmul2(q2[kt][1], sC);
+        fa[i][3] = hfms2(q2[kt][1], sC, fa[i][2]);
+        const uint4 z4 = zkw[kt >> 1];
+        const uint32_t z0 = zscale<BITS>((kt & 1) ? z4.z : z4.x, i);
+        const uint32_t z8 = zscale<BITS>((kt & 1) ? z4.w : z4.y, i);
+        const uint32_t qa[4] = {q2[kt][0], 0u, q2[kt][1], 0u};
+        mma_f16(kb, qa, z0, z8);
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const uint2 w = *reinterpret_cast<const uint2*>(kcw + (mt * 32 + lane) * NW + 2 * j);
+        const uint32_t X = w.x, Y = w.y, XS = w.x >> 8, YS = w.y >> 8;
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+          const uint32_t m = F::mask(i);
+          mma_f16(sc[2 * mt], fa[i], X & m, Y & m);
+          mma_f16(sc[2 * mt + 1], fa[i], XS & m, YS & m);
+        }
+      }
+    }
+
+    // (2) softmax of head gid over tokens 8 n + 2 tig, +1
+    const float kzs = kb[0] * sl2;
+    float y[2 * MT][2];
+    float t = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < 2 * MT; ++n) {
+      y[n][0] = sc[n][0] + sc[n][2];
+      y[n][1] = sc[n][1] + sc[n][3];
+      t = fmaxf(t, fmaxf(y[n][0], y[n][1]));
+    }
+    t = fmaxf(t, __shfl_xor_sync(FULL, t, 1));
+    t = fmaxf(t, __shfl_xor_sync(FULL, t, 2));
+    t = fmaf(t, scl, kzs);
+    if (__any_sync(FULL, t > m_lim)) {
+      const float m_new = fmaxf(m_run, t);
+      const float alpha = ex2(m_run - m_new);
+      m_run = m_new;
+      m_lim = m_new + kLazy;
+      l_run *= alpha;
+      // acc and vb columns are heads 2 tig, 2 tig + 1: fetch their factors
+      const float a0 = __shfl_sync(FULL, alpha, 8 * tig);
+      const float a1 = __shfl_sync(FULL, alpha, 8 * tig + 4);
+#pragma unroll
+      for (int mc = 0; mc < KT; ++mc) {
+        acc[mc][0] *= a0;
+        acc[mc][1] *= a1;
+        acc[mc][2] *= a0;
+        acc[mc][3] *= a1;
+      }
+      vb[0] *= a0;
+      vb[1] *= a1;
+      vb[2] *= a0;
+      vb[3] *= a1;
+    }
+    const float off = kzs - m_run;
+    uint32_t P[2 * MT];
+#pragma unroll
+    for (int n = 0; n < 2 * MT; ++n) {
+      const float p0 = ex2(fmaf(y[n][0], scl, off)), p1 = ex2(fmaf(y[n][1], scl, off));
+      l_run += p0 + p1;
+      P[n] = pack_h2(p0, p1);
+    }
+
+    // (3) P . V: B = p~ * s of head gid for tokens (2 tig, +1) and (2 tig + 8, +9),
+    //     high part and exact low part as two MMAs into the same accumulator
+#pragma unroll
+    for (int ktt = 0; ktt < MT; ++ktt) {
+      uint32_t s01[CPG], s89[CPG];
+      load_cpg<CPG>(sv32 + (ktt * 8 + tig) * CPG, s01);
+      load_cpg<CPG>(sv32 + (ktt * 8 + 4 + tig) * CPG, s89);
+      {
+        uint32_t za[4] = {0u, 0u, 0u, 0u};
+        if (gid < CPG) {
+          za[0] = zv32[(ktt * 8 + tig) * CPG + gid];
+          za[2] = zv32[(ktt * 8 + 4 + tig) * CPG + gid];
+        }
+        mma_f16(vb, za, P[2 * ktt], P[2 * ktt + 1]);
+      }
+      uint32_t h0 = 0u, h1 = 0u, l0 = 0u, l1 = 0u;
+#pragma unroll
+      for (int j = 0; j < NW / 2; ++j) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vcw + (ktt * 32 + lane) * NW + 2 * j);
+        const uint32_t X = w.x, Y = w.y, XS = w.x >> 8, YS = w.y >> 8;
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+          const int mc = TPW * j + i;
+          const int cg = mc * 16 / G;
+          if (mc == 0 || (mc - 1) * 16 / G != cg) {
+            h0 = hmul2(P[2 * ktt], s01[cg]);
+            l0 = hfms2(P[2 * ktt], s01[cg], h0);
+            h1 = hmul2(P[2 * ktt + 1], s89[cg]);
+            l1 = hfms2(P[2 * ktt + 1], s89[cg], h1);
+          }
+          const uint32_t m = F::mask(i);
+          const uint32_t af[4] = {X & m, Y & m, XS & m, YS & m};
+          mma_f16(acc[mc], af, h0, h1);
+          mma_f16(acc[mc], af, l0, l1);
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void store(const QArgs& a, int warp, int lane, bool ok, float* st_o, float* st_ml) {
+    constexpr unsigned FULL = 0xffffffffu;
+    const int gid = lane >> 2, tig = lane & 3;
+    float l = l_run;
+    l += __shfl_xor_sync(FULL, l, 1);
+    l += __shfl_xor_sync(FULL, l, 2);
+    const int h0 = 2 * tig, h1 = 2 * tig + 1;
+#pragma unroll
+    for (int mc = 0; mc < KT; ++mc) {
+      const int cg = mc * 16 / G;
+      const float zb0 = __shfl_sync(FULL, vb[0], cg * 4 + tig);
+      const float zb1 = __shfl_sync(FULL, vb[1], cg * 4 + tig);
+      const float uf = pow2i(24 - BITS * (mc % TPW));
+      if (h0 < a.g) {
+        float* wo = st_o + (warp * HEADS + h0) * D + mc * 16 + gid;
+        wo[0] = acc[mc][0] * uf + zb0;
+        wo[8] = acc[mc][2] * uf + zb0;
+      }
+      if (h1 < a.g) {
+        float* wo = st_o + (warp * HEADS + h1) * D + mc * 16 + gid;
+        wo[0] = acc[mc][1] * uf + zb1;
+        wo[8] = acc[mc][3] * uf + zb1;
+      }
+    }
+    if (gid < a.g && tig == 0) {
+      st_ml[(warp * HEADS + gid) * 2] = ok ? m_run : -INFINITY;
+      st_ml[(warp * HEADS + gid) * 2 + 1] = ok ? l : 0.f;
+    }
+  }
+};
+
+// Processes this warp's stages of unit u's quantised segment (the prefetch
+// pipeline runs on across segments) and leaves the warp's state in its slot.
+template <int BITS, int G, int D, int NT>
+__device__ __forceinline__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, int u, int64_t qs0,
+                                          int my_nq, int& iq, int& issued, IssuePtr& ip, int& islot, int& cslot,
+                                          uint32_t& cphase, bool& ok, float* st_o, float* st_ml) {
+  using C = QCfg<BITS, G, D, NT>;
+  using Body = std::conditional_t<NT == 1, TokM<BITS, G, D>, HeadM<BITS, G, D>>;
+  constexpr unsigned FULL = 0xffffffffu;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = u / a.Hkv, h = u - b * a.Hkv;
   // the score MMAs accumulate scores * 2^-24; undo it together with the softmax scale
   const float scl = a.scale_log2 * 16777216.0f;
-
-  float acc[C::KT][NT][4];
-  float vb[NT][4];
-  float m_run[NT], l_run[NT];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    m_run[nt] = -INFINITY;
-    l_run[nt] = 0.f;
-    vb[nt][0] = vb[nt][1] = vb[nt][2] = vb[nt][3] = 0.f;
-#pragma unroll
-    for (int mc = 0; mc < C::KT; ++mc) acc[mc][nt][0] = acc[mc][nt][1] = acc[mc][nt][2] = acc[mc][nt][3] = 0.f;
-  }
+  Body body;
+  body.init(a, b, h, lane);
 
   // this warp's stages of the segment: local stages ls0, ls0 + kQNW, ...
   // (qs: index inside the quantised zone; this warp's i-th one is qs0 + kQNW i)
@@ -299,6 +693,7 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
       ls0 = static_cast<int>(s_first - seg_lo);
     }
   }
+#pragma unroll 1
   for (int kk = 0; kk < n_seg; ++kk, ++iq) {
     if (!ok) continue;
     if (issued < my_nq && issued <= iq + C::NST - 1) {
@@ -318,219 +713,17 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
       for (int k = iq; k < issued; ++k) mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
       continue;
     }
-    const int64_t g0 = static_cast<int64_t>(ls0 + kk * kQNW) * C::NG;
-    const int n_here = a.P.ng - g0 < C::NG ? static_cast<int>(a.P.ng - g0) : C::NG;
+    if constexpr (C::NG == 1) {
+      body.group(ring + slot * C::STAGE, lane, scl, a.scale_log2);
+    } else {
+      const int64_t g0 = static_cast<int64_t>(ls0 + kk * kQNW) * C::NG;
+      const int n_here = a.P.ng - g0 < C::NG ? static_cast<int>(a.P.ng - g0) : C::NG;
 #pragma unroll 1
-    for (int gi = 0; gi < (C::NG == 1 ? 1 : n_here); ++gi) {
-      const unsigned char* rs = ring + slot * C::STAGE + gi * C::REC;
-      const uint32_t* kcw = reinterpret_cast<const uint32_t*>(rs);
-      const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
-      const uint4* skw = reinterpret_cast<const uint4*>(rs + C::OFF_SK) + tig * (C::KT / 2);
-      const uint4* zkw = reinterpret_cast<const uint4*>(rs + C::OFF_ZK) + tig * (C::KT / 2);
-      const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);  // [G/2][CPG] token pairs
-      const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
-
-      // (1) scores of the group's MT token tiles in one pass over the channel
-      //     tiles kt.  Per kt the key scales are folded into q right before
-      //     use (fp16 high part in part-0 columns, low part in part-1
-      //     columns); lane tig's scale words for (kt, h) are word 2kt + h of
-      //     its run.  The zero-point term sum_c q_c z_c comes from the zeros
-      //     times 2^(bits i) (exact) against q2s, in both columns of a head
-      //     (only the high one is used).
-      float sc[MT][NT][4];
-      float kb[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        kb[nt][0] = kb[nt][1] = kb[nt][2] = kb[nt][3] = 0.f;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) sc[mt][nt][0] = sc[mt][nt][1] = sc[mt][nt][2] = sc[mt][nt][3] = 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < NW / 2; ++j) {
-        uint2 w[MT];
-        uint32_t xs[MT], ys[MT];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          w[mt] = *reinterpret_cast<const uint2*>(kcw + (mt * 32 + lane) * NW + 2 * j);
-          xs[mt] = w[mt].x >> 8;
-          ys[mt] = w[mt].y >> 8;
-        }
-#pragma unroll
-        for (int i = 0; i < F::TPW; ++i) {
-          const int kt = F::TPW * j + i;
-          const uint4 s4 = skw[kt >> 1];
-          const uint32_t sA = (kt & 1) ? s4.z : s4.x, sC = (kt & 1) ? s4.w : s4.y;
-          const uint32_t m = F::mask(i);
-          uint32_t fa[NT], fc[NT];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const uint32_t qa = q2s[kt][nt][0], qc = q2s[kt][nt][1];
-            fa[nt] = hfma2(qa, sA, hmul2(hmul2(qa, sA), kap));
-            fc[nt] = hfma2(qc, sC, hmul2(hmul2(qc, sC), kap));
-          }
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            const uint32_t af[4] = {w[mt].x & m, xs[mt] & m, w[mt].y & m, ys[mt] & m};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_f16(sc[mt][nt], af, fa[nt], fc[nt]);
-          }
-          const uint4 z4 = zkw[kt >> 1];
-          uint32_t z0 = (kt & 1) ? z4.z : z4.x, z8 = (kt & 1) ? z4.w : z4.y;
-          if (i > 0) {
-            const uint32_t f2 = static_cast<uint32_t>(15 + BITS * i) << 10;  // fp16 2^(bits i)
-            z0 = hmul2(z0, f2 | (f2 << 16));
-            z8 = hmul2(z8, f2 | (f2 << 16));
-          }
-          const uint32_t za[4] = {z0, z0, z8, z8};
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_f16(kb[nt], za, q2s[kt][nt][0], q2s[kt][nt][1]);
-        }
-      }
-
-      // (2) softmax per head nt*4 + tig over the lane's tokens 16 mt + gid (+8);
-      //     the running max is raised only when a score exceeds it by more
-      //     than 2^8 (lazy rescale; p <= 256 keeps every fp16/fp32 value in range)
-      float x[NT][2 * MT], tmax[NT];
-      bool need = false;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const float kz = kb[nt][0] * 5.9604644775390625e-8f;  // zero-point term in the 2^-24 domain
-        float t = -INFINITY;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          x[nt][2 * mt] = (sc[mt][nt][0] + sc[mt][nt][1] + kz) * scl;
-          x[nt][2 * mt + 1] = (sc[mt][nt][2] + sc[mt][nt][3] + kz) * scl;
-          t = fmaxf(t, fmaxf(x[nt][2 * mt], x[nt][2 * mt + 1]));
-        }
-        t = warp_max_xor(t, 4);
-        t = warp_max_xor(t, 8);
-        t = warp_max_xor(t, 16);
-        tmax[nt] = t;
-        need |= t > m_run[nt] + 8.f;
-      }
-      if (__any_sync(FULL, need)) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const float m_new = fmaxf(m_run[nt], tmax[nt]);
-          const float alpha = ex2(m_run[nt] - m_new);
-          m_run[nt] = m_new;
-          l_run[nt] *= alpha;
-#pragma unroll
-          for (int mc = 0; mc < C::KT; ++mc) {
-            acc[mc][nt][0] *= alpha;
-            acc[mc][nt][1] *= alpha;
-            acc[mc][nt][2] *= alpha;
-            acc[mc][nt][3] *= alpha;
-          }
-          vb[nt][0] *= alpha;
-          vb[nt][1] *= alpha;
-          vb[nt][2] *= alpha;
-          vb[nt][3] *= alpha;
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        unsigned short* ph = reinterpret_cast<unsigned short*>(Ph + (nt * 4 + tig) * G + gid);
-        unsigned short* pl = reinterpret_cast<unsigned short*>(Pl + (nt * 4 + tig) * G + gid);
-        float ls = 0.f;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const float p0 = ex2(x[nt][2 * mt] - m_run[nt]), p1 = ex2(x[nt][2 * mt + 1] - m_run[nt]);
-          ls += p0 + p1;
-          // p as fp16 high + low parts (tokens 16mt + gid and +8), split once for the value side
-          const uint32_t hh = pack_h2(p0, p1);
-          const float2 f = unpack_h2(hh);
-          const uint32_t ll = pack_h2(p0 - f.x, p1 - f.y);
-          ph[16 * mt] = static_cast<unsigned short>(hh);
-          ph[16 * mt + 8] = static_cast<unsigned short>(hh >> 16);
-          pl[16 * mt] = static_cast<unsigned short>(ll);
-          pl[16 * mt + 8] = static_cast<unsigned short>(ll >> 16);
-        }
-        l_run[nt] += ls;
-      }
-      __syncwarp();
-
-      // (3) P . V over the group's MT token tiles
-#pragma unroll
-      for (int ktt = 0; ktt < MT; ++ktt) {
-        const int t0 = ktt * 16 + 2 * tig;  // tokens t0, t0+1, t0+8, t0+9
-        uint32_t ph01[NT], ph89[NT], plm01[NT], plm89[NT], phn01[NT], phn89[NT];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int hh = nt * 4 + (gid >> 1);
-          ph01[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0);
-          ph89[nt] = *reinterpret_cast<const uint32_t*>(Ph + hh * G + t0 + 8);
-          const uint32_t pl01 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0);
-          const uint32_t pl89 = *reinterpret_cast<const uint32_t*>(Pl + hh * G + t0 + 8);
-          plm01[nt] = hmul2(pl01, mu);
-          plm89[nt] = hmul2(pl89, mu);
-          phn01[nt] = hmul2(ph01[nt], kap);
-          phn89[nt] = hmul2(ph89[nt], kap);
-          // value zero-point term: A = z_v^T (row = value group gid), B = p (high or low column)
-          uint32_t za[4] = {0u, 0u, 0u, 0u};
-          if (gid < C::CPG) {
-            za[0] = zv32[(t0 >> 1) * C::CPG + gid];
-            za[2] = zv32[((t0 + 8) >> 1) * C::CPG + gid];
-          }
-          mma_f16(vb[nt], za, part ? pl01 : ph01[nt], part ? pl89 : ph89[nt]);
-        }
-        // folded p*s per value group, made right before the channel tiles
-        // that use it: high part (part 0) or low part (part 1)
-        uint32_t s01[C::CPG], s89[C::CPG];
-        load_cpg<C::CPG>(sv32 + (t0 >> 1) * C::CPG, s01);
-        load_cpg<C::CPG>(sv32 + ((t0 + 8) >> 1) * C::CPG, s89);
-        uint32_t wv[NW];
-        load_words(vcw + (ktt * 32 + lane) * NW, wv);
-        uint32_t pf[NT][2];
-#pragma unroll
-        for (int j = 0; j < NW / 2; ++j) {
-          const uint32_t X = wv[2 * j], Y = wv[2 * j + 1], xsv = X >> 8, ysv = Y >> 8;
-#pragma unroll
-          for (int i = 0; i < F::TPW; ++i) {
-            const int mc = F::TPW * j + i;  // 16-channel tile
-            const int cg = mc * 16 / G;
-            if (mc == 0 || (mc - 1) * 16 / G != cg) {
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                pf[nt][0] = hfma2(plm01[nt], s01[cg], hfma2(ph01[nt], s01[cg], hmul2(phn01[nt], s01[cg])));
-                pf[nt][1] = hfma2(plm89[nt], s89[cg], hfma2(ph89[nt], s89[cg], hmul2(phn89[nt], s89[cg])));
-              }
-            }
-            const uint32_t af[4] = {X & F::mask(i), Y & F::mask(i), xsv & F::mask(i), ysv & F::mask(i)};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_f16(acc[mc][nt], af, pf[nt][0], pf[nt][1]);
-          }
-        }
-      }
-      __syncwarp();
+      for (int gi = 0; gi < n_here; ++gi) body.group(ring + slot * C::STAGE + gi * C::REC, lane, scl, a.scale_log2);
     }
+    __syncwarp();
   }
-
-  // ---- this warp's state -> its slot, natural channel order
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int hh = nt * 4 + tig;
-    float l = l_run[nt];
-    l += __shfl_xor_sync(FULL, l, 4);
-    l += __shfl_xor_sync(FULL, l, 8);
-    l += __shfl_xor_sync(FULL, l, 16);
-    const float vbs = vb[nt][0] + vb[nt][1];  // value-zero term of group gid, head hh
-#pragma unroll
-    for (int mc = 0; mc < C::KT; ++mc) {
-      const int cg = mc * 16 / G;
-      const float zb = __shfl_sync(FULL, vbs, cg * 4 + tig);
-      const float uf = pow2i(24 - BITS * (mc % F::TPW));  // undo the code encoding of this tile
-      if (hh < a.g) {
-        float* wo = st_o + (warp * C::HEADS + hh) * D + mc * 16 + gid;
-        wo[0] = (acc[mc][nt][0] + acc[mc][nt][1]) * uf + zb;
-        wo[8] = (acc[mc][nt][2] + acc[mc][nt][3]) * uf + zb;
-      }
-    }
-    if (hh < a.g && gid == 0) {
-      st_ml[(warp * C::HEADS + hh) * 2] = ok ? m_run[nt] : -INFINITY;
-      st_ml[(warp * C::HEADS + hh) * 2 + 1] = ok ? l : 0.f;
-    }
-  }
+  body.store(a, warp, lane, ok, st_o, st_ml);
 }
 
 // -------------------------------------------------------- bf16 residual part
@@ -538,7 +731,7 @@ __device__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, i
 // not pipelined; the residual is a few percent of the bytes).  Leaves the
 // warp's state in its slot.
 template <int D, int NT, int HEADS>
-__device__ __noinline__ void residual_seg(const QArgs& a, unsigned char* ring, float* P_s, uint64_t* bar, int& rph, int u,
+__device__ __forceinline__ void residual_seg(const QArgs& a, unsigned char* ring, float* P_s, uint64_t* bar, int& rph, int u,
                              int64_t first_s, int64_t end_s, int64_t seg_b, bool& ok, float* st_o, float* st_ml) {
   constexpr int KT = D / 16;
   constexpr int ROW_B = D * 2;
@@ -846,7 +1039,7 @@ __global__ void __launch_bounds__(128) combine_kernel(CArgs a) {
 }
 
 template <int BITS, int G, int D, int NT>
-__global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kernel(QArgs a) {
+__global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 3)) draft_quant_kernel(QArgs a) {
   using C = QCfg<BITS, G, D, NT>;
   extern __shared__ __align__(128) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -859,7 +1052,7 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
   if (B0 >= B1) return;  // the host sizes the grid so that this never happens
   const int seg0 = P.seg_of(B0), seg1 = P.seg_of(B1 - 1);
   unsigned char* ring = smem + warp * C::WARP_B;
-  float* P_res = reinterpret_cast<float*>(ring + C::RING);  // residual scores share the p buffer
+  float* P_res = reinterpret_cast<float*>(ring + C::RING);  // residual tile scores
   float* st_o = reinterpret_cast<float*>(smem + C::STATE_OFF);
   float* st_ml = reinterpret_cast<float*>(smem + C::ML_OFF);
   float* mw = reinterpret_cast<float*>(smem + C::MW_OFF);
@@ -1242,9 +1435,12 @@ vc_status vc_debug_quant_partition(const vc_attn_shape* shape, const vc_quant_ca
 //
 // The array's address is looked up once per device, with that device
 // current, on the first call made on it (cudaGetSymbolAddress); make that
-// first call before any stream capture.  Every call shares the one array:
-// each call clears the words that must start at zero, and calls that
-// overlap on the GPU (other streams, other host threads) race on it.
+// first call before any stream capture.  Every call shares the one array,
+// and calls that overlap on the GPU (other streams, other host threads) race
+// on it.  Only its flag word must start at zero: a device array is zero when
+// the module loads, kernels only OR bits into the word, and
+// vc_draft_attn_quant_noalloc_flags reads and clears it, so a timed-out call
+// stays visible until the caller asks.  The block partials need no clearing.
 namespace vc {
 namespace {
 
@@ -1296,14 +1492,26 @@ vc_status vc_draft_attn_quant_noalloc(const vc_attn_shape* shape, const vc_quant
   st = vc::noalloc_scratch(&scratch);
   if (st != VC_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the flag word must start at zero; partials need no clearing
-  if (cudaMemsetAsync(scratch, 0, p.off_ml, s) != cudaSuccess)
-    return vc::set_error(VC_ERR_CUDA, "vc_draft_attn_quant_noalloc: clearing the scratch failed: %s",
-                         cudaGetErrorString(cudaGetLastError()));
   vc::QArgs a = vc::make_args(*shape, *cache, q);
   vc::bind_scratch(a, p, scratch, out);
   vc::launch_quant(*shape, *cache, a, p, s);
   return vc::launch_status("vc_draft_attn_quant_noalloc");
+}
+
+vc_status vc_draft_attn_quant_noalloc_flags(uint32_t* host_flags, void* stream) {
+  VC_REQUIRE(host_flags != nullptr, "vc_draft_attn_quant_noalloc_flags: null output");
+  void* scratch = nullptr;
+  vc_status st = vc::noalloc_scratch(&scratch);
+  if (st != VC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, scratch, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemsetAsync(scratch, 0, sizeof(uint32_t), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+    return vc::set_error(VC_ERR_CUDA, "vc_draft_attn_quant_noalloc_flags: %s",
+                         cudaGetErrorString(cudaGetLastError()));
+  *host_flags = v;
+  vc::clear_error();
+  return VC_OK;
 }
 
 }  // extern "C"

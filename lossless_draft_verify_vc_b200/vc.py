@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
             "vc_accept": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_size_t, c_void_p]),
             "vc_workspace_flags": (c_int, [c_void_p, c_size_t, P(c_uint32), c_void_p]),
+            "vc_draft_attn_quant_noalloc_flags": (c_int, [P(c_uint32), c_void_p]),
             "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
             "vc_debug_quant_partition": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_int, c_void_p, c_int,
                                                  P(c_int), P(c_int), P(c_int64), P(c_int64)]),
@@ -229,6 +230,14 @@ def vc_accept(logits, B: int, K: int, V: int, draft, target, accept_len, correct
 def vc_workspace_flags(ws, stream=None) -> int:
     v = c_uint32(0)
     _check(lib().vc_workspace_flags(_p(ws), ws.numel(), ctypes.byref(v), _stream(stream)))
+    return int(v.value)
+
+
+def vc_draft_attn_quant_noalloc_flags(stream=None) -> int:
+    """Flags set by vc_draft_attn_quant_noalloc calls on the current device
+    since the last read (read and cleared)."""
+    v = c_uint32(0)
+    _check(lib().vc_draft_attn_quant_noalloc_flags(ctypes.byref(v), _stream(stream)))
     return int(v.value)
 
 

@@ -21,16 +21,18 @@ pytestmark = pytest.mark.gpu
 dev = "cuda"
 
 
-def _inputs(seed, B=2, Hq=8, Hkv=2, D=128, T=32 * 40 + 128, R=128):
+def _inputs(seed, B=2, Hq=8, Hkv=2, D=128, T=32 * 40 + 128, R=128, bits=2, G=32):
     k, v = synth.kv_full(B, Hkv, T, D, seed=seed)
-    cache = Q.build_quant_cache(np32(k), np32(v), 2, 32, R)
+    cache = Q.build_quant_cache(np32(k), np32(v), bits, G, R)
     q = synth.normal((B, Hq, D), seed=seed + 1)
     return cache, quant_cache_to_torch(cache, dev), q.to(dev), vc.shape(B, Hq, Hkv, D)
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
+@pytest.mark.parametrize("cfg", [dict(), dict(Hq=16, T=64 * 24 + 100, R=100, bits=4, G=64)],
+                         ids=["2bit-g32-gqa4", "4bit-g64-gqa8"])
+def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row(cfg):
     for seed in (101, 202):
-        cache, tc, q, sh = _inputs(seed)
+        cache, tc, q, sh = _inputs(seed, **cfg)
         qc = vc.quant_cache(tc)
         ws = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, qc))
         ref = torch.empty(q.shape, device=dev)
@@ -40,6 +42,24 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
         torch.cuda.synchronize()
         assert row_rel_err(np32(got), np32(ref)) <= ATTN_TOL
         assert row_rel_err(np32(got), A.draft_attention_quant(np32(q), cache)) <= ATTN_TOL
+    # no bounded wait gave up in these calls
+    assert vc.vc_draft_attn_quant_noalloc_flags() == 0
+
+
+def test_noalloc_calls_allocate_nothing():
+    cache, tc, q, sh = _inputs(303)
+    qc = vc.quant_cache(tc)
+    out = torch.empty(q.shape, device=dev)
+    vc.vc_draft_attn_quant_noalloc(sh, qc, q, out)  # first call: looks up the scratch array
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    reserved0 = torch.cuda.memory_reserved()
+    for _ in range(20):
+        vc.vc_draft_attn_quant_noalloc(sh, qc, q, out)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_reserved() == reserved0
 
 
 def test_noalloc_refuses_a_call_larger_than_its_scratch():
