@@ -396,16 +396,20 @@ VC_API vc_status vc_debug_gather(const vc_attn_shape* shape, const vc_sparse_cac
 
 /* vc_debug_quant_partition reports, without touching a GPU, how
  * vc_draft_attn_quant cuts one call into blocks when at most target_blocks
- * blocks are allowed (the real call uses SMs x resident blocks).  The call is
- * one axis of stages: every (request, head) unit's residual rows, 16 per
- * stage, then every unit's quantised groups (n_quant_stages of the n_stages
- * stages).  Block k owns stages [first_stage[k], first_stage[k+1]);
- * *max_segments is the most unit parts (quantised or residual part of one
- * unit) one block touches.  first_stage may be NULL; else it needs
- * max_blocks >= *n_blocks + 1 entries. */
+ * blocks are allowed (the real call uses SMs x resident blocks).  Each
+ * (request, KV head) unit is an axis of *residual_tiles tiles of 16 residual
+ * rows followed by *quant_stages quantised stages.  With
+ * *blocks_per_unit >= 1 every unit is cut into that many contiguous pieces of
+ * equal cost, one per block; with *blocks_per_unit == 0 (more units than
+ * blocks) each block takes whole units.  Every unit ends up in
+ * *partials_per_unit block partials.  block_ranges may be NULL; else it
+ * needs max_blocks >= *n_blocks rows of six int32: first unit, end unit,
+ * residual tiles [r0, r1) and quantised stages [q0, q1) of that block
+ * (unit-local indices, the same for every unit of the block). */
 VC_API vc_status vc_debug_quant_partition(const vc_attn_shape* shape, const vc_quant_cache* cache,
-                                          int target_blocks, int64_t* first_stage, int max_blocks, int* n_blocks,
-                                          int* max_segments, int64_t* n_stages, int64_t* n_quant_stages);
+                                          int target_blocks, int32_t* block_ranges, int max_blocks, int* n_blocks,
+                                          int* blocks_per_unit, int* partials_per_unit, int* residual_tiles,
+                                          int* quant_stages);
 
 #ifdef __cplusplus
 }

@@ -49,7 +49,12 @@ namespace {
 
 constexpr int kQNW = 4;          // warps per block
 constexpr int kResRows = 16;     // residual rows per stage
-constexpr int kResCostWeight = 2;  // residual stages are not pipelined: count their bytes twice
+// A residual tile (16 bf16 K and V rows, fetched without a pipeline, so its
+// time is mostly one memory round trip) costs about 4/3 of its bytes in
+// quantised-stage bytes (measured on B200: a tile takes the time of ~3.6
+// 2-bit group-32 records)
+constexpr int kResCostNum = 4, kResCostDen = 3;
+constexpr int kMergeFloats = 512;  // shared-memory area of the final per-unit merge (2 KB)
 
 template <int BITS, int G, int D, int NT>
 struct QCfg {
@@ -60,70 +65,110 @@ struct QCfg {
   static constexpr int OFF_ZK = 2 * CB + 2 * D;
   static constexpr int OFF_SV = 2 * CB + 4 * D;
   static constexpr int OFF_ZV = 2 * CB + 6 * D;
-  static constexpr int NG = REC >= 3072 ? 1 : 3072 / REC;  // records per stage
+  static constexpr int HEADS = 4 * NT;
+  static constexpr int STATE_W = HEADS * D * 4;  // one warp's unnormalised o, fp32 [HEADS][D]
+  static constexpr int NG0 = REC >= 3072 ? 1 : 3072 / REC;
+  // records per stage (a stage slot also holds a warp's state at a segment end)
+  static constexpr int NG = NG0 * REC >= STATE_W ? NG0 : (STATE_W + REC - 1) / REC;
   static constexpr int STAGE = NG * REC;
-  static constexpr int NST0 = (NT == 1 ? 9216 : 18432) / STAGE;
-  static constexpr int NST = NST0 < 2 ? 2 : (NST0 > 4 ? 4 : NST0);  // ring depth
-  static constexpr int RSTAGE = 2 * kResRows * D * 2;                // 16 K + 16 V bf16 rows
+  static constexpr bool PIPE = NT == 1 && NG == 1;  // software-pipelined group loop (TokM)
+  static constexpr int NST0 = (PIPE ? 12288 : 18432) / STAGE;
+  static constexpr int NMIN = PIPE ? 3 : 2;
+  static constexpr int NST = NST0 < NMIN ? NMIN : (NST0 > 4 ? 4 : NST0);  // ring depth
+  static constexpr int RSTAGE = 2 * kResRows * D * 2;                      // 16 K + 16 V bf16 rows
+  // the ring also holds a residual tile; a warp's residual state is written over
+  // its last tile once that is consumed
   static constexpr int RING0 = NST * STAGE > RSTAGE ? NST * STAGE : RSTAGE;
   static constexpr int RING = (RING0 + 127) / 128 * 128;
-  static constexpr int HEADS = 4 * NT;
   static constexpr int RP_B = HEADS * kResRows * 4;  // residual tile scores, fp32 [HEADS][16]
   static constexpr int WARP_B = RING + RP_B;
-  static constexpr int STATE_OFF = kQNW * WARP_B;                       // fp32 [kQNW][HEADS][D]
-  static constexpr int ML_OFF = STATE_OFF + kQNW * HEADS * D * 4;       // fp32 [kQNW][HEADS][2]
-  static constexpr int MW_OFF = ML_OFF + kQNW * HEADS * 2 * 4;          // merge weights + (M, L)
+  static constexpr int ML_OFF = kQNW * WARP_B;                  // fp32 [kQNW][HEADS][2]
+  static constexpr int SO_OFF = ML_OFF + kQNW * HEADS * 2 * 4;  // int [kQNW]: where each warp's state is
+  static constexpr int MW_OFF = SO_OFF + kQNW * 4;              // merge weights + (M, L)
   static constexpr int MW_FLOATS = kQNW * HEADS + 2 * HEADS;
-  static constexpr int BAR_OFF = (MW_OFF + MW_FLOATS * 4 + 15) / 16 * 16;
+  static constexpr int MA_OFF = (MW_OFF + MW_FLOATS * 4 + 15) / 16 * 16;  // unit merge area
+  // block-shared query fragments of TokM (all warps of a block work on one
+  // unit at a time): uint4 [KT][32 lanes]
+  static constexpr int QSM_OFF = MA_OFF + kMergeFloats * 4;
+  static constexpr int QSM_B = NT == 1 ? (D / 16) * 32 * 16 : 0;
+  static constexpr int FLAG_OFF = QSM_OFF + QSM_B;
+  static constexpr int BAR_OFF = (FLAG_OFF + 4 + 15) / 16 * 16;
   static constexpr int SMEM_B = BAR_OFF + kQNW * (NST + 1) * 8;
   static constexpr int KT = D / 16;   // channel tiles
   static constexpr int CPG = D / G;   // value groups per token
   static_assert(G % 32 == 0, "group must be a multiple of 32");
   static_assert(REC % 16 == 0 && STAGE % 16 == 0, "bulk copies need 16-byte multiples");
+  static_assert(STAGE >= STATE_W, "a stage slot holds a warp state");
+  static_assert(RSTAGE >= STATE_W, "a residual tile area holds a warp state");
   static_assert(WARP_B % 128 == 0, "warp areas stay 128-byte aligned");
 };
 
-// The stage axis and its cut into blocks; the same arithmetic runs on the
-// host (planning, workspace size) and on the device.
-//   stage s <  RZ : residual stage s % sr of unit s / sr            (cost cr)
-//   stage s >= RZ : quantised stage (s - RZ) % sq of unit (s - RZ) / sq (cost cq)
-// The residual zone comes first so that a unit's last partial (whose block
-// finishes the unit) comes from the quantised zone, spread over many blocks.
-// Block k owns the stages whose start cost c_s satisfies
-// ceil(k C / n) <= c_s < ceil((k + 1) C / n); equivalently the block of stage
-// s is floor(c_s n / C).  The host keeps n <= C / max(cq, cr), so every block
-// owns at least one stage.  Segments along the axis: the residual part of
-// unit u (id u), then the quantised part of unit u (id U + u).
-struct Partition {
+// The work of one call and its cut into blocks; the same arithmetic runs on
+// the host (planning, workspace size) and on the device.  Unit u (one
+// request's KV head) is an axis of sr residual tiles (16 bf16 rows each,
+// cost cr) followed by sq quantised stages (NG group records each, cost cq).
+//  * bpu >= 1 (at most as many units as blocks): every unit is cut into bpu
+//    contiguous pieces of equal cost (piece j starts at axis index A(j),
+//    the first index whose start cost is >= ceil(j Cu / bpu)); block k owns
+//    piece k % bpu of unit k / bpu.  The host keeps bpu <= Cu / max(cq, cr),
+//    so no piece is empty.
+//  * bpu == 0 (more units than blocks): block k owns the whole units
+//    [k U / nblk, (k + 1) U / nblk).
+// A block's work on one unit is at most two segments, its residual tiles and
+// its quantised stages, each ending in one block partial.  Every unit has
+// the same partials: with bpu >= 1, the residual partials of pieces
+// 0 .. jr - 1 and the quantised partials of pieces jq .. bpu - 1
+// (np = jr + bpu - jq); with bpu == 0, one of each kind.
+struct UPart {
   int64_t ng;      // groups per unit
-  int64_t RZ;      // stages in the residual zone = U * sr
-  int64_t S_tot;   // all stages = RZ + U * sq
-  int64_t cq, cr;  // cost of one quantised / residual stage
-  int64_t C;       // total cost
-  int U, sq, sr, nblk;
+  int64_t cq, cr;  // cost of one quantised stage / residual tile
+  int U, sq, sr;   // units, quantised stages and residual tiles per unit
+  int bpu;         // blocks per unit (0: units per block >= 1)
+  int nblk;        // blocks in the grid
+  int upb;         // most units of one block (1 when bpu >= 1)
+  int jr, jq, np;  // pieces with residual / first piece with quantised stages / partials per unit
 
-  __host__ __device__ int64_t cost(int64_t s) const { return s < RZ ? s * cr : RZ * cr + (s - RZ) * cq; }
-  __host__ __device__ int64_t first(int k) const {
-    if (k <= 0) return 0;
-    if (k >= nblk) return S_tot;
-    const int64_t T = (static_cast<int64_t>(k) * C + nblk - 1) / nblk;
-    if (RZ > 0 && T <= (RZ - 1) * cr) return (T + cr - 1) / cr;
-    const int64_t base = RZ * cr;
-    if (T <= base) return RZ;
-    const int64_t s = RZ + (T - base + cq - 1) / cq;
-    return s < S_tot ? s : S_tot;
+  __host__ __device__ int64_t ucost() const { return static_cast<int64_t>(sr) * cr + static_cast<int64_t>(sq) * cq; }
+  // first unit-axis index of piece j (bpu >= 1)
+  __host__ __device__ int axis_first(int j) const {
+    if (j <= 0) return 0;
+    if (j >= bpu) return sr + sq;
+    const int64_t T = (static_cast<int64_t>(j) * ucost() + bpu - 1) / bpu;
+    if (sr > 0 && T <= static_cast<int64_t>(sr - 1) * cr) return static_cast<int>((T + cr - 1) / cr);
+    const int64_t base = static_cast<int64_t>(sr) * cr;
+    if (T <= base) return sr;
+    const int64_t s = sr + (T - base + cq - 1) / cq;
+    return s < sr + sq ? static_cast<int>(s) : sr + sq;
   }
-  __host__ __device__ int block_of(int64_t s) const {
-    const int64_t k = cost(s) * nblk / C;
-    return k < nblk ? static_cast<int>(k) : nblk - 1;
+  // units [u0, u1) and unit-local residual tiles [r0, r1) / quantised stages [q0, q1) of block k
+  __host__ __device__ void block_range(int k, int& u0, int& u1, int& r0, int& r1, int& q0, int& q1) const {
+    if (bpu > 0) {
+      u0 = k / bpu;
+      u1 = u0 + 1;
+      const int j = k - u0 * bpu;
+      const int a0 = axis_first(j), a1 = axis_first(j + 1);
+      r0 = a0 < sr ? a0 : sr;
+      r1 = a1 < sr ? a1 : sr;
+      q0 = a0 > sr ? a0 - sr : 0;
+      q1 = a1 > sr ? a1 - sr : 0;
+    } else {
+      u0 = static_cast<int>(static_cast<int64_t>(k) * U / nblk);
+      u1 = static_cast<int>(static_cast<int64_t>(k + 1) * U / nblk);
+      r0 = 0, r1 = sr, q0 = 0, q1 = sq;
+    }
   }
-  __host__ __device__ int seg_of(int64_t s) const {
-    return s < RZ ? static_cast<int>(s / sr) : U + static_cast<int>((s - RZ) / sq);
+  // slot of partial p (0 <= p < np) of unit u; a block's slots are
+  // k * 2 upb + 2 (unit - u0) + (0 residual, 1 quantised)
+  __host__ __device__ int64_t partial_slot(int u, int p) const {
+    if (bpu > 0) {
+      const int j = p < jr ? p : jq + (p - jr);
+      return 2 * (static_cast<int64_t>(u) * bpu + j) + (p < jr ? 0 : 1);
+    }
+    const int k = static_cast<int>((static_cast<int64_t>(u + 1) * nblk + U - 1) / U) - 1;
+    const int u0 = static_cast<int>(static_cast<int64_t>(k) * U / nblk);
+    const int kind = (sr > 0 && p == 0) ? 0 : 1;
+    return static_cast<int64_t>(k) * 2 * upb + 2 * (u - u0) + kind;
   }
-  __host__ __device__ int64_t seg_begin(int seg) const {
-    return seg < U ? static_cast<int64_t>(seg) * sr : RZ + static_cast<int64_t>(seg - U) * sq;
-  }
-  __host__ __device__ int64_t seg_end(int seg) const { return seg_begin(seg) + (seg < U ? sr : sq); }
 };
 
 struct QArgs {
@@ -131,12 +176,13 @@ struct QArgs {
   const __nv_bfloat16* kr;
   const __nv_bfloat16* vr;
   const __nv_bfloat16* q;
-  Partition P;
+  UPart P;
   int R, R_cap;
   int Hq, Hkv, g;
   int MAXS;  // partial slots per block
   float scale_log2;
   uint32_t* flags;
+  uint32_t* tickets;  // [U] partials of each unit written so far in this call (back to 0 after it)
   float* part_o;      // [nblk * MAXS][g][D]
   float* part_ml;     // [nblk * MAXS][g][2]
   float* out;         // [B][Hq][D]
@@ -196,35 +242,40 @@ __device__ __forceinline__ void load_cpg(const uint32_t* p, uint32_t (&w)[CPG]) 
   }
 }
 
-// Where this warp's next quantised stage to fetch lives: unit u, stage ls of
-// that unit (both < 2^31: units are capped at 2^24, groups per unit at 2^30).
-// Advancing by kQNW stages needs no division.
+// Where this warp's next quantised stage to fetch lives: unit u, unit-local
+// stage ls.  Warp w takes the stages q0 + w, q0 + w + kQNW, ... < q1 of each
+// of its block's units in turn.
 struct IssuePtr {
   int u, ls;
-  __device__ void start(const Partition& P, int64_t s) {
-    u = static_cast<int>(s / P.sq);
-    ls = static_cast<int>(s - static_cast<int64_t>(u) * P.sq);
-  }
-  __device__ void advance(const Partition& P) {
-    ls += kQNW;
-    while (ls >= P.sq) {
-      ls -= P.sq;
-      ++u;
-    }
-  }
+  const uint8_t* src;  // record of group ls * NG of unit u
 };
+
+template <typename C>
+__device__ __forceinline__ void issue_start(const QArgs& a, IssuePtr& ip, int u, int ls) {
+  ip.u = u;
+  ip.ls = ls;
+  ip.src = a.rec + (static_cast<int64_t>(u) * a.P.ng + static_cast<int64_t>(ls) * C::NG) * C::REC;
+}
+
+template <typename C>
+__device__ __forceinline__ void issue_advance(const QArgs& a, IssuePtr& ip, int q_first, int q_end) {
+  ip.ls += kQNW;
+  ip.src += kQNW * C::STAGE;
+  if (ip.ls >= q_end) issue_start<C>(a, ip, ip.u + 1, q_first);
+}
 
 // One bulk copy of this warp's next quantised stage (at ip) into ring slot `slot`.
 template <typename C>
 __device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring, uint64_t* bars, int lane, int slot,
                                             const IssuePtr& ip) {
-  const int64_t g0 = static_cast<int64_t>(ip.ls) * C::NG;
-  const int64_t left = a.P.ng - g0;
-  const uint32_t bytes = static_cast<uint32_t>((left < C::NG ? left : C::NG) * C::REC);
+  uint32_t bytes = C::STAGE;
+  if constexpr (C::NG > 1) {  // a unit's last stage may hold fewer groups
+    const int64_t left = a.P.ng - static_cast<int64_t>(ip.ls) * C::NG;
+    if (left < C::NG) bytes = static_cast<uint32_t>(left * C::REC);
+  }
   if (lane == 0) {
     mbar_arrive_expect_tx(&bars[slot], bytes);
-    bulk_g2s(ring + slot * C::STAGE, a.rec + (static_cast<int64_t>(ip.u) * a.P.ng + g0) * C::REC, bytes,
-             &bars[slot]);
+    bulk_g2s(ring + slot * C::STAGE, ip.src, bytes, &bars[slot]);
   }
 }
 
@@ -244,10 +295,17 @@ __device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring,
 //     needs, and no data moves between lanes.
 //
 // Both: values D[chan][col] = codes^T[chan][token] x pfold[token][col].
-// The softmax weights p (<= 2^kLazyLog2 by the lazy running maximum) are
+// The softmax weights p (<= 2^kLazy by the lazy running maximum) are
 // rounded once to fp16 (p~) for the value side; the softmax denominator
 // sums the fp32 p.  p~ * s is split into an fp16 high part and the exact
 // fp16 remainder (one fma), so the value operand carries ~22 bits.
+//
+// Each body has three steps per group: keys() (scores of the group into
+// registers), softmax() (running max and sum, weights in the value MMA's
+// operand layout) and values() (P . V into the accumulators).  TokM runs
+// them software-pipelined: values() of group j and keys() of group j + 1
+// form one straight-line block, so the long MMA and load latencies of one
+// overlap the other's independent work.
 
 constexpr float kLazy = 8.f;  // raise the running max only when a score exceeds it by > 2^8
 
@@ -277,15 +335,21 @@ __device__ __forceinline__ uint32_t zscale(uint32_t z, int i) {
 template <int BITS, int G, int D>
 struct TokM {
   using F = Frag<BITS>;
+  using C = QCfg<BITS, G, D, 1>;
   static constexpr int KT = D / 16, TPW = F::TPW, NW = 2 * KT / TPW, MT = G / 16, CPG = D / G;
   static constexpr int HEADS = 4;
-  uint32_t qs[KT][2];  // q * 2^-(bits i), negated in low-part lanes
-  uint32_t qm[KT][2];  // q * 2^-(bits i) in low-part lanes, 0 in high-part lanes
+  // per (kt, lane) in block-shared memory: (qs0, qs1, qm0, qm1) with
+  //   qs = q * 2^-(bits i), negated in low-part lanes,
+  //   qm = q * 2^-(bits i) in low-part lanes, 0 in high-part lanes
+  const uint4* qsm;
   float acc[KT][4];    // D[channel][col]
   float vb[4];         // value zero-point term: D[value group][col]
   float m_run, m_lim, l_run;
+  float sc[MT][4], kb[4];          // scores of the group keys() read last
+  uint32_t PA[MT][2], PB[MT][2];  // its weights, after softmax()
 
-  __device__ __forceinline__ void init(const QArgs& a, int b, int h, int lane) {
+  // Query fragments of unit (b, h) into the block-shared area (one warp).
+  __device__ __forceinline__ static void write_q(const QArgs& a, int b, int h, int lane, uint4* q_sm) {
     const int gid = lane >> 2, tig = lane & 3, part = gid & 1;
     const int hh = gid >> 1;
     const bool hv = hh < a.g;
@@ -297,11 +361,14 @@ struct TokM {
       const float2 hi = unpack_bf2(*reinterpret_cast<const uint32_t*>(qp + kt * 16 + 8 + 2 * tig));
       const uint32_t q0 = hv ? pack_h2(lo.x * f, lo.y * f) : 0u;
       const uint32_t q1 = hv ? pack_h2(hi.x * f, hi.y * f) : 0u;
-      qs[kt][0] = part ? q0 ^ 0x80008000u : q0;
-      qs[kt][1] = part ? q1 ^ 0x80008000u : q1;
-      qm[kt][0] = part ? q0 : 0u;
-      qm[kt][1] = part ? q1 : 0u;
+      q_sm[kt * 32 + lane] = make_uint4(part ? q0 ^ 0x80008000u : q0, part ? q1 ^ 0x80008000u : q1,
+                                        part ? q0 : 0u, part ? q1 : 0u);
     }
+  }
+
+  __device__ __forceinline__ void init(const QArgs& a, int b, int h, int lane, const uint4* q_sm) {
+    (void)a, (void)b, (void)h, (void)lane;
+    qsm = q_sm;
 #pragma unroll
     for (int mc = 0; mc < KT; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
     vb[0] = vb[1] = vb[2] = vb[3] = 0.f;
@@ -310,23 +377,15 @@ struct TokM {
     l_run = 0.f;
   }
 
-  // One group record at rs (shared memory).
-  __device__ __forceinline__ void group(const unsigned char* rs, int lane, float scl, float sl2) {
-    constexpr unsigned FULL = 0xffffffffu;
-    using C = QCfg<BITS, G, D, 1>;
-    const int gid = lane >> 2, tig = lane & 3;
+  // (1) scores: per channel tile kt the key scales are folded into q right
+  //     before use (high part in part-0 columns, low part in part-1
+  //     columns); the zero-point term sum_c q_c z_c is an MMA of the zeros
+  //     (times 2^(bits i), exact) against the signed q in the high columns.
+  __device__ __forceinline__ void keys(const unsigned char* rs, int lane) {
+    const int tig = lane & 3;
     const uint32_t* kcw = reinterpret_cast<const uint32_t*>(rs);
-    const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
     const uint4* skw = reinterpret_cast<const uint4*>(rs + C::OFF_SK) + tig * (KT / 2);
     const uint4* zkw = reinterpret_cast<const uint4*>(rs + C::OFF_ZK) + tig * (KT / 2);
-    const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);  // [G/2][CPG] token pairs
-    const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
-
-    // (1) scores: per channel tile kt the key scales are folded into q right
-    //     before use (high part in part-0 columns, low part in part-1
-    //     columns); the zero-point term sum_c q_c z_c is an MMA of the zeros
-    //     (times 2^(bits i), exact) against the signed q in the high columns.
-    float sc[MT][4], kb[4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
     kb[0] = kb[1] = kb[2] = kb[3] = 0.f;
@@ -343,8 +402,9 @@ struct TokM {
         const int kt = TPW * j + i;
         const uint4 s4 = skw[kt >> 1];
         const uint32_t sA = (kt & 1) ? s4.z : s4.x, sC = (kt & 1) ? s4.w : s4.y;
-        const uint32_t fa = hfma2(qm[kt][0], sA, hmul2(qs[kt][0], sA));
-        const uint32_t fc = hfma2(qm[kt][1], sC, hmul2(qs[kt][1], sC));
+        const uint4 qq = qsm[kt * 32 + lane];  // (qs0, qs1, qm0, qm1)
+        const uint32_t fa = hfma2(qq.z, sA, hmul2(qq.x, sA));
+        const uint32_t fc = hfma2(qq.w, sC, hmul2(qq.y, sC));
         const uint32_t m = F::mask(i);
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
@@ -355,12 +415,15 @@ struct TokM {
         const uint32_t z0 = zscale<BITS>((kt & 1) ? z4.z : z4.x, i);
         const uint32_t z8 = zscale<BITS>((kt & 1) ? z4.w : z4.y, i);
         const uint32_t za[4] = {z0, z0, z8, z8};
-        mma_f16(kb, za, qs[kt][0], qs[kt][1]);
+        mma_f16(kb, za, qq.x, qq.y);
       }
     }
+  }
 
-    // (2) softmax of head tig over the lane's tokens 16 mt + gid (+8); the
-    //     scores sit in the 2^-24 domain of the code encoding
+  // (2) softmax of head tig over the lane's tokens 16 mt + gid (+8); the
+  //     scores sit in the 2^-24 domain of the code encoding
+  __device__ __forceinline__ void softmax(float scl, float sl2) {
+    constexpr unsigned FULL = 0xffffffffu;
     const float kzs = kb[0] * sl2;
     float x[MT][2];
     float t = -INFINITY;
@@ -395,7 +458,6 @@ struct TokM {
     // (p, -p) in a head's (high, low) columns for PA and (0, p) for PB;
     // after the transpose lane (gid, tig) holds its column's entries for
     // tokens 2 tig, 2 tig + 1 of the block.
-    uint32_t PA[MT][2], PB[MT][2];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
@@ -406,10 +468,16 @@ struct TokM {
         PB[mt][hf] = movm_t(pack_h2(0.f, p));
       }
     }
+  }
 
-    // (3) P . V: per 16-token tile, the folded operand of value group cg is
-    //     high (part 0 columns: 0 + fp16(p~ s)) or low (part 1 columns:
-    //     p~ s - fp16(p~ s), exact) -- the same two instructions in every lane
+  // (3) P . V: per 16-token tile, the folded operand of value group cg is
+  //     high (part 0 columns: 0 + fp16(p~ s)) or low (part 1 columns:
+  //     p~ s - fp16(p~ s), exact) -- the same two instructions in every lane
+  __device__ __forceinline__ void values(const unsigned char* rs, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
+    const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);  // [G/2][CPG] token pairs
+    const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
 #pragma unroll
     for (int ktt = 0; ktt < MT; ++ktt) {
       uint32_t s01[CPG], s89[CPG];
@@ -445,8 +513,9 @@ struct TokM {
     }
   }
 
-  // This warp's state -> its slot (natural channel order, unnormalised).
-  __device__ __forceinline__ void store(const QArgs& a, int warp, int lane, bool ok, float* st_o, float* st_ml) {
+  // This warp's state -> wst [HEADS][D] (natural channel order, unnormalised)
+  // and wml [HEADS][2].
+  __device__ __forceinline__ void store(const QArgs& a, int lane, bool ok, float* wst, float* wml) {
     constexpr unsigned FULL = 0xffffffffu;
     const int gid = lane >> 2, tig = lane & 3;
     const int hh = tig;
@@ -461,14 +530,14 @@ struct TokM {
       const float zb = __shfl_sync(FULL, vbs, cg * 4 + tig);
       const float uf = pow2i(24 - BITS * (mc % TPW));  // undo the code encoding of this tile
       if (hh < a.g) {
-        float* wo = st_o + (warp * HEADS + hh) * D + mc * 16 + gid;
+        float* wo = wst + hh * D + mc * 16 + gid;
         wo[0] = (acc[mc][0] + acc[mc][1]) * uf + zb;
         wo[8] = (acc[mc][2] + acc[mc][3]) * uf + zb;
       }
     }
     if (hh < a.g && gid == 0) {
-      st_ml[(warp * HEADS + hh) * 2] = ok ? m_run : -INFINITY;
-      st_ml[(warp * HEADS + hh) * 2 + 1] = ok ? l : 0.f;
+      wml[hh * 2] = ok ? m_run : -INFINITY;
+      wml[hh * 2 + 1] = ok ? l : 0.f;
     }
   }
 };
@@ -476,14 +545,18 @@ struct TokM {
 template <int BITS, int G, int D>
 struct HeadM {
   using F = Frag<BITS>;
+  using C = QCfg<BITS, G, D, 2>;
   static constexpr int KT = D / 16, TPW = F::TPW, NW = 2 * KT / TPW, MT = G / 16, CPG = D / G;
   static constexpr int HEADS = 8;
   uint32_t q2[KT][2];  // head gid: q * 2^-(bits i), channel pairs (2 tig, +1), (2 tig + 8, +9)
   float acc[KT][4];    // D[channel][head]: (channel gid, heads 2 tig, 2 tig + 1), channel + 8
   float vb[4];         // D[value group][head]
   float m_run, m_lim, l_run;  // head gid
+  float sc[2 * MT][4], kb[4];  // n-tile n: tokens 8 n .. 8 n + 7
+  uint32_t P[2 * MT];          // p~ of head gid, tokens 8 n + 2 tig, +1
 
-  __device__ __forceinline__ void init(const QArgs& a, int b, int h, int lane) {
+  __device__ __forceinline__ void init(const QArgs& a, int b, int h, int lane, const uint4* q_sm) {
+    (void)q_sm;
     const int gid = lane >> 2, tig = lane & 3;
     const bool hv = gid < a.g;
     const __nv_bfloat16* qp = a.q + (static_cast<size_t>(b) * a.Hq + h * a.g + (hv ? gid : 0)) * D;
@@ -503,21 +576,14 @@ struct HeadM {
     l_run = 0.f;
   }
 
-  __device__ __forceinline__ void group(const unsigned char* rs, int lane, float scl, float sl2) {
-    constexpr unsigned FULL = 0xffffffffu;
-    using C = QCfg<BITS, G, D, 2>;
-    const int gid = lane >> 2, tig = lane & 3;
+  // (1) scores: rows gid (high part of head gid's q*s) and gid + 8 (its low
+  //     part); zero-point term from rows = q (unfolded) against the zeros
+  //     broadcast over the columns
+  __device__ __forceinline__ void keys(const unsigned char* rs, int lane) {
+    const int tig = lane & 3;
     const uint32_t* kcw = reinterpret_cast<const uint32_t*>(rs);
-    const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
     const uint4* skw = reinterpret_cast<const uint4*>(rs + C::OFF_SK) + tig * (KT / 2);
     const uint4* zkw = reinterpret_cast<const uint4*>(rs + C::OFF_ZK) + tig * (KT / 2);
-    const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);
-    const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
-
-    // (1) scores, n-tile nt = tokens 8 nt .. 8 nt + 7: rows gid (high part of
-    //     head gid's q*s) and gid + 8 (its low part); zero-point term from
-    //     rows = q (unfolded) against the zeros broadcast over the columns
-    float sc[2 * MT][4], kb[4];
 #pragma unroll
     for (int n = 0; n < 2 * MT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
     kb[0] = kb[1] = kb[2] = kb[3] = 0.f;
@@ -551,8 +617,12 @@ struct HeadM {
         }
       }
     }
+  }
 
-    // (2) softmax of head gid over tokens 8 n + 2 tig, +1
+  // (2) softmax of head gid over tokens 8 n + 2 tig, +1
+  __device__ __forceinline__ void softmax(float scl, float sl2) {
+    constexpr unsigned FULL = 0xffffffffu;
+    const int tig = threadIdx.x & 3;
     const float kzs = kb[0] * sl2;
     float y[2 * MT][2];
     float t = -INFINITY;
@@ -587,16 +657,21 @@ struct HeadM {
       vb[3] *= a1;
     }
     const float off = kzs - m_run;
-    uint32_t P[2 * MT];
 #pragma unroll
     for (int n = 0; n < 2 * MT; ++n) {
       const float p0 = ex2(fmaf(y[n][0], scl, off)), p1 = ex2(fmaf(y[n][1], scl, off));
       l_run += p0 + p1;
       P[n] = pack_h2(p0, p1);
     }
+  }
 
-    // (3) P . V: B = p~ * s of head gid for tokens (2 tig, +1) and (2 tig + 8, +9),
-    //     high part and exact low part as two MMAs into the same accumulator
+  // (3) P . V: B = p~ * s of head gid for tokens (2 tig, +1) and (2 tig + 8, +9),
+  //     high part and exact low part as two MMAs into the same accumulator
+  __device__ __forceinline__ void values(const unsigned char* rs, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t* vcw = reinterpret_cast<const uint32_t*>(rs + C::OFF_VC);
+    const uint32_t* sv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_SV);
+    const uint32_t* zv32 = reinterpret_cast<const uint32_t*>(rs + C::OFF_ZV);
 #pragma unroll
     for (int ktt = 0; ktt < MT; ++ktt) {
       uint32_t s01[CPG], s89[CPG];
@@ -634,7 +709,7 @@ struct HeadM {
     }
   }
 
-  __device__ __forceinline__ void store(const QArgs& a, int warp, int lane, bool ok, float* st_o, float* st_ml) {
+  __device__ __forceinline__ void store(const QArgs& a, int lane, bool ok, float* wst, float* wml) {
     constexpr unsigned FULL = 0xffffffffu;
     const int gid = lane >> 2, tig = lane & 3;
     float l = l_run;
@@ -648,82 +723,150 @@ struct HeadM {
       const float zb1 = __shfl_sync(FULL, vb[1], cg * 4 + tig);
       const float uf = pow2i(24 - BITS * (mc % TPW));
       if (h0 < a.g) {
-        float* wo = st_o + (warp * HEADS + h0) * D + mc * 16 + gid;
+        float* wo = wst + h0 * D + mc * 16 + gid;
         wo[0] = acc[mc][0] * uf + zb0;
         wo[8] = acc[mc][2] * uf + zb0;
       }
       if (h1 < a.g) {
-        float* wo = st_o + (warp * HEADS + h1) * D + mc * 16 + gid;
+        float* wo = wst + h1 * D + mc * 16 + gid;
         wo[0] = acc[mc][1] * uf + zb1;
         wo[8] = acc[mc][3] * uf + zb1;
       }
     }
     if (gid < a.g && tig == 0) {
-      st_ml[(warp * HEADS + gid) * 2] = ok ? m_run : -INFINITY;
-      st_ml[(warp * HEADS + gid) * 2 + 1] = ok ? l : 0.f;
+      wml[gid * 2] = ok ? m_run : -INFINITY;
+      wml[gid * 2 + 1] = ok ? l : 0.f;
     }
   }
 };
 
-// Processes this warp's stages of unit u's quantised segment (the prefetch
-// pipeline runs on across segments) and leaves the warp's state in its slot.
+// A warp's ring of NST stage slots.  Stage i (the warp's i-th quantised
+// stage) lives in slot i mod NST and completes phase (i / NST) mod 2 of that
+// slot's mbarrier.  A slot is refilled (the stage NST later is issued into
+// it) only once the stage it holds is released.
+struct WarpRing {
+  int issued;     // stages issued
+  int head;       // next stage to wait for
+  int tail;       // next stage to release
+  int hslot;
+  uint32_t hphase;
+  int q_first, q_end;  // this warp's first quantised stage in a unit, and the block's end
+  IssuePtr ip;
+};
+
+template <typename C>
+__device__ __forceinline__ void ring_issue_next(const QArgs& a, unsigned char* ring, uint64_t* bars, int lane,
+                                                WarpRing& r, int slot, int my_nq) {
+  if (r.issued < my_nq) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    issue_stage<C>(a, ring, bars, lane, slot, r.ip);
+    issue_advance<C>(a, r.ip, r.q_first, r.q_end);
+    ++r.issued;
+  }
+}
+
+// Waits for stage r.head; returns its slot or -1 if the bounded wait gave up
+// (then every stage still in flight is drained and the warp stops).
+template <typename C>
+__device__ __forceinline__ int ring_wait(const QArgs& a, uint64_t* bars, WarpRing& r, bool& ok) {
+  constexpr unsigned FULL = 0xffffffffu;
+  const int slot = r.hslot;
+  if (!__all_sync(FULL, mbar_wait_bounded(&bars[slot], r.hphase, a.flags))) {  // warp-uniform
+    ok = false;
+    for (int k = r.head; k < r.issued; ++k)
+      mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
+    return -1;
+  }
+  ++r.head;
+  r.hslot = slot + 1 == C::NST ? 0 : slot + 1;
+  r.hphase ^= r.hslot == 0 ? 1u : 0u;
+  return slot;
+}
+
+// Processes this warp's stages of unit u's quantised segment and leaves the
+// warp's state in the slot of its last stage of the segment (that slot is
+// released, and refilled, only after the block has merged the warp states:
+// *state_slot returns it, -1 if the warp had no stage here).
 template <int BITS, int G, int D, int NT>
-__device__ __forceinline__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, int u, int64_t qs0,
-                                          int my_nq, int& iq, int& issued, IssuePtr& ip, int& islot, int& cslot,
-                                          uint32_t& cphase, bool& ok, float* st_o, float* st_ml) {
+__device__ __forceinline__ void quant_seg(const QArgs& a, unsigned char* ring, uint64_t* bars, int u, int n_seg,
+                                          int my_nq, WarpRing& r, bool& ok, float* wml, int& state_slot,
+                                          const uint4* q_sm) {
   using C = QCfg<BITS, G, D, NT>;
   using Body = std::conditional_t<NT == 1, TokM<BITS, G, D>, HeadM<BITS, G, D>>;
-  constexpr unsigned FULL = 0xffffffffu;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   const int b = u / a.Hkv, h = u - b * a.Hkv;
   // the score MMAs accumulate scores * 2^-24; undo it together with the softmax scale
   const float scl = a.scale_log2 * 16777216.0f;
+  const float sl2 = a.scale_log2;
   Body body;
-  body.init(a, b, h, lane);
+  body.init(a, b, h, lane, q_sm);
+  state_slot = -1;
 
-  // this warp's stages of the segment: local stages ls0, ls0 + kQNW, ...
-  // (qs: index inside the quantised zone; this warp's i-th one is qs0 + kQNW i)
-  int n_seg = 0, ls0 = 0;
-  {
-    const int64_t seg_lo = static_cast<int64_t>(u) * a.P.sq, seg_hi = seg_lo + a.P.sq;
-    const int64_t s_first = qs0 + static_cast<int64_t>(iq) * kQNW;
-    if (iq < my_nq && s_first < seg_hi) {
-      const int64_t n = (seg_hi - s_first + kQNW - 1) / kQNW;
-      n_seg = n < my_nq - iq ? static_cast<int>(n) : my_nq - iq;
-      ls0 = static_cast<int>(s_first - seg_lo);
-    }
-  }
+  // this warp's stages of the segment: r.head .. r.head + n_seg - 1, unit-local
+  // stages r.q_first + kQNW kk
+  auto stage_ptr = [&](int slot) { return ring + slot * C::STAGE; };
+  if (n_seg > 0 && ok) {
+    if constexpr (C::PIPE) {
+      static_assert(C::NG == 1, "the pipelined loop takes one group per stage");
+      int s_cur = ring_wait<C>(a, bars, r, ok);
+      if (s_cur >= 0) {
+        body.keys(stage_ptr(s_cur), lane);
+        body.softmax(scl, sl2);
 #pragma unroll 1
-  for (int kk = 0; kk < n_seg; ++kk, ++iq) {
-    if (!ok) continue;
-    if (issued < my_nq && issued <= iq + C::NST - 1) {
-      fence_proxy_async_smem();
-      __syncwarp();
-      issue_stage<C>(a, ring, bars, lane, islot, ip);
-      ip.advance(a.P);
-      ++issued;
-      islot = islot + 1 == C::NST ? 0 : islot + 1;
-    }
-    const int slot = cslot;  // = iq mod NST, with phase cphase = (iq / NST) mod 2
-    cslot = cslot + 1 == C::NST ? 0 : cslot + 1;
-    const uint32_t phase = cphase;
-    cphase ^= cslot == 0 ? 1u : 0u;
-    if (!__all_sync(FULL, mbar_wait_bounded(&bars[slot], phase, a.flags))) {  // warp-uniform
-      ok = false;
-      for (int k = iq; k < issued; ++k) mbar_wait_bounded(&bars[k % C::NST], (k / C::NST) & 1, nullptr, 100000000ull);
-      continue;
-    }
-    if constexpr (C::NG == 1) {
-      body.group(ring + slot * C::STAGE, lane, scl, a.scale_log2);
+        for (int kk = 1; kk < n_seg; ++kk) {
+          const int s_nxt = ring_wait<C>(a, bars, r, ok);
+          if (s_nxt < 0) break;
+          body.values(stage_ptr(s_cur), lane);
+          body.keys(stage_ptr(s_nxt), lane);
+          __syncwarp();
+          ring_issue_next<C>(a, ring, bars, lane, r, s_cur, my_nq);  // stage tail + NST into the freed slot
+          ++r.tail;
+          body.softmax(scl, sl2);
+          s_cur = s_nxt;
+        }
+        if (ok) {
+          body.values(stage_ptr(s_cur), lane);
+          __syncwarp();
+          state_slot = s_cur;
+        }
+      }
     } else {
-      const int64_t g0 = static_cast<int64_t>(ls0 + kk * kQNW) * C::NG;
-      const int n_here = a.P.ng - g0 < C::NG ? static_cast<int>(a.P.ng - g0) : C::NG;
 #pragma unroll 1
-      for (int gi = 0; gi < n_here; ++gi) body.group(ring + slot * C::STAGE + gi * C::REC, lane, scl, a.scale_log2);
+      for (int kk = 0; kk < n_seg; ++kk) {
+        const int s_cur = ring_wait<C>(a, bars, r, ok);
+        if (s_cur < 0) break;
+        const unsigned char* rs = stage_ptr(s_cur);
+        if constexpr (C::NG == 1) {
+          body.keys(rs, lane);
+          body.softmax(scl, sl2);
+          body.values(rs, lane);
+        } else {
+          const int64_t gs = static_cast<int64_t>(r.q_first + kQNW * kk) * C::NG;
+          const int n_here = a.P.ng - gs < C::NG ? static_cast<int>(a.P.ng - gs) : C::NG;
+#pragma unroll 1
+          for (int gi = 0; gi < n_here; ++gi) {
+            body.keys(rs + gi * C::REC, lane);
+            body.softmax(scl, sl2);
+            body.values(rs + gi * C::REC, lane);
+          }
+        }
+        __syncwarp();
+        if (kk + 1 < n_seg) {
+          ring_issue_next<C>(a, ring, bars, lane, r, s_cur, my_nq);
+          ++r.tail;
+        } else {
+          state_slot = s_cur;
+        }
+      }
     }
-    __syncwarp();
   }
-  body.store(a, warp, lane, ok, st_o, st_ml);
+  if (state_slot >= 0) {
+    body.store(a, lane, ok, reinterpret_cast<float*>(stage_ptr(state_slot)), wml);
+  } else if (lane < C::HEADS) {
+    wml[lane * 2] = -INFINITY;  // no state from this warp
+    wml[lane * 2 + 1] = 0.f;
+  }
 }
 
 // -------------------------------------------------------- bf16 residual part
@@ -731,12 +874,13 @@ __device__ __forceinline__ void quant_seg(const QArgs& a, unsigned char* ring, u
 // not pipelined; the residual is a few percent of the bytes).  Leaves the
 // warp's state in its slot.
 template <int D, int NT, int HEADS>
-__device__ __forceinline__ void residual_seg(const QArgs& a, unsigned char* ring, float* P_s, uint64_t* bar, int& rph, int u,
-                             int64_t first_s, int64_t end_s, int64_t seg_b, bool& ok, float* st_o, float* st_ml) {
+__device__ __forceinline__ void residual_seg(const QArgs& a, unsigned char* ring, float* P_s, uint64_t* bar,
+                                             int& rph, int u, int t_first, int t_end, bool& ok, float* wst,
+                                             float* wml) {
   constexpr int KT = D / 16;
   constexpr int ROW_B = D * 2;
   constexpr unsigned FULL = 0xffffffffu;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int part = gid & 1;
   const int b = u / a.Hkv, h = u - b * a.Hkv;
@@ -765,8 +909,8 @@ __device__ __forceinline__ void residual_seg(const QArgs& a, unsigned char* ring
 #pragma unroll
     for (int mc = 0; mc < KT; ++mc) acc[mc][nt][0] = acc[mc][nt][1] = acc[mc][nt][2] = acc[mc][nt][3] = 0.f;
   }
-  for (int64_t s = first_s; s < end_s && ok; s += kQNW) {
-    const int t0 = static_cast<int>(s - seg_b) * kResRows;
+  for (int t = t_first; t < t_end && ok; t += kQNW) {
+    const int t0 = t * kResRows;
     const int nv = a.R - t0 < kResRows ? a.R - t0 : kResRows;  // rows of this tile inside the window
     fence_proxy_async_smem();
     __syncwarp();
@@ -864,239 +1008,254 @@ __device__ __forceinline__ void residual_seg(const QArgs& a, unsigned char* ring
     if (hh < a.g) {
 #pragma unroll
       for (int mc = 0; mc < KT; ++mc) {
-        float* wo = st_o + (warp * HEADS + hh) * D + mc * 16 + gid;
+        float* wo = wst + hh * D + mc * 16 + gid;
         wo[0] = acc[mc][nt][0] + acc[mc][nt][1];
         wo[8] = acc[mc][nt][2] + acc[mc][nt][3];
       }
       if (gid == 0) {
-        st_ml[(warp * HEADS + hh) * 2] = ok ? m_run[nt] : -INFINITY;
-        st_ml[(warp * HEADS + hh) * 2 + 1] = ok ? l : 0.f;
+        wml[hh * 2] = ok ? m_run[nt] : -INFINITY;
+        wml[hh * 2 + 1] = ok ? l : 0.f;
       }
     }
   }
 }
 
-// Number of block partials of unit u and the slot of partial p of it.  A
-// unit's partials are those of its residual segment (blocks block_of(begin)
-// .. block_of(end - 1)) followed by those of its quantised segment.  Every
-// block after the first one of a segment starts inside it, so its local
-// segment index is 0; only the first block's index needs computing.
-struct UnitPartials {
-  int seg[2];
-  int kb[2];
-  int cnt[2];
-  int loc0[2];
-  __device__ void init(const Partition& P, int u) {
-    int n = 0;
-    if (P.sr > 0) seg[n++] = u;
-    if (P.sq > 0) seg[n++] = P.U + u;
-    for (int i = 0; i < 2; ++i) {
-      if (i < n) {
-        kb[i] = P.block_of(P.seg_begin(seg[i]));
-        cnt[i] = P.block_of(P.seg_end(seg[i]) - 1) - kb[i] + 1;
-        loc0[i] = seg[i] - P.seg_of(P.first(kb[i]));
-      } else {
-        seg[i] = 0, kb[i] = 0, cnt[i] = 0, loc0[i] = 0;
-      }
-    }
-  }
-  __device__ int total() const { return cnt[0] + cnt[1]; }
-  __device__ int64_t slot(int maxs, int p) const {
-    const int i = p < cnt[0] ? 0 : 1;
-    const int pl = i ? p - cnt[0] : p;
-    return static_cast<int64_t>(kb[i] + pl) * maxs + (pl == 0 ? loc0[i] : 0);
-  }
-};
-
-// Block-wide: merges the kQNW warp states of segment `seg` (local index j of
-// block k) into the block's partial of that segment.
+// Block-wide: merges the kQNW warp states of a segment into the block's
+// partial of that segment (partial slot `slot`).  Warp w's state is at
+// byte offset st_off[w] of shared memory (-1: that warp had nothing here).
 template <int D, int HEADS>
-__device__ __forceinline__ void merge_segment(const QArgs& a, int k, int j, const float* st_o, const float* st_ml,
-                                           float* mw) {
+__device__ __forceinline__ void merge_segment(const QArgs& a, int64_t slot, const unsigned char* smem,
+                                              const int* st_off, const float* st_ml, float* mw) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int g = a.g;
-  float* wts = mw;               // [kQNW][HEADS]
+  float* wts = mw;                // [kQNW][HEADS]
   float* ML = mw + kQNW * HEADS;  // [HEADS][2]
   for (int r = tid; r < g; r += nthr) {
     float M = -INFINITY;
-    for (int w = 0; w < kQNW; ++w) M = fmaxf(M, st_ml[(w * HEADS + r) * 2]);
+    for (int w = 0; w < kQNW; ++w)
+      if (st_off[w] >= 0) M = fmaxf(M, st_ml[(w * HEADS + r) * 2]);
     float L = 0.f;
     for (int w = 0; w < kQNW; ++w) {
       const float mw_ = st_ml[(w * HEADS + r) * 2];
-      const float sc = (mw_ == -INFINITY) ? 0.f : ex2(mw_ - M);
+      const float sc = (st_off[w] < 0 || mw_ == -INFINITY) ? 0.f : ex2(mw_ - M);
       wts[w * HEADS + r] = sc;
-      L += sc * st_ml[(w * HEADS + r) * 2 + 1];
+      L += sc > 0.f ? sc * st_ml[(w * HEADS + r) * 2 + 1] : 0.f;
     }
     ML[2 * r] = M;
     ML[2 * r + 1] = L;
   }
   __syncthreads();
-  const int64_t slot = static_cast<int64_t>(k) * a.MAXS + j;
   float* po = a.part_o + slot * g * D;
   float* pml = a.part_ml + slot * g * 2;
   for (int e = tid; e < g * D; e += nthr) {
-    const int r = e / D, d = e - r * D;
+    const int r = e / D;
     float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < kQNW; ++w) acc += wts[w * HEADS + r] * st_o[(w * HEADS + r) * D + d];
+    for (int w = 0; w < kQNW; ++w) {
+      const float wt = wts[w * HEADS + r];
+      if (wt > 0.f) acc += wt * reinterpret_cast<const float*>(smem + st_off[w])[e];
+    }
     po[e] = acc;
   }
   for (int r = tid; r < g; r += nthr) {
     pml[2 * r] = ML[2 * r];
     pml[2 * r + 1] = ML[2 * r + 1];
   }
-  __syncthreads();  // the warp slots are reused by the next segment
+  fence_proxy_async_smem();  // the state slots are refilled by bulk copies after this
+  __syncthreads();
 }
 
-// Merges every unit's block partials into out.  One block of 128 threads per
-// (unit, head r): warp w takes partials w, w + 4, ...; each lane keeps a
-// running online-softmax merge (M, L, D/32 channels) of them, loading a
-// partial's (m, l) and its channel slice together (independent loads, one
-// round trip); the four warp states are then merged through shared memory.
-struct CArgs {
-  Partition P;
-  int MAXS, g, Hq, Hkv;
-  const float* part_o;
-  const float* part_ml;
-  float* out;
-};
-
+// After the block wrote its partial of unit u: the block that writes the
+// unit's last partial (a per-unit ticket counts them) merges all of them
+// into the output and resets the ticket for the next call.  Partials come
+// from other SMs, so they are read past L1 (ld.global.cg).  The merge is on
+// the kernel's tail, so it is latency-bound: the partials' slots and merge
+// weights are staged in shared memory once, then each thread owns output
+// float4s and keeps up to 16 partial loads in flight.
+// After the block wrote its partial of unit u (and passed the barrier that
+// follows those writes): the block that writes the unit's last partial (a
+// per-unit ticket counts them) merges all of them into the output and resets
+// the ticket for the next call.  Partials come from other SMs, so they are
+// read past L1 (ld.global.cg).  The merge sits on the kernel's tail and is
+// latency-bound, so it takes two rounds of loads: (1) lane p of warp r reads
+// partial p's (max, sum) of head r, the warp reduces the maximum and the sum
+// and stages the weights; (2) each thread owns output float4s and keeps up to
+// 16 partial loads in flight.
 template <int D>
-__global__ void __launch_bounds__(128) combine_kernel(CArgs a) {
-  __shared__ float wsum[4][D];
-  __shared__ float wml[4][2];
-  // launched as a programmatic dependent of draft_quant_kernel: wait until that
-  // grid has completed and its partials are visible
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  const int u = blockIdx.x, r = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+__device__ __forceinline__ void unit_finish(const QArgs& a, int u, float* ma, int* s_flag) {
+  constexpr unsigned FULL = 0xffffffffu;
+  const int np = a.P.np;
+  if (threadIdx.x == 1) {
+    // lane 1 of warp 0 issues no bulk copies, so its fence waits on no copy
+    // in flight; it orders the block's partial writes (seen through the
+    // barrier) before the ticket
+    __threadfence();
+    const unsigned old = atomicAdd(a.tickets + u, 1u);
+    const int last = old + 1u == static_cast<unsigned>(np) ? 1 : 0;
+    if (last) {
+      __threadfence();    // the other blocks' partials are visible past this point
+      a.tickets[u] = 0u;  // every partial of u is in; no other block touches it in this call
+    }
+    *s_flag = last;
+  }
+  __syncthreads();
+  if (!*s_flag) return;
   const int g = a.g;
-  UnitPartials up;
-  up.init(a.P, u);
-  const int np = up.total();
-  constexpr int PER = D / 32;  // channels per lane
-  float acc[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  float M = -INFINITY, L = 0.f;
-  for (int p0 = warp; p0 < np; p0 += 8) {  // two partials of this warp per trip
-    float v[2][PER];
-    float2 ml[2];
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int p = p0 + 4 * t;
-      if (p < np) {
-        const int64_t slot = up.slot(a.MAXS, p);
-        ml[t] = *reinterpret_cast<const float2*>(a.part_ml + slot * g * 2 + 2 * r);
-        const float* src = a.part_o + (slot * g + r) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 x = *reinterpret_cast<const float4*>(src);
-          v[t][0] = x.x, v[t][1] = x.y, v[t][2] = x.z, v[t][3] = x.w;
-        } else {
-          const float2 x = *reinterpret_cast<const float2*>(src);
-          v[t][0] = x.x, v[t][1] = x.y;
-        }
-      } else {
-        ml[t] = make_float2(-INFINITY, 0.f);
-#pragma unroll
-        for (int i = 0; i < PER; ++i) v[t][i] = 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // merge area: (M, L) of 8 heads | slot of each partial | weights [np][g]
+  float* MLs = ma;
+  int* SL = reinterpret_cast<int*>(ma + 16);
+  float* W = ma + 16 + np;
+  const bool staged = 16 + np * (g + 1) <= kMergeFloats;
+  if (staged)
+    for (int p = threadIdx.x; p < np; p += blockDim.x) SL[p] = static_cast<int>(a.P.partial_slot(u, p));
+  __syncthreads();
+  auto slot_of = [&](int p) -> int64_t { return staged ? static_cast<int64_t>(SL[p]) : a.P.partial_slot(u, p); };
+  // (1) per head: online max and sum over the partials, one load per lane and pass
+  for (int r = warp; r < g; r += kQNW) {
+    float M = -INFINITY, L = 0.f;
+    for (int p = lane; p < np; p += 32) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + (slot_of(p) * g + r) * 2));
+      if (ml.x != -INFINITY) {
+        const float Mn = fmaxf(M, ml.x);
+        L = (M == -INFINITY ? 0.f : L * ex2(M - Mn)) + ml.y * ex2(ml.x - Mn);
+        M = Mn;
       }
     }
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      if (ml[t].x == -INFINITY) continue;
-      const float Mn = fmaxf(M, ml[t].x);
-      const float ro = M == -INFINITY ? 0.f : ex2(M - Mn);
-      const float rn = ex2(ml[t].x - Mn);
-      L = L * ro + ml[t].y * rn;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) acc[i] = acc[i] * ro + v[t][i] * rn;
+    for (int o = 16; o > 0; o >>= 1) {
+      const float Mo = __shfl_xor_sync(FULL, M, o), Lo = __shfl_xor_sync(FULL, L, o);
+      const float Mn = fmaxf(M, Mo);
+      L = (M == -INFINITY ? 0.f : L * ex2(M - Mn)) + (Mo == -INFINITY ? 0.f : Lo * ex2(Mo - Mn));
       M = Mn;
     }
+    if (staged)
+      for (int p = lane; p < np; p += 32) {
+        const float m = __ldcg(a.part_ml + (slot_of(p) * g + r) * 2);
+        W[p * g + r] = (M == -INFINITY || m == -INFINITY) ? 0.f : ex2(m - M);
+      }
+    if (lane == 0) {
+      MLs[2 * r] = M;
+      MLs[2 * r + 1] = L;
+    }
   }
-  if (lane == 0) {
-    wml[warp][0] = M;
-    wml[warp][1] = L;
-  }
-#pragma unroll
-  for (int i = 0; i < PER; ++i) wsum[warp][lane * PER + i] = acc[i];
   __syncthreads();
-  float Mb = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < 4; ++w) Mb = fmaxf(Mb, wml[w][0]);
-  float f[4], Lb = 0.f;
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    f[w] = wml[w][0] == -INFINITY ? 0.f : ex2(wml[w][0] - Mb);
-    Lb += f[w] * wml[w][1];
-  }
+  // (2) weighted sum of the partials' o
   const int b = u / a.Hkv, h = u - b * a.Hkv;
-  float* o = a.out + (static_cast<size_t>(b) * a.Hq + h * g + r) * D;
-  for (int d = tid; d < D; d += 128) {
-    const float t = (f[0] * wsum[0][d] + f[1] * wsum[1][d]) + (f[2] * wsum[2][d] + f[3] * wsum[3][d]);
-    o[d] = Lb > 0.f ? t / Lb : 0.f;
+  float4* out = reinterpret_cast<float4*>(a.out + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(h) * g) * D);
+  constexpr int UNR = 16;
+  for (int e4 = threadIdx.x; e4 < g * D / 4; e4 += blockDim.x) {
+    const int r = e4 / (D / 4);
+    const float M = MLs[2 * r], L = MLs[2 * r + 1];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < np; p0 += UNR) {
+      float4 v[UNR];
+      float w[UNR];
+#pragma unroll
+      for (int i = 0; i < UNR; ++i) {
+        const int p = p0 + i;
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        w[i] = 0.f;
+        if (p < np) {
+          const int64_t sl = slot_of(p);
+          if (staged) {
+            w[i] = W[p * g + r];
+          } else {
+            const float m = __ldcg(a.part_ml + (sl * g + r) * 2);
+            w[i] = (M == -INFINITY || m == -INFINITY) ? 0.f : ex2(m - M);
+          }
+          if (w[i] > 0.f) v[i] = __ldcg(reinterpret_cast<const float4*>(a.part_o + sl * g * D) + e4);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < UNR; ++i) {
+        acc.x += w[i] * v[i].x;
+        acc.y += w[i] * v[i].y;
+        acc.z += w[i] * v[i].z;
+        acc.w += w[i] * v[i].w;
+      }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    out[e4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
+  __syncthreads();  // the merge area and flag are reused by the next unit
 }
 
 template <int BITS, int G, int D, int NT>
-__global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 3)) draft_quant_kernel(QArgs a) {
+__global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kernel(QArgs a) {
   using C = QCfg<BITS, G, D, NT>;
   extern __shared__ __align__(128) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x;
-  const Partition& P = a.P;
-  // let the combine grid be scheduled as this grid's blocks retire (it waits
-  // for this grid's completion before reading anything)
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-  const int64_t B0 = P.first(k), B1 = P.first(k + 1);
-  if (B0 >= B1) return;  // the host sizes the grid so that this never happens
-  const int seg0 = P.seg_of(B0), seg1 = P.seg_of(B1 - 1);
+  const UPart& P = a.P;
   unsigned char* ring = smem + warp * C::WARP_B;
   float* P_res = reinterpret_cast<float*>(ring + C::RING);  // residual tile scores
-  float* st_o = reinterpret_cast<float*>(smem + C::STATE_OFF);
   float* st_ml = reinterpret_cast<float*>(smem + C::ML_OFF);
+  int* st_off = reinterpret_cast<int*>(smem + C::SO_OFF);
   float* mw = reinterpret_cast<float*>(smem + C::MW_OFF);
+  float* ma = reinterpret_cast<float*>(smem + C::MA_OFF);
+  int* s_flag = reinterpret_cast<int*>(smem + C::FLAG_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + warp * (C::NST + 1);
-
-  // this warp's quantised stages: s = sQ0 + kQNW i (s >= RZ), i < my_nq
-  const int64_t lo_q = B0 > P.RZ ? B0 : P.RZ;
-  const int64_t off_q = lo_q - B0;
-  const int64_t sQ0 = B0 + warp + (off_q <= warp ? 0 : (off_q - warp + kQNW - 1) / kQNW) * kQNW;
-  const int my_nq = sQ0 < B1 ? static_cast<int>((B1 - sQ0 + kQNW - 1) / kQNW) : 0;
   if (lane == 0)
     for (int s = 0; s <= C::NST; ++s) mbar_init(&bars[s], 1);
   fence_mbar_init();
   __syncwarp();
-  bool ok = true, primed = false;
-  int iq = 0, issued = 0, rph = 0, islot = 0, cslot = 0;
-  uint32_t cphase = 0;
-  IssuePtr ip;
-  for (int seg = seg0; seg <= seg1; ++seg) {
-    if (seg >= P.U) {
-      if (!primed) {  // the ring is free of residual tiles from here on
-        primed = true;
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (my_nq > 0) ip.start(P, sQ0 - P.RZ);
-        while (issued < my_nq && issued < C::NST - 1) {
-          issue_stage<C>(a, ring, bars, lane, islot, ip);
-          ip.advance(P);
-          ++issued;
-          islot = islot + 1 == C::NST ? 0 : islot + 1;
-        }
-      }
-      quant_seg<BITS, G, D, NT>(a, ring, bars, seg - P.U, sQ0 - P.RZ, my_nq, iq, issued, ip, islot, cslot, cphase,
-                                ok, st_o, st_ml);
-    } else {
-      const int64_t sb = P.seg_begin(seg), se = P.seg_end(seg);
-      const int64_t lo = sb > B0 ? sb : B0;
-      const int64_t off = lo - B0;
-      const int64_t i0 = off <= warp ? 0 : (off - warp + kQNW - 1) / kQNW;
-      residual_seg<D, NT, C::HEADS>(a, ring, P_res, &bars[C::NST], rph, seg,
-                                    B0 + warp + i0 * kQNW, se < B1 ? se : B1, sb, ok, st_o, st_ml);
+  int u0, u1, r0, r1, q0, q1;
+  P.block_range(k, u0, u1, r0, r1, q0, q1);
+  // this warp's quantised stages: q0 + warp + kQNW i < q1 of every unit of the block
+  const int per_unit = q1 - q0 - warp > 0 ? (q1 - q0 - warp + kQNW - 1) / kQNW : 0;
+  const int my_nq = (u1 - u0) * per_unit;
+  // Launched as a programmatic dependent of the previous kernel in the
+  // stream: nothing global is read or written before that grid completed.
+  // The next kernel may then be scheduled as this grid's blocks retire (it
+  // waits the same way).
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  bool ok = true;
+  int rph = 0;
+  float* wml = st_ml + warp * C::HEADS * 2;
+  const int64_t slot0 = static_cast<int64_t>(k) * 2 * P.upb;
+
+  // residual tiles of each unit (the ring is not primed yet)
+  if (r1 > r0) {
+    for (int u = u0; u < u1; ++u) {
+      residual_seg<D, NT, C::HEADS>(a, ring, P_res, &bars[C::NST], rph, u, r0 + warp, r1, ok,
+                                    reinterpret_cast<float*>(ring), wml);
+      if (lane == 0) st_off[warp] = static_cast<int>(ring - smem);
+      __syncthreads();
+      merge_segment<D, C::HEADS>(a, slot0 + 2 * (u - u0), smem, st_off, st_ml, mw);
+      unit_finish<D>(a, u, ma, s_flag);
     }
-    __syncthreads();
-    merge_segment<D, C::HEADS>(a, k, seg - seg0, st_o, st_ml, mw);
+  }
+  if (q1 > q0) {
+    WarpRing r;
+    r.issued = 0, r.head = 0, r.tail = 0, r.hslot = 0, r.hphase = 0u;
+    r.q_first = q0 + warp, r.q_end = q1;
+    issue_start<C>(a, r.ip, u0, q0 + warp);
+    fence_proxy_async_smem();
+    __syncwarp();
+    while (r.issued < my_nq && r.issued < C::NST) {
+      issue_stage<C>(a, ring, bars, lane, r.issued, r.ip);
+      issue_advance<C>(a, r.ip, r.q_first, r.q_end);
+      ++r.issued;
+    }
+    uint4* q_sm = reinterpret_cast<uint4*>(smem + C::QSM_OFF);
+    for (int u = u0; u < u1; ++u) {
+      if constexpr (NT == 1) {  // the unit's query fragments, shared by the block's warps
+        if (warp == 0) TokM<BITS, G, D>::write_q(a, u / a.Hkv, u - (u / a.Hkv) * a.Hkv, lane, q_sm);
+        __syncthreads();
+      }
+      int state_slot = -1;
+      quant_seg<BITS, G, D, NT>(a, ring, bars, u, per_unit, my_nq, r, ok, wml, state_slot, q_sm);
+      if (lane == 0) st_off[warp] = state_slot >= 0 ? static_cast<int>(ring + state_slot * C::STAGE - smem) : -1;
+      __syncthreads();
+      merge_segment<D, C::HEADS>(a, slot0 + 2 * (u - u0) + 1, smem, st_off, st_ml, mw);
+      if (state_slot >= 0) {  // the deferred slot is free again: refill it
+        ring_issue_next<C>(a, ring, bars, lane, r, state_slot, my_nq);
+        ++r.tail;
+      }
+      unit_finish<D>(a, u, ma, s_flag);
+    }
   }
 }
 
@@ -1170,9 +1329,9 @@ __global__ void __launch_bounds__(32) debug_dequant_kernel(const uint8_t* recs, 
 }
 
 struct QPlan {
-  Partition P;
+  UPart P;
   int MAXS;
-  size_t off_ml, off_o, total;
+  size_t off_tk, off_ml, off_o, total;
 };
 
 // Blocks per SM for one kernel instance (cached per device).
@@ -1199,32 +1358,41 @@ int quant_occupancy() {
 QPlan make_plan(const vc_attn_shape& sh, const vc_quant_cache& c, int ng_per_stage, int rec_bytes,
                 int64_t target_blocks) {
   QPlan p{};
-  Partition& P = p.P;
+  UPart& P = p.P;
   P.U = sh.B * sh.Hkv;
   P.ng = c.L_q / c.group;
   P.sq = static_cast<int>((P.ng + ng_per_stage - 1) / ng_per_stage);
   P.sr = (c.R + kResRows - 1) / kResRows;
-  P.RZ = static_cast<int64_t>(P.U) * P.sr;
-  P.S_tot = P.RZ + static_cast<int64_t>(P.U) * P.sq;
   P.cq = P.sq > 0 ? static_cast<int64_t>(ng_per_stage) * rec_bytes : 1;
-  P.cr = P.sr > 0 ? static_cast<int64_t>(kResRows) * 4 * sh.D * kResCostWeight : 1;
-  P.C = P.RZ * P.cr + (P.S_tot - P.RZ) * P.cq;
-  const int64_t mx = P.sq > 0 && P.sr > 0 ? (P.cq > P.cr ? P.cq : P.cr) : (P.sq > 0 ? P.cq : P.cr);
-  int64_t n = target_blocks;
-  if (n > P.S_tot) n = P.S_tot;
-  if (n > P.C / mx) n = P.C / mx;
-  if (n < 1) n = 1;
-  P.nblk = static_cast<int>(n);
-  int maxs = 1;
-  for (int k = 0; k < P.nblk; ++k) {
-    const int64_t b0 = P.first(k), b1 = P.first(k + 1);
-    const int segs = P.seg_of(b1 - 1) - P.seg_of(b0) + 1;
-    if (segs > maxs) maxs = segs;
+  P.cr = P.sr > 0 ? static_cast<int64_t>(kResRows) * 4 * sh.D * kResCostNum / kResCostDen : 1;
+  if (target_blocks < 1) target_blocks = 1;
+  if (P.U <= target_blocks) {
+    const int64_t mx = P.sq > 0 && P.sr > 0 ? (P.cq > P.cr ? P.cq : P.cr) : (P.sq > 0 ? P.cq : P.cr);
+    int64_t bpu = target_blocks / P.U;
+    if (bpu > P.ucost() / mx) bpu = P.ucost() / mx;  // every piece holds at least one tile or stage
+    if (bpu < 1) bpu = 1;
+    P.bpu = static_cast<int>(bpu);
+    P.nblk = P.U * P.bpu;
+    P.upb = 1;
+    int jr = 0, jq = P.bpu;
+    for (int j = 0; j < P.bpu; ++j) {
+      if (P.axis_first(j) < P.sr) jr = j + 1;
+      if (jq == P.bpu && P.axis_first(j + 1) > P.sr) jq = j;
+    }
+    P.jr = jr, P.jq = jq;
+    P.np = jr + (P.bpu - jq);
+  } else {
+    P.bpu = 0;
+    P.nblk = static_cast<int>(target_blocks);
+    P.upb = static_cast<int>((P.U + target_blocks - 1) / target_blocks);
+    P.jr = P.jq = 0;
+    P.np = (P.sr > 0 ? 1 : 0) + (P.sq > 0 ? 1 : 0);
   }
-  p.MAXS = maxs;
+  p.MAXS = 2 * P.upb;
   const int g = sh.Hq / sh.Hkv;
-  const size_t slots = static_cast<size_t>(P.nblk) * maxs;
-  p.off_ml = align_up(sizeof(WsHeader), 256);
+  const size_t slots = static_cast<size_t>(P.nblk) * p.MAXS;
+  p.off_tk = align_up(sizeof(WsHeader), 256);
+  p.off_ml = align_up(p.off_tk + static_cast<size_t>(P.U) * 4, 256);
   p.off_o = align_up(p.off_ml + slots * g * 2 * 4, 256);
   p.total = align_up(p.off_o + slots * g * sh.D * 4, 256);
   return p;
@@ -1241,27 +1409,19 @@ template <int BITS, int G, int D, int NT>
 void launch_t(const QArgs& a, const QPlan& p, cudaStream_t s) {
   using C = QCfg<BITS, G, D, NT>;
   quant_occupancy<BITS, G, D, NT>();  // sets the shared-memory attribute once per device
-  draft_quant_kernel<BITS, G, D, NT><<<p.P.nblk, kQNW * 32, C::SMEM_B, s>>>(a);
-  CArgs c{};
-  c.P = p.P;
-  c.MAXS = p.MAXS;
-  c.g = a.g;
-  c.Hq = a.Hq;
-  c.Hkv = a.Hkv;
-  c.part_o = a.part_o;
-  c.part_ml = a.part_ml;
-  c.out = a.out;
+  // programmatic dependent launch: the grid may be scheduled while the
+  // previous kernel of the stream drains; it waits for it before reading
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.P.U), static_cast<unsigned>(a.g));
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
+  cfg.gridDim = dim3(static_cast<unsigned>(p.P.nblk));
+  cfg.blockDim = dim3(kQNW * 32);
+  cfg.dynamicSmemBytes = C::SMEM_B;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, combine_kernel<D>, c);
+  cudaLaunchKernelEx(&cfg, draft_quant_kernel<BITS, G, D, NT>, a);
 }
 
 template <int BITS, int G, int D>
@@ -1343,6 +1503,7 @@ void bind_scratch(QArgs& a, const QPlan& p, void* scratch, float* out) {
   a.P = p.P;
   a.MAXS = p.MAXS;
   a.flags = reinterpret_cast<uint32_t*>(w);
+  a.tickets = reinterpret_cast<uint32_t*>(w + p.off_tk);
   a.part_ml = reinterpret_cast<float*>(w + p.off_ml);
   a.part_o = reinterpret_cast<float*>(w + p.off_o);
   a.out = out;
@@ -1399,23 +1560,29 @@ vc_status vc_debug_dequant(const vc_attn_shape* shape, const vc_quant_cache* cac
 }
 
 vc_status vc_debug_quant_partition(const vc_attn_shape* shape, const vc_quant_cache* cache, int target_blocks,
-                                   int64_t* first_stage, int max_blocks, int* n_blocks, int* max_segments,
-                                   int64_t* n_stages, int64_t* n_quant_stages) {
+                                   int32_t* block_ranges, int max_blocks, int* n_blocks, int* blocks_per_unit,
+                                   int* partials_per_unit, int* residual_tiles, int* quant_stages) {
   vc_status st = vc::check_quant(shape, cache, "vc_debug_quant_partition");
   if (st != VC_OK) return st;
   VC_REQUIRE(target_blocks >= 1, "vc_debug_quant_partition: target_blocks must be >= 1");
-  VC_REQUIRE(n_blocks && max_segments && n_stages && n_quant_stages, "vc_debug_quant_partition: null output");
+  VC_REQUIRE(n_blocks && blocks_per_unit && partials_per_unit && residual_tiles && quant_stages,
+             "vc_debug_quant_partition: null output");
   vc::QPlan p{};
   if (!vc::quant_plan(*shape, *cache, &p, target_blocks))
     return vc::set_error(VC_ERR_UNSUPPORTED, "vc_debug_quant_partition: no kernel for this configuration");
   *n_blocks = p.P.nblk;
-  *max_segments = p.MAXS;
-  *n_stages = p.P.S_tot;
-  *n_quant_stages = p.P.S_tot - p.P.RZ;
-  if (first_stage) {
-    VC_REQUIRE(max_blocks >= p.P.nblk + 1, "vc_debug_quant_partition: first_stage needs %d entries",
-               p.P.nblk + 1);
-    for (int k = 0; k <= p.P.nblk; ++k) first_stage[k] = p.P.first(k);
+  *blocks_per_unit = p.P.bpu;
+  *partials_per_unit = p.P.np;
+  *residual_tiles = p.P.sr;
+  *quant_stages = p.P.sq;
+  if (block_ranges) {
+    VC_REQUIRE(max_blocks >= p.P.nblk, "vc_debug_quant_partition: block_ranges needs %d rows", p.P.nblk);
+    for (int k = 0; k < p.P.nblk; ++k) {
+      int u0, u1, r0, r1, q0, q1;
+      p.P.block_range(k, u0, u1, r0, r1, q0, q1);
+      int32_t* row = block_ranges + 6 * static_cast<size_t>(k);
+      row[0] = u0, row[1] = u1, row[2] = r0, row[3] = r1, row[4] = q0, row[5] = q1;
+    }
   }
   return VC_OK;
 }

@@ -100,7 +100,7 @@ def lib() -> ctypes.CDLL:
             "vc_draft_attn_quant_noalloc_flags": (c_int, [P(c_uint32), c_void_p]),
             "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
             "vc_debug_quant_partition": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_int, c_void_p, c_int,
-                                                 P(c_int), P(c_int), P(c_int64), P(c_int64)]),
+                                                 P(c_int), P(c_int), P(c_int), P(c_int), P(c_int)]),
             "vc_kvstream_create": (c_int, [P(c_void_p), c_int, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p,
                                            c_void_p]),
             "vc_kvstream_prefetch": (c_int, [c_void_p, c_int]),
@@ -247,18 +247,22 @@ def vc_debug_dequant(sh, qc, k_out, v_out, stream=None):
 
 def vc_debug_quant_partition(sh, qc, target_blocks: int) -> dict:
     """How vc_draft_attn_quant cuts a call into at most target_blocks blocks
-    (no GPU needed): first stage of every block plus the stage counts."""
+    (no GPU needed): per block its units and unit-local residual tiles and
+    quantised stages, plus the per-unit counts."""
     L = lib()
-    nb, ms = ctypes.c_int(), ctypes.c_int()
-    ns, nqs = ctypes.c_int64(), ctypes.c_int64()
-    _check(L.vc_debug_quant_partition(ctypes.byref(sh), ctypes.byref(qc), int(target_blocks), None, 0,
-                                      ctypes.byref(nb), ctypes.byref(ms), ctypes.byref(ns), ctypes.byref(nqs)))
-    first = (ctypes.c_int64 * (nb.value + 1))()
-    _check(L.vc_debug_quant_partition(ctypes.byref(sh), ctypes.byref(qc), int(target_blocks), first,
-                                      nb.value + 1, ctypes.byref(nb), ctypes.byref(ms), ctypes.byref(ns),
-                                      ctypes.byref(nqs)))
-    return dict(first=list(first), n_blocks=nb.value, max_segments=ms.value, n_stages=ns.value,
-                n_quant_stages=nqs.value)
+    nb, bpu, npu, sr, sq = (ctypes.c_int() for _ in range(5))
+
+    def call(rows, n):
+        _check(L.vc_debug_quant_partition(ctypes.byref(sh), ctypes.byref(qc), int(target_blocks), rows, n,
+                                          ctypes.byref(nb), ctypes.byref(bpu), ctypes.byref(npu), ctypes.byref(sr),
+                                          ctypes.byref(sq)))
+
+    call(None, 0)
+    rows = (ctypes.c_int32 * (6 * nb.value))()
+    call(rows, nb.value)
+    blocks = [tuple(rows[6 * k:6 * k + 6]) for k in range(nb.value)]
+    return dict(blocks=blocks, n_blocks=nb.value, blocks_per_unit=bpu.value, partials_per_unit=npu.value,
+                residual_tiles=sr.value, quant_stages=sq.value)
 
 
 def vc_debug_gather(sh, sc, k_out, v_out, ws=None, stream=None):
