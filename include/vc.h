@@ -394,6 +394,15 @@ VC_API vc_status vc_debug_dequant(const vc_attn_shape* shape, const vc_quant_cac
 VC_API vc_status vc_debug_gather(const vc_attn_shape* shape, const vc_sparse_cache* cache, void* k_out, void* v_out,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* vc_debug_wait_timeout runs the bounded on-chip wait every hot-path kernel
+ * uses on an mbarrier that nothing ever completes, giving up after limit_ns
+ * (1 us .. 100 ms): the wait must return, OR VC_FLAG_WAIT_TIMEOUT into
+ * *flags (device uint32) and write 2 to *result (device uint32; 1 would mean
+ * the wait completed).  The kernel ends normally and the context stays
+ * usable; this is how the library's device-side failure path is tested
+ * without faulting or hanging a GPU. */
+VC_API vc_status vc_debug_wait_timeout(uint32_t* flags, uint32_t* result, int64_t limit_ns, void* stream);
+
 /* vc_debug_quant_partition reports, without touching a GPU, how
  * vc_draft_attn_quant cuts one call into blocks when at most target_blocks
  * blocks are allowed (the real call uses SMs x resident blocks).  Each

@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
             "vc_workspace_flags": (c_int, [c_void_p, c_size_t, P(c_uint32), c_void_p]),
             "vc_draft_attn_quant_noalloc_flags": (c_int, [P(c_uint32), c_void_p]),
             "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
+            "vc_debug_wait_timeout": (c_int, [c_void_p, c_void_p, ctypes.c_int64, c_void_p]),
             "vc_debug_quant_partition": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_int, c_void_p, c_int,
                                                  P(c_int), P(c_int), P(c_int), P(c_int), P(c_int)]),
             "vc_kvstream_create": (c_int, [P(c_void_p), c_int, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p,
@@ -243,6 +244,12 @@ def vc_draft_attn_quant_noalloc_flags(stream=None) -> int:
 
 def vc_debug_dequant(sh, qc, k_out, v_out, stream=None):
     _check(lib().vc_debug_dequant(ctypes.byref(sh), ctypes.byref(qc), _p(k_out), _p(v_out), _stream(stream)))
+
+
+def vc_debug_wait_timeout(flags, result, limit_ns: int, stream=None):
+    """Bounded on-chip wait on an mbarrier that never completes (device
+    uint32 flags and result; see include/vc.h)."""
+    _check(lib().vc_debug_wait_timeout(_p(flags), _p(result), int(limit_ns), _stream(stream)))
 
 
 def vc_debug_quant_partition(sh, qc, target_blocks: int) -> dict:

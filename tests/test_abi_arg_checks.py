@@ -182,3 +182,11 @@ def test_sched_create_rejects(L, n_req, policy, timeout_ms, req):
     st = L.vc_sched_create(ctypes.byref(handle), n_req, reqs, 2, 30, policy, 0, timeout_ms)
     _expect_invalid(L, st, "vc_sched_create")
     assert not handle.value
+
+
+def test_wait_timeout_export_rejects_before_any_launch(L):
+    # null pointers and limits outside 1 us .. 100 ms are refused on the host
+    assert L.vc_debug_wait_timeout(None, 16, 1000000, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_debug_wait_timeout(16, None, 1000000, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_debug_wait_timeout(16, 16, 999, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_debug_wait_timeout(16, 16, 200000000, None) == vc.VC_ERR_INVALID_ARG

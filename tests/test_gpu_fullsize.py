@@ -5,6 +5,8 @@ oracle recomputes sampled (request, KV head) units one by one on the host.
 
 Workloads: Llama-3.1-8B shapes (8 requests x 32K, KIVI-2 group 32, 128-row
 residual), the 500K context, the Llama-70B shape (g = 8, 4-bit group 64),
+each both on random records and with sampled units holding oracle-quantised
+draws with lognormal key outliers,
 the Qwen-32B shape (g = 5, 25000 kept rows of 100000), and acceptance over
 the Llama vocabulary (128256 bf16 logits, 31 rows, 8 requests)."""
 
@@ -16,6 +18,7 @@ from lossless_draft_verify_vc_b200 import synth
 from lossless_draft_verify_vc_b200 import vc
 from oracle import accept as ACC
 from oracle import attention as A
+from oracle import quant as Q
 from tests.vcutil import ATTN_TOL, np32, row_rel_err
 
 pytestmark = pytest.mark.gpu
@@ -55,6 +58,48 @@ def test_quant_draft_full_size_sampled(B, Hq, Hkv, D, T, bits, G, R, units):
     for u in units:
         b, h = divmod(u, Hkv)
         want = A.draft_attention_quant(np32(q[b:b + 1, h * g:(h + 1) * g]), _unit_cache(c, b, h, D))
+        assert row_rel_err(got[b:b + 1, h * g:(h + 1) * g], want) <= ATTN_TOL, (b, h)
+    del c, ws, out
+    _free()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D,T,bits,G,R,units", [
+    (8, 32, 8, 128, 32768, 2, 32, 128, [0, 13, 37, 63]),    # Llama-3.1-8B, 8 x 32K
+    (1, 32, 8, 128, 500000, 2, 32, 128, [3]),                # 500K context
+    (1, 64, 8, 128, 131072, 4, 64, 128, [2, 7]),             # Llama-70B shape, 4-bit group 64, g = 8
+])
+def test_quant_draft_full_size_realistic_units(B, Hq, Hkv, D, T, bits, G, R, units):
+    """The numerically hardest regime at full context: the sampled units hold
+    real draws (keys with lognormal per-channel outliers, values N(0, 1))
+    quantised by the oracle, so scores span the outlier channels' range and
+    the long softmax sums stress the folded-operand precision; the other
+    units are random records.  Each sampled unit is compared with the oracle
+    on its own quantised cache."""
+    c = synth.random_quant_cache(B, Hkv, T - R, R, D, bits, G, seed=T + 7 * bits, device=dev)
+    oracle_units = {}
+    for u in units:
+        b, h = divmod(u, Hkv)
+        k, v = synth.kv_full(1, 1, T, D, seed=1000 + u)
+        oc = Q.build_quant_cache(np32(k), np32(v), bits, G, R)
+        c["records"][b, h].copy_(torch.from_numpy(np.ascontiguousarray(oc["records"][0, 0])).to(dev))
+        c["k_res"][b, h, :R].copy_(k[0, 0, T - R:].to(dev))
+        c["v_res"][b, h, :R].copy_(v[0, 0, T - R:].to(dev))
+        oracle_units[u] = oc
+        del k, v
+    q = synth.normal((B, Hq, D), seed=6, device=dev)
+    sh = vc.shape(B, Hq, Hkv, D)
+    qc = vc.quant_cache(c)
+    ws = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, qc))
+    out = torch.full((B, Hq, D), float("nan"), device=dev)
+    vc.vc_draft_attn_quant(sh, qc, q, out, ws)
+    torch.cuda.synchronize()
+    assert vc.vc_workspace_flags(ws) == 0
+    g = Hq // Hkv
+    got = np32(out)
+    assert np.isfinite(got).all()
+    for u in units:
+        b, h = divmod(u, Hkv)
+        want = A.draft_attention_quant(np32(q[b:b + 1, h * g:(h + 1) * g]), oracle_units[u])
         assert row_rel_err(got[b:b + 1, h * g:(h + 1) * g], want) <= ATTN_TOL, (b, h)
     del c, ws, out
     _free()
