@@ -74,6 +74,7 @@ typedef enum vc_dtype { VC_F32 = 0, VC_BF16 = 1, VC_F16 = 2 } vc_dtype;
 /* Device-side flags reported through the workspace (bit mask). */
 #define VC_FLAG_BAD_INDEX 1u   /* a kept position was outside [0, T_store) */
 #define VC_FLAG_WAIT_TIMEOUT 2u /* a bounded on-chip wait gave up */
+#define VC_FLAG_RANGE 4u        /* a quantisation scale or zero fell outside the fp16 range */
 
 /* Message for the last error returned on the calling thread ("" if none). */
 VC_API const char* vc_last_error(void);
@@ -232,6 +233,38 @@ VC_API vc_status vc_draft_attn_quant_noalloc_flags(uint32_t* host_flags, void* s
 VC_API size_t vc_draft_attn_sparse_workspace_size(const vc_attn_shape* shape, const vc_sparse_cache* cache);
 VC_API vc_status vc_draft_attn_sparse(const vc_attn_shape* shape, const vc_sparse_cache* cache, const void* q,
                                float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- building the compressed caches on the GPU -------------------------------
+ * A compressor is known to the system only through the positions it drops and
+ * the bit width it stores (menfem.com source page, "Key Contributions"); these
+ * calls produce both kinds of draft cache from one layer's full bf16 cache.
+ *
+ * vc_quantize_cache: the oldest L_q rows of every (request, KV head) of
+ * k, v (bf16 [B][Hkv][T][D]) become group records in the layout of
+ * vc_quant_cache (records uint8 [B][Hkv][L_q / group][REC]), the newest
+ * T - L_q rows are copied to rows 0 .. T - L_q - 1 of k_res, v_res (bf16
+ * [B][Hkv][R_cap][D]).  Rule (the library's reading of KIVI-style
+ * quantisation): per group s = fp16((max - min) / (2^bits - 1)) and
+ * z = fp16(min), rounded to nearest even; code = clamp(rint((x - z) / s),
+ * 0, 2^bits - 1) with the stored s and z, half to even, as an exact
+ * division decides; s == 0 gives code 0.  The records equal the oracle's
+ * byte for byte.  A scale or zero outside the fp16 range raises
+ * VC_FLAG_RANGE in the workspace's flag word.  bits 2|4, group 32|64,
+ * D 64|128, L_q a multiple of group, T - L_q <= R_cap.
+ * vc_compact_kept: for each (request, KV head) the rows idx[..][j] of k, v
+ * (bf16 [B][Hkv][T_store][D]) go to row j of k_out, v_out (bf16
+ * [B][Hkv][n_keep][D]): the kept-row pool the token-dropped draft reads with
+ * slots 0 .. n_keep - 1.  An index outside [0, T_store) writes a zero row and
+ * raises VC_FLAG_BAD_INDEX (ws may be NULL).
+ * Both need a workspace of vc_compress_workspace_size() bytes (a flag word,
+ * zeroed once). */
+VC_API size_t vc_compress_workspace_size(void);
+VC_API vc_status vc_quantize_cache(const vc_attn_shape* shape, const void* k, const void* v, int64_t T, int bits,
+                                   int group, int64_t L_q, void* records, void* k_res, void* v_res, int R_cap,
+                                   void* ws, size_t ws_bytes, void* stream);
+VC_API vc_status vc_compact_kept(const vc_attn_shape* shape, const void* k, const void* v, int64_t T_store,
+                                 const int32_t* idx, int n_keep, void* k_out, void* v_out, void* ws,
+                                 size_t ws_bytes, void* stream);
 
 /* ---- block verification attention -----------------------------------------
  * One pass over the full cache scores every drafted position at once and

@@ -1,0 +1,305 @@
+// vc_compress.cu -- building the compressed draft caches on the GPU:
+//   vc_quantize_cache   full bf16 K, V -> group records (KIVI-style uniform
+//                       quantisation, keys per channel, values per token) +
+//                       the bf16 residual window;
+//   vc_compact_kept     full bf16 K, V + kept positions -> a kept-row pool.
+//
+// A compressor is known to the system only through the positions it drops
+// and the bit width it stores ("VeriCache: Turning Lossy KV Cache into
+// Lossless LLM Inference", menfem.com, "Key Contributions"); these two
+// kernels produce exactly those two kinds of cache in the layouts the draft
+// kernels read (include/vc.h).
+//
+// Quantisation rule (the library's reading, identical to the oracle's):
+// per group, s = fp16(round-to-nearest((max - min) / (2^b - 1))),
+// z = fp16(min), code = clamp(rint((x - z) / s), 0, 2^b - 1) with the STORED
+// s and z, half to even; s == 0 gives code 0.  The quotient is evaluated so
+// that every code equals the one an exact float64 division gives: x - z of
+// a bf16 and an fp16 value is exact in float64, the quotient is first taken
+// as (x - z) * (1 / s) and, when it lies within 1e-9 of a rounding tie
+// (k + 1/2), recomputed with an IEEE float64 division.
+#include "vc_common.cuh"
+
+namespace vc {
+namespace {
+
+constexpr uint32_t kRangeFlag = VC_FLAG_RANGE;
+
+// fp16 bits of v rounded to nearest even, or a range flag when |v| > 65504
+__device__ __forceinline__ uint16_t to_half_checked(double v, uint32_t* flags) {
+  if (!(fabs(v) <= 65504.0)) {
+    if (flags) atomicOr(flags, kRangeFlag);
+  }
+  const __half h = __double2half(v);
+  return __half_as_ushort(h);
+}
+
+__device__ __forceinline__ double half_bits_to_double(uint16_t b) {
+  return static_cast<double>(__half2float(__ushort_as_half(b)));
+}
+
+// code = clamp(rint((x - z) / s), 0, levels); s == 0 -> 0
+__device__ __forceinline__ uint32_t quant_code(float x, double s, double z, double inv_s, int levels) {
+  if (s == 0.0) return 0u;
+  const double d = static_cast<double>(x) - z;  // exact: x is bf16, z is fp16
+  double q = d * inv_s;
+  const double f = q - floor(q);
+  if (fabs(f - 0.5) < 1e-9) q = d / s;  // near a tie: the exact quotient decides
+  double r = rint(q);
+  r = r < 0.0 ? 0.0 : (r > levels ? static_cast<double>(levels) : r);
+  return static_cast<uint32_t>(r);
+}
+
+template <int BITS, int G, int D>
+struct QuantLayout {
+  static constexpr int CB = G * D * BITS / 8;
+  static constexpr int REC = 2 * CB + 8 * D;
+  static constexpr int KT = D / 16;
+  static constexpr int TPW = 8 / BITS;
+  static constexpr int NW = 2 * KT / TPW;  // words per lane per 16-token tile
+  static constexpr int CPG = D / G;
+  static constexpr int WORDS = CB / 4;     // 32-bit words of one code block
+};
+
+// One block of 128 threads per (group, unit).  The group's K and V rows are
+// staged in shared memory (bf16), the parameters and reciprocal scales
+// computed, then every thread assembles whole 32-bit words of the
+// fragment-native code blocks (the order in which the draft kernel's lanes
+// consume them), computing each code where it is packed, and the block
+// writes words and parameters as one record.
+template <int BITS, int G, int D>
+__global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __restrict__ k,
+                                                       const __nv_bfloat16* __restrict__ v, int64_t T,
+                                                       int64_t ng, uint8_t* __restrict__ records, uint32_t* flags) {
+  using L = QuantLayout<BITS, G, D>;
+  constexpr int levels = (1 << BITS) - 1;
+  __shared__ __align__(16) __nv_bfloat16 ks[G][D];
+  __shared__ __align__(16) __nv_bfloat16 vs[G][D];
+  __shared__ uint16_t skz[2][D];          // key scale, key zero (natural channel order)
+  __shared__ uint16_t svz[2][G][L::CPG];  // value scale, value zero per (token, value group)
+  __shared__ double kinv[D];
+  __shared__ double vinv[G][L::CPG];
+  const int tid = threadIdx.x;
+  const int64_t grp = blockIdx.x;
+  const int64_t unit = blockIdx.y;
+  const uint4* kg = reinterpret_cast<const uint4*>(k + (unit * T + grp * G) * D);
+  const uint4* vg = reinterpret_cast<const uint4*>(v + (unit * T + grp * G) * D);
+  for (int e = tid; e < G * D / 8; e += 128) {  // stage the group's rows, 16-byte loads
+    reinterpret_cast<uint4*>(&ks[0][0])[e] = kg[e];
+    reinterpret_cast<uint4*>(&vs[0][0])[e] = vg[e];
+  }
+  __syncthreads();
+  auto K = [&](int t, int c) { return __bfloat162float(ks[t][c]); };
+  auto V = [&](int t, int c) { return __bfloat162float(vs[t][c]); };
+
+  // key parameters: channel c over the group's G tokens
+  for (int c = tid; c < D; c += 128) {
+    float mn = K(0, c), mx = mn;
+    for (int t = 1; t < G; ++t) mn = fminf(mn, K(t, c)), mx = fmaxf(mx, K(t, c));
+    skz[0][c] = to_half_checked((static_cast<double>(mx) - static_cast<double>(mn)) / levels, flags);
+    skz[1][c] = to_half_checked(static_cast<double>(mn), flags);
+    const double sd = half_bits_to_double(skz[0][c]);
+    kinv[c] = sd != 0.0 ? 1.0 / sd : 0.0;
+  }
+  // value parameters: token t, value group cg over its G channels
+  for (int e = tid; e < G * L::CPG; e += 128) {
+    const int t = e / L::CPG, cg = e % L::CPG;
+    float mn = V(t, cg * G), mx = mn;
+    for (int c = 1; c < G; ++c) mn = fminf(mn, V(t, cg * G + c)), mx = fmaxf(mx, V(t, cg * G + c));
+    svz[0][t][cg] = to_half_checked((static_cast<double>(mx) - static_cast<double>(mn)) / levels, flags);
+    svz[1][t][cg] = to_half_checked(static_cast<double>(mn), flags);
+    const double sd = half_bits_to_double(svz[0][t][cg]);
+    vinv[t][cg] = sd != 0.0 ? 1.0 / sd : 0.0;
+  }
+  __syncthreads();
+  auto kcode = [&](int t, int c) -> uint32_t {
+    return quant_code(K(t, c), half_bits_to_double(skz[0][c]), half_bits_to_double(skz[1][c]), kinv[c], levels);
+  };
+  auto vcode = [&](int t, int c) -> uint32_t {
+    const int cg = c / G;
+    return quant_code(V(t, c), half_bits_to_double(svz[0][t][cg]), half_bits_to_double(svz[1][t][cg]), vinv[t][cg],
+                      levels);
+  };
+
+  uint8_t* rec = records + (unit * ng + grp) * L::REC;
+  uint32_t* kw = reinterpret_cast<uint32_t*>(rec);
+  uint32_t* vw = reinterpret_cast<uint32_t*>(rec + L::CB);
+  // code words: word index = (tt * 32 + lane) * NW + w, w = 2 j + (0: X, 1: Y);
+  // local tile i of pair j covers channel (key) / channel-row (value) tile TPW j + i;
+  // first register's codes at bits [b i] and [16 + b i], second's at [8 + b i], [24 + b i]
+  for (int wi = tid; wi < L::WORDS; wi += 128) {
+    const int w = wi % L::NW, rest = wi / L::NW;
+    const int lane = rest % 32, tt = rest / 32;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int j = w >> 1, isY = w & 1;
+    uint32_t kword = 0, vword = 0;
+#pragma unroll
+    for (int i = 0; i < L::TPW; ++i) {
+      const int ct = L::TPW * j + i;
+      {  // keys: X = (reg0: token gid, reg1: token gid + 8) at channels 16 ct + 2 tig (+8 in Y)
+        const int c = 16 * ct + 2 * tig + (isY ? 8 : 0);
+        const int t0 = 16 * tt + gid, t1 = t0 + 8;
+        kword |= kcode(t0, c) << (BITS * i);
+        kword |= kcode(t0, c + 1) << (16 + BITS * i);
+        kword |= kcode(t1, c) << (8 + BITS * i);
+        kword |= kcode(t1, c + 1) << (24 + BITS * i);
+      }
+      {  // values: X = (reg0: channel gid, reg2: tokens + 8), Y = (reg1: channel gid + 8, reg3)
+        const int c = 16 * ct + gid + (isY ? 8 : 0);
+        const int t0 = 16 * tt + 2 * tig, t1 = t0 + 8;
+        vword |= vcode(t0, c) << (BITS * i);
+        vword |= vcode(t0 + 1, c) << (16 + BITS * i);
+        vword |= vcode(t1, c) << (8 + BITS * i);
+        vword |= vcode(t1 + 1, c) << (24 + BITS * i);
+      }
+    }
+    kw[wi] = kword;
+    vw[wi] = vword;
+  }
+  // key parameters in fragment order: channel c = 16 kt + 8 h + 2 t + e at
+  // fp16 slot 2 (t * 2 (D/16) + 2 kt + h) + e
+  uint16_t* sk = reinterpret_cast<uint16_t*>(rec + 2 * L::CB);
+  uint16_t* zk = sk + D;
+  for (int c = tid; c < D; c += 128) {
+    const int kt = c >> 4, h = (c >> 3) & 1, t = (c >> 1) & 3, e = c & 1;
+    const int slot = 2 * (t * 2 * L::KT + 2 * kt + h) + e;
+    sk[slot] = skz[0][c];
+    zk[slot] = skz[1][c];
+  }
+  // value parameters pair-interleaved: [G/2][CPG][2]
+  uint16_t* sv = zk + D;
+  uint16_t* zv = sv + D;
+  for (int e = tid; e < G * L::CPG; e += 128) {
+    const int t = e / L::CPG, cg = e % L::CPG;
+    const int slot = ((t >> 1) * L::CPG + cg) * 2 + (t & 1);
+    sv[slot] = svz[0][t][cg];
+    zv[slot] = svz[1][t][cg];
+  }
+}
+
+// The newest R rows of every unit into the residual buffers (rows 0..R-1 of R_cap).
+__global__ void copy_residual_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int64_t T, int64_t L_q,
+                                     int R, int R_cap, int D, uint4* __restrict__ kr, uint4* __restrict__ vr,
+                                     int64_t units) {
+  const int vec = D / 8;  // uint4 per row
+  const int64_t n = units * R * vec;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t u = e / (static_cast<int64_t>(R) * vec);
+    const int64_t rem = e - u * R * vec;
+    const int64_t r = rem / vec, x = rem - r * vec;
+    kr[(u * R_cap + r) * vec + x] = k[(u * T + L_q + r) * vec + x];
+    vr[(u * R_cap + r) * vec + x] = v[(u * T + L_q + r) * vec + x];
+  }
+}
+
+// Kept rows into the pool: one warp per (unit, kept row); lanes 0-15 copy the
+// K row, lanes 16-31 the V row, 16 bytes each per step.  An index outside
+// [0, T_store) writes a zero row and raises VC_FLAG_BAD_INDEX.
+__global__ void compact_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                               int64_t T_store, const int32_t* __restrict__ idx, int n_keep, int D, int64_t units,
+                               __nv_bfloat16* __restrict__ ko, __nv_bfloat16* __restrict__ vo, uint32_t* flags) {
+  const int lane = threadIdx.x & 31;
+  const int vec = D / 8;
+  const int64_t rows = units * n_keep;
+  for (int64_t rw = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) / 32; rw < rows;
+       rw += static_cast<int64_t>(gridDim.x) * blockDim.x / 32) {
+    const int64_t u = rw / n_keep;
+    const int32_t p = idx[rw];
+    const bool okp = p >= 0 && p < T_store;
+    if (!okp && lane == 0 && flags) atomicOr(flags, VC_FLAG_BAD_INDEX);
+    const bool isv = lane >= 16;
+    const int l = lane & 15;
+    const uint4* src = reinterpret_cast<const uint4*>((isv ? v : k) + (u * T_store + (okp ? p : 0)) * D);
+    uint4* dst = reinterpret_cast<uint4*>((isv ? vo : ko) + rw * D);
+    for (int x = l; x < vec; x += 16) dst[x] = okp ? src[x] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <typename F>
+bool dispatch_q(int bits, int group, int D, F&& f) {
+#define VC_QQ_CASE(BI, GR, DD)                                                                                \
+  if (bits == BI && group == GR && D == DD) {                                                                 \
+    f(std::integral_constant<int, BI>{}, std::integral_constant<int, GR>{}, std::integral_constant<int, DD>{}); \
+    return true;                                                                                              \
+  }
+  VC_QQ_CASE(2, 32, 128) VC_QQ_CASE(2, 64, 128) VC_QQ_CASE(4, 32, 128) VC_QQ_CASE(4, 64, 128)
+  VC_QQ_CASE(2, 32, 64) VC_QQ_CASE(2, 64, 64) VC_QQ_CASE(4, 32, 64) VC_QQ_CASE(4, 64, 64)
+#undef VC_QQ_CASE
+  return false;
+}
+
+}  // namespace
+}  // namespace vc
+
+extern "C" {
+
+size_t vc_compress_workspace_size(void) { return vc::align_up(sizeof(vc::WsHeader), 256); }
+
+vc_status vc_quantize_cache(const vc_attn_shape* shape, const void* k, const void* v, int64_t T, int bits, int group,
+                            int64_t L_q, void* records, void* k_res, void* v_res, int R_cap, void* ws,
+                            size_t ws_bytes, void* stream) {
+  VC_REQUIRE(shape, "vc_quantize_cache: null shape");
+  const vc_attn_shape& sh = *shape;
+  VC_REQUIRE(sh.B >= 1 && sh.Hkv >= 1, "vc_quantize_cache: need B >= 1 and Hkv >= 1");
+  VC_REQUIRE(sh.D == 64 || sh.D == 128, "vc_quantize_cache: head dim must be 64 or 128 (got %d)", sh.D);
+  VC_REQUIRE(bits == 2 || bits == 4, "vc_quantize_cache: bits must be 2 or 4 (got %d)", bits);
+  VC_REQUIRE(group == 32 || group == 64, "vc_quantize_cache: group must be 32 or 64 (got %d)", group);
+  VC_REQUIRE(L_q >= 0 && L_q % group == 0 && L_q <= T, "vc_quantize_cache: need 0 <= L_q <= T, L_q a multiple of group");
+  VC_REQUIRE(T >= 1, "vc_quantize_cache: T must be >= 1");
+  const int64_t R = T - L_q;
+  VC_REQUIRE(R <= R_cap, "vc_quantize_cache: the %lld newest rows do not fit the residual (R_cap %d)",
+             static_cast<long long>(R), R_cap);
+  VC_REQUIRE(k && v && ws, "vc_quantize_cache: null k, v or workspace");
+  VC_REQUIRE(L_q == 0 || records, "vc_quantize_cache: null records");
+  VC_REQUIRE(R == 0 || (k_res && v_res), "vc_quantize_cache: null residual buffers");
+  VC_REQUIRE(vc::aligned16(k) && vc::aligned16(v) && vc::aligned16(records) && vc::aligned16(k_res) &&
+                 vc::aligned16(v_res) && vc::aligned16(ws),
+             "vc_quantize_cache: pointers must be 16-byte aligned");
+  VC_REQUIRE(ws_bytes >= vc_compress_workspace_size(), "vc_quantize_cache: workspace too small");
+  VC_REQUIRE(L_q / group <= 2147483647 && static_cast<int64_t>(sh.B) * sh.Hkv <= 65535,
+             "vc_quantize_cache: too many groups or units");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* flags = static_cast<uint32_t*>(ws);
+  const int64_t ng = L_q / group;
+  const int64_t units = static_cast<int64_t>(sh.B) * sh.Hkv;
+  if (ng > 0) {
+    vc::dispatch_q(bits, group, sh.D, [&](auto BI, auto GR, auto DD) {
+      dim3 grid(static_cast<unsigned>(ng), static_cast<unsigned>(units));
+      vc::quantize_kernel<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value><<<grid, 128, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), T, ng,
+          static_cast<uint8_t*>(records), flags);
+    });
+  }
+  if (R > 0) {
+    const int64_t n = units * R * (sh.D / 8);
+    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 148 * 8));
+    vc::copy_residual_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), T,
+                                                     L_q, static_cast<int>(R), R_cap, sh.D, static_cast<uint4*>(k_res),
+                                                     static_cast<uint4*>(v_res), units);
+  }
+  return vc::launch_status("vc_quantize_cache");
+}
+
+vc_status vc_compact_kept(const vc_attn_shape* shape, const void* k, const void* v, int64_t T_store,
+                          const int32_t* idx, int n_keep, void* k_out, void* v_out, void* ws, size_t ws_bytes,
+                          void* stream) {
+  VC_REQUIRE(shape, "vc_compact_kept: null shape");
+  const vc_attn_shape& sh = *shape;
+  VC_REQUIRE(sh.B >= 1 && sh.Hkv >= 1, "vc_compact_kept: need B >= 1 and Hkv >= 1");
+  VC_REQUIRE(sh.D == 64 || sh.D == 128, "vc_compact_kept: head dim must be 64 or 128 (got %d)", sh.D);
+  VC_REQUIRE(T_store >= 1 && n_keep >= 1, "vc_compact_kept: need T_store >= 1 and n_keep >= 1");
+  VC_REQUIRE(k && v && idx && k_out && v_out, "vc_compact_kept: null pointer");
+  VC_REQUIRE(vc::aligned16(k) && vc::aligned16(v) && vc::aligned16(k_out) && vc::aligned16(v_out),
+             "vc_compact_kept: K/V pointers must be 16-byte aligned");
+  VC_REQUIRE(ws == nullptr || ws_bytes >= vc_compress_workspace_size(), "vc_compact_kept: workspace too small");
+  const int64_t units = static_cast<int64_t>(sh.B) * sh.Hkv;
+  const int64_t rows = units * n_keep;
+  const int blocks = static_cast<int>(std::min<int64_t>((rows * 32 + 255) / 256, 148 * 16));
+  vc::compact_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), T_store, idx, n_keep, sh.D, units,
+      static_cast<__nv_bfloat16*>(k_out), static_cast<__nv_bfloat16*>(v_out), static_cast<uint32_t*>(ws));
+  return vc::launch_status("vc_compact_kept");
+}
+
+}  // extern "C"

@@ -27,6 +27,7 @@ VC_ERR_WORKSPACE = -5
 VC_F32, VC_BF16, VC_F16 = 0, 1, 2
 VC_FLAG_BAD_INDEX = 1
 VC_FLAG_WAIT_TIMEOUT = 2
+VC_FLAG_RANGE = 4
 
 
 class VcError(RuntimeError):
@@ -100,6 +101,12 @@ def lib() -> ctypes.CDLL:
             "vc_draft_attn_quant_noalloc_flags": (c_int, [P(c_uint32), c_void_p]),
             "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
             "vc_debug_wait_timeout": (c_int, [c_void_p, c_void_p, ctypes.c_int64, c_void_p]),
+            "vc_compress_workspace_size": (c_size_t, []),
+            "vc_quantize_cache": (c_int, [P(vc_attn_shape), c_void_p, c_void_p, ctypes.c_int64, c_int, c_int,
+                                          ctypes.c_int64, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_size_t,
+                                          c_void_p]),
+            "vc_compact_kept": (c_int, [P(vc_attn_shape), c_void_p, c_void_p, ctypes.c_int64, c_void_p, c_int,
+                                        c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
             "vc_debug_quant_partition": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_int, c_void_p, c_int,
                                                  P(c_int), P(c_int), P(c_int), P(c_int), P(c_int)]),
             "vc_kvstream_create": (c_int, [P(c_void_p), c_int, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p,
@@ -244,6 +251,25 @@ def vc_draft_attn_quant_noalloc_flags(stream=None) -> int:
 
 def vc_debug_dequant(sh, qc, k_out, v_out, stream=None):
     _check(lib().vc_debug_dequant(ctypes.byref(sh), ctypes.byref(qc), _p(k_out), _p(v_out), _stream(stream)))
+
+
+def vc_compress_workspace_size() -> int:
+    return lib().vc_compress_workspace_size()
+
+
+def vc_quantize_cache(sh, k, v, T: int, bits: int, group: int, L_q: int, records, k_res, v_res, R_cap: int, ws,
+                      stream=None):
+    """Full bf16 K, V [B, Hkv, T, D] -> group records of the oldest L_q rows
+    plus the residual rows (see include/vc.h)."""
+    _check(lib().vc_quantize_cache(ctypes.byref(sh), _p(k), _p(v), int(T), int(bits), int(group), int(L_q),
+                                   _p(records), _p(k_res), _p(v_res), int(R_cap), _p(ws), ws.numel(),
+                                   _stream(stream)))
+
+
+def vc_compact_kept(sh, k, v, T_store: int, idx, n_keep: int, k_out, v_out, ws=None, stream=None):
+    """Kept rows of k, v into a pool [B, Hkv, n_keep, D] (see include/vc.h)."""
+    _check(lib().vc_compact_kept(ctypes.byref(sh), _p(k), _p(v), int(T_store), _p(idx), int(n_keep), _p(k_out),
+                                 _p(v_out), _p(ws), ws.numel() if ws is not None else 0, _stream(stream)))
 
 
 def vc_debug_wait_timeout(flags, result, limit_ns: int, stream=None):

@@ -190,3 +190,23 @@ def test_wait_timeout_export_rejects_before_any_launch(L):
     assert L.vc_debug_wait_timeout(16, None, 1000000, None) == vc.VC_ERR_INVALID_ARG
     assert L.vc_debug_wait_timeout(16, 16, 999, None) == vc.VC_ERR_INVALID_ARG
     assert L.vc_debug_wait_timeout(16, 16, 200000000, None) == vc.VC_ERR_INVALID_ARG
+
+
+def test_compression_calls_reject_before_any_launch(L):
+    import ctypes
+    sh = vc.shape(1, 4, 2, 128)
+    ws = 256
+    ok = dict(k=16, v=16, T=160, bits=2, group=32, L_q=128, records=16, k_res=16, v_res=16, R_cap=32)
+
+    def quant(**kw):
+        a = dict(ok, **kw)
+        return L.vc_quantize_cache(ctypes.byref(sh), a["k"], a["v"], a["T"], a["bits"], a["group"], a["L_q"],
+                                   a["records"], a["k_res"], a["v_res"], a["R_cap"], ws, 256, None)
+    for bad in (dict(bits=3), dict(group=48), dict(L_q=100), dict(L_q=200), dict(R_cap=16), dict(k=None),
+                dict(records=None), dict(k_res=None), dict(k=17)):
+        assert quant(**bad) == vc.VC_ERR_INVALID_ARG, bad
+    assert L.vc_compress_workspace_size() >= 16
+    # compaction: zero kept rows, null index list, misaligned pool
+    assert L.vc_compact_kept(ctypes.byref(sh), 16, 16, 100, 16, 0, 16, 16, None, 0, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_compact_kept(ctypes.byref(sh), 16, 16, 100, None, 8, 16, 16, None, 0, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_compact_kept(ctypes.byref(sh), 16, 16, 100, 16, 8, 18, 16, None, 0, None) == vc.VC_ERR_INVALID_ARG
