@@ -13,11 +13,12 @@
 // Quantisation rule (the library's reading, identical to the oracle's):
 // per group, s = fp16(round-to-nearest((max - min) / (2^b - 1))),
 // z = fp16(min), code = clamp(rint((x - z) / s), 0, 2^b - 1) with the STORED
-// s and z, half to even; s == 0 gives code 0.  The quotient is evaluated so
-// that every code equals the one an exact float64 division gives: x - z of
-// a bf16 and an fp16 value is exact in float64, the quotient is first taken
-// as (x - z) * (1 / s) and, when it lies within 1e-9 of a rounding tie
-// (k + 1/2), recomputed with an IEEE float64 division.
+// s and z, half to even; s == 0 gives code 0.  Every code equals the one the
+// float64 quotient gives: the quotient is first taken in fp32 as
+// (x - z) * (1 / s), whose error is below 2^-18 for the quotients that are
+// not clamped (|q| <= 16); only when that lands within 2^-12 of a rounding
+// tie (k + 1/2) is it recomputed as an IEEE float64 division of the exact
+// float64 difference.
 #include "vc_common.cuh"
 
 namespace vc {
@@ -38,15 +39,17 @@ __device__ __forceinline__ double half_bits_to_double(uint16_t b) {
   return static_cast<double>(__half2float(__ushort_as_half(b)));
 }
 
-// code = clamp(rint((x - z) / s), 0, levels); s == 0 -> 0
-__device__ __forceinline__ uint32_t quant_code(float x, double s, double z, double inv_s, int levels) {
-  if (s == 0.0) return 0u;
-  const double d = static_cast<double>(x) - z;  // exact: x is bf16, z is fp16
-  double q = d * inv_s;
-  const double f = q - floor(q);
-  if (fabs(f - 0.5) < 1e-9) q = d / s;  // near a tie: the exact quotient decides
-  double r = rint(q);
-  r = r < 0.0 ? 0.0 : (r > levels ? static_cast<double>(levels) : r);
+// code = clamp(rint((x - z) / s), 0, levels); s == 0 -> 0 (inv_s is then 0).
+// sz points at the stored (scale, zero) fp16 bits, read only on the slow path.
+__device__ __forceinline__ uint32_t quant_code(float x, float2 zi, int levels, const uint16_t* s_bits,
+                                               const uint16_t* z_bits) {
+  const float q = (x - zi.x) * zi.y;
+  float r = rintf(q);
+  if (fabsf(fabsf(q - r) - 0.5f) < 2.44140625e-4f && zi.y != 0.f) {  // near a tie: the exact quotient decides
+    const double sd = half_bits_to_double(*s_bits), zd = half_bits_to_double(*z_bits);
+    r = static_cast<float>(rint((static_cast<double>(x) - zd) / sd));
+  }
+  r = fminf(fmaxf(r, 0.f), static_cast<float>(levels));
   return static_cast<uint32_t>(r);
 }
 
@@ -77,8 +80,8 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __re
   __shared__ __align__(16) __nv_bfloat16 vs[G][D];
   __shared__ uint16_t skz[2][D];          // key scale, key zero (natural channel order)
   __shared__ uint16_t svz[2][G][L::CPG];  // value scale, value zero per (token, value group)
-  __shared__ double kinv[D];
-  __shared__ double vinv[G][L::CPG];
+  __shared__ float2 kzi[D];           // key zero, 1 / key scale (0 when the scale is 0), fp32
+  __shared__ float2 vzi[G][L::CPG];   // the same per value group
   const int tid = threadIdx.x;
   const int64_t grp = blockIdx.x;
   const int64_t unit = blockIdx.y;
@@ -98,8 +101,8 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __re
     for (int t = 1; t < G; ++t) mn = fminf(mn, K(t, c)), mx = fmaxf(mx, K(t, c));
     skz[0][c] = to_half_checked((static_cast<double>(mx) - static_cast<double>(mn)) / levels, flags);
     skz[1][c] = to_half_checked(static_cast<double>(mn), flags);
-    const double sd = half_bits_to_double(skz[0][c]);
-    kinv[c] = sd != 0.0 ? 1.0 / sd : 0.0;
+    const float sf = __half2float(__ushort_as_half(skz[0][c]));
+    kzi[c] = make_float2(__half2float(__ushort_as_half(skz[1][c])), sf != 0.f ? 1.f / sf : 0.f);
   }
   // value parameters: token t, value group cg over its G channels
   for (int e = tid; e < G * L::CPG; e += 128) {
@@ -108,17 +111,13 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __re
     for (int c = 1; c < G; ++c) mn = fminf(mn, V(t, cg * G + c)), mx = fmaxf(mx, V(t, cg * G + c));
     svz[0][t][cg] = to_half_checked((static_cast<double>(mx) - static_cast<double>(mn)) / levels, flags);
     svz[1][t][cg] = to_half_checked(static_cast<double>(mn), flags);
-    const double sd = half_bits_to_double(svz[0][t][cg]);
-    vinv[t][cg] = sd != 0.0 ? 1.0 / sd : 0.0;
+    const float sf = __half2float(__ushort_as_half(svz[0][t][cg]));
+    vzi[t][cg] = make_float2(__half2float(__ushort_as_half(svz[1][t][cg])), sf != 0.f ? 1.f / sf : 0.f);
   }
   __syncthreads();
-  auto kcode = [&](int t, int c) -> uint32_t {
-    return quant_code(K(t, c), half_bits_to_double(skz[0][c]), half_bits_to_double(skz[1][c]), kinv[c], levels);
-  };
   auto vcode = [&](int t, int c) -> uint32_t {
     const int cg = c / G;
-    return quant_code(V(t, c), half_bits_to_double(svz[0][t][cg]), half_bits_to_double(svz[1][t][cg]), vinv[t][cg],
-                      levels);
+    return quant_code(V(t, c), vzi[t][cg], levels, &svz[0][t][cg], &svz[1][t][cg]);
   };
 
   uint8_t* rec = records + (unit * ng + grp) * L::REC;
@@ -139,10 +138,13 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __re
       {  // keys: X = (reg0: token gid, reg1: token gid + 8) at channels 16 ct + 2 tig (+8 in Y)
         const int c = 16 * ct + 2 * tig + (isY ? 8 : 0);
         const int t0 = 16 * tt + gid, t1 = t0 + 8;
-        kword |= kcode(t0, c) << (BITS * i);
-        kword |= kcode(t0, c + 1) << (16 + BITS * i);
-        kword |= kcode(t1, c) << (8 + BITS * i);
-        kword |= kcode(t1, c + 1) << (24 + BITS * i);
+        const float2 z0 = kzi[c], z1 = kzi[c + 1];
+        const float2 x0 = unpack_bf2(*reinterpret_cast<const uint32_t*>(&ks[t0][c]));
+        const float2 x1 = unpack_bf2(*reinterpret_cast<const uint32_t*>(&ks[t1][c]));
+        kword |= quant_code(x0.x, z0, levels, &skz[0][c], &skz[1][c]) << (BITS * i);
+        kword |= quant_code(x0.y, z1, levels, &skz[0][c + 1], &skz[1][c + 1]) << (16 + BITS * i);
+        kword |= quant_code(x1.x, z0, levels, &skz[0][c], &skz[1][c]) << (8 + BITS * i);
+        kword |= quant_code(x1.y, z1, levels, &skz[0][c + 1], &skz[1][c + 1]) << (24 + BITS * i);
       }
       {  // values: X = (reg0: channel gid, reg2: tokens + 8), Y = (reg1: channel gid + 8, reg3)
         const int c = 16 * ct + gid + (isY ? 8 : 0);
