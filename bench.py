@@ -374,6 +374,8 @@ def run_gpu(args, w, rank, world):
            + h_lg.numel() * h_lg.element_size() + h_dt.numel() * h_dt.element_size())
     d2h = h_out.numel() * h_out.element_size() + h_res.numel() * h_res.element_size()
 
+    compress = time_compress(w, dev, inp) if rank == 0 else None
+
     streamed = None
     if w.get("streamed_too"):
         streamed = time_streamed_verify(args, w, dev, inp, sh, ws_v, out_v, stream)
@@ -381,8 +383,56 @@ def run_gpu(args, w, rank, world):
     total_ms, draft_ms, verify_ms, accept_ms, e2e_total_ms, e2e_draft_ms = max_over_ranks(
         [total_ms, draft_ms, verify_ms, accept_ms, e2e_total_ms, e2e_draft_ms], dev)
     return dict(total_ms=total_ms, draft_ms=draft_ms, verify_ms=verify_ms, accept_ms=accept_ms,
-                e2e_total_ms=e2e_total_ms, e2e_draft_ms=e2e_draft_ms, h2d=h2d, d2h=d2h, clocks=clk,
+                e2e_total_ms=e2e_total_ms, e2e_draft_ms=e2e_draft_ms, h2d=h2d, d2h=d2h, clocks=clk, compress=compress,
                 streamed=streamed)
+
+
+def time_compress(w, dev, inp):
+    """Building the draft caches on the GPU for one layer of the workload:
+    quantising its full K and V into group records + residual, and gathering
+    25% kept rows into a kept-row pool.  Device time per call (CUDA events,
+    inputs larger than L2) and algorithmic bytes (full rows read, records and
+    residual or pool rows written)."""
+    import torch
+    from lossless_draft_verify_vc_b200 import synth, vc
+    B, Hkv, D, T, R, G, bits = w["B"], w["Hkv"], w["D"], w["T"], w["R"], w["G"], w["bits"]
+    k, v = inp["kvs"][0]
+    k2, v2 = inp["kvs"][1 % len(inp["kvs"])]
+    L_q = T - R
+    rec_b = 2 * G * D * bits // 8 + 8 * D
+    records = torch.empty((B, Hkv, L_q // G, rec_b), dtype=torch.uint8, device=dev)
+    kr = torch.empty((B, Hkv, R, D), dtype=torch.bfloat16, device=dev)
+    vr = torch.empty_like(kr)
+    ws = vc.workspace(vc.vc_compress_workspace_size(), dev)
+    sh = inp["sh"]
+    n_keep = T // 4
+    idx = synth.kept_positions(B, Hkv, T, n_keep, seed=77, device=dev)
+    ko = torch.empty((B, Hkv, n_keep, D), dtype=torch.bfloat16, device=dev)
+    vo = torch.empty_like(ko)
+
+    def timed(fn, n=10):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) * 1e3 / n
+
+    q_us = timed(lambda i: vc.vc_quantize_cache(sh, k if i % 2 else k2, v if i % 2 else v2, T, bits, G, L_q,
+                                                records, kr, vr, R, ws))
+    c_us = timed(lambda i: vc.vc_compact_kept(sh, k if i % 2 else k2, v if i % 2 else v2, T, idx, n_keep, ko, vo,
+                                              ws))
+    flags = vc.vc_workspace_flags(ws)
+    q_bytes = 2 * B * Hkv * T * D * 2 + records.numel() + 2 * B * Hkv * R * D * 2
+    c_bytes = 2 * 2 * B * Hkv * n_keep * D * 2 + idx.numel() * 4
+    del records, kr, vr, ko, vo
+    return dict(quantize_us=q_us, quantize_gbps=q_bytes / (q_us * 1e-6) / 1e9, quantize_bytes=q_bytes,
+                compact_us=c_us, compact_gbps=c_bytes / (c_us * 1e-6) / 1e9, compact_bytes=c_bytes,
+                compact_kept_per_head=n_keep, flags=flags)
 
 
 def time_streamed_verify(args, w, dev, inp, sh, ws_v, out_v, comp):
@@ -795,6 +845,16 @@ def resident_line(args, w, rank, world, config, peak, peak_kind):
         "gpu_launches": (K * NL + 2 * NL + 1) * args.steps,
         "clocks": r["clocks"],
     }
+    if r.get("compress"):
+        cp = r["compress"]
+        line["compress"] = {
+            "note": "building one layer's draft caches on the GPU (vc_quantize_cache: full K/V -> group records "
+                    "+ residual; vc_compact_kept: 25% kept rows -> pool); device time per call",
+            "quantize_us": cp["quantize_us"], "quantize_gbps": cp["quantize_gbps"],
+            "quantize_frac_of_hbm_peak": cp["quantize_gbps"] / peak, "quantize_bytes": cp["quantize_bytes"],
+            "compact_us": cp["compact_us"], "compact_gbps": cp["compact_gbps"],
+            "compact_frac_of_hbm_peak": cp["compact_gbps"] / peak, "compact_bytes": cp["compact_bytes"],
+            "flags": cp["flags"]}
     if r.get("streamed"):
         sv = r["streamed"]
         line["verify_streamed"] = {"round_us": sv["round_us"], "link_gbps": sv["link_gbps"],
