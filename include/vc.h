@@ -75,6 +75,7 @@ typedef enum vc_dtype { VC_F32 = 0, VC_BF16 = 1, VC_F16 = 2 } vc_dtype;
 #define VC_FLAG_BAD_INDEX 1u   /* a kept position was outside [0, T_store) */
 #define VC_FLAG_WAIT_TIMEOUT 2u /* a bounded on-chip wait gave up */
 #define VC_FLAG_RANGE 4u        /* a quantisation scale or zero fell outside the fp16 range */
+#define VC_FLAG_BAD_LENGTH 8u   /* a per-request length or accepted length was invalid; that request was skipped */
 
 /* Message for the last error returned on the calling thread ("" if none). */
 VC_API const char* vc_last_error(void);
@@ -162,6 +163,13 @@ typedef struct vc_quant_cache {
   int64_t L_q;
   int R;
   int R_cap;
+  /* Optional device int32 [B][2]: the (L_q, R) of each request, for caches
+   * maintained on the device across rounds (vc_cache_commit).  When set, L_q
+   * above is the record capacity in tokens (records holds L_q / group records
+   * per (request, KV head)), R above is ignored, and request b uses its own
+   * lens[b] = (L_q_b, R_b) with L_q_b a multiple of group, L_q_b <= L_q and
+   * R_b <= R_cap.  NULL: every request has L_q and R. */
+  const int32_t* lens;
 } vc_quant_cache;
 
 /* One layer of a token-dropped draft cache: every (request, KV head) keeps
@@ -265,6 +273,30 @@ VC_API vc_status vc_quantize_cache(const vc_attn_shape* shape, const void* k, co
 VC_API vc_status vc_compact_kept(const vc_attn_shape* shape, const void* k, const void* v, int64_t T_store,
                                  const int32_t* idx, int n_keep, void* k_out, void* v_out, void* ws,
                                  size_t ws_bytes, void* stream);
+
+/* ---- cache maintenance around a round -----------------------------------------
+ * After acceptance, a round keeps the accepted prefix plus the verifier's
+ * correction and discards the rest of the draft (devshah.ca page, "The Core
+ * Idea", the worked example's Emit / Discard lines).  The library's reading:
+ * before a round the caches hold every committed token but the newest (x);
+ * the verification block is (x, d_1 .. d_K), nq = K + 1 rows whose exact K, V
+ * the verifier computes; with a = accept_len[b] the rows x, d_1 .. d_a
+ * (a + 1 rows) are committed and d_(a+1) .. d_K rolled back.
+ * vc_cache_commit appends those rows of k_new, v_new (bf16 [B][Hkv][nq][D],
+ * this layer's block rows) to the bf16 residual of each request's quantised
+ * cache; when the residual would exceed R_cap, its oldest `group` rows first
+ * become one group record (vc_quantize_cache's rule, byte-identical to it)
+ * at index L_q_b / group and the residual keeps the rest.  cache->lens (device
+ * [B][2]) is required and is updated in place; accept_len is a device int32
+ * [B] (vc_accept's output): nothing is read back to the host.  Needs
+ * nq <= group and R_cap >= group + nq - 1.  A request with an accepted length
+ * outside [0, nq), invalid lengths or no record capacity left is left
+ * unchanged and raises VC_FLAG_BAD_LENGTH.  The full bf16 cache needs no data
+ * movement: its committed length simply grows by a + 1.  Workspace: a flag
+ * word of vc_compress_workspace_size() bytes. */
+VC_API vc_status vc_cache_commit(const vc_attn_shape* shape, const vc_quant_cache* cache, const void* k_new,
+                                 const void* v_new, int nq, const int32_t* accept_len, void* ws, size_t ws_bytes,
+                                 void* stream);
 
 /* ---- block verification attention -----------------------------------------
  * One pass over the full cache scores every drafted position at once and

@@ -71,9 +71,9 @@ struct QuantLayout {
 // consume them), computing each code where it is packed, and the block
 // writes words and parameters as one record.
 template <int BITS, int G, int D>
-__global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __restrict__ k,
-                                                       const __nv_bfloat16* __restrict__ v, int64_t T,
-                                                       int64_t ng, uint8_t* __restrict__ records, uint32_t* flags) {
+__device__ __forceinline__ void quantize_group(const __nv_bfloat16* __restrict__ kgp,
+                                               const __nv_bfloat16* __restrict__ vgp, uint8_t* __restrict__ rec,
+                                               uint32_t* flags) {
   using L = QuantLayout<BITS, G, D>;
   constexpr int levels = (1 << BITS) - 1;
   __shared__ __align__(16) __nv_bfloat16 ks[G][D];
@@ -83,10 +83,8 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __re
   __shared__ float2 kzi[D];           // key zero, 1 / key scale (0 when the scale is 0), fp32
   __shared__ float2 vzi[G][L::CPG];   // the same per value group
   const int tid = threadIdx.x;
-  const int64_t grp = blockIdx.x;
-  const int64_t unit = blockIdx.y;
-  const uint4* kg = reinterpret_cast<const uint4*>(k + (unit * T + grp * G) * D);
-  const uint4* vg = reinterpret_cast<const uint4*>(v + (unit * T + grp * G) * D);
+  const uint4* kg = reinterpret_cast<const uint4*>(kgp);
+  const uint4* vg = reinterpret_cast<const uint4*>(vgp);
   for (int e = tid; e < G * D / 8; e += 128) {  // stage the group's rows, 16-byte loads
     reinterpret_cast<uint4*>(&ks[0][0])[e] = kg[e];
     reinterpret_cast<uint4*>(&vs[0][0])[e] = vg[e];
@@ -120,7 +118,6 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __re
     return quant_code(V(t, c), vzi[t][cg], levels, &svz[0][t][cg], &svz[1][t][cg]);
   };
 
-  uint8_t* rec = records + (unit * ng + grp) * L::REC;
   uint32_t* kw = reinterpret_cast<uint32_t*>(rec);
   uint32_t* vw = reinterpret_cast<uint32_t*>(rec + L::CB);
   // code words: word index = (tt * 32 + lane) * NW + w, w = 2 j + (0: X, 1: Y);
@@ -179,6 +176,16 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __re
   }
 }
 
+template <int BITS, int G, int D>
+__global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16* __restrict__ k,
+                                                       const __nv_bfloat16* __restrict__ v, int64_t T,
+                                                       int64_t ng, uint8_t* __restrict__ records, uint32_t* flags) {
+  using L = QuantLayout<BITS, G, D>;
+  const int64_t grp = blockIdx.x, unit = blockIdx.y;
+  quantize_group<BITS, G, D>(k + (unit * T + grp * G) * D, v + (unit * T + grp * G) * D,
+                             records + (unit * ng + grp) * L::REC, flags);
+}
+
 // The newest R rows of every unit into the residual buffers (rows 0..R-1 of R_cap).
 __global__ void copy_residual_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int64_t T, int64_t L_q,
                                      int R, int R_cap, int D, uint4* __restrict__ kr, uint4* __restrict__ vr,
@@ -215,6 +222,108 @@ __global__ void compact_kernel(const __nv_bfloat16* __restrict__ k, const __nv_b
     const uint4* src = reinterpret_cast<const uint4*>((isv ? v : k) + (u * T_store + (okp ? p : 0)) * D);
     uint4* dst = reinterpret_cast<uint4*>((isv ? vo : ko) + rw * D);
     for (int x = l; x < vec; x += 16) dst[x] = okp ? src[x] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// ---- cache maintenance after a round (vc_cache_commit) -----------------------
+// Per request b: a = accept_len[b] accepted drafts, n = a + 1 rows of the
+// verifier's block (x, d_1 .. d_a) are committed.  lens[b] = (L_q, R) of the
+// request's quantised cache.  If R + n > R_cap the oldest `group` residual
+// rows become record L_q / group and the residual keeps rows group .. R - 1;
+// the n rows are appended after the residual.  Three launches in stream
+// order, all deciding from the same (lens, accept_len): re-quantise, rewrite
+// the residual, update lens.  A request whose accepted length is outside
+// [0, nq) or whose records would exceed the capacity is left unchanged and
+// raises VC_FLAG_BAD_LENGTH.
+struct CommitDecision {
+  bool valid, requant;
+  int L_q, R, n;
+};
+
+__device__ __forceinline__ CommitDecision commit_decision(const int32_t* lens, const int32_t* accept, int b, int nq,
+                                                          int R_cap, int G, int64_t ng_cap) {
+  CommitDecision d;
+  d.L_q = lens[2 * b];
+  d.R = lens[2 * b + 1];
+  const int a = accept[b];
+  d.n = a + 1;
+  d.requant = d.R + d.n > R_cap;
+  d.valid = a >= 0 && a < nq && d.R >= 0 && d.R <= R_cap && d.L_q >= 0 && d.L_q % G == 0 &&
+            (!d.requant || (d.R >= G && d.L_q / G < ng_cap));
+  return d;
+}
+
+template <int BITS, int G, int D>
+__global__ void __launch_bounds__(128) commit_requant_kernel(const __nv_bfloat16* __restrict__ k_res,
+                                                             const __nv_bfloat16* __restrict__ v_res, int R_cap,
+                                                             uint8_t* __restrict__ records, int64_t ng_cap,
+                                                             const int32_t* __restrict__ lens,
+                                                             const int32_t* __restrict__ accept, int Hkv, int nq,
+                                                             uint32_t* flags) {
+  using L = QuantLayout<BITS, G, D>;
+  const int64_t u = blockIdx.x;
+  const int b = static_cast<int>(u / Hkv);
+  const CommitDecision d = commit_decision(lens, accept, b, nq, R_cap, G, ng_cap);
+  if (!d.valid) {
+    if (threadIdx.x == 0 && u % Hkv == 0 && flags) atomicOr(flags, VC_FLAG_BAD_LENGTH);
+    return;
+  }
+  if (!d.requant) return;
+  quantize_group<BITS, G, D>(k_res + u * R_cap * D, v_res + u * R_cap * D,
+                             records + (u * ng_cap + d.L_q / G) * L::REC, flags);
+}
+
+// Residual rewrite of one unit: rows kept (group .. R - 1 after a re-quantisation,
+// else none move) are staged in shared memory and written back from row 0,
+// then the n committed rows follow.
+__global__ void __launch_bounds__(256) commit_residual_kernel(__nv_bfloat16* __restrict__ k_res,
+                                                              __nv_bfloat16* __restrict__ v_res, int R_cap, int D,
+                                                              const __nv_bfloat16* __restrict__ k_new,
+                                                              const __nv_bfloat16* __restrict__ v_new, int nq,
+                                                              const int32_t* __restrict__ lens,
+                                                              const int32_t* __restrict__ accept, int Hkv, int G,
+                                                              int64_t ng_cap) {
+  extern __shared__ __align__(16) uint4 stage[];
+  const int64_t u = blockIdx.x;
+  const int b = static_cast<int>(u / Hkv);
+  const CommitDecision d = commit_decision(lens, accept, b, nq, R_cap, G, ng_cap);
+  if (!d.valid) return;
+  const int vec = D / 8;  // uint4 per row
+  uint4* kr = reinterpret_cast<uint4*>(k_res + u * R_cap * D);
+  uint4* vr = reinterpret_cast<uint4*>(v_res + u * R_cap * D);
+  int dst = d.R;
+  if (d.requant) {
+    const int kept = d.R - G;
+    for (int e = threadIdx.x; e < kept * vec; e += blockDim.x) {
+      stage[e] = kr[G * vec + e];
+      stage[kept * vec + e] = vr[G * vec + e];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kept * vec; e += blockDim.x) {
+      kr[e] = stage[e];
+      vr[e] = stage[kept * vec + e];
+    }
+    dst = kept;
+  }
+  const uint4* kn = reinterpret_cast<const uint4*>(k_new + u * nq * D);
+  const uint4* vn = reinterpret_cast<const uint4*>(v_new + u * nq * D);
+  for (int e = threadIdx.x; e < d.n * vec; e += blockDim.x) {
+    kr[dst * vec + e] = kn[e];
+    vr[dst * vec + e] = vn[e];
+  }
+}
+
+__global__ void commit_lens_kernel(int32_t* lens, const int32_t* accept, int B, int nq, int R_cap, int G,
+                                   int64_t ng_cap) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
+    const CommitDecision d = commit_decision(lens, accept, b, nq, R_cap, G, ng_cap);
+    if (!d.valid) continue;
+    if (d.requant) {
+      lens[2 * b] = d.L_q + G;
+      lens[2 * b + 1] = d.R + d.n - G;
+    } else {
+      lens[2 * b + 1] = d.R + d.n;
+    }
   }
 }
 
@@ -302,6 +411,52 @@ vc_status vc_compact_kept(const vc_attn_shape* shape, const void* k, const void*
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), T_store, idx, n_keep, sh.D, units,
       static_cast<__nv_bfloat16*>(k_out), static_cast<__nv_bfloat16*>(v_out), static_cast<uint32_t*>(ws));
   return vc::launch_status("vc_compact_kept");
+}
+
+vc_status vc_cache_commit(const vc_attn_shape* shape, const vc_quant_cache* cache, const void* k_new,
+                          const void* v_new, int nq, const int32_t* accept_len, void* ws, size_t ws_bytes,
+                          void* stream) {
+  VC_REQUIRE(shape && cache, "vc_cache_commit: null shape or cache");
+  const vc_attn_shape& sh = *shape;
+  const vc_quant_cache& c = *cache;
+  VC_REQUIRE(sh.B >= 1 && sh.Hkv >= 1 && static_cast<int64_t>(sh.B) * sh.Hkv <= 65535,
+             "vc_cache_commit: need 1 <= B * Hkv <= 65535");
+  VC_REQUIRE(sh.D == 64 || sh.D == 128, "vc_cache_commit: head dim must be 64 or 128 (got %d)", sh.D);
+  VC_REQUIRE(c.bits == 2 || c.bits == 4, "vc_cache_commit: bits must be 2 or 4 (got %d)", c.bits);
+  VC_REQUIRE(c.group == 32 || c.group == 64, "vc_cache_commit: group must be 32 or 64 (got %d)", c.group);
+  VC_REQUIRE(c.lens != nullptr, "vc_cache_commit: the cache needs per-request lengths (lens)");
+  VC_REQUIRE(c.L_q >= 0 && c.L_q % c.group == 0, "vc_cache_commit: record capacity L_q must be a multiple of group");
+  VC_REQUIRE(nq >= 1 && nq <= c.group, "vc_cache_commit: need 1 <= nq <= group (got nq %d)", nq);
+  VC_REQUIRE(c.R_cap >= c.group + nq - 1,
+             "vc_cache_commit: R_cap must be >= group + nq - 1 so an overflowing residual holds a whole group");
+  VC_REQUIRE(c.records && c.k_res && c.v_res && k_new && v_new && accept_len && ws,
+             "vc_cache_commit: null pointer");
+  VC_REQUIRE(vc::aligned16(c.records) && vc::aligned16(c.k_res) && vc::aligned16(c.v_res) &&
+                 vc::aligned16(k_new) && vc::aligned16(v_new),
+             "vc_cache_commit: cache and block pointers must be 16-byte aligned");
+  VC_REQUIRE(ws_bytes >= vc_compress_workspace_size(), "vc_cache_commit: workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* flags = static_cast<uint32_t*>(ws);
+  const int64_t units = static_cast<int64_t>(sh.B) * sh.Hkv;
+  const int64_t ng_cap = c.L_q / c.group;
+  int32_t* lens = const_cast<int32_t*>(c.lens);
+  const auto* kres = static_cast<const __nv_bfloat16*>(c.k_res);
+  const auto* vres = static_cast<const __nv_bfloat16*>(c.v_res);
+  vc::dispatch_q(c.bits, c.group, sh.D, [&](auto BI, auto GR, auto DD) {
+    vc::commit_requant_kernel<decltype(BI)::value, decltype(GR)::value, decltype(DD)::value>
+        <<<static_cast<unsigned>(units), 128, 0, s>>>(kres, vres, c.R_cap, static_cast<uint8_t*>(const_cast<void*>(c.records)),
+                                                      ng_cap, lens, accept_len, sh.Hkv, nq, flags);
+  });
+  const size_t smem = static_cast<size_t>(c.R_cap) * sh.D * 2 * 2;
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(vc::commit_residual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+  vc::commit_residual_kernel<<<static_cast<unsigned>(units), 256, smem, s>>>(
+      static_cast<__nv_bfloat16*>(const_cast<void*>(c.k_res)), static_cast<__nv_bfloat16*>(const_cast<void*>(c.v_res)),
+      c.R_cap, sh.D, static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), nq, lens,
+      accept_len, sh.Hkv, c.group, ng_cap);
+  vc::commit_lens_kernel<<<1, 128, 0, s>>>(lens, accept_len, sh.B, nq, c.R_cap, c.group, ng_cap);
+  return vc::launch_status("vc_cache_commit");
 }
 
 }  // extern "C"

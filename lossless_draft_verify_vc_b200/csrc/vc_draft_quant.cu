@@ -177,12 +177,13 @@ struct QArgs {
   const __nv_bfloat16* vr;
   const __nv_bfloat16* q;
   UPart P;
-  int R, R_cap;
+  int R, R_cap, group;
   int Hq, Hkv, g;
   int MAXS;  // partial slots per block
   float scale_log2;
   uint32_t* flags;
   uint32_t* tickets;  // [U] partials of each unit written so far in this call (back to 0 after it)
+  const int32_t* lens;  // optional [B][2] per-request (L_q, R); NULL: P.ng groups and R rows everywhere
   float* part_o;      // [nblk * MAXS][g][D]
   float* part_ml;     // [nblk * MAXS][g][2]
   float* out;         // [B][Hq][D]
@@ -242,26 +243,64 @@ __device__ __forceinline__ void load_cpg(const uint32_t* p, uint32_t (&w)[CPG]) 
   }
 }
 
+// Groups and residual rows of unit u's request (per-request lengths when the
+// cache carries them; the planned capacity is then an upper bound).
+// Clamped to the planned capacity, so a length the host did not validate can
+// never make a kernel read past the buffers.
+__device__ __forceinline__ int64_t unit_groups(const QArgs& a, int u) {
+  if (!a.lens) return a.P.ng;
+  const int64_t g = a.lens[2 * (u / a.Hkv)] / a.group;
+  return g < 0 ? 0 : (g > a.P.ng ? a.P.ng : g);
+}
+__device__ __forceinline__ int unit_res_rows(const QArgs& a, int u) {
+  if (!a.lens) return a.R;
+  const int r = a.lens[2 * (u / a.Hkv) + 1];
+  return r < 0 ? 0 : (r > a.R_cap ? a.R_cap : r);
+}
+
 // Where this warp's next quantised stage to fetch lives: unit u, unit-local
 // stage ls.  Warp w takes the stages q0 + w, q0 + w + kQNW, ... < q1 of each
 // of its block's units in turn.
 struct IssuePtr {
   int u, ls;
+  int qend;            // end of unit u's quantised stages in this block
   const uint8_t* src;  // record of group ls * NG of unit u
 };
 
+// End of unit u's quantised stages in a block whose planned range ends at q1:
+// with per-request lengths, a request's own stage count can be smaller.
 template <typename C>
-__device__ __forceinline__ void issue_start(const QArgs& a, IssuePtr& ip, int u, int ls) {
-  ip.u = u;
-  ip.ls = ls;
-  ip.src = a.rec + (static_cast<int64_t>(u) * a.P.ng + static_cast<int64_t>(ls) * C::NG) * C::REC;
+__device__ __forceinline__ int unit_qend(const QArgs& a, int u, int q1) {
+  if (!a.lens) return q1;
+  const int sq_u = static_cast<int>((unit_groups(a, u) + C::NG - 1) / C::NG);
+  return sq_u < q1 ? sq_u : q1;
+}
+
+// This warp's stage count in unit u: stages q_first, q_first + kQNW, ... < qend.
+__device__ __forceinline__ int warp_stage_count(int q_first, int qend) {
+  return qend > q_first ? (qend - q_first + kQNW - 1) / kQNW : 0;
 }
 
 template <typename C>
-__device__ __forceinline__ void issue_advance(const QArgs& a, IssuePtr& ip, int q_first, int q_end) {
+__device__ __forceinline__ void issue_start(const QArgs& a, IssuePtr& ip, int u, int ls, int q1) {
+  ip.u = u;
+  ip.ls = ls;
+  ip.qend = unit_qend<C>(a, u, q1);
+  ip.src = a.rec + (static_cast<int64_t>(u) * a.P.ng + static_cast<int64_t>(ls) * C::NG) * C::REC;
+}
+
+// Next stage of this warp: the next one in the unit, else the first one of
+// the next unit of the block that holds any (a unit with none is skipped).
+template <typename C>
+__device__ __forceinline__ void issue_advance(const QArgs& a, IssuePtr& ip, int q_first, int u_end, int q1) {
   ip.ls += kQNW;
   ip.src += kQNW * C::STAGE;
-  if (ip.ls >= q_end) issue_start<C>(a, ip, ip.u + 1, q_first);
+  if (ip.ls >= ip.qend) {
+    int u = ip.u + 1;
+    while (u < u_end && warp_stage_count(q_first, unit_qend<C>(a, u, q1)) == 0) ++u;
+    if (u < u_end) issue_start<C>(a, ip, u, q_first, q1);
+    else ip.u = u;
+  }
 }
 
 // One bulk copy of this warp's next quantised stage (at ip) into ring slot `slot`.
@@ -750,7 +789,8 @@ struct WarpRing {
   int tail;       // next stage to release
   int hslot;
   uint32_t hphase;
-  int q_first, q_end;  // this warp's first quantised stage in a unit, and the block's end
+  int q_first, q_end;  // this warp's first quantised stage in a unit, and the block's planned end
+  int u_end;           // end of the block's units
   IssuePtr ip;
 };
 
@@ -761,7 +801,7 @@ __device__ __forceinline__ void ring_issue_next(const QArgs& a, unsigned char* r
     fence_proxy_async_smem();
     __syncwarp();
     issue_stage<C>(a, ring, bars, lane, slot, r.ip);
-    issue_advance<C>(a, r.ip, r.q_first, r.q_end);
+    issue_advance<C>(a, r.ip, r.q_first, r.u_end, r.q_end);
     ++r.issued;
   }
 }
@@ -843,7 +883,8 @@ __device__ __forceinline__ void quant_seg(const QArgs& a, unsigned char* ring, u
           body.values(rs, lane);
         } else {
           const int64_t gs = static_cast<int64_t>(r.q_first + kQNW * kk) * C::NG;
-          const int n_here = a.P.ng - gs < C::NG ? static_cast<int>(a.P.ng - gs) : C::NG;
+          const int64_t ng_u = unit_groups(a, u);
+          const int n_here = ng_u - gs < C::NG ? static_cast<int>(ng_u - gs) : C::NG;
 #pragma unroll 1
           for (int gi = 0; gi < n_here; ++gi) {
             body.keys(rs + gi * C::REC, lane);
@@ -909,9 +950,11 @@ __device__ __forceinline__ void residual_seg(const QArgs& a, unsigned char* ring
 #pragma unroll
     for (int mc = 0; mc < KT; ++mc) acc[mc][nt][0] = acc[mc][nt][1] = acc[mc][nt][2] = acc[mc][nt][3] = 0.f;
   }
+  const int R_u = unit_res_rows(a, u);
   for (int t = t_first; t < t_end && ok; t += kQNW) {
     const int t0 = t * kResRows;
-    const int nv = a.R - t0 < kResRows ? a.R - t0 : kResRows;  // rows of this tile inside the window
+    if (t0 >= R_u) break;  // (per-request lengths) past this request's residual
+    const int nv = R_u - t0 < kResRows ? R_u - t0 : kResRows;  // rows of this tile inside the window
     fence_proxy_async_smem();
     __syncwarp();
     if (nv < kResRows) {
@@ -950,7 +993,7 @@ __device__ __forceinline__ void residual_seg(const QArgs& a, unsigned char* ring
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const bool v0 = t0 + gid < a.R, v1 = t0 + gid + 8 < a.R;
+      const bool v0 = t0 + gid < R_u, v1 = t0 + gid + 8 < R_u;
       float x[2] = {v0 ? (sc[nt][0] + sc[nt][1]) * a.scale_log2 : -INFINITY,
                     v1 ? (sc[nt][2] + sc[nt][3]) * a.scale_log2 : -INFINITY};
       float t = fmaxf(x[0], x[1]);
@@ -1203,14 +1246,16 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
   int u0, u1, r0, r1, q0, q1;
   P.block_range(k, u0, u1, r0, r1, q0, q1);
   // this warp's quantised stages: q0 + warp + kQNW i < q1 of every unit of the block
-  const int per_unit = q1 - q0 - warp > 0 ? (q1 - q0 - warp + kQNW - 1) / kQNW : 0;
-  const int my_nq = (u1 - u0) * per_unit;
+  // (< the request's own stage count with per-request lengths)
   // Launched as a programmatic dependent of the previous kernel in the
   // stream: nothing global is read or written before that grid completed.
   // The next kernel may then be scheduled as this grid's blocks retire (it
   // waits the same way).
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  int my_nq = 0;
+  if (q1 > q0)
+    for (int u = u0; u < u1; ++u) my_nq += warp_stage_count(q0 + warp, unit_qend<C>(a, u, q1));
   bool ok = true;
   int rph = 0;
   float* wml = st_ml + warp * C::HEADS * 2;
@@ -1230,13 +1275,17 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
   if (q1 > q0) {
     WarpRing r;
     r.issued = 0, r.head = 0, r.tail = 0, r.hslot = 0, r.hphase = 0u;
-    r.q_first = q0 + warp, r.q_end = q1;
-    issue_start<C>(a, r.ip, u0, q0 + warp);
+    r.q_first = q0 + warp, r.q_end = q1, r.u_end = u1;
+    {
+      int uf = u0;  // first unit where this warp has a stage
+      while (uf < u1 && warp_stage_count(q0 + warp, unit_qend<C>(a, uf, q1)) == 0) ++uf;
+      issue_start<C>(a, r.ip, uf < u1 ? uf : u0, q0 + warp, q1);
+    }
     fence_proxy_async_smem();
     __syncwarp();
     while (r.issued < my_nq && r.issued < C::NST) {
       issue_stage<C>(a, ring, bars, lane, r.issued, r.ip);
-      issue_advance<C>(a, r.ip, r.q_first, r.q_end);
+      issue_advance<C>(a, r.ip, r.q_first, r.u_end, r.q_end);
       ++r.issued;
     }
     uint4* q_sm = reinterpret_cast<uint4*>(smem + C::QSM_OFF);
@@ -1246,7 +1295,8 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
         __syncthreads();
       }
       int state_slot = -1;
-      quant_seg<BITS, G, D, NT>(a, ring, bars, u, per_unit, my_nq, r, ok, wml, state_slot, q_sm);
+      const int n_u = warp_stage_count(q0 + warp, unit_qend<C>(a, u, q1));
+      quant_seg<BITS, G, D, NT>(a, ring, bars, u, n_u, my_nq, r, ok, wml, state_slot, q_sm);
       if (lane == 0) st_off[warp] = state_slot >= 0 ? static_cast<int>(ring + state_slot * C::STAGE - smem) : -1;
       __syncthreads();
       merge_segment<D, C::HEADS>(a, slot0 + 2 * (u - u0) + 1, smem, st_off, st_ml, mw);
@@ -1362,7 +1412,8 @@ QPlan make_plan(const vc_attn_shape& sh, const vc_quant_cache& c, int ng_per_sta
   P.U = sh.B * sh.Hkv;
   P.ng = c.L_q / c.group;
   P.sq = static_cast<int>((P.ng + ng_per_stage - 1) / ng_per_stage);
-  P.sr = (c.R + kResRows - 1) / kResRows;
+  const int Rp = c.lens ? c.R_cap : c.R;  // per-request lengths: plan for the capacity
+  P.sr = (Rp + kResRows - 1) / kResRows;
   P.cq = P.sq > 0 ? static_cast<int64_t>(ng_per_stage) * rec_bytes : 1;
   P.cr = P.sr > 0 ? static_cast<int64_t>(kResRows) * 4 * sh.D * kResCostNum / kResCostDen : 1;
   if (target_blocks < 1) target_blocks = 1;
@@ -1459,15 +1510,20 @@ vc_status check_quant(const vc_attn_shape* sh, const vc_quant_cache* c, const ch
   VC_REQUIRE(c->group == 32 || c->group == 64, "%s: group must be 32 or 64 (got %d)", who, c->group);
   VC_REQUIRE(c->L_q >= 0 && c->L_q % c->group == 0, "%s: L_q must be a non-negative multiple of group", who);
   VC_REQUIRE(c->L_q / c->group < (int64_t(1) << 30), "%s: L_q too large", who);
-  VC_REQUIRE(c->R >= 0 && c->R <= c->R_cap, "%s: need 0 <= R <= R_cap", who);
-  VC_REQUIRE(c->L_q + c->R >= 1, "%s: the cache holds no token", who);
+  if (c->lens == nullptr) {
+    VC_REQUIRE(c->R >= 0 && c->R <= c->R_cap, "%s: need 0 <= R <= R_cap", who);
+    VC_REQUIRE(c->L_q + c->R >= 1, "%s: the cache holds no token", who);
+  } else {
+    VC_REQUIRE(c->R_cap >= 0 && c->L_q + c->R_cap >= 1, "%s: the cache has no capacity", who);
+    VC_REQUIRE(reinterpret_cast<uintptr_t>(c->lens) % 8 == 0, "%s: lens must be 8-byte aligned", who);
+  }
   VC_REQUIRE(static_cast<int64_t>(sh->B) * sh->Hkv <= (int64_t(1) << 24), "%s: too many (request, head) pairs",
              who);
   if (c->L_q > 0) {
     VC_REQUIRE(c->records, "%s: null group-record pointer", who);
     VC_REQUIRE(aligned16(c->records), "%s: group records must be 16-byte aligned", who);
   }
-  if (c->R > 0) {
+  if ((c->lens ? c->R_cap : c->R) > 0) {
     VC_REQUIRE(c->k_res && c->v_res, "%s: null residual pointer", who);
     VC_REQUIRE(aligned16(c->k_res) && aligned16(c->v_res), "%s: residual arrays must be 16-byte aligned", who);
   }
@@ -1482,6 +1538,8 @@ QArgs make_args(const vc_attn_shape& sh, const vc_quant_cache& c, const void* q)
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.R = c.R;
   a.R_cap = c.R_cap;
+  a.group = c.group;
+  a.lens = c.lens;
   a.Hq = sh.Hq;
   a.Hkv = sh.Hkv;
   a.g = sh.Hq / sh.Hkv;

@@ -28,6 +28,7 @@ VC_F32, VC_BF16, VC_F16 = 0, 1, 2
 VC_FLAG_BAD_INDEX = 1
 VC_FLAG_WAIT_TIMEOUT = 2
 VC_FLAG_RANGE = 4
+VC_FLAG_BAD_LENGTH = 8
 
 
 class VcError(RuntimeError):
@@ -42,7 +43,8 @@ class vc_attn_shape(Structure):
 
 class vc_quant_cache(Structure):
     _fields_ = [("records", c_void_p), ("k_res", c_void_p), ("v_res", c_void_p),
-                ("bits", c_int), ("group", c_int), ("L_q", c_int64), ("R", c_int), ("R_cap", c_int)]
+                ("bits", c_int), ("group", c_int), ("L_q", c_int64), ("R", c_int), ("R_cap", c_int),
+                ("lens", c_void_p)]
 
 
 class vc_sparse_cache(Structure):
@@ -102,6 +104,8 @@ def lib() -> ctypes.CDLL:
             "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
             "vc_debug_wait_timeout": (c_int, [c_void_p, c_void_p, ctypes.c_int64, c_void_p]),
             "vc_compress_workspace_size": (c_size_t, []),
+            "vc_cache_commit": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_int, c_void_p,
+                                        c_void_p, c_size_t, c_void_p]),
             "vc_quantize_cache": (c_int, [P(vc_attn_shape), c_void_p, c_void_p, ctypes.c_int64, c_int, c_int,
                                           ctypes.c_int64, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_size_t,
                                           c_void_p]),
@@ -162,11 +166,13 @@ def shape(B: int, Hq: int, Hkv: int, D: int, sm_scale: float = 0.0) -> vc_attn_s
 
 def quant_cache(t: dict) -> vc_quant_cache:
     """Descriptor of a quantised cache given as a dict of CUDA tensors with the
-    keys records, k_res, v_res and ints bits, group, L_q, R, R_cap (the layout
+    keys records, k_res, v_res and ints bits, group, L_q, R, R_cap, and an
+    optional int32 tensor lens [B, 2] of per-request (L_q, R) (the layout
     documented in vc.h).  The descriptor holds raw device pointers; it keeps
     references to the tensors so they stay allocated while it lives."""
     d = vc_quant_cache(_p(t["records"]), _p(t.get("k_res")), _p(t.get("v_res")),
-                       int(t["bits"]), int(t["group"]), int(t["L_q"]), int(t["R"]), int(t["R_cap"]))
+                       int(t["bits"]), int(t["group"]), int(t["L_q"]), int(t["R"]), int(t["R_cap"]),
+                       _p(t.get("lens")))
     d._keep = dict(t)
     return d
 
@@ -264,6 +270,13 @@ def vc_quantize_cache(sh, k, v, T: int, bits: int, group: int, L_q: int, records
     _check(lib().vc_quantize_cache(ctypes.byref(sh), _p(k), _p(v), int(T), int(bits), int(group), int(L_q),
                                    _p(records), _p(k_res), _p(v_res), int(R_cap), _p(ws), ws.numel(),
                                    _stream(stream)))
+
+
+def vc_cache_commit(sh, qc, k_new, v_new, nq: int, accept_len, ws, stream=None):
+    """Commit one round's accepted rows into a device-maintained quantised
+    cache (qc.lens required; see include/vc.h)."""
+    _check(lib().vc_cache_commit(ctypes.byref(sh), ctypes.byref(qc), _p(k_new), _p(v_new), int(nq), _p(accept_len),
+                                 _p(ws), ws.numel(), _stream(stream)))
 
 
 def vc_compact_kept(sh, k, v, T_store: int, idx, n_keep: int, k_out, v_out, ws=None, stream=None):

@@ -210,3 +210,27 @@ def test_compression_calls_reject_before_any_launch(L):
     assert L.vc_compact_kept(ctypes.byref(sh), 16, 16, 100, 16, 0, 16, 16, None, 0, None) == vc.VC_ERR_INVALID_ARG
     assert L.vc_compact_kept(ctypes.byref(sh), 16, 16, 100, None, 8, 16, 16, None, 0, None) == vc.VC_ERR_INVALID_ARG
     assert L.vc_compact_kept(ctypes.byref(sh), 16, 16, 100, 16, 8, 18, 16, None, 0, None) == vc.VC_ERR_INVALID_ARG
+
+
+def test_cache_commit_rejects_before_any_launch(L):
+    import ctypes
+    sh = vc.shape(2, 8, 2, 128)
+
+    def qc(**kw):
+        c = vc.vc_quant_cache()
+        c.records, c.k_res, c.v_res, c.lens = 16, 16, 16, 16
+        c.bits, c.group, c.L_q, c.R, c.R_cap = 2, 32, 320, 0, 128
+        for k, v in kw.items():
+            setattr(c, k, v)
+        return c
+
+    def commit(c, nq=31, k_new=16, accept=16, ws=16):
+        return L.vc_cache_commit(ctypes.byref(sh), ctypes.byref(c), k_new, 16, nq, accept, ws, 256, None)
+    assert commit(qc(lens=None)) == vc.VC_ERR_INVALID_ARG      # needs per-request lengths
+    assert commit(qc(), nq=33) == vc.VC_ERR_INVALID_ARG        # nq > group
+    assert commit(qc(R_cap=40)) == vc.VC_ERR_INVALID_ARG       # R_cap < group + nq - 1
+    assert commit(qc(L_q=100)) == vc.VC_ERR_INVALID_ARG        # capacity not a multiple of group
+    assert commit(qc(bits=3)) == vc.VC_ERR_INVALID_ARG
+    assert commit(qc(), k_new=None) == vc.VC_ERR_INVALID_ARG
+    assert commit(qc(), accept=None) == vc.VC_ERR_INVALID_ARG
+    assert commit(qc(), k_new=24) == vc.VC_ERR_INVALID_ARG     # misaligned block rows
