@@ -6,10 +6,13 @@
 // correction (the bonus token when all K agree) -- devshah.ca page "VeriCache:
 // making lossy KV compression exact", section "The Core Idea".
 //
-// Layout of the work: grid (S, B*(K+1)).  Block (c, row) scans chunk c of one
-// logit row with 16-byte streaming loads and reduces (value, index) pairs
-// under the rule "larger value wins, NaN beats every number, ties go to the
-// lower index".  The last block of a row (atomic ticket, no waiting) merges
+// Layout of the work: grid (S, B*(K+1)), S chosen so the grid is about one
+// wave of 512-thread blocks.  Block (c, row) scans chunk c of one logit row
+// with 16-byte streaming loads, eight in flight per thread, and reduces
+// (value, index) pairs under the rule "larger value wins, NaN beats every
+// number, ties go to the lower index".  Inside a thread the indices only
+// grow, so a later value replaces the kept one only if it is strictly larger
+// or a NaN over a number; the index rule decides between threads and blocks.  The last block of a row (atomic ticket, no waiting) merges
 // the S partials into target[row]; the last row of a request computes the
 // accepted length and the correction.  Tickets reset themselves, so the
 // workspace stays ready for the next call.
@@ -20,9 +23,9 @@
 namespace vc {
 namespace {
 
-constexpr int kAcceptThreads = 256;
-constexpr int kAcceptChunk = 16384;  // vocabulary entries per block
+constexpr int kAcceptThreads = 512;
 constexpr int kAcceptMaxSplit = 16;
+constexpr int kAcceptInFlight = 8;  // 16-byte loads in flight per thread
 
 struct Best {
   float v;
@@ -62,20 +65,27 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return r;
 }
 
+// x at a larger index than every value taken so far by this thread
+__device__ __forceinline__ void take_later(Best& b, float x, int i) {
+  if (x > b.v || (x != x && b.v == b.v) || b.i == INT_MAX) {
+    b.v = x;
+    b.i = i;
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ void take_vec(Best& b, uint4 w, int base) {
   if constexpr (sizeof(T) == 4) {
-    take(b, __uint_as_float(w.x), base + 0);
-    take(b, __uint_as_float(w.y), base + 1);
-    take(b, __uint_as_float(w.z), base + 2);
-    take(b, __uint_as_float(w.w), base + 3);
+    take_later(b, __uint_as_float(w.x), base + 0);
+    take_later(b, __uint_as_float(w.y), base + 1);
+    take_later(b, __uint_as_float(w.z), base + 2);
+    take_later(b, __uint_as_float(w.w), base + 3);
   } else {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float2 f = unpack_bf2(ws[j]);
-      take(b, f.x, base + 2 * j);
-      take(b, f.y, base + 2 * j + 1);
+      take_later(b, __uint_as_float(ws[j] << 16), base + 2 * j);             // bf16 -> fp32 is a shift
+      take_later(b, __uint_as_float(ws[j] & 0xffff0000u), base + 2 * j + 1);
     }
   }
 }
@@ -105,32 +115,30 @@ __global__ void __launch_bounds__(kAcceptThreads) accept_kernel(const T* __restr
   const int v1 = min(V, v0 + chunk);
 
   Best b{-INFINITY, INT_MAX};
-  // scalar head up to 16-byte alignment, vector body, scalar tail
+  // scalar head up to 16-byte alignment, vector body, scalar tail; each
+  // thread sees its indices in increasing order (head, then vectors j,
+  // j + threads, ..., then the tail), so take_later applies
   const uintptr_t addr0 = reinterpret_cast<uintptr_t>(p + v0);
   int head = static_cast<int>(((16 - (addr0 & 15)) & 15) / sizeof(T));
   if (v0 + head > v1) head = v1 - v0;
   const int a = v0 + head;
   const int nvec = (v1 - a) / VEC;
-  if (threadIdx.x < head) take(b, to_f32(p[v0 + threadIdx.x]), v0 + threadIdx.x);
-  // four independent 16-byte loads in flight per thread before they are used
-  // (the comparison rule does not depend on the order values are taken in)
-  int j = threadIdx.x;
-  for (; j + 3 * kAcceptThreads < nvec; j += 4 * kAcceptThreads) {
-    const int b0 = a + j * VEC;
-    const auto x0 = ld_stream(p + b0);
-    const auto x1 = ld_stream(p + b0 + kAcceptThreads * VEC);
-    const auto x2 = ld_stream(p + b0 + 2 * kAcceptThreads * VEC);
-    const auto x3 = ld_stream(p + b0 + 3 * kAcceptThreads * VEC);
-    take_vec<T>(b, x0, b0);
-    take_vec<T>(b, x1, b0 + kAcceptThreads * VEC);
-    take_vec<T>(b, x2, b0 + 2 * kAcceptThreads * VEC);
-    take_vec<T>(b, x3, b0 + 3 * kAcceptThreads * VEC);
+  if (threadIdx.x < head) take_later(b, to_f32(p[v0 + threadIdx.x]), v0 + threadIdx.x);
+  // kAcceptInFlight independent 16-byte loads per thread before any is used
+  for (int j0 = threadIdx.x; j0 < nvec; j0 += kAcceptInFlight * kAcceptThreads) {
+    uint4 x[kAcceptInFlight];
+#pragma unroll
+    for (int f = 0; f < kAcceptInFlight; ++f) {
+      const int j = j0 + f * kAcceptThreads;
+      x[f] = j < nvec ? ld_stream(p + a + j * VEC) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int f = 0; f < kAcceptInFlight; ++f) {
+      const int j = j0 + f * kAcceptThreads;
+      if (j < nvec) take_vec<T>(b, x[f], a + j * VEC);
+    }
   }
-  for (; j < nvec; j += kAcceptThreads) {
-    const int base = a + j * VEC;
-    take_vec<T>(b, ld_stream(p + base), base);
-  }
-  for (int t = a + nvec * VEC + threadIdx.x; t < v1; t += kAcceptThreads) take(b, to_f32(p[t]), t);
+  for (int t = a + nvec * VEC + threadIdx.x; t < v1; t += kAcceptThreads) take_later(b, to_f32(p[t]), t);
 
   __shared__ Best red[kAcceptThreads / 32];
   b = warp_best(b);
@@ -179,9 +187,14 @@ struct AcceptPlan {
 
 AcceptPlan plan_accept(int B, int K, int V) {
   AcceptPlan pl{};
-  pl.S = (V + kAcceptChunk - 1) / kAcceptChunk;
-  if (pl.S > kAcceptMaxSplit) pl.S = kAcceptMaxSplit;
-  if (pl.S < 1) pl.S = 1;
+  // about one wave of blocks (4 blocks of 512 threads per SM), no chunk shorter than 8 loads per thread
+  const int64_t nrows = static_cast<int64_t>(B) * (K + 1);
+  const int64_t wave = 4 * static_cast<int64_t>(sm_count());
+  int64_t S = (wave + nrows - 1) / nrows;
+  const int64_t smax = (V + 8 * kAcceptThreads - 1) / (8 * kAcceptThreads);
+  if (S > smax) S = smax;
+  if (S > kAcceptMaxSplit) S = kAcceptMaxSplit;
+  pl.S = S < 1 ? 1 : static_cast<int>(S);
   pl.chunk = (V + pl.S - 1) / pl.S;
   pl.chunk = (pl.chunk + 7) / 8 * 8;
   pl.S = (V + pl.chunk - 1) / pl.chunk;
