@@ -14,24 +14,26 @@
 //   sum_t p_t v_hat[t]c = sum_t (p_t s_t) code[t][c] + sum_t p_t z_t
 // so the codes enter the tensor cores as exact small integers (fp16), and the
 // scales are folded into the other operand once per group.  The folded
-// operands q*s and p*s are split into an fp16 high part and an fp16 low
-// part (two MMA columns each), which keeps ~22 significant bits; the zero
-// terms are separate small MMAs with exact fp16 products.  Accumulation is
-// fp32.  The result equals attention over fp32-dequantised values up to fp32
-// rounding (the oracle dequantises with one fp32 FMA per element).
+// operands q*s and p~*s are split into an fp16 high part and an fp16 low
+// part (two MMA columns each), which keeps ~22 significant bits; p~ is the
+// softmax weight rounded once to fp16 (the denominator sums the fp32
+// weights); the zero terms are separate small MMAs with exact fp16
+// products.  Accumulation is fp32.
 //
-// Work layout.  The job is one axis of STAGES: first every (request, KV
-// head) unit's bf16 residual, 16 rows per stage, then every unit's quantised
-// groups, NG consecutive group records per stage.  A persistent grid of
-// (SMs x resident blocks) blocks cuts that axis into equal-cost contiguous
-// ranges (Partition); inside a block the 4 warps take the range's stages
-// round-robin.  A quantised stage is ONE bulk copy of contiguous records into
-// the warp's private ring (NST stages deep, completed on mbarriers, waits
-// bounded).  Wherever the range crosses from one unit's segment to the next,
-// the block merges its warps' online-softmax states into one partial of that
-// segment; a second launch (combine_kernel, one block per (unit, head))
-// merges each unit's partials into the output.  All g query heads of a GQA
-// group share each record (they are the MMA's N columns).
+// Work layout.  Every (request, KV head) unit is an axis of residual tiles
+// (16 bf16 rows) followed by quantised stages (NG consecutive group records,
+// ONE bulk copy).  A persistent grid of (SMs x resident blocks) blocks takes
+// the units in equal-cost pieces (UPart): with fewer units than blocks each
+// unit is cut into bpu contiguous pieces, otherwise each block owns whole
+// units.  Inside a block the 4 warps take the piece's stages round-robin,
+// each through its own shared-memory ring (NST stages deep, completed on
+// mbarriers, waits bounded); at the end of each segment (the residual tiles,
+// then the quantised stages) the block merges its warps' online-softmax
+// states into one partial of the unit.  The block that finishes a unit's
+// last partial (a per-unit ticket) merges the unit's partials into the
+// output, so a call is one launch (a programmatic dependent launch: its
+// prologue overlaps the previous kernel's tail).  All g query heads of a GQA
+// group share each record (they are MMA columns or rows).
 //
 // MMA arrangement (mma.sync m16n8k16, fp16 x fp16 -> fp32):
 //   scores:  D[token][col] = codes[token][chan] x qfold[chan][col]
