@@ -160,6 +160,52 @@ def read_peaks():
         return 6650.0, "fallback"
 
 
+def read_tensor_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s): the measured cuBLAS burst figure
+    when the box carries one, else the fallback measured earlier on this kind
+    of box."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def time_resident_verify_layer(w, dev, reps: int = 20):
+    """One layer's block verification with the full K and V resident in HBM
+    (the workload's request shape), timed alone with CUDA events over `reps`
+    calls alternating two layers (each larger than L2): the HBM and the
+    tensor-pipe fractions of the kernel, which the host link hides when the
+    cache is streamed."""
+    import torch
+    from lossless_draft_verify_vc_b200 import synth, vc
+    B, Hq, Hkv, D, T, nq = w["B"], w["Hq"], w["Hkv"], w["D"], w["T"], w["K"] + 1
+    sh = vc.shape(B, Hq, Hkv, D)
+    kv = [synth.kv_full(B, Hkv, T, D, seed=70 + l, device=dev) for l in range(2)]
+    q = synth.normal((B, nq, Hq, D), 72, dev)
+    out = torch.empty(B, nq, Hq, D, device=dev)
+    ws = vc.workspace(vc.vc_verify_attn_workspace_size(sh, T, nq), dev)
+    comp = torch.cuda.current_stream(dev)
+    for l in range(4):
+        vc.vc_verify_attn(sh, q, kv[l % 2][0], kv[l % 2][1], T, nq, out, None, ws, comp)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for l in range(reps):
+        vc.vc_verify_attn(sh, q, kv[l % 2][0], kv[l % 2][1], T, nq, out, None, ws, comp)
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    byt = 4 * T * Hkv * D * B
+    flops = 4 * nq * Hq * T * D * B
+    del kv
+    torch.cuda.empty_cache()
+    return dict(us_per_layer=us, hbm_gbps=byt / (us * 1e-6) / 1e9, tflops=flops / (us * 1e-6) / 1e12,
+                bytes_per_layer=byt, flops_per_layer=flops, reps=reps)
+
+
 def kernel_source_hash(files) -> str:
     h = hashlib.sha256()
     for f in files:
@@ -742,6 +788,21 @@ def _common(args, config, value, peak, peak_kind, r, dtype):
             "config": config, "clocks": r["clocks"]}
 
 
+def resident_verify_block(w, peak, peak_kind):
+    """JSON block for one resident verification layer of a streamed workload."""
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    rv = time_resident_verify_layer(w, dev)
+    tp, tk = read_tensor_peak()
+    rv.update({"hbm_frac": rv["hbm_gbps"] / peak, "hbm_peak_kind": f"{peak_kind} hbm_gbs (burst copy)",
+               "tensor_frac": rv["tflops"] / tp, "tensor_peak_tflops": tp,
+               "tensor_peak_kind": f"{tk} bf16 dense (burst)",
+               "note": "one layer of the workload's request with the full K and V in HBM, timed alone; flops = "
+                       "4 nq Hq T D (the two products, algorithmic; the kernel runs P.V twice, as bf16 high and "
+                       "low parts)"})
+    return rv
+
+
 def streamed_line(args, w, rank, world, config, peak, peak_kind):
     r = run_streamed(args, w, rank, world)
     K, NL = w["K"], w["NL"]
@@ -768,6 +829,7 @@ def streamed_line(args, w, rank, world, config, peak, peak_kind):
         # per step: K*NL token-drop draft calls and NL verify calls (each an
         # attention kernel + its chunk-merge kernel), one accept kernel
         "gpu_launches": (2 * K * NL + 2 * NL + 1) * args.steps,
+        "verify_resident_layer": resident_verify_block(w, peak, peak_kind),
     })
     return line
 
@@ -798,6 +860,7 @@ def stagger_line(args, w, rank, world, config, peak, peak_kind):
                      "frac": db / (r["draft_ms"] * 1e3 / (K * NL) * 1e-6) / 1e9 / peak, "traffic": None,
                      "algorithmic_bytes_per_launch": db},
         "gpu_launches": 2 * K * NL,
+        "verify_resident_layer": resident_verify_block(w, peak, peak_kind),
     })
     return line
 

@@ -9,9 +9,13 @@
 //
 // Design.  For one (request, KV head) the nq query rows of all g heads of the
 // GQA group form the MMA's M dimension (row r = position i * g + head), so each
-// K/V tile is read from HBM once for the whole group.  Blocks split the
-// context (split-K) and merge through the workspace.  Per block:
-//   * Q (<= 128 rows) is staged once into shared memory in the 128-byte
+// K/V tile is read from HBM once for the whole group.  When nq * g exceeds
+// 128 rows (g = 5 or 8 with 31 rows), the rows form two row tiles of <= 128
+// rows, and ONE block computes both against each K/V tile it loads: two
+// softmax warpgroups, two S double buffers and two O accumulators fill the
+// 512 TMEM columns.  Blocks split the context (split-K) and merge through
+// the workspace.  Per block:
+//   * Q (<= 128 rows per row tile) is staged once into shared memory in the 128-byte
 //     swizzled K-major layout by tiled TMA (a 3-D map over positions x heads
 //     x channels: the g heads of nqt positions are the tile's rows), the
 //     first request of the block so that it does not queue behind K and V;
@@ -24,7 +28,7 @@
 //     the tensor pipe's queue while the softmax warps work, so no row waits
 //     for it.  S is double buffered: S of tile i + 1 is computed while the
 //     softmax of tile i runs;
-//   * each of the 128 softmax threads owns one row: it reads its scores from TMEM,
+//   * each softmax thread owns one row of its warpgroup's row tile: it reads its scores from TMEM,
 //     applies the causal mask (row i sees keys 0 .. T - nq + i), updates an
 //     online softmax with lazy rescaling (O is rescaled only when the running
 //     maximum grows by more than 8 in log2 units), and writes P back to TMEM
@@ -39,6 +43,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "vc_splitk.cuh"
 #include "vc_tc.cuh"
 
@@ -46,28 +52,43 @@ namespace vc {
 namespace {
 
 constexpr int kVBN = 64;        // keys per tile
-constexpr int kVThreads = 128;  // softmax warpgroup: thread r owns row r
-constexpr int kVBlock = kVThreads + 64;  // + the MMA warp + the loader warp
-constexpr int kVIssuer = kVThreads;      // the MMA warp's elected thread
-constexpr int kVLoader = kVThreads + 32; // the loader warp's elected thread
-constexpr int kVTmemCols = 256;
-// TMEM column map: two S buffers of kVBN fp32 columns (tile i in buffer
-// i & 1), each overwritten by its P -- high part in the first kVBN / 2
-// columns, low part in the next (bf16 pairs) -- then O, D fp32 columns.
+constexpr int kVThreads = 128;  // one softmax warpgroup: thread r owns row r of its row tile
+// Block of RTC row tiles: RTC softmax warpgroups, then the MMA warp and the
+// loader warp.
+template <int RTC>
+struct VBlk {
+  static constexpr int SOFTMAX = RTC * kVThreads;
+  static constexpr int THREADS = SOFTMAX + 64;
+  static constexpr int ISSUER = SOFTMAX;       // the MMA warp's elected thread
+  static constexpr int LOADER = SOFTMAX + 32;  // the loader warp's elected thread
+  static constexpr uint32_t TMEM_COLS = RTC * 256;
+};
+// TMEM column map of row tile rt (base rt * 256): two S buffers of kVBN fp32
+// columns (tile i in buffer i & 1), each overwritten by its P -- high part in
+// the first kVBN / 2 columns, low part in the next (bf16 pairs) -- then O,
+// D fp32 columns.
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColPlo = kVBN / 2;  // offset of P's low part inside a buffer
 constexpr uint32_t kColO = 2 * kVBN;
+constexpr uint32_t kColTile = 256;      // columns of one row tile
 
-template <int D>
+template <int D, int RTC>
 struct VCfg {
   static constexpr int HALVES = D / 64;              // 128-byte swizzle atoms across D
-  static constexpr int Q_B = 128 * D * 2;            // 128 rows
+  static constexpr int QT_B = 128 * D * 2;           // one row tile: 128 rows
+  static constexpr int Q_B = RTC * QT_B;
   static constexpr int KV_B = kVBN * D * 2;          // one of K or V per stage
   static constexpr int STAGE_B = 2 * KV_B;
+  // K/V stages in flight per block (measured on B200: 4 stages for the
+  // two-row-tile block were no faster than 2)
+  static constexpr int NS = 2;
   static constexpr int Q_OFF = 0;
-  static constexpr int ST_OFF = Q_B;                 // 2 stages
-  static constexpr int BAR_OFF = ST_OFF + 2 * STAGE_B;
-  static constexpr int SMEM_B = BAR_OFF + 128 + 1024;  // 9 barriers + TMEM slot (76 B); + alignment slack
+  static constexpr int ST_OFF = Q_B;
+  static constexpr int BAR_OFF = ST_OFF + NS * STAGE_B;
+  // barriers: K full / K free / V full / V free per stage, S and P.V per S
+  // buffer, Q, drain; then the TMEM address slot
+  static constexpr int NBAR = 4 * NS + 6;
+  static constexpr int SMEM_B = BAR_OFF + NBAR * 8 + 16 + 1024;  // + alignment slack
 };
 
 struct VArgs {
@@ -81,21 +102,24 @@ struct VArgs {
 
 // Block-wide barrier of the softmax warps and the MMA warp only (the loader
 // warp runs its own loop); returns whether any participant passed true.
+template <int RTC>
 __device__ __forceinline__ bool mma_group_sync_or(bool v) {
   uint32_t r;
   asm volatile(
       "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
       : "=r"(r)
-      : "r"(v ? 1u : 0u), "n"(kVThreads + 32)
+      : "r"(v ? 1u : 0u), "n"(VBlk<RTC>::SOFTMAX + 32)
       : "memory");
   return r != 0;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                           const __grid_constant__ CUtensorMap tm_k,
-                                                           const __grid_constant__ CUtensorMap tm_v, VArgs a) {
-  using C = VCfg<D>;
+template <int D, int RTC>
+__global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                     const __grid_constant__ CUtensorMap tm_k,
+                                                                     const __grid_constant__ CUtensorMap tm_v,
+                                                                     VArgs a) {
+  using C = VCfg<D, RTC>;
+  using K = VBlk<RTC>;
   // the chunk-merge launch that follows may be scheduled as this grid's blocks
   // retire; it waits for this grid's completion before reading the partials
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
@@ -103,31 +127,38 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_s = smem + C::Q_OFF;
   unsigned char* st_s = smem + C::ST_OFF;
-  uint64_t* bar_k = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);  // [2] K slot landed
-  uint64_t* bar_v = bar_k + 2;                                        // [2] V slot landed
-  uint64_t* bar_s = bar_k + 4;                                        // [2] S buffer computed
-  uint64_t* bar_pv = bar_k + 6;                                       // [2] P.V of that buffer done
-  uint64_t* bar_q = bar_k + 8;                                        // Q staged
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_k + 9);
+  constexpr int NS = C::NS;
+  uint64_t* bar_k = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);  // [NS] K stage landed
+  uint64_t* bar_kf = bar_k + NS;                                      // [NS] K stage read by its S MMAs
+  uint64_t* bar_v = bar_kf + NS;                                      // [NS] V stage landed
+  uint64_t* bar_vf = bar_v + NS;                                      // [NS] V stage read by its P.V MMAs
+  uint64_t* bar_s = bar_vf + NS;                                      // [2] S buffer computed
+  uint64_t* bar_pv = bar_s + 2;                                       // [2] P.V of that buffer done
+  uint64_t* bar_q = bar_pv + 2;                                       // Q staged
+  uint64_t* bar_dr = bar_q + 1;                                       // drain after a give-up
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_dr + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int chunk = blockIdx.x;
   const int unit = blockIdx.y;  // b * Hkv + h
-  const int rt = blockIdx.z;    // row tile
+  // row tile of this thread: blockIdx.z when a block takes one row tile, its
+  // warpgroup when the block takes all of them (RTC == 2)
+  const int wg = RTC == 1 ? 0 : (tid < K::SOFTMAX ? tid / kVThreads : 0);
+  const int rt = RTC == 1 ? static_cast<int>(blockIdx.z) : wg;
   const int b = unit / a.Hkv, h = unit - b * a.Hkv;
   const int i0 = rt * a.nqt;
-  const int nq_t = min(a.nqt, a.nq - i0);
-  const int M = nq_t * a.g;  // valid rows
+  const int nq_t = max(0, min(a.nqt, a.nq - i0));
+  const int M = nq_t * a.g;  // valid rows of this thread's row tile
   const int64_t k_begin = static_cast<int64_t>(chunk) * a.tiles_per_chunk * kVBN;
   const int64_t k_end = min(a.T, k_begin + static_cast<int64_t>(a.tiles_per_chunk) * kVBN);
   const int ntiles = static_cast<int>((k_end - k_begin + kVBN - 1) / kVBN);
-  const bool softmax_thread = tid < kVThreads;
+  const bool softmax_thread = tid < K::SOFTMAX;
   bool fail = false;
 
-  // K (v = 0) or V (v = 1) of tile i into slot i & 1; loader only
+  // K (v = 0) or V (v = 1) of tile i into stage i % NS; loader only
   auto issue_load = [&](int i, int v) {
-    unsigned char* dst = st_s + (i & 1) * C::STAGE_B + v * C::KV_B;
-    uint64_t* bar = v ? &bar_v[i & 1] : &bar_k[i & 1];
+    unsigned char* dst = st_s + (i % NS) * C::STAGE_B + v * C::KV_B;
+    uint64_t* bar = v ? &bar_v[i % NS] : &bar_k[i % NS];
     const int y = static_cast<int>(k_begin + static_cast<int64_t>(i) * kVBN);
     mbar_arrive_expect_tx(bar, C::KV_B);
 #pragma unroll
@@ -135,30 +166,36 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
       tc::tma_load_3d(dst + hf * kVBN * 128, v ? &tm_v : &tm_k, hf * 64, y, unit, bar);
   };
 
-  // The loader owns the barriers' initialisation and requests Q, then the
-  // first two tiles; nobody else touches a barrier before the block-wide
-  // barrier below.
-  if (tid == kVLoader) {
-    for (int j = 0; j < 9; ++j) mbar_init(&bar_k[j], 1);
+  // The loader owns the barriers' initialisation and requests Q (every row
+  // tile of the block), then the first NS tiles; nobody else touches a
+  // barrier before the block-wide barrier below.
+  if (tid == K::LOADER) {
+    for (int j = 0; j < C::NBAR; ++j) mbar_init(&bar_k[j], 1);
     fence_mbar_init();
     fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar_q, C::HALVES * 128 * a.g * a.nqt);
+    mbar_arrive_expect_tx(bar_q, RTC * C::HALVES * 128 * a.g * a.nqt);
 #pragma unroll
-    for (int hf = 0; hf < C::HALVES; ++hf)
-      tc::tma_load_3d(q_s + hf * (128 * 128), &tm_q, hf * 64, h * a.g, b * a.nq + i0, bar_q);
-    for (int j = 0; j < 2 && j < ntiles; ++j) {
+    for (int t = 0; t < RTC; ++t) {
+      const int rtq = RTC == 1 ? rt : t;
+#pragma unroll
+      for (int hf = 0; hf < C::HALVES; ++hf)
+        tc::tma_load_3d(q_s + t * C::QT_B + hf * (128 * 128), &tm_q, hf * 64, h * a.g, b * a.nq + rtq * a.nqt, bar_q);
+    }
+    for (int j = 0; j < NS && j < ntiles; ++j) {
       issue_load(j, 0);
       issue_load(j, 1);
     }
   }
-  if (warp == 0) tc::alloc(tmem_slot, kVTmemCols);
+  if (warp == 0) tc::alloc(tmem_slot, K::TMEM_COLS);
 
   // ---- Q rows past the TMA tile's g * nqt rows are zeros (rows of the tile
   //      whose position is past nq hold finite data and are never stored)
-  if (softmax_thread && tid >= a.g * a.nqt) {
+  const int r = tid - wg * kVThreads;  // row of this softmax thread in its row tile
+  unsigned char* q_t = q_s + wg * C::QT_B;
+  if (softmax_thread && r >= a.g * a.nqt) {
 #pragma unroll
     for (int c = 0; c < D / 8; ++c)
-      *reinterpret_cast<uint4*>(q_s + (c >> 3) * (128 * 128) + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) =
+      *reinterpret_cast<uint4*>(q_t + (c >> 3) * (128 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4)) =
           make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
@@ -170,31 +207,36 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, kVBN, false);
   constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(128, D, true);
   const uint32_t q_base = smem_addr(q_s);
-  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;  // this warp's TMEM lanes
+  // this warp's TMEM lanes and its row tile's columns
+  const uint32_t lane_off = (static_cast<uint32_t>((warp & 3) * 32) << 16) + static_cast<uint32_t>(wg) * kColTile;
 
   // row state
-  const int r = tid;
   const int i_row = i0 + (r < M ? r / a.g : 0);
   const int64_t vis_end = a.T - a.nq + i_row + 1;  // keys [0, vis_end) visible to this row
   float m_run = -INFINITY, l_run = 0.f;
 
-  // S = Q K^T of tile i into buffer i & 1: MMA thread, once tile i's K has landed
+  // S = Q K^T of tile i into buffer i & 1 of every row tile: MMA thread, once
+  // tile i's K has landed; when those MMAs complete, the S buffer is ready
+  // for the softmax and the K stage free for the loader
   auto issue_s = [&](int i) -> bool {
-    const uint32_t ks_addr = smem_addr(st_s + (i & 1) * C::STAGE_B);
-    if (!mbar_wait_bounded(&bar_k[i & 1], (i >> 1) & 1, a.flags)) return false;
+    const uint32_t ks_addr = smem_addr(st_s + (i % NS) * C::STAGE_B);
+    if (!mbar_wait_bounded(&bar_k[i % NS], (i / NS) & 1, a.flags)) return false;
     tc::fence_after_sync();
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int hf = kk >> 2, ko = (kk & 3) * 32;
-      const uint64_t ad = tc::smem_desc_sw128(q_base + hf * (128 * 128) + ko, 16, 1024);
-      const uint64_t bd = tc::smem_desc_sw128(ks_addr + hf * (kVBN * 128) + ko, 16, 1024);
-      tc::mma_ss(tmem + kColS + (i & 1) * kVBN, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-    }
+    for (int t = 0; t < RTC; ++t)
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int hf = kk >> 2, ko = (kk & 3) * 32;
+        const uint64_t ad = tc::smem_desc_sw128(q_base + t * C::QT_B + hf * (128 * 128) + ko, 16, 1024);
+        const uint64_t bd = tc::smem_desc_sw128(ks_addr + hf * (kVBN * 128) + ko, 16, 1024);
+        tc::mma_ss(tmem + t * kColTile + kColS + (i & 1) * kVBN, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+      }
     tc::commit(&bar_s[i & 1]);
+    tc::commit(&bar_kf[i % NS]);
     return true;
   };
 
-  if (tid == kVIssuer) {
+  if (tid == K::ISSUER) {
     if (!mbar_wait_bounded(bar_q, 0, a.flags)) fail = true;
     if (!fail && ntiles > 0 && !issue_s(0)) fail = true;
     if (!fail && ntiles > 1 && !issue_s(1)) fail = true;
@@ -206,18 +248,19 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   // exits on their common barrier's OR, so they leave together; the loader
   // stops at its first failed wait.  All meet again after the loop.
   constexpr unsigned FULL = 0xffffffffu;
-  int nk = ntiles < 2 ? ntiles : 2, nv = nk;  // K / V tiles issued so far (loader)
-  if (warp == kVLoader / 32) {
-    // ---- loader: K of tile j once S of tile j - 2 is done, V of tile j once
-    //      P.V of tile j - 2 is done, in the order those happen (S of tile
-    //      j - 1 finishes before P.V of tile j - 2, so K runs a tile ahead).
-    //      The next completion of the awaited barrier needs this very load,
-    //      so its phase cannot run ahead of the wait.
-    if (tid == kVLoader) {
+  int nk = ntiles < NS ? ntiles : NS, nv = nk;  // K / V tiles issued so far (loader)
+  if (warp == K::LOADER / 32) {
+    // ---- loader: K of tile j once the S MMAs of tile j - NS released its
+    //      stage, V of tile j once the P.V MMAs of tile j - NS did, in the
+    //      order those happen (K runs a tile ahead of V).  A stage's "free"
+    //      barrier completes once per tile that used the stage, and its next
+    //      completion needs this very load, so its phase cannot run ahead of
+    //      the wait.
+    if (tid == K::LOADER) {
       while (nk < ntiles || nv < ntiles) {
         const bool is_k = nk < ntiles && nk <= nv + 1;
         const int j = is_k ? nk : nv;
-        if (!mbar_wait_bounded(is_k ? &bar_s[j & 1] : &bar_pv[j & 1], ((j - 2) >> 1) & 1, a.flags)) {
+        if (!mbar_wait_bounded(is_k ? &bar_kf[j % NS] : &bar_vf[j % NS], (j / NS - 1) & 1, a.flags)) {
           fail = true;
           break;
         }
@@ -231,8 +274,8 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   } else {
     for (int i = 0; i < ntiles; ++i) {
       const int s = i & 1;
-      const uint32_t vs_addr = smem_addr(st_s + s * C::STAGE_B) + C::KV_B;
-      if (softmax_thread) {  // warp-uniform: warps 0-3
+      const uint32_t vs_addr = smem_addr(st_s + (i % NS) * C::STAGE_B) + C::KV_B;
+      if (softmax_thread) {  // warp-uniform
         if (!fail && !mbar_wait_bounded(&bar_s[s], (i >> 1) & 1, a.flags)) fail = true;
         tc::fence_after_sync();
         bool wfail = __any_sync(FULL, fail);
@@ -289,11 +332,18 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
             plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
           }
         l_run = l_run * alpha + psum;
-        // the previous P.V must be done before O is touched
-        if (i > 0 && !fail && !mbar_wait_bounded(&bar_pv[(i - 1) & 1], ((i - 1) >> 1) & 1, a.flags)) fail = true;
-        tc::fence_after_sync();
+        // O is rescaled only when a row of the warp raised its maximum (rare
+        // with the lazy rule); only then must the previous P.V be done first.
+        // P goes over this tile's own S buffer, which no MMA in flight reads,
+        // so storing it needs no wait: the softmax of tile i overlaps P.V of
+        // tile i - 1.
+        const bool rescale = __any_sync(FULL, alpha != 1.f);  // warp-uniform
+        if (rescale) {
+          if (i > 0 && !fail && !mbar_wait_bounded(&bar_pv[(i - 1) & 1], ((i - 1) >> 1) & 1, a.flags)) fail = true;
+          tc::fence_after_sync();
+        }
         wfail = __any_sync(FULL, fail);
-        if (!wfail && __any_sync(FULL, alpha != 1.f)) {  // warp-uniform: lanes without a new max scale by 1
+        if (!wfail && rescale) {  // lanes without a new max scale by 1
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
@@ -311,26 +361,31 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
         }
         tc::fence_before_sync();
       }
-      if (mma_group_sync_or(fail)) break;
-      if (tid == kVIssuer) {
+      if (mma_group_sync_or<RTC>(fail)) break;
+      if (tid == K::ISSUER) {
         tc::fence_after_sync();
-        if (!mbar_wait_bounded(&bar_v[s], (i >> 1) & 1, a.flags)) fail = true;
+        if (!mbar_wait_bounded(&bar_v[i % NS], (i / NS) & 1, a.flags)) fail = true;
         if (!fail) {
-          const uint32_t pcol = kColS + s * kVBN;
 #pragma unroll
-          for (int j = 0; j < kVBN / 16; ++j) {
-            const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
-            tc::mma_ts(tmem + kColO, tmem + pcol + 8 * j, vd, IDESC_PV, (i > 0 || j > 0) ? 1u : 0u);
-          }
+          for (int t = 0; t < RTC; ++t) {
+            const uint32_t pcol = t * kColTile + kColS + s * kVBN;
+            const uint32_t ocol = t * kColTile + kColO;
 #pragma unroll
-          for (int j = 0; j < kVBN / 16; ++j) {
-            const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
-            tc::mma_ts(tmem + kColO, tmem + pcol + kColPlo + 8 * j, vd, IDESC_PV, 1u);
+            for (int j = 0; j < kVBN / 16; ++j) {
+              const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
+              tc::mma_ts(tmem + ocol, tmem + pcol + 8 * j, vd, IDESC_PV, (i > 0 || j > 0) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < kVBN / 16; ++j) {
+              const uint64_t vd = tc::smem_desc_sw128(vs_addr + j * 2048, kVBN * 128, 1024);
+              tc::mma_ts(tmem + ocol, tmem + pcol + kColPlo + 8 * j, vd, IDESC_PV, 1u);
+            }
           }
           tc::commit(&bar_pv[s]);
+          tc::commit(&bar_vf[i % NS]);
         }
         if (!fail && i + 2 < ntiles) {
-          // P.V of tile i done: its S buffer takes tile i + 2
+          // P.V of tile i done: its S buffers take tile i + 2
           if (!mbar_wait_bounded(&bar_pv[s], (i >> 1) & 1, a.flags) || !issue_s(i + 2)) fail = true;
         }
       }
@@ -342,21 +397,20 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
     fail = true;
   tc::fence_after_sync();
   const bool aborted = __syncthreads_or(fail) != 0;
-  if (aborted && tid == kVIssuer) {
-    // let MMAs already issued finish before TMEM is released (bounded)
-    for (int j = 0; j < 4; ++j) {
-      mbar_wait_bounded(&bar_s[j >> 1], j & 1, nullptr, 100000000ull);
-      mbar_wait_bounded(&bar_pv[j >> 1], j & 1, nullptr, 100000000ull);
-    }
+  if (aborted && tid == K::ISSUER) {
+    // let MMAs already issued finish before TMEM is released: a commit
+    // arrives once every earlier MMA of this thread is done (bounded wait)
+    tc::commit(bar_dr);
+    mbar_wait_bounded(bar_dr, 0, nullptr, 100000000ull);
   }
-  if (aborted && tid == kVLoader) {
+  if (aborted && tid == K::LOADER) {
     // and the loads still in flight: Q, and the last tile issued into each
-    // slot (earlier ones into it were consumed, hence landed)
+    // stage (earlier ones into it were consumed, hence landed)
     mbar_wait_bounded(bar_q, 0, nullptr, 100000000ull);
     for (int v = 0; v < 2; ++v) {
       const int n = v ? nv : nk;
-      for (int j = n - 2; j < n; ++j)
-        if (j >= 0) mbar_wait_bounded(v ? &bar_v[j & 1] : &bar_k[j & 1], (j >> 1) & 1, nullptr, 100000000ull);
+      for (int j = n - NS; j < n; ++j)
+        if (j >= 0) mbar_wait_bounded(v ? &bar_v[j % NS] : &bar_k[j % NS], (j / NS) & 1, nullptr, 100000000ull);
     }
   }
   __syncthreads();
@@ -411,7 +465,7 @@ __global__ void __launch_bounds__(kVBlock) verify_kernel(const __grid_constant__
   __syncthreads();
   if (warp == 0) {
     tc::fence_after_sync();
-    tc::dealloc(tmem, kVTmemCols);
+    tc::dealloc(tmem, K::TMEM_COLS);
   }
 }
 
@@ -479,22 +533,24 @@ bool make_q_map(CUtensorMap* m, const void* base, int64_t positions, int Hq, int
 
 struct VPlan {
   int nqt, RT, C, tiles_per_chunk;
+  int RTC;  // row tiles per block (RT when two row tiles share each K/V tile, else 1)
   size_t off_ml, off_o, total;
 };
 
 // Resident blocks per SM of one instance (cached per device; also sets the
 // kernel's shared-memory attribute on that device).
-template <int D>
+template <int D, int RTC>
 int verify_occupancy() {
-  using C = VCfg<D>;
+  using C = VCfg<D, RTC>;
   static int cache[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (cache[dev] == 0) {
-    cudaFuncSetAttribute(verify_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
+    cudaFuncSetAttribute(verify_kernel<D, RTC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, verify_kernel<D>, kVBlock, C::SMEM_B) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, verify_kernel<D, RTC>, VBlk<RTC>::THREADS, C::SMEM_B) !=
+            cudaSuccess ||
         n < 1)
       n = 1;
     cache[dev] = n;
@@ -502,7 +558,7 @@ int verify_occupancy() {
   return cache[dev];
 }
 
-// Split of the context into C chunks per (unit, row tile): the C that
+// Split of the context into C chunks per unit: the C that
 // minimises waves x (tiles per chunk + 2), where a wave is SMs x resident
 // blocks and the 2 stands for a block's fixed cost (its query load, pipeline
 // fill and partial write).
@@ -511,12 +567,21 @@ VPlan plan_verify(const vc_attn_shape& sh, int64_t T, int nq) {
   const int g = sh.Hq / sh.Hkv;
   p.nqt = 128 / g;
   if (p.nqt > nq) p.nqt = nq;
-  p.RT = (nq + p.nqt - 1) / p.nqt;
+  p.RT = (nq + p.nqt - 1) / p.nqt;  // 1 or 2 (nq <= 32, g <= 8)
   const int units = sh.B * sh.Hkv;
+  // Two row tiles: one block per unit computes both against each K/V tile it
+  // loads (K/V read once), or one block per row tile (two blocks per SM).
+  // Measured on B200 at 31 rows: with 8 (request, KV head) units the shared
+  // block is 16% faster (g = 8 at 131K keys, g = 5 at 100K), with 32 units
+  // (4 x 32K, g = 8) it is 5-8% slower -- its tile loop is bound by the
+  // tensor pipe's round trips, not by HBM, so it pays off only when the
+  // separate blocks' second read of K/V is what limits them.
+  p.RTC = (p.RT == 2 && units <= 16) ? 2 : 1;
   const int64_t tiles = (T + kVBN - 1) / kVBN;
-  const int occ = sh.D == 128 ? verify_occupancy<128>() : verify_occupancy<64>();
+  const int occ = p.RTC == 2 ? (sh.D == 128 ? verify_occupancy<128, 2>() : verify_occupancy<64, 2>())
+                             : (sh.D == 128 ? verify_occupancy<128, 1>() : verify_occupancy<64, 1>());
   const int64_t slots = static_cast<int64_t>(occ) * sm_count();
-  const int64_t n = static_cast<int64_t>(units) * p.RT;
+  const int64_t n = static_cast<int64_t>(units) * (p.RT / p.RTC);
   int64_t c = 1, best = -1;
   for (int64_t cc = 1; cc <= tiles && cc <= 256; ++cc) {
     const int64_t waves = (n * cc + slots - 1) / slots;
@@ -591,14 +656,21 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
   a.o.lse = lse;
   a.o.part_ml = reinterpret_cast<float*>(w + p.off_ml);
   a.o.part_o = reinterpret_cast<float*>(w + p.off_o);
-  dim3 grid(p.C, units, p.RT);
+  dim3 grid(p.C, units, p.RT / p.RTC);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto go = [&](auto DD, auto RR) {
+    constexpr int Dv = decltype(DD)::value, Rv = decltype(RR)::value;
+    vc::verify_occupancy<Dv, Rv>();  // sets the shared-memory attribute once per device
+    vc::verify_kernel<Dv, Rv><<<grid, vc::VBlk<Rv>::THREADS, vc::VCfg<Dv, Rv>::SMEM_B, s>>>(tq, tk, tv, a);
+  };
+  using I128 = std::integral_constant<int, 128>;
+  using I64 = std::integral_constant<int, 64>;
+  using R1 = std::integral_constant<int, 1>;
+  using R2 = std::integral_constant<int, 2>;
   if (shape->D == 128) {
-    vc::verify_occupancy<128>();  // sets the shared-memory attribute once per device
-    vc::verify_kernel<128><<<grid, vc::kVBlock, vc::VCfg<128>::SMEM_B, s>>>(tq, tk, tv, a);
+    if (p.RTC == 2) go(I128{}, R2{}); else go(I128{}, R1{});
   } else {
-    vc::verify_occupancy<64>();
-    vc::verify_kernel<64><<<grid, vc::kVBlock, vc::VCfg<64>::SMEM_B, s>>>(tq, tk, tv, a);
+    if (p.RTC == 2) go(I64{}, R2{}); else go(I64{}, R1{});
   }
   if (p.C > 1) {  // chunk partials -> output rows (and lse)
     const int rows_cap = p.nqt * a.g;

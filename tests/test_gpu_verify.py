@@ -43,8 +43,10 @@ def test_tiny_single_layer_eight_rows():
 
 @pytest.mark.parametrize("B,nq,Hq,Hkv,D,T", [
     (2, 31, 32, 8, 128, 2000),   # Llama-style GQA, K = 30 drafts + 1
-    (1, 31, 40, 8, 128, 3001),   # g = 5: two row tiles
-    (1, 31, 64, 8, 128, 1500),   # g = 8: two row tiles
+    (1, 31, 40, 8, 128, 3001),   # g = 5: two row tiles in one block (8 units)
+    (1, 31, 64, 8, 128, 1500),   # g = 8: two row tiles in one block
+    (3, 31, 64, 8, 128, 700),    # g = 8, 24 units: one block per row tile
+    (2, 31, 16, 2, 64, 900),     # g = 8, D = 64, two row tiles in one block
     (1, 1, 4, 4, 128, 100),      # one row, g = 1
     (1, 32, 4, 1, 64, 32),       # T == nq: the block is the whole cache
     (1, 31, 4, 1, 128, 96),      # one full tile plus a ragged tail

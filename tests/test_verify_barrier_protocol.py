@@ -10,17 +10,20 @@ kernel's three roles with random latencies and checks that precondition at
 every wait, that every role finishes (no deadlock), and that every load and
 MMA happens exactly once:
 
-* loader: Q, K and V of tiles 0 and 1, then K of tile j once S of tile j - 2
-  is done and V of tile j once P.V of tile j - 2 is done, in the order those
-  happen (K one tile ahead of V);
+* loader: Q, K and V of tiles 0 .. NS - 1 (NS stages: 2, or 4 when one block
+  takes two row tiles), then K of tile j once the S MMAs of tile j - NS
+  released stage j mod NS and V of tile j once the P.V MMAs of tile j - NS
+  did, in the order those happen (K one tile ahead of V);
 * MMA thread: S of tiles 0 and 1 (after Q and their K), then per tile i,
   after the softmax group's barrier: P.V(i) once V(i) landed, and S(i + 2)
-  into S buffer i & 1 once P.V(i) is done and K(i + 2) landed;
-* softmax group: per tile i, wait S(i), work, wait P.V(i - 1), barrier.
+  into S buffer i & 1 once P.V(i) is done and K(i + 2) landed; each S group
+  also releases its K stage, each P.V group its V stage;
+* softmax group: per tile i, wait S(i), work, wait P.V(i - 1) when it
+  rescales O (the lazy rule makes that rare), barrier.
 
-Barriers: k0 k1 v0 v1 (slots), s0 s1 (S buffers), pv0 pv1 (P.V per buffer),
-q.  The tensor pipe runs MMA groups in issue order; a commit fires when its
-group ends.
+Barriers: k<j> v<j> (stage landed), kf<j> vf<j> (stage released) for
+j < NS, s0 s1 (S buffers), pv0 pv1 (P.V per buffer), q.  The tensor pipe
+runs MMA groups in issue order; a group's commits fire when it ends.
 """
 
 import heapq
@@ -89,7 +92,8 @@ class _Sim:
         elif kind == "mma":
             start = max(self.t, self.pipe_free)
             self.pipe_free = start + req[2]
-            self.fire_after(self.pipe_free - self.t, req[1])
+            for name in (req[1] if isinstance(req[1], tuple) else (req[1],)):
+                self.fire_after(self.pipe_free - self.t, name)
             self.schedule(self.rng.uniform(0, req[2]), gen)  # the issue may block part of the time
         elif kind == "group":
             self.group.append(gen)
@@ -99,21 +103,21 @@ class _Sim:
                 self.group = []
 
 
-def _run_protocol(n, rng):
+def _run_protocol(n, rng, NS):
     sim = _Sim(rng)
     finished = []
 
     def loader():
         yield ("load", "q")
-        for j in range(min(2, n)):
-            yield ("load", f"k{j & 1}")
-            yield ("load", f"v{j & 1}")
-        nk = nv = min(2, n)
+        for j in range(min(NS, n)):
+            yield ("load", f"k{j % NS}")
+            yield ("load", f"v{j % NS}")
+        nk = nv = min(NS, n)
         while nk < n or nv < n:
             is_k = nk < n and nk <= nv + 1
             j = nk if is_k else nv
-            yield ("wait", (f"s{j & 1}" if is_k else f"pv{j & 1}"), (j - 2) >> 1)
-            yield ("load", (f"k{j & 1}" if is_k else f"v{j & 1}"))
+            yield ("wait", (f"kf{j % NS}" if is_k else f"vf{j % NS}"), j // NS - 1)
+            yield ("load", (f"k{j % NS}" if is_k else f"v{j % NS}"))
             if is_k:
                 nk = j + 1
             else:
@@ -122,8 +126,8 @@ def _run_protocol(n, rng):
 
     def mma():
         def issue_s(i):
-            yield ("wait", f"k{i & 1}", i >> 1)
-            yield ("mma", f"s{i & 1}", rng.uniform(3, 30))
+            yield ("wait", f"k{i % NS}", i // NS)
+            yield ("mma", (f"s{i & 1}", f"kf{i % NS}"), rng.uniform(3, 30))
 
         yield ("sleep", rng.uniform(0, 20))
         yield ("wait", "q", 0)
@@ -131,8 +135,8 @@ def _run_protocol(n, rng):
             yield from issue_s(i)
         for i in range(n):
             yield ("group",)
-            yield ("wait", f"v{i & 1}", i >> 1)
-            yield ("mma", f"pv{i & 1}", rng.uniform(5, 60))
+            yield ("wait", f"v{i % NS}", i // NS)
+            yield ("mma", (f"pv{i & 1}", f"vf{i % NS}"), rng.uniform(5, 60))
             if i + 2 < n:
                 yield ("wait", f"pv{i & 1}", i >> 1)
                 yield from issue_s(i + 2)
@@ -143,7 +147,7 @@ def _run_protocol(n, rng):
         for i in range(n):
             yield ("wait", f"s{i & 1}", i >> 1)
             yield ("sleep", rng.uniform(5, 80))
-            if i > 0:
+            if i > 0 and rng.random() < 0.3:  # only a warp that rescales O waits for P.V(i - 1)
                 yield ("wait", f"pv{(i - 1) & 1}", (i - 1) >> 1)
             yield ("group",)
         yield ("wait", f"pv{(n - 1) & 1}", (n - 1) >> 1)
@@ -153,16 +157,19 @@ def _run_protocol(n, rng):
         sim.schedule(0.0, g)
     sim.run()
     assert sorted(finished) == ["loader", "mma", "softmax"], "a role never finished (deadlock)"
-    for kind in ("k", "v", "s", "pv"):
+    for kind in ("s", "pv"):
         assert sim.done(f"{kind}0") + sim.done(f"{kind}1") == n, kind
+    for kind in ("k", "v", "kf", "vf"):
+        assert sum(sim.done(f"{kind}{j}") for j in range(NS)) == n, kind
     assert sim.done("q") == 1
 
 
+@pytest.mark.parametrize("NS", [2, 4])
 @pytest.mark.parametrize("ntiles", list(range(1, 12)))
-def test_parity_waits_never_early_or_late(ntiles):
-    rng = random.Random(1000 + ntiles)
+def test_parity_waits_never_early_or_late(ntiles, NS):
+    rng = random.Random(1000 + ntiles + 100 * NS)
     for _ in range(150):
-        _run_protocol(ntiles, rng)
+        _run_protocol(ntiles, rng, NS)
 
 
 def test_model_catches_a_wait_on_a_stale_phase():
