@@ -58,6 +58,12 @@ WORKLOADS = {
     "llama-70b-4x131k-4bit-stagger": dict(kind="stagger", NL=80, B=1, n_req=4, Hq=64, Hkv=8, D=128, T=131072,
                                           bits=4, G=64, R=128, K=30, V=128256, logits="bf16", p_mismatch=0.2,
                                           host_pool=2),
+    # remote prefix caching: each request's compressed prefix cache arrives over an emulated 1.2 GB/s remote
+    # link, its full cache is streamed for verification over an emulated 40 GB/s local link
+    "llama-3.1-8b-4x32k-kivi2-remote-prefix": dict(kind="remote", NL=32, B=1, n_req=4, Hq=32, Hkv=8, D=128,
+                                                   T=32768, bits=2, G=32, R=128, K=30, V=128256, logits="bf16",
+                                                   p_mismatch=0.2, host_pool=2, remote_gbps=1.2, local_gbps=40.0,
+                                                   rounds=2),
 }
 
 
@@ -676,6 +682,107 @@ def run_stagger(args, w, rank, world):
                 link_bytes_per_request=2 * hk[0].numel() * hk[0].element_size() * NL, host_pool_layers=len(hk))
 
 
+def run_remote(args, w, rank, world):
+    """Remote prefix caching: every request's compressed cache (all layers:
+    group records and residual) starts in pinned host memory and reaches the
+    GPU over the emulated remote link before the request's first draft; each
+    round then drafts from it (HBM) and verifies against the full cache
+    streamed over the emulated local link.  One run = the fetches plus
+    `rounds` rounds of every request, by the scheduler in lock-step and in
+    the staggered order."""
+    import torch
+    from lossless_draft_verify_vc_b200 import synth, vc
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    vc.lib()
+    NL, B, Hq, Hkv, D, T, K, V, n = (w["NL"], w["B"], w["Hq"], w["Hkv"], w["D"], w["T"], w["K"], w["V"],
+                                     w["n_req"])
+    nq = K + 1
+    sh = vc.shape(B, Hq, Hkv, D)
+    hk, hv = host_pool(w, torch.bfloat16, w["host_pool"])
+    copy, remote = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    reqs, keep, fetch = [], [], []
+    accepted = 0
+    for i in range(n):
+        seed0 = 1000 * rank + 100 * i
+        caches, src, dst = [], [], []
+        for l in range(NL):
+            c = synth.random_quant_cache(B, Hkv, T - w["R"], w["R"], D, w["bits"], w["G"], seed=seed0 + l,
+                                         device=dev)
+            for key in ("records", "k_res", "v_res"):
+                src.append(c[key].cpu().pin_memory())
+                dst.append(c[key])
+                c[key].zero_()  # the device copy is filled by the fetch
+            caches.append(c)
+        qcs = [vc.quant_cache(c) for c in caches]
+        q_draft = synth.normal((K, NL, B, Hq, D), seed0 + 1, dev)
+        q_ver = synth.normal((NL, B, nq, Hq, D), seed0 + 2, dev)
+        toks = synth.tokens((B, K), V, seed0 + 3, dev)
+        lens = synth.geometric_accept_lengths(B, K, w["p_mismatch"], seed0 + 3)
+        accepted += sum(a + 1 for a in lens)
+        logits = synth.planted_logits(B, K, V, toks.cpu(), lens, seed0 + 4, device="cpu",
+                                      dtype=torch.bfloat16).to(dev)
+        st_k = [torch.empty_like(hk[0], device=dev) for _ in range(2)]
+        st_v = [torch.empty_like(hv[0], device=dev) for _ in range(2)]
+        out = dict(d=torch.empty(B, Hq, D, device=dev), v=torch.empty(B, nq, Hq, D, device=dev),
+                   t=torch.empty(B, K + 1, dtype=torch.int32, device=dev),
+                   a=torch.empty(B, dtype=torch.int32, device=dev), c=torch.empty(B, dtype=torch.int32, device=dev))
+        dws = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, qcs[0]), dev)
+        vws = vc.workspace(vc.vc_verify_attn_workspace_size(sh, T, nq), dev)
+        aws = vc.workspace(vc.vc_accept_workspace_size(B, K, V), dev)
+        stream = torch.cuda.Stream(dev)
+        reqs.append(vc.make_sched_request(sh, vc.VC_DRAFT_QUANT, qcs, q_draft, out["d"], dws,
+                                          [hk[l % len(hk)] for l in range(NL)], [hv[l % len(hv)] for l in range(NL)],
+                                          st_k, st_v, q_ver, out["v"], vws, T, nq, logits, V, toks, out["t"],
+                                          out["a"], out["c"], aws, stream))
+        keep.append((caches, qcs, out, lens, q_draft))
+        fetch.append((src, dst))
+    fetch_bytes = sum(t.numel() * t.element_size() for src, _ in fetch for t in src)
+    rounds = w.get("rounds", 2)
+    # draft kernel alone (request 0, its cache fetched once directly)
+    for a_, b_ in zip(*fetch[0]):
+        b_.copy_(a_)
+    qcs0, q_draft0, out0 = keep[0][1], keep[0][4], keep[0][2]["d"]
+    dws0 = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, qcs0[0]), dev)
+    comp = torch.cuda.current_stream(dev)
+    for l in range(NL):
+        vc.vc_draft_attn_quant(sh, qcs0[l], q_draft0[0, l], out0, dws0, comp)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for t in range(K):
+        for l in range(NL):
+            vc.vc_draft_attn_quant(sh, qcs0[l], q_draft0[t, l], out0, dws0, comp)
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    draft_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
+    res = {}
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    for name, pol in (("lockstep", vc.VC_SCHED_LOCKSTEP), ("stagger", vc.VC_SCHED_STAGGER)):
+        sch = vc.Sched(reqs, NL, K, pol, copy, timeout_ms=30000)
+        sch.set_links(remote, w["remote_gbps"], w["local_gbps"])
+        for i, (src, dst) in enumerate(fetch):
+            sch.set_fetch(i, src, dst)
+        if world > 1:
+            torch.distributed.barrier()
+        st = sch.run_rounds(rounds)
+        torch.cuda.synchronize(dev)
+        sch.close()
+        for k in ("elapsed_ms", "fetch_ms", "link_busy_ms", "first_draft_ms"):
+            st[k] = max_over_ranks([st[k]], dev)[0]
+        for (_, _, out, lens, _) in keep:
+            assert out["a"].cpu().tolist() == lens, "acceptance mismatch under the scheduler"
+        res[name] = st
+    clk = clocks.stop()
+    return dict(draft_ms=draft_ms, sched=res, clocks=clk, fetch_bytes=fetch_bytes,
+                link_bytes_per_request_round=2 * hk[0].numel() * hk[0].element_size() * NL,
+                host_pool_layers=len(hk), rounds=rounds, tokens_per_run=accepted * rounds)
+
+
 # ----------------------------------------------------------------------------- oracle leg
 def oracle_sample(w, budget_s: float):
     """Time the oracle's quantised draft attention on (request 0, KV head 0)
@@ -740,8 +847,12 @@ def main():
     if w["kind"] != "resident" or w.get("streamed_too"):
         config.update(full_kv="pinned host memory, streamed per layer",
                       host_pool_layers=w.get("host_pool", 2))
-    if w["kind"] == "stagger":
+    if w["kind"] in ("stagger", "remote"):
         config.update(requests=w["n_req"])
+    if w["kind"] == "remote":
+        config.update(full_kv="pinned host memory, streamed per layer over the emulated local link",
+                      draft_cache="pinned host memory, fetched over the emulated remote link",
+                      remote_gbps=w["remote_gbps"], local_gbps=w["local_gbps"])
 
     if args.impl == "reference":
         if rank != 0:
@@ -772,6 +883,8 @@ def main():
         line = streamed_line(args, w, rank, world, config, peak, peak_kind)
     elif w["kind"] == "stagger":
         line = stagger_line(args, w, rank, world, config, peak, peak_kind)
+    elif w["kind"] == "remote":
+        line = remote_line(args, w, rank, world, config, peak, peak_kind)
     else:
         line = resident_line(args, w, rank, world, config, peak, peak_kind)
     if rank == 0:
@@ -861,6 +974,43 @@ def stagger_line(args, w, rank, world, config, peak, peak_kind):
                      "algorithmic_bytes_per_launch": db},
         "gpu_launches": 2 * K * NL,
         "verify_resident_layer": resident_verify_block(w, peak, peak_kind),
+    })
+    return line
+
+
+def remote_line(args, w, rank, world, config, peak, peak_kind):
+    r = run_remote(args, w, rank, world)
+    K, NL, n = w["K"], w["NL"], w["n_req"]
+    db = draft_bytes_per_layer(w)
+    value = whole_job_rate(db * K * NL, 1, world, r["draft_ms"])
+    lk, sg = r["sched"]["lockstep"], r["sched"]["stagger"]
+    achieved = db / (r["draft_ms"] * 1e3 / (K * NL) * 1e-6) / 1e9
+    local_bytes = r["link_bytes_per_request_round"] * n * r["rounds"]
+    line = _common(args, config, value, peak, peak_kind, r, "int2 codes + bf16 -> fp16/bf16 MMA, fp32 accumulate")
+
+    def pol(st):
+        return {"ms_per_run": st["elapsed_ms"], "tokens_per_s": r["tokens_per_run"] / (st["elapsed_ms"] * 1e-3),
+                "remote_gbps": r["fetch_bytes"] / (st["fetch_ms"] * 1e-3) / 1e9,
+                "remote_busy_frac": st["fetch_ms"] / st["elapsed_ms"],
+                "local_gbps_while_streaming": local_bytes / (st["link_busy_ms"] * 1e-3) / 1e9,
+                "local_busy_frac": st["link_busy_ms"] / st["elapsed_ms"],
+                "last_first_draft_ms": st["first_draft_ms"]}
+
+    line.update({
+        "ms_per_step": sg["elapsed_ms"],
+        "draft_frac_of_hbm_peak": value / world / peak,
+        "remote_prefix": {"lockstep": pol(lk), "stagger": pol(sg), "speedup": lk["elapsed_ms"] / sg["elapsed_ms"],
+                          "remote_link_gbps_set": w["remote_gbps"], "local_link_gbps_set": w["local_gbps"],
+                          "fetch_bytes": r["fetch_bytes"], "rounds_per_run": r["rounds"],
+                          "tokens_per_run": r["tokens_per_run"],
+                          "note": "one run = every request's compressed cache fetched over the remote link, then "
+                                  "`rounds` draft/verify/accept rounds per request; tokens = accepted drafts + the "
+                                  "correction per round (planted acceptance)"},
+        "roofline": {"kernel": "vc_draft_attn_quant (draft_quant_kernel)", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)", "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "algorithmic_bytes_per_launch": db},
+        # the timed draft loop: K * NL draft kernels
+        "gpu_launches": K * NL,
     })
     return line
 

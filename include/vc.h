@@ -359,6 +359,27 @@ VC_API vc_status vc_kvstream_acquire(vc_kvstream* s, int layer, void* compute_st
 VC_API vc_status vc_kvstream_release(vc_kvstream* s, int layer, void* compute_stream);
 VC_API vc_status vc_kvstream_destroy(vc_kvstream* s);
 
+/* ---- bandwidth-limited links ---------------------------------------------------
+ * Remote prefix caching sends the compressed cache to the serving GPU over a
+ * slow network while the full cache stays reachable over a fast local link
+ * (menfem.com source page, "Key Contributions" (two deployment pipelines),
+ * "Methodology": 1.2 GB/s remote against 40 GB/s local).  A vc_link emulates
+ * a host -> device link of `gbps` GB/s on the GPU's own bus: copies run on
+ * `stream` in chunks of chunk_bytes (0: 8 MiB), each released no sooner than
+ * its size / gbps after the previous one started (a one-thread kernel sleeps
+ * on the device clock; bounded at 60 s per chunk, after which it sets
+ * VC_FLAG_WAIT_TIMEOUT and lets the copy proceed).  gbps == 0: unpaced.
+ *   vc_link_copy   asynchronous host -> device copy on the link's stream
+ *                  (src should be pinned host memory); returns at once.
+ *   vc_link_flags  reads and clears the link's flag word (synchronous).
+ *   vc_link_destroy waits for the link's stream, then frees the link.
+ * The link allocates 64 bytes of device memory for its clock. */
+typedef struct vc_link vc_link;
+VC_API vc_status vc_link_create(vc_link** out, void* stream, double gbps, size_t chunk_bytes);
+VC_API vc_status vc_link_copy(vc_link* link, void* dst, const void* src, size_t bytes);
+VC_API vc_status vc_link_flags(vc_link* link, uint32_t* host_flags);
+VC_API vc_status vc_link_destroy(vc_link* link);
+
 /* ---- cross-request staggering scheduler -------------------------------------
  * Drafting is bound by HBM bandwidth and verification by the host link, so
  * the pages interleave different requests' draft and verify phases instead
@@ -418,11 +439,13 @@ typedef struct vc_sched_request {
 } vc_sched_request;
 typedef struct vc_sched_stats {
   double elapsed_ms;      /* device time from the first enqueued work to the last completion */
-  double link_busy_ms;    /* device time the copy stream spent copying */
+  double link_busy_ms;    /* device time the copy stream spent copying (verification streaming) */
   double draft_ms;        /* summed device time of the draft phases */
   double verify_ms;       /* summed device time of the verify + accept phases */
   int rounds;
   int requests;
+  double fetch_ms;        /* summed device time of the requests' fetches over the remote link */
+  double first_draft_ms;  /* device time from the start to the last request's first draft */
 } vc_sched_stats;
 typedef struct vc_sched vc_sched;
 VC_API vc_status vc_sched_create(vc_sched** out, int n_requests, const vc_sched_request* reqs, int n_layers,
@@ -430,16 +453,39 @@ VC_API vc_status vc_sched_create(vc_sched** out, int n_requests, const vc_sched_
 VC_API vc_status vc_sched_run_rounds(vc_sched* s, int n_rounds, vc_sched_stats* stats);
 VC_API vc_status vc_sched_destroy(vc_sched* s);
 
+/* Remote prefix caching (the pages' second deployment pipeline; see the
+ * links above).  vc_sched_set_links paces the scheduler's transfers:
+ *   remote_stream, remote_gbps  the link that fetches requests' compressed
+ *                               caches (vc_sched_set_fetch); gbps 0: unpaced
+ *   local_gbps                  the verification streaming on copy_stream
+ *                               (0: unpaced, the bus's own speed)
+ *   chunk_bytes                 pacing chunk (0: 8 MiB)
+ * vc_sched_set_fetch gives request r a list of n host -> device copies
+ * (src pinned host, dst device, bytes each; the arrays are copied) that
+ * every vc_sched_run_rounds call performs over the remote link, in request
+ * order, before r's first draft of that call.  VC_SCHED_STAGGER lets r draft
+ * as soon as its own fetch is done (other requests' fetches continue on the
+ * remote link while r drafts and verifies); VC_SCHED_LOCKSTEP starts the
+ * first drafts only when every fetch is done.  Both return
+ * VC_ERR_INVALID_ARG for bad arguments. */
+VC_API vc_status vc_sched_set_links(vc_sched* s, void* remote_stream, double remote_gbps, double local_gbps,
+                                    size_t chunk_bytes);
+VC_API vc_status vc_sched_set_fetch(vc_sched* s, int request, int n, const void* const* src, void* const* dst,
+                                    const size_t* bytes);
+
 /* Host-only model of the same policy on a simulated timeline (no GPU): each
- * request's draft takes draft_ms of the GPU (drafts share the GPU one at a
- * time) and its verification verify_ms of the link (one at a time).  Writes
- * the finishing time of the last round to *makespan_ms.  A request index
- * `never_done` >= 0 makes that request's first verification never complete,
- * which exercises the timeout path (VC_ERR_TIMEOUT after timeout_ms of
- * simulated time without progress).  Used by the CPU tests of the policy. */
-VC_API vc_status vc_sched_simulate(int n_requests, int n_rounds, int policy, const double* draft_ms,
-                                   const double* verify_ms, int never_done, double timeout_ms,
-                                   double* makespan_ms);
+ * request's fetch takes fetch_ms of the remote link (fetch_ms may be NULL:
+ * no fetches; fetches run one at a time in request order, all enqueued at
+ * the start), its draft draft_ms of the GPU (drafts share the GPU one at a
+ * time) and its verification verify_ms of the local link (one at a time).
+ * Writes the finishing time of the last round to *makespan_ms.  A request
+ * index `never_done` >= 0 makes that request's first verification never
+ * complete, which exercises the timeout path (VC_ERR_TIMEOUT after
+ * timeout_ms of simulated time without progress).  Used by the CPU tests
+ * of the policy. */
+VC_API vc_status vc_sched_simulate(int n_requests, int n_rounds, int policy, const double* fetch_ms,
+                                   const double* draft_ms, const double* verify_ms, int never_done,
+                                   double timeout_ms, double* makespan_ms);
 
 /* ---- workspace flags -------------------------------------------------------
  * Copies the device-side flag word of a workspace to *host_flags and clears

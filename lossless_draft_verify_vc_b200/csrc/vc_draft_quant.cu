@@ -57,6 +57,7 @@ constexpr int kResRows = 16;     // residual rows per stage
 // 2-bit group-32 records)
 constexpr int kResCostNum = 4, kResCostDen = 3;
 constexpr int kMergeFloats = 512;  // shared-memory area of the final per-unit merge (2 KB)
+constexpr int kMinWarpStages = 8;  // measured on B200: 1 x 32K keys 26.0 -> 22.8 us per call, larger shapes unchanged
 
 template <int BITS, int G, int D, int NT>
 struct QCfg {
@@ -1423,6 +1424,11 @@ QPlan make_plan(const vc_attn_shape& sh, const vc_quant_cache& c, int ng_per_sta
     const int64_t mx = P.sq > 0 && P.sr > 0 ? (P.cq > P.cr ? P.cq : P.cr) : (P.sq > 0 ? P.cq : P.cr);
     int64_t bpu = target_blocks / P.U;
     if (bpu > P.ucost() / mx) bpu = P.ucost() / mx;  // every piece holds at least one tile or stage
+    // every warp gets at least kMinWarpStages quantised stages: the last
+    // block of a unit merges all of the unit's partials at the call's end,
+    // so more blocks than that shorten the stages but lengthen the merge
+    const int64_t cap = P.sq / (static_cast<int64_t>(kQNW) * kMinWarpStages);
+    if (P.sq > 0 && bpu > cap) bpu = cap;
     if (bpu < 1) bpu = 1;
     P.bpu = static_cast<int>(bpu);
     P.nblk = P.U * P.bpu;

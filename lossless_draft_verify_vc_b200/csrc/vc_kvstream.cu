@@ -49,9 +49,16 @@ vc_status KvStream::prefetch(int layer, cudaEvent_t t0, cudaEvent_t t1) {
   if (slot_used[s] && cudaStreamWaitEvent(copy_stream, released[s], 0) != cudaSuccess)
     return set_error(VC_ERR_CUDA, "vc_kvstream_prefetch: wait failed");
   if (t0) cudaEventRecord(t0, copy_stream);
-  if (cudaMemcpyAsync(dev_k[s], host_k[layer], bytes_per_layer, cudaMemcpyHostToDevice, copy_stream) != cudaSuccess ||
-      cudaMemcpyAsync(dev_v[s], host_v[layer], bytes_per_layer, cudaMemcpyHostToDevice, copy_stream) != cudaSuccess)
+  if (link) {
+    vc_status st = link->copy(dev_k[s], host_k[layer], bytes_per_layer);
+    if (st == VC_OK) st = link->copy(dev_v[s], host_v[layer], bytes_per_layer);
+    if (st != VC_OK) return st;
+  } else if (cudaMemcpyAsync(dev_k[s], host_k[layer], bytes_per_layer, cudaMemcpyHostToDevice, copy_stream) !=
+                 cudaSuccess ||
+             cudaMemcpyAsync(dev_v[s], host_v[layer], bytes_per_layer, cudaMemcpyHostToDevice, copy_stream) !=
+                 cudaSuccess) {
     return set_error(VC_ERR_CUDA, "vc_kvstream_prefetch: copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+  }
   if (t1) cudaEventRecord(t1, copy_stream);
   if (cudaEventRecord(copied[s], copy_stream) != cudaSuccess)
     return set_error(VC_ERR_CUDA, "vc_kvstream_prefetch: event record failed");

@@ -5,6 +5,7 @@
 #include <vector>
 
 #include "vc_common.cuh"
+#include "vc_link.h"
 
 namespace vc {
 
@@ -20,6 +21,7 @@ struct KvStream {
   cudaEvent_t copied[2] = {nullptr, nullptr};
   cudaEvent_t released[2] = {nullptr, nullptr};
   cudaStream_t copy_stream = nullptr;
+  PacedLink* link = nullptr;  // optional: copies go through this link (on copy_stream) at its rate
 
   vc_status init(int n_layers, const void* const* hk, const void* const* hv, size_t bytes, void* const* dk,
                  void* const* dv, cudaStream_t cs);

@@ -65,7 +65,8 @@ class vc_sched_request(Structure):
 
 class vc_sched_stats(Structure):
     _fields_ = [("elapsed_ms", ctypes.c_double), ("link_busy_ms", ctypes.c_double), ("draft_ms", ctypes.c_double),
-                ("verify_ms", ctypes.c_double), ("rounds", c_int), ("requests", c_int)]
+                ("verify_ms", ctypes.c_double), ("rounds", c_int), ("requests", c_int),
+                ("fetch_ms", ctypes.c_double), ("first_draft_ms", ctypes.c_double)]
 
 
 VC_DRAFT_QUANT, VC_DRAFT_SPARSE = 0, 1
@@ -123,8 +124,14 @@ def lib() -> ctypes.CDLL:
                                         c_int]),
             "vc_sched_run_rounds": (c_int, [c_void_p, c_int, P(vc_sched_stats)]),
             "vc_sched_destroy": (c_int, [c_void_p]),
-            "vc_sched_simulate": (c_int, [c_int, c_int, c_int, P(ctypes.c_double), P(ctypes.c_double), c_int,
-                                          ctypes.c_double, P(ctypes.c_double)]),
+            "vc_sched_simulate": (c_int, [c_int, c_int, c_int, P(ctypes.c_double), P(ctypes.c_double),
+                                          P(ctypes.c_double), c_int, ctypes.c_double, P(ctypes.c_double)]),
+            "vc_sched_set_links": (c_int, [c_void_p, c_void_p, ctypes.c_double, ctypes.c_double, c_size_t]),
+            "vc_sched_set_fetch": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+            "vc_link_create": (c_int, [P(c_void_p), c_void_p, ctypes.c_double, c_size_t]),
+            "vc_link_copy": (c_int, [c_void_p, c_void_p, c_void_p, c_size_t]),
+            "vc_link_flags": (c_int, [c_void_p, P(c_uint32)]),
+            "vc_link_destroy": (c_int, [c_void_p]),
             "vc_debug_gather": (c_int, [P(vc_attn_shape), P(vc_sparse_cache), c_void_p, c_void_p, c_void_p,
                                         c_size_t, c_void_p]),
         }
@@ -375,11 +382,30 @@ class Sched:
                                      _stream(copy_stream), int(timeout_ms)))
         self.h = h
 
+    def set_links(self, remote_stream, remote_gbps: float, local_gbps: float = 0.0, chunk_bytes: int = 0):
+        self._keep.append(remote_stream)
+        _check(lib().vc_sched_set_links(self.h, _stream(remote_stream), float(remote_gbps), float(local_gbps),
+                                        int(chunk_bytes)))
+
+    def set_fetch(self, request: int, src, dst):
+        """Copies (pinned host tensor -> device tensor of the same size) that
+        bring the request's compressed cache over the remote link."""
+        n = len(src)
+        sa = (c_void_p * n)(*[_p(t) for t in src])
+        da = (c_void_p * n)(*[_p(t) for t in dst])
+        ba = (c_size_t * n)(*[t.numel() * t.element_size() for t in src])
+        for a, b in zip(src, dst):
+            assert a.numel() * a.element_size() == b.numel() * b.element_size()
+        self._keep.append((src, dst))
+        _check(lib().vc_sched_set_fetch(self.h, int(request), n, ctypes.cast(sa, c_void_p), ctypes.cast(da, c_void_p),
+                                        ctypes.cast(ba, c_void_p)))
+
     def run_rounds(self, n_rounds: int) -> dict:
         st = vc_sched_stats()
         _check(lib().vc_sched_run_rounds(self.h, int(n_rounds), ctypes.byref(st)))
         return dict(elapsed_ms=st.elapsed_ms, link_busy_ms=st.link_busy_ms, draft_ms=st.draft_ms,
-                    verify_ms=st.verify_ms, rounds=st.rounds, requests=st.requests)
+                    verify_ms=st.verify_ms, rounds=st.rounds, requests=st.requests, fetch_ms=st.fetch_ms,
+                    first_draft_ms=st.first_draft_ms)
 
     def close(self):
         if self.h:
@@ -427,12 +453,49 @@ def make_sched_request(sh, kind, caches, draft_q, draft_out, draft_ws, host_k, h
 
 
 def vc_sched_simulate(draft_ms, verify_ms, n_rounds: int, policy: int, never_done: int = -1,
-                      timeout_ms: float = 1e9) -> float:
+                      timeout_ms: float = 1e9, fetch_ms=None) -> float:
     """Makespan of the scheduling policy on a simulated timeline (host only)."""
     n = len(draft_ms)
     d = (ctypes.c_double * n)(*draft_ms)
     v = (ctypes.c_double * n)(*verify_ms)
+    f = (ctypes.c_double * n)(*fetch_ms) if fetch_ms is not None else None
     out = ctypes.c_double()
-    _check(lib().vc_sched_simulate(n, int(n_rounds), int(policy), d, v, int(never_done), float(timeout_ms),
+    _check(lib().vc_sched_simulate(n, int(n_rounds), int(policy), f, d, v, int(never_done), float(timeout_ms),
                                    ctypes.byref(out)))
     return out.value
+
+
+# ---- bandwidth-limited link --------------------------------------------------------
+
+class Link:
+    """Handle of a vc_link: host -> device copies on `stream` at `gbps` GB/s
+    (0: unpaced), in chunks of chunk_bytes (0: 8 MiB)."""
+
+    def __init__(self, stream, gbps: float, chunk_bytes: int = 0):
+        h = c_void_p()
+        self._keep = [stream]
+        _check(lib().vc_link_create(ctypes.byref(h), _stream(stream), float(gbps), int(chunk_bytes)))
+        self.h = h
+
+    def copy(self, dst, src):
+        n = src.numel() * src.element_size()
+        assert dst.numel() * dst.element_size() >= n
+        self._keep.append((dst, src))
+        _check(lib().vc_link_copy(self.h, _p(dst), _p(src), n))
+
+    def flags(self) -> int:
+        v = c_uint32(0)
+        _check(lib().vc_link_flags(self.h, ctypes.byref(v)))
+        return int(v.value)
+
+    def close(self):
+        if self.h:
+            _check(lib().vc_link_destroy(self.h))
+            self.h = None
+            self._keep = []
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

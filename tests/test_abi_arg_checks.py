@@ -184,6 +184,29 @@ def test_sched_create_rejects(L, n_req, policy, timeout_ms, req):
     assert not handle.value
 
 
+@pytest.mark.parametrize("out,gbps,chunk", [
+    (False, 1.2, 0),          # null output
+    (True, -1.0, 0),          # negative rate
+    (True, 2e4, 0),           # absurd rate
+    (True, 1.2, 100),         # chunk below 4 KiB
+    (True, 1.2, (1 << 32) + 16),  # chunk above 4 GiB
+])
+def test_link_create_rejects_before_allocating(L, out, gbps, chunk):
+    handle = ctypes.c_void_p(0)
+    st = L.vc_link_create(ctypes.byref(handle) if out else None, None, gbps, chunk)
+    _expect_invalid(L, st, "vc_link_create")
+    assert not handle.value
+
+
+def test_link_and_remote_fetch_calls_reject_null_objects(L):
+    _expect_invalid(L, L.vc_link_copy(None, A, A, 16), "vc_link_copy")
+    flags = ctypes.c_uint32(0)
+    _expect_invalid(L, L.vc_link_flags(None, ctypes.byref(flags)), "vc_link_flags")
+    assert L.vc_link_destroy(None) == 0
+    _expect_invalid(L, L.vc_sched_set_links(None, None, 1.2, 40.0, 0), "vc_sched_set_links")
+    _expect_invalid(L, L.vc_sched_set_fetch(None, 0, 0, None, None, None), "vc_sched_set_fetch")
+
+
 def test_wait_timeout_export_rejects_before_any_launch(L):
     # null pointers and limits outside 1 us .. 100 ms are refused on the host
     assert L.vc_debug_wait_timeout(None, 16, 1000000, None) == vc.VC_ERR_INVALID_ARG

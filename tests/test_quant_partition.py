@@ -90,8 +90,12 @@ def test_partition_covers_every_tile_and_stage_once_in_balanced_pieces(Bq, Hq, H
             assert (u0, u1) == (k // bpu, k // bpu + 1)
             c = (r1 - r0) * cr + (q1 - q0) * cq
             assert abs(c - unit_cost / bpu) <= max(cq if sq else 0, cr if sr else 0) + 1, (k, c, unit_cost / bpu)
-        # as many blocks as fit, up to one piece per tile or stage
-        assert bpu == min(target // U, unit_cost // max(cq if sq else 0, cr if sr else 0))
+        # as many blocks as fit, up to one piece per tile or stage, and at least 8
+        # quantised stages per warp (4 warps per block) when the unit has any
+        want = min(target // U, unit_cost // max(cq if sq else 0, cr if sr else 0))
+        if sq:
+            want = min(want, sq // (4 * 8))
+        assert bpu == max(1, want)
     else:
         assert U > target and n == target
         per = [u1 - u0 for (u0, u1, *_rest) in p["blocks"]]

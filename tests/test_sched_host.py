@@ -6,6 +6,10 @@ servers: a draft takes D of the GPU, a verification V of the link.  For n
 equal requests and R rounds the two policies have closed forms:
   lock-step: every round is n drafts then n verifications -> R * n * (D + V)
   stagger  : link-bound (V >= D): D + R * n * V; GPU-bound: R * n * D + V
+Remote prefix caching adds a fetch per request on a third one-at-a-time
+server (the remote link), all fetches enqueued at the start in request
+order; lock-step starts drafting only after every fetch, stagger as soon as
+the request's own fetch is done.
 """
 
 import ctypes
@@ -106,3 +110,42 @@ def test_invalid_arguments_are_refused_before_any_device_call():
     sh2 = vc.shape(1, 4, 2, 96)
     assert L.vc_verify_attn_workspace_size(ctypes.byref(sh2), 100, 4) == 0
     assert L.vc_accept(16, 0, 1, 65, 10, 16, 16, 16, 16, 16, 1 << 20, None) == vc.VC_ERR_INVALID_ARG
+
+
+def test_fetch_closed_forms_two_requests():
+    # fetches 0-10 and 10-20; stagger: request 0 drafts 10-11, verifies 11-16,
+    # request 1 drafts 20-21, verifies 21-26; lock-step: drafts 20-22, then
+    # verifications 22-27 and 27-32
+    f, d, v = [10.0, 10.0], [1.0, 1.0], [5.0, 5.0]
+    assert vc.vc_sched_simulate(d, v, 1, vc.VC_SCHED_STAGGER, fetch_ms=f) == pytest.approx(26.0)
+    assert vc.vc_sched_simulate(d, v, 1, vc.VC_SCHED_LOCKSTEP, fetch_ms=f) == pytest.approx(32.0)
+
+
+@pytest.mark.parametrize("n,R,F,D,V", [(4, 3, 40.0, 2.0, 10.0), (3, 2, 100.0, 5.0, 20.0)])
+def test_fetch_bound_closed_forms(n, R, F, D, V):
+    # the remote link dominates (F >= R * (D + V)): with stagger, every request's
+    # rounds run while the next fetch is on the link, so only the last
+    # request's rounds extend past the fetches
+    assert F >= R * (D + V)
+    f, d, v = [F] * n, [D] * n, [V] * n
+    assert vc.vc_sched_simulate(d, v, R, vc.VC_SCHED_STAGGER, fetch_ms=f) == pytest.approx(n * F + R * (D + V))
+    assert vc.vc_sched_simulate(d, v, R, vc.VC_SCHED_LOCKSTEP, fetch_ms=f) == pytest.approx(n * F + R * n * (D + V))
+
+
+def test_fetch_stagger_never_slower_and_no_fetch_changes_nothing():
+    rng = random.Random(1)
+    for _ in range(200):
+        n = rng.randint(1, 5)
+        R = rng.randint(1, 3)
+        f = [rng.uniform(0.0, 40) for _ in range(n)]
+        d = [rng.uniform(0.5, 20) for _ in range(n)]
+        v = [rng.uniform(0.5, 20) for _ in range(n)]
+        lock = vc.vc_sched_simulate(d, v, R, vc.VC_SCHED_LOCKSTEP, fetch_ms=f)
+        stag = vc.vc_sched_simulate(d, v, R, vc.VC_SCHED_STAGGER, fetch_ms=f)
+        assert stag <= lock + 1e-9
+        # the remote link and the last request's own chain bound it from below
+        assert stag >= sum(f) - 1e-9
+        assert stag >= max(R * sum(d), R * sum(v)) - 1e-9
+        for pol in (vc.VC_SCHED_LOCKSTEP, vc.VC_SCHED_STAGGER):
+            assert vc.vc_sched_simulate(d, v, R, pol, fetch_ms=[0.0] * n) == pytest.approx(
+                vc.vc_sched_simulate(d, v, R, pol))
