@@ -73,6 +73,28 @@ __device__ __forceinline__ void take_later(Best& b, float x, int i) {
   }
 }
 
+// Largest of a 16-byte vector of logits, NaN if any is NaN (max.NaN).
+__device__ __forceinline__ float max_nan_f32(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t max_nan_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <typename T>
+__device__ __forceinline__ float vec_max(uint4 w) {
+  if constexpr (sizeof(T) == 4) {
+    return max_nan_f32(max_nan_f32(__uint_as_float(w.x), __uint_as_float(w.y)),
+                       max_nan_f32(__uint_as_float(w.z), __uint_as_float(w.w)));
+  } else {
+    const uint32_t m = max_nan_bf16x2(max_nan_bf16x2(w.x, w.y), max_nan_bf16x2(w.z, w.w));
+    return max_nan_f32(__uint_as_float(m << 16), __uint_as_float(m & 0xffff0000u));  // bf16 -> fp32 is a shift
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ void take_vec(Best& b, uint4 w, int base) {
   if constexpr (sizeof(T) == 4) {
@@ -124,7 +146,16 @@ __global__ void __launch_bounds__(kAcceptThreads) accept_kernel(const T* __restr
   const int a = v0 + head;
   const int nvec = (v1 - a) / VEC;
   if (threadIdx.x < head) take_later(b, to_f32(p[v0 + threadIdx.x]), v0 + threadIdx.x);
-  // kAcceptInFlight independent 16-byte loads per thread before any is used
+  // Vector body, two passes over the thread's own vectors: (1) the running
+  // maximum of whole vectors (max.NaN, a few instructions per 16 bytes) and
+  // the first vector that reached it -- a later vector replaces it only if
+  // its maximum is strictly larger or a NaN over a number, so ties keep the
+  // earlier vector; (2) that one vector is read again (from L2) and its
+  // first element equal to the maximum (or its first NaN) is the thread's
+  // candidate.  kAcceptInFlight independent loads per thread before any is
+  // used.
+  float vrun = -INFINITY;
+  int vbest = -1;  // element index of the vector holding vrun first
   for (int j0 = threadIdx.x; j0 < nvec; j0 += kAcceptInFlight * kAcceptThreads) {
     uint4 x[kAcceptInFlight];
 #pragma unroll
@@ -135,8 +166,19 @@ __global__ void __launch_bounds__(kAcceptThreads) accept_kernel(const T* __restr
 #pragma unroll
     for (int f = 0; f < kAcceptInFlight; ++f) {
       const int j = j0 + f * kAcceptThreads;
-      if (j < nvec) take_vec<T>(b, x[f], a + j * VEC);
+      if (j < nvec) {
+        const float m = vec_max<T>(x[f]);
+        if (vbest < 0 || m > vrun || (m != m && vrun == vrun)) {
+          vrun = m;
+          vbest = a + j * VEC;
+        }
+      }
     }
+  }
+  if (vbest >= 0) {
+    Best vb{-INFINITY, INT_MAX};
+    take_vec<T>(vb, *reinterpret_cast<const uint4*>(p + vbest), vbest);
+    take_later(b, vb.v, vb.i);
   }
   for (int t = a + nvec * VEC + threadIdx.x; t < v1; t += kAcceptThreads) take_later(b, to_f32(p[t]), t);
 
@@ -185,12 +227,31 @@ struct AcceptPlan {
   size_t off_row, off_req, off_part, total;
 };
 
+// Resident accept blocks per SM (cached per device).
+int accept_occupancy() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, accept_kernel<__nv_bfloat16>, kAcceptThreads, 0) !=
+            cudaSuccess ||
+        n < 1)
+      n = 1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 AcceptPlan plan_accept(int B, int K, int V) {
   AcceptPlan pl{};
-  // about one wave of blocks (4 blocks of 512 threads per SM), no chunk shorter than 8 loads per thread
+  // at most one wave of blocks: S chunks per row with rows * S <= SMs x
+  // resident blocks (a partial second wave would double the time of its
+  // blocks), no chunk shorter than 8 loads per thread
   const int64_t nrows = static_cast<int64_t>(B) * (K + 1);
-  const int64_t wave = 4 * static_cast<int64_t>(sm_count());
-  int64_t S = (wave + nrows - 1) / nrows;
+  const int64_t wave = static_cast<int64_t>(accept_occupancy()) * sm_count();
+  int64_t S = wave / nrows;
   const int64_t smax = (V + 8 * kAcceptThreads - 1) / (8 * kAcceptThreads);
   if (S > smax) S = smax;
   if (S > kAcceptMaxSplit) S = kAcceptMaxSplit;
