@@ -58,6 +58,10 @@ WORKLOADS = {
     "llama-70b-4x131k-4bit-stagger": dict(kind="stagger", NL=80, B=1, n_req=4, Hq=64, Hkv=8, D=128, T=131072,
                                           bits=4, G=64, R=128, K=30, V=128256, logits="bf16", p_mismatch=0.2,
                                           host_pool=2),
+    # the verification pass through 32 decoder layers with random bf16 weights (Llama-3.1-8B dimensions),
+    # full KV resident: tokens verified per second, comparable only in kind (no trained weights)
+    "llama-3.1-8b-32k-layers-verify": dict(kind="layers", NL=32, B=8, Hq=32, Hkv=8, D=128, T=32768, K=30,
+                                           d_model=4096, d_ff=14336, V=128256),
     # remote prefix caching: each request's compressed prefix cache arrives over an emulated 1.2 GB/s remote
     # link, its full cache is streamed for verification over an emulated 40 GB/s local link
     "llama-3.1-8b-4x32k-kivi2-remote-prefix": dict(kind="remote", NL=32, B=1, n_req=4, Hq=32, Hkv=8, D=128,
@@ -823,6 +827,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama-3.1-8b-32k-kivi2", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--kernel", default="", choices=["", "draft", "verify", "accept"],
+                    help="time one kernel of the workload alone (a per-kernel line for profiler captures; "
+                         "not the benchmark line)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small cases for profiler captures; 0 = the workload's)")
     args = ap.parse_args()
@@ -844,15 +851,22 @@ def main():
         config.update(bits=w["bits"], group=w["G"], residual=w["R"])
     if "n_keep" in w:
         config.update(kept_per_head=w["n_keep"], kept_row_pool="idx = pool slots 0..n_keep-1")
-    if w["kind"] != "resident" or w.get("streamed_too"):
+    if w["kind"] not in ("resident", "layers") or w.get("streamed_too"):
         config.update(full_kv="pinned host memory, streamed per layer",
                       host_pool_layers=w.get("host_pool", 2))
     if w["kind"] in ("stagger", "remote"):
         config.update(requests=w["n_req"])
+    if w["kind"] == "layers":
+        config.update(full_kv="resident in HBM", d_model=w["d_model"], d_ff=w["d_ff"],
+                      weights="random bf16 (no trained weights)")
     if w["kind"] == "remote":
         config.update(full_kv="pinned host memory, streamed per layer over the emulated local link",
                       draft_cache="pinned host memory, fetched over the emulated remote link",
                       remote_gbps=w["remote_gbps"], local_gbps=w["local_gbps"])
+
+    if args.kernel:
+        print(json.dumps(kernel_line(args, w, peak, peak_kind)), flush=True)
+        return
 
     if args.impl == "reference":
         if rank != 0:
@@ -885,6 +899,8 @@ def main():
         line = stagger_line(args, w, rank, world, config, peak, peak_kind)
     elif w["kind"] == "remote":
         line = remote_line(args, w, rank, world, config, peak, peak_kind)
+    elif w["kind"] == "layers":
+        line = layers_line(args, w, rank, world, config, peak, peak_kind)
     else:
         line = resident_line(args, w, rank, world, config, peak, peak_kind)
     if rank == 0:
@@ -899,6 +915,83 @@ def _common(args, config, value, peak, peak_kind, r, dtype):
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": dtype, "data": "synthetic (seeded random KV, queries and logits; no model weights)",
             "config": config, "clocks": r["clocks"]}
+
+
+def kernel_line(args, w, peak, peak_kind):
+    """One kernel of the workload timed alone with CUDA events: the quantised
+    or token-dropped draft attention of one layer, one resident
+    verification layer, or one acceptance call over the round's logits."""
+    import torch
+    from lossless_draft_verify_vc_b200 import synth, vc
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    vc.lib()
+    B = w["B"]
+    reps = max(args.steps, 3) * 10
+    comp = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if args.kernel == "verify":
+        rv = time_resident_verify_layer(w, dev, reps=reps)
+        return {"kernel": "vc_verify_attn", "workload": args.workload, "us": rv["us_per_layer"],
+                "gbps": rv["hbm_gbps"], "frac_of_hbm_peak": rv["hbm_gbps"] / peak, "tflops": rv["tflops"],
+                "peak_kind": peak_kind, "calls": reps}
+    if args.kernel == "accept":
+        K, V = w["K"], w["V"]
+        dt = torch.bfloat16 if w["logits"] == "bf16" else torch.float32
+        toks = synth.tokens((B, K), V, seed=3)
+        lens = synth.geometric_accept_lengths(B, K, w["p_mismatch"], seed=3)
+        lg = [synth.planted_logits(B, K, V, toks, lens, seed=4 + i, dtype=dt).to(dev) for i in range(4)]
+        d = toks.to(dev)
+        tgt = torch.empty(B, K + 1, dtype=torch.int32, device=dev)
+        acc = torch.empty(B, dtype=torch.int32, device=dev)
+        cor = torch.empty_like(acc)
+        ws = vc.workspace(vc.vc_accept_workspace_size(B, K, V), dev)
+        for i in range(5):
+            vc.vc_accept(lg[i % 4], B, K, V, d, tgt, acc, cor, ws, comp)
+        torch.cuda.synchronize(dev)
+        assert acc.cpu().tolist() == lens
+        e0.record(comp)
+        for i in range(reps):
+            vc.vc_accept(lg[i % 4], B, K, V, d, tgt, acc, cor, ws, comp)
+        e1.record(comp)
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        nb = B * (K + 1) * V * lg[0].element_size()
+        return {"kernel": "vc_accept", "workload": args.workload, "us": us, "gbps": nb / us / 1e3,
+                "frac_of_hbm_peak": nb / us / 1e3 / peak, "peak_kind": peak_kind, "calls": reps}
+    # draft attention of one layer
+    nl = 3
+    sh = vc.shape(B, w["Hq"], w["Hkv"], w["D"])
+    q = synth.normal((nl, B, w["Hq"], w["D"]), 7, dev)
+    out = torch.empty(B, w["Hq"], w["D"], device=dev)
+    if "bits" in w:
+        caches = [vc.quant_cache(synth.random_quant_cache(B, w["Hkv"], w["T"] - w["R"], w["R"], w["D"], w["bits"],
+                                                          w["G"], seed=l, device=dev)) for l in range(nl)]
+        ws = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, caches[0]), dev)
+        call = lambda i: vc.vc_draft_attn_quant(sh, caches[i % nl], q[i % nl], out, ws, comp)
+        nb, name = draft_bytes_per_layer(w), "vc_draft_attn_quant"
+    else:
+        keep = []
+        caches = []
+        for l in range(nl):
+            k, v = synth.kv_full(B, w["Hkv"], w["n_keep"], w["D"], seed=40 + l, device=dev)
+            idx = torch.arange(w["n_keep"], dtype=torch.int32, device=dev).expand(B, w["Hkv"], -1).contiguous()
+            keep.append((k, v, idx))
+            caches.append(vc.sparse_cache(k, v, idx))
+        ws = vc.workspace(vc.vc_draft_attn_sparse_workspace_size(sh, caches[0]), dev)
+        call = lambda i: vc.vc_draft_attn_sparse(sh, caches[i % nl], q[i % nl], out, ws, comp)
+        nb, name = sparse_bytes_per_layer(w), "vc_draft_attn_sparse"
+    for i in range(6):
+        call(i)
+    torch.cuda.synchronize(dev)
+    e0.record(comp)
+    for i in range(reps):
+        call(i)
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    return {"kernel": name, "workload": args.workload, "us": us, "gbps": nb / us / 1e3,
+            "frac_of_hbm_peak": nb / us / 1e3 / peak, "peak_kind": peak_kind, "calls": reps}
 
 
 def resident_verify_block(w, peak, peak_kind):
@@ -1011,6 +1104,74 @@ def remote_line(args, w, rank, world, config, peak, peak_kind):
                      "frac": achieved / peak, "traffic": None, "algorithmic_bytes_per_launch": db},
         # the timed draft loop: K * NL draft kernels
         "gpu_launches": K * NL,
+    })
+    return line
+
+
+def layers_line(args, w, rank, world, config, peak, peak_kind):
+    """The verification pass through NL decoder layers (vc_verify_layer) on
+    random bf16 weights with the full KV resident: each layer reads its
+    weights and its full K and V once."""
+    import torch
+    from lossless_draft_verify_vc_b200 import synth, vc
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    vc.lib()
+    NL, B, Hq, Hkv, D, T, dm, dff = w["NL"], w["B"], w["Hq"], w["Hkv"], w["D"], w["T"], w["d_model"], w["d_ff"]
+    nq = w["K"] + 1
+    ls = vc.layer_shape(dm, dff, Hq, Hkv, D)
+    g = torch.Generator(device=dev).manual_seed(1000 * rank + 5)
+
+    def r(shape, s):
+        return (torch.randn(shape, generator=g, device=dev) * s).to(torch.bfloat16)
+
+    layers = []
+    for _ in range(NL):
+        W = dict(w1=(1 + 0.1 * torch.randn(dm, generator=g, device=dev)).to(torch.bfloat16),
+                 w2=(1 + 0.1 * torch.randn(dm, generator=g, device=dev)).to(torch.bfloat16),
+                 wqkv=r(((Hq + 2 * Hkv) * D, dm), dm ** -0.5), wo=r((dm, Hq * D), (Hq * D) ** -0.5),
+                 wgu=r((2 * dff, dm), dm ** -0.5), wd=r((dm, dff), dff ** -0.5))
+        k, v = synth.kv_full(B, Hkv, T, D, seed=len(layers), device=dev)
+        layers.append((vc.layer_weights(W), W, k, v))
+    x0 = synth.normal((B, nq, dm), 3, dev)
+    x = x0.clone()
+    ws = vc.workspace(vc.vc_verify_layer_workspace_size(ls, B, nq, T), dev)
+    comp = torch.cuda.current_stream(dev)
+
+    def one_pass():
+        x.copy_(x0)
+        for lw, _, k, v in layers:
+            vc.vc_verify_layer(ls, lw, B, nq, T, x, k, v, ws, comp)
+
+    for _ in range(args.warmup):
+        one_pass()
+    torch.cuda.synchronize(dev)
+    assert torch.isfinite(x.float()).all()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for _ in range(args.steps):
+        one_pass()
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0] / args.steps
+    wbytes = sum(t.numel() * t.element_size() for _, W, _, _ in layers for t in W.values())
+    kvbytes = NL * 4 * T * Hkv * D * B
+    value = (wbytes + kvbytes) * world / (ms * 1e-3) / 1e9
+    line = _common(args, config, value, peak, peak_kind, dict(clocks=clk), "bf16 weights and KV, fp32 accumulate")
+    line.update({
+        "ms_per_step": ms,
+        "note": "value = weight + full-KV bytes read per verification pass / pass time (GB/s); random weights, "
+                "so tokens/s are comparable only in kind",
+        "verify_pass": {"ms": ms, "tokens_verified_per_s": B * nq * world / (ms * 1e-3),
+                        "weight_bytes": wbytes, "kv_bytes": kvbytes, "frac_of_hbm_peak": value / world / peak,
+                        "layers": NL, "rows_per_request": nq},
+        # per layer: 2 norms, rotary, attention + combine, convert, SwiGLU (+ 4 cuBLAS GEMMs)
+        "gpu_launches": NL * 7 * args.steps,
     })
     return line
 

@@ -359,6 +359,41 @@ VC_API vc_status vc_kvstream_acquire(vc_kvstream* s, int layer, void* compute_st
 VC_API vc_status vc_kvstream_release(vc_kvstream* s, int layer, void* compute_stream);
 VC_API vc_status vc_kvstream_destroy(vc_kvstream* s);
 
+/* ---- one verifier decoder layer on caller-given weights --------------------
+ * Verification is one pass of the same model over the drafted block with the
+ * full cache (devshah.ca page, "The Core Idea"; drafter and verifier share
+ * the weights, menfem.com source page, "Methodology").  vc_verify_layer runs
+ * one Llama-style pre-norm decoder layer over the block:
+ *   h = RMSNorm(x) w1; [q | k | v] = h Wqkv^T; rotary embedding (rotate-half
+ *   pairs j, j + D/2, angle = position * rope_theta^(-2j/D)) of q and k at
+ *   positions T - nq + i; the block's k and v written into the full cache
+ *   rows T - nq .. T - 1; o = vc_verify_attn; x += o Wo^T;
+ *   h2 = RMSNorm(x) w2; [g | u] = h2 Wgu^T; x += (silu(g) u) Wd^T.
+ * Activations are bf16 between the steps (each step's result is rounded to
+ * bf16 once); the projections are cuBLAS bf16 GEMMs with fp32 accumulation.
+ *   x        bf16 [B][nq][d_model], read and overwritten with the layer output
+ *   k_cache, v_cache  bf16 [B][Hkv][T][D] (full cache, resident); rows
+ *            T - nq .. T - 1 are overwritten with the block's k and v
+ *   weights  bf16 row-major [out][in]: w1, w2 [d_model]; wqkv
+ *            [(Hq + 2 Hkv) D][d_model]; wo [d_model][Hq D]; wgu
+ *            [2 d_ff][d_model] (gate rows, then up rows); wd [d_model][d_ff]
+ * D in {64, 128}, Hq/Hkv <= 8, nq <= 32, d_model and d_ff multiples of 8,
+ * every pointer 16-byte aligned.  The workspace (size from the query) also
+ * holds cuBLAS's scratch.  Returns VC_ERR_INVALID_ARG on bad arguments
+ * before any launch. */
+typedef struct vc_layer_shape {
+  int d_model, d_ff, Hq, Hkv, D;
+  float rms_eps;     /* e.g. 1e-5 */
+  float rope_theta;  /* e.g. 500000 */
+} vc_layer_shape;
+typedef struct vc_layer_weights {
+  const void *w1, *wqkv, *wo, *w2, *wgu, *wd;
+} vc_layer_weights;
+VC_API size_t vc_verify_layer_workspace_size(const vc_layer_shape* shape, int B, int nq, int64_t T);
+VC_API vc_status vc_verify_layer(const vc_layer_shape* shape, const vc_layer_weights* weights, int B, int nq,
+                                 int64_t T, void* x, void* k_cache, void* v_cache, void* ws, size_t ws_bytes,
+                                 void* stream);
+
 /* ---- bandwidth-limited links ---------------------------------------------------
  * Remote prefix caching sends the compressed cache to the serving GPU over a
  * slow network while the full cache stays reachable over a fast local link

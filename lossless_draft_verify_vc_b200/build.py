@@ -69,7 +69,7 @@ def build(verbose: bool = False, extra_flags=None) -> str:
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         list(ex.map(run, jobs))
     if jobs or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        run([nvcc, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart", "-lcuda"])
+        run([nvcc, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart", "-lcuda", "-lcublas"])
     return LIB
 
 

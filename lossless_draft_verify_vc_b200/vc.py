@@ -69,6 +69,16 @@ class vc_sched_stats(Structure):
                 ("fetch_ms", ctypes.c_double), ("first_draft_ms", ctypes.c_double)]
 
 
+class vc_layer_shape(Structure):
+    _fields_ = [("d_model", c_int), ("d_ff", c_int), ("Hq", c_int), ("Hkv", c_int), ("D", c_int),
+                ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float)]
+
+
+class vc_layer_weights(Structure):
+    _fields_ = [("w1", c_void_p), ("wqkv", c_void_p), ("wo", c_void_p), ("w2", c_void_p), ("wgu", c_void_p),
+                ("wd", c_void_p)]
+
+
 VC_DRAFT_QUANT, VC_DRAFT_SPARSE = 0, 1
 VC_SCHED_LOCKSTEP, VC_SCHED_STAGGER = 0, 1
 
@@ -129,6 +139,9 @@ def lib() -> ctypes.CDLL:
             "vc_sched_set_links": (c_int, [c_void_p, c_void_p, ctypes.c_double, ctypes.c_double, c_size_t]),
             "vc_sched_set_fetch": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
             "vc_link_create": (c_int, [P(c_void_p), c_void_p, ctypes.c_double, c_size_t]),
+            "vc_verify_layer_workspace_size": (c_size_t, [P(vc_layer_shape), c_int, c_int, c_int64]),
+            "vc_verify_layer": (c_int, [P(vc_layer_shape), P(vc_layer_weights), c_int, c_int, c_int64, c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
             "vc_link_copy": (c_int, [c_void_p, c_void_p, c_void_p, c_size_t]),
             "vc_link_flags": (c_int, [c_void_p, P(c_uint32)]),
             "vc_link_destroy": (c_int, [c_void_p]),
@@ -499,3 +512,27 @@ class Link:
             self.close()
         except Exception:
             pass
+
+
+# ---- one verifier decoder layer ------------------------------------------------------
+
+def layer_shape(d_model: int, d_ff: int, Hq: int, Hkv: int, D: int, rms_eps: float = 1e-5,
+                rope_theta: float = 500000.0) -> vc_layer_shape:
+    return vc_layer_shape(d_model, d_ff, Hq, Hkv, D, rms_eps, rope_theta)
+
+
+def layer_weights(w: dict) -> vc_layer_weights:
+    """Descriptor of a layer's bf16 weights given as a dict of CUDA tensors
+    w1, wqkv, wo, w2, wgu, wd (keeps references to them)."""
+    d = vc_layer_weights(*[_p(w[k]) for k in ("w1", "wqkv", "wo", "w2", "wgu", "wd")])
+    d._keep = w
+    return d
+
+
+def vc_verify_layer_workspace_size(ls, B: int, nq: int, T: int) -> int:
+    return lib().vc_verify_layer_workspace_size(ctypes.byref(ls), int(B), int(nq), int(T))
+
+
+def vc_verify_layer(ls, lw, B: int, nq: int, T: int, x, k_cache, v_cache, ws, stream=None):
+    _check(lib().vc_verify_layer(ctypes.byref(ls), ctypes.byref(lw), int(B), int(nq), int(T), _p(x), _p(k_cache),
+                                 _p(v_cache), _p(ws), ws.numel(), _stream(stream)))

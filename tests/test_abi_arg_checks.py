@@ -207,6 +207,24 @@ def test_link_and_remote_fetch_calls_reject_null_objects(L):
     _expect_invalid(L, L.vc_sched_set_fetch(None, 0, 0, None, None, None), "vc_sched_set_fetch")
 
 
+@pytest.mark.parametrize("shape,B,nq,T,wnull,x", [
+    ((256, 512, 8, 2, 96), 1, 4, 100, False, A),     # head dim
+    ((256, 512, 6, 4, 64), 1, 4, 100, False, A),     # Hq not a multiple of Hkv
+    ((250, 512, 8, 2, 64), 1, 4, 100, False, A),     # d_model not a multiple of 8
+    ((256, 512, 8, 2, 64), 1, 33, 100, False, A),    # nq > 32
+    ((256, 512, 8, 2, 64), 1, 4, 3, False, A),       # T < nq
+    ((256, 512, 8, 2, 64), 1, 4, 100, True, A),      # a null weight
+    ((256, 512, 8, 2, 64), 1, 4, 100, False, M),     # misaligned x
+])
+def test_verify_layer_rejects_before_any_launch(L, shape, B, nq, T, wnull, x):
+    ls = vc.layer_shape(*shape)
+    lw = vc.vc_layer_weights(*([A] * 6))
+    if wnull:
+        lw.wo = None
+    st = L.vc_verify_layer(ctypes.byref(ls), ctypes.byref(lw), B, nq, T, x, A, A, A, WS, None)
+    _expect_invalid(L, st, "vc_verify_layer")
+
+
 def test_wait_timeout_export_rejects_before_any_launch(L):
     # null pointers and limits outside 1 us .. 100 ms are refused on the host
     assert L.vc_debug_wait_timeout(None, 16, 1000000, None) == vc.VC_ERR_INVALID_ARG
