@@ -389,10 +389,20 @@ vc_status vc_draft_attn_sparse(const vc_attn_shape* shape, const vc_sparse_cache
   if (pl.S > 1) {  // chunk partials -> output rows
     const vc::SparseRowMap map{a.g, shape->Hq, shape->Hkv, shape->D};
     const int64_t n_rows = static_cast<int64_t>(shape->B) * shape->Hkv * a.g;
-    if (shape->D == 128)
-      vc::launch_splitk_combine<128>(a.o, pl.S, a.g, n_rows, map, s);
-    else
-      vc::launch_splitk_combine<64>(a.o, pl.S, a.g, n_rows, map, s);
+    // tens of chunks per row: one block per row keeps each thread's loads
+    // few and independent (one warp per row above kWideMaxS chunks)
+    const bool wide = pl.S >= 16 && pl.S <= vc::kWideMaxS;
+    if (shape->D == 128) {
+      if (wide)
+        vc::launch_splitk_combine_wide<128>(a.o, pl.S, a.g, n_rows, map, s);
+      else
+        vc::launch_splitk_combine<128>(a.o, pl.S, a.g, n_rows, map, s);
+    } else {
+      if (wide)
+        vc::launch_splitk_combine_wide<64>(a.o, pl.S, a.g, n_rows, map, s);
+      else
+        vc::launch_splitk_combine<64>(a.o, pl.S, a.g, n_rows, map, s);
+    }
   }
   return vc::launch_status("vc_draft_attn_sparse");
 }

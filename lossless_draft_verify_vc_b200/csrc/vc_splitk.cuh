@@ -2,7 +2,9 @@
 // in-block merge of per-warp online-softmax states into a per-chunk partial
 // (splitk_store; the token-dropped draft -- verification stores its one
 // state per row straight from tensor memory), and the cross-chunk merge as a
-// separate launch with one warp per output row (splitk_combine_kernel; both).
+// separate launch with one warp per output row (splitk_combine_kernel; both)
+// or, for many chunks and few rows, one block per row
+// (splitk_combine_wide_kernel; the token-dropped draft).
 //
 // A partial of one (unit, chunk) holds, per query row r < rows:
 //   o[r][0..D)  unnormalised sum_j 2^(s_j - m) v_j
@@ -139,6 +141,80 @@ __global__ void __launch_bounds__(128) splitk_combine_kernel(SplitKOut o, int S,
   if (o.lse && lane == 0) o.lse[lse_off] = lse_from(M, L);
 }
 
+// Cross-chunk merge for many chunks and few rows (the token-dropped draft:
+// g rows per unit, tens of chunks): one 256-thread block per output row.
+// The chunks' (m, l) are reduced by all threads at once; each of 8 warps
+// then sums every 8th chunk's o (lane l owns channels D/32 l ..), so a
+// thread keeps ~S/8 independent loads in flight instead of S, and the 8
+// warp sums meet in shared memory.  S <= kWideMaxS.
+constexpr int kWideMaxS = 2048;
+
+template <int D, typename Map>
+__global__ void __launch_bounds__(256) splitk_combine_wide_kernel(SplitKOut o, int S, int rows_cap, int64_t n_rows,
+                                                                  Map map) {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  constexpr int PER = D / 32;
+  __shared__ float wts[kWideMaxS];
+  __shared__ float red[8][D];
+  __shared__ float ml[2][8];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t fr = blockIdx.x;
+  int unit, r;
+  size_t out_off, lse_off;
+  if (fr >= n_rows || !map.locate(fr, unit, r, out_off, lse_off)) return;  // block-uniform
+  const size_t stride_ml = static_cast<size_t>(rows_cap) * 2;
+  const float* pml = o.part_ml + static_cast<size_t>(unit) * S * stride_ml + 2 * r;
+  float m = -INFINITY;
+  for (int s = tid; s < S; s += 256) m = fmaxf(m, __ldcg(pml + s * stride_ml));
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, x));
+  if (lane == 0) ml[0][warp] = m;
+  __syncthreads();
+  float M = ml[0][0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) M = fmaxf(M, ml[0][w]);
+  float l = 0.f;
+  for (int s = tid; s < S; s += 256) {
+    const float ms = __ldcg(pml + s * stride_ml);
+    const float w = (ms == -INFINITY || M == -INFINITY) ? 0.f : ex2(ms - M);
+    wts[s] = w;
+    if (w > 0.f) l += w * __ldcg(pml + s * stride_ml + 1);
+  }
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) l += __shfl_xor_sync(0xffffffffu, l, x);
+  if (lane == 0) ml[1][warp] = l;
+  __syncthreads();
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) L += ml[1][w];
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  const float* po = o.part_o + (static_cast<size_t>(unit) * S * rows_cap + r) * D + lane * PER;
+#pragma unroll 8
+  for (int s = warp; s < S; s += 8) {
+    const float w = wts[s];
+    const float* src = po + static_cast<size_t>(s) * rows_cap * D;
+    if constexpr (PER == 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+      acc[0] += w * v.x, acc[1] += w * v.y, acc[2] += w * v.z, acc[3] += w * v.w;
+    } else {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+      acc[0] += w * v.x, acc[1] += w * v.y;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) red[warp][lane * PER + i] = acc[i];
+  __syncthreads();
+  if (tid < D) {
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += red[w][tid];
+    o.out[out_off + tid] = L > 0.f ? sum / L : 0.f;
+  }
+  if (o.lse && tid == 0) o.lse[lse_off] = lse_from(M, L);
+}
+
 // Host: launches splitk_combine_kernel<D> as a programmatic dependent of the
 // kernel just enqueued on s.
 template <int D, typename Map>
@@ -155,6 +231,23 @@ inline void launch_splitk_combine(const SplitKOut& o, int S, int rows_cap, int64
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaLaunchKernelEx(&cfg, splitk_combine_kernel<D, Map>, o, S, rows_cap, n_rows, map);
+}
+
+// Host: the wide merge (one block per row) as a programmatic dependent.
+template <int D, typename Map>
+inline void launch_splitk_combine_wide(const SplitKOut& o, int S, int rows_cap, int64_t n_rows, const Map& map,
+                                       cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_rows));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, splitk_combine_wide_kernel<D, Map>, o, S, rows_cap, n_rows, map);
 }
 
 }  // namespace vc
