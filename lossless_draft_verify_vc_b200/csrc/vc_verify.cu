@@ -676,10 +676,19 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
     const int rows_cap = p.nqt * a.g;
     const vc::VerifyRowMap map{rows_cap, p.RT, shape->Hkv, nq, p.nqt, a.g, shape->Hq, shape->D};
     const int64_t n_rows = static_cast<int64_t>(units) * p.RT * rows_cap;
-    if (shape->D == 128)
-      vc::launch_splitk_combine<128>(a.o, p.C, rows_cap, n_rows, map, s);
-    else
-      vc::launch_splitk_combine<64>(a.o, p.C, rows_cap, n_rows, map, s);
+    // many chunks (long contexts, few units): one block per row
+    const bool wide = p.C >= 16 && p.C <= vc::kWideMaxS;
+    if (shape->D == 128) {
+      if (wide)
+        vc::launch_splitk_combine_wide<128>(a.o, p.C, rows_cap, n_rows, map, s);
+      else
+        vc::launch_splitk_combine<128>(a.o, p.C, rows_cap, n_rows, map, s);
+    } else {
+      if (wide)
+        vc::launch_splitk_combine_wide<64>(a.o, p.C, rows_cap, n_rows, map, s);
+      else
+        vc::launch_splitk_combine<64>(a.o, p.C, rows_cap, n_rows, map, s);
+    }
   }
   return vc::launch_status("vc_verify_attn");
 }
