@@ -317,6 +317,10 @@ def build_inputs(w, dev, rank):
     ldt = torch.bfloat16 if w["logits"] == "bf16" else torch.float32
     logits = synth.planted_logits(B, K, w["V"], draft_tok.cpu(), lens, seed0 + 4, device="cpu", dtype=ldt).to(dev)
     sh = vc.shape(B, Hq, Hkv, D)
+    # the draft caches are written once before the loop and never by a kernel
+    # of the step: the draft kernel may start copying records early
+    for c in caches:
+        c["flags"] = vc.VC_CACHE_STATIC
     qcs = [vc.quant_cache(c) for c in caches]
     return dict(caches=caches, kvs=kvs, q_draft=q_draft, q_ver=q_ver, draft_tok=draft_tok, logits=logits,
                 lens=lens, sh=sh, qcs=qcs)
@@ -965,8 +969,9 @@ def kernel_line(args, w, peak, peak_kind):
     q = synth.normal((nl, B, w["Hq"], w["D"]), 7, dev)
     out = torch.empty(B, w["Hq"], w["D"], device=dev)
     if "bits" in w:
-        caches = [vc.quant_cache(synth.random_quant_cache(B, w["Hkv"], w["T"] - w["R"], w["R"], w["D"], w["bits"],
-                                                          w["G"], seed=l, device=dev)) for l in range(nl)]
+        caches = [vc.quant_cache(dict(synth.random_quant_cache(B, w["Hkv"], w["T"] - w["R"], w["R"], w["D"],
+                                                               w["bits"], w["G"], seed=l, device=dev),
+                                      flags=vc.VC_CACHE_STATIC)) for l in range(nl)]
         ws = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, caches[0]), dev)
         call = lambda i: vc.vc_draft_attn_quant(sh, caches[i % nl], q[i % nl], out, ws, comp)
         nb, name = draft_bytes_per_layer(w), "vc_draft_attn_quant"

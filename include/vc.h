@@ -170,7 +170,14 @@ typedef struct vc_quant_cache {
    * lens[b] = (L_q_b, R_b) with L_q_b a multiple of group, L_q_b <= L_q and
    * R_b <= R_cap.  NULL: every request has L_q and R. */
   const int32_t* lens;
+  /* VC_CACHE_STATIC: the records, residual rows and lens are not written by
+   * the kernel that precedes this call in the stream (e.g. the previous
+   * layer's draft call), so the draft kernel may start copying its first
+   * records before that kernel has finished.  0: it waits first (always
+   * safe; required right after vc_cache_commit or any other writer). */
+  int flags;
 } vc_quant_cache;
+#define VC_CACHE_STATIC 1
 
 /* One layer of a token-dropped draft cache: every (request, KV head) keeps
  * the same number n_keep of positions (the pages restrict the method to equal

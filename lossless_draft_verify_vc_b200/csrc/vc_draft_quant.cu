@@ -187,6 +187,7 @@ struct QArgs {
   uint32_t* flags;
   uint32_t* tickets;  // [U] partials of each unit written so far in this call (back to 0 after it)
   const int32_t* lens;  // optional [B][2] per-request (L_q, R); NULL: P.ng groups and R rows everywhere
+  int cache_flags;      // VC_CACHE_STATIC: the first stages may be fetched before the stream dependency
   float* part_o;      // [nblk * MAXS][g][D]
   float* part_ml;     // [nblk * MAXS][g][2]
   float* out;         // [B][Hq][D]
@@ -1248,22 +1249,41 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
   __syncwarp();
   int u0, u1, r0, r1, q0, q1;
   P.block_range(k, u0, u1, r0, r1, q0, q1);
-  // this warp's quantised stages: q0 + warp + kQNW i < q1 of every unit of the block
-  // (< the request's own stage count with per-request lengths)
-  // Launched as a programmatic dependent of the previous kernel in the
-  // stream: nothing global is read or written before that grid completed.
-  // The next kernel may then be scheduled as this grid's blocks retire (it
-  // waits the same way).
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-  int my_nq = 0;
-  if (q1 > q0)
-    for (int u = u0; u < u1; ++u) my_nq += warp_stage_count(q0 + warp, unit_qend<C>(a, u, q1));
   bool ok = true;
   int rph = 0;
   float* wml = st_ml + warp * C::HEADS * 2;
   const int64_t slot0 = static_cast<int64_t>(k) * 2 * P.upb;
-
+  // this warp's quantised stages: q0 + warp + kQNW i < q1 of every unit of the
+  // block (< the request's own stage count with per-request lengths)
+  WarpRing r;
+  int my_nq = 0;
+  auto prime = [&]() {
+    for (int u = u0; u < u1; ++u) my_nq += warp_stage_count(q0 + warp, unit_qend<C>(a, u, q1));
+    r.issued = 0, r.head = 0, r.tail = 0, r.hslot = 0, r.hphase = 0u;
+    r.q_first = q0 + warp, r.q_end = q1, r.u_end = u1;
+    int uf = u0;  // first unit where this warp has a stage
+    while (uf < u1 && warp_stage_count(q0 + warp, unit_qend<C>(a, uf, q1)) == 0) ++uf;
+    issue_start<C>(a, r.ip, uf < u1 ? uf : u0, q0 + warp, q1);
+    fence_proxy_async_smem();
+    __syncwarp();
+    while (r.issued < my_nq && r.issued < C::NST) {
+      issue_stage<C>(a, ring, bars, lane, r.issued, r.ip);
+      issue_advance<C>(a, r.ip, r.q_first, r.u_end, r.q_end);
+      ++r.issued;
+    }
+  };
+  // Launched as a programmatic dependent of the previous kernel in the
+  // stream: nothing global is read or written before that grid completed,
+  // except, when the caller declares the cache static (VC_CACHE_STATIC: the
+  // previous kernel does not write it), the first NST stages of group
+  // records of a block without residual tiles, whose copies then overlap the
+  // previous kernel's tail.  (A block with residual tiles stages them in its
+  // ring first and primes the ring after them.)  The next kernel may be
+  // scheduled as this grid's blocks retire (it waits the same way).
+  const bool early = (a.cache_flags & VC_CACHE_STATIC) != 0 && r1 <= r0;
+  if (early && q1 > q0) prime();
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   // residual tiles of each unit (the ring is not primed yet)
   if (r1 > r0) {
     for (int u = u0; u < u1; ++u) {
@@ -1275,22 +1295,9 @@ __global__ void __launch_bounds__(kQNW * 32, (NT == 1 ? 4 : 2)) draft_quant_kern
       unit_finish<D>(a, u, ma, s_flag);
     }
   }
+  if (!early && q1 > q0) prime();
+
   if (q1 > q0) {
-    WarpRing r;
-    r.issued = 0, r.head = 0, r.tail = 0, r.hslot = 0, r.hphase = 0u;
-    r.q_first = q0 + warp, r.q_end = q1, r.u_end = u1;
-    {
-      int uf = u0;  // first unit where this warp has a stage
-      while (uf < u1 && warp_stage_count(q0 + warp, unit_qend<C>(a, uf, q1)) == 0) ++uf;
-      issue_start<C>(a, r.ip, uf < u1 ? uf : u0, q0 + warp, q1);
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    while (r.issued < my_nq && r.issued < C::NST) {
-      issue_stage<C>(a, ring, bars, lane, r.issued, r.ip);
-      issue_advance<C>(a, r.ip, r.q_first, r.u_end, r.q_end);
-      ++r.issued;
-    }
     uint4* q_sm = reinterpret_cast<uint4*>(smem + C::QSM_OFF);
     for (int u = u0; u < u1; ++u) {
       if constexpr (NT == 1) {  // the unit's query fragments, shared by the block's warps
@@ -1548,6 +1555,7 @@ QArgs make_args(const vc_attn_shape& sh, const vc_quant_cache& c, const void* q)
   a.R_cap = c.R_cap;
   a.group = c.group;
   a.lens = c.lens;
+  a.cache_flags = c.flags;
   a.Hq = sh.Hq;
   a.Hkv = sh.Hkv;
   a.g = sh.Hq / sh.Hkv;

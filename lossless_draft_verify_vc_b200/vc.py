@@ -44,7 +44,7 @@ class vc_attn_shape(Structure):
 class vc_quant_cache(Structure):
     _fields_ = [("records", c_void_p), ("k_res", c_void_p), ("v_res", c_void_p),
                 ("bits", c_int), ("group", c_int), ("L_q", c_int64), ("R", c_int), ("R_cap", c_int),
-                ("lens", c_void_p)]
+                ("lens", c_void_p), ("flags", c_int)]
 
 
 class vc_sparse_cache(Structure):
@@ -80,6 +80,7 @@ class vc_layer_weights(Structure):
 
 
 VC_DRAFT_QUANT, VC_DRAFT_SPARSE = 0, 1
+VC_CACHE_STATIC = 1
 VC_SCHED_LOCKSTEP, VC_SCHED_STAGGER = 0, 1
 
 _lib = None
@@ -188,11 +189,11 @@ def quant_cache(t: dict) -> vc_quant_cache:
     """Descriptor of a quantised cache given as a dict of CUDA tensors with the
     keys records, k_res, v_res and ints bits, group, L_q, R, R_cap, and an
     optional int32 tensor lens [B, 2] of per-request (L_q, R) (the layout
-    documented in vc.h).  The descriptor holds raw device pointers; it keeps
+    documented in vc.h) and optional int flags (VC_CACHE_STATIC).  The descriptor holds raw device pointers; it keeps
     references to the tensors so they stay allocated while it lives."""
     d = vc_quant_cache(_p(t["records"]), _p(t.get("k_res")), _p(t.get("v_res")),
                        int(t["bits"]), int(t["group"]), int(t["L_q"]), int(t["R"]), int(t["R_cap"]),
-                       _p(t.get("lens")))
+                       _p(t.get("lens")), int(t.get("flags", 0)))
     d._keep = dict(t)
     return d
 

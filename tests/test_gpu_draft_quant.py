@@ -111,3 +111,31 @@ def test_explicit_scale_and_repeat():
     vc.vc_draft_attn_quant(sh, vc.quant_cache(tc), q, out2, ws)
     torch.cuda.synchronize()
     assert np.array_equal(np32(out2), got)
+
+
+def test_static_cache_flag_changes_nothing_but_the_start():
+    """VC_CACHE_STATIC lets the kernel copy its first records before the
+    previous kernel of the stream ends; the results must be bit-identical to
+    the same calls without it, in a chain of back-to-back calls over
+    alternating caches (each call overlapping the previous one's tail)."""
+    B, Hq, Hkv, D, G, R = 3, 12, 3, 128, 32, 128
+    caches = []
+    for s_ in range(2):
+        k, v, cache = make(B, Hkv, 32 * 40 + R, D, 2, G, R, seed=300 + s_)
+        caches.append(quant_cache_to_torch(cache, dev))
+    qs = [synth.normal((B, Hq, D), seed=400 + i).to(dev) for i in range(6)]
+    sh = vc.shape(B, Hq, Hkv, D)
+    outs = {}
+    for flags in (0, vc.VC_CACHE_STATIC):
+        qcs = [vc.quant_cache(dict(c, flags=flags)) for c in caches]
+        ws = vc.workspace(vc.vc_draft_attn_quant_workspace_size(sh, qcs[0]))
+        res = []
+        for i, q in enumerate(qs):
+            out = torch.empty(B, Hq, D, device=dev)
+            vc.vc_draft_attn_quant(sh, qcs[i % 2], q, out, ws)
+            res.append(out)
+        torch.cuda.synchronize()
+        assert vc.vc_workspace_flags(ws) == 0
+        outs[flags] = [np32(o) for o in res]
+    for a_, b_ in zip(outs[0], outs[vc.VC_CACHE_STATIC]):
+        assert np.array_equal(a_, b_)
