@@ -1,6 +1,6 @@
 // vc_tc.cuh -- thin inline-PTX wrappers for the sm_100a 5th-generation tensor
 // core (tcgen05: MMA into tensor memory, TMEM allocation, loads/stores) and
-// for tiled TMA loads.  Only single-CTA forms are used, and no TMA load uses
+// for tiled TMA loads and stores.  Only single-CTA forms are used, and no TMA load uses
 // cluster multicast.
 #pragma once
 
@@ -115,6 +115,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, 
       "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
       : "memory");
 }
+
+// Tiled 3-D TMA store from shared memory (bulk-group completion); elements
+// of the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];\n" ::"l"(tmap),
+               "r"(x), "r"(y), "r"(z), "r"(smem_addr(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// Waits until every committed bulk store of this thread has read its shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
 
 }  // namespace tc
 }  // namespace vc

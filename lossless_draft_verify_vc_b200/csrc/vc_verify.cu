@@ -37,12 +37,14 @@
 //   * O += P_hi V + P_lo V as tcgen05.mma with A read from TMEM and V from
 //     shared memory (MN-major), accumulating in TMEM;
 //   * at the end each softmax thread moves its O row from TMEM to the output
-//     (one chunk) or to its chunk's partial, which splitk_combine_kernel
-//     merges in a programmatic-dependent launch.
+//     (one chunk) or, through shared memory and a TMA store, to its chunk's
+//     partial, which splitk_combine_kernel merges in a programmatic-dependent
+//     launch.
 // All waits are bounded; TMEM is always released.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <type_traits>
 
 #include "vc_splitk.cuh"
@@ -71,6 +73,9 @@ constexpr uint32_t kColS = 0;
 constexpr uint32_t kColPlo = kVBN / 2;  // offset of P's low part inside a buffer
 constexpr uint32_t kColO = 2 * kVBN;
 constexpr uint32_t kColTile = 256;      // columns of one row tile
+// One box of a partial's O rows in shared memory for the TMA store: 32 fp32
+// channels (128 bytes) x up to 128 rows.
+constexpr int kOBox = 128 * 128;
 
 template <int D, int RTC>
 struct VCfg {
@@ -89,6 +94,8 @@ struct VCfg {
   // buffer, Q, drain; then the TMEM address slot
   static constexpr int NBAR = 4 * NS + 6;
   static constexpr int SMEM_B = BAR_OFF + NBAR * 8 + 16 + 1024;  // + alignment slack
+  // the partials' O boxes reuse the Q and K/V area after the tile loop
+  static_assert(RTC * (D / 32) * kOBox <= BAR_OFF, "O boxes must fit below the barriers");
 };
 
 struct VArgs {
@@ -117,6 +124,7 @@ template <int D, int RTC>
 __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                      const __grid_constant__ CUtensorMap tm_k,
                                                                      const __grid_constant__ CUtensorMap tm_v,
+                                                                     const __grid_constant__ CUtensorMap tm_o,
                                                                      VArgs a) {
   using C = VCfg<D, RTC>;
   using K = VBlk<RTC>;
@@ -415,47 +423,68 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
   }
   __syncthreads();
   const bool ok = !aborted;
-  // ---- O rows straight from TMEM: with one chunk the normalised output rows
-  //      (and lse), otherwise this chunk's partial (unnormalised O, m, l) for
-  //      splitk_combine_kernel.  Rows past M are not stored.
+  // ---- O rows from TMEM: with one chunk the normalised output rows (and
+  //      lse) straight to global memory; otherwise this chunk's partial
+  //      (unnormalised O, m, l) for splitk_combine_kernel.  A partial's O
+  //      rows are contiguous in the workspace, so the softmax threads write
+  //      them into shared memory (free once the last P.V is done) in the
+  //      128-byte-swizzled layout of the partials' tensor map -- one box of
+  //      32 channels x the row tile's rows per 16 KB, bank-conflict free --
+  //      and the loader thread stores the boxes with TMA: coalesced full
+  //      lines instead of one 512-byte row per lane.  Rows past M are never
+  //      read back.
   if (softmax_thread && ok) {
     const bool live = r < M;
     const bool any = ntiles > 0;
-    float* dst = nullptr;
-    float sc = 1.f;
-    const size_t orow = (static_cast<size_t>(b) * a.nq + i0 + r / a.g) * a.Hq + h * a.g + r % a.g;
     const int rows_cap = a.nqt * a.g;
-    const size_t slot = (static_cast<size_t>(unit) * a.RT + rt) * a.C + chunk;
-    if (a.C == 1) {
-      dst = a.o.out + orow * D;
-      sc = (any && l_run > 0.f) ? 1.f / l_run : 0.f;
-    } else {
-      dst = a.o.part_o + (slot * rows_cap + r) * D;
-    }
-#pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      if (any) {
-        tc::ld32(tmem + lane_off + kColO + c0, o);  // warp-collective: every lane
-        tc::wait_ld();
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] = 0u;
-      }
-      if (live) {
-        float4* d4 = reinterpret_cast<float4*>(dst + c0);
-#pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          d4[j / 4] = make_float4(__uint_as_float(o[j]) * sc, __uint_as_float(o[j + 1]) * sc,
-                                  __uint_as_float(o[j + 2]) * sc, __uint_as_float(o[j + 3]) * sc);
-      }
-    }
     const float m_out = any ? m_run : -INFINITY;
     const float l_out = any ? l_run : 0.f;
-    if (live) {
-      if (a.C == 1) {
-        if (a.o.lse) a.o.lse[orow] = lse_from(m_out, l_out);
-      } else {
+    if (a.C == 1) {
+      const size_t orow = (static_cast<size_t>(b) * a.nq + i0 + r / a.g) * a.Hq + h * a.g + r % a.g;
+      float* dst = a.o.out + orow * D;
+      const float sc = (any && l_run > 0.f) ? 1.f / l_run : 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (any) {
+          tc::ld32(tmem + lane_off + kColO + c0, o);  // warp-collective: every lane
+          tc::wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+        if (live) {
+          float4* d4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            d4[j / 4] = make_float4(__uint_as_float(o[j]) * sc, __uint_as_float(o[j + 1]) * sc,
+                                    __uint_as_float(o[j + 2]) * sc, __uint_as_float(o[j + 3]) * sc);
+        }
+      }
+      if (live && a.o.lse) a.o.lse[orow] = lse_from(m_out, l_out);
+    } else {
+      unsigned char* ob = smem + wg * (D / 32) * kOBox + r * 128;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (any) {
+          tc::ld32(tmem + lane_off + kColO + c0, o);  // warp-collective: every lane
+          tc::wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+        if (r < rows_cap) {
+          unsigned char* row = ob + (c0 / 32) * kOBox;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4*>(row + ((q ^ (r & 7)) << 4)) =
+                make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();  // the boxes are read by the TMA store (async proxy)
+      if (live) {
+        const size_t slot = (static_cast<size_t>(unit) * a.RT + rt) * a.C + chunk;
         a.o.part_ml[(slot * rows_cap + r) * 2] = m_out;
         a.o.part_ml[(slot * rows_cap + r) * 2 + 1] = l_out;
       }
@@ -466,6 +495,17 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
   if (warp == 0) {
     tc::fence_after_sync();
     tc::dealloc(tmem, K::TMEM_COLS);
+  }
+  if (a.C > 1 && ok && tid == K::LOADER) {
+#pragma unroll 1
+    for (int t = 0; t < RTC; ++t) {
+      const int rts = RTC == 1 ? rt : t;
+      const int slot = (unit * a.RT + rts) * a.C + chunk;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tc::tma_store_3d(&tm_o, smem + (t * (D / 32) + c) * kOBox, c * 32, 0, slot);
+    }
+    tc::bulk_commit();
+    tc::bulk_wait_read();  // the shared memory must outlive the stores' reads
   }
 }
 
@@ -513,6 +553,21 @@ bool make_kv_map(CUtensorMap* m, const void* base, int64_t T, int D, int units) 
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over the chunk partials' O [slots][rows_cap][D] fp32 with a box of
+// 32 channels x rows_cap rows x 1 slot, 128-byte swizzle (the kernel's
+// shared-memory layout of a box).
+bool make_part_map(CUtensorMap* m, float* base, int rows_cap, int D, int64_t slots) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows_cap), static_cast<cuuint64_t>(slots)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(rows_cap) * D * 4};
+  cuuint32_t box[3] = {32, static_cast<cuuint32_t>(rows_cap), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -656,12 +711,16 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
   a.o.lse = lse;
   a.o.part_ml = reinterpret_cast<float*>(w + p.off_ml);
   a.o.part_o = reinterpret_cast<float*>(w + p.off_o);
+  CUtensorMap to;
+  memset(&to, 0, sizeof(to));
+  if (p.C > 1 && !vc::make_part_map(&to, a.o.part_o, p.nqt * a.g, shape->D, static_cast<int64_t>(units) * p.RT * p.C))
+    return vc::set_error(VC_ERR_CUDA, "vc_verify_attn: could not encode the partials' tensor map");
   dim3 grid(p.C, units, p.RT / p.RTC);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto go = [&](auto DD, auto RR) {
     constexpr int Dv = decltype(DD)::value, Rv = decltype(RR)::value;
     vc::verify_occupancy<Dv, Rv>();  // sets the shared-memory attribute once per device
-    vc::verify_kernel<Dv, Rv><<<grid, vc::VBlk<Rv>::THREADS, vc::VCfg<Dv, Rv>::SMEM_B, s>>>(tq, tk, tv, a);
+    vc::verify_kernel<Dv, Rv><<<grid, vc::VBlk<Rv>::THREADS, vc::VCfg<Dv, Rv>::SMEM_B, s>>>(tq, tk, tv, to, a);
   };
   using I128 = std::integral_constant<int, 128>;
   using I64 = std::integral_constant<int, 64>;
