@@ -307,7 +307,8 @@ __device__ __forceinline__ void issue_advance(const QArgs& a, IssuePtr& ip, int 
   }
 }
 
-// One bulk copy of this warp's next quantised stage (at ip) into ring slot `slot`.
+// One bulk copy of this warp's next quantised stage (at ip) into ring slot
+// `slot`; the records are read once per call (evict-first in L2).
 template <typename C>
 __device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring, uint64_t* bars, int lane, int slot,
                                             const IssuePtr& ip) {
@@ -318,7 +319,7 @@ __device__ __forceinline__ void issue_stage(const QArgs& a, unsigned char* ring,
   }
   if (lane == 0) {
     mbar_arrive_expect_tx(&bars[slot], bytes);
-    bulk_g2s(ring + slot * C::STAGE, ip.src, bytes, &bars[slot]);
+    bulk_g2s_once(ring + slot * C::STAGE, ip.src, bytes, &bars[slot]);
   }
 }
 
@@ -970,8 +971,8 @@ __device__ __forceinline__ void residual_seg(const QArgs& a, unsigned char* ring
     // the tile's K rows and V rows are contiguous: two bulk copies
     if (lane == 0) {
       mbar_arrive_expect_tx(bar, 2u * nv * ROW_B);
-      bulk_g2s(ring, kr + static_cast<size_t>(t0) * D, nv * ROW_B, bar);
-      bulk_g2s(ring + kResRows * ROW_B, vr + static_cast<size_t>(t0) * D, nv * ROW_B, bar);
+      bulk_g2s_once(ring, kr + static_cast<size_t>(t0) * D, nv * ROW_B, bar);
+      bulk_g2s_once(ring + kResRows * ROW_B, vr + static_cast<size_t>(t0) * D, nv * ROW_B, bar);
     }
     __syncwarp();
     if (!__all_sync(FULL, mbar_wait_bounded(bar, rph & 1, a.flags))) {  // warp-uniform

@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kSpNW * 32) draft_sparse_kernel(SpArgs a) {
     }
     __syncwarp();
     const __nv_bfloat16* src = (lane < 16 ? kh : vh) + static_cast<size_t>(pos) * D;
-    bulk_g2s(ring + s * C::STAGE_B + lane * C::RS, src, C::ROW_B, &bars[s]);
+    bulk_g2s_once(ring + s * C::STAGE_B + lane * C::RS, src, C::ROW_B, &bars[s]);
   };
 
   // Q fragments: rows 0..7 = query heads of this group (zero beyond g),

@@ -116,6 +116,25 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// An L2 cache policy that evicts the lines it tags first: for data read
+// once (a stream of K/V tiles), so that it does not push out what is read
+// again soon (the chunk partials that the merge reads back).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+
+// tma_load_3d with an L2 cache policy (from l2_evict_first and the like).
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+      "{%2, %3, %4}], [%5], %6;\n" ::"r"(smem_addr(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
 // Tiled 3-D TMA store from shared memory (bulk-group completion); elements
 // of the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int x, int y, int z) {

@@ -163,7 +163,9 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
   const bool softmax_thread = tid < K::SOFTMAX;
   bool fail = false;
 
-  // K (v = 0) or V (v = 1) of tile i into stage i % NS; loader only
+  // K (v = 0) or V (v = 1) of tile i into stage i % NS; loader only.  K and
+  // V are read once: their lines go first when L2 needs room.
+  const uint64_t kv_policy = tc::l2_evict_first();
   auto issue_load = [&](int i, int v) {
     unsigned char* dst = st_s + (i % NS) * C::STAGE_B + v * C::KV_B;
     uint64_t* bar = v ? &bar_v[i % NS] : &bar_k[i % NS];
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
     mbar_arrive_expect_tx(bar, C::KV_B);
 #pragma unroll
     for (int hf = 0; hf < C::HALVES; ++hf)
-      tc::tma_load_3d(dst + hf * kVBN * 128, v ? &tm_v : &tm_k, hf * 64, y, unit, bar);
+      tc::tma_load_3d_hint(dst + hf * kVBN * 128, v ? &tm_v : &tm_k, hf * 64, y, unit, bar, kv_policy);
   };
 
   // The loader owns the barriers' initialisation and requests Q (every row
