@@ -90,9 +90,9 @@ struct VCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int ST_OFF = Q_B;
   static constexpr int BAR_OFF = ST_OFF + NS * STAGE_B;
-  // barriers: K full / K free / V full / V free per stage, S and P.V per S
-  // buffer, Q, drain; then the TMEM address slot
-  static constexpr int NBAR = 4 * NS + 6;
+  // barriers: K full / K free / V full / V free per stage, S, P and P.V per
+  // S buffer, Q, drain; then the TMEM address slot and the abort flag
+  static constexpr int NBAR = 4 * NS + 8;
   static constexpr int SMEM_B = BAR_OFF + NBAR * 8 + 16 + 1024;  // + alignment slack
   // the partials' O boxes reuse the Q and K/V area after the tile loop
   static_assert(RTC * (D / 32) * kOBox <= BAR_OFF, "O boxes must fit below the barriers");
@@ -106,19 +106,6 @@ struct VArgs {
   uint32_t* flags;
   SplitKOut o;
 };
-
-// Block-wide barrier of the softmax warps and the MMA warp only (the loader
-// warp runs its own loop); returns whether any participant passed true.
-template <int RTC>
-__device__ __forceinline__ bool mma_group_sync_or(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"(v ? 1u : 0u), "n"(VBlk<RTC>::SOFTMAX + 32)
-      : "memory");
-  return r != 0;
-}
 
 template <int D, int RTC>
 __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -141,10 +128,12 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
   uint64_t* bar_v = bar_kf + NS;                                      // [NS] V stage landed
   uint64_t* bar_vf = bar_v + NS;                                      // [NS] V stage read by its P.V MMAs
   uint64_t* bar_s = bar_vf + NS;                                      // [2] S buffer computed
-  uint64_t* bar_pv = bar_s + 2;                                       // [2] P.V of that buffer done
+  uint64_t* bar_p = bar_s + 2;                                        // [2] P of that buffer stored
+  uint64_t* bar_pv = bar_p + 2;                                       // [2] P.V of that buffer done
   uint64_t* bar_q = bar_pv + 2;                                       // Q staged
   uint64_t* bar_dr = bar_q + 1;                                       // drain after a give-up
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_dr + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);  // a wait gave up
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int chunk = blockIdx.x;
@@ -181,6 +170,9 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
   // barrier before the block-wide barrier below.
   if (tid == K::LOADER) {
     for (int j = 0; j < C::NBAR; ++j) mbar_init(&bar_k[j], 1);
+    mbar_init(&bar_p[0], K::SOFTMAX / 32);  // one arrival per softmax warp
+    mbar_init(&bar_p[1], K::SOFTMAX / 32);
+    *s_abort = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(bar_q, RTC * C::HALVES * 128 * a.g * a.nqt);
@@ -225,12 +217,27 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
   const int64_t vis_end = a.T - a.nq + i_row + 1;  // keys [0, vis_end) visible to this row
   float m_run = -INFINITY, l_run = 0.f;
 
+  // Bounded wait that also gives up as soon as another thread of the block
+  // has given up (*s_abort), so that a failure ends the block promptly.
+  auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+      if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+      if (*s_abort != 0) return false;
+      if (global_timer_ns() - t0 > 2000000000ull) {
+        atomicOr(a.flags, VC_FLAG_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  };
+
   // S = Q K^T of tile i into buffer i & 1 of every row tile: MMA thread, once
   // tile i's K has landed; when those MMAs complete, the S buffer is ready
   // for the softmax and the K stage free for the loader
   auto issue_s = [&](int i) -> bool {
     const uint32_t ks_addr = smem_addr(st_s + (i % NS) * C::STAGE_B);
-    if (!mbar_wait_bounded(&bar_k[i % NS], (i / NS) & 1, a.flags)) return false;
+    if (!wait_or_abort(&bar_k[i % NS], (i / NS) & 1)) return false;
     tc::fence_after_sync();
 #pragma unroll
     for (int t = 0; t < RTC; ++t)
@@ -250,13 +257,15 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
     if (!mbar_wait_bounded(bar_q, 0, a.flags)) fail = true;
     if (!fail && ntiles > 0 && !issue_s(0)) fail = true;
     if (!fail && ntiles > 1 && !issue_s(1)) fail = true;
+    if (fail) *s_abort = 1;
   }
 
   // Failure handling: every wait is bounded; a thread that sees a timeout sets
-  // its sticky `fail`.  tcgen05.ld / st are warp-collective, so each warp
-  // decides them with __any_sync; the tile loop of the softmax and MMA warps
-  // exits on their common barrier's OR, so they leave together; the loader
-  // stops at its first failed wait.  All meet again after the loop.
+  // its sticky `fail` and the block's abort flag, and every other wait gives
+  // up once it sees the flag.  tcgen05.ld / st are warp-collective, so each
+  // warp decides them with __any_sync; a softmax warp that gives up still
+  // arrives on its P barrier (after setting the flag), so the MMA thread does
+  // not wait for it.  All meet again after the loop.
   constexpr unsigned FULL = 0xffffffffu;
   int nk = ntiles < NS ? ntiles : NS, nv = nk;  // K / V tiles issued so far (loader)
   if (warp == K::LOADER / 32) {
@@ -270,8 +279,9 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
       while (nk < ntiles || nv < ntiles) {
         const bool is_k = nk < ntiles && nk <= nv + 1;
         const int j = is_k ? nk : nv;
-        if (!mbar_wait_bounded(is_k ? &bar_kf[j % NS] : &bar_vf[j % NS], (j / NS - 1) & 1, a.flags)) {
+        if (!wait_or_abort(is_k ? &bar_kf[j % NS] : &bar_vf[j % NS], (j / NS - 1) & 1)) {
           fail = true;
+          *s_abort = 1;
           break;
         }
         issue_load(j, is_k ? 0 : 1);
@@ -281,100 +291,123 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
           nv = j + 1;
       }
     }
-  } else {
+    __syncwarp();  // the other lanes wait here, not in a barrier poll
+  } else if (softmax_thread) {
+    // ---- softmax warps: S of tile i -> P of tile i (over S), then one
+    //      arrival per warp on the buffer's "P stored" barrier; they go on
+    //      to tile i + 1 without waiting for the MMA warp
     for (int i = 0; i < ntiles; ++i) {
       const int s = i & 1;
-      const uint32_t vs_addr = smem_addr(st_s + (i % NS) * C::STAGE_B) + C::KV_B;
-      if (softmax_thread) {  // warp-uniform
-        if (!fail && !mbar_wait_bounded(&bar_s[s], (i >> 1) & 1, a.flags)) fail = true;
-        tc::fence_after_sync();
-        bool wfail = __any_sync(FULL, fail);
-        uint32_t sr[2][32];
-        if (!wfail) {
-          tc::ld32(tmem + lane_off + kColS + s * kVBN, sr[0]);
-          tc::ld32(tmem + lane_off + kColS + s * kVBN + 32, sr[1]);
-          tc::wait_ld();
-        } else {
+      if (__any_sync(FULL, *s_abort != 0)) {
+        fail = true;
+        break;
+      }
+      if (!fail && !wait_or_abort(&bar_s[s], (i >> 1) & 1)) fail = true;
+      tc::fence_after_sync();
+      bool wfail = __any_sync(FULL, fail);
+      uint32_t sr[2][32];
+      if (!wfail) {
+        tc::ld32(tmem + lane_off + kColS + s * kVBN, sr[0]);
+        tc::ld32(tmem + lane_off + kColS + s * kVBN + 32, sr[1]);
+        tc::wait_ld();
+      } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) sr[0][j] = sr[1][j] = 0u;
-        }
-        const int64_t t0 = k_begin + static_cast<int64_t>(i) * kVBN;
-        const int64_t lim = min(vis_end, k_end) - t0;  // keys [t0, t0 + lim) are live
-        // raw scores; the scale (> 0) is applied in the exponent's FMA below
-        float tmax = -INFINITY;
-        if (__all_sync(FULL, lim >= kVBN)) {  // whole tile visible to the warp's rows: no mask
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; ++j) tmax = fmaxf(tmax, __uint_as_float(sr[c][j]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
-              sr[c][j] = __float_as_uint(x);
-              tmax = fmaxf(tmax, x);
-            }
-        }
-        tmax *= a.scale_log2;
-        // lazy rescale: keep the stale maximum unless the new one exceeds it by > 8
-        float m_use = m_run;
-        float alpha = 1.f;
-        if (tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY)) {
-          m_use = tmax;
-          if (m_run != -INFINITY) alpha = ex2(m_run - m_use);
-          m_run = m_use;
-        }
-        const float m_sub = m_use == -INFINITY ? 0.f : m_use;
-        uint32_t phi[32], plo[32];
-        float psum = 0.f;
+        for (int j = 0; j < 32; ++j) sr[0][j] = sr[1][j] = 0u;
+      }
+      const int64_t t0 = k_begin + static_cast<int64_t>(i) * kVBN;
+      const int64_t lim = min(vis_end, k_end) - t0;  // keys [t0, t0 + lim) are live
+      // raw scores; the scale (> 0) is applied in the exponent's FMA below
+      float tmax = -INFINITY;
+      if (__all_sync(FULL, lim >= kVBN)) {  // whole tile visible to the warp's rows: no mask
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, -m_sub));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, -m_sub));
-            psum += p0 + p1;
-            const uint32_t hw = pack_bf2(p0, p1);
-            const float2 hf = unpack_bf2(hw);
-            phi[c * 16 + j / 2] = hw;
-            plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
-          }
-        l_run = l_run * alpha + psum;
-        // O is rescaled only when a row of the warp raised its maximum (rare
-        // with the lazy rule); only then must the previous P.V be done first.
-        // P goes over this tile's own S buffer, which no MMA in flight reads,
-        // so storing it needs no wait: the softmax of tile i overlaps P.V of
-        // tile i - 1.
-        const bool rescale = __any_sync(FULL, alpha != 1.f);  // warp-uniform
-        if (rescale) {
-          if (i > 0 && !fail && !mbar_wait_bounded(&bar_pv[(i - 1) & 1], ((i - 1) >> 1) & 1, a.flags)) fail = true;
-          tc::fence_after_sync();
-        }
-        wfail = __any_sync(FULL, fail);
-        if (!wfail && rescale) {  // lanes without a new max scale by 1
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tc::ld32(tmem + lane_off + kColO + c0, o);
-            tc::wait_ld();
+          for (int j = 0; j < 32; ++j) tmax = fmaxf(tmax, __uint_as_float(sr[c][j]));
+      } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tc::st32(tmem + lane_off + kColO + c0, o);
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float x = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
+            sr[c][j] = __float_as_uint(x);
+            tmax = fmaxf(tmax, x);
           }
-        }
-        if (!wfail) {  // P over this tile's S, read above
-          tc::st32(tmem + lane_off + kColS + s * kVBN, phi);
-          tc::st32(tmem + lane_off + kColS + s * kVBN + kColPlo, plo);
-          tc::wait_st();
-        }
-        tc::fence_before_sync();
       }
-      if (mma_group_sync_or<RTC>(fail)) break;
-      if (tid == K::ISSUER) {
+      tmax *= a.scale_log2;
+      // lazy rescale: keep the stale maximum unless the new one exceeds it by > 8
+      float m_use = m_run;
+      float alpha = 1.f;
+      if (tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY)) {
+        m_use = tmax;
+        if (m_run != -INFINITY) alpha = ex2(m_run - m_use);
+        m_run = m_use;
+      }
+      const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+      uint32_t phi[32], plo[32];
+      float psum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, -m_sub));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, -m_sub));
+          psum += p0 + p1;
+          const uint32_t hw = pack_bf2(p0, p1);
+          const float2 hf = unpack_bf2(hw);
+          phi[c * 16 + j / 2] = hw;
+          plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
+        }
+      l_run = l_run * alpha + psum;
+      // O is rescaled only when a row of the warp raised its maximum (rare
+      // with the lazy rule); only then must the previous P.V be done first.
+      // P goes over this tile's own S buffer, which no MMA in flight reads,
+      // so storing it needs no wait: the softmax of tile i overlaps P.V of
+      // tile i - 1.
+      const bool rescale = __any_sync(FULL, alpha != 1.f);  // warp-uniform
+      if (rescale) {
+        if (i > 0 && !fail && !wait_or_abort(&bar_pv[(i - 1) & 1], ((i - 1) >> 1) & 1)) fail = true;
         tc::fence_after_sync();
-        if (!mbar_wait_bounded(&bar_v[i % NS], (i / NS) & 1, a.flags)) fail = true;
+      }
+      wfail = __any_sync(FULL, fail);
+      if (!wfail && rescale) {  // lanes without a new max scale by 1
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tc::ld32(tmem + lane_off + kColO + c0, o);
+          tc::wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tc::st32(tmem + lane_off + kColO + c0, o);
+        }
+      }
+      if (!wfail) {  // P over this tile's S, read above
+        tc::st32(tmem + lane_off + kColS + s * kVBN, phi);
+        tc::st32(tmem + lane_off + kColS + s * kVBN + kColPlo, plo);
+        tc::wait_st();
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (wfail) {
+        if ((tid & 31) == 0) *s_abort = 1;  // seen by the MMA thread after its wait below
+        __syncwarp();
+      }
+      if ((tid & 31) == 0) mbar_arrive(&bar_p[s]);
+      if (wfail) {
+        fail = true;
+        break;
+      }
+    }
+  } else if (warp == K::ISSUER / 32) {
+    if (tid == K::ISSUER) {
+      // ---- MMA thread: P.V of tile i once every softmax warp stored P (and
+      //      any rescale of O); once that P.V is done, S of tile i + 2 into the
+      //      same buffer
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i & 1;
+        const uint32_t vs_addr = smem_addr(st_s + (i % NS) * C::STAGE_B) + C::KV_B;
+        if (!wait_or_abort(&bar_p[s], (i >> 1) & 1) || *s_abort != 0) fail = true;
+        tc::fence_after_sync();
+        if (!fail && !wait_or_abort(&bar_v[i % NS], (i / NS) & 1)) fail = true;
         if (!fail) {
 #pragma unroll
           for (int t = 0; t < RTC; ++t) {
@@ -396,15 +429,19 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
         }
         if (!fail && i + 2 < ntiles) {
           // P.V of tile i done: its S buffers take tile i + 2
-          if (!mbar_wait_bounded(&bar_pv[s], (i >> 1) & 1, a.flags) || !issue_s(i + 2)) fail = true;
+          if (!wait_or_abort(&bar_pv[s], (i >> 1) & 1) || !issue_s(i + 2)) fail = true;
+        }
+        if (fail) {
+          *s_abort = 1;
+          break;
         }
       }
     }
+    __syncwarp();
   }
 
   // ---- drain, read O, release TMEM
-  if (!fail && ntiles > 0 && !mbar_wait_bounded(&bar_pv[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, a.flags))
-    fail = true;
+  if (!fail && ntiles > 0 && !wait_or_abort(&bar_pv[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1)) fail = true;
   tc::fence_after_sync();
   const bool aborted = __syncthreads_or(fail) != 0;
   if (aborted && tid == K::ISSUER) {
