@@ -345,17 +345,21 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
       const float m_sub = m_use == -INFINITY ? 0.f : m_use;
       uint32_t phi[32], plo[32];
       float psum = 0.f;
+      // pairs of columns in packed fp32x2 arithmetic (each half rounds as the
+      // scalar instruction would)
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_sub, -m_sub);
+      const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
       for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, -m_sub));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, -m_sub));
+          const float2 e = __ffma2_rn(make_float2(__uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1])), sc2, nm2);
+          const float p0 = ex2(e.x), p1 = ex2(e.y);
           psum += p0 + p1;
           const uint32_t hw = pack_bf2(p0, p1);
-          const float2 hf = unpack_bf2(hw);
+          const float2 lo = __ffma2_rn(unpack_bf2(hw), neg1, make_float2(p0, p1));  // p - bf16(p), exact
           phi[c * 16 + j / 2] = hw;
-          plo[c * 16 + j / 2] = pack_bf2(p0 - hf.x, p1 - hf.y);
+          plo[c * 16 + j / 2] = pack_bf2(lo.x, lo.y);
         }
       l_run = l_run * alpha + psum;
       // O is rescaled only when a row of the warp raised its maximum (rare
