@@ -16,7 +16,7 @@
 // s and z, half to even; s == 0 gives code 0.  Every code equals the one the
 // float64 quotient gives: the quotient is first taken in fp32 as
 // (x - z) * (1 / s), whose error is below 2^-18 for the quotients that are
-// not clamped (|q| <= 16); only when that lands within 2^-12 of a rounding
+// not clamped (|q| <= 16); only when that lands within 2^-17 of a rounding
 // tie (k + 1/2) is it recomputed as an IEEE float64 division of the exact
 // float64 difference.
 #include "vc_common.cuh"
@@ -35,22 +35,114 @@ __device__ __forceinline__ uint16_t to_half_checked(double v, uint32_t* flags) {
   return __half_as_ushort(h);
 }
 
-__device__ __forceinline__ double half_bits_to_double(uint16_t b) {
-  return static_cast<double>(__half2float(__ushort_as_half(b)));
+// Codes of a pair of elements (one bf16x2 register): clamp(rint((x - z) / s),
+// 0, levels), returned as code(lo) | code(hi) << 16.  Fast form: the
+// quotient in fp32 as (x - z) * (1 / s), both halves in one packed fp32x2
+// instruction each; its error is at most 3 * 2^-24 * |q| < 2^-18 where
+// 0 <= q <= 15.5, so a quotient farther than 2^-17 from a rounding tie
+// rounds as the exact one does, and `near` is set for the others (exact
+// ties are common: bf16 data, fp16 scale and zero).  Rounding adds
+// 1.5 * 2^23, which leaves rint(q) in the low mantissa bits.  Clamping
+// before rounding gives the same codes as clamping after it; a NaN quotient
+// (zero or scale outside fp16) gives code 0.
+template <int BITS>
+__device__ __forceinline__ uint32_t codes2_fast(uint32_t xb, float2 negz, float2 inv, bool& near) {
+  constexpr float levels = static_cast<float>((1 << BITS) - 1);
+  constexpr float kMagic = 12582912.0f;                // 1.5 * 2^23
+  constexpr float kTie = 0.5f - 7.62939453125e-6f;     // 0.5 - 2^-17
+  const float2 x = unpack_bf2(xb);
+  const float2 q = __fmul2_rn(__fadd2_rn(x, negz), inv);
+  const float2 qc = make_float2(fminf(fmaxf(q.x, 0.f), levels), fminf(fmaxf(q.y, 0.f), levels));
+  const float2 m = __fadd2_rn(qc, make_float2(kMagic, kMagic));
+  const float2 e = __ffma2_rn(__fadd2_rn(m, make_float2(-kMagic, -kMagic)), make_float2(-1.f, -1.f), qc);
+  near = fabsf(e.x) > kTie || fabsf(e.y) > kTie;
+  return __byte_perm(__float_as_uint(m.x), __float_as_uint(m.y), 0x5410);
 }
 
-// code = clamp(rint((x - z) / s), 0, levels); s == 0 -> 0 (inv_s is then 0).
-// sz points at the stored (scale, zero) fp16 bits, read only on the slow path.
-__device__ __forceinline__ uint32_t quant_code(float x, float2 zi, int levels, const uint16_t* s_bits,
-                                               const uint16_t* z_bits) {
-  const float q = (x - zi.x) * zi.y;
-  float r = rintf(q);
-  if (fabsf(fabsf(q - r) - 0.5f) < 2.44140625e-4f && zi.y != 0.f) {  // near a tie: the exact quotient decides
-    const double sd = half_bits_to_double(*s_bits), zd = half_bits_to_double(*z_bits);
-    r = static_cast<float>(rint((static_cast<double>(x) - zd) / sd));
+// Code of one element as the float64 rule gives it: rint of the float64
+// quotient of the float64 difference by the stored scale (out of line: it
+// runs only where x - z is not exact in fp32, which needs exponents ~2^24
+// apart).
+template <int BITS>
+__device__ __noinline__ uint32_t code_f64(float x, float negz, float s) {
+  const double r = rint((static_cast<double>(x) + static_cast<double>(negz)) / static_cast<double>(s));
+  return static_cast<uint32_t>(fmin(fmax(r, 0.0), static_cast<double>((1 << BITS) - 1)));
+}
+
+// Code of one element whose fp32 quotient may sit on the wrong side of a
+// tie T = k + 1/2.  When d = fp32(x - z) is exact (its two-sum error is
+// zero), d and T s are exact fp32 numbers, and the sign of d - T s (one
+// fused multiply-add, so the sign is exact) tells whether (x - z) / s lies
+// above, below or on T; on T the even neighbour wins.  Any other quotient is
+// at least ~2^-24 T from T, so the float64 quotient falls on the same side.
+template <int BITS>
+__device__ __forceinline__ uint32_t code_near(float x, float negz, float inv, float s) {
+  constexpr float levels = static_cast<float>((1 << BITS) - 1);
+  if (s == 0.f) return 0u;
+  const float d = __fadd_rn(x, negz);
+  const float bv = __fsub_rn(d, x), av = __fsub_rn(d, bv);
+  const float err = __fadd_rn(__fsub_rn(x, av), __fsub_rn(negz, bv));
+  if (err != 0.f) return code_f64<BITS>(x, negz, s);
+  const float qc = fminf(fmaxf(__fmul_rn(d, inv), 0.f), levels);
+  const float r = rintf(qc);
+  if (fabsf(qc - r) <= 0.25f) return static_cast<uint32_t>(r);  // not near a tie
+  const float T = qc > r ? r + 0.5f : r - 0.5f;
+  const float t = fmaf(-T, s, d);
+  const float lo = T - 0.5f;
+  float c = t > 0.f ? T + 0.5f : (t < 0.f ? lo : ((static_cast<int>(lo) & 1) == 0 ? lo : T + 0.5f));
+  c = fminf(fmaxf(c, 0.f), levels);
+  return static_cast<uint32_t>(c);
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t codes2_near(uint32_t xb, float2 negz, float2 inv, float2 sc) {
+  const float2 x = unpack_bf2(xb);
+  return code_near<BITS>(x.x, negz.x, inv.x, sc.x) | (code_near<BITS>(x.y, negz.y, inv.y, sc.y) << 16);
+}
+
+// Per-lane fix-up of a word pair whose fast codes include pairs near a tie
+// (bit 4 i + register of nm): the tile's registers are loaded again and the
+// near pairs recomputed with code_near.  Warp-collective (ldmatrix); out of
+// line so that the common path keeps few registers.
+//   base: the staged K (isv false) or V rows; RS their stride in bytes;
+//   z, iv, sc: (-zero, 1 / scale, scale) per key channel, or per token of
+//   value group cg at z + cg * G (G floats per group).
+template <int BITS, int G, int RS, int TPW>
+__device__ __noinline__ uint2 fix_words(uint2 w, uint32_t nm, bool isv, int tt, int j, const unsigned char* base,
+                                        const float* z, const float* iv, const float* sc) {
+  constexpr uint32_t levels = (1u << BITS) - 1u;
+  const int lane = threadIdx.x & 31, tig = lane & 3, mi = lane >> 3, ri = lane & 7;
+  const int wsh = isv ? 0 : 1, osh = isv ? 1 : 0;
+  for (int i = 0; i < TPW; ++i) {
+    if (!__any_sync(0xffffffffu, (nm >> (4 * i)) & 0xfu)) continue;
+    const int ct = TPW * j + i;
+    uint32_t r[4];
+    int o0;
+    const float *zp = z, *ip = iv, *sp = sc;
+    if (!isv) {
+      ldsm_x4(r, base + (16 * tt + 8 * (mi & 1) + ri) * RS + (16 * ct + 8 * (mi >> 1)) * 2);
+      o0 = 16 * ct + 2 * tig;
+    } else {
+      ldsm_x4_t(r, base + (16 * tt + 8 * (mi >> 1) + ri) * RS + (16 * ct + 8 * (mi & 1)) * 2);
+      const int cg = 16 * ct / G;
+      zp += cg * G, ip += cg * G, sp += cg * G;
+      o0 = 16 * tt + 2 * tig;
+    }
+    for (int k = 0; k < 4; ++k) {
+      if (!((nm >> (4 * i + k)) & 1u)) continue;
+      const int o = o0 + (k < 2 ? 0 : 8);
+      const uint32_t p = codes2_near<BITS>(r[k], *reinterpret_cast<const float2*>(zp + o),
+                                           *reinterpret_cast<const float2*>(ip + o),
+                                           *reinterpret_cast<const float2*>(sp + o));
+      const int sh = 8 * ((k >> osh) & 1) + BITS * i;
+      const uint32_t field = (levels | (levels << 16)) << sh;
+      if ((k >> wsh) & 1)
+        w.y = (w.y & ~field) | (p << sh);
+      else
+        w.x = (w.x & ~field) | (p << sh);
+    }
   }
-  r = fminf(fmaxf(r, 0.f), static_cast<float>(levels));
-  return static_cast<uint32_t>(r);
+  return w;
 }
 
 template <int BITS, int G, int D>
@@ -60,119 +152,164 @@ struct QuantLayout {
   static constexpr int KT = D / 16;
   static constexpr int TPW = 8 / BITS;
   static constexpr int NW = 2 * KT / TPW;  // words per lane per 16-token tile
+  static constexpr int NJ = KT / TPW;      // word pairs (X, Y) per lane per 16-token tile
   static constexpr int CPG = D / G;
   static constexpr int WORDS = CB / 4;     // 32-bit words of one code block
 };
 
 // One block of 128 threads per (group, unit).  The group's K and V rows are
-// staged in shared memory (bf16), the parameters and reciprocal scales
-// computed, then every thread assembles whole 32-bit words of the
-// fragment-native code blocks (the order in which the draft kernel's lanes
-// consume them), computing each code where it is packed, and the block
-// writes words and parameters as one record.
+// staged in shared memory (bf16, rows padded by 16 bytes so that the eight
+// 16-byte rows of an ldmatrix hit distinct banks).  Parameters: keys per
+// channel by one thread each, values per (token, value group) by one warp
+// per token row with shuffles.  Codes: a warp takes one (16-token tile,
+// word pair) of K or V at a time; ldmatrix (transposed for V) hands every
+// lane the elements of its fragment-native code words directly (the order in
+// which the draft kernel's lanes consume them), so each lane computes and
+// packs whole words and stores them.
 template <int BITS, int G, int D>
 __device__ __forceinline__ void quantize_group(const __nv_bfloat16* __restrict__ kgp,
                                                const __nv_bfloat16* __restrict__ vgp, uint8_t* __restrict__ rec,
                                                uint32_t* flags) {
   using L = QuantLayout<BITS, G, D>;
   constexpr int levels = (1 << BITS) - 1;
-  __shared__ __align__(16) __nv_bfloat16 ks[G][D];
-  __shared__ __align__(16) __nv_bfloat16 vs[G][D];
-  __shared__ uint16_t skz[2][D];          // key scale, key zero (natural channel order)
-  __shared__ uint16_t svz[2][G][L::CPG];  // value scale, value zero per (token, value group)
-  __shared__ float2 kzi[D];           // key zero, 1 / key scale (0 when the scale is 0), fp32
-  __shared__ float2 vzi[G][L::CPG];   // the same per value group
-  const int tid = threadIdx.x;
+  constexpr int RS = 2 * D + 16;  // bytes per staged row
+  constexpr int TT = G / 16, TPW = L::TPW, NJ = L::NJ, NW = L::NW, CPG = L::CPG;
+  constexpr int EPL = D / 32;     // channels per lane in a row
+  constexpr int LPG = G / EPL;    // lanes per value group
+  __shared__ __align__(16) unsigned char ks[G * RS];
+  __shared__ __align__(16) unsigned char vs[G * RS];
+  __shared__ __align__(8) float kzn[D], kin[D], ksc[D];             // -zero, 1 / scale (0 if 0), scale
+  __shared__ __align__(8) float vzn[CPG][G], vin[CPG][G], vsc[CPG][G];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint4* kg = reinterpret_cast<const uint4*>(kgp);
   const uint4* vg = reinterpret_cast<const uint4*>(vgp);
-  for (int e = tid; e < G * D / 8; e += 128) {  // stage the group's rows, 16-byte loads
-    reinterpret_cast<uint4*>(&ks[0][0])[e] = kg[e];
-    reinterpret_cast<uint4*>(&vs[0][0])[e] = vg[e];
+  for (int e = tid; e < G * D / 8; e += 128) {  // stage the group's rows, 16-byte streaming loads
+    const int t = e / (D / 8), c8 = e - t * (D / 8);
+    *reinterpret_cast<uint4*>(ks + t * RS + c8 * 16) = __ldcs(kg + e);
+    *reinterpret_cast<uint4*>(vs + t * RS + c8 * 16) = __ldcs(vg + e);
   }
   __syncthreads();
-  auto K = [&](int t, int c) { return __bfloat162float(ks[t][c]); };
-  auto V = [&](int t, int c) { return __bfloat162float(vs[t][c]); };
-
-  // key parameters: channel c over the group's G tokens
-  for (int c = tid; c < D; c += 128) {
-    float mn = K(0, c), mx = mn;
-    for (int t = 1; t < G; ++t) mn = fminf(mn, K(t, c)), mx = fmaxf(mx, K(t, c));
-    skz[0][c] = to_half_checked((static_cast<double>(mx) - static_cast<double>(mn)) / levels, flags);
-    skz[1][c] = to_half_checked(static_cast<double>(mn), flags);
-    const float sf = __half2float(__ushort_as_half(skz[0][c]));
-    kzi[c] = make_float2(__half2float(__ushort_as_half(skz[1][c])), sf != 0.f ? 1.f / sf : 0.f);
-  }
-  // value parameters: token t, value group cg over its G channels
-  for (int e = tid; e < G * L::CPG; e += 128) {
-    const int t = e / L::CPG, cg = e % L::CPG;
-    float mn = V(t, cg * G), mx = mn;
-    for (int c = 1; c < G; ++c) mn = fminf(mn, V(t, cg * G + c)), mx = fmaxf(mx, V(t, cg * G + c));
-    svz[0][t][cg] = to_half_checked((static_cast<double>(mx) - static_cast<double>(mn)) / levels, flags);
-    svz[1][t][cg] = to_half_checked(static_cast<double>(mn), flags);
-    const float sf = __half2float(__ushort_as_half(svz[0][t][cg]));
-    vzi[t][cg] = make_float2(__half2float(__ushort_as_half(svz[1][t][cg])), sf != 0.f ? 1.f / sf : 0.f);
-  }
-  __syncthreads();
-  auto vcode = [&](int t, int c) -> uint32_t {
-    const int cg = c / G;
-    return quant_code(V(t, c), vzi[t][cg], levels, &svz[0][t][cg], &svz[1][t][cg]);
-  };
-
-  uint32_t* kw = reinterpret_cast<uint32_t*>(rec);
-  uint32_t* vw = reinterpret_cast<uint32_t*>(rec + L::CB);
-  // code words: word index = (tt * 32 + lane) * NW + w, w = 2 j + (0: X, 1: Y);
-  // local tile i of pair j covers channel (key) / channel-row (value) tile TPW j + i;
-  // first register's codes at bits [b i] and [16 + b i], second's at [8 + b i], [24 + b i]
-  for (int wi = tid; wi < L::WORDS; wi += 128) {
-    const int w = wi % L::NW, rest = wi / L::NW;
-    const int lane = rest % 32, tt = rest / 32;
-    const int gid = lane >> 2, tig = lane & 3;
-    const int j = w >> 1, isY = w & 1;
-    uint32_t kword = 0, vword = 0;
-#pragma unroll
-    for (int i = 0; i < L::TPW; ++i) {
-      const int ct = L::TPW * j + i;
-      {  // keys: X = (reg0: token gid, reg1: token gid + 8) at channels 16 ct + 2 tig (+8 in Y)
-        const int c = 16 * ct + 2 * tig + (isY ? 8 : 0);
-        const int t0 = 16 * tt + gid, t1 = t0 + 8;
-        const float2 z0 = kzi[c], z1 = kzi[c + 1];
-        const float2 x0 = unpack_bf2(*reinterpret_cast<const uint32_t*>(&ks[t0][c]));
-        const float2 x1 = unpack_bf2(*reinterpret_cast<const uint32_t*>(&ks[t1][c]));
-        kword |= quant_code(x0.x, z0, levels, &skz[0][c], &skz[1][c]) << (BITS * i);
-        kword |= quant_code(x0.y, z1, levels, &skz[0][c + 1], &skz[1][c + 1]) << (16 + BITS * i);
-        kword |= quant_code(x1.x, z0, levels, &skz[0][c], &skz[1][c]) << (8 + BITS * i);
-        kword |= quant_code(x1.y, z1, levels, &skz[0][c + 1], &skz[1][c + 1]) << (24 + BITS * i);
-      }
-      {  // values: X = (reg0: channel gid, reg2: tokens + 8), Y = (reg1: channel gid + 8, reg3)
-        const int c = 16 * ct + gid + (isY ? 8 : 0);
-        const int t0 = 16 * tt + 2 * tig, t1 = t0 + 8;
-        vword |= vcode(t0, c) << (BITS * i);
-        vword |= vcode(t0 + 1, c) << (16 + BITS * i);
-        vword |= vcode(t1, c) << (8 + BITS * i);
-        vword |= vcode(t1 + 1, c) << (24 + BITS * i);
-      }
-    }
-    kw[wi] = kword;
-    vw[wi] = vword;
-  }
-  // key parameters in fragment order: channel c = 16 kt + 8 h + 2 t + e at
-  // fp16 slot 2 (t * 2 (D/16) + 2 kt + h) + e
+  auto Kf = [&](int t, int c) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ks + t * RS + 2 * c)); };
   uint16_t* sk = reinterpret_cast<uint16_t*>(rec + 2 * L::CB);
   uint16_t* zk = sk + D;
-  for (int c = tid; c < D; c += 128) {
-    const int kt = c >> 4, h = (c >> 3) & 1, t = (c >> 1) & 3, e = c & 1;
-    const int slot = 2 * (t * 2 * L::KT + 2 * kt + h) + e;
-    sk[slot] = skz[0][c];
-    zk[slot] = skz[1][c];
-  }
-  // value parameters pair-interleaved: [G/2][CPG][2]
   uint16_t* sv = zk + D;
   uint16_t* zv = sv + D;
-  for (int e = tid; e < G * L::CPG; e += 128) {
-    const int t = e / L::CPG, cg = e % L::CPG;
-    const int slot = ((t >> 1) * L::CPG + cg) * 2 + (t & 1);
-    sv[slot] = svz[0][t][cg];
-    zv[slot] = svz[1][t][cg];
+
+  // key parameters: channel c over the group's G tokens; stored in fragment
+  // order, channel c = 16 kt + 8 h + 2 t + e at fp16 slot 2 (t * 2 (D/16) + 2 kt + h) + e
+  for (int c = tid; c < D; c += 128) {
+    float mn = Kf(0, c), mx = mn;
+    for (int t = 1; t < G; ++t) mn = fminf(mn, Kf(t, c)), mx = fmaxf(mx, Kf(t, c));
+    const uint16_t sb = to_half_checked((static_cast<double>(mx) - static_cast<double>(mn)) / levels, flags);
+    const uint16_t zb = to_half_checked(static_cast<double>(mn), flags);
+    const int kt = c >> 4, h = (c >> 3) & 1, tq = (c >> 1) & 3, e = c & 1;
+    const int slot = 2 * (tq * 2 * L::KT + 2 * kt + h) + e;
+    sk[slot] = sb;
+    zk[slot] = zb;
+    const float sf = __half2float(__ushort_as_half(sb));
+    kzn[c] = -__half2float(__ushort_as_half(zb));
+    kin[c] = sf != 0.f ? 1.f / sf : 0.f;
+    ksc[c] = sf;
+  }
+  // value parameters: token t, value group cg over its G channels; the
+  // minimum and maximum by one warp per token row (lane l holds channels
+  // EPL l ..), then one thread per (token, value group) forms the
+  // parameters; stored pair-interleaved [G/2][CPG][2]
+  for (int t = warp; t < G; t += 4) {
+    float mn, mx;
+    if constexpr (EPL == 4) {
+      const uint2 w = *reinterpret_cast<const uint2*>(vs + t * RS + 8 * lane);
+      const float2 a = unpack_bf2(w.x), b = unpack_bf2(w.y);
+      mn = fminf(fminf(a.x, a.y), fminf(b.x, b.y));
+      mx = fmaxf(fmaxf(a.x, a.y), fmaxf(b.x, b.y));
+    } else {
+      const float2 a = unpack_bf2(*reinterpret_cast<const uint32_t*>(vs + t * RS + 4 * lane));
+      mn = fminf(a.x, a.y);
+      mx = fmaxf(a.x, a.y);
+    }
+#pragma unroll
+    for (int m = 1; m < LPG; m <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, m));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+    }
+    if (lane % LPG == 0) {
+      vsc[lane / LPG][t] = mn;  // staged here until the parameters replace them
+      vin[lane / LPG][t] = mx;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < G * CPG; e += 128) {
+    const int cg = e / G, t = e - cg * G;
+    const float mn = vsc[cg][t], mx = vin[cg][t];
+    const uint16_t sb = to_half_checked((static_cast<double>(mx) - static_cast<double>(mn)) / levels, flags);
+    const uint16_t zb = to_half_checked(static_cast<double>(mn), flags);
+    const int slot = ((t >> 1) * CPG + cg) * 2 + (t & 1);
+    sv[slot] = sb;
+    zv[slot] = zb;
+    const float sf = __half2float(__ushort_as_half(sb));
+    vzn[cg][t] = -__half2float(__ushort_as_half(zb));
+    vin[cg][t] = sf != 0.f ? 1.f / sf : 0.f;
+    vsc[cg][t] = sf;
+  }
+  __syncthreads();
+
+  // code words: word index = (tt * 32 + lane) * NW + w, w = 2 j + (0: X, 1: Y);
+  // local tile i of pair j covers channel (key) / channel-row (value) tile
+  // TPW j + i; first register's codes at bits [b i] and [16 + b i], second's
+  // at [8 + b i], [24 + b i].  ldmatrix row providers: lane 8 mi + ri.
+  const int gid = lane >> 2, tig = lane & 3, mi = lane >> 3, ri = lane & 7;
+  uint32_t* kw = reinterpret_cast<uint32_t*>(rec);
+  uint32_t* vw = reinterpret_cast<uint32_t*>(rec + L::CB);
+  for (int item = warp; item < 2 * TT * NJ; item += 4) {  // warp-uniform
+    const bool isv = item >= TT * NJ;
+    const int it = isv ? item - TT * NJ : item;
+    const int tt = it / NJ, j = it - tt * NJ;
+    uint32_t X = 0u, Y = 0u;
+    uint32_t nm = 0u;  // pairs of this lane near a tie: bit 4 i + register
+    // keys: r0 / r1 = tokens gid / gid + 8 at channels 16 ct + 2 tig (+1), r2 /
+    // r3 the same at channels + 8: X = r0 | r1 << 8, Y = r2 | r3 << 8.
+    // values (transposed): r0 / r1 = channel gid / gid + 8 at tokens
+    // 16 tt + 2 tig (+1), r2 / r3 the same at tokens + 8: X = r0 | r2 << 8,
+    // Y = r1 | r3 << 8.  Register k goes to word (k >> wsh) & 1 of (X, Y) at
+    // offset 8 ((k >> osh) & 1); its parameters are those of the first (k < 2:
+    // keys channel c, values tokens t0) or the second pair (c + 8, t0 + 8).
+    const int wsh = isv ? 0 : 1, osh = isv ? 1 : 0;
+#pragma unroll
+    for (int i = 0; i < TPW; ++i) {
+      const int ct = TPW * j + i;
+      uint32_t r[4];
+      const float *zp, *ip;
+      int o0;
+      if (!isv) {
+        ldsm_x4(r, ks + (16 * tt + 8 * (mi & 1) + ri) * RS + (16 * ct + 8 * (mi >> 1)) * 2);
+        zp = kzn, ip = kin, o0 = 16 * ct + 2 * tig;
+      } else {
+        ldsm_x4_t(r, vs + (16 * tt + 8 * (mi >> 1) + ri) * RS + (16 * ct + 8 * (mi & 1)) * 2);
+        const int cg = 16 * ct / G;
+        zp = &vzn[cg][0], ip = &vin[cg][0], o0 = 16 * tt + 2 * tig;
+      }
+      const float2 za = *reinterpret_cast<const float2*>(zp + o0), ia = *reinterpret_cast<const float2*>(ip + o0);
+      const float2 zb = *reinterpret_cast<const float2*>(zp + o0 + 8), ib = *reinterpret_cast<const float2*>(ip + o0 + 8);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        bool nr;
+        const uint32_t p = codes2_fast<BITS>(r[k], k < 2 ? za : zb, k < 2 ? ia : ib, nr);
+        nm |= (nr ? 1u : 0u) << (4 * i + k);
+        const uint32_t placed = p << (8 * ((k >> osh) & 1) + BITS * i);
+        if ((k >> wsh) & 1)
+          Y |= placed;
+        else
+          X |= placed;
+      }
+    }
+    if (__any_sync(0xffffffffu, nm != 0u)) {  // some lane holds a pair near a tie
+      const uint2 w = isv ? fix_words<BITS, G, RS, TPW>(make_uint2(X, Y), nm, true, tt, j, vs, &vzn[0][0], &vin[0][0],
+                                                        &vsc[0][0])
+                          : fix_words<BITS, G, RS, TPW>(make_uint2(X, Y), nm, false, tt, j, ks, kzn, kin, ksc);
+      X = w.x, Y = w.y;
+    }
+    uint32_t* dst = (isv ? vw : kw) + (tt * 32 + lane) * NW + 2 * j;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(X, Y);
   }
 }
 
