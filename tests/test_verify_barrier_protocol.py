@@ -15,15 +15,20 @@ MMA happens exactly once:
   released stage j mod NS and V of tile j once the P.V MMAs of tile j - NS
   did, in the order those happen (K one tile ahead of V);
 * MMA thread: S of tiles 0 and 1 (after Q and their K), then per tile i,
-  after the softmax group's barrier: P.V(i) once V(i) landed, and S(i + 2)
-  into S buffer i & 1 once P.V(i) is done and K(i + 2) landed; each S group
-  also releases its K stage, each P.V group its V stage;
-* softmax group: per tile i, wait S(i), work, wait P.V(i - 1) when it
-  rescales O (the lazy rule makes that rare), barrier.
+  once every softmax warp has stored P(i) (barrier p<i & 1>): P.V(i) once
+  V(i) landed, and S(i + 2) into S buffer i & 1 once P.V(i) is done and
+  K(i + 2) landed; each S group also releases its K stage, each P.V group
+  its V stage;
+* softmax warps (4, or 8 when one block takes two row tiles), each on its
+  own clock: per tile i, wait S(i), work, wait P.V(i - 1) when it rescales
+  O (the lazy rule makes that rare), store P, arrive on p<i & 1> and go on
+  to tile i + 1 without waiting for the MMA thread; at the end wait for the
+  last P.V.
 
 Barriers: k<j> v<j> (stage landed), kf<j> vf<j> (stage released) for
-j < NS, s0 s1 (S buffers), pv0 pv1 (P.V per buffer), q.  The tensor pipe
-runs MMA groups in issue order; a group's commits fire when it ends.
+j < NS, s0 s1 (S buffers), p0 p1 (P stored: one arrival per softmax warp
+completes a phase), pv0 pv1 (P.V per buffer), q.  The tensor pipe runs MMA
+groups in issue order; a group's commits fire when it ends.
 """
 
 import heapq
@@ -40,6 +45,7 @@ class _Sim:
         self.waiters = {}
         self.pipe_free = 0.0
         self.group = []
+        self.arrivals = {}
 
     def done(self, name):
         return self.count.get(name, 0)
@@ -95,6 +101,14 @@ class _Sim:
             for name in (req[1] if isinstance(req[1], tuple) else (req[1],)):
                 self.fire_after(self.pipe_free - self.t, name)
             self.schedule(self.rng.uniform(0, req[2]), gen)  # the issue may block part of the time
+        elif kind == "arrive":  # one arrival; the phase completes at `count` arrivals
+            _, name, count = req
+            a = self.arrivals.get(name, 0) + 1
+            if a == count:
+                a = 0
+                self.complete(name)
+            self.arrivals[name] = a
+            self.schedule(0.0, gen)
         elif kind == "group":
             self.group.append(gen)
             if len(self.group) == 2:
@@ -103,9 +117,10 @@ class _Sim:
                 self.group = []
 
 
-def _run_protocol(n, rng, NS):
+def _run_protocol(n, rng, NS, warps, stale_p_wait=False):
     sim = _Sim(rng)
     finished = []
+    stored = [0] * n  # softmax warps that have stored P of each tile
 
     def loader():
         yield ("load", "q")
@@ -134,7 +149,8 @@ def _run_protocol(n, rng, NS):
         for i in range(min(2, n)):
             yield from issue_s(i)
         for i in range(n):
-            yield ("group",)
+            yield ("wait", f"p{i & 1}", max(0, (i >> 1) - 1) if stale_p_wait else i >> 1)
+            assert stored[i] == warps, f"P.V({i}) issued before every warp stored P({i})"
             yield ("wait", f"v{i % NS}", i // NS)
             yield ("mma", (f"pv{i & 1}", f"vf{i % NS}"), rng.uniform(5, 60))
             if i + 2 < n:
@@ -149,14 +165,17 @@ def _run_protocol(n, rng, NS):
             yield ("sleep", rng.uniform(5, 80))
             if i > 0 and rng.random() < 0.3:  # only a warp that rescales O waits for P.V(i - 1)
                 yield ("wait", f"pv{(i - 1) & 1}", (i - 1) >> 1)
-            yield ("group",)
+            yield ("sleep", rng.uniform(0, 10))  # P stored
+            stored[i] += 1
+            yield ("arrive", f"p{i & 1}", warps)
         yield ("wait", f"pv{(n - 1) & 1}", (n - 1) >> 1)
         finished.append("softmax")
 
-    for g in (loader(), mma(), softmax()):
+    for g in (loader(), mma(), *[softmax() for _ in range(warps)]):
         sim.schedule(0.0, g)
     sim.run()
-    assert sorted(finished) == ["loader", "mma", "softmax"], "a role never finished (deadlock)"
+    assert sorted(finished) == ["loader", "mma"] + ["softmax"] * warps, "a role never finished (deadlock)"
+    assert sim.done("p0") + sim.done("p1") == n
     for kind in ("s", "pv"):
         assert sim.done(f"{kind}0") + sim.done(f"{kind}1") == n, kind
     for kind in ("k", "v", "kf", "vf"):
@@ -164,12 +183,12 @@ def _run_protocol(n, rng, NS):
     assert sim.done("q") == 1
 
 
-@pytest.mark.parametrize("NS", [2, 4])
+@pytest.mark.parametrize("NS,warps", [(2, 4), (2, 8), (4, 8)])
 @pytest.mark.parametrize("ntiles", list(range(1, 12)))
-def test_parity_waits_never_early_or_late(ntiles, NS):
-    rng = random.Random(1000 + ntiles + 100 * NS)
-    for _ in range(150):
-        _run_protocol(ntiles, rng, NS)
+def test_parity_waits_never_early_or_late(ntiles, NS, warps):
+    rng = random.Random(1000 + ntiles + 100 * NS + warps)
+    for _ in range(100):
+        _run_protocol(ntiles, rng, NS, warps)
 
 
 def test_model_catches_a_wait_on_a_stale_phase():
@@ -211,3 +230,13 @@ def test_model_catches_a_wait_on_a_stale_phase():
     with pytest.raises(AssertionError):
         for _ in range(50):
             bad_run(8)
+
+
+def test_model_catches_a_p_wait_on_a_stale_phase():
+    """Planting a mistake in the model: an MMA thread that waits for the "P
+    stored" phase of tile i - 2 instead of tile i issues P.V before every
+    softmax warp has stored P; the checker must notice in one of the runs."""
+    rng = random.Random(11)
+    with pytest.raises(AssertionError):
+        for _ in range(50):
+            _run_protocol(8, rng, 2, 4, stale_p_wait=True)
