@@ -86,6 +86,27 @@ def test_zero_scales_and_exact_ties_round_half_to_even():
     assert list(vc_[0, 1, 7, 2:5]) == [0, 2, 2]
 
 
+def test_tie_whose_fp32_difference_is_inexact():
+    """x - z not exact in fp32 next to a tie: z = -1000, s = 400 (max 200),
+    x = 2^-30, so (x - z) / s = 2.5 + 2^-30 / 400 rounds up to 3, while the
+    fp32 difference (1000) would sit exactly on the tie and round to even (2).
+    Keys (channel 3 of group 0) and values (token 5, value group 0)."""
+    B, Hkv, D, G, bits = 1, 1, 64, 32, 2
+    k, v = synth.kv_full(B, Hkv, G, D, seed=8, key_outliers=False)
+    k = k.float()
+    v = v.float()
+    k[0, 0, :, 3] = torch.linspace(-900.0, 100.0, G)
+    k[0, 0, 0, 3], k[0, 0, 1, 3], k[0, 0, 2, 3] = -1000.0, 200.0, 2.0 ** -30
+    v[0, 0, 5, 0:32] = torch.linspace(-900.0, 100.0, 32)
+    v[0, 0, 5, 0], v[0, 0, 5, 1], v[0, 0, 5, 2] = -1000.0, 200.0, 2.0 ** -30
+    k, v = k.to(torch.bfloat16), v.to(torch.bfloat16)
+    assert k[0, 0, 2, 3].item() == 2.0 ** -30 and v[0, 0, 5, 2].item() == 2.0 ** -30
+    check_against_oracle(k, v, bits, G, 0)
+    kc, sk, zk, vc_, sv, zv = Q.cache_parts(Q.build_quant_cache(np32(k), np32(v), bits, G, 0))
+    assert sk[0, 0, 0, 3] == 400.0 and zk[0, 0, 0, 3] == -1000.0 and kc[0, 0, 2, 3] == 3
+    assert vc_[0, 0, 5, 2] == 3
+
+
 def test_scale_outside_fp16_is_flagged():
     B, Hkv, D, G = 1, 1, 64, 32
     k, v = synth.kv_full(B, Hkv, G, D, seed=4)
