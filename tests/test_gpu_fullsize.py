@@ -179,7 +179,8 @@ def test_accept_full_size_every_row():
 
 def test_streamed_verify_full_layer_bit_identical():
     """One Qwen-32B-shaped layer (409.6 MB of K and V) streamed from pinned
-    host memory gives bit-identical results to the resident call."""
+    host memory gives bit-identical results to the resident call, and one
+    streamed (request, KV head) unit of the second layer matches the oracle."""
     B, Hq, Hkv, D, T, nq, NL = 1, 40, 8, 128, 100000, 31, 2
     kv = [synth.kv_full(B, Hkv, T, D, seed=60 + l) for l in range(NL)]
     hk = [k.pin_memory() for k, _ in kv]
@@ -210,5 +211,9 @@ def test_streamed_verify_full_layer_bit_identical():
     ks.close()
     for l in range(NL):
         assert torch.equal(outs[l], resident[l]), l
+    g, h = Hq // Hkv, 5
+    want, _ = A.verify_attention(np32(q[1][:, :, h * g:(h + 1) * g]), np32(kv[1][0][:, h:h + 1]).astype(np.float64),
+                                 np32(kv[1][1][:, h:h + 1]).astype(np.float64))
+    assert row_rel_err(np32(outs[1])[:, :, h * g:(h + 1) * g], want) <= ATTN_TOL
     del stage_k, stage_v, ws
     _free()
