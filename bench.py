@@ -831,7 +831,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama-3.1-8b-32k-kivi2", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
-    ap.add_argument("--kernel", default="", choices=["", "draft", "verify", "accept"],
+    ap.add_argument("--kernel", default="", choices=["", "draft", "verify", "accept", "compress"],
                     help="time one kernel of the workload alone (a per-kernel line for profiler captures; "
                          "not the benchmark line)")
     ap.add_argument("--layers", type=int, default=0,
@@ -924,7 +924,8 @@ def _common(args, config, value, peak, peak_kind, r, dtype):
 def kernel_line(args, w, peak, peak_kind):
     """One kernel of the workload timed alone with CUDA events: the quantised
     or token-dropped draft attention of one layer, one resident
-    verification layer, or one acceptance call over the round's logits."""
+    verification layer, one acceptance call over the round's logits, or the
+    GPU compression of one layer (quantiser and kept-row compaction)."""
     import torch
     from lossless_draft_verify_vc_b200 import synth, vc
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -939,6 +940,17 @@ def kernel_line(args, w, peak, peak_kind):
         return {"kernel": "vc_verify_attn", "workload": args.workload, "us": rv["us_per_layer"],
                 "gbps": rv["hbm_gbps"], "frac_of_hbm_peak": rv["hbm_gbps"] / peak, "tflops": rv["tflops"],
                 "peak_kind": peak_kind, "calls": reps}
+    if args.kernel == "compress":
+        if "bits" not in w:
+            return {"kernel": "vc_quantize_cache", "workload": args.workload,
+                    "unavailable": "the workload's draft cache is token-dropped, not quantised"}
+        kvs = [synth.kv_full(B, w["Hkv"], w["T"], w["D"], seed=s, device=dev) for s in (1, 2)]
+        cp = time_compress(w, dev, {"kvs": kvs, "sh": vc.shape(B, w["Hq"], w["Hkv"], w["D"])})
+        return {"kernel": "vc_quantize_cache + vc_compact_kept", "workload": args.workload,
+                "quantize_us": cp["quantize_us"], "quantize_gbps": cp["quantize_gbps"],
+                "quantize_frac_of_hbm_peak": cp["quantize_gbps"] / peak, "compact_us": cp["compact_us"],
+                "compact_gbps": cp["compact_gbps"], "compact_frac_of_hbm_peak": cp["compact_gbps"] / peak,
+                "flags": cp["flags"], "peak_kind": peak_kind}
     if args.kernel == "accept":
         K, V = w["K"], w["V"]
         dt = torch.bfloat16 if w["logits"] == "bf16" else torch.float32
