@@ -20,9 +20,10 @@
 //     x channels: the g heads of nqt positions are the tile's rows), the
 //     first request of the block so that it does not queue behind K and V;
 //   * K and V tiles of BN = 64 keys stream in through 2-slot rings of tiled
-//     TMA loads (3-D tensor maps, rows past T read as zeros, no multicast),
-//     K and V on barriers of their own: a K slot is refilled as soon as the
-//     S that read it is done, a V slot once its P.V is done;
+//     TMA loads (3-D tensor maps, rows past T read as zeros, no multicast,
+//     evict-first in L2), K and V on barriers of their own: a K slot is
+//     refilled as soon as the S that read it is done, a V slot once its P.V
+//     is done;
 //   * a loader warp issues the TMA loads, an MMA warp issues tcgen05.mma:
 //     S = Q K^T into tensor memory (TMEM), and P.V; the MMA warp blocks on
 //     the tensor pipe's queue while the softmax warps work, so no row waits
@@ -33,7 +34,9 @@
 //     online softmax with lazy rescaling (O is rescaled only when the running
 //     maximum grows by more than 8 in log2 units), and writes P back to TMEM
 //     over its own S as a bf16 high part and a bf16 low part (P keeps ~16
-//     bits);
+//     bits); each softmax warp then arrives on that S buffer's "P stored"
+//     mbarrier and goes straight on to the next tile -- the MMA thread waits
+//     on the barrier, the softmax warps never wait for the MMA thread;
 //   * O += P_hi V + P_lo V as tcgen05.mma with A read from TMEM and V from
 //     shared memory (MN-major), accumulating in TMEM;
 //   * at the end each softmax thread moves its O row from TMEM to the output
