@@ -94,55 +94,13 @@ __device__ __forceinline__ uint32_t code_near(float x, float negz, float inv, fl
   return static_cast<uint32_t>(c);
 }
 
+// Both codes of a register pair with code_near (out of line: it runs only
+// for the rare pairs near a tie, and inlined in every tile it would cost the
+// common path registers and code size).
 template <int BITS>
-__device__ __forceinline__ uint32_t codes2_near(uint32_t xb, float2 negz, float2 inv, float2 sc) {
+__device__ __noinline__ uint32_t codes2_near(uint32_t xb, float2 negz, float2 inv, float2 sc) {
   const float2 x = unpack_bf2(xb);
   return code_near<BITS>(x.x, negz.x, inv.x, sc.x) | (code_near<BITS>(x.y, negz.y, inv.y, sc.y) << 16);
-}
-
-// Per-lane fix-up of a word pair whose fast codes include pairs near a tie
-// (bit 4 i + register of nm): the tile's registers are loaded again and the
-// near pairs recomputed with code_near.  Warp-collective (ldmatrix); out of
-// line so that the common path keeps few registers.
-//   base: the staged K (isv false) or V rows; RS their stride in bytes;
-//   z, iv, sc: (-zero, 1 / scale, scale) per key channel, or per token of
-//   value group cg at z + cg * G (G floats per group).
-template <int BITS, int G, int RS, int TPW>
-__device__ __noinline__ uint2 fix_words(uint2 w, uint32_t nm, bool isv, int tt, int j, const unsigned char* base,
-                                        const float* z, const float* iv, const float* sc) {
-  constexpr uint32_t levels = (1u << BITS) - 1u;
-  const int lane = threadIdx.x & 31, tig = lane & 3, mi = lane >> 3, ri = lane & 7;
-  const int wsh = isv ? 0 : 1, osh = isv ? 1 : 0;
-  for (int i = 0; i < TPW; ++i) {
-    if (!__any_sync(0xffffffffu, (nm >> (4 * i)) & 0xfu)) continue;
-    const int ct = TPW * j + i;
-    uint32_t r[4];
-    int o0;
-    const float *zp = z, *ip = iv, *sp = sc;
-    if (!isv) {
-      ldsm_x4(r, base + (16 * tt + 8 * (mi & 1) + ri) * RS + (16 * ct + 8 * (mi >> 1)) * 2);
-      o0 = 16 * ct + 2 * tig;
-    } else {
-      ldsm_x4_t(r, base + (16 * tt + 8 * (mi >> 1) + ri) * RS + (16 * ct + 8 * (mi & 1)) * 2);
-      const int cg = 16 * ct / G;
-      zp += cg * G, ip += cg * G, sp += cg * G;
-      o0 = 16 * tt + 2 * tig;
-    }
-    for (int k = 0; k < 4; ++k) {
-      if (!((nm >> (4 * i + k)) & 1u)) continue;
-      const int o = o0 + (k < 2 ? 0 : 8);
-      const uint32_t p = codes2_near<BITS>(r[k], *reinterpret_cast<const float2*>(zp + o),
-                                           *reinterpret_cast<const float2*>(ip + o),
-                                           *reinterpret_cast<const float2*>(sp + o));
-      const int sh = 8 * ((k >> osh) & 1) + BITS * i;
-      const uint32_t field = (levels | (levels << 16)) << sh;
-      if ((k >> wsh) & 1)
-        w.y = (w.y & ~field) | (p << sh);
-      else
-        w.x = (w.x & ~field) | (p << sh);
-    }
-  }
-  return w;
 }
 
 template <int BITS, int G, int D>
@@ -154,7 +112,6 @@ struct QuantLayout {
   static constexpr int NW = 2 * KT / TPW;  // words per lane per 16-token tile
   static constexpr int NJ = KT / TPW;      // word pairs (X, Y) per lane per 16-token tile
   static constexpr int CPG = D / G;
-  static constexpr int WORDS = CB / 4;     // 32-bit words of one code block
 };
 
 // One block of 128 threads per (group, unit).  The group's K and V rows are
@@ -257,7 +214,7 @@ __device__ __forceinline__ void quantize_group(const __nv_bfloat16* __restrict__
   // local tile i of pair j covers channel (key) / channel-row (value) tile
   // TPW j + i; first register's codes at bits [b i] and [16 + b i], second's
   // at [8 + b i], [24 + b i].  ldmatrix row providers: lane 8 mi + ri.
-  const int gid = lane >> 2, tig = lane & 3, mi = lane >> 3, ri = lane & 7;
+  const int tig = lane & 3, mi = lane >> 3, ri = lane & 7;
   uint32_t* kw = reinterpret_cast<uint32_t*>(rec);
   uint32_t* vw = reinterpret_cast<uint32_t*>(rec + L::CB);
   for (int item = warp; item < 2 * TT * NJ; item += 4) {  // warp-uniform
@@ -265,7 +222,6 @@ __device__ __forceinline__ void quantize_group(const __nv_bfloat16* __restrict__
     const int it = isv ? item - TT * NJ : item;
     const int tt = it / NJ, j = it - tt * NJ;
     uint32_t X = 0u, Y = 0u;
-    uint32_t nm = 0u;  // pairs of this lane near a tie: bit 4 i + register
     // keys: r0 / r1 = tokens gid / gid + 8 at channels 16 ct + 2 tig (+1), r2 /
     // r3 the same at channels + 8: X = r0 | r1 << 8, Y = r2 | r3 << 8.
     // values (transposed): r0 / r1 = channel gid / gid + 8 at tokens
@@ -290,23 +246,34 @@ __device__ __forceinline__ void quantize_group(const __nv_bfloat16* __restrict__
       }
       const float2 za = *reinterpret_cast<const float2*>(zp + o0), ia = *reinterpret_cast<const float2*>(ip + o0);
       const float2 zb = *reinterpret_cast<const float2*>(zp + o0 + 8), ib = *reinterpret_cast<const float2*>(ip + o0 + 8);
+      uint32_t nmi = 0u;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         bool nr;
         const uint32_t p = codes2_fast<BITS>(r[k], k < 2 ? za : zb, k < 2 ? ia : ib, nr);
-        nm |= (nr ? 1u : 0u) << (4 * i + k);
+        nmi |= (nr ? 1u : 0u) << k;
         const uint32_t placed = p << (8 * ((k >> osh) & 1) + BITS * i);
         if ((k >> wsh) & 1)
           Y |= placed;
         else
           X |= placed;
       }
-    }
-    if (__any_sync(0xffffffffu, nm != 0u)) {  // some lane holds a pair near a tie
-      const uint2 w = isv ? fix_words<BITS, G, RS, TPW>(make_uint2(X, Y), nm, true, tt, j, vs, &vzn[0][0], &vin[0][0],
-                                                        &vsc[0][0])
-                          : fix_words<BITS, G, RS, TPW>(make_uint2(X, Y), nm, false, tt, j, ks, kzn, kin, ksc);
-      X = w.x, Y = w.y;
+      // pairs of this tile near a tie (rare per pair, but some lane meets one
+      // in most word pairs): their codes again, exactly
+      if (__any_sync(0xffffffffu, nmi != 0u) && nmi != 0u) {
+        const float* sp = isv ? &vsc[16 * ct / G][0] : ksc;
+        const float2 sa = *reinterpret_cast<const float2*>(sp + o0), sb = *reinterpret_cast<const float2*>(sp + o0 + 8);
+        for (int k = 0; k < 4; ++k) {
+          if (!((nmi >> k) & 1u)) continue;
+          const uint32_t p = codes2_near<BITS>(r[k], k < 2 ? za : zb, k < 2 ? ia : ib, k < 2 ? sa : sb);
+          const int sh = 8 * ((k >> osh) & 1) + BITS * i;
+          const uint32_t field = static_cast<uint32_t>(levels | (levels << 16)) << sh;
+          if ((k >> wsh) & 1)
+            Y = (Y & ~field) | (p << sh);
+          else
+            X = (X & ~field) | (p << sh);
+        }
+      }
     }
     uint32_t* dst = (isv ? vw : kw) + (tt * 32 + lane) * NW + 2 * j;
     *reinterpret_cast<uint2*>(dst) = make_uint2(X, Y);
