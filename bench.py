@@ -26,6 +26,7 @@ the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -248,7 +249,7 @@ class ClockSampler:
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,timestamp")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
@@ -256,18 +257,30 @@ class ClockSampler:
         self.path = None
 
     def start(self):
+        """Starts sampling every 100 ms and returns once the first sample is
+        written (at most ~3 s), so that the timed region that follows is
+        covered; samples before this point and after stop() are dropped by
+        their timestamps."""
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
+        self.t0 = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        for _ in range(60):
+            if os.path.getsize(self.path) > 0 or self.proc.poll() is not None:
+                break
+            time.sleep(0.05)
+        self.t0 = time.time()
 
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        t1 = time.time()
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -280,6 +293,15 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.path)
+
+        def stamp(r):
+            try:
+                return datetime.datetime.strptime(r[9], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except (ValueError, IndexError):
+                return None
+
+        inside = [r for r in rows if self.t0 is not None and stamp(r) is not None and self.t0 - 0.1 <= stamp(r) <= t1]
+        rows = inside or rows  # keep every sample when the window holds none (a very short region)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
 
