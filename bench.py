@@ -92,25 +92,30 @@ def sparse_bytes_per_layer(w) -> int:
     return w["n_keep"] * w["Hkv"] * (4 * w["D"] + 4) * w["B"]
 
 
-def measure_pcie_h2d(dev, nbytes: int = 1 << 30, reps: int = 5) -> float:
+def measure_pcie_h2d(dev, srcs=(), nbytes: int = 1 << 30, reps: int = 5) -> float:
     """Pinned host -> device copy bandwidth (GB/s, best of reps) of one
-    cudaMemcpyAsync of nbytes: the host-link peak the streamed verification
-    is measured against."""
+    cudaMemcpyAsync: the host-link peak the streamed verification is
+    measured against.  Copies a fresh pinned buffer of nbytes and each of
+    `srcs` (pinned host tensors: the streamed layers themselves, whose host
+    memory may sit elsewhere than a fresh buffer); the best rate counts."""
     import torch
-    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
-    d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     st = torch.cuda.Stream(dev)
     best = 0.0
-    with torch.cuda.stream(st):
-        d.copy_(h, non_blocking=True)
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(st)
+    fresh = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    for h in (fresh, *srcs):
+        d = torch.empty_like(h, device=dev)
+        nb = h.numel() * h.element_size()
+        with torch.cuda.stream(st):
             d.copy_(h, non_blocking=True)
-            e1.record(st)
-            e1.synchronize()
-            best = max(best, nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
-    del h, d
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                d.copy_(h, non_blocking=True)
+                e1.record(st)
+                e1.synchronize()
+                best = max(best, nb / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+        del d
+    del fresh
     return best
 
 
@@ -524,8 +529,8 @@ def time_streamed_verify(args, w, dev, inp, sh, ws_v, out_v, comp):
     import torch
     from lossless_draft_verify_vc_b200 import vc
     NL, T, nq = w["NL"], w["T"], w["K"] + 1
-    pcie = measure_pcie_h2d(dev)
     hk, hv = host_pool(w, torch.bfloat16, w.get("host_pool", 2))
+    pcie = measure_pcie_h2d(dev, (hk[0], hv[0]))
     host_k = [hk[l % len(hk)] for l in range(NL)]
     host_v = [hv[l % len(hv)] for l in range(NL)]
     stage_k = [torch.empty_like(hk[0], device=dev) for _ in range(2)]
@@ -582,8 +587,8 @@ def run_streamed(args, w, rank, world):
     tgt = torch.empty(B, K + 1, dtype=torch.int32, device=dev)
     acc = torch.empty(B, dtype=torch.int32, device=dev)
     cor = torch.empty(B, dtype=torch.int32, device=dev)
-    pcie = measure_pcie_h2d(dev)
     hk, hv = host_pool(w, torch.bfloat16, w["host_pool"])
+    pcie = measure_pcie_h2d(dev, (hk[0], hv[0]))
     host_k = [hk[l % len(hk)] for l in range(NL)]
     host_v = [hv[l % len(hv)] for l in range(NL)]
     stage_k = [torch.empty_like(hk[0], device=dev) for _ in range(2)]
@@ -645,8 +650,8 @@ def run_stagger(args, w, rank, world):
                                      w["n_req"])
     nq = K + 1
     sh = vc.shape(B, Hq, Hkv, D)
-    pcie = measure_pcie_h2d(dev)
     hk, hv = host_pool(w, torch.bfloat16, w["host_pool"])
+    pcie = measure_pcie_h2d(dev, (hk[0], hv[0]))
     copy = torch.cuda.Stream(dev)
     reqs, keep = [], []
     for i in range(n):
