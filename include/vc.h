@@ -556,6 +556,21 @@ VC_API vc_status vc_debug_gather(const vc_attn_shape* shape, const vc_sparse_cac
  * without faulting or hanging a GPU. */
 VC_API vc_status vc_debug_wait_timeout(uint32_t* flags, uint32_t* result, int64_t limit_ns, void* stream);
 
+/* vc_debug_verify_abort is vc_verify_attn with its failure path forced: in
+ * every block the K tile with block-local index skip_tile (>= 0) is never
+ * requested, and the tile loop's waits give up after limit_ns (1 us ..
+ * 100 ms) instead of 2 s.  A block that has that tile stops: the wait on it
+ * ORs VC_FLAG_WAIT_TIMEOUT into the workspace's flag word and raises the
+ * block's abort flag, every other wait of the block then gives up, the
+ * block drains its MMAs and copies, releases its tensor memory and returns;
+ * its output rows are not valid.  Blocks with fewer tiles finish normally.
+ * Same arguments and checks as vc_verify_attn otherwise.  Test only: it
+ * shows a timed-out wait ending the kernel and leaving the context usable
+ * without faulting or hanging a GPU. */
+VC_API vc_status vc_debug_verify_abort(const vc_attn_shape* shape, const void* q, const void* k, const void* v,
+                                       int64_t T, int nq, float* out, float* lse, void* ws, size_t ws_bytes,
+                                       int skip_tile, int64_t limit_ns, void* stream);
+
 /* vc_debug_quant_partition reports, without touching a GPU, how
  * vc_draft_attn_quant cuts one call into blocks when at most target_blocks
  * blocks are allowed (the real call uses SMs x resident blocks).  Each

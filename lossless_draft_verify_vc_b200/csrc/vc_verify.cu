@@ -108,6 +108,11 @@ struct VArgs {
   float scale_log2;
   uint32_t* flags;
   SplitKOut o;
+  // failure-path test only (vc_debug_verify_abort): the block-local K tile
+  // that is never requested (-1: none) and the give-up limit of the tile
+  // loop's waits
+  int skip_k;
+  uint64_t wait_ns;
 };
 
 template <int D, int RTC>
@@ -162,6 +167,7 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
     unsigned char* dst = st_s + (i % NS) * C::STAGE_B + v * C::KV_B;
     uint64_t* bar = v ? &bar_v[i % NS] : &bar_k[i % NS];
     const int y = static_cast<int>(k_begin + static_cast<int64_t>(i) * kVBN);
+    if (v == 0 && i == a.skip_k) return;  // failure-path test: this tile never lands
     mbar_arrive_expect_tx(bar, C::KV_B);
 #pragma unroll
     for (int hf = 0; hf < C::HALVES; ++hf)
@@ -228,7 +234,7 @@ __global__ void __launch_bounds__(VBlk<RTC>::THREADS) verify_kernel(const __grid
     for (;;) {
       if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
       if (*s_abort != 0) return false;
-      if (global_timer_ns() - t0 > 2000000000ull) {
+      if (global_timer_ns() - t0 > a.wait_ns) {
         atomicOr(a.flags, VC_FLAG_WAIT_TIMEOUT);
         return false;
       }
@@ -724,8 +730,13 @@ size_t vc_verify_attn_workspace_size(const vc_attn_shape* shape, int64_t T, int 
   return vc::plan_verify(*shape, T, nq).total;
 }
 
-vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* k, const void* v, int64_t T, int nq,
-                         float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace vc {
+namespace {
+vc_status verify_launch(const vc_attn_shape* shape, const void* q, const void* k, const void* v, int64_t T, int nq,
+                        float* out, float* lse, void* ws, size_t ws_bytes, void* stream, int skip_k,
+                        uint64_t wait_ns) {
   vc_status st = vc::check_verify(shape, T, nq, "vc_verify_attn");
   if (st != VC_OK) return st;
   VC_REQUIRE(q && k && v && out && ws, "vc_verify_attn: null pointer argument");
@@ -753,6 +764,8 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
   const float sm = shape->sm_scale > 0.f ? shape->sm_scale : 1.0f / sqrtf(static_cast<float>(shape->D));
   a.scale_log2 = sm * 1.4426950408889634f;
   a.flags = reinterpret_cast<uint32_t*>(w);
+  a.skip_k = skip_k;
+  a.wait_ns = wait_ns;
   a.o.out = out;
   a.o.lse = lse;
   a.o.part_ml = reinterpret_cast<float*>(w + p.off_ml);
@@ -796,6 +809,25 @@ vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* 
     }
   }
   return vc::launch_status("vc_verify_attn");
+}
+}  // namespace
+}  // namespace vc
+
+extern "C" {
+
+vc_status vc_verify_attn(const vc_attn_shape* shape, const void* q, const void* k, const void* v, int64_t T, int nq,
+                         float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return vc::verify_launch(shape, q, k, v, T, nq, out, lse, ws, ws_bytes, stream, -1, 2000000000ull);
+}
+
+vc_status vc_debug_verify_abort(const vc_attn_shape* shape, const void* q, const void* k, const void* v, int64_t T,
+                                int nq, float* out, float* lse, void* ws, size_t ws_bytes, int skip_tile,
+                                int64_t limit_ns, void* stream) {
+  VC_REQUIRE(skip_tile >= 0, "vc_debug_verify_abort: skip_tile must be >= 0 (got %d)", skip_tile);
+  VC_REQUIRE(limit_ns >= 1000 && limit_ns <= 100000000,
+             "vc_debug_verify_abort: limit must be 1 us .. 100 ms (got %lld ns)", static_cast<long long>(limit_ns));
+  return vc::verify_launch(shape, q, k, v, T, nq, out, lse, ws, ws_bytes, stream, skip_tile,
+                           static_cast<uint64_t>(limit_ns));
 }
 
 }  // extern "C"

@@ -115,6 +115,9 @@ def lib() -> ctypes.CDLL:
             "vc_draft_attn_quant_noalloc_flags": (c_int, [P(c_uint32), c_void_p]),
             "vc_debug_dequant": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_void_p]),
             "vc_debug_wait_timeout": (c_int, [c_void_p, c_void_p, ctypes.c_int64, c_void_p]),
+            "vc_debug_verify_abort": (c_int, [P(vc_attn_shape), c_void_p, c_void_p, c_void_p, c_int64, c_int,
+                                              c_void_p, c_void_p, c_void_p, c_size_t, c_int, ctypes.c_int64,
+                                              c_void_p]),
             "vc_compress_workspace_size": (c_size_t, []),
             "vc_cache_commit": (c_int, [P(vc_attn_shape), P(vc_quant_cache), c_void_p, c_void_p, c_int, c_void_p,
                                         c_void_p, c_size_t, c_void_p]),
@@ -310,6 +313,15 @@ def vc_debug_wait_timeout(flags, result, limit_ns: int, stream=None):
     """Bounded on-chip wait on an mbarrier that never completes (device
     uint32 flags and result; see include/vc.h)."""
     _check(lib().vc_debug_wait_timeout(_p(flags), _p(result), int(limit_ns), _stream(stream)))
+
+
+def vc_debug_verify_abort(sh, q, k, v, T: int, nq: int, out, lse, ws, skip_tile: int, limit_ns: int,
+                          stream=None):
+    """vc_verify_attn with K tile skip_tile of every block never requested
+    and the tile loop's waits giving up after limit_ns (see include/vc.h)."""
+    _check(lib().vc_debug_verify_abort(ctypes.byref(sh), _p(q), _p(k), _p(v), int(T), int(nq), _p(out), _p(lse),
+                                       _p(ws), ws.numel() if hasattr(ws, "numel") else 1 << 62, int(skip_tile),
+                                       int(limit_ns), _stream(stream)))
 
 
 def vc_debug_quant_partition(sh, qc, target_blocks: int) -> dict:
